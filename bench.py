@@ -1,0 +1,369 @@
+#!/usr/bin/env python
+"""Throughput of the PRISM sequence-mixer scan forward on B200.
+
+One step = one prism_scan_fwd call (ShortConv anchor, residual chain, rank-(L-1)
+residual write, gated-delta chunk scan, readout) over one batch of synthetic
+inputs already resident in HBM.  Default workload: one 130M-LM-shaped layer
+(B=16, T=2048, H=6, d_k=d_v=128, L=4, chunk=64, ShortConv width 4, bf16).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank scans its own batch
+(independent replicas sharded by batch, no collective on the data path:
+weak scaling).  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the slow, obviously correct
+definition) on the host cores instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "PRISM scan fwd tokens/s on 1 B200; achieved fraction of TC/HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {
+    "chunk_tc": "linear_attention_sequence_shortconv_b200/csrc/chunk_tc_kernel.cu",
+    "recurrent": "linear_attention_sequence_shortconv_b200/csrc/recurrent_kernel.cu",
+}
+
+
+# ---------------------------------------------------------------- workload arithmetic
+def algorithmic_work(w, lengths=None):
+    """Algorithmic bytes and FLOPs of one scan over workload ``w``.
+
+    Per token-head: bytes = q,k,v,o (4 d elements) + u, gain (2 m d elements) in the
+    I/O dtype, plus gamma, beta (fp32) and alpha (m fp32); per sequence-head the
+    final state (d_v d_k fp32) and S0 if given.  FLOPs (chunk form, dense C x C
+    blocks): 10 C d + 8 C m d + 6 d^2 + 2 m d^2 per token-head (d = d_k = d_v).
+    Only valid tokens count for right-padded batches.
+    """
+    es = 2 if w.dtype == "bf16" else 4
+    d, m, C = w.d_k, w.m, w.chunk
+    valid_tokens = int(lengths.sum()) if lengths is not None else w.B * w.T
+    token_heads = valid_tokens * w.H
+    per_th = es * (2 * w.d_k + 2 * w.d_v) + es * m * (w.d_k + w.d_v) + 4 * (2 + m)
+    state = w.B * w.H * w.d_v * w.d_k * 4 * (2 if w.with_s0 else 1)
+    flops_th = 10 * C * d + 8 * C * m * d + 6 * d * d + 2 * m * d * d
+    return {"tokens": valid_tokens, "token_heads": token_heads,
+            "bytes": token_heads * per_th + state, "flops": token_heads * flops_th}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sha256_of(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of ``kernel`` and this workload; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = rec.get(kernel, {}).get(workload)
+    if not e or e.get("source_sha256") != sha256_of(KERNEL_SOURCES[kernel]):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r for r in csv.reader(io.StringIO(f.read())) if len(r) >= 9]
+        os.unlink(self.file.name)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle (reference arm / baseline)
+def time_oracle(w, budget_s, rows=None, tokens=None):
+    """Time the fp64 oracle on a bounded sample of workload ``w``: the first
+    ``tokens`` steps of the first ``rows`` batch rows, all heads."""
+    from linear_attention_sequence_shortconv_b200 import synth
+    from oracle import prism_seq
+
+    rows = rows or 1
+    tokens = tokens or w.T
+    sample = w.replace(B=rows, T=tokens, lengths_lo=None)
+    x = synth.to_float64_numpy(synth.make_inputs(sample))
+    if w.L == 1:
+        x["u"] = x["alpha"] = x["gain"] = None
+    wall0, cpu0 = time.perf_counter(), time.process_time()
+    prism_seq(**x)
+    wall = time.perf_counter() - wall0
+    cpu = time.process_time() - cpu0
+    cores = max(1, round(cpu / wall)) if wall > 0 else 1
+    return {"tokens": rows * tokens, "seconds": wall, "cores": cores,
+            "sample": f"first {tokens} steps of {rows} batch row(s) x {w.H} heads of {w.name}"}
+
+
+def calibrate_oracle_tokens(w, target_s):
+    probe = time_oracle(w, 0, rows=1, tokens=min(w.T, 64))
+    per_tok = probe["seconds"] / probe["tokens"]
+    return max(8, min(w.T, int(target_s / max(per_tok, 1e-9))))
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    steps, warmup = args.steps, args.warmup
+    budget = 120.0
+    tokens = calibrate_oracle_tokens(w, budget / max(1, steps + warmup))
+    for _ in range(warmup):
+        time_oracle(w, 0, rows=1, tokens=tokens)
+    times, cores, sample = [], 1, ""
+    for _ in range(steps):
+        r = time_oracle(w, 0, rows=1, tokens=tokens)
+        times.append(r["seconds"])
+        cores = max(cores, r["cores"])
+        sample = r["sample"]
+    ms = 1e3 * sum(times) / len(times)
+    value = tokens / (ms / 1e3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, n):
+    return {"workload": f"{w.name}: B={w.B} T={w.T} H={w.H} d_k={w.d_k} d_v={w.d_v} L={w.L} chunk={w.chunk} "
+                        f"W={w.W} {w.dtype}" + (f" lengths~U{{{w.lengths_lo}..{w.T}}}" if w.lengths_lo else ""),
+            "B": w.B, "T": w.T, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "L": w.L, "chunk": w.chunk, "W": w.W,
+            "parallelism": f"dp{n} (independent replicas, batch-sharded; no collective)",
+            "l2": "flushed between timed steps (256 MiB write); inputs also exceed L2"}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import linear_attention_sequence_shortconv_b200 as prism
+    from linear_attention_sequence_shortconv_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wr = w.replace(seed=w.seed + rank)   # each rank scans its own batch
+    host_inputs = synth.make_inputs(wr)
+    d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in host_inputs.items()}
+    io_dtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    o = torch.empty((w.B, w.T, w.H, w.d_v), dtype=io_dtype, device=dev)
+    S = torch.empty((w.B, w.H, w.d_v, w.d_k), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        prism.scan_fwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"], d["conv_w"],
+                       L=w.L, chunk=w.chunk, S0=d["S0"], lengths=d["lengths"], o=o, S_final=S, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if prism.stream_status() != 0:
+        raise SystemExit("device status word reports an error after warm-up")
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    if prism.stream_status() != 0:
+        raise SystemExit("device status word reports an error in the timed region")
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_local = sum(per_step) / K
+    ms = torch.tensor([ms_local], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    ms = float(ms.item())
+    work = algorithmic_work(w, host_inputs["lengths"].numpy() if host_inputs["lengths"] is not None else None)
+    value = world * work["tokens"] / (ms / 1e3)
+
+    # end to end through the host-buffer entry point: pinned host inputs -> HBM,
+    # scan, o and S_final back to host, every step
+    e2e = None
+    if not args.no_e2e:
+        pinned = {n: (t.pin_memory() if isinstance(t, torch.Tensor) else None) for n, t in host_inputs.items()}
+        pinned["o"] = torch.empty(o.shape, dtype=io_dtype).pin_memory()
+        pinned["S_final"] = torch.empty(S.shape, dtype=torch.float32).pin_memory()
+        devbuf = {n: torch.empty_like(t, device=dev) for n, t in pinned.items() if t is not None}
+        K2 = max(1, min(K, args.e2e_steps))
+        for _ in range(2):
+            prism.scan_fwd_host(pinned, devbuf, L=w.L, chunk=w.chunk, stream=stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K2):
+            prism.scan_fwd_host(pinned, devbuf, L=w.L, chunk=w.chunk, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = torch.tensor([e0.elapsed_time(e1) / K2], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        h2d = sum(t.numel() * t.element_size() for n, t in pinned.items()
+                  if t is not None and n not in ("o", "S_final"))
+        d2h = pinned["o"].numel() * pinned["o"].element_size() + S.numel() * 4
+        e2e = {"value": world * work["tokens"] / (float(ems.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K2,
+               "api": "prism_scan_fwd_host (C ABI, pinned host buffers)"}
+
+    # the dominant (only) kernel of a step: roofline against measured HBM bandwidth
+    use_tc = prism.uses_tensor_cores(w.d_k, w.d_v, w.L, w.W, w.chunk,
+                                     prism.PRISM_BF16 if w.dtype == "bf16" else prism.PRISM_FP32)
+    kernel = "chunk_tc" if use_tc else "recurrent"
+    peaks, peak_kind = load_peaks()
+    t_s = ms / 1e3
+    achieved = work["bytes"] / t_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(kernel, w.name),
+                "kernel": kernel, "peak_source": f"{peak_kind} (MEASURED_PEAKS hbm_gbs burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": work["bytes"], "algorithmic_flops_per_launch": work["flops"],
+                "tensor_frac_of_peak": work["flops"] / t_s / 1e12 / peaks["bf16_tflops"],
+                "roofline_time_us": 1e6 * max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                                               work["flops"] / (peaks["bf16_tflops"] * 1e12))}
+    roofline["roofline_frac"] = roofline["roofline_time_us"] / (ms * 1e3)
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 4 if w.T >= 1024 else 16
+        r = time_oracle(w, 0, rows=min(rows, w.B), tokens=min(w.T, 2048))
+        cpu_baseline = {"value": r["tokens"] / r["seconds"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                        "sample": r["sample"], "seconds": r["seconds"]}
+
+    clk = clocks.summary()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded; shapes and distributions of the method's workloads)",
+            "config": workload_config(w, world), "roofline": roofline, "cpu_baseline": cpu_baseline,
+            "e2e": e2e, "gpu_launches": K, "clocks": clk,
+            "tokens_per_step_per_gpu": work["tokens"],
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="lm_130m")
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    from linear_attention_sequence_shortconv_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,183 @@
+/*
+ * prism.h - C ABI of the PRISM sequence-mixer scan for NVIDIA B200 (sm_100a).
+ *
+ * The operation (forward only), per batch row b and head h, with the state
+ * S in R^{d_v x d_k} (S0, or zeros), m = L - 1 residual steps and a ShortConv of
+ * width W:
+ *
+ *   a_t     = sum_{i<W} conv_w[h,:,i] * v_{t-i}      depthwise causal ShortConv anchor
+ *   r_{t,0} = v_t - a_t                               anchor residual
+ *   r_{t,l} = (1 - gain_{t,l}) * r_{t,l-1}            linearised residual chain, l = 1..m
+ *   S_t     = gamma_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *             + sum_l alpha_{t,l} r_{t,l} u_{t,l}^T    gated-delta write + rank-m residual write
+ *   o_t     = S_t q_t                                 post-update readout
+ *
+ * Sources (web pages on PRISM, Parallel Residual Iterative Sequence Model):
+ *   - "ICML 2026 | 当线性注意力学会"写入前思考"：并行化的多步记忆写入" (Tencent Ads
+ *     write-up): section 核心迭代形式 (the step-size x residual x direction write),
+ *     消除 Token 间串行 (forget path kept as GDN, ShortConv anchor replaces the
+ *     global state), 消除 Step 间串行 (closed-form element-wise residual chain),
+ *     架构形式 (write = GDN write + low-rank residual; L = 1 is exactly GDN),
+ *     混合架构是必然 (the anchor window covers the last 3-4 tokens).
+ *   - "PRISM: Parallel Residual Iterative Sequence Model" technical summary,
+ *     sections 2.1 (S_t = S_{t-1} A_t + B_t, A_t the rank-1 gated-delta
+ *     transition) and 2.2 (two-stage proxy: anchor from a short convolution,
+ *     then L parallel refinement steps with gain, residual and direction).
+ *   - ICML 2026 poster abstract of the same paper (short-convolution anchor,
+ *     rank-L accumulation).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers (except in prism_scan_fwd_host),
+ *     owned by the caller.  The library never allocates or frees device memory
+ *     and never synchronises, except prism_stream_status.  Work is enqueued on
+ *     `stream` (0 = legacy default stream).
+ *   - Layouts are dense, row-major, token-major:
+ *       q, k    [B, T, H, d_k]          dtype
+ *       v       [B, T, H, d_v]          dtype
+ *       gamma   [B, T, H]               fp32, decay gate in (0, 1]
+ *       beta    [B, T, H]               fp32, delta-rule step size
+ *       u       [B, T, H, L-1, d_k]     dtype, residual-write directions (NULL iff L == 1)
+ *       alpha   [B, T, H, L-1]          fp32, residual step sizes        (NULL iff L == 1)
+ *       gain    [B, T, H, L-1, d_v]     dtype, per-channel gains g       (NULL iff L == 1)
+ *       conv_w  [H, d_v, W]             fp32, ShortConv taps, tap i multiplies v_{t-i}
+ *       S0      [B, H, d_v, d_k]        fp32 or NULL (zeros)
+ *       lengths [B]                     int32 or NULL (every row has T valid steps);
+ *                                       right padding: steps t >= lengths[b] leave S
+ *                                       unchanged and write o_t = 0
+ *       o       [B, T, H, d_v]          dtype (output)
+ *       S_final [B, H, d_v, d_k]        fp32 (output) or NULL: state after the last
+ *                                       valid step of each row
+ *     dtype is PRISM_BF16 (bfloat16) or PRISM_FP32.  Arithmetic is fp32 with an
+ *     fp32 state; bf16 outputs are rounded to nearest even.
+ *   - Every device pointer must be 16-byte aligned.
+ *   - Return value: PRISM_OK or a PRISM_ERR_* code.  All argument checks run
+ *     before anything is enqueued; on an error nothing is launched and the
+ *     outputs are untouched.  Launch failures return PRISM_ERR_CUDA.  Device-side
+ *     errors (a bounded wait that expired) are recorded in a per-device status
+ *     word that prism_stream_status reports.
+ */
+#ifndef PRISM_H_
+#define PRISM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* prism_stream_t; /* same type as cudaStream_t */
+
+#define PRISM_VERSION_MAJOR 0
+#define PRISM_VERSION_MINOR 1
+#define PRISM_VERSION_PATCH 0
+
+enum prism_dtype {
+  PRISM_BF16 = 0,
+  PRISM_FP32 = 1
+};
+
+enum prism_status {
+  PRISM_OK = 0,
+  PRISM_ERR_INVALID_ARG = 1, /* NULL where required, non-positive size, L < 1, W < 1, ... */
+  PRISM_ERR_UNSUPPORTED = 2, /* valid but not implemented: head size, width, alignment, device */
+  PRISM_ERR_WORKSPACE = 3,   /* workspace smaller than prism_scan_fwd_workspace_size() */
+  PRISM_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  PRISM_ERR_TIMEOUT = 5      /* a bounded device-side wait expired (from prism_stream_status) */
+};
+
+/* Limits of this build (checked; larger values return PRISM_ERR_UNSUPPORTED). */
+#define PRISM_MAX_HEAD_DIM 128 /* d_k, d_v in {16, 32, 64, 128} */
+#define PRISM_MAX_L 16         /* 1 <= L <= 16 */
+#define PRISM_MAX_W 8          /* 1 <= W <= 8 */
+
+/*
+ * prism_scan_fwd - the whole mixer forward: ShortConv anchor, residual chain,
+ * rank-(L-1) residual write and gated-delta write inside one scan, readout.
+ * Defined by the sources above (write-up 核心迭代形式 / 架构形式, summary 2.1-2.2).
+ *
+ * chunk: chunk length of the chunkwise-parallel evaluation, a power of two in
+ *   [16, 64].  The result does not depend on it beyond rounding.  The bf16
+ *   tensor-core path runs chunk == 64 with d_k == d_v in {64, 128} and
+ *   L - 1 <= 3; every other supported shape runs the fp32 CUDA-core path, which
+ *   evaluates the recurrence token by token.
+ * workspace / workspace_bytes: device scratch of at least
+ *   prism_scan_fwd_workspace_size(...) bytes (may be NULL when that is 0).
+ * Errors: PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED, PRISM_ERR_WORKSPACE,
+ *   PRISM_ERR_CUDA, as described above.
+ */
+int prism_scan_fwd(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const void* u, const float* alpha, const void* gain,
+                   const float* conv_w, const float* S0, const int32_t* lengths,
+                   int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
+                   int dtype, void* o, float* S_final,
+                   void* workspace, size_t workspace_bytes, prism_stream_t stream);
+
+/* Bytes of device workspace prism_scan_fwd needs for these sizes (0 if none).
+ * Returns 0 for invalid sizes as well; prism_scan_fwd reports those. */
+size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L,
+                                     int W, int chunk, int dtype);
+
+/*
+ * prism_scan_fwd_host - the same operation on HOST buffers: copies every input
+ * from host memory into the caller's device buffers, runs prism_scan_fwd on
+ * them, and copies o (and S_final if both pointers are given) back to host
+ * memory, all enqueued on `stream` with cudaMemcpyAsync (pinned host memory
+ * makes the copies asynchronous).  host_* are host pointers with the layouts
+ * above, dev_* the device buffers of the same sizes; dk, dv are d_k, d_v.  The
+ * call returns once the work is enqueued; synchronise `stream` before reading
+ * host_o / host_S_final.
+ */
+int prism_scan_fwd_host(const void* host_q, const void* host_k, const void* host_v,
+                        const float* host_gamma, const float* host_beta,
+                        const void* host_u, const float* host_alpha, const void* host_gain,
+                        const float* host_conv_w, const float* host_S0, const int32_t* host_lengths,
+                        void* dev_q, void* dev_k, void* dev_v, float* dev_gamma, float* dev_beta,
+                        void* dev_u, float* dev_alpha, void* dev_gain, float* dev_conv_w,
+                        float* dev_S0, int32_t* dev_lengths,
+                        int B, int T, int H, int dk, int dv, int L, int W, int chunk,
+                        int dtype, void* dev_o, float* dev_S_final, void* host_o, float* host_S_final,
+                        void* workspace, size_t workspace_bytes, prism_stream_t stream);
+
+/*
+ * prism_prologue_fwd - steps before the scan, on their own: the ShortConv
+ * anchor, the anchor residual and the closed-form residual chain, giving the
+ * residual-write vectors rho_{t,l} = alpha_{t,l} r_{t,l} (write-up 消除 Step
+ * 间串行: the chain is element-wise and linear, so it has a closed form).
+ * Inputs as for prism_scan_fwd (L >= 2); lengths may be NULL.
+ * rho_out: [B, T, H, L-1, d_v] fp32 device buffer; rows t >= lengths[b] are
+ * written as 0.  Errors as for prism_scan_fwd.
+ */
+int prism_prologue_fwd(const void* v, const float* alpha, const void* gain,
+                       const float* conv_w, const int32_t* lengths,
+                       int B, int T, int H, int d_v, int L, int W, int dtype,
+                       float* rho_out, prism_stream_t stream);
+
+/* 1 if prism_scan_fwd runs these sizes on the tcgen05 tensor-core chunk
+ * kernel, 0 if on the CUDA-core token-by-token kernel (sizes as for
+ * prism_scan_fwd; unsupported sizes also give 0). */
+int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype);
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the
+ * synchronisation itself failed. */
+int prism_stream_status(prism_stream_t stream);
+
+/* Test hook: the spin limit of the device-side bounded waits (0 restores the
+ * default).  A tiny limit makes those waits give up and record
+ * PRISM_ERR_TIMEOUT instead of waiting, which tests the error path without
+ * hanging a GPU.  Host-side setting; applies to launches made after the call. */
+void prism_set_spin_limit(long long limit);
+
+/* Static description of a status code; never NULL. */
+const char* prism_status_string(int code);
+
+/* (major << 16) | (minor << 8) | patch */
+int prism_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRISM_H_ */

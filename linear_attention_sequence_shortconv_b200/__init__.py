@@ -1,0 +1,23 @@
+"""PRISM sequence-mixer scan for NVIDIA B200 (sm_100a).
+
+The compute lives in ``libprism.so`` (hand-written CUDA kernels behind the C
+ABI of include/prism.h); this package is its thin Python binding plus the
+seeded synthetic input generator.  Build the library with
+``python -m linear_attention_sequence_shortconv_b200.build``.
+"""
+from ._lib import (  # noqa: F401
+    EXPORTS,
+    PRISM_BF16,
+    PRISM_FP32,
+    PrismError,
+    lib,
+    prologue_fwd,
+    scan_fwd,
+    scan_fwd_host,
+    set_spin_limit,
+    status_string,
+    stream_status,
+    uses_tensor_cores,
+    version,
+    workspace_size,
+)

@@ -1,0 +1,224 @@
+"""ctypes binding of ``libprism.so`` (argument marshalling only).
+
+Every step of the scan runs in the library's CUDA kernels; this module only
+checks tensor dtypes/devices, allocates outputs with torch and passes raw
+pointers plus torch's current stream.  There is no CPU fallback: if the
+library is missing or the tensors are not on a CUDA device, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libprism.so")
+
+PRISM_BF16 = 0
+PRISM_FP32 = 1
+STATUS = {
+    0: "PRISM_OK",
+    1: "PRISM_ERR_INVALID_ARG",
+    2: "PRISM_ERR_UNSUPPORTED",
+    3: "PRISM_ERR_WORKSPACE",
+    4: "PRISM_ERR_CUDA",
+    5: "PRISM_ERR_TIMEOUT",
+}
+
+# Every symbol include/prism.h declares.
+EXPORTS = (
+    "prism_scan_fwd",
+    "prism_scan_fwd_workspace_size",
+    "prism_scan_fwd_host",
+    "prism_prologue_fwd",
+    "prism_scan_fwd_uses_tensor_cores",
+    "prism_stream_status",
+    "prism_set_spin_limit",
+    "prism_status_string",
+    "prism_version",
+)
+
+
+class PrismError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library once (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m linear_attention_sequence_shortconv_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, fp, i32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    ci, cs = ctypes.c_int, ctypes.c_size_t
+    L.prism_scan_fwd.argtypes = [vp, vp, vp, fp, fp, vp, fp, vp, fp, fp, i32p,
+                                 ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, fp, vp, cs, vp]
+    L.prism_scan_fwd.restype = ci
+    L.prism_scan_fwd_workspace_size.argtypes = [ci] * 9
+    L.prism_scan_fwd_workspace_size.restype = cs
+    L.prism_scan_fwd_host.argtypes = ([vp] * 11 + [vp] * 11 + [ci] * 9 + [vp, vp, vp, vp, vp, cs, vp])
+    L.prism_scan_fwd_host.restype = ci
+    L.prism_prologue_fwd.argtypes = [vp, fp, vp, fp, i32p, ci, ci, ci, ci, ci, ci, ci, fp, vp]
+    L.prism_prologue_fwd.restype = ci
+    L.prism_scan_fwd_uses_tensor_cores.argtypes = [ci] * 6
+    L.prism_scan_fwd_uses_tensor_cores.restype = ci
+    L.prism_stream_status.argtypes = [vp]
+    L.prism_stream_status.restype = ci
+    L.prism_set_spin_limit.argtypes = [ctypes.c_longlong]
+    L.prism_set_spin_limit.restype = None
+    L.prism_status_string.argtypes = [ci]
+    L.prism_status_string.restype = ctypes.c_char_p
+    L.prism_version.argtypes = []
+    L.prism_version.restype = ci
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().prism_status_string(int(code)).decode()
+
+
+def version() -> Tuple[int, int, int]:
+    v = lib().prism_version()
+    return (v >> 16) & 0xFF, (v >> 8) & 0xFF, v & 0xFF
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return PRISM_BF16
+    if t.dtype == torch.float32:
+        return PRISM_FP32
+    raise TypeError(f"q/k/v/u/gain must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtype=None, required=True):
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype_code) -> int:
+    return int(lib().prism_scan_fwd_workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype_code))
+
+
+def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 64,
+             S0=None, lengths=None, want_state: bool = True, o=None, S_final=None,
+             workspace=None, stream=None):
+    """PRISM mixer forward on CUDA tensors; returns (o, S_final or None).
+
+    Shapes as in include/prism.h: q, k [B,T,H,d_k]; v [B,T,H,d_v]; gamma, beta
+    [B,T,H] fp32; u [B,T,H,L-1,d_k]; alpha [B,T,H,L-1] fp32; gain [B,T,H,L-1,d_v];
+    conv_w [H,d_v,W] fp32; S0 [B,H,d_v,d_k] fp32 or None; lengths [B] int32 or None.
+    """
+    dt = q.dtype
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, dt)
+    for name, t in (("gamma", gamma), ("beta", beta), ("conv_w", conv_w)):
+        _check(t, name, torch.float32)
+    if L > 1:
+        _check(u, "u", dt)
+        _check(gain, "gain", dt)
+        _check(alpha, "alpha", torch.float32)
+    _check(S0, "S0", torch.float32, required=False)
+    _check(lengths, "lengths", torch.int32, required=False)
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    W = conv_w.shape[-1]
+    if o is None:
+        o = torch.empty((B, T, H, d_v), dtype=dt, device=q.device)
+    if want_state and S_final is None:
+        S_final = torch.empty((B, H, d_v, d_k), dtype=torch.float32, device=q.device)
+    ws_bytes = workspace_size(B, T, H, d_k, d_v, L, W, chunk, code)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    rc = lib().prism_scan_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+        _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
+        _ptr(conv_w), _ptr(S0), _ptr(lengths),
+        B, T, H, d_k, d_v, L, W, chunk, code,
+        _ptr(o), _ptr(S_final if want_state else None),
+        _ptr(workspace), ws_bytes if workspace is not None else 0, _stream_handle(stream))
+    if rc != 0:
+        raise PrismError(rc, "prism_scan_fwd")
+    return o, (S_final if want_state else None)
+
+
+def scan_fwd_host(host: dict, dev: dict, L: int, chunk: int = 64, stream=None):
+    """The host-buffer entry point: ``host`` holds pinned CPU tensors (inputs and
+    the outputs ``o``/``S_final``), ``dev`` CUDA tensors of the same shapes.
+    Enqueues H2D copies, the scan and D2H copies on ``stream``; does not sync."""
+    names = ("q", "k", "v", "gamma", "beta", "u", "alpha", "gain", "conv_w", "S0", "lengths")
+    q = host["q"]
+    B, T, H, d_k = q.shape
+    d_v = host["v"].shape[-1]
+    W = host["conv_w"].shape[-1]
+    code = _dtype_code(q)
+    ws_bytes = workspace_size(B, T, H, d_k, d_v, L, W, chunk, code)
+    ws = dev.get("workspace")
+    rc = lib().prism_scan_fwd_host(
+        *[_ptr(host.get(n)) for n in names], *[_ptr(dev.get(n) if host.get(n) is not None else None) for n in names],
+        B, T, H, d_k, d_v, L, W, chunk, code,
+        _ptr(dev["o"]), _ptr(dev.get("S_final")), _ptr(host["o"]), _ptr(host.get("S_final")),
+        _ptr(ws), ws_bytes if ws is not None else 0, _stream_handle(stream))
+    if rc != 0:
+        raise PrismError(rc, "prism_scan_fwd_host")
+
+
+def prologue_fwd(v, alpha, gain, conv_w, L: int, lengths=None, stream=None):
+    """rho_{t,l} = alpha_{t,l} r_{t,l} as [B,T,H,L-1,d_v] fp32 (CUDA)."""
+    code = _dtype_code(v)
+    _check(v, "v")
+    _check(gain, "gain", v.dtype)
+    _check(alpha, "alpha", torch.float32)
+    _check(conv_w, "conv_w", torch.float32)
+    _check(lengths, "lengths", torch.int32, required=False)
+    B, T, H, d_v = v.shape
+    rho = torch.empty((B, T, H, L - 1, d_v), dtype=torch.float32, device=v.device)
+    rc = lib().prism_prologue_fwd(_ptr(v), _ptr(alpha), _ptr(gain), _ptr(conv_w), _ptr(lengths),
+                                  B, T, H, d_v, L, conv_w.shape[-1], code, _ptr(rho),
+                                  _stream_handle(stream))
+    if rc != 0:
+        raise PrismError(rc, "prism_prologue_fwd")
+    return rho
+
+
+def uses_tensor_cores(d_k, d_v, L, W, chunk, dtype_code) -> bool:
+    """True if prism_scan_fwd runs these sizes on the tcgen05 chunk kernel."""
+    return bool(lib().prism_scan_fwd_uses_tensor_cores(d_k, d_v, L, W, chunk, dtype_code))
+
+
+def stream_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(lib().prism_stream_status(_stream_handle(stream)))
+
+
+def set_spin_limit(limit: int) -> None:
+    lib().prism_set_spin_limit(int(limit))

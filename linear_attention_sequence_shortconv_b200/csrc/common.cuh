@@ -1,0 +1,71 @@
+// Shared device helpers of the PRISM scan kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "prism.h"
+
+namespace prism {
+
+// Sizes and pointers of one prism_scan_fwd call (device pointers).
+struct ScanParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* gamma;
+  const float* beta;
+  const void* u;
+  const float* alpha;
+  const void* gain;
+  const float* conv_w;
+  const float* S0;
+  const int32_t* lengths;
+  void* o;
+  float* S_final;
+  int B, T, H, d_k, d_v, L, W, chunk;
+  int* status;            // per-device status word (PRISM_OK / PRISM_ERR_TIMEOUT)
+  long long spin_limit;   // bound of every device-side wait
+};
+
+// ---------------------------------------------------------------- element I/O
+template <typename T>
+__device__ __forceinline__ float ld1(const T* p);
+template <>
+__device__ __forceinline__ float ld1<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ld1<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(__ldg(p));
+}
+
+// four consecutive elements starting at p (p 4-element aligned)
+template <typename T>
+__device__ __forceinline__ float4 ld4(const T* p);
+template <>
+__device__ __forceinline__ float4 ld4<float>(const float* p) {
+  return __ldg(reinterpret_cast<const float4*>(p));
+}
+template <>
+__device__ __forceinline__ float4 ld4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  uint2 raw = __ldg(reinterpret_cast<const uint2*>(p));
+  __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162*>(&raw.x);
+  __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162*>(&raw.y);
+  float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+template <typename T>
+__device__ __forceinline__ void st1(T* p, float x);
+template <>
+__device__ __forceinline__ void st1<float>(float* p, float x) { *p = x; }
+template <>
+__device__ __forceinline__ void st1<__nv_bfloat16>(__nv_bfloat16* p, float x) {
+  *p = __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicCAS(status, PRISM_OK, code);
+}
+
+}  // namespace prism

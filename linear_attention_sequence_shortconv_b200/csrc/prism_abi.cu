@@ -1,0 +1,209 @@
+// C ABI of the PRISM scan: argument checks, launch planning, status word.
+// Declarations and documentation: include/prism.h.
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace prism {
+cudaError_t launch_recurrent_scan(const ScanParams& p, int dtype, cudaStream_t stream);
+cudaError_t launch_prologue(const void* v, const float* alpha, const void* gain, const float* conv_w,
+                            const int32_t* lengths, int B, int T, int H, int d_v, int L, int W,
+                            int dtype, float* rho, cudaStream_t stream);
+bool chunk_tc_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
+cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream);
+}  // namespace prism
+
+namespace {
+
+// One status word per device: kernels record PRISM_ERR_TIMEOUT here when a
+// bounded wait gives up; prism_stream_status reads and clears it.
+__device__ int g_status_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+int* g_status_ptr[kMaxDevices] = {};
+int g_arch_ok[kMaxDevices] = {};  // 0 unknown, 1 sm_100, -1 other
+constexpr long long kDefaultSpinLimit = 1ll << 26;
+std::atomic<long long> g_spin_limit{kDefaultSpinLimit};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+// Device-side status word address and architecture check for the current device.
+int device_setup(int** status_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PRISM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_arch_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return PRISM_ERR_CUDA;
+    g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  if (g_arch_ok[dev] != 1) return PRISM_ERR_UNSUPPORTED;
+  if (!g_status_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return PRISM_ERR_CUDA;
+    g_status_ptr[dev] = static_cast<int*>(ptr);
+  }
+  *status_out = g_status_ptr[dev];
+  return PRISM_OK;
+}
+
+int check_sizes(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype) {
+  if (B < 1 || T < 1 || H < 1 || d_k < 1 || d_v < 1 || L < 1 || W < 1 || chunk < 1)
+    return PRISM_ERR_INVALID_ARG;
+  if (dtype != PRISM_BF16 && dtype != PRISM_FP32) return PRISM_ERR_INVALID_ARG;
+  if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return PRISM_ERR_UNSUPPORTED;
+  if (L > PRISM_MAX_L || W > PRISM_MAX_W) return PRISM_ERR_UNSUPPORTED;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return PRISM_ERR_UNSUPPORTED;
+  // element counts must fit the 64-bit index arithmetic with a wide margin
+  const double elems = (double)B * T * H * (double)(L > 1 ? L - 1 : 1) * (d_k > d_v ? d_k : d_v);
+  if (elems > 9.0e15) return PRISM_ERR_UNSUPPORTED;
+  return PRISM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int prism_version(void) {
+  return (PRISM_VERSION_MAJOR << 16) | (PRISM_VERSION_MINOR << 8) | PRISM_VERSION_PATCH;
+}
+
+const char* prism_status_string(int code) {
+  switch (code) {
+    case PRISM_OK: return "PRISM_OK";
+    case PRISM_ERR_INVALID_ARG: return "PRISM_ERR_INVALID_ARG: a required pointer is NULL or a size is out of range";
+    case PRISM_ERR_UNSUPPORTED: return "PRISM_ERR_UNSUPPORTED: valid arguments this build does not implement (head size, width, chunk, alignment or device)";
+    case PRISM_ERR_WORKSPACE: return "PRISM_ERR_WORKSPACE: workspace smaller than prism_scan_fwd_workspace_size()";
+    case PRISM_ERR_CUDA: return "PRISM_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+    case PRISM_ERR_TIMEOUT: return "PRISM_ERR_TIMEOUT: a bounded device-side wait expired";
+    default: return "PRISM: unknown status code";
+  }
+}
+
+void prism_set_spin_limit(long long limit) {
+  g_spin_limit.store(limit > 0 ? limit : kDefaultSpinLimit);
+}
+
+size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
+                                     int dtype) {
+  (void)B; (void)T; (void)H; (void)d_k; (void)d_v; (void)L; (void)W; (void)chunk; (void)dtype;
+  return 0;
+}
+
+int prism_scan_fwd(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
+                   const void* u, const float* alpha, const void* gain, const float* conv_w,
+                   const float* S0, const int32_t* lengths, int B, int T, int H, int d_k, int d_v,
+                   int L, int W, int chunk, int dtype, void* o, float* S_final, void* workspace,
+                   size_t workspace_bytes, prism_stream_t stream) {
+  int rc = check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype);
+  if (rc != PRISM_OK) return rc;
+  if (!q || !k || !v || !gamma || !beta || !conv_w || !o) return PRISM_ERR_INVALID_ARG;
+  if (L > 1 && (!u || !alpha || !gain)) return PRISM_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, gamma, beta, conv_w, o, S0, lengths, S_final,
+                        L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return PRISM_ERR_UNSUPPORTED;
+  const size_t need = prism_scan_fwd_workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return PRISM_ERR_WORKSPACE;
+  int* status = nullptr;
+  rc = device_setup(&status);
+  if (rc != PRISM_OK) return rc;
+
+  prism::ScanParams p{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr,
+                      L > 1 ? gain : nullptr, conv_w, S0, lengths, o, S_final,
+                      B, T, H, d_k, d_v, L, W, chunk, status, g_spin_limit.load()};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err;
+  if (prism::chunk_tc_supported(d_k, d_v, L, W, chunk, dtype))
+    err = prism::launch_chunk_tc(p, s);
+  else
+    err = prism::launch_recurrent_scan(p, dtype, s);
+  return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+int prism_scan_fwd_host(const void* host_q, const void* host_k, const void* host_v, const float* host_gamma,
+                        const float* host_beta, const void* host_u, const float* host_alpha, const void* host_gain,
+                        const float* host_conv_w, const float* host_S0, const int32_t* host_lengths, void* dev_q,
+                        void* dev_k, void* dev_v, float* dev_gamma, float* dev_beta, void* dev_u, float* dev_alpha,
+                        void* dev_gain, float* dev_conv_w, float* dev_S0, int32_t* dev_lengths, int B, int T,
+                        int H, int dk, int dv, int L, int W, int chunk, int dtype, void* dev_o,
+                        float* dev_S_final, void* host_o, float* host_S_final, void* workspace,
+                        size_t workspace_bytes, prism_stream_t stream) {
+  int rc = check_sizes(B, T, H, dk, dv, L, W, chunk, dtype);
+  if (rc != PRISM_OK) return rc;
+  if (!host_q || !host_k || !host_v || !host_gamma || !host_beta || !host_conv_w || !host_o) return PRISM_ERR_INVALID_ARG;
+  if (L > 1 && (!host_u || !host_alpha || !host_gain)) return PRISM_ERR_INVALID_ARG;
+  if ((host_S0 && !dev_S0) || (host_lengths && !dev_lengths)) return PRISM_ERR_INVALID_ARG;
+  const size_t es = dtype == PRISM_FP32 ? 4 : 2;
+  const size_t toks = (size_t)B * T * H;
+  const size_t m = (size_t)(L - 1);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  struct Copy { void* dst; const void* src; size_t bytes; };
+  const Copy in[] = {
+      {dev_q, host_q, toks * dk * es}, {dev_k, host_k, toks * dk * es}, {dev_v, host_v, toks * dv * es},
+      {dev_gamma, host_gamma, toks * 4}, {dev_beta, host_beta, toks * 4},
+      {dev_u, L > 1 ? host_u : nullptr, toks * m * dk * es}, {dev_alpha, L > 1 ? host_alpha : nullptr, toks * m * 4},
+      {dev_gain, L > 1 ? host_gain : nullptr, toks * m * dv * es},
+      {dev_conv_w, host_conv_w, (size_t)H * dv * W * 4},
+      {dev_S0, host_S0, (size_t)B * H * dv * dk * 4}, {dev_lengths, host_lengths, (size_t)B * 4}};
+  for (const Copy& c : in) {
+    if (!c.src || c.bytes == 0) continue;
+    if (!c.dst) return PRISM_ERR_INVALID_ARG;
+    if (cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return PRISM_ERR_CUDA;
+  }
+  rc = prism_scan_fwd(dev_q, dev_k, dev_v, dev_gamma, dev_beta, dev_u, dev_alpha, dev_gain, dev_conv_w,
+                      host_S0 ? dev_S0 : nullptr, host_lengths ? dev_lengths : nullptr, B, T, H, dk, dv, L, W,
+                      chunk, dtype, dev_o, host_S_final ? dev_S_final : nullptr, workspace, workspace_bytes,
+                      stream);
+  if (rc != PRISM_OK) return rc;
+  if (cudaMemcpyAsync(host_o, dev_o, toks * dv * es, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return PRISM_ERR_CUDA;
+  if (host_S_final && dev_S_final &&
+      cudaMemcpyAsync(host_S_final, dev_S_final, (size_t)B * H * dv * dk * 4, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess)
+    return PRISM_ERR_CUDA;
+  return PRISM_OK;
+}
+
+int prism_prologue_fwd(const void* v, const float* alpha, const void* gain, const float* conv_w,
+                       const int32_t* lengths, int B, int T, int H, int d_v, int L, int W, int dtype,
+                       float* rho_out, prism_stream_t stream) {
+  int rc = check_sizes(B, T, H, d_v, d_v, L, W, 64, dtype);
+  if (rc != PRISM_OK) return rc;
+  if (L < 2 || !v || !alpha || !gain || !conv_w || !rho_out) return PRISM_ERR_INVALID_ARG;
+  const void* ptrs[] = {v, alpha, gain, conv_w, lengths, rho_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return PRISM_ERR_UNSUPPORTED;
+  int* status = nullptr;
+  rc = device_setup(&status);
+  if (rc != PRISM_OK) return rc;
+  cudaError_t err = prism::launch_prologue(v, alpha, gain, conv_w, lengths, B, T, H, d_v, L, W, dtype,
+                                           rho_out, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype) {
+  if (check_sizes(1, 1, 1, d_k, d_v, L, W, chunk, dtype) != PRISM_OK) return 0;
+  return prism::chunk_tc_supported(d_k, d_v, L, W, chunk, dtype) ? 1 : 0;
+}
+
+int prism_stream_status(prism_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return PRISM_ERR_CUDA;
+  int* status = nullptr;
+  int rc = device_setup(&status);
+  if (rc != PRISM_OK) return rc;
+  int value = 0, zero = 0;
+  if (cudaMemcpy(&value, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (value != PRISM_OK && cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return PRISM_ERR_CUDA;
+  return value;
+}
+
+}  // extern "C"

@@ -1,0 +1,97 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/prism.h declares, and rejects bad arguments before it
+touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_sequence_shortconv_b200 as prism
+from linear_attention_sequence_shortconv_b200 import build as prism_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "prism.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    prism_build.build()
+    return prism.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(prism_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(prism.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_version_matches_header(L):
+    text = open(HEADER).read()
+    ver = tuple(int(re.search(rf"#define PRISM_VERSION_{k}\s+(\d+)", text).group(1)) for k in ("MAJOR", "MINOR", "PATCH"))
+    assert prism.version() == ver
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert prism.status_string(code).startswith("PRISM")
+    assert "unknown" in prism.status_string(99)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails before any CUDA call
+
+
+def call(lib_, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, gamma=FAKE, beta=FAKE, u=FAKE, alpha=FAKE, gain=FAKE, conv_w=FAKE,
+             S0=None, lengths=None, B=2, T=8, H=2, d_k=64, d_v=64, L=4, W=4, chunk=64, dtype=0,
+             o=FAKE, S_final=None)
+    a.update(kw)
+    return lib_.prism_scan_fwd(a["q"], a["k"], a["v"], a["gamma"], a["beta"], a["u"], a["alpha"], a["gain"],
+                            a["conv_w"], a["S0"], a["lengths"], a["B"], a["T"], a["H"], a["d_k"], a["d_v"],
+                            a["L"], a["W"], a["chunk"], a["dtype"], a["o"], a["S_final"], None, 0, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), 1), (dict(T=0), 1), (dict(H=-1), 1), (dict(L=0), 1), (dict(W=0), 1), (dict(dtype=7), 1),
+    (dict(q=None), 1), (dict(o=None), 1), (dict(conv_w=None), 1), (dict(u=None), 1), (dict(alpha=None), 1),
+    (dict(d_k=48), 2), (dict(d_v=256), 2), (dict(L=17), 2), (dict(W=9), 2), (dict(chunk=48), 2),
+    (dict(chunk=128), 2), (dict(q=FAKE + 8), 2), (dict(gamma=FAKE + 4), 2), (dict(S_final=FAKE + 2), 2),
+])
+def test_invalid_arguments(L, kw, code):
+    assert call(L, **kw) == code
+
+
+def test_L1_needs_no_residual_inputs(L):
+    # L = 1 ignores u/alpha/gain: with them NULL the checks pass up to the first
+    # device query, so only check that NULL residual inputs are not rejected as
+    # invalid when a size error is also present (the size error wins).
+    assert call(L, L=1, u=None, alpha=None, gain=None, B=0) == 1
+
+
+def test_workspace_size_query(L):
+    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) >= 0
+
+
+def test_prologue_invalid_arguments(L):
+    rc = L.prism_prologue_fwd(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 64, 1, 4, 0, FAKE, None)
+    assert rc == 1   # L must be >= 2
+    rc = L.prism_prologue_fwd(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 64, 4, 4, 0, FAKE + 4, None)
+    assert rc == 2   # misaligned output
+
+
+def test_host_entry_invalid_arguments(L):
+    args = [FAKE] * 11 + [FAKE] * 11 + [2, 8, 2, 64, 64, 4, 4, 64, 0] + [FAKE, FAKE, FAKE, FAKE, None, 0, None]
+    bad = list(args)
+    bad[0] = None      # host q
+    assert L.prism_scan_fwd_host(*bad) == 1
+    bad = list(args)
+    bad[22] = 0        # B = 0
+    assert L.prism_scan_fwd_host(*bad) == 1

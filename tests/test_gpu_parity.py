@@ -1,0 +1,180 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Bars (max-abs-relative error, per (batch, head) slice): 2e-2 for bf16 inputs
+and outputs with fp32 accumulation, 1e-4 for the fp32 build.  The oracle
+consumes exactly the (already rounded) inputs the GPU sees.
+"""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_sequence_shortconv_b200 import synth
+from oracle import gdn_seq, max_abs_rel_err, residual_chain
+from tests.helpers import TOL, gpu_run, oracle_run, rel_err
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+
+# Reduced versions of every workload: several chunks, a ragged tail (T not a
+# multiple of 64), and the same head sizes, L, W and dtypes as the full ones.
+REDUCED = {
+    "tiny_fp32": W["tiny_fp32"],
+    "tiny_fp32_s0": W["tiny_fp32"].replace(with_s0=True, seed=1),
+    "gdn_l1": W["gdn_l1"].replace(B=2, T=300, H=2),
+    "recsys": W["recsys"].replace(B=6, T=333, lengths_lo=40),
+    "lm_130m": W["lm_130m"].replace(B=2, T=200, H=3, with_s0=True),
+    "long_ctx": W["long_ctx"].replace(T=150, H=2),
+    "lm_fp32": W["lm_130m"].replace(B=1, T=130, H=2, dtype="fp32"),
+    "d32_L16_W8": synth.Workload("d32", B=2, T=97, H=3, d_k=32, d_v=32, L=16, chunk=32, W=8),
+    "dk64_dv128_W1": synth.Workload("mixed", B=1, T=77, H=2, d_k=64, d_v=128, L=3, chunk=64, W=1),
+}
+
+
+@pytest.mark.parametrize("name", list(REDUCED))
+def test_parity_reduced(name):
+    w = REDUCED[name]
+    inp = synth.make_inputs(w)
+    o, S = gpu_run(inp, w)
+    o_ref, S_ref = oracle_run(inp, w)
+    tol = TOL[w.dtype]
+    assert max_abs_rel_err(o, o_ref) <= tol, name
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= tol, name
+    if w.lengths_lo is not None:
+        lens = inp["lengths"].numpy()
+        for b, n in enumerate(lens):
+            assert np.all(o[b, n:] == 0)
+
+
+def test_L1_full_config_equals_plain_gdn():
+    """The L = 1 workload (B=4, H=4, T=1024, d=64, bf16) against the separately
+    written gated-delta recurrence."""
+    w = W["gdn_l1"]
+    inp = synth.make_inputs(w)
+    o, S = gpu_run(inp, w)
+    x = synth.to_float64_numpy(inp)
+    o_ref, S_ref = gdn_seq(x["q"], x["k"], x["v"], x["gamma"], x["beta"])
+    assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("name,pairs", [
+    ("lm_130m", [(0, 0), (7, 3), (15, 5)]),
+    ("recsys", [(0, 0), (77, 1), (127, 0)]),
+])
+def test_parity_full_size_sampled(name, pairs):
+    """Full-size workloads in the launch configuration the bench times; the
+    oracle evaluates a sample of (batch, head) chains over the whole sequence."""
+    w = W[name]
+    inp = synth.make_inputs(w)
+    o, S = gpu_run(inp, w)
+    outs, states = oracle_run(inp, w, bh=pairs)
+    for (b, h), o_ref, S_ref in zip(pairs, outs, states):
+        assert rel_err(o[b, :, h], o_ref) <= TOL[w.dtype], (b, h)
+        assert rel_err(S[b, h], S_ref) <= TOL[w.dtype], (b, h)
+
+
+def test_long_context_full_size_final_state_sampled():
+    """Long context (B=1, T=65536, H=8, d=128, L=8): outputs and the returned
+    final state of one head against the oracle over all 65536 steps."""
+    w = W["long_ctx"]
+    inp = synth.make_inputs(w)
+    o, S = gpu_run(inp, w)
+    outs, states = oracle_run(inp, w, bh=[(0, 5)])
+    assert rel_err(o[0, :, 5], outs[0]) <= TOL["bf16"]
+    assert rel_err(S[0, 5], states[0]) <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("T", [1, 2, 3, 63, 64, 65])
+def test_short_and_boundary_lengths(T):
+    w = synth.Workload("edge", B=2, T=T, H=2, d_k=64, d_v=64, L=4, chunk=64, with_s0=True)
+    inp = synth.make_inputs(w)
+    o, S = gpu_run(inp, w)
+    o_ref, S_ref = oracle_run(inp, w)
+    assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
+
+
+def test_empty_and_full_rows_in_one_batch():
+    """lengths = 0 (empty row: o = 0, S_final = S0), 1, T-1 and T in one batch."""
+    w = synth.Workload("ragged", B=4, T=130, H=2, d_k=128, d_v=128, L=4, chunk=64, with_s0=True)
+    inp = synth.make_inputs(w)
+    inp["lengths"] = torch.tensor([0, 1, 129, 130], dtype=torch.int32)
+    o, S = gpu_run(inp, w)
+    o_ref, S_ref = oracle_run(inp, w)
+    assert np.all(o[0] == 0)
+    np.testing.assert_array_equal(S[0], inp["S0"][0].numpy())
+    assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
+
+
+def test_bitwise_deterministic():
+    w = W["lm_130m"].replace(B=3, T=257, H=2)
+    inp = synth.make_inputs(w)
+    o1, S1 = gpu_run(inp, w)
+    o2, S2 = gpu_run(inp, w)
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+
+
+def test_state_only_optional():
+    w = REDUCED["lm_130m"]
+    inp = synth.make_inputs(w)
+    o1, _ = gpu_run(inp, w, want_state=False)
+    o2, _ = gpu_run(inp, w)
+    assert np.array_equal(o1, o2)
+
+
+# ---------------------------------------------------------------- prologue
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_prologue_kernel(dtype):
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    w = synth.Workload("pro", B=3, T=70, H=2, d_k=64, d_v=64, L=5, chunk=64, lengths_lo=10, dtype=dtype)
+    inp = synth.make_inputs(w)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    rho = prism.prologue_fwd(d["v"], d["alpha"], d["gain"], d["conv_w"], L=w.L, lengths=d["lengths"])
+    torch.cuda.synchronize()
+    x = synth.to_float64_numpy(inp)
+    ref = x["alpha"][..., None] * residual_chain(x["v"], x["conv_w"], x["gain"])
+    valid = np.arange(w.T)[None, :] < x["lengths"][:, None]
+    ref = np.where(valid[:, :, None, None, None], ref, 0.0)
+    got = rho.cpu().numpy()
+    assert np.abs(got - ref).max() <= 1e-5 * max(np.abs(ref).max(), 1.0)
+
+
+# ---------------------------------------------------------------- host entry point
+def test_host_entry_point_matches_device_entry_point():
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    w = REDUCED["recsys"]
+    inp = synth.make_inputs(w)
+    o_dev, S_dev = gpu_run(inp, w)
+    host = {n: (t.pin_memory() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    host["o"] = torch.empty(o_dev.shape, dtype=torch.bfloat16).pin_memory()
+    host["S_final"] = torch.empty(S_dev.shape, dtype=torch.float32).pin_memory()
+    dev = {n: torch.empty_like(t, device="cuda") for n, t in host.items() if isinstance(t, torch.Tensor)}
+    prism.scan_fwd_host(host, dev, L=w.L, chunk=w.chunk)
+    torch.cuda.synchronize()
+    assert np.array_equal(host["o"].float().numpy(), o_dev)
+    assert np.array_equal(host["S_final"].numpy(), S_dev)
+
+
+# ---------------------------------------------------------------- errors
+def test_argument_errors_raise_before_launch():
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    w = REDUCED["lm_130m"]
+    inp = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in synth.make_inputs(w).items()}
+    with pytest.raises(prism.PrismError) as e:
+        prism.scan_fwd(inp["q"], inp["k"], inp["v"], inp["gamma"], inp["beta"], inp["u"], inp["alpha"],
+                       inp["gain"], inp["conv_w"], L=w.L, chunk=48)
+    assert e.value.code == 2
+    misaligned = inp["q"].data_ptr() + 2
+    rc = prism.lib().prism_scan_fwd(misaligned, inp["k"].data_ptr(), inp["v"].data_ptr(),
+                                    inp["gamma"].data_ptr(), inp["beta"].data_ptr(), inp["u"].data_ptr(),
+                                    inp["alpha"].data_ptr(), inp["gain"].data_ptr(), inp["conv_w"].data_ptr(),
+                                    None, None, 1, 8, 1, 128, 128, 4, 4, 64, 0,
+                                    inp["v"].data_ptr(), None, None, 0, None)
+    assert rc == 2
+    assert prism.stream_status() == 0
