@@ -351,6 +351,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="lm_130m")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (smaller profiling captures)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -360,6 +362,8 @@ def main():
     from linear_attention_sequence_shortconv_b200 import synth
 
     w = synth.WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = w.replace(B=args.batch, name=f"{w.name}_b{args.batch}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

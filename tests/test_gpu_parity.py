@@ -178,3 +178,33 @@ def test_argument_errors_raise_before_launch():
                                     inp["v"].data_ptr(), None, None, 0, None)
     assert rc == 2
     assert prism.stream_status() == 0
+
+
+# ---------------------------------------------------------------- paths and device-side errors
+def test_tensor_core_path_is_taken_for_the_benchmarked_shapes():
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    for name in ("lm_130m", "recsys", "gdn_l1"):
+        w = W[name]
+        assert prism.uses_tensor_cores(w.d_k, w.d_v, w.L, w.W, w.chunk, prism.PRISM_BF16), name
+    assert not prism.uses_tensor_cores(128, 128, 4, 4, 64, prism.PRISM_FP32)
+
+
+def test_bounded_wait_timeout_is_reported_and_recovers():
+    """A spin limit of one poll makes the chunk kernel's first wait give up: the
+    kernel records PRISM_ERR_TIMEOUT, drains its own copies, frees TMEM and
+    exits; the context stays usable and the next call is correct."""
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    w = REDUCED["lm_130m"]
+    inp = synth.make_inputs(w)
+    prism.set_spin_limit(1)
+    try:
+        gpu_run(inp, w)
+        assert prism.stream_status() == 5
+    finally:
+        prism.set_spin_limit(0)
+    assert prism.stream_status() == 0
+    o, S = gpu_run(inp, w)
+    o_ref, S_ref = oracle_run(inp, w)
+    assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
