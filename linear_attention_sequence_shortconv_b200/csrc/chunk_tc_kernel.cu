@@ -47,7 +47,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kC = 64;           // chunk length
-constexpr int kThreads = 256;    // 8 warps: warp w reads TMEM lanes 32*(w%4).., column half w/4
+constexpr int kThreads = 512;    // 16 warps: warp w reads TMEM lanes 32*(w%4).., column quarter w/4
 constexpr uint32_t kAtom = 16384;  // one 128-row, 128-byte-wide swizzle atom column
 constexpr long long kDrainLimit = 1ll << 26;
 
@@ -66,15 +66,15 @@ struct Layout {
   static constexpr uint32_t SZ_BQ = M * kAtom;  // [Bku;QU] (128 x 64m), later P~ (64m x D)
   static constexpr uint32_t OFF_TQ = OFF_BQ + SZ_BQ;
   static constexpr uint32_t OFF_SXA = OFF_TQ + kAtom;  // S bf16 | A,T fp32 | X^T, Delta~^T
-  static constexpr uint32_t OFF_SMALL = OFF_SXA + 2 * kAtom;
-  static constexpr uint32_t BYTES = OFF_SMALL + 1024;
+  static constexpr uint32_t OFF_SMALL = OFF_SXA + 2 * kAtom;  // gate tables, barriers
+  static constexpr uint32_t BYTES = OFF_SMALL + 2048;
   // + alignment slack; never below 116 KB so that one CTA (and one 512-column TMEM
   // allocation) is resident per SM
   static constexpr uint32_t SMEM_ALLOC = (BYTES + 1024 > 116u * 1024u) ? BYTES + 1024 : 116u * 1024u;
   static_assert(SMEM_ALLOC <= 232448, "exceeds the 227 KB opt-in shared memory of sm_100");
   static constexpr int LDA = 68;  // fp32 row stride of A / T in the SXA region
   static_assert(SZ_BQ >= SZ_P, "P~ must fit where [Bku;QU] was");
-  static_assert(64 * LDA * 4 + 3 * 256 * 4 <= 2 * kAtom, "A/T + Y scratch must fit in SXA");
+  static_assert(64 * LDA * 4 + 1024 * 4 <= 2 * kAtom, "A/T + inverse scratch must fit in SXA");
 };
 
 struct TcArgs {
@@ -119,6 +119,24 @@ __device__ __forceinline__ void ld_bf16x8(const __nv_bfloat16* p, float* x) {
   }
 }
 
+__device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* x) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float2 f = __bfloat1622float2(h[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+}
+
+// element e (0..7) of 8 packed bf16
+__device__ __forceinline__ float bf16_at(const uint4& u, int e) {
+  const uint32_t w = e < 2 ? u.x : e < 4 ? u.y : e < 6 ? u.z : u.w;
+  return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+
 // Warp-uniform bounded wait (lane 0 polls, the result is broadcast).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit, int* status) {
   bool ok = true;
@@ -136,7 +154,8 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t base, int kk, uint32_t lbo) 
 template <int D, int M>
 __global__ void __launch_bounds__(kThreads, 1)
     prism_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                          const __grid_constant__ CUtensorMap map_u, TcArgs p) {
+                          const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_v,
+                          const __grid_constant__ CUtensorMap map_g, TcArgs p) {
   using Ly = Layout<D, M>;
   constexpr int NA = Ly::NA, UR = Ly::UR, LDA = Ly::LDA;
   extern __shared__ uint8_t smem_raw[];
@@ -147,21 +166,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sBQ = sm + Ly::OFF_BQ;
   uint8_t* sTQ = sm + Ly::OFF_TQ;
   uint8_t* sSXA = sm + Ly::OFF_SXA;
-  float* sG = reinterpret_cast<float*>(sm + Ly::OFF_SMALL);  // [64] cumulative log decay
-  float* sBeta = sG + 64;                                     // [64]
-  float* sCdec = sG + 128;                                    // [64] exp(G_63 - G_i)
-  uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + Ly::OFF_SMALL + 768);
+  float* sG = reinterpret_cast<float*>(sm + Ly::OFF_SMALL);  // [2][64] in-chunk cumulative log decay
+  float* sBeta = sG + 128;                                    // [2][64]
+  float* sCdec = sG + 256;                                    // [64] exp(G_63 - G_t)
+  float* sEp = sG + 320;                                      // [64] exp(G_t)
+  float* sEn = sG + 384;                                      // [64] exp(-G_t) (fast path only)
+  uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + Ly::OFF_SMALL + 1792);
   uint64_t* bar_mma = bar_load + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_load + 2);
   int* s_abort = reinterpret_cast<int*>(bar_load + 3);
-  float* sA = reinterpret_cast<float*>(sSXA);          // [64][LDA] fp32: A, then T in place
-  float* sY = sA + 64 * LDA;                           // [3][16][16] fp32 scratch of the inverse
-  uint8_t* sX = sSXA;                                  // X^T      bf16 [128][64] K-major
-  uint8_t* sDl = sSXA + kAtom;                         // Delta~^T bf16 [128][64] K-major
+  float* sA = reinterpret_cast<float*>(sSXA);  // [64][LDA] fp32: A, then T in place
+  float* sY = sA + 64 * LDA;                   // inverse scratch (<= 32x32 fp32)
+  uint8_t* sX = sSXA;                          // X^T      bf16 [128][64] K-major
+  uint8_t* sDl = sSXA + kAtom;                 // Delta~^T bf16 [128][64] K-major
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q4 = warp & 3, hf = warp >> 2;
-  const int row = 32 * q4 + lane;  // TMEM lane of this thread
+  const int q4 = warp & 3, cq = warp >> 2;  // TMEM lane quarter, column quarter
+  const int row = 32 * q4 + lane;           // TMEM lane of this thread
+  const bool srow = q4 < 2 * NA;            // this warp owns state rows c = row < D
   const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
   const int T = p.T, H = p.H;
   const int len = p.lengths ? min(max(p.lengths[b], 0), T) : T;
@@ -175,7 +197,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     *s_abort = 0;
     tma_prefetch_desc(&map_q);
     tma_prefetch_desc(&map_k);
-    if (M > 0) tma_prefetch_desc(&map_u);
+    tma_prefetch_desc(&map_v);
+    if (M > 0) {
+      tma_prefetch_desc(&map_u);
+      tma_prefetch_desc(&map_g);
+    }
   }
   if (warp == 0) {
     tmem_alloc(s_tmem, 512);
@@ -187,12 +213,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *s_tmem;
   const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);  // this warp's lane base
   constexpr uint32_t R1 = 0, D3 = 256, RS = 384;
+  constexpr int SP = D / 64;  // 16-column pieces of a state-row quarter
 
   const uint32_t aKQ = smem_u32(sKQ), aU = smem_u32(sU), aP = smem_u32(sP), aBQ = smem_u32(sBQ);
   const uint32_t aTQ = smem_u32(sTQ), aS = smem_u32(sSXA), aX = smem_u32(sX), aDl = smem_u32(sDl);
   constexpr uint32_t kLoadBytes = 2 * NA * 8192 + NA * UR * 128;
   uint32_t ph_load = 0, ph_mma = 0;
-  // (thread 0) phase of a TMA batch / MMA commit that is in flight and not yet observed, or -1
+  // (thread 0) phase of a TMA batch / MMA commit in flight and not yet observed, or -1
   int load_inflight = -1, mma_inflight = -1;
 
   auto issue_loads = [&](int t0) {
@@ -204,57 +231,155 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (M > 0) tma_load_5d(sU + a * Ly::U_ATOM, &map_u, bar_load, 64 * a, 0, h, t0, b);
     }
   };
+  auto prefetch_tiles_l2 = [&](int t0) {
+#pragma unroll
+    for (int a = 0; a < NA; ++a) {
+      tma_prefetch_l2_4d(&map_k, 64 * a, h, t0, b);
+      tma_prefetch_l2_4d(&map_q, 64 * a, h, t0, b);
+      tma_prefetch_l2_4d(&map_v, 64 * a, h, t0, b);
+      if (M > 0) {
+        tma_prefetch_l2_5d(&map_u, 64 * a, 0, h, t0, b);
+        tma_prefetch_l2_5d(&map_g, 64 * a, 0, h, t0, b);
+      }
+    }
+  };
 
-  // ---- initial state: RS <- S0 (or 0), bf16 copy -> SXA (A operand of MMA3)
-  const bool lane_ok = row < D;  // state rows c in [0, D)
-  if (q4 < NA * 2) {             // warps that own real state rows (all for D=128, lanes < 64 for D=64)
+  constexpr int CPT = D / 8;           // threads per token in the prologue
+  constexpr int TPP = kThreads / CPT;  // tokens per prologue pass
+  const int pc8 = (tid % CPT) * 8;
+  // ShortConv taps of the prologue's 8 channels: conv_w[h, pc8 .. pc8+7, 0 .. W-1], contiguous
+  const float* cwp = p.conv_w + ((size_t)h * D + pc8) * p.W;
+
+  // Chunk prologue: gate prefix (warp 0) and rho_{i,l} = alpha_{i,l} r_{i,l} -> P (bf16).
+  auto prologue = [&](int n, int buf) {
+    const int t0 = n * kC;
+    const int nv = min(kC, len - t0);
+    if (warp == 0) {  // G_t = sum_{j<=t} log gamma_j; padded steps: gamma = 1, beta = 0
+      float lg[2], bt[2];
 #pragma unroll
-    for (int cc = 0; cc < D / 64; ++cc) {
-      const int j0 = hf * (D / 2) + 32 * cc;
-      float s[32];
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        const bool valid = t < nv;
+        const size_t th = ((size_t)b * T + t0 + t) * H + h;
+        lg[e] = valid ? __logf(__ldg(p.gamma + th)) : 0.f;
+        bt[e] = valid ? __ldg(p.beta + th) : 0.f;
+      }
+      float x = lg[0] + lg[1];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) s[e] = 0.f;
-      if (p.S0 && lane_ok) {
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+      }
+      sG[buf * 64 + 2 * lane] = x - lg[1];
+      sG[buf * 64 + 2 * lane + 1] = x;
+      sBeta[buf * 64 + 2 * lane] = bt[0];
+      sBeta[buf * 64 + 2 * lane + 1] = bt[1];
+    }
+    if (M > 0) {
+#pragma unroll 1
+      for (int pass = 0; pass < kC / TPP; ++pass) {
+        const int i = pass * TPP + tid / CPT;
+        const int t = t0 + i;
+        float r[8];
+        if (i < nv) {
+          // every global load of this pass first (independent requests in flight together)
+          const size_t th = ((size_t)b * T + t) * H + h;
+          const __nv_bfloat16* vp = p.v + th * D + pc8;
+          uint4 vraw[4];
+          vraw[0] = ldg16(vp);
+#pragma unroll
+          for (int w = 1; w < 4; ++w)
+            vraw[w] = (w < p.W && t - w >= 0) ? ldg16(vp - (size_t)w * H * D) : make_uint4(0u, 0u, 0u, 0u);
+          uint4 graw[M > 0 ? M : 1];
+          float al[M > 0 ? M : 1];
+#pragma unroll
+          for (int l = 0; l < M; ++l) {
+            graw[l] = ldg16(p.gain + (th * M + l) * D + pc8);
+            al[l] = __ldg(p.alpha + th * M + l);
+          }
+          if (p.W == 4) {  // taps of one channel are one aligned float4
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float4 c4 = __ldg(reinterpret_cast<const float4*>(cwp) + e);
+              const float v0 = bf16_at(vraw[0], e);
+              r[e] = v0 - (c4.x * v0 + c4.y * bf16_at(vraw[1], e) + c4.z * bf16_at(vraw[2], e) +
+                           c4.w * bf16_at(vraw[3], e));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float v0 = bf16_at(vraw[0], e);
+              float a = __ldg(cwp + e * p.W) * v0;
+#pragma unroll
+              for (int w = 1; w < 4; ++w)
+                if (w < p.W) a += __ldg(cwp + e * p.W + w) * bf16_at(vraw[w], e);
+              r[e] = v0 - a;
+            }
+          }
+#pragma unroll
+          for (int l = 0; l < M; ++l) {
+            float gg[8], rho[8];
+            unpack_bf16x8(graw[l], gg);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              r[e] *= 1.f - gg[e];
+              rho[e] = al[l] * r[e];
+            }
+            st_bf16x8(sP, sw128_offset(i * M + l, pc8, Ly::U_ATOM), rho);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) r[e] = 0.f;
+#pragma unroll
+          for (int l = 0; l < M; ++l) st_bf16x8(sP, sw128_offset(i * M + l, pc8, Ly::U_ATOM), r);
+        }
+      }
+    }
+  };
+
+  // ---- initial state: RS <- S0 (or 0), bf16 copy -> SXA (A operand of MMA3); chunk 0 prologue
+  if (srow) {
+#pragma unroll
+    for (int pc = 0; pc < SP; ++pc) {
+      const int j0 = cq * (D / 4) + 16 * pc;
+      float s[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) s[e] = 0.f;
+      if (p.S0) {
         const float4* src = reinterpret_cast<const float4*>(p.S0 + (((size_t)b * H + h) * D + row) * D + j0);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           float4 f = __ldg(src + e);
           s[4 * e] = f.x; s[4 * e + 1] = f.y; s[4 * e + 2] = f.z; s[4 * e + 3] = f.w;
         }
       }
-      tmem_st32(tl + RS + j0, s);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st_bf16x8(sSXA, sw128_offset(row, j0 + 8 * e, kAtom), s + 8 * e);
+      tmem_st16(tl + RS + j0, s);
+      st_bf16x8(sSXA, sw128_offset(row, j0, kAtom), s);
+      st_bf16x8(sSXA, sw128_offset(row, j0 + 8, kAtom), s + 8);
     }
   }
   if (tid == 0 && nchunks > 0) {
     issue_loads(0);
     load_inflight = (int)ph_load;
   }
+  if (nchunks > 0) prologue(0, 0);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
-
-  // ShortConv taps of the 8 channels this thread handles in the prologue
-  constexpr int CPT = D / 8;           // threads per token in the prologue
-  constexpr int TPP = kThreads / CPT;  // tokens per prologue pass
-  const int pc8 = (tid % CPT) * 8;
-  float cw[4][8];
-#pragma unroll
-  for (int w = 0; w < 4; ++w)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) cw[w][e] = (w < p.W) ? __ldg(p.conv_w + ((size_t)h * D + pc8 + e) * p.W + w) : 0.f;
 
   bool aborted = false;
   for (int n = 0; n < nchunks && !aborted; ++n) {
     const int t0 = n * kC;
     const int nv = min(kC, len - t0);
+    const int cur = n & 1;
+    const float* G = sG + cur * 64;
+    const float* Bt = sBeta + cur * 64;
 
-    // ---------------- A: wait for K,Q,U; MMA1 + MMA3; prologue; decay prefix
-    bool ok = warp_wait(bar_load, ph_load, lim, p.status);
+    // ---------------- A: wait for K,Q,U; MMA1 + MMA3; per-chunk decay tables; L2 prefetch of chunk n+1
     if (tid == 0) {
-      if (ok) load_inflight = -1;
+      const bool ok = mbar_wait(bar_load, ph_load, lim, p.status);
       if (ok) {
+        load_inflight = -1;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4 * NA; ++kk) {
@@ -267,124 +392,115 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16(tmem + D3, kdesc(aS, kk, kAtom), kdesc(aKQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
         mma_commit(bar_mma);
         mma_inflight = (int)ph_mma;
+        if (n + 1 < nchunks) prefetch_tiles_l2(t0 + kC);
+      } else {
+        *s_abort = 1;
       }
     }
     ph_load ^= 1;
-    if (!ok && lane == 0) atomicExch(s_abort, 1);
-    // in-chunk cumulative log decay and step sizes (padded steps: gamma = 1, beta = 0)
+    if (warp == 1 && n + 1 < nchunks) {
+      // the next chunk's gates are token-major spans [b, t0+64 .. t0+128, :]: prefetch their L2 lines
+      const int tn = t0 + kC, te = min(tn + kC, T);
+      const char* g0 = reinterpret_cast<const char*>(p.gamma + ((size_t)b * T + tn) * H);
+      const char* b0 = reinterpret_cast<const char*>(p.beta + ((size_t)b * T + tn) * H);
+      const char* a0 = reinterpret_cast<const char*>(p.alpha + ((size_t)b * T + tn) * H * (M > 0 ? M : 1));
+      const int gbytes = (te - tn) * H * 4, abytes = M > 0 ? gbytes * M : 0;
+      for (int off = lane * 128; off < gbytes; off += 32 * 128) {
+        prefetch_l2(g0 + off);
+        prefetch_l2(b0 + off);
+      }
+      for (int off = lane * 128; off < abytes; off += 32 * 128) prefetch_l2(a0 + off);
+    }
+    const bool fast = G[63] >= -60.f;  // exp(-G) stays finite: factor D[t,i] = e^{G_t} e^{-G_i}
     if (tid < 64) {
-      const bool valid = tid < nv;
-      const size_t th = ((size_t)b * T + t0 + tid) * H + h;
-      const float g = valid ? __logf(__ldg(p.gamma + th)) : 0.f;
-      float x = g;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += y;
-      }
-      sG[tid] = x;
-      sBeta[tid] = valid ? __ldg(p.beta + th) : 0.f;
+      sEp[tid] = __expf(G[tid]);
+      sEn[tid] = fast ? __expf(-G[tid]) : 0.f;
+      sCdec[tid] = __expf(G[63] - G[tid]);
     }
-    // prologue: rho_{i,l} = alpha_{i,l} prod_{j<=l}(1 - g_j) (v_i - sum_w cw_w v_{i-w}) -> P (bf16)
-    if (M > 0) {
-#pragma unroll 1
-      for (int pass = 0; pass < kC / TPP; ++pass) {
-        const int i = pass * TPP + tid / CPT;
-        const int t = t0 + i;
-        if (i < nv) {
-          float vv[8], r[8];
-          const size_t th = ((size_t)b * T + t) * H + h;
-          ld_bf16x8(p.v + th * D + pc8, vv);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) r[e] = vv[e] - cw[0][e] * vv[e];
-#pragma unroll
-          for (int w = 1; w < 4; ++w) {
-            if (w < p.W && t - w >= 0) {
-              float hv[8];
-              ld_bf16x8(p.v + (th - (size_t)w * H) * D + pc8, hv);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) r[e] -= cw[w][e] * hv[e];
-            }
-          }
-#pragma unroll
-          for (int l = 0; l < M; ++l) {
-            float gg[8], rho[8];
-            ld_bf16x8(p.gain + (th * M + l) * D + pc8, gg);
-            const float al = __ldg(p.alpha + th * M + l);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              r[e] *= 1.f - gg[e];
-              rho[e] = al * r[e];
-            }
-            st_bf16x8(sP, sw128_offset(i * M + l, pc8, Ly::U_ATOM), rho);
-          }
-        } else {
-          float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int l = 0; l < M; ++l) st_bf16x8(sP, sw128_offset(i * M + l, pc8, Ly::U_ATOM), z);
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid >= 32 && tid < 64) sG[tid] += sG[31];  // combine the two warp scans
     __syncthreads();
     if (*s_abort) { aborted = true; break; }
 
-    // ---------------- B: epilogue of MMA1 -> A (fp32), [Bku;QU], QK (bf16)
-    ok = warp_wait(bar_mma, ph_mma, lim, p.status);
+    // ---------------- B: epilogue of MMA1 -> A (fp32), [Bku;QU], QK (bf16); then issue MMA2
+    bool ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) mma_inflight = -1;
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
-    if (tid < 64) sCdec[tid] = __expf(sG[63] - sG[tid]);
     if (ok) {
       const bool krow = row < 64;
       const int t = krow ? row : row - 64;
-      const float Gt = sG[t];
-      const float bt = krow ? sBeta[t] : 1.f;
-      constexpr int NCH = (64 + UR) / 32;  // 32-column pieces of R1
-#pragma unroll 1
-      for (int ch = hf * (NCH / 2); ch < (hf + 1) * (NCH / 2); ++ch) {
-        const int j0 = 32 * ch;
-        float x[32];
-        tmem_ld32(tl + R1 + j0, x);
-        if (j0 < 64) {
+      const int tlim = krow ? t : t + 1;  // keep column i < tlim
+      const float Gt = G[t];
+      const float rs = (krow ? Bt[t] : 1.f) * sEp[t];
+      constexpr int NP = (64 + UR) / 16;  // 16-column pieces of R1
+      constexpr int PQ = NP / 4;           // pieces of this thread's column quarter
+      constexpr int PB = PQ >= 2 ? 2 : 1;  // pieces per TMEM wait
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = j0 + e;
-            const bool keep = krow ? (i < t) : (i <= t);
-            x[e] = keep ? bt * __expf(Gt - sG[i]) * x[e] : 0.f;
-          }
+      for (int pb = 0; pb < PQ; pb += PB) {
+      uint32_t raw[PB][16];
+#pragma unroll
+      for (int k = 0; k < PB; ++k)
+        if (pb + k < PQ) tmem_ld16_async(tl + R1 + 16 * (cq * PQ + pb + k), raw[k]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < PB; ++k) {
+        if (pb + k >= PQ) break;
+        const int pc = pb + k;
+        const int j0 = 16 * (cq * PQ + pc);
+        float x[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i = (j0 < 64) ? j0 + e : (j0 - 64 + e) / (M > 0 ? M : 1);
+          float f;
+          if (fast)
+            f = rs * sEn[i];
+          else
+            f = (krow ? Bt[t] : 1.f) * __expf(Gt - G[i]);
+          x[e] = (i < tlim) ? f * __uint_as_float(raw[k][e]) : 0.f;
+        }
+        if (j0 < 64) {
           if (krow) {
             float4* dst = reinterpret_cast<float4*>(sA + t * LDA + j0);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
           } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) st_bf16x8(sTQ, sw128_offset(row, j0 + 8 * e, kAtom), x + 8 * e);
+            st_bf16x8(sTQ, sw128_offset(row, j0, kAtom), x);
+            st_bf16x8(sTQ, sw128_offset(row, j0 + 8, kAtom), x + 8);
           }
         } else {
-          const int k0 = j0 - 64;  // column (i,l) = k0 + e
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = (k0 + e) / (M > 0 ? M : 1);
-            const bool keep = krow ? (i < t) : (i <= t);
-            x[e] = keep ? bt * __expf(Gt - sG[i]) * x[e] : 0.f;
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) st_bf16x8(sBQ, sw128_offset(row, k0 + 8 * e, kAtom), x + 8 * e);
+          st_bf16x8(sBQ, sw128_offset(row, j0 - 64, kAtom), x);
+          st_bf16x8(sBQ, sw128_offset(row, j0 - 56, kAtom), x + 8);
         }
+      }
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (*s_abort) { aborted = true; break; }
+    if (tid == 0 && M > 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < UR / 16; ++kk)
+        mma_bf16(tmem + R1, mndesc(aP, kk, Ly::U_ATOM), kdesc(aBQ, kk, kAtom), idesc_bf16(128, 128, 1, 0), kk > 0);
+    }
 
-    // ---------------- C: T = (I + A)^{-1} in place (fp32), blocked by 16
+    // ---------------- C: rescale RS by exp(G_63); T = (I + A)^{-1} in place (fp32); issue MMA QK*T
+    if (srow) {
+      const float blast = sEp[63];
+#pragma unroll
+      for (int pc = 0; pc < SP; ++pc) {
+        const int j0 = cq * (D / 4) + 16 * pc;
+        float s[16];
+        tmem_ld16(tl + RS + j0, s);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) s[e] *= blast;
+        tmem_st16(tl + RS + j0, s);
+      }
+    }
+    // ---------------- C1: inverse
     {
-      // diagonal 16x16 blocks: thread (blk, j) solves column j by forward substitution
+      // (1) diagonal 16x16 blocks: thread (blk, j) solves column j by forward substitution
       float xcol[16];
       const int blk = tid >> 4, j = tid & 15;
       if (tid < 64) {
@@ -392,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < 16; ++r) {
           float acc = 0.f;
 #pragma unroll
-          for (int s = 0; s < r; ++s) acc += sA[(16 * blk + r) * LDA + 16 * blk + s] * xcol[s];
+          for (int s2 = 0; s2 < r; ++s2) acc += sA[(16 * blk + r) * LDA + 16 * blk + s2] * xcol[s2];
           xcol[r] = (r < j) ? 0.f : (r == j ? 1.f : -acc);
         }
       }
@@ -402,27 +518,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < 16; ++r) sA[(16 * blk + r) * LDA + 16 * blk + j] = xcol[r];
       }
       __syncthreads();
-      // block rows I = 1..3: Y_IJ = sum_{K=J}^{I-1} A_IK T_KJ, then T_IJ = -T_II Y_IJ
-#pragma unroll 1
-      for (int I = 1; I < 4; ++I) {
-        for (int e = tid; e < 256 * I; e += kThreads) {
-          const int J = e >> 8, r = (e >> 4) & 15, s = e & 15;
-          float acc = 0.f;
-          for (int kx = 16 * J; kx < 16 * I; ++kx) acc += sA[(16 * I + r) * LDA + kx] * sA[kx * LDA + 16 * J + s];
-          sY[e] = acc;
-        }
+      // (2) 16 -> 32: T_{I,I-1} = -T_II A_{I,I-1} T_{I-1,I-1} for I = 1, 3
+      {
+        const int pr = tid >> 8, r = (tid >> 4) & 15, s2 = tid & 15;
+        const int I = 2 * pr + 1, J = 2 * pr;
+        float acc = 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) acc += sA[(16 * I + r) * LDA + 16 * J + u] * sA[(16 * J + u) * LDA + 16 * J + s2];
+        sY[tid] = acc;
         __syncthreads();
-        for (int e = tid; e < 256 * I; e += kThreads) {
-          const int J = e >> 8, r = (e >> 4) & 15, s = e & 15;
-          float acc = 0.f;
-          for (int u = 0; u <= r; ++u) acc += sA[(16 * I + r) * LDA + 16 * I + u] * sY[(J << 8) + (u << 4) + s];
-          sA[(16 * I + r) * LDA + 16 * J + s] = -acc;
-        }
+        acc = 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (u <= r) acc += sA[(16 * I + r) * LDA + 16 * I + u] * sY[(pr << 8) + (u << 4) + s2];
+        __syncthreads();
+        sA[(16 * I + r) * LDA + 16 * J + s2] = -acc;
         __syncthreads();
       }
+      // ---------------- C3: inverse 32 -> 64
+      // (3) 32 -> 64: T[32:64, 0:32] = -T2 (A21 T1).  256 threads, 4 rows x 1 column each:
+      // the 4 row operands are float4 broadcasts, the column operand a conflict-free scalar.
+      if (tid < 256) {
+        const int r0 = (tid >> 5) * 4, s2 = tid & 31;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int u = 0; u < 32; u += 4) {  // Y2 = A21 T1
+          float tc[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) tc[k] = sA[(u + k) * LDA + s2];
+#pragma unroll
+          for (int i2 = 0; i2 < 4; ++i2) {
+            const float4 a = *reinterpret_cast<const float4*>(sA + (32 + r0 + i2) * LDA + u);
+            acc[i2] += a.x * tc[0] + a.y * tc[1] + a.z * tc[2] + a.w * tc[3];
+          }
+        }
+#pragma unroll
+        for (int i2 = 0; i2 < 4; ++i2) sY[(r0 + i2) * 32 + s2] = acc[i2];
+      }
+      __syncthreads();
+      if (tid < 256) {
+        const int r0 = (tid >> 5) * 4, s2 = tid & 31;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int u = 0; u < 32; u += 4) {  // T21 = -T2 Y2 (T2's upper triangle is zero)
+          float yc[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) yc[k] = sY[(u + k) * 32 + s2];
+#pragma unroll
+          for (int i2 = 0; i2 < 4; ++i2) {
+            const float4 a = *reinterpret_cast<const float4*>(sA + (32 + r0 + i2) * LDA + 32 + u);
+            acc[i2] += a.x * yc[0] + a.y * yc[1] + a.z * yc[2] + a.w * yc[3];
+          }
+        }
+        // rows 32..63, columns 0..31 held A21, which step (3a) has consumed
+#pragma unroll
+        for (int i2 = 0; i2 < 4; ++i2) sA[(32 + r0 + i2) * LDA + s2] = -acc[i2];
+      }
+      __syncthreads();
       // T (fp32, lower incl. unit diagonal; upper part holds A's zeros) -> bf16 rows 0..63 of TQ
-      for (int e = tid; e < 64 * 8; e += kThreads) {
-        const int t = e >> 3, c8 = (e & 7) * 8;
+      {
+        const int t = tid >> 3, c8 = (tid & 7) * 8;
         const float4 lo = *reinterpret_cast<const float4*>(sA + t * LDA + c8);
         const float4 hi = *reinterpret_cast<const float4*>(sA + t * LDA + c8 + 4);
         const float v8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
@@ -430,33 +585,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
-
-    // ---------------- D: MMA QK*T and MMA2; rescale RS by exp(G_63)
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + R1 + 128, kdesc(aTQ, kk, kAtom), mndesc(aTQ, kk, kAtom), idesc_bf16(128, 64, 0, 1), kk > 0);
-      if (M > 0) {
-#pragma unroll
-        for (int kk = 0; kk < UR / 16; ++kk)
-          mma_bf16(tmem + R1, mndesc(aP, kk, Ly::U_ATOM), kdesc(aBQ, kk, kAtom), idesc_bf16(128, 128, 1, 0), kk > 0);
-      }
       mma_commit(bar_mma);
       mma_inflight = (int)ph_mma;
     }
-    const float blast = __expf(sG[63]);
-    if (q4 < NA * 2) {
+    // ---------------- D: loads for X while the MMAs run
+    // values of v this thread needs for X, loaded while the MMAs run
+    // (padded steps have beta = 0, so any in-range token may stand in for them)
+    float vreg[16];
+    {
+      const int tb = 16 * cq;
+      const int rr = srow ? row : 0;
+      __nv_bfloat16 raw[16];
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int j0 = hf * (D / 2) + 32 * cc;
-        float s[32];
-        tmem_ld32(tl + RS + j0, s);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[e] *= blast;
-        tmem_st32(tl + RS + j0, s);
+      for (int e = 0; e < 16; ++e) {
+        const int t = min(t0 + tb + e, T - 1);
+        raw[e] = p.v[(((size_t)b * T + t) * H + h) * D + rr];
       }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) vreg[e] = __bfloat162float(raw[e]);
     }
 
     // ---------------- E: QKT -> TQ rows 64..127; P~ = diag(c) P -> BQ; X^T -> SXA; O partial
@@ -465,13 +618,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0 && ok) mma_inflight = -1;
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
-    float opart[32];
     if (ok) {
-      if (q4 >= 2) {  // lanes 64..127 hold (QK T)[t, i], t = row - 64; column half hf
-        float x[32];
-        tmem_ld32(tl + R1 + 128 + 32 * hf, x);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) st_bf16x8(sTQ, sw128_offset(row, 32 * hf + 8 * e, kAtom), x + 8 * e);
+      float opart[16];
+      if (q4 >= 2) {  // lanes 64..127 hold (QK T)[t, i], t = row - 64
+        float x[16];
+        tmem_ld16(tl + R1 + 128 + 16 * cq, x);
+        st_bf16x8(sTQ, sw128_offset(row, 16 * cq, kAtom), x);
+        st_bf16x8(sTQ, sw128_offset(row, 16 * cq + 8, kAtom), x + 8);
       }
       if (M > 0) {
         for (int e = tid; e < UR * D / 8; e += kThreads) {
@@ -490,37 +643,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_bf16x8(sBQ, off, f);
         }
       }
-      if (q4 < NA * 2) {  // state rows c = row; tokens t = 32*hf + e
-        const int tb = 32 * hf;
-        float y[32], d2[32];
-        tmem_ld32(tl + D3 + tb, y);
-        if (M > 0) tmem_ld32(tl + R1 + tb, d2);
+      if (srow) {  // state row c = row; tokens t = 16*cq + e
+        const int tb = 16 * cq;
+        float y[16], d2[16];
+        tmem_ld16(tl + D3 + tb, y);
+        if (M > 0) tmem_ld16(tl + R1 + tb, d2);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int t = tb + e;
-          const float bet = sBeta[t];
-          const float vtc = (t < nv) ? __bfloat162float(p.v[(((size_t)b * T + t0 + t) * H + h) * D + row]) : 0.f;
-          float xv = bet * (vtc - __expf(sG[t]) * y[e]);
+        for (int e = 0; e < 16; ++e) {
+          float xv = Bt[tb + e] * (vreg[e] - sEp[tb + e] * y[e]);
           if (M > 0) xv -= d2[e];
           y[e] = xv;
         }
+        st_bf16x8(sX, sw128_offset(row, tb, kAtom), y);
+        st_bf16x8(sX, sw128_offset(row, tb + 8, kAtom), y + 8);
+        tmem_ld16(tl + D3 + 64 + tb, opart);
+        if (M > 0) tmem_ld16(tl + R1 + 64 + tb, d2);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) st_bf16x8(sX, sw128_offset(row, tb + 8 * e, kAtom), y + 8 * e);
-        tmem_ld32(tl + D3 + 64 + tb, opart);
-        if (M > 0) tmem_ld32(tl + R1 + 64 + tb, d2);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          opart[e] *= __expf(sG[tb + e]);
+        for (int e = 0; e < 16; ++e) {
+          opart[e] *= sEp[tb + e];
           if (M > 0) opart[e] += d2[e];
         }
+        tmem_st16(tl + D3 + 64 + tb, opart);  // parked until step G (no MMA writes D3 before then)
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (*s_abort) { aborted = true; break; }
-
-    // ---------------- F: MMA4 (Delta^T | (QKT X)^T) and MMA5a (RS += P~^T U)
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -535,33 +684,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_inflight = (int)ph_mma;
     }
 
-    // ---------------- G: Delta~^T -> SXA; o = O partial + (QKT X)
+    // ---------------- F: next chunk's prologue while MMA4 / MMA5a run (P_n is no longer read)
+    if (n + 1 < nchunks) prologue(n + 1, cur ^ 1);
+    fence_proxy_async_smem();
+
+    // ---------------- G: Delta~^T -> SXA; o = O partial + (QKT X); issue MMA5b
+    // (the prologue above has no barrier of its own; the wait below orders it)
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) mma_inflight = -1;
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
-    if (ok && q4 < NA * 2) {
-      const int tb = 32 * hf;
-      float x[32];
-      tmem_ld32(tl + R1 + 128 + tb, x);
+    if (ok && srow) {
+      const int tb = 16 * cq;
+      float x[16];
+      tmem_ld16(tl + R1 + 128 + tb, x);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) x[e] *= sCdec[tb + e];
+      for (int e = 0; e < 16; ++e) x[e] *= sCdec[tb + e];
+      st_bf16x8(sDl, sw128_offset(row, tb, kAtom), x);
+      st_bf16x8(sDl, sw128_offset(row, tb + 8, kAtom), x + 8);
+      float opart[16];
+      tmem_ld16(tl + R1 + 192 + tb, x);
+      tmem_ld16(tl + D3 + 64 + tb, opart);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) st_bf16x8(sDl, sw128_offset(row, tb + 8 * e, kAtom), x + 8 * e);
-      tmem_ld32(tl + R1 + 192 + tb, x);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
+      for (int e = 0; e < 16; ++e) {
         const int t = t0 + tb + e;
-        if (t < T) p.o[(((size_t)b * T + t) * H + h) * D + row] = __float2bfloat16_rn(tb + e < nv ? opart[e] + x[e] : 0.f);
+        if (t < T)
+          p.o[(((size_t)b * T + t) * H + h) * D + row] = __float2bfloat16_rn(tb + e < nv ? opart[e] + x[e] : 0.f);
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (*s_abort) { aborted = true; break; }
-
-    // ---------------- H: MMA5b (RS += Delta~^T K)
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -583,19 +738,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
-    if (ok && q4 < NA * 2) {
+    if (ok && srow) {
       const bool last = n + 1 == nchunks;
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int j0 = hf * (D / 2) + 32 * cc;
-        float s[32];
-        tmem_ld32(tl + RS + j0, s);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) st_bf16x8(sSXA, sw128_offset(row, j0 + 8 * e, kAtom), s + 8 * e);
+      for (int pc = 0; pc < SP; ++pc) {
+        const int j0 = cq * (D / 4) + 16 * pc;
+        float s[16];
+        tmem_ld16(tl + RS + j0, s);
+        st_bf16x8(sSXA, sw128_offset(row, j0, kAtom), s);
+        st_bf16x8(sSXA, sw128_offset(row, j0 + 8, kAtom), s + 8);
         if (last && p.S_final) {
           float4* dst = reinterpret_cast<float4*>(p.S_final + (((size_t)b * H + h) * D + row) * D + j0);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) dst[e] = make_float4(s[4 * e], s[4 * e + 1], s[4 * e + 2], s[4 * e + 3]);
+          for (int e = 0; e < 4; ++e) dst[e] = make_float4(s[4 * e], s[4 * e + 1], s[4 * e + 2], s[4 * e + 3]);
         }
       }
     }
@@ -607,15 +762,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (!aborted) {
     // rows with no valid token: S_final = S0 (still in RS); zero the outputs past the last chunk
-    if (nchunks == 0 && p.S_final && q4 < NA * 2) {
+    if (nchunks == 0 && p.S_final && srow) {
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int j0 = hf * (D / 2) + 32 * cc;
-        float s[32];
-        tmem_ld32(tl + RS + j0, s);
+      for (int pc = 0; pc < SP; ++pc) {
+        const int j0 = cq * (D / 4) + 16 * pc;
+        float s[16];
+        tmem_ld16(tl + RS + j0, s);
         float4* dst = reinterpret_cast<float4*>(p.S_final + (((size_t)b * H + h) * D + row) * D + j0);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dst[e] = make_float4(s[4 * e], s[4 * e + 1], s[4 * e + 2], s[4 * e + 3]);
+        for (int e = 0; e < 4; ++e) dst[e] = make_float4(s[4 * e], s[4 * e + 1], s[4 * e + 2], s[4 * e + 3]);
       }
     }
     const int tz = nchunks * kC;
@@ -673,24 +828,27 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
   });
   if (attr_err != cudaSuccess) return attr_err;
   const cuuint64_t B = p.B, T = p.T, H = p.H;
-  CUtensorMap mq, mk, mu;
+  CUtensorMap mq, mk, mu, mv, mg;
   const cuuint64_t dims4[4] = {(cuuint64_t)D, H, T, B};
   const cuuint64_t str4[3] = {(cuuint64_t)D * 2, H * D * 2, T * H * D * 2};
   const cuuint32_t box4[4] = {64, 1, 64, 1};
-  if (!encode(&mq, p.q, 4, dims4, str4, box4) || !encode(&mk, p.k, 4, dims4, str4, box4))
+  if (!encode(&mq, p.q, 4, dims4, str4, box4) || !encode(&mk, p.k, 4, dims4, str4, box4) ||
+      !encode(&mv, p.v, 4, dims4, str4, box4))
     return cudaErrorInvalidValue;
   if (M > 0) {
     const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)M, H, T, B};
     const cuuint64_t str5[4] = {(cuuint64_t)D * 2, (cuuint64_t)M * D * 2, H * M * D * 2, T * H * M * D * 2};
     const cuuint32_t box5[5] = {64, (cuuint32_t)M, 1, 64, 1};
-    if (!encode(&mu, p.u, 5, dims5, str5, box5)) return cudaErrorInvalidValue;
+    if (!encode(&mu, p.u, 5, dims5, str5, box5) || !encode(&mg, p.gain, 5, dims5, str5, box5))
+      return cudaErrorInvalidValue;
   } else {
     mu = mk;
+    mg = mk;
   }
   TcArgs a{static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha,
            static_cast<const __nv_bfloat16*>(p.gain), p.conv_w, p.S0, p.lengths,
            static_cast<__nv_bfloat16*>(p.o), p.S_final, p.B, p.T, p.H, p.W, p.status, p.spin_limit};
-  prism_chunk_tc_kernel<D, M><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, a);
+  prism_chunk_tc_kernel<D, M><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, a);
   return cudaGetLastError();
 }
 
