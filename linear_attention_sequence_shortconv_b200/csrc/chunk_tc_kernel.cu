@@ -78,6 +78,9 @@ struct Layout {
 };
 
 struct TcArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* u;
   const __nv_bfloat16* v;
   const float* gamma;
   const float* beta;
@@ -231,15 +234,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (M > 0) tma_load_5d(sU + a * Ly::U_ATOM, &map_u, bar_load, 64 * a, 0, h, t0, b);
     }
   };
-  auto prefetch_tiles_l2 = [&](int t0) {
+  // L2 prefetch of the next chunk's k, q, v (D bf16 per token) and u, gain (M*D bf16 per
+  // token): one 128-byte line per thread and request, spread over all threads.
+  auto prefetch_next_l2 = [&](int t0) {
+    constexpr int LK = D * 2 / 128, LU = M * D * 2 / 128;  // 128-byte lines per token
+    constexpr int LT = 3 * LK + 2 * LU;
+    const int i = tid & 63;
+    if (t0 + i < T) {
+      const size_t th = ((size_t)b * T + t0 + i) * H + h;
+      const char* kp = reinterpret_cast<const char*>(p.k + th * D);
+      const char* qp = reinterpret_cast<const char*>(p.q + th * D);
+      const char* vp = reinterpret_cast<const char*>(p.v + th * D);
+      const char* up = reinterpret_cast<const char*>(p.u + th * M * D);
+      const char* gp = reinterpret_cast<const char*>(p.gain + th * M * D);
 #pragma unroll
-    for (int a = 0; a < NA; ++a) {
-      tma_prefetch_l2_4d(&map_k, 64 * a, h, t0, b);
-      tma_prefetch_l2_4d(&map_q, 64 * a, h, t0, b);
-      tma_prefetch_l2_4d(&map_v, 64 * a, h, t0, b);
-      if (M > 0) {
-        tma_prefetch_l2_5d(&map_u, 64 * a, 0, h, t0, b);
-        tma_prefetch_l2_5d(&map_g, 64 * a, 0, h, t0, b);
+      for (int r = tid >> 6; r < LT; r += kThreads / 64) {
+        const char* ptr = r < LK ? kp + r * 128
+                        : r < 2 * LK ? qp + (r - LK) * 128
+                        : r < 3 * LK ? vp + (r - 2 * LK) * 128
+                        : r < 3 * LK + LU ? up + (r - 3 * LK) * 128
+                        : gp + (r - 3 * LK - LU) * 128;
+        prefetch_l2(ptr);
       }
     }
   };
@@ -280,58 +295,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int pass = 0; pass < kC / TPP; ++pass) {
         const int i = pass * TPP + tid / CPT;
         const int t = t0 + i;
-        float r[8];
+        // every global load of the pass first (independent requests in flight together)
+        uint4 vraw[4], graw[M > 0 ? M : 1];
+        float al[M > 0 ? M : 1];
         if (i < nv) {
-          // every global load of this pass first (independent requests in flight together)
           const size_t th = ((size_t)b * T + t) * H + h;
           const __nv_bfloat16* vp = p.v + th * D + pc8;
-          uint4 vraw[4];
           vraw[0] = ldg16(vp);
 #pragma unroll
           for (int w = 1; w < 4; ++w)
             vraw[w] = (w < p.W && t - w >= 0) ? ldg16(vp - (size_t)w * H * D) : make_uint4(0u, 0u, 0u, 0u);
-          uint4 graw[M > 0 ? M : 1];
-          float al[M > 0 ? M : 1];
 #pragma unroll
           for (int l = 0; l < M; ++l) {
             graw[l] = ldg16(p.gain + (th * M + l) * D + pc8);
             al[l] = __ldg(p.alpha + th * M + l);
           }
-          if (p.W == 4) {  // taps of one channel are one aligned float4
+        } else {  // padded step: rho = 0
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float4 c4 = __ldg(reinterpret_cast<const float4*>(cwp) + e);
-              const float v0 = bf16_at(vraw[0], e);
-              r[e] = v0 - (c4.x * v0 + c4.y * bf16_at(vraw[1], e) + c4.z * bf16_at(vraw[2], e) +
-                           c4.w * bf16_at(vraw[3], e));
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float v0 = bf16_at(vraw[0], e);
-              float a = __ldg(cwp + e * p.W) * v0;
-#pragma unroll
-              for (int w = 1; w < 4; ++w)
-                if (w < p.W) a += __ldg(cwp + e * p.W + w) * bf16_at(vraw[w], e);
-              r[e] = v0 - a;
-            }
-          }
+          for (int w = 0; w < 4; ++w) vraw[w] = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
           for (int l = 0; l < M; ++l) {
-            float gg[8], rho[8];
-            unpack_bf16x8(graw[l], gg);
+            graw[l] = make_uint4(0u, 0u, 0u, 0u);
+            al[l] = 0.f;
+          }
+        }
+        float r[8];
+        if (p.W == 4) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              r[e] *= 1.f - gg[e];
-              rho[e] = al[l] * r[e];
-            }
-            st_bf16x8(sP, sw128_offset(i * M + l, pc8, Ly::U_ATOM), rho);
+          for (int e = 0; e < 8; ++e) {  // taps of one channel: one aligned float4 (L1-resident)
+            const float4 c4e = __ldg(reinterpret_cast<const float4*>(cwp) + e);
+            const float v0 = bf16_at(vraw[0], e);
+            r[e] = v0 - (c4e.x * v0 + c4e.y * bf16_at(vraw[1], e) + c4e.z * bf16_at(vraw[2], e) +
+                         c4e.w * bf16_at(vraw[3], e));
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) r[e] = 0.f;
+          for (int e = 0; e < 8; ++e) {
+            const float v0 = bf16_at(vraw[0], e);
+            float a = __ldg(cwp + e * p.W) * v0;
 #pragma unroll
-          for (int l = 0; l < M; ++l) st_bf16x8(sP, sw128_offset(i * M + l, pc8, Ly::U_ATOM), r);
+            for (int w = 1; w < 4; ++w)
+              if (w < p.W) a += __ldg(cwp + e * p.W + w) * bf16_at(vraw[w], e);
+            r[e] = v0 - a;
+          }
+        }
+#pragma unroll
+        for (int l = 0; l < M; ++l) {
+          float rho[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            r[e] *= 1.f - bf16_at(graw[l], e);
+            rho[e] = al[l] * r[e];
+          }
+          st_bf16x8(sP, sw128_offset(i * M + l, pc8, Ly::U_ATOM), rho);
         }
       }
     }
@@ -392,12 +408,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16(tmem + D3, kdesc(aS, kk, kAtom), kdesc(aKQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
         mma_commit(bar_mma);
         mma_inflight = (int)ph_mma;
-        if (n + 1 < nchunks) prefetch_tiles_l2(t0 + kC);
       } else {
         *s_abort = 1;
       }
     }
     ph_load ^= 1;
+    if (n + 1 < nchunks) prefetch_next_l2(t0 + kC);
     if (warp == 1 && n + 1 < nchunks) {
       // the next chunk's gates are token-major spans [b, t0+64 .. t0+128, :]: prefetch their L2 lines
       const int tn = t0 + kC, te = min(tn + kC, T);
@@ -448,15 +464,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pc = pb + k;
         const int j0 = 16 * (cq * PQ + pc);
         float x[16];
+        if (fast) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i = (j0 < 64) ? j0 + e : (j0 - 64 + e) / (M > 0 ? M : 1);
-          float f;
-          if (fast)
-            f = rs * sEn[i];
-          else
-            f = (krow ? Bt[t] : 1.f) * __expf(Gt - G[i]);
-          x[e] = (i < tlim) ? f * __uint_as_float(raw[k][e]) : 0.f;
+          for (int e = 0; e < 16; ++e) {
+            const int i = (j0 < 64) ? j0 + e : (j0 - 64 + e) / (M > 0 ? M : 1);
+            x[e] = (i < tlim) ? rs * sEn[i] * __uint_as_float(raw[k][e]) : 0.f;
+          }
+        } else {
+          const float bk = krow ? Bt[t] : 1.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int i = (j0 < 64) ? j0 + e : (j0 - 64 + e) / (M > 0 ? M : 1);
+            x[e] = (i < tlim) ? bk * __expf(Gt - G[i]) * __uint_as_float(raw[k][e]) : 0.f;
+          }
         }
         if (j0 < 64) {
           if (krow) {
@@ -845,7 +865,8 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
     mu = mk;
     mg = mk;
   }
-  TcArgs a{static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha,
+  TcArgs a{static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
+           static_cast<const __nv_bfloat16*>(p.u), static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha,
            static_cast<const __nv_bfloat16*>(p.gain), p.conv_w, p.S0, p.lengths,
            static_cast<__nv_bfloat16*>(p.o), p.S_final, p.B, p.T, p.H, p.W, p.status, p.spin_limit};
   prism_chunk_tc_kernel<D, M><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, a);
