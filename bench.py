@@ -92,6 +92,29 @@ def recorded_traffic(kernel, workload):
     return e.get("dram_bytes_per_launch")
 
 
+# ---------------------------------------------------------------- multi-rank plumbing
+def rank_workload(w, rank):
+    """The batch rank ``rank`` scans: same shape, its own seed (independent
+    replicas sharded by batch; no data crosses ranks)."""
+    return w.replace(seed=w.seed + rank)
+
+
+def max_over_ranks(x, dist, device):
+    """Max of a per-rank float over all ranks (the job's time is its slowest rank)."""
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(tokens_per_rank, world, ms_per_step):
+    """Whole-job tokens/s: the tokens every rank processed per step over the
+    slowest rank's time per step."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -229,7 +252,7 @@ def run_ours(args, w):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    wr = w.replace(seed=w.seed + rank)   # each rank scans its own batch
+    wr = rank_workload(w, rank)   # each rank scans its own batch
     host_inputs = synth.make_inputs(wr)
     d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in host_inputs.items()}
     io_dtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
@@ -266,13 +289,9 @@ def run_ours(args, w):
     if prism.stream_status() != 0:
         raise SystemExit("device status word reports an error in the timed region")
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms_local = sum(per_step) / K
-    ms = torch.tensor([ms_local], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    ms = float(ms.item())
+    ms = max_over_ranks(sum(per_step) / K, dist, dev)
     work = algorithmic_work(w, host_inputs["lengths"].numpy() if host_inputs["lengths"] is not None else None)
-    value = world * work["tokens"] / (ms / 1e3)
+    value = aggregate_throughput(work["tokens"], world, ms)
 
     # end to end through the host-buffer entry point: pinned host inputs -> HBM,
     # scan, o and S_final back to host, every step
@@ -294,13 +313,11 @@ def run_ours(args, w):
             prism.scan_fwd_host(pinned, devbuf, L=w.L, chunk=w.chunk, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = torch.tensor([e0.elapsed_time(e1) / K2], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        ems = max_over_ranks(e0.elapsed_time(e1) / K2, dist, dev)
         h2d = sum(t.numel() * t.element_size() for n, t in pinned.items()
                   if t is not None and n not in ("o", "S_final"))
         d2h = pinned["o"].numel() * pinned["o"].element_size() + S.numel() * 4
-        e2e = {"value": world * work["tokens"] / (float(ems.item()) / 1e3), "unit": UNIT,
+        e2e = {"value": aggregate_throughput(work["tokens"], world, ems), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K2,
                "api": "prism_scan_fwd_host (C ABI, pinned host buffers)"}
 
