@@ -49,7 +49,7 @@ using namespace sm100;
 constexpr int kC = 64;           // chunk length
 constexpr int kThreads = 512;    // 16 warps: warp w reads TMEM lanes 32*(w%4).., column quarter w/4
 constexpr uint32_t kAtom = 16384;  // one 128-row, 128-byte-wide swizzle atom column
-constexpr long long kDrainLimit = 1ll << 26;
+constexpr long long kDrainLimit = 1ll << 18;  // polls of up to 20 us each
 
 template <int D, int M>
 struct Layout {
@@ -158,7 +158,8 @@ template <int D, int M>
 __global__ void __launch_bounds__(kThreads, 1)
     prism_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                           const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_v,
-                          const __grid_constant__ CUtensorMap map_g, TcArgs p) {
+                          const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_o,
+                          TcArgs p) {
   using Ly = Layout<D, M>;
   constexpr int NA = Ly::NA, UR = Ly::UR, LDA = Ly::LDA;
   extern __shared__ uint8_t smem_raw[];
@@ -231,7 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < NA; ++a) {
       tma_load_4d(sKQ + a * kAtom, &map_k, bar_load, 64 * a, h, t0, b);
       tma_load_4d(sKQ + a * kAtom + 8192, &map_q, bar_load, 64 * a, h, t0, b);
-      if (M > 0) tma_load_5d(sU + a * Ly::U_ATOM, &map_u, bar_load, 64 * a, 0, h, t0, b);
+#pragma unroll
+      for (int l = 0; l < M; ++l)  // direction-major rows: row l*64 + i
+        tma_load_5d(sU + a * Ly::U_ATOM + l * 8192, &map_u, bar_load, 64 * a, l, h, t0, b);
     }
   };
   // L2 prefetch of the next chunk's k, q, v (D bf16 per token) and u, gain (M*D bf16 per
@@ -290,6 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       sBeta[buf * 64 + 2 * lane] = bt[0];
       sBeta[buf * 64 + 2 * lane + 1] = bt[1];
     }
+    __syncthreads();  // the chunk's decay prefix is needed below
+    // Fast path (chunk log-decay >= -60): write P~ = diag(c) P with c_i = e^{G_63 - G_i}; the
+    // U-columns of [Bku;QU] then carry e^{G_t - G_63} instead of e^{G_t - G_i} (same product).
+    const float G63 = sG[buf * 64 + 63];
+    const bool pfast = G63 >= -60.f;
     if (M > 0) {
 #pragma unroll 1
       for (int pass = 0; pass < kC / TPP; ++pass) {
@@ -319,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             al[l] = 0.f;
           }
         }
+        const float ci = pfast ? __expf(G63 - sG[buf * 64 + i]) : 1.f;
         float r[8];
         if (p.W == 4) {
 #pragma unroll
@@ -342,12 +351,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int l = 0; l < M; ++l) {
           float rho[8];
+          const float alc = al[l] * ci;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             r[e] *= 1.f - bf16_at(graw[l], e);
-            rho[e] = al[l] * r[e];
+            rho[e] = alc * r[e];
           }
-          st_bf16x8(sP, sw128_offset(i * M + l, pc8, Ly::U_ATOM), rho);
+          st_bf16x8(sP, sw128_offset(l * 64 + i, pc8, Ly::U_ATOM), rho);
         }
       }
     }
@@ -448,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tlim = krow ? t : t + 1;  // keep column i < tlim
       const float Gt = G[t];
       const float rs = (krow ? Bt[t] : 1.f) * sEp[t];
+      const float rsu = fast ? (krow ? Bt[t] : 1.f) * __expf(Gt - G[63]) : 0.f;
       constexpr int NP = (64 + UR) / 16;  // 16-column pieces of R1
       constexpr int PQ = NP / 4;           // pieces of this thread's column quarter
       constexpr int PB = PQ >= 2 ? 2 : 1;  // pieces per TMEM wait
@@ -464,18 +475,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pc = pb + k;
         const int j0 = 16 * (cq * PQ + pc);
         float x[16];
-        if (fast) {
+        if (j0 < 64) {  // K / Q columns: D[t,i] = e^{G_t - G_i}
+          if (fast) {
+            float en[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int i = (j0 < 64) ? j0 + e : (j0 - 64 + e) / (M > 0 ? M : 1);
-            x[e] = (i < tlim) ? rs * sEn[i] * __uint_as_float(raw[k][e]) : 0.f;
+            for (int e = 0; e < 16; e += 4) {
+              const float4 f = *reinterpret_cast<const float4*>(sEn + j0 + e);
+              en[e] = f.x; en[e + 1] = f.y; en[e + 2] = f.z; en[e + 3] = f.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x[e] = (j0 + e < tlim) ? rs * en[e] * __uint_as_float(raw[k][e]) : 0.f;
+          } else {
+            const float bk = krow ? Bt[t] : 1.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              x[e] = (j0 + e < tlim) ? bk * __expf(Gt - G[j0 + e]) * __uint_as_float(raw[k][e]) : 0.f;
           }
-        } else {
-          const float bk = krow ? Bt[t] : 1.f;
+        } else {  // U columns (l, i): fast path e^{G_t - G_63} (P holds P~), else e^{G_t - G_i}
+          const int i0 = (j0 - 64) & 63;
+          if (fast) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int i = (j0 < 64) ? j0 + e : (j0 - 64 + e) / (M > 0 ? M : 1);
-            x[e] = (i < tlim) ? bk * __expf(Gt - G[i]) * __uint_as_float(raw[k][e]) : 0.f;
+            for (int e = 0; e < 16; ++e) x[e] = (i0 + e < tlim) ? rsu * __uint_as_float(raw[k][e]) : 0.f;
+          } else {
+            const float bk = krow ? Bt[t] : 1.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              x[e] = (i0 + e < tlim) ? bk * __expf(Gt - G[i0 + e]) * __uint_as_float(raw[k][e]) : 0.f;
           }
         }
         if (j0 < 64) {
@@ -556,45 +581,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
       }
       // ---------------- C3: inverse 32 -> 64
-      // (3) 32 -> 64: T[32:64, 0:32] = -T2 (A21 T1).  256 threads, 4 rows x 1 column each:
-      // the 4 row operands are float4 broadcasts, the column operand a conflict-free scalar.
-      if (tid < 256) {
-        const int r0 = (tid >> 5) * 4, s2 = tid & 31;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
+      // (3) 32 -> 64: T[32:64, 0:32] = -T2 (A21 T1).  Each thread: 2 rows x 1 column; the row
+      // operands are float4 broadcasts, the column operand a conflict-free scalar.
+      {
+        const int r0 = (tid >> 5) * 2, s2 = tid & 31;
+        float acc[2] = {0.f, 0.f};
+#pragma unroll 4
         for (int u = 0; u < 32; u += 4) {  // Y2 = A21 T1
           float tc[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) tc[k] = sA[(u + k) * LDA + s2];
 #pragma unroll
-          for (int i2 = 0; i2 < 4; ++i2) {
+          for (int i2 = 0; i2 < 2; ++i2) {
             const float4 a = *reinterpret_cast<const float4*>(sA + (32 + r0 + i2) * LDA + u);
             acc[i2] += a.x * tc[0] + a.y * tc[1] + a.z * tc[2] + a.w * tc[3];
           }
         }
 #pragma unroll
-        for (int i2 = 0; i2 < 4; ++i2) sY[(r0 + i2) * 32 + s2] = acc[i2];
-      }
-      __syncthreads();
-      if (tid < 256) {
-        const int r0 = (tid >> 5) * 4, s2 = tid & 31;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
+        for (int i2 = 0; i2 < 2; ++i2) sY[(r0 + i2) * 32 + s2] = acc[i2];
+        __syncthreads();
+        acc[0] = acc[1] = 0.f;
+#pragma unroll 4
         for (int u = 0; u < 32; u += 4) {  // T21 = -T2 Y2 (T2's upper triangle is zero)
           float yc[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) yc[k] = sY[(u + k) * 32 + s2];
 #pragma unroll
-          for (int i2 = 0; i2 < 4; ++i2) {
+          for (int i2 = 0; i2 < 2; ++i2) {
             const float4 a = *reinterpret_cast<const float4*>(sA + (32 + r0 + i2) * LDA + 32 + u);
             acc[i2] += a.x * yc[0] + a.y * yc[1] + a.z * yc[2] + a.w * yc[3];
           }
         }
         // rows 32..63, columns 0..31 held A21, which step (3a) has consumed
 #pragma unroll
-        for (int i2 = 0; i2 < 4; ++i2) sA[(32 + r0 + i2) * LDA + s2] = -acc[i2];
+        for (int i2 = 0; i2 < 2; ++i2) sA[(32 + r0 + i2) * LDA + s2] = -acc[i2];
+        __syncthreads();
       }
-      __syncthreads();
       // T (fp32, lower incl. unit diagonal; upper part holds A's zeros) -> bf16 rows 0..63 of TQ
       {
         const int t = tid >> 3, c8 = (tid & 7) * 8;
@@ -646,11 +668,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_bf16x8(sTQ, sw128_offset(row, 16 * cq, kAtom), x);
         st_bf16x8(sTQ, sw128_offset(row, 16 * cq + 8, kAtom), x + 8);
       }
-      if (M > 0) {
+      if (M > 0 && !fast) {  // exact path: P~ = diag(c) P into the [Bku;QU] buffer
         for (int e = tid; e < UR * D / 8; e += kThreads) {
           const int r = e / (D / 8), c8 = (e % (D / 8)) * 8;
           const uint32_t off = sw128_offset(r, c8, Ly::U_ATOM);
-          const float sc = sCdec[r / (M > 0 ? M : 1)];
+          const float sc = sCdec[r & 63];
           uint4 u = *reinterpret_cast<const uint4*>(sP + off);
           __nv_bfloat162* hx = reinterpret_cast<__nv_bfloat162*>(&u);
           float f[8];
@@ -698,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (M > 0) {
 #pragma unroll
         for (int kk = 0; kk < UR / 16; ++kk)
-          mma_bf16(tmem + RS, mndesc(aBQ, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
+          mma_bf16(tmem + RS, mndesc(fast ? aP : aBQ, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
       }
       mma_commit(bar_mma);
       mma_inflight = (int)ph_mma;
@@ -726,12 +748,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       float opart[16];
       tmem_ld16(tl + R1 + 192 + tb, x);
       tmem_ld16(tl + D3 + 64 + tb, opart);
+      // o tile [64 tokens][D] bf16 in the X buffer (MMA4 has consumed X), stored by TMA below
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int t = t0 + tb + e;
-        if (t < T)
-          p.o[(((size_t)b * T + t) * H + h) * D + row] = __float2bfloat16_rn(tb + e < nv ? opart[e] + x[e] : 0.f);
-      }
+      for (int e = 0; e < 16; ++e)
+        *reinterpret_cast<__nv_bfloat16*>(sX + sw128_offset(tb + e, row, 8192)) =
+            __float2bfloat16_rn(tb + e < nv ? opart[e] + x[e] : 0.f);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -744,6 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_bf16(tmem + RS, kdesc(aDl, kk, kAtom), mndesc(aKQ, kk, kAtom), idesc_bf16(128, D, 0, 1), 1);
       mma_commit(bar_mma);
       mma_inflight = (int)ph_mma;
+#pragma unroll
+      for (int a = 0; a < NA; ++a) tma_store_4d(&map_o, sX + a * 8192, 64 * a, h, t0, b);
+      bulk_commit_group();
     }
 
     // ---------------- I: next chunk's loads; S_{n+1} -> bf16 SXA (and S_final)
@@ -757,6 +781,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
+    if (tid == 0) bulk_wait_read_all();  // the o tile in SXA has been read by the TMA store
+    __syncthreads();
     tc_fence_after();
     if (ok && srow) {
       const bool last = n + 1 == nchunks;
@@ -804,6 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (load_inflight >= 0) mbar_wait(bar_load, (uint32_t)load_inflight, kDrainLimit, p.status);
     if (mma_inflight >= 0) mbar_wait(bar_mma, (uint32_t)mma_inflight, kDrainLimit, p.status);
   }
+  if (tid == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -848,17 +875,17 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
   });
   if (attr_err != cudaSuccess) return attr_err;
   const cuuint64_t B = p.B, T = p.T, H = p.H;
-  CUtensorMap mq, mk, mu, mv, mg;
+  CUtensorMap mq, mk, mu, mv, mg, mo;
   const cuuint64_t dims4[4] = {(cuuint64_t)D, H, T, B};
   const cuuint64_t str4[3] = {(cuuint64_t)D * 2, H * D * 2, T * H * D * 2};
   const cuuint32_t box4[4] = {64, 1, 64, 1};
   if (!encode(&mq, p.q, 4, dims4, str4, box4) || !encode(&mk, p.k, 4, dims4, str4, box4) ||
-      !encode(&mv, p.v, 4, dims4, str4, box4))
+      !encode(&mv, p.v, 4, dims4, str4, box4) || !encode(&mo, p.o, 4, dims4, str4, box4))
     return cudaErrorInvalidValue;
   if (M > 0) {
     const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)M, H, T, B};
     const cuuint64_t str5[4] = {(cuuint64_t)D * 2, (cuuint64_t)M * D * 2, H * M * D * 2, T * H * M * D * 2};
-    const cuuint32_t box5[5] = {64, (cuuint32_t)M, 1, 64, 1};
+    const cuuint32_t box5[5] = {64, 1, 1, 64, 1};
     if (!encode(&mu, p.u, 5, dims5, str5, box5) || !encode(&mg, p.gain, 5, dims5, str5, box5))
       return cudaErrorInvalidValue;
   } else {
@@ -869,7 +896,7 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
            static_cast<const __nv_bfloat16*>(p.u), static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha,
            static_cast<const __nv_bfloat16*>(p.gain), p.conv_w, p.S0, p.lengths,
            static_cast<__nv_bfloat16*>(p.o), p.S_final, p.B, p.T, p.H, p.W, p.status, p.spin_limit};
-  prism_chunk_tc_kernel<D, M><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, a);
+  prism_chunk_tc_kernel<D, M><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, mo, a);
   return cudaGetLastError();
 }
 

@@ -24,7 +24,7 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 int* g_status_ptr[kMaxDevices] = {};
 int g_arch_ok[kMaxDevices] = {};  // 0 unknown, 1 sm_100, -1 other
-constexpr long long kDefaultSpinLimit = 1ll << 26;
+constexpr long long kDefaultSpinLimit = 1ll << 18;  // polls; each may suspend up to 20 us
 std::atomic<long long> g_spin_limit{kDefaultSpinLimit};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
