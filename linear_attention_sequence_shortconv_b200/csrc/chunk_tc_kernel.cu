@@ -265,14 +265,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int CPT = D / 8;           // threads per token in the prologue
   constexpr int TPP = kThreads / CPT;  // tokens per prologue pass
   const int pc8 = (tid % CPT) * 8;
-  // ShortConv taps of the prologue's 8 channels: conv_w[h, pc8 .. pc8+7, 0 .. W-1], contiguous
-  const float* cwp = p.conv_w + ((size_t)h * D + pc8) * p.W;
+  // ShortConv taps of this head, conv_w[h, :, :] (D*W <= 4*D fp32), staged in shared memory
+  // for the prologue tap-major ([w][c]: a lane's 8 channels of one tap are 32 contiguous
+  // bytes, so a token's 16 lanes read 512 contiguous bytes): one element per thread.
+  const float* cw_head = p.conv_w + (size_t)h * D * p.W;
+  const bool tap_thread = tid < D * p.W;
 
-  // Chunk prologue: gate prefix (warp 0) and rho_{i,l} = alpha_{i,l} r_{i,l} -> P (bf16).
-  auto prologue = [&](int n, int buf) {
+  // Gate prefix of chunk n into buffer buf (one warp): G_t = sum_{j<=t} log gamma_j and
+  // beta_t; padded steps count as gamma = 1, beta = 0.
+  auto gate_scan = [&](int n, int buf) {
     const int t0 = n * kC;
     const int nv = min(kC, len - t0);
-    if (warp == 0) {  // G_t = sum_{j<=t} log gamma_j; padded steps: gamma = 1, beta = 0
+    {
       float lg[2], bt[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -293,68 +297,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       sBeta[buf * 64 + 2 * lane] = bt[0];
       sBeta[buf * 64 + 2 * lane + 1] = bt[1];
     }
-    __syncthreads();  // the chunk's decay prefix is needed below
+  };
+
+  // Chunk prologue: rho_{i,l} = alpha_{i,l} r_{i,l} -> P (bf16); needs the chunk's gate prefix in buf.
+  auto prologue = [&](int n, int buf, const float* taps) {
+    const int t0 = n * kC;
+    const int nv = min(kC, len - t0);
     // Fast path (chunk log-decay >= -60): write P~ = diag(c) P with c_i = e^{G_63 - G_i}; the
     // U-columns of [Bku;QU] then carry e^{G_t - G_63} instead of e^{G_t - G_i} (same product).
     const float G63 = sG[buf * 64 + 63];
     const bool pfast = G63 >= -60.f;
     if (M > 0) {
-#pragma unroll 1
-      for (int pass = 0; pass < kC / TPP; ++pass) {
+      constexpr int NPASS = kC / TPP;
+      // every global load of every pass first (independent requests in flight together)
+      uint4 vraw[NPASS][4], graw[NPASS][M > 0 ? M : 1];
+      float al[NPASS][M > 0 ? M : 1];
+#pragma unroll
+      for (int pass = 0; pass < NPASS; ++pass) {
         const int i = pass * TPP + tid / CPT;
         const int t = t0 + i;
-        // every global load of the pass first (independent requests in flight together)
-        uint4 vraw[4], graw[M > 0 ? M : 1];
-        float al[M > 0 ? M : 1];
         if (i < nv) {
           const size_t th = ((size_t)b * T + t) * H + h;
           const __nv_bfloat16* vp = p.v + th * D + pc8;
-          vraw[0] = ldg16(vp);
+          vraw[pass][0] = ldg16(vp);
 #pragma unroll
           for (int w = 1; w < 4; ++w)
-            vraw[w] = (w < p.W && t - w >= 0) ? ldg16(vp - (size_t)w * H * D) : make_uint4(0u, 0u, 0u, 0u);
+            vraw[pass][w] = (w < p.W && t - w >= 0) ? ldg16(vp - (size_t)w * H * D) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
           for (int l = 0; l < M; ++l) {
-            graw[l] = ldg16(p.gain + (th * M + l) * D + pc8);
-            al[l] = __ldg(p.alpha + th * M + l);
+            graw[pass][l] = ldg16(p.gain + (th * M + l) * D + pc8);
+            al[pass][l] = __ldg(p.alpha + th * M + l);
           }
         } else {  // padded step: rho = 0
 #pragma unroll
-          for (int w = 0; w < 4; ++w) vraw[w] = make_uint4(0u, 0u, 0u, 0u);
+          for (int w = 0; w < 4; ++w) vraw[pass][w] = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
           for (int l = 0; l < M; ++l) {
-            graw[l] = make_uint4(0u, 0u, 0u, 0u);
-            al[l] = 0.f;
+            graw[pass][l] = make_uint4(0u, 0u, 0u, 0u);
+            al[pass][l] = 0.f;
           }
         }
+      }
+#pragma unroll
+      for (int pass = 0; pass < NPASS; ++pass) {
+        const int i = pass * TPP + tid / CPT;
         const float ci = pfast ? __expf(G63 - sG[buf * 64 + i]) : 1.f;
         float r[8];
-        if (p.W == 4) {
+        {
+          float a[8];
+          const float4 lo0 = *reinterpret_cast<const float4*>(taps + pc8);
+          const float4 hi0 = *reinterpret_cast<const float4*>(taps + pc8 + 4);
+          const float t0v[8] = {lo0.x, lo0.y, lo0.z, lo0.w, hi0.x, hi0.y, hi0.z, hi0.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {  // taps of one channel: one aligned float4 (L1-resident)
-            const float4 c4e = __ldg(reinterpret_cast<const float4*>(cwp) + e);
-            const float v0 = bf16_at(vraw[0], e);
-            r[e] = v0 - (c4e.x * v0 + c4e.y * bf16_at(vraw[1], e) + c4e.z * bf16_at(vraw[2], e) +
-                         c4e.w * bf16_at(vraw[3], e));
+          for (int e = 0; e < 8; ++e) a[e] = t0v[e] * bf16_at(vraw[pass][0], e);
+#pragma unroll
+          for (int w = 1; w < 4; ++w) {
+            if (w < p.W) {
+              const float4 lo = *reinterpret_cast<const float4*>(taps + w * D + pc8);
+              const float4 hi = *reinterpret_cast<const float4*>(taps + w * D + pc8 + 4);
+              const float tw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) a[e] += tw[e] * bf16_at(vraw[pass][w], e);
+            }
           }
-        } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float v0 = bf16_at(vraw[0], e);
-            float a = __ldg(cwp + e * p.W) * v0;
-#pragma unroll
-            for (int w = 1; w < 4; ++w)
-              if (w < p.W) a += __ldg(cwp + e * p.W + w) * bf16_at(vraw[w], e);
-            r[e] = v0 - a;
-          }
+          for (int e = 0; e < 8; ++e) r[e] = bf16_at(vraw[pass][0], e) - a[e];
         }
 #pragma unroll
         for (int l = 0; l < M; ++l) {
           float rho[8];
-          const float alc = al[l] * ci;
+          const float alc = al[pass][l] * ci;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            r[e] *= 1.f - bf16_at(graw[l], e);
+            r[e] *= 1.f - bf16_at(graw[pass][l], e);
             rho[e] = alc * r[e];
           }
           st_bf16x8(sP, sw128_offset(l * 64 + i, pc8, Ly::U_ATOM), rho);
@@ -388,7 +403,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     issue_loads(0);
     load_inflight = (int)ph_load;
   }
-  if (nchunks > 0) prologue(0, 0);
+  float* taps0 = reinterpret_cast<float*>(sBQ);  // free until chunk 0's epilogue
+  if (nchunks > 0 && warp == 0) gate_scan(0, 0);
+  if (M > 0 && tap_thread) taps0[(tid % p.W) * D + tid / p.W] = __ldg(cw_head + tid);
+  __syncthreads();
+  if (nchunks > 0) prologue(0, 0, taps0);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -545,7 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------- C1: inverse
     {
-      // (1) diagonal 16x16 blocks: thread (blk, j) solves column j by forward substitution
+      // (1) diagonal 16x16 blocks: thread (blk, j) solves column j by forward substitution;
+      // meanwhile warp 2 computes the next chunk's gate prefix (its lines were prefetched in A)
+      if (warp == 2 && n + 1 < nchunks) gate_scan(n + 1, cur ^ 1);
       float xcol[16];
       const int blk = tid >> 4, j = tid & 15;
       if (tid < 64) {
@@ -601,8 +622,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i2 = 0; i2 < 2; ++i2) sY[(r0 + i2) * 32 + s2] = acc[i2];
         __syncthreads();
         acc[0] = acc[1] = 0.f;
+        const int ulim = r0 + 2;  // T2 is lower triangular: only u <= r0 + 1 contribute (warp-uniform)
 #pragma unroll 4
-        for (int u = 0; u < 32; u += 4) {  // T21 = -T2 Y2 (T2's upper triangle is zero)
+        for (int u = 0; u < ulim; u += 4) {  // T21 = -T2 Y2
           float yc[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) yc[k] = sY[(u + k) * 32 + s2];
@@ -639,6 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------- D: loads for X while the MMAs run
     // values of v this thread needs for X, loaded while the MMAs run
+    const float tap_reg = (M > 0 && tap_thread) ? __ldg(cw_head + tid) : 0.f;
     // (padded steps have beta = 0, so any in-range token may stand in for them)
     float vreg[16];
     {
@@ -727,7 +750,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------- F: next chunk's prologue while MMA4 / MMA5a run (P_n is no longer read)
-    if (n + 1 < nchunks) prologue(n + 1, cur ^ 1);
+    if (n + 1 < nchunks) {
+      float* taps = reinterpret_cast<float*>(sDl);  // Delta~ is written only after MMA4 completes
+      if (M > 0 && tap_thread) taps[(tid % p.W) * D + tid / p.W] = tap_reg;
+      __syncthreads();
+      prologue(n + 1, cur ^ 1, taps);
+      __syncthreads();  // every thread is done with the staged taps before Delta~ overwrites them
+    }
     fence_proxy_async_smem();
 
     // ---------------- G: Delta~^T -> SXA; o = O partial + (QKT X); issue MMA5b
