@@ -221,43 +221,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t aKQ = smem_u32(sKQ), aU = smem_u32(sU), aP = smem_u32(sP), aBQ = smem_u32(sBQ);
   const uint32_t aTQ = smem_u32(sTQ), aS = smem_u32(sSXA), aX = smem_u32(sX), aDl = smem_u32(sDl);
-  constexpr uint32_t kLoadBytes = 2 * NA * 8192 + NA * UR * 128;
   uint32_t ph_load = 0, ph_mma = 0;
   // (thread 0) phase of a TMA batch / MMA commit in flight and not yet observed, or -1
   int load_inflight = -1, mma_inflight = -1;
+  bool load_open = false;  // (thread 0) next chunk's Q/U loads issued, closing arrival not yet made
 
-  auto issue_loads = [&](int t0) {
-    mbar_arrive_expect_tx(bar_load, kLoadBytes);
+  // The next chunk's tiles are loaded as soon as their buffers are free: Q once MMA1/MMA3 have
+  // read it, U once MMA5a has, K (with the arrival that closes the phase) once MMA5b has.
+  auto load_q = [&](int t0) {
+    load_open = true;
+    mbar_expect_tx(bar_load, NA * 8192);
 #pragma unroll
-    for (int a = 0; a < NA; ++a) {
-      tma_load_4d(sKQ + a * kAtom, &map_k, bar_load, 64 * a, h, t0, b);
-      tma_load_4d(sKQ + a * kAtom + 8192, &map_q, bar_load, 64 * a, h, t0, b);
+    for (int a = 0; a < NA; ++a) tma_load_4d(sKQ + a * kAtom + 8192, &map_q, bar_load, 64 * a, h, t0, b);
+  };
+  auto load_u = [&](int t0) {
+    if (M > 0) {
+      load_open = true;
+      mbar_expect_tx(bar_load, NA * UR * 128);
 #pragma unroll
-      for (int l = 0; l < M; ++l)  // direction-major rows: row l*64 + i
-        tma_load_5d(sU + a * Ly::U_ATOM + l * 8192, &map_u, bar_load, 64 * a, l, h, t0, b);
+      for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int l = 0; l < M; ++l)  // direction-major rows: row l*64 + i
+          tma_load_5d(sU + a * Ly::U_ATOM + l * 8192, &map_u, bar_load, 64 * a, l, h, t0, b);
     }
+  };
+  auto load_k_arrive = [&](int t0) {
+    load_open = false;
+    mbar_arrive_expect_tx(bar_load, NA * 8192);
+#pragma unroll
+    for (int a = 0; a < NA; ++a) tma_load_4d(sKQ + a * kAtom, &map_k, bar_load, 64 * a, h, t0, b);
+  };
+  auto issue_loads = [&](int t0) {
+    load_q(t0);
+    load_u(t0);
+    load_k_arrive(t0);
   };
   // L2 prefetch of the next chunk's k, q, v (D bf16 per token) and u, gain (M*D bf16 per
   // token): one 128-byte line per thread and request, spread over all threads.
   auto prefetch_next_l2 = [&](int t0) {
     constexpr int LK = D * 2 / 128, LU = M * D * 2 / 128;  // 128-byte lines per token
-    constexpr int LT = 3 * LK + 2 * LU;
-    const int i = tid & 63;
+    const int i = tid & 63, g = tid >> 6;                   // 8 groups of 64 threads
     if (t0 + i < T) {
       const size_t th = ((size_t)b * T + t0 + i) * H + h;
-      const char* kp = reinterpret_cast<const char*>(p.k + th * D);
-      const char* qp = reinterpret_cast<const char*>(p.q + th * D);
-      const char* vp = reinterpret_cast<const char*>(p.v + th * D);
-      const char* up = reinterpret_cast<const char*>(p.u + th * M * D);
-      const char* gp = reinterpret_cast<const char*>(p.gain + th * M * D);
+      if (g < 3) {  // k, q, v: LK lines each
+        const __nv_bfloat16* base = g == 0 ? p.k : (g == 1 ? p.q : p.v);
+        const char* ptr = reinterpret_cast<const char*>(base + th * D);
 #pragma unroll
-      for (int r = tid >> 6; r < LT; r += kThreads / 64) {
-        const char* ptr = r < LK ? kp + r * 128
-                        : r < 2 * LK ? qp + (r - LK) * 128
-                        : r < 3 * LK ? vp + (r - 2 * LK) * 128
-                        : r < 3 * LK + LU ? up + (r - 3 * LK) * 128
-                        : gp + (r - 3 * LK - LU) * 128;
-        prefetch_l2(ptr);
+        for (int r = 0; r < LK; ++r) prefetch_l2(ptr + r * 128);
+      } else if (M > 0) {  // u (groups 3..4) and gain (groups 5..7): LU lines each, split
+        const bool is_u = g < 5;
+        const int part = is_u ? g - 3 : g - 5, nparts = is_u ? 2 : 3;
+        const char* ptr = reinterpret_cast<const char*>((is_u ? p.u : p.gain) + th * M * D);
+        for (int r = part; r < LU; r += nparts) prefetch_l2(ptr + r * 128);
       }
     }
   };
@@ -272,31 +287,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool tap_thread = tid < D * p.W;
 
   // Gate prefix of chunk n into buffer buf (one warp): G_t = sum_{j<=t} log gamma_j and
-  // beta_t; padded steps count as gamma = 1, beta = 0.
-  auto gate_scan = [&](int n, int buf) {
+  // beta_t; padded steps count as gamma = 1, beta = 0.  gate_load issues the loads (lane owns
+  // tokens 2*lane, 2*lane+1), gate_scan finishes from those registers.
+  auto gate_load = [&](int n, float (&gl)[4]) {
     const int t0 = n * kC;
     const int nv = min(kC, len - t0);
-    {
-      float lg[2], bt[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int t = 2 * lane + e;
-        const bool valid = t < nv;
-        const size_t th = ((size_t)b * T + t0 + t) * H + h;
-        lg[e] = valid ? __logf(__ldg(p.gamma + th)) : 0.f;
-        bt[e] = valid ? __ldg(p.beta + th) : 0.f;
-      }
-      float x = lg[0] + lg[1];
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += y;
-      }
-      sG[buf * 64 + 2 * lane] = x - lg[1];
-      sG[buf * 64 + 2 * lane + 1] = x;
-      sBeta[buf * 64 + 2 * lane] = bt[0];
-      sBeta[buf * 64 + 2 * lane + 1] = bt[1];
+    for (int e = 0; e < 2; ++e) {
+      const int t = 2 * lane + e;
+      const bool valid = t < nv;
+      const size_t th = ((size_t)b * T + min(t0 + t, T - 1)) * H + h;
+      gl[e] = valid ? __ldg(p.gamma + th) : 1.f;
+      gl[2 + e] = valid ? __ldg(p.beta + th) : 0.f;
     }
+  };
+  auto gate_scan = [&](const float (&gl)[4], int buf) {
+    const float lg0 = __logf(gl[0]), lg1 = __logf(gl[1]);
+    float x = lg0 + lg1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    sG[buf * 64 + 2 * lane] = x - lg1;
+    sG[buf * 64 + 2 * lane + 1] = x;
+    sBeta[buf * 64 + 2 * lane] = gl[2];
+    sBeta[buf * 64 + 2 * lane + 1] = gl[3];
   };
 
   // Chunk prologue: rho_{i,l} = alpha_{i,l} r_{i,l} -> P (bf16); needs the chunk's gate prefix in buf.
@@ -404,7 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     load_inflight = (int)ph_load;
   }
   float* taps0 = reinterpret_cast<float*>(sBQ);  // free until chunk 0's epilogue
-  if (nchunks > 0 && warp == 0) gate_scan(0, 0);
+  if (nchunks > 0 && warp == 0) {
+    float gl[4];
+    gate_load(0, gl);
+    gate_scan(gl, 0);
+  }
   if (M > 0 && tap_thread) taps0[(tid % p.W) * D + tid / p.W] = __ldg(cw_head + tid);
   __syncthreads();
   if (nchunks > 0) prologue(0, 0, taps0);
@@ -468,8 +488,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- B: epilogue of MMA1 -> A (fp32), [Bku;QU], QK (bf16); then issue MMA2
     bool ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
-    if (tid == 0 && ok) mma_inflight = -1;
+    if (tid == 0 && ok) {
+      mma_inflight = -1;
+      if (n + 1 < nchunks) load_q(t0 + kC);  // MMA1 and MMA3 have read Q
+    }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
+    float gl_next[4] = {1.f, 1.f, 0.f, 0.f};  // warp 2: next chunk's gates, scanned during C1
+    if (warp == 2 && n + 1 < nchunks) gate_load(n + 1, gl_next);
     tc_fence_after();
     if (ok) {
       const bool krow = row < 64;
@@ -550,23 +575,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------- C: rescale RS by exp(G_63); T = (I + A)^{-1} in place (fp32); issue MMA QK*T
-    if (srow) {
+    // the tap element this thread stages for the next prologue, and the values of v it needs for
+    // X, loaded here so their latency hides behind the inverse
+    const float tap_reg = (M > 0 && tap_thread) ? __ldg(cw_head + tid) : 0.f;
+    // (padded steps have beta = 0, so any in-range token may stand in for them)
+    __nv_bfloat16 vraw16[16];  // converted where X is formed, so the loads are not waited on here
+    {
+      const int tb = 16 * cq;
+      const int rr = srow ? row : 0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int t = min(t0 + tb + e, T - 1);
+        vraw16[e] = p.v[(((size_t)b * T + t) * H + h) * D + rr];
+      }
+    }
+    if (srow) {  // RS <- exp(G_63) RS, ahead of MMA5a / MMA5b accumulating into it
       const float blast = sEp[63];
+      uint32_t rr[SP][16];
+#pragma unroll
+      for (int pc = 0; pc < SP; ++pc) tmem_ld16_async(tl + RS + cq * (D / 4) + 16 * pc, rr[pc]);
+      tmem_wait_ld();
 #pragma unroll
       for (int pc = 0; pc < SP; ++pc) {
-        const int j0 = cq * (D / 4) + 16 * pc;
         float s[16];
-        tmem_ld16(tl + RS + j0, s);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) s[e] *= blast;
-        tmem_st16(tl + RS + j0, s);
+        for (int e = 0; e < 16; ++e) s[e] = __uint_as_float(rr[pc][e]) * blast;
+        tmem_st16_async(tl + RS + cq * (D / 4) + 16 * pc, s);
       }
+      tmem_wait_st();
     }
     // ---------------- C1: inverse
     {
       // (1) diagonal 16x16 blocks: thread (blk, j) solves column j by forward substitution;
       // meanwhile warp 2 computes the next chunk's gate prefix (its lines were prefetched in A)
-      if (warp == 2 && n + 1 < nchunks) gate_scan(n + 1, cur ^ 1);
+      if (warp == 2 && n + 1 < nchunks) gate_scan(gl_next, cur ^ 1);
       float xcol[16];
       const int blk = tid >> 4, j = tid & 15;
       if (tid < 64) {
@@ -659,24 +701,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar_mma);
       mma_inflight = (int)ph_mma;
     }
-    // ---------------- D: loads for X while the MMAs run
-    // values of v this thread needs for X, loaded while the MMAs run
-    const float tap_reg = (M > 0 && tap_thread) ? __ldg(cw_head + tid) : 0.f;
-    // (padded steps have beta = 0, so any in-range token may stand in for them)
-    float vreg[16];
-    {
-      const int tb = 16 * cq;
-      const int rr = srow ? row : 0;
-      __nv_bfloat16 raw[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int t = min(t0 + tb + e, T - 1);
-        raw[e] = p.v[(((size_t)b * T + t) * H + h) * D + rr];
-      }
-#pragma unroll
-      for (int e = 0; e < 16; ++e) vreg[e] = __bfloat162float(raw[e]);
-    }
-
     // ---------------- E: QKT -> TQ rows 64..127; P~ = diag(c) P -> BQ; X^T -> SXA; O partial
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
@@ -715,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (M > 0) tmem_ld16(tl + R1 + tb, d2);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float xv = Bt[tb + e] * (vreg[e] - sEp[tb + e] * y[e]);
+          float xv = Bt[tb + e] * (__bfloat162float(vraw16[e]) - sEp[tb + e] * y[e]);
           if (M > 0) xv -= d2[e];
           y[e] = xv;
         }
@@ -760,10 +784,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async_smem();
 
     // ---------------- G: Delta~^T -> SXA; o = O partial + (QKT X); issue MMA5b
-    // (the prologue above has no barrier of its own; the wait below orders it)
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
-    if (tid == 0 && ok) mma_inflight = -1;
+    if (tid == 0 && ok) {
+      mma_inflight = -1;
+      if (n + 1 < nchunks) load_u(t0 + kC);  // MMA5a has read U
+    }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
     if (ok && srow) {
@@ -805,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       if (ok) mma_inflight = -1;
       if (ok && n + 1 < nchunks) {
-        issue_loads(t0 + kC);
+        load_k_arrive(t0 + kC);  // MMA5b has read K
         load_inflight = (int)ph_load;
       }
     }
@@ -856,6 +882,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (tid == 0) {
     // drain this CTA's own copies and MMAs before giving the memory back
+    if (load_open) {  // close the phase so the copies already issued can complete it
+      mbar_arrive(bar_load);
+      load_inflight = (int)ph_load;
+    }
     if (load_inflight >= 0) mbar_wait(bar_load, (uint32_t)load_inflight, kDrainLimit, p.status);
     if (mma_inflight >= 0) mbar_wait(bar_mma, (uint32_t)mma_inflight, kDrainLimit, p.status);
   }
