@@ -620,7 +620,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           xcol[r] = (r < j) ? 0.f : (r == j ? 1.f : -acc);
         }
       }
+      tc_fence_before();  // the RS rescale above is ordered before MMA5a below
       __syncthreads();
+      if (tid == 0 && fast && M > 0) {
+        // Fast path: MMA5a (RS += P~^T U) needs only P~ (= P), U and the rescaled RS, so it runs
+        // under the inverse; it completes before the next prologue overwrites P.
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < UR / 16; ++kk)
+          mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
+      }
       if (tid < 64) {
 #pragma unroll
         for (int r = 0; r < 16; ++r) sA[(16 * blk + r) * LDA + 16 * blk + j] = xcol[r];
@@ -704,7 +713,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- E: QKT -> TQ rows 64..127; P~ = diag(c) P -> BQ; X^T -> SXA; O partial
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
-    if (tid == 0 && ok) mma_inflight = -1;
+    if (tid == 0 && ok) {
+      mma_inflight = -1;
+      if (fast && n + 1 < nchunks) load_u(t0 + kC);  // fast path: MMA5a (issued in C) has read U
+    }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
     if (ok) {
@@ -764,16 +776,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + R1 + 128, kdesc(aX, kk, kAtom), kdesc(aTQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
-      if (M > 0) {
+      if (M > 0 && !fast) {  // exact path: P~ was copied into the [Bku;QU] buffer in this step
 #pragma unroll
         for (int kk = 0; kk < UR / 16; ++kk)
-          mma_bf16(tmem + RS, mndesc(fast ? aP : aBQ, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
+          mma_bf16(tmem + RS, mndesc(aBQ, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
       }
       mma_commit(bar_mma);
       mma_inflight = (int)ph_mma;
     }
 
-    // ---------------- F: next chunk's prologue while MMA4 / MMA5a run (P_n is no longer read)
+    // ---------------- F: next chunk's prologue while MMA4 (and, on the exact path, MMA5a) run;
+    // P is no longer read: MMA2 and the fast-path MMA5a completed before step E's wait
     if (n + 1 < nchunks) {
       float* taps = reinterpret_cast<float*>(sDl);  // Delta~ is written only after MMA4 completes
       if (M > 0 && tap_thread) taps[(tid % p.W) * D + tid / p.W] = tap_reg;
@@ -788,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ph_mma ^= 1;
     if (tid == 0 && ok) {
       mma_inflight = -1;
-      if (n + 1 < nchunks) load_u(t0 + kC);  // MMA5a has read U
+      if (!fast && n + 1 < nchunks) load_u(t0 + kC);  // exact path: MMA5a has read U
     }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
