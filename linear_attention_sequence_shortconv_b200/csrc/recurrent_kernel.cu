@@ -11,63 +11,54 @@
 // The rows of S are independent recurrences: row c only needs (S k)_c, a dot
 // product inside the row.  Each row is held by LPR lanes (EPL = d_k / LPR fp32
 // elements per lane), so the two per-token reductions are log2(LPR)-step warp
-// shuffles.  Blocks of 64 threads carry 64 / LPR rows of one (batch, head), so
-// even 8 (batch, head) chains of 128 rows fill 128 blocks.  The next token's
-// inputs are loaded one token ahead into registers (directions and gains too
-// when L - 1 <= MPF), so the loop waits on the shuffles, not on memory.
+// shuffles.  Blocks of 64 threads carry 64 / LPR rows of one (batch, head), so a
+// handful of (batch, head) chains still spreads over many SMs.
+//
+// The loop over tokens is sequential, so its inputs must be on-chip when it gets
+// to them: tiles of TT tokens (k, q, u of the head; v and gains of the block's
+// rows; gamma, beta, alpha) stream into double-buffered shared memory with
+// cp.async while the previous tile is being scanned.
 #include "common.cuh"
 
 namespace prism {
 namespace {
 
 constexpr int kBlock = 64;
-constexpr int MPF = 7;  // residual directions prefetched one token ahead
+constexpr int kTileBytes = 48 * 1024;  // per buffer
 
-// Groups of 4 consecutive row elements kept in their I/O encoding until used: bf16 as one
-// 8-byte word pair, fp32 as a float4.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 template <typename T>
-struct Raw4;
+__device__ __forceinline__ float to_f(T x);
 template <>
-struct Raw4<float> {
-  float4 w;
-  __device__ void load(const float* p) { w = __ldg(reinterpret_cast<const float4*>(p)); }
-  __device__ float4 get() const { return w; }
-};
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
 template <>
-struct Raw4<__nv_bfloat16> {
-  uint2 w;
-  __device__ void load(const __nv_bfloat16* p) { w = __ldg(reinterpret_cast<const uint2*>(p)); }
-  __device__ float4 get() const {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-  }
-};
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-template <typename T, int EPL>
-struct RowVec {  // the EPL elements one lane holds of a d_k vector
-  Raw4<T> r[EPL / 4];
-  __device__ void load(const T* p) {
-#pragma unroll
-    for (int e = 0; e < EPL / 4; ++e) r[e].load(p + 4 * e);
-  }
-  __device__ float dot(const float* s) const {
-    float acc = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL / 4; ++e) {
-      const float4 f = r[e].get();
-      acc += s[4 * e] * f.x + s[4 * e + 1] * f.y + s[4 * e + 2] * f.z + s[4 * e + 3] * f.w;
-    }
-    return acc;
-  }
-  __device__ void axpy(float a, float* s) const {  // s += a * this
-#pragma unroll
-    for (int e = 0; e < EPL / 4; ++e) {
-      const float4 f = r[e].get();
-      s[4 * e] += a * f.x; s[4 * e + 1] += a * f.y; s[4 * e + 2] += a * f.z; s[4 * e + 3] += a * f.w;
-    }
-  }
-};
+// 4 consecutive elements from shared memory as fp32
+template <typename T>
+__device__ __forceinline__ float4 ld4_smem(const T* p);
+template <>
+__device__ __forceinline__ float4 ld4_smem<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
+template <>
+__device__ __forceinline__ float4 ld4_smem<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
 
 template <int LPR>
 __device__ __forceinline__ float row_sum(float x) {
@@ -76,24 +67,48 @@ __device__ __forceinline__ float row_sum(float x) {
   return x;
 }
 
-// Inputs of one token for one row-lane.
-template <typename T, int EPL, int MP>
-struct Tok {
-  RowVec<T, EPL> k, q, u[MP > 0 ? MP : 1];
-  float v, gam, bet, g[MP > 0 ? MP : 1], al[MP > 0 ? MP : 1];
+// Shared-memory layout of one tile of TT tokens (byte offsets, each 16-byte aligned).
+struct TileLayout {
+  int TT, dk, m, rpb, es;
+  int off_k, off_q, off_u, off_v, off_g, off_gam, off_bet, off_al, bytes;
+  __host__ __device__ TileLayout(int TT_, int dk_, int m_, int rpb_, int es_)
+      : TT(TT_), dk(dk_), m(m_), rpb(rpb_), es(es_) {
+    auto al16 = [](int x) { return (x + 15) & ~15; };
+    off_k = 0;
+    off_q = al16(off_k + TT * dk * es);
+    off_u = al16(off_q + TT * dk * es);
+    off_v = al16(off_u + TT * m * dk * es);
+    off_g = al16(off_v + TT * rpb * es);
+    off_gam = al16(off_g + TT * m * rpb * es);
+    off_bet = al16(off_gam + TT * 4);
+    off_al = al16(off_bet + TT * 4);
+    bytes = al16(off_al + TT * m * 4);
+  }
 };
 
-template <typename T, int LPR, int EPL, int MP>
-__global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p) {
+template <typename T>
+int tile_tokens(int dk, int m, int rpb) {
+  for (int TT = 32; TT > 1; TT >>= 1)
+    if (TileLayout(TT, dk, m, rpb, sizeof(T)).bytes <= kTileBytes) return TT;
+  return 1;
+}
+
+template <typename T, int LPR, int EPL>
+__global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, int TT) {
   constexpr int RPB = kBlock / LPR;  // rows per block
-  const int j = threadIdx.x % LPR;   // lane within the row: owns d_k elements EPL*j .. EPL*j+EPL-1
-  const int row = blockIdx.x * RPB + threadIdx.x / LPR;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int tid = threadIdx.x;
+  const int j = tid % LPR;  // lane within the row: owns d_k elements EPL*j .. EPL*j+EPL-1
+  const int lrow = tid / LPR;
+  const int row0 = blockIdx.x * RPB;
+  const int row = row0 + lrow;
   const int h = blockIdx.y, b = blockIdx.z;
   const int T_ = p.T, H = p.H, dk = p.d_k, dv = p.d_v, m = p.L - 1, W = p.W;
   const bool row_ok = row < dv;
   const int c = row_ok ? row : dv - 1;  // idle rows shadow the last real row (no stores)
   const int len = p.lengths ? min(max(p.lengths[b], 0), T_) : T_;
-  const bool prefetch_dirs = (m <= MP);
+  const TileLayout L(TT, dk, m, RPB, (int)sizeof(T));
+  const int nrows = min(RPB, dv - row0);  // rows of this block that exist
 
   const T* q = static_cast<const T*>(p.q);
   const T* k = static_cast<const T*>(p.k);
@@ -101,6 +116,61 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p) {
   const T* u = static_cast<const T*>(p.u);
   const T* g = static_cast<const T*>(p.gain);
   T* o = static_cast<T*>(p.o);
+
+  // cooperative async load of tile `ti` (tokens ti*TT ..) into buffer `buf`
+  auto load_tile = [&](int ti, int buf) {
+    uint8_t* base = smem + buf * L.bytes;
+    const int t0 = ti * TT, nt = min(TT, len - t0);
+    const int vec = 16 / (int)sizeof(T);  // elements per 16-byte chunk
+    const int kchunks = dk / vec;
+    // k, q: [nt][dk]
+    for (int e = tid; e < nt * kchunks; e += kBlock) {
+      const int i = e / kchunks, cc = e % kchunks;
+      const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+      cp_async16(base + L.off_k + (i * dk + cc * vec) * sizeof(T), k + tok * dk + cc * vec);
+      cp_async16(base + L.off_q + (i * dk + cc * vec) * sizeof(T), q + tok * dk + cc * vec);
+    }
+    // u: [nt][m][dk] (contiguous per token)
+    for (int e = tid; e < nt * m * kchunks; e += kBlock) {
+      const int i = e / (m * kchunks), r = e % (m * kchunks);
+      const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+      cp_async16(base + L.off_u + ((size_t)i * m * dk + r * vec) * sizeof(T), u + tok * m * dk + r * vec);
+    }
+    // v, gains of this block's rows: [nt][rpb], [nt][m][rpb] (a block's rows are contiguous:
+    // 16-byte copies when the whole block exists, element copies at a ragged d_v edge)
+    const int rbytes = RPB * (int)sizeof(T);
+    if (nrows == RPB && rbytes % 16 == 0) {
+      const int rch = rbytes / 16;
+      for (int e = tid; e < nt * (1 + m) * rch; e += kBlock) {
+        const int i = e / ((1 + m) * rch), r = e % ((1 + m) * rch), l = r / rch, cc = r % rch;
+        const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+        const T* src = (l == 0 ? v + tok * dv : g + (tok * m + (l - 1)) * dv) + row0 + cc * (16 / (int)sizeof(T));
+        uint8_t* dst = base + (l == 0 ? L.off_v + i * rbytes : L.off_g + (i * m + (l - 1)) * rbytes) + cc * 16;
+        cp_async16(dst, src);
+      }
+    } else {
+      for (int e = tid; e < nt * (1 + m) * nrows; e += kBlock) {
+        const int i = e / ((1 + m) * nrows), r = e % ((1 + m) * nrows), l = r / nrows, cr = r % nrows;
+        const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+        const T* src = l == 0 ? v + tok * dv + row0 + cr : g + (tok * m + (l - 1)) * dv + row0 + cr;
+        T* dst = reinterpret_cast<T*>(base + (l == 0 ? L.off_v : L.off_g)) +
+                 (l == 0 ? i * RPB + cr : (i * m + (l - 1)) * RPB + cr);
+        if (sizeof(T) == 4)
+          cp_async4(dst, src);
+        else
+          *dst = *src;  // 2-byte elements at a ragged edge: plain copy (cp.async needs >= 4 bytes)
+      }
+    }
+    // gates: gamma, beta [nt], alpha [nt][m]
+    for (int e = tid; e < nt * (2 + m); e += kBlock) {
+      const int i = e / (2 + m), r = e % (2 + m);
+      const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+      const float* src = r == 0 ? p.gamma + tok : (r == 1 ? p.beta + tok : p.alpha + tok * m + (r - 2));
+      float* dst = reinterpret_cast<float*>(base + (r == 0 ? L.off_gam : (r == 1 ? L.off_bet : L.off_al))) +
+                   (r < 2 ? i : i * m + (r - 2));
+      cp_async4(dst, src);
+    }
+  };
 
   float w[PRISM_MAX_W];
 #pragma unroll
@@ -113,79 +183,89 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p) {
   const size_t sbase = (((size_t)b * H + h) * dv + c) * dk + EPL * j;
 #pragma unroll
   for (int e = 0; e < EPL; e += 4) {
-    const float4 f = p.S0 ? __ldg(reinterpret_cast<const float4*>(p.S0 + sbase + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 f =
+        p.S0 ? __ldg(reinterpret_cast<const float4*>(p.S0 + sbase + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
     s[e] = f.x; s[e + 1] = f.y; s[e + 2] = f.z; s[e + 3] = f.w;
   }
 
-  auto fetch = [&](int t, Tok<T, EPL, MP>& x) {
-    const size_t tok = ((size_t)b * T_ + t) * H + h;
-    x.k.load(k + tok * dk + EPL * j);
-    x.q.load(q + tok * dk + EPL * j);
-    x.v = ld1<T>(v + tok * dv + c);
-    x.gam = __ldg(p.gamma + tok);
-    x.bet = __ldg(p.beta + tok);
-    if (prefetch_dirs) {
+  const int ntiles = (len + TT - 1) / TT;
+  if (ntiles > 0) load_tile(0, 0);
+  cp_async_commit();
+  for (int ti = 0; ti < ntiles; ++ti) {
+    const int buf = ti & 1;
+    if (ti + 1 < ntiles) load_tile(ti + 1, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait_1();  // tile ti has landed (the next may still be in flight)
+    __syncthreads();
+    const uint8_t* base = smem + buf * L.bytes;
+    const T* sk_ = reinterpret_cast<const T*>(base + L.off_k);
+    const T* sq_ = reinterpret_cast<const T*>(base + L.off_q);
+    const T* su_ = reinterpret_cast<const T*>(base + L.off_u);
+    const T* sv_ = reinterpret_cast<const T*>(base + L.off_v);
+    const T* sg_ = reinterpret_cast<const T*>(base + L.off_g);
+    const float* sgam = reinterpret_cast<const float*>(base + L.off_gam);
+    const float* sbet = reinterpret_cast<const float*>(base + L.off_bet);
+    const float* sal = reinterpret_cast<const float*>(base + L.off_al);
+    const int t0 = ti * TT, nt = min(TT, len - t0);
+    const int cr = row_ok ? lrow : 0;
+    for (int i = 0; i < nt; ++i) {
+      const T* kk = sk_ + i * dk + EPL * j;
+      float sk = 0.f;
 #pragma unroll
-      for (int l = 0; l < MP; ++l) {
-        if (l < m) {
-          const size_t tl = tok * m + l;
-          x.u[l].load(u + tl * dk + EPL * j);
-          x.g[l] = ld1<T>(g + tl * dv + c);
-          x.al[l] = __ldg(p.alpha + tl);
-        }
+      for (int e = 0; e < EPL; e += 4) {
+        const float4 f = ld4_smem<T>(kk + e);
+        sk += s[e] * f.x + s[e + 1] * f.y + s[e + 2] * f.z + s[e + 3] * f.w;
       }
-    }
-  };
+      sk = row_sum<LPR>(sk);
 
-  Tok<T, EPL, MP> cur, nxt;
-  if (len > 0) fetch(0, cur);
-  for (int t = 0; t < len; ++t) {
-    if (t + 1 < len) fetch(t + 1, nxt);
-    const size_t tok = ((size_t)b * T_ + t) * H + h;
-
-    // (S_{t-1} k_t)_c
-    const float sk = row_sum<LPR>(cur.k.dot(s));
-
-    // ShortConv anchor and anchor residual
-    const float vt = cur.v;
-    float a = w[0] * vt;
+      // ShortConv anchor and anchor residual
+      const float vt = to_f<T>(sv_[i * RPB + cr]);
+      float a = w[0] * vt;
 #pragma unroll
-    for (int i = 1; i < PRISM_MAX_W; ++i) a += w[i] * hist[i - 1];
-    float r = vt - a;
+      for (int z = 1; z < PRISM_MAX_W; ++z) a += w[z] * hist[z - 1];
+      float r = vt - a;
 #pragma unroll
-    for (int i = PRISM_MAX_W - 1; i > 0; --i) hist[i] = hist[i - 1];
-    hist[0] = vt;
+      for (int z = PRISM_MAX_W - 1; z > 0; --z) hist[z] = hist[z - 1];
+      hist[0] = vt;
 
-    // gated delta write: gamma S (I - beta k k^T) + beta v k^T
-    const float gam = cur.gam;
-    const float coef = cur.bet * (vt - gam * sk);
+      // gated delta write: gamma S (I - beta k k^T) + beta v k^T
+      const float gam = sgam[i];
+      const float coef = sbet[i] * (vt - gam * sk);
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) s[e] *= gam;
-    cur.k.axpy(coef, s);
-
-    // rank-m residual write
-    if (prefetch_dirs) {
-#pragma unroll
-      for (int l = 0; l < MP; ++l) {
-        if (l < m) {
-          r *= 1.f - cur.g[l];
-          cur.u[l].axpy(cur.al[l] * r, s);
-        }
+      for (int e = 0; e < EPL; e += 4) {
+        const float4 f = ld4_smem<T>(kk + e);
+        s[e] = gam * s[e] + coef * f.x;
+        s[e + 1] = gam * s[e + 1] + coef * f.y;
+        s[e + 2] = gam * s[e + 2] + coef * f.z;
+        s[e + 3] = gam * s[e + 3] + coef * f.w;
       }
-    } else {
+      // rank-m residual write
       for (int l = 0; l < m; ++l) {
-        const size_t tl = tok * m + l;
-        r *= 1.f - ld1<T>(g + tl * dv + c);
-        RowVec<T, EPL> uu;
-        uu.load(u + tl * dk + EPL * j);
-        uu.axpy(__ldg(p.alpha + tl) * r, s);
+        r *= 1.f - to_f<T>(sg_[(i * m + l) * RPB + cr]);
+        const float rho = sal[i * m + l] * r;
+        const T* uu = su_ + ((size_t)i * m + l) * dk + EPL * j;
+#pragma unroll
+        for (int e = 0; e < EPL; e += 4) {
+          const float4 f = ld4_smem<T>(uu + e);
+          s[e] += rho * f.x;
+          s[e + 1] += rho * f.y;
+          s[e + 2] += rho * f.z;
+          s[e + 3] += rho * f.w;
+        }
       }
+      const T* qq = sq_ + i * dk + EPL * j;
+      float oq = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; e += 4) {
+        const float4 f = ld4_smem<T>(qq + e);
+        oq += s[e] * f.x + s[e + 1] * f.y + s[e + 2] * f.z + s[e + 3] * f.w;
+      }
+      oq = row_sum<LPR>(oq);
+      if (row_ok && j == 0) st1<T>(o + (((size_t)b * T_ + t0 + i) * H + h) * dv + c, oq);
     }
-
-    const float oq = row_sum<LPR>(cur.q.dot(s));
-    if (row_ok && j == 0) st1<T>(o + tok * dv + c, oq);
-    cur = nxt;
+    __syncthreads();  // the buffer is refilled next iteration
   }
+  cp_async_wait_0();
   if (row_ok && j == 0)
     for (int t = len; t < T_; ++t) st1<T>(o + (((size_t)b * T_ + t) * H + h) * dv + c, 0.f);
   if (row_ok && p.S_final) {
@@ -198,12 +278,13 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p) {
 template <typename T, int LPR, int EPL>
 cudaError_t launch_shape(const ScanParams& p, cudaStream_t stream) {
   constexpr int RPB = kBlock / LPR;
+  const int TT = tile_tokens<T>(p.d_k, p.L - 1, RPB);
+  const int smem = 2 * TileLayout(TT, p.d_k, p.L - 1, RPB, sizeof(T)).bytes;
+  cudaError_t err =
+      cudaFuncSetAttribute(recurrent_scan_kernel<T, LPR, EPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
   dim3 grid((p.d_v + RPB - 1) / RPB, p.H, p.B);
-  constexpr int MPMAX = sizeof(T) == 2 ? MPF : 3;  // fp32 inputs: prefetch at most 3 directions
-  if (p.L - 1 <= 3)
-    recurrent_scan_kernel<T, LPR, EPL, 3><<<grid, kBlock, 0, stream>>>(p);
-  else
-    recurrent_scan_kernel<T, LPR, EPL, MPMAX><<<grid, kBlock, 0, stream>>>(p);
+  recurrent_scan_kernel<T, LPR, EPL><<<grid, kBlock, smem, stream>>>(p, TT);
   return cudaGetLastError();
 }
 
