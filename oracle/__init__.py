@@ -6,6 +6,7 @@ CPU-baseline leg of ``bench.py`` may import it.  The library never does.
 from .prism_oracle import (  # noqa: F401
     affine_maps,
     gdn_seq,
+    gelu,
     max_abs_rel_err,
     prism_chunked,
     prism_seq,

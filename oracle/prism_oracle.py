@@ -49,6 +49,7 @@ import numpy as np
 __all__ = [
     "shortconv_anchor",
     "residual_chain",
+    "gelu",
     "residual_write",
     "affine_maps",
     "prism_seq",
@@ -91,39 +92,55 @@ def shortconv_anchor(v, conv_w) -> np.ndarray:
     return a
 
 
-def residual_chain(v, conv_w, gain) -> np.ndarray:
-    """Residuals r_{t,1..L-1} of the linearised chain.
+def gelu(x):
+    """GELU(x) = x * Phi(x) = 0.5 x (1 + erf(x / sqrt(2))), the exact (erf) form."""
+    from scipy.special import erf
+
+    x = _f64(x)
+    return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))
+
+
+def residual_chain(v, conv_w, gain, chain: str = "linear") -> np.ndarray:
+    """Residuals r_{t,1..L-1} of the residual chain.
 
     [summary] sec. 2.2: the residual is reduced greedily step by step starting
-    from the anchor residual; [blog] "消除 Step 间串行": with the nonlinearity
-    absorbed into the preconditioner the chain is an element-wise linear
-    recurrence.  Here r_0 = v - a and r_l = (1 - g_l) * r_{l-1}, taken one step
-    at a time (the closed form is a test).
+    from the anchor residual, r^{(l+1)} = r^{(l)} - delta^{(l)} with
+    delta^{(l)} = GELU(p^{(l)} * r^{(l)}).
+
+    chain = "linear" (the path the library runs by default): [blog] "消除 Step
+    间串行": with the nonlinearity absorbed into the preconditioner the chain is
+    an element-wise linear recurrence, r_l = (1 - g_l) * r_{l-1}, g the
+    per-channel gain.  chain = "gelu": the exact step above with p = gain,
+    r_l = r_{l-1} - GELU(g_l * r_{l-1}).  Both start at r_0 = v - a and are taken
+    one step at a time (the linear closed form is a test).
 
     gain: [B,T,H,m,d_v] with m = L-1.  Returns r: [B,T,H,m,d_v].
     """
+    if chain not in ("linear", "gelu"):
+        raise ValueError(f"unknown chain {chain!r}")
     v = _f64(v)
     gain = _f64(gain)
     m = gain.shape[3]
     r = v - shortconv_anchor(v, conv_w)
     out = np.empty(gain.shape, dtype=np.float64)
     for l in range(m):
-        r = (1.0 - gain[:, :, :, l, :]) * r
+        g = gain[:, :, :, l, :]
+        r = (1.0 - g) * r if chain == "linear" else r - gelu(g * r)
         out[:, :, :, l, :] = r
     return out
 
 
-def residual_write(v, u, alpha, gain, conv_w) -> np.ndarray:
+def residual_write(v, u, alpha, gain, conv_w, chain: str = "linear") -> np.ndarray:
     """Per-token residual write dS_res,t = sum_l alpha_{t,l} r_{t,l} u_{t,l}^T
     ([blog] "核心迭代形式" and "架构形式": the write is the GDN write plus a
     low-rank correction).  Returns [B,T,H,d_v,d_k]."""
-    r = residual_chain(v, conv_w, gain)
+    r = residual_chain(v, conv_w, gain, chain)
     u = _f64(u)
     alpha = _f64(alpha)
     return np.einsum("bthl,bthlc,bthlj->bthcj", alpha, r, u)
 
 
-def affine_maps(k, v, gamma, beta, u, alpha, gain, conv_w, lengths=None):
+def affine_maps(k, v, gamma, beta, u, alpha, gain, conv_w, lengths=None, chain: str = "linear"):
     """The pair (A_t, B_t) of the state update S_t = S_{t-1} A_t + B_t
     ([summary] sec. 2.1: forgetting A_t is the rank-1 gated-delta transition,
     all expressiveness sits in the injection B_t; [blog] "背景": this linear form
@@ -142,14 +159,14 @@ def affine_maps(k, v, gamma, beta, u, alpha, gain, conv_w, lengths=None):
     A = gamma[..., None, None] * (eye - beta[..., None, None] * k[..., :, None] * k[..., None, :])
     Bt = beta[..., None, None] * v[..., :, None] * k[..., None, :]
     if u is not None and np.asarray(u).shape[3] > 0:
-        Bt = Bt + residual_write(v, u, alpha, gain, conv_w)
+        Bt = Bt + residual_write(v, u, alpha, gain, conv_w, chain)
     valid = _valid_mask(B, T, lengths)[:, :, None, None, None]
     A = np.where(valid, A, eye)
     Bt = np.where(valid, Bt, 0.0)
     return A, Bt
 
 
-def prism_seq(q, k, v, gamma, beta, u, alpha, gain, conv_w, S0=None, lengths=None):
+def prism_seq(q, k, v, gamma, beta, u, alpha, gain, conv_w, S0=None, lengths=None, chain: str = "linear"):
     """Token-by-token PRISM scan (the definition in the module docstring).
 
     Shapes (token-major): q, k [B,T,H,d_k]; v [B,T,H,d_v]; gamma, beta [B,T,H];
@@ -166,7 +183,7 @@ def prism_seq(q, k, v, gamma, beta, u, alpha, gain, conv_w, S0=None, lengths=Non
     m = 0 if u is None else np.asarray(u).shape[3]
     if m > 0:
         u, alpha = _f64(u), _f64(alpha)
-        r = residual_chain(v, conv_w, gain)
+        r = residual_chain(v, conv_w, gain, chain)
     S = np.zeros((B, H, dv, dk)) if S0 is None else _f64(S0).copy()
     o = np.zeros((B, T, H, dv))
     valid = _valid_mask(B, T, lengths)
@@ -215,7 +232,7 @@ def gdn_seq(q, k, v, gamma, beta, S0=None, lengths=None):
     return o, S
 
 
-def prism_chunked(q, k, v, gamma, beta, u, alpha, gain, conv_w, chunk, S0=None, lengths=None):
+def prism_chunked(q, k, v, gamma, beta, u, alpha, gain, conv_w, chunk, S0=None, lengths=None, chain: str = "linear"):
     """Chunkwise-parallel form of the same scan, fp64 (the decomposition the
     tensor-core path uses; the chunkwise scan is how the method keeps GDN-class
     throughput, [blog] "消除 Token 间串行").
@@ -242,7 +259,7 @@ def prism_chunked(q, k, v, gamma, beta, u, alpha, gain, conv_w, chunk, S0=None, 
     if m > 0:
         u = _f64(u)
         alpha = np.where(valid[:, :, None, None], _f64(alpha), 0.0)
-        rho = alpha[..., None] * residual_chain(v, conv_w, gain)       # [B,T,H,m,dv]
+        rho = alpha[..., None] * residual_chain(v, conv_w, gain, chain)  # [B,T,H,m,dv]
     S = np.zeros((B, H, dv, dk)) if S0 is None else _f64(S0).copy()
     o = np.zeros((B, T, H, dv))
     # move heads next to batch: [B,H,T,...]

@@ -377,3 +377,61 @@ def test_max_abs_rel_err_metric():
     assert max_abs_rel_err(x, ref) == pytest.approx(0.05)
     x[0, 1, 1, 2] = 1e-3   # an all-zero slice uses the 1e-6 floor
     assert max_abs_rel_err(x, ref) == pytest.approx(1e3)
+
+
+# ---------------------------------------------------------------- exact GELU chain (NEXT variant)
+def test_gelu_matches_library():
+    """The oracle's GELU is the exact erf form: torch's gelu(approximate='none') and the
+    standard library's math.erf give the same numbers."""
+    import math
+
+    import torch
+
+    x = np.linspace(-6, 6, 97)
+    ours = __import__("oracle").gelu(x)
+    ref = torch.nn.functional.gelu(torch.tensor(x, dtype=torch.float64), approximate="none").numpy()
+    np.testing.assert_allclose(ours, ref, rtol=1e-14, atol=1e-15)
+    for xi, oi in zip(x[::8], ours[::8]):
+        assert abs(oi - 0.5 * xi * (1.0 + math.erf(xi / math.sqrt(2.0)))) < 1e-14
+
+
+def test_gelu_chain_special_cases():
+    """p = 0: GELU(0) = 0, nothing is removed, every r_l equals r_0.  A single step
+    against a hand-evaluated GELU (math.erf), and the linear chain is unchanged."""
+    import math
+
+    rng = np.random.default_rng(20)
+    d = rand_inputs(rng, L=4)
+    r = residual_chain(d["v"], d["conv_w"], np.zeros_like(d["gain"]), chain="gelu")
+    r0 = d["v"] - shortconv_anchor(d["v"], d["conv_w"])
+    for l in range(3):
+        np.testing.assert_array_equal(r[:, :, :, l], r0)
+    v = np.array([[[[0.7, -1.3]]]])              # B=T=H=1, d_v=2
+    w = np.zeros((1, 2, 1))                      # no anchor: r_0 = v
+    p = np.array([[[[[2.0, 0.5]]]]])             # one step
+    r1 = residual_chain(v, w, p, chain="gelu")[0, 0, 0, 0]
+    for c in range(2):
+        x = p[0, 0, 0, 0, c] * v[0, 0, 0, c]
+        ref = v[0, 0, 0, c] - 0.5 * x * (1.0 + math.erf(x / math.sqrt(2.0)))
+        assert abs(r1[c] - ref) < 1e-15
+    np.testing.assert_array_equal(residual_chain(d["v"], d["conv_w"], d["gain"]),
+                                  residual_chain(d["v"], d["conv_w"], d["gain"], chain="linear"))
+
+
+@pytest.mark.parametrize("chunk", [4, 64])
+def test_gelu_chain_chunked_equals_sequential(chunk):
+    rng = np.random.default_rng(21)
+    d = rand_inputs(rng, B=2, T=70, H=2, dk=8, dv=6, L=4, s0=True, lengths=np.array([70, 33]))
+    o, S = prism_seq(**d, chain="gelu")
+    oc, Sc = prism_chunked(**d, chunk=chunk, chain="gelu")
+    assert max_abs_rel_err(oc, o) < 1e-10
+    assert max_abs_rel_err(Sc, S, slice_axes=(0, 1)) < 1e-10
+
+
+def test_gelu_chain_rank():
+    rng = np.random.default_rng(22)
+    d = rand_inputs(rng, B=1, T=5, H=1, dk=12, dv=12, L=5)
+    dS = residual_write(d["v"], d["u"], d["alpha"], d["gain"], d["conv_w"], chain="gelu")
+    for t in range(5):
+        s = np.linalg.svd(dS[0, t, 0], compute_uv=False)
+        assert int((s > 1e-10 * s[0]).sum()) == 4
