@@ -77,6 +77,13 @@ enum prism_dtype {
   PRISM_FP32 = 1
 };
 
+/* Residual chain step.  Exact: gist.science PRISM explainer, 2.2 Input-Anchored Loop
+ * Unrolling (Residual Update).  Linearised: ICML 2026 PRISM write-up, 消除 Step 间串行. */
+enum prism_chain {
+  PRISM_CHAIN_LINEAR = 0, /* r_l = (1 - g_l) * r_{l-1}: the linearised chain (default) */
+  PRISM_CHAIN_GELU = 1    /* r_l = r_{l-1} - GELU(g_l * r_{l-1}), GELU(x) = x Phi(x) (erf form) */
+};
+
 enum prism_status {
   PRISM_OK = 0,
   PRISM_ERR_INVALID_ARG = 1, /* NULL where required, non-positive size, L < 1, W < 1, ... */
@@ -113,6 +120,21 @@ int prism_scan_fwd(const void* q, const void* k, const void* v,
                    int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
                    int dtype, void* o, float* S_final,
                    void* workspace, size_t workspace_bytes, prism_stream_t stream);
+
+/*
+ * prism_scan_fwd_ex - prism_scan_fwd with the residual chain selected by `chain`
+ * (PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU; any other value is PRISM_ERR_INVALID_ARG).
+ * For PRISM_CHAIN_GELU the `gain` tensor holds the predictor output p of the exact
+ * refinement step r <- r - GELU(p * r) (gist.science PRISM explainer, 2.2), any real value.
+ * prism_scan_fwd is prism_scan_fwd_ex with PRISM_CHAIN_LINEAR.
+ */
+int prism_scan_fwd_ex(const void* q, const void* k, const void* v,
+                      const float* gamma, const float* beta,
+                      const void* u, const float* alpha, const void* gain,
+                      const float* conv_w, const float* S0, const int32_t* lengths,
+                      int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
+                      int dtype, void* o, float* S_final,
+                      void* workspace, size_t workspace_bytes, prism_stream_t stream, int chain);
 
 /* Bytes of device workspace prism_scan_fwd needs for these sizes (0 if none).
  * Returns 0 for invalid sizes as well; prism_scan_fwd reports those. */
@@ -158,6 +180,12 @@ int prism_prologue_fwd(const void* v, const float* alpha, const void* gain,
  * kernel, 0 if on the CUDA-core token-by-token kernel (sizes as for
  * prism_scan_fwd; unsupported sizes also give 0). */
 int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype);
+
+/* prism_prologue_fwd with the residual chain selected by `chain` (see prism_scan_fwd_ex). */
+int prism_prologue_fwd_ex(const void* v, const float* alpha, const void* gain,
+                          const float* conv_w, const int32_t* lengths,
+                          int B, int T, int H, int d_v, int L, int W, int dtype,
+                          float* rho_out, prism_stream_t stream, int chain);
 
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the

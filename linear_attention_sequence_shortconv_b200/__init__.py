@@ -9,6 +9,8 @@ from ._lib import (  # noqa: F401
     EXPORTS,
     PRISM_BF16,
     PRISM_FP32,
+    PRISM_CHAIN_GELU,
+    PRISM_CHAIN_LINEAR,
     PrismError,
     lib,
     prologue_fwd,

@@ -18,6 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libprism.so")
 
 PRISM_BF16 = 0
 PRISM_FP32 = 1
+PRISM_CHAIN_LINEAR = 0
+PRISM_CHAIN_GELU = 1
 STATUS = {
     0: "PRISM_OK",
     1: "PRISM_ERR_INVALID_ARG",
@@ -30,9 +32,11 @@ STATUS = {
 # Every symbol include/prism.h declares.
 EXPORTS = (
     "prism_scan_fwd",
+    "prism_scan_fwd_ex",
     "prism_scan_fwd_workspace_size",
     "prism_scan_fwd_host",
     "prism_prologue_fwd",
+    "prism_prologue_fwd_ex",
     "prism_scan_fwd_uses_tensor_cores",
     "prism_stream_status",
     "prism_set_spin_limit",
@@ -65,12 +69,16 @@ def lib() -> ctypes.CDLL:
     L.prism_scan_fwd.argtypes = [vp, vp, vp, fp, fp, vp, fp, vp, fp, fp, i32p,
                                  ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, fp, vp, cs, vp]
     L.prism_scan_fwd.restype = ci
+    L.prism_scan_fwd_ex.argtypes = L.prism_scan_fwd.argtypes + [ci]
+    L.prism_scan_fwd_ex.restype = ci
     L.prism_scan_fwd_workspace_size.argtypes = [ci] * 9
     L.prism_scan_fwd_workspace_size.restype = cs
     L.prism_scan_fwd_host.argtypes = ([vp] * 11 + [vp] * 11 + [ci] * 9 + [vp, vp, vp, vp, vp, cs, vp])
     L.prism_scan_fwd_host.restype = ci
     L.prism_prologue_fwd.argtypes = [vp, fp, vp, fp, i32p, ci, ci, ci, ci, ci, ci, ci, fp, vp]
     L.prism_prologue_fwd.restype = ci
+    L.prism_prologue_fwd_ex.argtypes = L.prism_prologue_fwd.argtypes + [ci]
+    L.prism_prologue_fwd_ex.restype = ci
     L.prism_scan_fwd_uses_tensor_cores.argtypes = [ci] * 6
     L.prism_scan_fwd_uses_tensor_cores.restype = ci
     L.prism_stream_status.argtypes = [vp]
@@ -111,6 +119,15 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"q/k/v/u/gain must be bfloat16 or float32, got {t.dtype}")
 
 
+CHAINS = {"linear": PRISM_CHAIN_LINEAR, "gelu": PRISM_CHAIN_GELU}
+
+
+def _chain_code(chain: str) -> int:
+    if chain not in CHAINS:
+        raise ValueError(f"chain must be one of {sorted(CHAINS)}, got {chain!r}")
+    return CHAINS[chain]
+
+
 def _check(t: Optional[torch.Tensor], name: str, dtype=None, required=True):
     if t is None:
         if required:
@@ -130,8 +147,11 @@ def workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype_code) -> int:
 
 def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 64,
              S0=None, lengths=None, want_state: bool = True, o=None, S_final=None,
-             workspace=None, stream=None):
+             workspace=None, stream=None, chain: str = "linear"):
     """PRISM mixer forward on CUDA tensors; returns (o, S_final or None).
+
+    ``chain`` picks the residual chain step: "linear" r <- (1 - g) r, or "gelu"
+    r <- r - GELU(g r) (exact erf GELU; ``gain`` then holds the predictor p).
 
     Shapes as in include/prism.h: q, k [B,T,H,d_k]; v [B,T,H,d_v]; gamma, beta
     [B,T,H] fp32; u [B,T,H,L-1,d_k]; alpha [B,T,H,L-1] fp32; gain [B,T,H,L-1,d_v];
@@ -159,15 +179,16 @@ def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 
     ws_bytes = workspace_size(B, T, H, d_k, d_v, L, W, chunk, code)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    rc = lib().prism_scan_fwd(
+    chain_code = _chain_code(chain)
+    rc = lib().prism_scan_fwd_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
         _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
         _ptr(conv_w), _ptr(S0), _ptr(lengths),
         B, T, H, d_k, d_v, L, W, chunk, code,
         _ptr(o), _ptr(S_final if want_state else None),
-        _ptr(workspace), ws_bytes if workspace is not None else 0, _stream_handle(stream))
+        _ptr(workspace), ws_bytes if workspace is not None else 0, _stream_handle(stream), chain_code)
     if rc != 0:
-        raise PrismError(rc, "prism_scan_fwd")
+        raise PrismError(rc, "prism_scan_fwd_ex")
     return o, (S_final if want_state else None)
 
 
@@ -192,8 +213,9 @@ def scan_fwd_host(host: dict, dev: dict, L: int, chunk: int = 64, stream=None):
         raise PrismError(rc, "prism_scan_fwd_host")
 
 
-def prologue_fwd(v, alpha, gain, conv_w, L: int, lengths=None, stream=None):
+def prologue_fwd(v, alpha, gain, conv_w, L: int, lengths=None, stream=None, chain: str = "linear"):
     """rho_{t,l} = alpha_{t,l} r_{t,l} as [B,T,H,L-1,d_v] fp32 (CUDA)."""
+    chain_code = _chain_code(chain)
     code = _dtype_code(v)
     _check(v, "v")
     _check(gain, "gain", v.dtype)
@@ -202,11 +224,11 @@ def prologue_fwd(v, alpha, gain, conv_w, L: int, lengths=None, stream=None):
     _check(lengths, "lengths", torch.int32, required=False)
     B, T, H, d_v = v.shape
     rho = torch.empty((B, T, H, L - 1, d_v), dtype=torch.float32, device=v.device)
-    rc = lib().prism_prologue_fwd(_ptr(v), _ptr(alpha), _ptr(gain), _ptr(conv_w), _ptr(lengths),
-                                  B, T, H, d_v, L, conv_w.shape[-1], code, _ptr(rho),
-                                  _stream_handle(stream))
+    rc = lib().prism_prologue_fwd_ex(_ptr(v), _ptr(alpha), _ptr(gain), _ptr(conv_w), _ptr(lengths),
+                                     B, T, H, d_v, L, conv_w.shape[-1], code, _ptr(rho),
+                                     _stream_handle(stream), chain_code)
     if rc != 0:
-        raise PrismError(rc, "prism_prologue_fwd")
+        raise PrismError(rc, "prism_prologue_fwd_ex")
     return rho
 
 

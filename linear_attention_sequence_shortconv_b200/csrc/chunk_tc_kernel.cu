@@ -111,28 +111,7 @@ __device__ __forceinline__ void st_bf16x8(uint8_t* base, uint32_t off, const flo
   *reinterpret_cast<uint4*>(base + off) = u;
 }
 
-__device__ __forceinline__ void ld_bf16x8(const __nv_bfloat16* p, float* x) {
-  uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    float2 f = __bfloat1622float2(h[e]);
-    x[2 * e] = f.x;
-    x[2 * e + 1] = f.y;
-  }
-}
-
 __device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
-
-__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* x) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    float2 f = __bfloat1622float2(h[e]);
-    x[2 * e] = f.x;
-    x[2 * e + 1] = f.y;
-  }
-}
 
 // element e (0..7) of 8 packed bf16
 __device__ __forceinline__ float bf16_at(const uint4& u, int e) {
@@ -154,7 +133,9 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t base, int kk, uint32_t lbo) 
   return sdesc_sw128(base + (uint32_t)kk * 2048u, lbo, 1024);
 }
 
-template <int D, int M>
+// CH: residual chain step (PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU), fixed at compile
+// time so the linear chain carries none of the GELU step's code or registers.
+template <int D, int M, int CH>
 __global__ void __launch_bounds__(kThreads, 1)
     prism_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                           const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_v,
@@ -385,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float alc = al[pass][l] * ci;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            r[e] *= 1.f - bf16_at(graw[pass][l], e);
+            r[e] = chain_step(r[e], bf16_at(graw[pass][l], e), CH);
             rho[e] = alc * r[e];
           }
           st_bf16x8(sP, sw128_offset(l * 64 + i, pc8, Ly::U_ATOM), rho);
@@ -936,13 +917,13 @@ bool encode(CUtensorMap* map, const void* ptr, int rank, const cuuint64_t* dims,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int M>
+template <int D, int M, int CH>
 cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
   using Ly = Layout<D, M>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(prism_chunk_tc_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(prism_chunk_tc_kernel<D, M, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     Ly::SMEM_ALLOC);
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -968,19 +949,25 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
            static_cast<const __nv_bfloat16*>(p.u), static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha,
            static_cast<const __nv_bfloat16*>(p.gain), p.conv_w, p.S0, p.lengths,
            static_cast<__nv_bfloat16*>(p.o), p.S_final, p.B, p.T, p.H, p.W, p.status, p.spin_limit};
-  prism_chunk_tc_kernel<D, M><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, mo, a);
+  prism_chunk_tc_kernel<D, M, CH><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, mo, a);
   return cudaGetLastError();
+}
+
+template <int D, int CH>
+cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
+  switch (p.L - 1) {
+    case 1: return launch_dm<D, 1, CH>(p, stream);
+    case 2: return launch_dm<D, 2, CH>(p, stream);
+    case 3: return launch_dm<D, 3, CH>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <int D>
 cudaError_t launch_d(const ScanParams& p, cudaStream_t stream) {
-  switch (p.L - 1) {
-    case 0: return launch_dm<D, 0>(p, stream);
-    case 1: return launch_dm<D, 1>(p, stream);
-    case 2: return launch_dm<D, 2>(p, stream);
-    case 3: return launch_dm<D, 3>(p, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  if (p.L == 1) return launch_dm<D, 0, PRISM_CHAIN_LINEAR>(p, stream);  // no residual chain at L = 1
+  if (p.chain == PRISM_CHAIN_GELU) return launch_dc<D, PRISM_CHAIN_GELU>(p, stream);
+  return launch_dc<D, PRISM_CHAIN_LINEAR>(p, stream);
 }
 
 }  // namespace

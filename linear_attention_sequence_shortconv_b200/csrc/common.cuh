@@ -27,7 +27,20 @@ struct ScanParams {
   int B, T, H, d_k, d_v, L, W, chunk;
   int* status;            // per-device status word (PRISM_OK / PRISM_ERR_TIMEOUT)
   long long spin_limit;   // bound of every device-side wait
+  int chain;              // PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU
 };
+
+// One step of the residual chain.  Exact form (gist.science PRISM explainer, 2.2
+// Input-Anchored Loop Unrolling, Residual Update): r <- r - GELU(p * r), GELU in its
+// erf form.  Linearised form (ICML 2026 PRISM write-up, 消除 Step 间串行: the GELU is
+// absorbed into the preconditioner): r <- (1 - g) r.
+__device__ __forceinline__ float chain_step(float r, float g, int chain) {
+  if (chain == PRISM_CHAIN_GELU) {
+    const float x = g * r;
+    return r - 0.5f * x * (1.f + erff(x * 0.7071067811865476f));
+  }
+  return r * (1.f - g);
+}
 
 // ---------------------------------------------------------------- element I/O
 template <typename T>

@@ -9,7 +9,7 @@ namespace prism {
 cudaError_t launch_recurrent_scan(const ScanParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_prologue(const void* v, const float* alpha, const void* gain, const float* conv_w,
                             const int32_t* lengths, int B, int T, int H, int d_v, int L, int W,
-                            int dtype, float* rho, cudaStream_t stream);
+                            int dtype, float* rho, cudaStream_t stream, int chain);
 bool chunk_tc_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
 cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream);
 }  // namespace prism
@@ -101,6 +101,16 @@ int prism_scan_fwd(const void* q, const void* k, const void* v, const float* gam
                    const float* S0, const int32_t* lengths, int B, int T, int H, int d_k, int d_v,
                    int L, int W, int chunk, int dtype, void* o, float* S_final, void* workspace,
                    size_t workspace_bytes, prism_stream_t stream) {
+  return prism_scan_fwd_ex(q, k, v, gamma, beta, u, alpha, gain, conv_w, S0, lengths, B, T, H, d_k, d_v, L, W,
+                           chunk, dtype, o, S_final, workspace, workspace_bytes, stream, PRISM_CHAIN_LINEAR);
+}
+
+int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
+                      const void* u, const float* alpha, const void* gain, const float* conv_w,
+                      const float* S0, const int32_t* lengths, int B, int T, int H, int d_k, int d_v,
+                      int L, int W, int chunk, int dtype, void* o, float* S_final, void* workspace,
+                      size_t workspace_bytes, prism_stream_t stream, int chain) {
+  if (chain != PRISM_CHAIN_LINEAR && chain != PRISM_CHAIN_GELU) return PRISM_ERR_INVALID_ARG;
   int rc = check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype);
   if (rc != PRISM_OK) return rc;
   if (!q || !k || !v || !gamma || !beta || !conv_w || !o) return PRISM_ERR_INVALID_ARG;
@@ -117,7 +127,7 @@ int prism_scan_fwd(const void* q, const void* k, const void* v, const float* gam
 
   prism::ScanParams p{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr,
                       L > 1 ? gain : nullptr, conv_w, S0, lengths, o, S_final,
-                      B, T, H, d_k, d_v, L, W, chunk, status, g_spin_limit.load()};
+                      B, T, H, d_k, d_v, L, W, chunk, status, g_spin_limit.load(), chain};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (prism::chunk_tc_supported(d_k, d_v, L, W, chunk, dtype))
@@ -175,6 +185,14 @@ int prism_scan_fwd_host(const void* host_q, const void* host_k, const void* host
 int prism_prologue_fwd(const void* v, const float* alpha, const void* gain, const float* conv_w,
                        const int32_t* lengths, int B, int T, int H, int d_v, int L, int W, int dtype,
                        float* rho_out, prism_stream_t stream) {
+  return prism_prologue_fwd_ex(v, alpha, gain, conv_w, lengths, B, T, H, d_v, L, W, dtype, rho_out, stream,
+                               PRISM_CHAIN_LINEAR);
+}
+
+int prism_prologue_fwd_ex(const void* v, const float* alpha, const void* gain, const float* conv_w,
+                          const int32_t* lengths, int B, int T, int H, int d_v, int L, int W, int dtype,
+                          float* rho_out, prism_stream_t stream, int chain) {
+  if (chain != PRISM_CHAIN_LINEAR && chain != PRISM_CHAIN_GELU) return PRISM_ERR_INVALID_ARG;
   int rc = check_sizes(B, T, H, d_v, d_v, L, W, 64, dtype);
   if (rc != PRISM_OK) return rc;
   if (L < 2 || !v || !alpha || !gain || !conv_w || !rho_out) return PRISM_ERR_INVALID_ARG;
@@ -185,7 +203,7 @@ int prism_prologue_fwd(const void* v, const float* alpha, const void* gain, cons
   rc = device_setup(&status);
   if (rc != PRISM_OK) return rc;
   cudaError_t err = prism::launch_prologue(v, alpha, gain, conv_w, lengths, B, T, H, d_v, L, W, dtype,
-                                           rho_out, reinterpret_cast<cudaStream_t>(stream));
+                                           rho_out, reinterpret_cast<cudaStream_t>(stream), chain);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 

@@ -1,5 +1,5 @@
 // PRISM prologue on its own: ShortConv anchor, anchor residual and the
-// closed-form residual chain, giving rho_{t,l} = alpha_{t,l} r_{t,l}.
+// residual chain (closed-form linear or exact GELU steps), giving rho_{t,l} = alpha_{t,l} r_{t,l}.
 //
 // ICML 2026 PRISM write-up, 消除 Token 间串行 (a short convolution of the input
 // replaces the global state as the anchor) and 消除 Step 间串行 (with the GELU
@@ -20,7 +20,7 @@ struct PrologueParams {
   const float* conv_w;
   const int32_t* lengths;
   float* rho;
-  int B, T, H, d_v, L, W;
+  int B, T, H, d_v, L, W, chain;
 };
 
 template <typename T>
@@ -57,10 +57,10 @@ __global__ void __launch_bounds__(256) prologue_kernel(PrologueParams p) {
   for (int l = 0; l < m; ++l) {
     const size_t tl = tok * m + l;
     const float4 gg = ld4<T>(g + tl * dv + c0);
-    r.x *= 1.f - gg.x;
-    r.y *= 1.f - gg.y;
-    r.z *= 1.f - gg.z;
-    r.w *= 1.f - gg.w;
+    r.x = chain_step(r.x, gg.x, p.chain);
+    r.y = chain_step(r.y, gg.y, p.chain);
+    r.z = chain_step(r.z, gg.z, p.chain);
+    r.w = chain_step(r.w, gg.w, p.chain);
     const float al = __ldg(p.alpha + tl);
     out[(size_t)l * dv / 4] = make_float4(al * r.x, al * r.y, al * r.z, al * r.w);
   }
@@ -68,8 +68,8 @@ __global__ void __launch_bounds__(256) prologue_kernel(PrologueParams p) {
 
 cudaError_t launch_prologue(const void* v, const float* alpha, const void* gain, const float* conv_w,
                             const int32_t* lengths, int B, int T, int H, int d_v, int L, int W,
-                            int dtype, float* rho, cudaStream_t stream) {
-  PrologueParams p{v, alpha, gain, conv_w, lengths, rho, B, T, H, d_v, L, W};
+                            int dtype, float* rho, cudaStream_t stream, int chain) {
+  PrologueParams p{v, alpha, gain, conv_w, lengths, rho, B, T, H, d_v, L, W, chain};
   const size_t n = (size_t)B * T * H * (d_v / 4);
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (dtype == PRISM_FP32)

@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
       }
       // rank-m residual write
       for (int l = 0; l < m; ++l) {
-        r *= 1.f - to_f<T>(sg_[(i * m + l) * RPB + cr]);
+        r = chain_step(r, to_f<T>(sg_[(i * m + l) * RPB + cr]), p.chain);
         const float rho = sal[i * m + l] * r;
         const T* uu = su_ + ((size_t)i * m + l) * dk + EPL * j;
 #pragma unroll

@@ -9,18 +9,18 @@ from linear_attention_sequence_shortconv_b200 import synth
 TOL = {"bf16": 2e-2, "fp32": 1e-4}   # max-abs-relative error bars of the method's evaluation
 
 
-def gpu_run(inp: dict, w: synth.Workload, device="cuda:0", want_state=True, chunk=None):
+def gpu_run(inp: dict, w: synth.Workload, device="cuda:0", want_state=True, chunk=None, chain="linear"):
     import linear_attention_sequence_shortconv_b200 as prism
 
     d = {n: (t.to(device) if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
     o, S = prism.scan_fwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"],
                           d["conv_w"], L=w.L, chunk=chunk or w.chunk, S0=d["S0"], lengths=d["lengths"],
-                          want_state=want_state)
+                          want_state=want_state, chain=chain)
     torch.cuda.synchronize()
     return o.float().cpu().numpy(), (S.cpu().numpy() if S is not None else None)
 
 
-def oracle_run(inp: dict, w: synth.Workload, bh=None):
+def oracle_run(inp: dict, w: synth.Workload, bh=None, chain="linear"):
     """fp64 oracle; ``bh`` = list of (b, h) pairs to evaluate (sampling), else all."""
     from oracle import prism_seq
 
@@ -28,7 +28,7 @@ def oracle_run(inp: dict, w: synth.Workload, bh=None):
     if w.L == 1:
         x["u"] = x["alpha"] = x["gain"] = None
     if bh is None:
-        return prism_seq(**x)
+        return prism_seq(**x, chain=chain)
     outs, states = [], []
     for b, h in bh:
         sl = {}
@@ -43,7 +43,7 @@ def oracle_run(inp: dict, w: synth.Workload, bh=None):
                 sl[n] = a[b:b + 1]
             else:
                 sl[n] = a[b:b + 1, :, h:h + 1]
-        o, S = prism_seq(**sl)
+        o, S = prism_seq(**sl, chain=chain)
         outs.append(o[0, :, 0])
         states.append(S[0, 0])
     return outs, states

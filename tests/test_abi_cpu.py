@@ -95,3 +95,12 @@ def test_host_entry_invalid_arguments(L):
     bad = list(args)
     bad[22] = 0        # B = 0
     assert L.prism_scan_fwd_host(*bad) == 1
+
+
+def test_unknown_residual_chain_is_rejected(L):
+    a = [FAKE] * 9 + [None, None, 2, 8, 2, 64, 64, 4, 4, 64, 0, FAKE, None, None, 0, None]
+    for chain in (-1, 2, 7):
+        assert L.prism_scan_fwd_ex(*a, chain) == 1
+        assert L.prism_prologue_fwd_ex(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 64, 4, 4, 0, FAKE, None, chain) == 1
+    with pytest.raises(ValueError):
+        prism._lib._chain_code("tanh")
