@@ -9,6 +9,7 @@ from .prism_oracle import (  # noqa: F401
     gelu,
     max_abs_rel_err,
     prism_chunked,
+    prism_decode_step,
     prism_seq,
     residual_chain,
     residual_write,

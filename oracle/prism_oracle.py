@@ -38,7 +38,10 @@ chunkwise form ``prism_chunked`` against the token loop; the rank of the
 residual write; the zero-state and frozen-state special cases; the anchor
 against a library FIR filter; an exact rational evaluation of the affine form
 S_t = S_{t-1} A_t + B_t; linearity; split invariance; masking against
-truncation; and a hand-worked two-token example under tests/golden/.
+truncation; and a hand-worked two-token example under tests/golden/.  The
+one-token decode step ``prism_decode_step`` is pinned to the same hand-worked
+example, to exact recall, and to the sequence form (token-by-token decoding
+and the continuation of a prefix).
 """
 from __future__ import annotations
 
@@ -55,6 +58,7 @@ __all__ = [
     "prism_seq",
     "gdn_seq",
     "prism_chunked",
+    "prism_decode_step",
     "max_abs_rel_err",
 ]
 
@@ -200,6 +204,46 @@ def prism_seq(q, k, v, gamma, beta, u, alpha, gain, conv_w, S0=None, lengths=Non
         S = np.where(ok, S_new, S)
         o[:, t] = np.where(valid[:, t][:, None, None], np.einsum("bhcj,bhj->bhc", S, qt), 0.0)
     return o, S
+
+
+def prism_decode_step(q, k, v, gamma, beta, u, alpha, gain, conv_w, conv_state, S, chain: str = "linear"):
+    """One recurrent step of the scan (the O(1)-state inference form of the same
+    recurrence: [blog] "背景" / "Rank-1 写入瓶颈", a linear-attention model keeps a
+    fixed-size state and updates it once per token).
+
+    The ShortConv history that the sequence form reads from v_{t-1..t-W+1} is
+    carried explicitly: conv_state [B,H,W-1,d_v] holds v_{t-W+1}, ..., v_{t-1}
+    (oldest first; zeros before the start of a sequence).
+
+    q, k [B,H,d_k]; v [B,H,d_v]; gamma, beta [B,H]; u [B,H,m,d_k] (or None when
+    m = 0); alpha [B,H,m]; gain [B,H,m,d_v]; conv_w [H,d_v,W]; S [B,H,d_v,d_k].
+    Returns (o [B,H,d_v], S_new, conv_state_new), fp64.
+    """
+    if chain not in ("linear", "gelu"):
+        raise ValueError(f"unknown chain {chain!r}")
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    gamma, beta, S = _f64(gamma), _f64(beta), _f64(S)
+    w = _f64(conv_w)
+    W = w.shape[2]
+    hist = _f64(conv_state) if W > 1 else np.zeros(v.shape[:2] + (0, v.shape[2]))
+    a = w[None, :, :, 0] * v
+    for i in range(1, W):
+        a = a + w[None, :, :, i] * hist[:, :, W - 1 - i]
+    r = v - a
+    bt = beta[..., None, None]
+    write = bt * v[..., :, None] * k[..., None, :]
+    m = 0 if u is None else np.asarray(u).shape[2]
+    if m > 0:
+        u, alpha, gain = _f64(u), _f64(alpha), _f64(gain)
+        for l in range(m):
+            g = gain[:, :, l]
+            r = (1.0 - g) * r if chain == "linear" else r - gelu(g * r)
+            write = write + alpha[:, :, l][..., None, None] * r[..., :, None] * u[:, :, l][..., None, :]
+    Sk = np.einsum("bhcj,bhj->bhc", S, k)
+    S_new = gamma[..., None, None] * (S - bt * Sk[..., :, None] * k[..., None, :]) + write
+    o = np.einsum("bhcj,bhj->bhc", S_new, q)
+    hist_new = np.concatenate([hist[:, :, 1:], v[:, :, None]], axis=2) if W > 1 else hist
+    return o, S_new, hist_new
 
 
 def gdn_seq(q, k, v, gamma, beta, S0=None, lengths=None):
