@@ -187,6 +187,44 @@ int prism_prologue_fwd_ex(const void* v, const float* alpha, const void* gain,
                           int B, int T, int H, int d_v, int L, int W, int dtype,
                           float* rho_out, prism_stream_t stream, int chain);
 
+/*
+ * prism_decode_step - one recurrent step of the scan for every (b, h): the O(1)-state
+ * inference form of the recurrence above (ICML 2026 PRISM write-up, 背景 and
+ * Rank-1 写入瓶颈: a linear-attention layer keeps a fixed-size state and updates it
+ * once per token).  For one token t and each (b, h):
+ *   a = w[h,:,0] v_t + sum_{i=1}^{W-1} w[h,:,i] v_{t-i}   (v_{t-i} taken from conv_state)
+ *   r_0 = v_t - a;  r_l = chain step of r_{l-1} with gain g_l (see prism_scan_fwd_ex)
+ *   S <- gamma S (I - beta k k^T) + beta v_t k^T + sum_l alpha_l r_l u_l^T;   o = S q
+ * Decoding tokens one at a time from S0 and a zero history gives what prism_scan_fwd
+ * gives for the whole sequence; decoding after prism_scan_fwd continues that sequence
+ * when S = its S_final and conv_state = its last W-1 values of v.
+ *
+ * Inputs (device pointers, contiguous, 16-byte aligned):
+ *   q, k        [B,H,d_k]      dtype
+ *   v           [B,H,d_v]      dtype
+ *   gamma, beta [B,H]          fp32
+ *   u           [B,H,L-1,d_k]  dtype   (NULL iff L == 1)
+ *   alpha       [B,H,L-1]      fp32    (NULL iff L == 1)
+ *   gain        [B,H,L-1,d_v]  dtype   (NULL iff L == 1)
+ *   conv_w      [H,d_v,W]      fp32
+ * In/out, updated in place:
+ *   conv_state  [B,H,W-1,d_v]  dtype   v_{t-W+1}, ..., v_{t-1}, oldest first (zeros at the
+ *                                      start of a sequence); becomes v_{t-W+2}, ..., v_t.
+ *                                      NULL iff W == 1.
+ *   S           [B,H,d_v,d_k]  fp32    the state before the token; becomes the state after it.
+ * Output:
+ *   o           [B,H,d_v]      dtype
+ * d_k, d_v in {16, 32, 64, 128} (independently); 1 <= L <= PRISM_MAX_L; 1 <= W <= PRISM_MAX_W;
+ * chain is PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU.  Enqueued on `stream`; allocates nothing;
+ * no synchronisation.  Errors as for prism_scan_fwd, returned before any launch.
+ */
+int prism_decode_step(const void* q, const void* k, const void* v,
+                      const float* gamma, const float* beta,
+                      const void* u, const float* alpha, const void* gain,
+                      const float* conv_w, void* conv_state, float* S,
+                      int B, int H, int d_k, int d_v, int L, int W, int dtype, int chain,
+                      void* o, prism_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the
  * synchronisation itself failed. */

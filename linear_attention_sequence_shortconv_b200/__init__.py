@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     PRISM_CHAIN_LINEAR,
     PrismError,
     lib,
+    decode_step,
     prologue_fwd,
     scan_fwd,
     scan_fwd_host,

@@ -37,6 +37,7 @@ EXPORTS = (
     "prism_scan_fwd_host",
     "prism_prologue_fwd",
     "prism_prologue_fwd_ex",
+    "prism_decode_step",
     "prism_scan_fwd_uses_tensor_cores",
     "prism_stream_status",
     "prism_set_spin_limit",
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.prism_prologue_fwd.restype = ci
     L.prism_prologue_fwd_ex.argtypes = L.prism_prologue_fwd.argtypes + [ci]
     L.prism_prologue_fwd_ex.restype = ci
+    L.prism_decode_step.argtypes = [vp] * 11 + [ci] * 8 + [vp, vp]
+    L.prism_decode_step.restype = ci
     L.prism_scan_fwd_uses_tensor_cores.argtypes = [ci] * 6
     L.prism_scan_fwd_uses_tensor_cores.restype = ci
     L.prism_stream_status.argtypes = [vp]
@@ -230,6 +233,42 @@ def prologue_fwd(v, alpha, gain, conv_w, L: int, lengths=None, stream=None, chai
     if rc != 0:
         raise PrismError(rc, "prism_prologue_fwd_ex")
     return rho
+
+
+def decode_step(q, k, v, gamma, beta, u, alpha, gain, conv_w, conv_state, S, L: int, o=None,
+                stream=None, chain: str = "linear"):
+    """One recurrent step for every (b, h) on CUDA tensors; returns o [B,H,d_v].
+
+    q, k [B,H,d_k]; v [B,H,d_v]; gamma, beta [B,H] fp32; u [B,H,L-1,d_k]; alpha
+    [B,H,L-1] fp32; gain [B,H,L-1,d_v]; conv_w [H,d_v,W] fp32.  ``conv_state``
+    [B,H,W-1,d_v] (v's dtype; None when W = 1) and ``S`` [B,H,d_v,d_k] fp32 are
+    updated in place.
+    """
+    chain_code = _chain_code(chain)
+    dt = q.dtype
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, dt)
+    for name, t in (("gamma", gamma), ("beta", beta), ("conv_w", conv_w), ("S", S)):
+        _check(t, name, torch.float32)
+    if L > 1:
+        _check(u, "u", dt)
+        _check(gain, "gain", dt)
+        _check(alpha, "alpha", torch.float32)
+    W = conv_w.shape[-1]
+    _check(conv_state, "conv_state", dt, required=W > 1)
+    B, H, d_k = q.shape
+    d_v = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, d_v), dtype=dt, device=q.device)
+    rc = lib().prism_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+        _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
+        _ptr(conv_w), _ptr(conv_state if W > 1 else None), _ptr(S),
+        B, H, d_k, d_v, L, W, code, chain_code, _ptr(o), _stream_handle(stream))
+    if rc != 0:
+        raise PrismError(rc, "prism_decode_step")
+    return o
 
 
 def uses_tensor_cores(d_k, d_v, L, W, chunk, dtype_code) -> bool:

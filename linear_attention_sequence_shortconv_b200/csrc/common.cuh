@@ -30,6 +30,23 @@ struct ScanParams {
   int chain;              // PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU
 };
 
+// Pointers and sizes of one prism_decode_step call (device pointers).
+struct DecodeParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* gamma;
+  const float* beta;
+  const void* u;
+  const float* alpha;
+  const void* gain;
+  const float* conv_w;
+  void* conv_state;
+  float* S;
+  void* o;
+  int B, H, d_k, d_v, L, W, chain;
+};
+
 // One step of the residual chain.  Exact form (gist.science PRISM explainer, 2.2
 // Input-Anchored Loop Unrolling, Residual Update): r <- r - GELU(p * r), GELU in its
 // erf form.  Linearised form (ICML 2026 PRISM write-up, 消除 Step 间串行: the GELU is

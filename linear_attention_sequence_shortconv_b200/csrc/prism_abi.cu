@@ -12,6 +12,7 @@ cudaError_t launch_prologue(const void* v, const float* alpha, const void* gain,
                             int dtype, float* rho, cudaStream_t stream, int chain);
 bool chunk_tc_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
 cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream);
+cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t stream);
 }  // namespace prism
 
 namespace {
@@ -222,6 +223,28 @@ int prism_stream_status(prism_stream_t stream) {
   if (value != PRISM_OK && cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return PRISM_ERR_CUDA;
   return value;
+}
+
+int prism_decode_step(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
+                      const void* u, const float* alpha, const void* gain, const float* conv_w,
+                      void* conv_state, float* S, int B, int H, int d_k, int d_v, int L, int W, int dtype,
+                      int chain, void* o, prism_stream_t stream) {
+  if (chain != PRISM_CHAIN_LINEAR && chain != PRISM_CHAIN_GELU) return PRISM_ERR_INVALID_ARG;
+  int rc = check_sizes(B, 1, H, d_k, d_v, L, W, 16, dtype);
+  if (rc != PRISM_OK) return rc;
+  if (!q || !k || !v || !gamma || !beta || !conv_w || !S || !o) return PRISM_ERR_INVALID_ARG;
+  if (L > 1 && (!u || !alpha || !gain)) return PRISM_ERR_INVALID_ARG;
+  if (W > 1 && !conv_state) return PRISM_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, gamma, beta, u, alpha, gain, conv_w, conv_state, S, o};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return PRISM_ERR_UNSUPPORTED;
+  int* status = nullptr;
+  rc = device_setup(&status);
+  if (rc != PRISM_OK) return rc;
+  prism::DecodeParams p{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr,
+                        conv_w, W > 1 ? conv_state : nullptr, S, o, B, H, d_k, d_v, L, W, chain};
+  cudaError_t err = prism::launch_decode_step(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
 }  // extern "C"

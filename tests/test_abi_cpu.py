@@ -104,3 +104,28 @@ def test_unknown_residual_chain_is_rejected(L):
         assert L.prism_prologue_fwd_ex(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 64, 4, 4, 0, FAKE, None, chain) == 1
     with pytest.raises(ValueError):
         prism._lib._chain_code("tanh")
+
+
+def decode_call(lib_, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, gamma=FAKE, beta=FAKE, u=FAKE, alpha=FAKE, gain=FAKE, conv_w=FAKE,
+             conv_state=FAKE, S=FAKE, B=2, H=2, d_k=64, d_v=64, L=4, W=4, dtype=0, chain=0, o=FAKE)
+    a.update(kw)
+    return lib_.prism_decode_step(a["q"], a["k"], a["v"], a["gamma"], a["beta"], a["u"], a["alpha"], a["gain"],
+                                  a["conv_w"], a["conv_state"], a["S"], a["B"], a["H"], a["d_k"], a["d_v"],
+                                  a["L"], a["W"], a["dtype"], a["chain"], a["o"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), 1), (dict(H=0), 1), (dict(L=0), 1), (dict(W=0), 1), (dict(dtype=3), 1), (dict(chain=2), 1),
+    (dict(S=None), 1), (dict(o=None), 1), (dict(conv_state=None), 1), (dict(u=None), 1), (dict(gain=None), 1),
+    (dict(d_k=48), 2), (dict(d_v=256), 2), (dict(L=17), 2), (dict(W=9), 2), (dict(S=FAKE + 4), 2),
+    (dict(conv_state=FAKE + 2), 2),
+])
+def test_decode_invalid_arguments(L, kw, code):
+    assert decode_call(L, **kw) == code
+
+
+def test_decode_optional_inputs(L):
+    # W = 1 needs no history and L = 1 no residual inputs: with those NULL the only
+    # error left is the size error planted here.
+    assert decode_call(L, W=1, conv_state=None, L=1, u=None, alpha=None, gain=None, B=0) == 1
