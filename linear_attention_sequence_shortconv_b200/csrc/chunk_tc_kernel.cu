@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_mma = bar_load + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_load + 2);
   int* s_abort = reinterpret_cast<int*>(bar_load + 3);
+  uint64_t* bar_drain = bar_load + 4;  // one commit on the abort path: every MMA issued has completed
   float* sA = reinterpret_cast<float*>(sSXA);  // [64][LDA] fp32: A, then T in place
   float* sY = sA + 64 * LDA;                   // inverse scratch (<= 32x32 fp32)
   uint8_t* sX = sSXA;                          // X^T      bf16 [128][64] K-major
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(bar_load, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_drain, 1);
     fence_mbar_init();
     *s_abort = 0;
     tma_prefetch_desc(&map_q);
@@ -391,7 +393,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           s[4 * e] = f.x; s[4 * e + 1] = f.y; s[4 * e + 2] = f.z; s[4 * e + 3] = f.w;
         }
       }
-      tmem_st16(tl + RS + j0, s);
       st_bf16x8(sSXA, sw128_offset(row, j0, kAtom), s);
       st_bf16x8(sSXA, sw128_offset(row, j0 + 8, kAtom), s + 8);
     }
@@ -408,6 +409,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (M > 0 && tap_thread) taps0[(tid % p.W) * D + tid / p.W] = __ldg(cw_head + tid);
   __syncthreads();
+  if (srow) {  // RS <- exp(G_63 of chunk 0) S0 (undecayed S0 when there is no chunk: S_final)
+    const float b0 = nchunks > 0 ? __expf(sG[63]) : 1.f;
+#pragma unroll
+    for (int pc = 0; pc < SP; ++pc) {
+      const int j0 = cq * (D / 4) + 16 * pc;
+      float s[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) s[e] = 0.f;
+      if (p.S0) {
+        const float4* src = reinterpret_cast<const float4*>(p.S0 + (((size_t)b * H + h) * D + row) * D + j0);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float4 f = __ldg(src + e);
+          s[4 * e] = b0 * f.x; s[4 * e + 1] = b0 * f.y; s[4 * e + 2] = b0 * f.z; s[4 * e + 3] = b0 * f.w;
+        }
+      }
+      tmem_st16(tl + RS + j0, s);
+    }
+  }
   if (nchunks > 0) prologue(0, 0, taps0);
   fence_proxy_async_smem();
   tc_fence_before();
@@ -433,11 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16(tmem + R1, a, a, idesc_bf16(128, 64, 0, 0), kk > 0);
           if (M > 0) mma_bf16(tmem + R1 + 64, a, kdesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, UR, 0, 0), kk > 0);
         }
+        mma_commit(bar_mma);  // step B waits for MMA1 only
+        mma_inflight = (int)ph_mma;
+        // MMA3 (read in step E) is covered by the next commit, after MMA2 and QK*T
 #pragma unroll
         for (int kk = 0; kk < 4 * NA; ++kk)
           mma_bf16(tmem + D3, kdesc(aS, kk, kAtom), kdesc(aKQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
-        mma_commit(bar_mma);
-        mma_inflight = (int)ph_mma;
       } else {
         *s_abort = 1;
       }
@@ -570,21 +591,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         vraw16[e] = p.v[(((size_t)b * T + t) * H + h) * D + rr];
       }
     }
-    if (srow) {  // RS <- exp(G_63) RS, ahead of MMA5a / MMA5b accumulating into it
-      const float blast = sEp[63];
-      uint32_t rr[SP][16];
-#pragma unroll
-      for (int pc = 0; pc < SP; ++pc) tmem_ld16_async(tl + RS + cq * (D / 4) + 16 * pc, rr[pc]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int pc = 0; pc < SP; ++pc) {
-        float s[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) s[e] = __uint_as_float(rr[pc][e]) * blast;
-        tmem_st16_async(tl + RS + cq * (D / 4) + 16 * pc, s);
-      }
-      tmem_wait_st();
-    }
     // ---------------- C1: inverse
     {
       // (1) diagonal 16x16 blocks: thread (blk, j) solves column j by forward substitution;
@@ -601,7 +607,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           xcol[r] = (r < j) ? 0.f : (r == j ? 1.f : -acc);
         }
       }
-      tc_fence_before();  // the RS rescale above is ordered before MMA5a below
       __syncthreads();
       if (tid == 0 && fast && M > 0) {
         // Fast path: MMA5a (RS += P~^T U) needs only P~ (= P), U and the rescaled RS, so it runs
@@ -834,7 +839,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (ok && srow) {
+      // RS <- exp(G_63 of chunk n+1) S_{n+1}, the decayed state MMA5a / MMA5b of chunk n+1
+      // accumulate onto; the bf16 copy (A operand of MMA3) and S_final stay undecayed
       const bool last = n + 1 == nchunks;
+      const float bnext = last ? 1.f : __expf(sG[(cur ^ 1) * 64 + 63]);
 #pragma unroll
       for (int pc = 0; pc < SP; ++pc) {
         const int j0 = cq * (D / 4) + 16 * pc;
@@ -842,12 +850,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(tl + RS + j0, s);
         st_bf16x8(sSXA, sw128_offset(row, j0, kAtom), s);
         st_bf16x8(sSXA, sw128_offset(row, j0 + 8, kAtom), s + 8);
-        if (last && p.S_final) {
-          float4* dst = reinterpret_cast<float4*>(p.S_final + (((size_t)b * H + h) * D + row) * D + j0);
+        if (last) {
+          if (p.S_final) {
+            float4* dst = reinterpret_cast<float4*>(p.S_final + (((size_t)b * H + h) * D + row) * D + j0);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_float4(s[4 * e], s[4 * e + 1], s[4 * e + 2], s[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) dst[e] = make_float4(s[4 * e], s[4 * e + 1], s[4 * e + 2], s[4 * e + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) s[e] *= bnext;
+          tmem_st16_async(tl + RS + j0, s);
         }
       }
+      tmem_wait_st();
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -882,6 +897,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (load_inflight >= 0) mbar_wait(bar_load, (uint32_t)load_inflight, kDrainLimit, p.status);
     if (mma_inflight >= 0) mbar_wait(bar_mma, (uint32_t)mma_inflight, kDrainLimit, p.status);
+    mma_commit(bar_drain);  // also covers MMAs issued after the last commit observed
+    mbar_wait(bar_drain, 0u, kDrainLimit, p.status);
   }
   if (tid == 0) bulk_wait_all();
   tc_fence_before();
