@@ -109,7 +109,12 @@ enum prism_status {
  *   L - 1 <= 3; every other supported shape runs the fp32 CUDA-core path, which
  *   evaluates the recurrence token by token.
  * workspace / workspace_bytes: device scratch of at least
- *   prism_scan_fwd_workspace_size(...) bytes (may be NULL when that is 0).
+ *   prism_scan_fwd_workspace_size(...) bytes (may be NULL when that is 0), 16-byte
+ *   aligned, owned by the caller, contents undefined on return.  The tensor-core
+ *   path keeps there the inverse T = (I + A)^{-1} of every 64-token chunk as bf16
+ *   (B * H * ceil(T / 64) * 8 KB), computed for all chunks at once before the scan;
+ *   the token-by-token path needs none.  Too small or NULL: PRISM_ERR_WORKSPACE,
+ *   before any launch.
  * Errors: PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED, PRISM_ERR_WORKSPACE,
  *   PRISM_ERR_CUDA, as described above.
  */

@@ -197,8 +197,9 @@ def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 
 
 def scan_fwd_host(host: dict, dev: dict, L: int, chunk: int = 64, stream=None):
     """The host-buffer entry point: ``host`` holds pinned CPU tensors (inputs and
-    the outputs ``o``/``S_final``), ``dev`` CUDA tensors of the same shapes.
-    Enqueues H2D copies, the scan and D2H copies on ``stream``; does not sync."""
+    the outputs ``o``/``S_final``), ``dev`` CUDA tensors of the same shapes (and
+    optionally ``workspace``, allocated here when missing).  Enqueues H2D copies,
+    the scan and D2H copies on ``stream``; does not sync."""
     names = ("q", "k", "v", "gamma", "beta", "u", "alpha", "gain", "conv_w", "S0", "lengths")
     q = host["q"]
     B, T, H, d_k = q.shape
@@ -207,6 +208,8 @@ def scan_fwd_host(host: dict, dev: dict, L: int, chunk: int = 64, stream=None):
     code = _dtype_code(q)
     ws_bytes = workspace_size(B, T, H, d_k, d_v, L, W, chunk, code)
     ws = dev.get("workspace")
+    if ws_bytes and ws is None:
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev["o"].device)
     rc = lib().prism_scan_fwd_host(
         *[_ptr(host.get(n)) for n in names], *[_ptr(dev.get(n) if host.get(n) is not None else None) for n in names],
         B, T, H, d_k, d_v, L, W, chunk, code,

@@ -4,7 +4,7 @@
 // in order, with the state S (d_v x d_k, fp32) resident in tensor memory.  Every
 // input element is read from HBM once and o is written once; the ShortConv
 // prologue (anchor, residual chain, residual-write vectors rho) runs inside the
-// same kernel.  Sources: ICML 2026 PRISM write-up (核心迭代形式, 消除 Token 间串行,
+// scan kernel.  Sources: ICML 2026 PRISM write-up (核心迭代形式, 消除 Token 间串行,
 // 消除 Step 间串行, 架构形式) and the PRISM technical summary (2.1, 2.2), which fix
 // the recurrence; its chunkwise form below is derived from that recurrence.
 //
@@ -20,15 +20,21 @@
 //   O   = diag(e^G) Q S_n^T + QU P + (QK T) X
 //   S_{n+1} = e^{G_63} S_n + Delta^T diag(c) K + P^T diag(c) U
 //
-// Tensor-core products (bf16 operands, fp32 accumulators in TMEM, M = 128):
-//   MMA1  [K;Q] x [K;U]^T          -> R1   (token rows; N = 64 + 64m)
+// Two launches per call.  The preparation kernel (one CTA per (b, h, chunk), all chunks
+// at once) computes T = (I + A)^{-1} of every chunk: A from K K^T on the tensor cores,
+// the inverse by blocked forward substitution in fp32 on CUDA cores, stored as bf16 in
+// the workspace.  The scan kernel then walks the chunks of each chain in order and
+// TMA-loads each chunk's T next to its K, Q and U tiles.
+//
+// Tensor-core products of the scan kernel (bf16 operands, fp32 accumulators in TMEM,
+// M = 128):
+//   MMA1  [K;Q] x [K;U]^T          -> R1   (token rows; N = 64 + 64m; only QK, Bku, QU used)
 //   MMA3  S_n  x [K;Q]^T           -> D3   (state rows c; N = 128)
 //   MMAQT [T;QK] x T               -> R1+128 (rows 64..127 = QK T)
 //   MMA2  P^T x [Bku;QU]^T         -> R1   ((Bku P)^T | (QU P)^T)
 //   MMA4  X^T x [T;QKT]^T          -> R1+128 (Delta^T | (QKT X)^T)
 //   MMA5  (diag(c)P)^T U + (diag(c)Delta)^T K  accumulated onto e^{G_63} S_n in RS
-// CUDA cores do the ShortConv prologue, the decay/mask epilogues and the 64x64
-// unit-lower-triangular inverse T (blocked forward substitution in fp32).
+// CUDA cores do the ShortConv prologue of the next chunk and the decay/mask epilogues.
 //
 // Smem operands use the 128-byte swizzle; K, Q and U arrive by TMA (zero fill past
 // T), everything else is written by the CTA's threads.  Every mbarrier wait is
@@ -65,16 +71,14 @@ struct Layout {
   static constexpr uint32_t OFF_BQ = OFF_P + SZ_P;
   static constexpr uint32_t SZ_BQ = M * kAtom;  // [Bku;QU] (128 x 64m), later P~ (64m x D)
   static constexpr uint32_t OFF_TQ = OFF_BQ + SZ_BQ;
-  static constexpr uint32_t OFF_SXA = OFF_TQ + kAtom;  // S bf16 | A,T fp32 | X^T, Delta~^T
+  static constexpr uint32_t OFF_SXA = OFF_TQ + kAtom;  // S bf16 | X^T, Delta~^T
   static constexpr uint32_t OFF_SMALL = OFF_SXA + 2 * kAtom;  // gate tables, barriers
   static constexpr uint32_t BYTES = OFF_SMALL + 2048;
   // + alignment slack; never below 116 KB so that one CTA (and one 512-column TMEM
   // allocation) is resident per SM
   static constexpr uint32_t SMEM_ALLOC = (BYTES + 1024 > 116u * 1024u) ? BYTES + 1024 : 116u * 1024u;
   static_assert(SMEM_ALLOC <= 232448, "exceeds the 227 KB opt-in shared memory of sm_100");
-  static constexpr int LDA = 68;  // fp32 row stride of A / T in the SXA region
   static_assert(SZ_BQ >= SZ_P, "P~ must fit where [Bku;QU] was");
-  static_assert(64 * LDA * 4 + 1024 * 4 <= 2 * kAtom, "A/T + inverse scratch must fit in SXA");
 };
 
 struct TcArgs {
@@ -91,7 +95,7 @@ struct TcArgs {
   const int32_t* lengths;
   __nv_bfloat16* o;
   float* S_final;
-  int B, T, H, W;
+  int B, T, H, W, NC;
   int* status;
   long long spin_limit;
 };
@@ -133,6 +137,276 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t base, int kk, uint32_t lbo) 
   return sdesc_sw128(base + (uint32_t)kk * 2048u, lbo, 1024);
 }
 
+// T = (I + A)^{-1} in place, for a strictly lower-triangular 64 x 64 fp32 A in sA (row
+// stride LDA, zeros on and above the diagonal), by blocked forward substitution: the four
+// 16 x 16 diagonal blocks column by column, then the 16 -> 32 and 32 -> 64 merges
+// T_21 = -T_22 A_21 T_11.  All kPrepThreads (128) threads call it (it synchronises
+// internally); on return sA holds T (unit lower triangular, zeros above).  sY: 1024 fp32.
+constexpr int kPrepThreads = 128;
+
+template <int LDA>
+__device__ __forceinline__ void invert_unit_lower64(float* sA, float* sY, int tid) {
+  // (1) diagonal blocks: thread (blk, j) solves column j of block blk
+  {
+    float xcol[16];
+    const int blk = tid >> 4, j = tid & 15;
+    if (tid < 64) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        float acc = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < r; ++s2) acc += sA[(16 * blk + r) * LDA + 16 * blk + s2] * xcol[s2];
+        xcol[r] = (r < j) ? 0.f : (r == j ? 1.f : -acc);
+      }
+    }
+    __syncthreads();
+    if (tid < 64) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) sA[(16 * blk + r) * LDA + 16 * blk + j] = xcol[r];
+    }
+    __syncthreads();
+  }
+  // (2) 16 -> 32: T_{I,I-1} = -T_II (A_{I,I-1} T_{I-1,I-1}) for I = 1, 3.  Thread: one row r
+  // of one of the two blocks, four consecutive columns.
+  {
+    const int pr = tid >> 6, r = (tid >> 2) & 15, c0 = (tid & 3) * 4;
+    const int I = 2 * pr + 1, J = 2 * pr;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const float a = sA[(16 * I + r) * LDA + 16 * J + u];
+      const float4 t = *reinterpret_cast<const float4*>(sA + (16 * J + u) * LDA + 16 * J + c0);
+      acc[0] += a * t.x;
+      acc[1] += a * t.y;
+      acc[2] += a * t.z;
+      acc[3] += a * t.w;
+    }
+    *reinterpret_cast<float4*>(sY + pr * 256 + r * 16 + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      if (u <= r) {
+        const float a = sA[(16 * I + r) * LDA + 16 * I + u];
+        const float4 y = *reinterpret_cast<const float4*>(sY + pr * 256 + u * 16 + c0);
+        acc[0] += a * y.x;
+        acc[1] += a * y.y;
+        acc[2] += a * y.z;
+        acc[3] += a * y.w;
+      }
+    }
+    *reinterpret_cast<float4*>(sA + (16 * I + r) * LDA + 16 * J + c0) =
+        make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+    __syncthreads();
+  }
+  // (3) 32 -> 64: T[32:64, 0:32] = -T2 (A21 T1).  Thread: two rows, four consecutive columns.
+  {
+    const int r0 = (tid >> 3) * 2, c0 = (tid & 7) * 4;
+    float acc[2][4] = {};
+#pragma unroll 8
+    for (int u = 0; u < 32; ++u) {  // Y2 = A21 T1
+      const float4 t = *reinterpret_cast<const float4*>(sA + u * LDA + c0);
+#pragma unroll
+      for (int i2 = 0; i2 < 2; ++i2) {
+        const float a = sA[(32 + r0 + i2) * LDA + u];
+        acc[i2][0] += a * t.x;
+        acc[i2][1] += a * t.y;
+        acc[i2][2] += a * t.z;
+        acc[i2][3] += a * t.w;
+      }
+    }
+#pragma unroll
+    for (int i2 = 0; i2 < 2; ++i2)
+      *reinterpret_cast<float4*>(sY + (r0 + i2) * 32 + c0) = make_float4(acc[i2][0], acc[i2][1], acc[i2][2], acc[i2][3]);
+    __syncthreads();
+#pragma unroll
+    for (int i2 = 0; i2 < 2; ++i2) acc[i2][0] = acc[i2][1] = acc[i2][2] = acc[i2][3] = 0.f;
+    const int ulim = r0 + 2;  // T2 is lower triangular: only u <= r0 + 1 contribute
+#pragma unroll 8
+    for (int u = 0; u < ulim; ++u) {  // T21 = -T2 Y2
+      const float4 y = *reinterpret_cast<const float4*>(sY + u * 32 + c0);
+#pragma unroll
+      for (int i2 = 0; i2 < 2; ++i2) {
+        const float a = sA[(32 + r0 + i2) * LDA + 32 + u];
+        acc[i2][0] += a * y.x;
+        acc[i2][1] += a * y.y;
+        acc[i2][2] += a * y.z;
+        acc[i2][3] += a * y.w;
+      }
+    }
+    // rows 32..63, columns 0..31 held A21, which the first product has consumed
+#pragma unroll
+    for (int i2 = 0; i2 < 2; ++i2)
+      *reinterpret_cast<float4*>(sA + (32 + r0 + i2) * LDA + c0) =
+          make_float4(-acc[i2][0], -acc[i2][1], -acc[i2][2], -acc[i2][3]);
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- chunk preparation
+// The part of every chunk that depends on neither the state nor the other chunks, done
+// for all (b, h, chunk) at once before the scan: the in-chunk gate prefix G, the masked
+// decayed Gram matrix A[t,i] = beta_t e^{G_t - G_i} k_t.k_i (i < t; K K^T on the tensor
+// cores) and T = (I + A)^{-1}, stored as bf16 [B, H, NC, 64, 64] in the workspace.
+// Taking the inverse off the scan's sequential chunk loop spreads it over every SM.
+struct PrepArgs {
+  const float* gamma;
+  const float* beta;
+  const int32_t* lengths;
+  __nv_bfloat16* Tws;
+  int T, H, NC;
+  int* status;
+  long long spin_limit;
+};
+
+constexpr int kPrepLDA = 68;  // fp32 row stride of A / T (bank-conflict padding)
+
+constexpr uint32_t kPrepAtom = 8192;  // 64 rows x 128 bytes: one swizzle-atom column of K
+
+template <int D>
+struct PrepLayout {
+  static constexpr int NA = D / 64;
+  // K tile: NA atom columns of 64 rows, 8 KB apart.  The M = 128 MMA also reads the 64
+  // rows that follow each one (the next atom column, or A below): those accumulator
+  // lanes are never read.
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_A = NA * kPrepAtom;             // [64][kPrepLDA] fp32
+  static constexpr uint32_t OFF_Y = OFF_A + 64 * kPrepLDA * 4;  // 1024 fp32 inverse scratch
+  static constexpr uint32_t OFF_SMALL = OFF_Y + 4096;           // G, beta [64] each; barriers
+  static constexpr uint32_t BYTES = OFF_SMALL + 1024;
+  static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;  // + alignment slack
+};
+
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads) prism_chunk_prep_kernel(const __grid_constant__ CUtensorMap map_k,
+                                                                       PrepArgs p) {
+  using Ly = PrepLayout<D>;
+  constexpr int NA = Ly::NA, LDA = kPrepLDA;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = sm + Ly::OFF_K;
+  float* sA = reinterpret_cast<float*>(sm + Ly::OFF_A);
+  float* sY = reinterpret_cast<float*>(sm + Ly::OFF_Y);
+  float* sG = reinterpret_cast<float*>(sm + Ly::OFF_SMALL);
+  float* sBeta = sG + 64;
+  uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + Ly::OFF_SMALL + 512);
+  uint64_t* bar_mma = bar_load + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_load + 2);
+  int* s_abort = reinterpret_cast<int*>(bar_load + 3);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % p.NC, bh = blockIdx.x / p.NC, b = bh / p.H, h = bh % p.H;
+  const int len = p.lengths ? min(max(p.lengths[b], 0), p.T) : p.T;
+  const int t0 = n * kC;
+  if (t0 >= len) return;  // the scan never reaches this chunk (uniform over the CTA)
+  const int nv = min(kC, len - t0);
+  const long long lim = p.spin_limit;
+
+  if (tid == 0) {  // the K tile is requested first: its latency overlaps the gate loads below
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    *s_abort = 0;
+    mbar_arrive_expect_tx(bar_load, NA * 8192);
+#pragma unroll
+    for (int a = 0; a < NA; ++a) tma_load_4d(sK + a * kPrepAtom, &map_k, bar_load, 64 * a, h, t0, b);
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, 64);
+    tmem_relinquish();
+  }
+  if (warp == 2) {  // gate prefix; lane owns tokens 2 lane, 2 lane + 1; padded steps: gamma = 1, beta = 0
+    float gl[2], bl[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int t = 2 * lane + e;
+      const bool valid = t < nv;
+      const size_t th = ((size_t)b * p.T + min(t0 + t, p.T - 1)) * p.H + h;
+      gl[e] = valid ? __ldg(p.gamma + th) : 1.f;
+      bl[e] = valid ? __ldg(p.beta + th) : 0.f;
+    }
+    const float lg0 = __logf(gl[0]), lg1 = __logf(gl[1]);
+    float x = lg0 + lg1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    sG[2 * lane] = x - lg1;
+    sG[2 * lane + 1] = x;
+    sBeta[2 * lane] = bl[0];
+    sBeta[2 * lane + 1] = bl[1];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  bool mma_issued = false;
+  if (tid == 0) {
+    if (mbar_wait(bar_load, 0, lim, p.status)) {
+      tc_fence_after();
+      // K K^T with M = 128 (accumulator lanes 64..127 are not read)
+      const uint32_t aK = smem_u32(sK);
+#pragma unroll
+      for (int kk = 0; kk < 4 * NA; ++kk)
+        mma_bf16(tmem, kdesc(aK, kk, kPrepAtom), kdesc(aK, kk, kPrepAtom), idesc_bf16(128, 64, 0, 0), kk > 0);
+      mma_commit(bar_mma);
+      mma_issued = true;
+    } else {
+      *s_abort = 1;
+    }
+  }
+  __syncthreads();
+  if (*s_abort == 0 && warp < 2) {  // TMEM lanes 0..63 = token rows t
+    const bool ok = warp_wait(bar_mma, 0, lim, p.status);
+    if (ok) {
+      tc_fence_after();
+      const int t = 32 * warp + lane;
+      const float Gt = sG[t], bt = sBeta[t];
+      const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        float x[16];
+        tmem_ld16(tl + 16 * pc, x);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i = 16 * pc + e;
+          x[e] = (i < t) ? bt * __expf(Gt - sG[i]) * x[e] : 0.f;
+        }
+        float4* dst = reinterpret_cast<float4*>(sA + t * LDA + 16 * pc);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+      }
+    } else if (lane == 0) {
+      atomicExch(s_abort, 1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*s_abort == 0) {
+    invert_unit_lower64<LDA>(sA, sY, tid);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // T -> bf16 rows of 128 bytes, 16 bytes per thread and pass
+      const int e = q * kPrepThreads + tid, t = e >> 3, c8 = (e & 7) * 8;
+      const float4 lo = *reinterpret_cast<const float4*>(sA + t * LDA + c8);
+      const float4 hi = *reinterpret_cast<const float4*>(sA + t * LDA + c8 + 4);
+      uint4 u;
+      u.x = pack_bf16x2(lo.x, lo.y);
+      u.y = pack_bf16x2(lo.z, lo.w);
+      u.z = pack_bf16x2(hi.x, hi.y);
+      u.w = pack_bf16x2(hi.z, hi.w);
+      *reinterpret_cast<uint4*>(p.Tws + (((size_t)bh * p.NC + n) * 64 + t) * 64 + c8) = u;
+    }
+  } else if (tid == 0) {  // drain this CTA's own copy and MMA before its memory is reused
+    mbar_wait(bar_load, 0, kDrainLimit, p.status);
+    if (mma_issued) mbar_wait(bar_mma, 0, kDrainLimit, p.status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+// ---------------------------------------------------------------- the scan
 // CH: residual chain step (PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU), fixed at compile
 // time so the linear chain carries none of the GELU step's code or registers.
 template <int D, int M, int CH>
@@ -140,9 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prism_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                           const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_v,
                           const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_o,
-                          TcArgs p) {
+                          const __grid_constant__ CUtensorMap map_t, TcArgs p) {
   using Ly = Layout<D, M>;
-  constexpr int NA = Ly::NA, UR = Ly::UR, LDA = Ly::LDA;
+  constexpr int NA = Ly::NA, UR = Ly::UR;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKQ = sm + Ly::OFF_KQ;
@@ -161,8 +435,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_load + 2);
   int* s_abort = reinterpret_cast<int*>(bar_load + 3);
   uint64_t* bar_drain = bar_load + 4;  // one commit on the abort path: every MMA issued has completed
-  float* sA = reinterpret_cast<float*>(sSXA);  // [64][LDA] fp32: A, then T in place
-  float* sY = sA + 64 * LDA;                   // inverse scratch (<= 32x32 fp32)
   uint8_t* sX = sSXA;                          // X^T      bf16 [128][64] K-major
   uint8_t* sDl = sSXA + kAtom;                 // Delta~^T bf16 [128][64] K-major
 
@@ -185,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&map_q);
     tma_prefetch_desc(&map_k);
     tma_prefetch_desc(&map_v);
+    tma_prefetch_desc(&map_t);
     if (M > 0) {
       tma_prefetch_desc(&map_u);
       tma_prefetch_desc(&map_g);
@@ -234,9 +507,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int a = 0; a < NA; ++a) tma_load_4d(sKQ + a * kAtom, &map_k, bar_load, 64 * a, h, t0, b);
   };
+  // T = (I + A)^{-1} of chunk nn (from the preparation kernel) -> rows 0..63 of TQ
+  auto load_t = [&](int nn) {
+    load_open = true;
+    mbar_expect_tx(bar_load, 8192);
+    tma_load_4d(sTQ, &map_t, bar_load, 0, 0, nn, bh);
+  };
   auto issue_loads = [&](int t0) {
     load_q(t0);
     load_u(t0);
+    load_t(t0 / kC);
     load_k_arrive(t0);
   };
   // L2 prefetch of the next chunk's k, q, v (D bf16 per token) and u, gain (M*D bf16 per
@@ -441,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* G = sG + cur * 64;
     const float* Bt = sBeta + cur * 64;
 
-    // ---------------- A: wait for K,Q,U; MMA1 + MMA3; per-chunk decay tables; L2 prefetch of chunk n+1
+    // ---------------- A: wait for K,Q,U,T; MMA1 + MMA3; per-chunk decay tables; L2 prefetch of chunk n+1
     if (tid == 0) {
       const bool ok = mbar_wait(bar_load, ph_load, lim, p.status);
       if (ok) {
@@ -487,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*s_abort) { aborted = true; break; }
 
-    // ---------------- B: epilogue of MMA1 -> A (fp32), [Bku;QU], QK (bf16); then issue MMA2
+    // ---------------- B: epilogue of MMA1 -> [Bku;QU], QK (bf16); then MMA2, MMA5a (fast), QK*T
     bool ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) {
@@ -495,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n + 1 < nchunks) load_q(t0 + kC);  // MMA1 and MMA3 have read Q
     }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
-    float gl_next[4] = {1.f, 1.f, 0.f, 0.f};  // warp 2: next chunk's gates, scanned during C1
+    float gl_next[4] = {1.f, 1.f, 0.f, 0.f};  // warp 2: next chunk's gates, scanned in step C
     if (warp == 2 && n + 1 < nchunks) gate_load(n + 1, gl_next);
     tc_fence_after();
     if (ok) {
@@ -520,6 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pb + k >= PQ) break;
         const int pc = pb + k;
         const int j0 = 16 * (cq * PQ + pc);
+        if (krow && j0 < 64) continue;  // K K^T: only the preparation kernel needs it (for T)
         float x[16];
         if (j0 < 64) {  // K / Q columns: D[t,i] = e^{G_t - G_i}
           if (fast) {
@@ -549,15 +830,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               x[e] = (i0 + e < tlim) ? bk * __expf(Gt - G[i0 + e]) * __uint_as_float(raw[k][e]) : 0.f;
           }
         }
-        if (j0 < 64) {
-          if (krow) {
-            float4* dst = reinterpret_cast<float4*>(sA + t * LDA + j0);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
-          } else {
-            st_bf16x8(sTQ, sw128_offset(row, j0, kAtom), x);
-            st_bf16x8(sTQ, sw128_offset(row, j0 + 8, kAtom), x + 8);
-          }
+        if (j0 < 64) {  // QK (rows 64..127 of TQ)
+          st_bf16x8(sTQ, sw128_offset(row, j0, kAtom), x);
+          st_bf16x8(sTQ, sw128_offset(row, j0 + 8, kAtom), x + 8);
         } else {
           st_bf16x8(sBQ, sw128_offset(row, j0 - 64, kAtom), x);
           st_bf16x8(sBQ, sw128_offset(row, j0 - 56, kAtom), x + 8);
@@ -569,16 +844,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (*s_abort) { aborted = true; break; }
-    if (tid == 0 && M > 0) {
+    if (tid == 0) {
       tc_fence_after();
+      if (M > 0) {
 #pragma unroll
-      for (int kk = 0; kk < UR / 16; ++kk)
-        mma_bf16(tmem + R1, mndesc(aP, kk, Ly::U_ATOM), kdesc(aBQ, kk, kAtom), idesc_bf16(128, 128, 1, 0), kk > 0);
+        for (int kk = 0; kk < UR / 16; ++kk)  // MMA2: (Bku P)^T | (QU P)^T
+          mma_bf16(tmem + R1, mndesc(aP, kk, Ly::U_ATOM), kdesc(aBQ, kk, kAtom), idesc_bf16(128, 128, 1, 0),
+                   kk > 0);
+        if (fast) {
+          // MMA5a (RS += P~^T U) needs only P~ (= P), U and the decayed RS: issued now, it
+          // completes before step E's wait, ahead of the next prologue overwriting P
+#pragma unroll
+          for (int kk = 0; kk < UR / 16; ++kk)
+            mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1),
+                     1);
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)  // [T;QK] x T: rows 64..127 = QK T
+        mma_bf16(tmem + R1 + 128, kdesc(aTQ, kk, kAtom), mndesc(aTQ, kk, kAtom), idesc_bf16(128, 64, 0, 1), kk > 0);
+      mma_commit(bar_mma);
+      mma_inflight = (int)ph_mma;
     }
 
-    // ---------------- C: rescale RS by exp(G_63); T = (I + A)^{-1} in place (fp32); issue MMA QK*T
-    // the tap element this thread stages for the next prologue, and the values of v it needs for
-    // X, loaded here so their latency hides behind the inverse
+    // ---------------- C: the next chunk's gate prefix; the tap element this thread stages for
+    // the next prologue and the values of v it needs for X (their latency hides behind the MMAs)
+    if (warp == 2 && n + 1 < nchunks) gate_scan(gl_next, cur ^ 1);
     const float tap_reg = (M > 0 && tap_thread) ? __ldg(cw_head + tid) : 0.f;
     // (padded steps have beta = 0, so any in-range token may stand in for them)
     __nv_bfloat16 vraw16[16];  // converted where X is formed, so the loads are not waited on here
@@ -590,111 +881,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = min(t0 + tb + e, T - 1);
         vraw16[e] = p.v[(((size_t)b * T + t) * H + h) * D + rr];
       }
-    }
-    // ---------------- C1: inverse
-    {
-      // (1) diagonal 16x16 blocks: thread (blk, j) solves column j by forward substitution;
-      // meanwhile warp 2 computes the next chunk's gate prefix (its lines were prefetched in A)
-      if (warp == 2 && n + 1 < nchunks) gate_scan(gl_next, cur ^ 1);
-      float xcol[16];
-      const int blk = tid >> 4, j = tid & 15;
-      if (tid < 64) {
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          float acc = 0.f;
-#pragma unroll
-          for (int s2 = 0; s2 < r; ++s2) acc += sA[(16 * blk + r) * LDA + 16 * blk + s2] * xcol[s2];
-          xcol[r] = (r < j) ? 0.f : (r == j ? 1.f : -acc);
-        }
-      }
-      __syncthreads();
-      if (tid == 0 && fast && M > 0) {
-        // Fast path: MMA5a (RS += P~^T U) needs only P~ (= P), U and the rescaled RS, so it runs
-        // under the inverse; it completes before the next prologue overwrites P.
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < UR / 16; ++kk)
-          mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
-      }
-      if (tid < 64) {
-#pragma unroll
-        for (int r = 0; r < 16; ++r) sA[(16 * blk + r) * LDA + 16 * blk + j] = xcol[r];
-      }
-      __syncthreads();
-      // (2) 16 -> 32: T_{I,I-1} = -T_II A_{I,I-1} T_{I-1,I-1} for I = 1, 3
-      {
-        const int pr = tid >> 8, r = (tid >> 4) & 15, s2 = tid & 15;
-        const int I = 2 * pr + 1, J = 2 * pr;
-        float acc = 0.f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) acc += sA[(16 * I + r) * LDA + 16 * J + u] * sA[(16 * J + u) * LDA + 16 * J + s2];
-        sY[tid] = acc;
-        __syncthreads();
-        acc = 0.f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (u <= r) acc += sA[(16 * I + r) * LDA + 16 * I + u] * sY[(pr << 8) + (u << 4) + s2];
-        __syncthreads();
-        sA[(16 * I + r) * LDA + 16 * J + s2] = -acc;
-        __syncthreads();
-      }
-      // ---------------- C3: inverse 32 -> 64
-      // (3) 32 -> 64: T[32:64, 0:32] = -T2 (A21 T1).  Each thread: 2 rows x 1 column; the row
-      // operands are float4 broadcasts, the column operand a conflict-free scalar.
-      {
-        const int r0 = (tid >> 5) * 2, s2 = tid & 31;
-        float acc[2] = {0.f, 0.f};
-#pragma unroll 4
-        for (int u = 0; u < 32; u += 4) {  // Y2 = A21 T1
-          float tc[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) tc[k] = sA[(u + k) * LDA + s2];
-#pragma unroll
-          for (int i2 = 0; i2 < 2; ++i2) {
-            const float4 a = *reinterpret_cast<const float4*>(sA + (32 + r0 + i2) * LDA + u);
-            acc[i2] += a.x * tc[0] + a.y * tc[1] + a.z * tc[2] + a.w * tc[3];
-          }
-        }
-#pragma unroll
-        for (int i2 = 0; i2 < 2; ++i2) sY[(r0 + i2) * 32 + s2] = acc[i2];
-        __syncthreads();
-        acc[0] = acc[1] = 0.f;
-        const int ulim = r0 + 2;  // T2 is lower triangular: only u <= r0 + 1 contribute (warp-uniform)
-#pragma unroll 4
-        for (int u = 0; u < ulim; u += 4) {  // T21 = -T2 Y2
-          float yc[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) yc[k] = sY[(u + k) * 32 + s2];
-#pragma unroll
-          for (int i2 = 0; i2 < 2; ++i2) {
-            const float4 a = *reinterpret_cast<const float4*>(sA + (32 + r0 + i2) * LDA + 32 + u);
-            acc[i2] += a.x * yc[0] + a.y * yc[1] + a.z * yc[2] + a.w * yc[3];
-          }
-        }
-        // rows 32..63, columns 0..31 held A21, which step (3a) has consumed
-#pragma unroll
-        for (int i2 = 0; i2 < 2; ++i2) sA[(32 + r0 + i2) * LDA + s2] = -acc[i2];
-        __syncthreads();
-      }
-      // T (fp32, lower incl. unit diagonal; upper part holds A's zeros) -> bf16 rows 0..63 of TQ
-      {
-        const int t = tid >> 3, c8 = (tid & 7) * 8;
-        const float4 lo = *reinterpret_cast<const float4*>(sA + t * LDA + c8);
-        const float4 hi = *reinterpret_cast<const float4*>(sA + t * LDA + c8 + 4);
-        const float v8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        st_bf16x8(sTQ, sw128_offset(t, c8, kAtom), v8);
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + R1 + 128, kdesc(aTQ, kk, kAtom), mndesc(aTQ, kk, kAtom), idesc_bf16(128, 64, 0, 1), kk > 0);
-      mma_commit(bar_mma);
-      mma_inflight = (int)ph_mma;
     }
     // ---------------- E: QKT -> TQ rows 64..127; P~ = diag(c) P -> BQ; X^T -> SXA; O partial
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
@@ -788,6 +974,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0 && ok) {
       mma_inflight = -1;
       if (!fast && n + 1 < nchunks) load_u(t0 + kC);  // exact path: MMA5a has read U
+      if (n + 1 < nchunks) load_t(n + 1);              // MMA4, the last reader of TQ, has completed
     }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
@@ -934,6 +1121,26 @@ bool encode(CUtensorMap* map, const void* ptr, int rank, const cuuint64_t* dims,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int num_chunks(int T) { return (T + kC - 1) / kC; }
+
+// T tiles of every (b, h, chunk) into the workspace: one CTA per tile.
+template <int D>
+cudaError_t launch_prep(const ScanParams& p, const CUtensorMap& mk, cudaStream_t stream) {
+  using Ly = PrepLayout<D>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(prism_chunk_prep_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Ly::SMEM_ALLOC);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int NC = num_chunks(p.T);
+  PrepArgs a{p.gamma, p.beta, p.lengths, static_cast<__nv_bfloat16*>(p.workspace), p.T, p.H, NC, p.status,
+             p.spin_limit};
+  prism_chunk_prep_kernel<D><<<p.B * p.H * NC, kPrepThreads, Ly::SMEM_ALLOC, stream>>>(mk, a);
+  return cudaGetLastError();
+}
+
 template <int D, int M, int CH>
 cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
   using Ly = Layout<D, M>;
@@ -945,6 +1152,7 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
   });
   if (attr_err != cudaSuccess) return attr_err;
   const cuuint64_t B = p.B, T = p.T, H = p.H;
+  const int NC = num_chunks(p.T);
   CUtensorMap mq, mk, mu, mv, mg, mo;
   const cuuint64_t dims4[4] = {(cuuint64_t)D, H, T, B};
   const cuuint64_t str4[3] = {(cuuint64_t)D * 2, H * D * 2, T * H * D * 2};
@@ -962,11 +1170,18 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
     mu = mk;
     mg = mk;
   }
+  CUtensorMap mt;  // T tiles [B*H][NC][64][64] bf16 in the workspace
+  const cuuint64_t dimsT[4] = {64, 64, (cuuint64_t)NC, B * H};
+  const cuuint64_t strT[3] = {128, 8192, (cuuint64_t)NC * 8192};
+  const cuuint32_t boxT[4] = {64, 64, 1, 1};
+  if (!encode(&mt, p.workspace, 4, dimsT, strT, boxT)) return cudaErrorInvalidValue;
+  cudaError_t err = launch_prep<D>(p, mk, stream);
+  if (err != cudaSuccess) return err;
   TcArgs a{static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
            static_cast<const __nv_bfloat16*>(p.u), static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha,
            static_cast<const __nv_bfloat16*>(p.gain), p.conv_w, p.S0, p.lengths,
-           static_cast<__nv_bfloat16*>(p.o), p.S_final, p.B, p.T, p.H, p.W, p.status, p.spin_limit};
-  prism_chunk_tc_kernel<D, M, CH><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, mo, a);
+           static_cast<__nv_bfloat16*>(p.o), p.S_final, p.B, p.T, p.H, p.W, NC, p.status, p.spin_limit};
+  prism_chunk_tc_kernel<D, M, CH><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, mo, mt, a);
   return cudaGetLastError();
 }
 
@@ -993,6 +1208,8 @@ bool chunk_tc_supported(int d_k, int d_v, int L, int W, int chunk, int dtype) {
   return dtype == PRISM_BF16 && chunk == kC && d_k == d_v && (d_k == 64 || d_k == 128) && L >= 1 && L <= 4 &&
          W >= 1 && W <= 4;
 }
+
+size_t chunk_tc_workspace_bytes(int B, int T, int H) { return (size_t)B * H * num_chunks(T) * 8192; }
 
 cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream) {
   if (p.d_k == 128) return launch_d<128>(p, stream);

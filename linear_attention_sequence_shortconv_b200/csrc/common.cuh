@@ -28,6 +28,7 @@ struct ScanParams {
   int* status;            // per-device status word (PRISM_OK / PRISM_ERR_TIMEOUT)
   long long spin_limit;   // bound of every device-side wait
   int chain;              // PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU
+  void* workspace;        // prism_scan_fwd_workspace_size() bytes (NULL when that is 0)
 };
 
 // Pointers and sizes of one prism_decode_step call (device pointers).

@@ -12,6 +12,7 @@ cudaError_t launch_prologue(const void* v, const float* alpha, const void* gain,
                             int dtype, float* rho, cudaStream_t stream, int chain);
 bool chunk_tc_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
 cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream);
+size_t chunk_tc_workspace_bytes(int B, int T, int H);
 cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t stream);
 }  // namespace prism
 
@@ -93,7 +94,9 @@ void prism_set_spin_limit(long long limit) {
 
 size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
                                      int dtype) {
-  (void)B; (void)T; (void)H; (void)d_k; (void)d_v; (void)L; (void)W; (void)chunk; (void)dtype;
+  if (check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype) != PRISM_OK) return 0;
+  // the tensor-core path keeps the inverse T of every chunk (bf16 64 x 64) in the workspace
+  if (prism::chunk_tc_supported(d_k, d_v, L, W, chunk, dtype)) return prism::chunk_tc_workspace_bytes(B, T, H);
   return 0;
 }
 
@@ -116,7 +119,7 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* 
   if (rc != PRISM_OK) return rc;
   if (!q || !k || !v || !gamma || !beta || !conv_w || !o) return PRISM_ERR_INVALID_ARG;
   if (L > 1 && (!u || !alpha || !gain)) return PRISM_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, gamma, beta, conv_w, o, S0, lengths, S_final,
+  const void* ptrs[] = {q, k, v, gamma, beta, conv_w, o, S0, lengths, S_final, workspace,
                         L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return PRISM_ERR_UNSUPPORTED;
@@ -128,7 +131,8 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* 
 
   prism::ScanParams p{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr,
                       L > 1 ? gain : nullptr, conv_w, S0, lengths, o, S_final,
-                      B, T, H, d_k, d_v, L, W, chunk, status, g_spin_limit.load(), chain};
+                      B, T, H, d_k, d_v, L, W, chunk, status, g_spin_limit.load(), chain,
+                      need > 0 ? workspace : nullptr};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (prism::chunk_tc_supported(d_k, d_v, L, W, chunk, dtype))
@@ -151,6 +155,8 @@ int prism_scan_fwd_host(const void* host_q, const void* host_k, const void* host
   if (!host_q || !host_k || !host_v || !host_gamma || !host_beta || !host_conv_w || !host_o) return PRISM_ERR_INVALID_ARG;
   if (L > 1 && (!host_u || !host_alpha || !host_gain)) return PRISM_ERR_INVALID_ARG;
   if ((host_S0 && !dev_S0) || (host_lengths && !dev_lengths)) return PRISM_ERR_INVALID_ARG;
+  const size_t need = prism_scan_fwd_workspace_size(B, T, H, dk, dv, L, W, chunk, dtype);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return PRISM_ERR_WORKSPACE;
   const size_t es = dtype == PRISM_FP32 ? 4 : 2;
   const size_t toks = (size_t)B * T * H;
   const size_t m = (size_t)(L - 1);

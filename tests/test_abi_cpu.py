@@ -49,14 +49,15 @@ def test_status_strings(L):
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails before any CUDA call
 
 
-def call(lib_, **kw):
+def call(lib_, workspace_ok=True, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, gamma=FAKE, beta=FAKE, u=FAKE, alpha=FAKE, gain=FAKE, conv_w=FAKE,
              S0=None, lengths=None, B=2, T=8, H=2, d_k=64, d_v=64, L=4, W=4, chunk=64, dtype=0,
              o=FAKE, S_final=None)
     a.update(kw)
+    ws, ws_bytes = (FAKE, 1 << 40) if workspace_ok else (None, 0)
     return lib_.prism_scan_fwd(a["q"], a["k"], a["v"], a["gamma"], a["beta"], a["u"], a["alpha"], a["gain"],
-                            a["conv_w"], a["S0"], a["lengths"], a["B"], a["T"], a["H"], a["d_k"], a["d_v"],
-                            a["L"], a["W"], a["chunk"], a["dtype"], a["o"], a["S_final"], None, 0, None)
+                               a["conv_w"], a["S0"], a["lengths"], a["B"], a["T"], a["H"], a["d_k"], a["d_v"],
+                               a["L"], a["W"], a["chunk"], a["dtype"], a["o"], a["S_final"], ws, ws_bytes, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -77,7 +78,17 @@ def test_L1_needs_no_residual_inputs(L):
 
 
 def test_workspace_size_query(L):
-    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) >= 0
+    # tensor-core path: one bf16 64 x 64 inverse per (b, h, chunk); other paths need none
+    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) == 16 * 6 * 32 * 64 * 64 * 2
+    assert prism.workspace_size(2, 100, 3, 64, 64, 2, 4, 64, 0) == 2 * 3 * 2 * 8192
+    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 1) == 0   # fp32: token-by-token kernel
+    assert prism.workspace_size(1, 64, 8, 128, 128, 8, 4, 64, 0) == 0       # L = 8: token-by-token kernel
+    assert prism.workspace_size(0, 64, 8, 128, 128, 4, 4, 64, 0) == 0       # invalid sizes
+
+
+def test_missing_workspace_is_rejected_before_launch(L):
+    # the tensor-core shapes need a workspace; without one the call fails before any launch
+    assert call(L, workspace_ok=False) == 3
 
 
 def test_prologue_invalid_arguments(L):
