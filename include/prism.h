@@ -146,6 +146,28 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v,
 size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L,
                                      int W, int chunk, int dtype);
 
+/* Size of the device-global scratch behind prism_scan_fwd_static. */
+#define PRISM_STATIC_WORKSPACE_BYTES (32u << 20)
+
+/*
+ * prism_scan_fwd_static - prism_scan_fwd_ex without a caller-supplied workspace and
+ * without any allocation: the scratch is a file-scope device array of
+ * PRISM_STATIC_WORKSPACE_BYTES (32 MiB, 256-byte aligned) inside the library, one per
+ * device, located once per device with cudaGetSymbolAddress.  Results are bit-for-bit
+ * those of prism_scan_fwd_ex with a workspace.  Sizes whose
+ * prism_scan_fwd_workspace_size() exceeds PRISM_STATIC_WORKSPACE_BYTES return
+ * PRISM_ERR_WORKSPACE before any launch (the 130M-LM layer, B=16 T=2048 H=6 d=128,
+ * needs 24 MiB).  Because the scratch is shared, calls on one device must not overlap
+ * in time: issue them on one stream or order them; calls on one stream may follow each
+ * other freely.  Other arguments, conventions and errors as for prism_scan_fwd_ex.
+ */
+int prism_scan_fwd_static(const void* q, const void* k, const void* v,
+                          const float* gamma, const float* beta,
+                          const void* u, const float* alpha, const void* gain,
+                          const float* conv_w, const float* S0, const int32_t* lengths,
+                          int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
+                          int dtype, void* o, float* S_final, prism_stream_t stream, int chain);
+
 /*
  * prism_scan_fwd_host - the same operation on HOST buffers: copies every input
  * from host memory into the caller's device buffers, runs prism_scan_fwd on

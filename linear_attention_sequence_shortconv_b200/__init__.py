@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     prologue_fwd,
     scan_fwd,
     scan_fwd_host,
+    scan_fwd_static,
     set_spin_limit,
     status_string,
     stream_status,

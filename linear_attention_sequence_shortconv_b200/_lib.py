@@ -35,6 +35,7 @@ EXPORTS = (
     "prism_scan_fwd_ex",
     "prism_scan_fwd_workspace_size",
     "prism_scan_fwd_host",
+    "prism_scan_fwd_static",
     "prism_prologue_fwd",
     "prism_prologue_fwd_ex",
     "prism_decode_step",
@@ -76,6 +77,9 @@ def lib() -> ctypes.CDLL:
     L.prism_scan_fwd_workspace_size.restype = cs
     L.prism_scan_fwd_host.argtypes = ([vp] * 11 + [vp] * 11 + [ci] * 9 + [vp, vp, vp, vp, vp, cs, vp])
     L.prism_scan_fwd_host.restype = ci
+    L.prism_scan_fwd_static.argtypes = [vp, vp, vp, fp, fp, vp, fp, vp, fp, fp, i32p,
+                                        ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, fp, vp, ci]
+    L.prism_scan_fwd_static.restype = ci
     L.prism_prologue_fwd.argtypes = [vp, fp, vp, fp, i32p, ci, ci, ci, ci, ci, ci, ci, fp, vp]
     L.prism_prologue_fwd.restype = ci
     L.prism_prologue_fwd_ex.argtypes = L.prism_prologue_fwd.argtypes + [ci]
@@ -192,6 +196,42 @@ def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 
         _ptr(workspace), ws_bytes if workspace is not None else 0, _stream_handle(stream), chain_code)
     if rc != 0:
         raise PrismError(rc, "prism_scan_fwd_ex")
+    return o, (S_final if want_state else None)
+
+
+def scan_fwd_static(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 64,
+                    S0=None, lengths=None, want_state: bool = True, o=None, S_final=None,
+                    stream=None, chain: str = "linear"):
+    """scan_fwd through prism_scan_fwd_static: no workspace argument, and the library
+    allocates nothing (its scratch is a device-global array); returns (o, S_final)."""
+    chain_code = _chain_code(chain)
+    dt = q.dtype
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, dt)
+    for name, t in (("gamma", gamma), ("beta", beta), ("conv_w", conv_w)):
+        _check(t, name, torch.float32)
+    if L > 1:
+        _check(u, "u", dt)
+        _check(gain, "gain", dt)
+        _check(alpha, "alpha", torch.float32)
+    _check(S0, "S0", torch.float32, required=False)
+    _check(lengths, "lengths", torch.int32, required=False)
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    W = conv_w.shape[-1]
+    if o is None:
+        o = torch.empty((B, T, H, d_v), dtype=dt, device=q.device)
+    if want_state and S_final is None:
+        S_final = torch.empty((B, H, d_v, d_k), dtype=torch.float32, device=q.device)
+    rc = lib().prism_scan_fwd_static(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+        _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
+        _ptr(conv_w), _ptr(S0), _ptr(lengths),
+        B, T, H, d_k, d_v, L, W, chunk, code,
+        _ptr(o), _ptr(S_final if want_state else None), _stream_handle(stream), chain_code)
+    if rc != 0:
+        raise PrismError(rc, "prism_scan_fwd_static")
     return o, (S_final if want_state else None)
 
 
