@@ -69,7 +69,10 @@ struct Layout {
   static constexpr uint32_t OFF_P = OFF_U + SZ_U;
   static constexpr uint32_t SZ_P = NA * U_ATOM;
   static constexpr uint32_t OFF_BQ = OFF_P + SZ_P;
-  static constexpr uint32_t SZ_BQ = M * kAtom;  // [Bku;QU] (128 x 64m), later P~ (64m x D)
+  // [Bku;QU] (128 x 64m); between MMA2 and the next epilogue, the next prologue's v tile
+  // (NA atom columns of 72 rows, 9 KB apart) and the ShortConv taps
+  static constexpr uint32_t SZ_VT = NA * 9216u + D * 16u;  // v tile + ShortConv taps (W <= 4)
+  static constexpr uint32_t SZ_BQ = M == 0 ? 0u : (M * kAtom > SZ_VT ? M * kAtom : SZ_VT);
   static constexpr uint32_t OFF_TQ = OFF_BQ + SZ_BQ;
   static constexpr uint32_t OFF_SXA = OFF_TQ + kAtom;  // S bf16 | X^T, Delta~^T
   static constexpr uint32_t OFF_SMALL = OFF_SXA + 2 * kAtom;  // gate tables, barriers
@@ -78,7 +81,6 @@ struct Layout {
   // allocation) is resident per SM
   static constexpr uint32_t SMEM_ALLOC = (BYTES + 1024 > 116u * 1024u) ? BYTES + 1024 : 116u * 1024u;
   static_assert(SMEM_ALLOC <= 232448, "exceeds the 227 KB opt-in shared memory of sm_100");
-  static_assert(SZ_BQ >= SZ_P, "P~ must fit where [Bku;QU] was");
 };
 
 struct TcArgs {
@@ -114,8 +116,6 @@ __device__ __forceinline__ void st_bf16x8(uint8_t* base, uint32_t off, const flo
   u.w = pack_bf16x2(x[6], x[7]);
   *reinterpret_cast<uint4*>(base + off) = u;
 }
-
-__device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
 // element e (0..7) of 8 packed bf16
 __device__ __forceinline__ float bf16_at(const uint4& u, int e) {
@@ -435,6 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_load + 2);
   int* s_abort = reinterpret_cast<int*>(bar_load + 3);
   uint64_t* bar_drain = bar_load + 4;  // one commit on the abort path: every MMA issued has completed
+  uint64_t* bar_pre = bar_load + 5;    // gain and v tiles of the next prologue
+  uint64_t* bar_mma1 = bar_load + 6;   // MMA1 of a chunk (issued while the previous one finishes)
   uint8_t* sX = sSXA;                          // X^T      bf16 [128][64] K-major
   uint8_t* sDl = sSXA + kAtom;                 // Delta~^T bf16 [128][64] K-major
 
@@ -452,6 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_load, 1);
     mbar_init(bar_mma, 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_pre, 1);
+    mbar_init(bar_mma1, 1);
     fence_mbar_init();
     *s_abort = 0;
     tma_prefetch_desc(&map_q);
@@ -477,7 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t aKQ = smem_u32(sKQ), aU = smem_u32(sU), aP = smem_u32(sP), aBQ = smem_u32(sBQ);
   const uint32_t aTQ = smem_u32(sTQ), aS = smem_u32(sSXA), aX = smem_u32(sX), aDl = smem_u32(sDl);
-  uint32_t ph_load = 0, ph_mma = 0;
+  uint32_t ph_load = 0, ph_mma = 0, ph_pre = 0, ph_mma1 = 0;
+  int pre_inflight = -1;  // (thread 0) phase of the prologue tiles in flight, or -1
   // (thread 0) phase of a TMA batch / MMA commit in flight and not yet observed, or -1
   int load_inflight = -1, mma_inflight = -1;
   bool load_open = false;  // (thread 0) next chunk's Q/U loads issued, closing arrival not yet made
@@ -519,27 +524,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     load_t(t0 / kC);
     load_k_arrive(t0);
   };
-  // L2 prefetch of the next chunk's k, q, v (D bf16 per token) and u, gain (M*D bf16 per
-  // token): one 128-byte line per thread and request, spread over all threads.
-  auto prefetch_next_l2 = [&](int t0) {
-    constexpr int LK = D * 2 / 128, LU = M * D * 2 / 128;  // 128-byte lines per token
-    const int i = tid & 63, g = tid >> 6;                   // 8 groups of 64 threads
-    if (t0 + i < T) {
-      const size_t th = ((size_t)b * T + t0 + i) * H + h;
-      if (g < 3) {  // k, q, v: LK lines each
-        const __nv_bfloat16* base = g == 0 ? p.k : (g == 1 ? p.q : p.v);
-        const char* ptr = reinterpret_cast<const char*>(base + th * D);
+  // Prologue tiles of chunk nn: its gain rows into P's buffer (the prologue turns them into
+  // P in place) and 72 rows of v, t0-8 .. t0+63 (the ShortConv history included; zero fill
+  // before the sequence start and past T), into the [Bku;QU] buffer.
+  constexpr uint32_t VT_ATOM = 72 * 128;
+  auto load_pre = [&](int nn) {
+    const int tn = nn * kC;
+    mbar_arrive_expect_tx(bar_pre, NA * (M * 8192 + VT_ATOM));
 #pragma unroll
-        for (int r = 0; r < LK; ++r) prefetch_l2(ptr + r * 128);
-      } else if (M > 0) {  // u (groups 3..4) and gain (groups 5..7): LU lines each, split
-        const bool is_u = g < 5;
-        const int part = is_u ? g - 3 : g - 5, nparts = is_u ? 2 : 3;
-        const char* ptr = reinterpret_cast<const char*>((is_u ? p.u : p.gain) + th * M * D);
-        for (int r = part; r < LU; r += nparts) prefetch_l2(ptr + r * 128);
-      }
+    for (int a = 0; a < NA; ++a) {
+      tma_load_4d(sBQ + a * VT_ATOM, &map_v, bar_pre, 64 * a, h, tn - 8, b);
+#pragma unroll
+      for (int l = 0; l < M; ++l)
+        tma_load_5d(sP + a * Ly::U_ATOM + l * 8192, &map_g, bar_pre, 64 * a, l, h, tn, b);
     }
+    pre_inflight = (int)ph_pre;
   };
-
+  // (thread 0) MMA1 of the chunk whose K, Q, U, T tiles are in flight on bar_load: [K;Q] x [K;U]^T
+  // into R1.  Issued as soon as those tiles are in, while the previous chunk's state pass runs.
+  auto issue_mma1 = [&]() -> bool {
+    if (!mbar_wait(bar_load, ph_load, lim, p.status)) return false;
+    load_inflight = -1;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < 4 * NA; ++kk) {
+      const uint64_t a = kdesc(aKQ, kk, kAtom);
+      mma_bf16(tmem + R1, a, a, idesc_bf16(128, 64, 0, 0), kk > 0);
+      if (M > 0) mma_bf16(tmem + R1 + 64, a, kdesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, UR, 0, 0), kk > 0);
+    }
+    mma_commit(bar_mma1);
+    return true;
+  };
   constexpr int CPT = D / 8;           // threads per token in the prologue
   constexpr int TPP = kThreads / CPT;  // tokens per prologue pass
   const int pc8 = (tid % CPT) * 8;
@@ -578,8 +593,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     sBeta[buf * 64 + 2 * lane + 1] = gl[3];
   };
 
-  // Chunk prologue: rho_{i,l} = alpha_{i,l} r_{i,l} -> P (bf16); needs the chunk's gate prefix in buf.
-  auto prologue = [&](int n, int buf, const float* taps) {
+  // Chunk prologue: rho_{i,l} = alpha_{i,l} r_{i,l} -> P (bf16), from the chunk's gain and v
+  // tiles (load_pre) and its alpha values (load_alpha); needs the chunk's gate prefix in buf.
+  constexpr int NPASS = kC / TPP;
+  constexpr int M1 = M > 0 ? M : 1;
+  auto load_alpha = [&](int n, float (&al)[NPASS][M1]) {
+    const int t0 = n * kC;
+    const int nv = min(kC, len - t0);
+#pragma unroll
+    for (int pass = 0; pass < NPASS; ++pass) {
+      const int i = pass * TPP + tid / CPT;
+      const size_t th = ((size_t)b * T + min(t0 + i, T - 1)) * H + h;
+#pragma unroll
+      for (int l = 0; l < M1; ++l) al[pass][l] = (M > 0 && i < nv) ? __ldg(p.alpha + th * M + l) : 0.f;
+    }
+  };
+  auto prologue = [&](int n, int buf, const float* taps, const float (&al)[NPASS][M1]) {
     const int t0 = n * kC;
     const int nv = min(kC, len - t0);
     // Fast path (chunk log-decay >= -60): write P~ = diag(c) P with c_i = e^{G_63 - G_i}; the
@@ -587,71 +616,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float G63 = sG[buf * 64 + 63];
     const bool pfast = G63 >= -60.f;
     if (M > 0) {
-      constexpr int NPASS = kC / TPP;
-      // every global load of every pass first (independent requests in flight together)
-      uint4 vraw[NPASS][4], graw[NPASS][M > 0 ? M : 1];
-      float al[NPASS][M > 0 ? M : 1];
 #pragma unroll
       for (int pass = 0; pass < NPASS; ++pass) {
         const int i = pass * TPP + tid / CPT;
-        const int t = t0 + i;
-        if (i < nv) {
-          const size_t th = ((size_t)b * T + t) * H + h;
-          const __nv_bfloat16* vp = p.v + th * D + pc8;
-          vraw[pass][0] = ldg16(vp);
+        if (i >= nv) {  // padded step: rho = 0
+          const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int w = 1; w < 4; ++w)
-            vraw[pass][w] = (w < p.W && t - w >= 0) ? ldg16(vp - (size_t)w * H * D) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-          for (int l = 0; l < M; ++l) {
-            graw[pass][l] = ldg16(p.gain + (th * M + l) * D + pc8);
-            al[pass][l] = __ldg(p.alpha + th * M + l);
-          }
-        } else {  // padded step: rho = 0
-#pragma unroll
-          for (int w = 0; w < 4; ++w) vraw[pass][w] = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-          for (int l = 0; l < M; ++l) {
-            graw[pass][l] = make_uint4(0u, 0u, 0u, 0u);
-            al[pass][l] = 0.f;
-          }
+          for (int l = 0; l < M; ++l) st_bf16x8(sP, sw128_offset(l * 64 + i, pc8, Ly::U_ATOM), z);
+          continue;
         }
-      }
-#pragma unroll
-      for (int pass = 0; pass < NPASS; ++pass) {
-        const int i = pass * TPP + tid / CPT;
         const float ci = pfast ? __expf(G63 - sG[buf * 64 + i]) : 1.f;
         float r[8];
         {
+          const uint4 v0 = *reinterpret_cast<const uint4*>(sBQ + sw128_offset(8 + i, pc8, VT_ATOM));
           float a[8];
           const float4 lo0 = *reinterpret_cast<const float4*>(taps + pc8);
           const float4 hi0 = *reinterpret_cast<const float4*>(taps + pc8 + 4);
           const float t0v[8] = {lo0.x, lo0.y, lo0.z, lo0.w, hi0.x, hi0.y, hi0.z, hi0.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) a[e] = t0v[e] * bf16_at(vraw[pass][0], e);
+          for (int e = 0; e < 8; ++e) a[e] = t0v[e] * bf16_at(v0, e);
 #pragma unroll
           for (int w = 1; w < 4; ++w) {
             if (w < p.W) {
+              const uint4 vw = *reinterpret_cast<const uint4*>(sBQ + sw128_offset(8 + i - w, pc8, VT_ATOM));
               const float4 lo = *reinterpret_cast<const float4*>(taps + w * D + pc8);
               const float4 hi = *reinterpret_cast<const float4*>(taps + w * D + pc8 + 4);
               const float tw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-              for (int e = 0; e < 8; ++e) a[e] += tw[e] * bf16_at(vraw[pass][w], e);
+              for (int e = 0; e < 8; ++e) a[e] += tw[e] * bf16_at(vw, e);
             }
           }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) r[e] = bf16_at(vraw[pass][0], e) - a[e];
+          for (int e = 0; e < 8; ++e) r[e] = bf16_at(v0, e) - a[e];
         }
 #pragma unroll
         for (int l = 0; l < M; ++l) {
+          const uint32_t off = sw128_offset(l * 64 + i, pc8, Ly::U_ATOM);
+          const uint4 g = *reinterpret_cast<const uint4*>(sP + off);  // gain, replaced by rho below
           float rho[8];
           const float alc = al[pass][l] * ci;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            r[e] = chain_step(r[e], bf16_at(graw[pass][l], e), CH);
+            r[e] = chain_step(r[e], bf16_at(g, e), CH);
             rho[e] = alc * r[e];
           }
-          st_bf16x8(sP, sw128_offset(l * 64 + i, pc8, Ly::U_ATOM), rho);
+          st_bf16x8(sP, off, rho);
         }
       }
     }
@@ -680,8 +689,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0 && nchunks > 0) {
     issue_loads(0);
     load_inflight = (int)ph_load;
+    if (M > 0) load_pre(0);
   }
-  float* taps0 = reinterpret_cast<float*>(sBQ);  // free until chunk 0's epilogue
+  float al0[NPASS][M1];
+  if (nchunks > 0) load_alpha(0, al0);
+  float* taps0 = reinterpret_cast<float*>(sTQ + 8192);  // rows 64..127 of TQ: free until chunk 0's epilogue
   if (nchunks > 0 && warp == 0) {
     float gl[4];
     gate_load(0, gl);
@@ -708,7 +720,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st16(tl + RS + j0, s);
     }
   }
-  if (nchunks > 0) prologue(0, 0, taps0);
+  if (nchunks > 0 && M > 0) {
+    const bool okp = warp_wait(bar_pre, ph_pre, lim, p.status);
+    if (okp) {
+      if (tid == 0) pre_inflight = -1;
+      prologue(0, 0, taps0, al0);
+    } else if (lane == 0) {
+      atomicExch(s_abort, 1);
+    }
+  }
+  ph_pre ^= 1;
+  if (tid == 0 && nchunks > 0 && !issue_mma1()) *s_abort = 1;
+  ph_load ^= 1;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -721,30 +744,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* G = sG + cur * 64;
     const float* Bt = sBeta + cur * 64;
 
-    // ---------------- A: wait for K,Q,U,T; MMA1 + MMA3; per-chunk decay tables; L2 prefetch of chunk n+1
+    // ---------------- A: MMA3 (S_n x [K;Q]^T; MMA1 was issued at the end of the previous chunk);
+    // per-chunk decay tables; L2 prefetch of the next chunk's gate lines
     if (tid == 0) {
-      const bool ok = mbar_wait(bar_load, ph_load, lim, p.status);
-      if (ok) {
-        load_inflight = -1;
-        tc_fence_after();
+      tc_fence_after();
+      // covered by the commit after MMA2 and QK*T (step E reads D3 after that one)
 #pragma unroll
-        for (int kk = 0; kk < 4 * NA; ++kk) {
-          const uint64_t a = kdesc(aKQ, kk, kAtom);
-          mma_bf16(tmem + R1, a, a, idesc_bf16(128, 64, 0, 0), kk > 0);
-          if (M > 0) mma_bf16(tmem + R1 + 64, a, kdesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, UR, 0, 0), kk > 0);
-        }
-        mma_commit(bar_mma);  // step B waits for MMA1 only
-        mma_inflight = (int)ph_mma;
-        // MMA3 (read in step E) is covered by the next commit, after MMA2 and QK*T
-#pragma unroll
-        for (int kk = 0; kk < 4 * NA; ++kk)
-          mma_bf16(tmem + D3, kdesc(aS, kk, kAtom), kdesc(aKQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
-      } else {
-        *s_abort = 1;
-      }
+      for (int kk = 0; kk < 4 * NA; ++kk)
+        mma_bf16(tmem + D3, kdesc(aS, kk, kAtom), kdesc(aKQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
     }
-    ph_load ^= 1;
-    if (n + 1 < nchunks) prefetch_next_l2(t0 + kC);
     if (warp == 1 && n + 1 < nchunks) {
       // the next chunk's gates are token-major spans [b, t0+64 .. t0+128, :]: prefetch their L2 lines
       const int tn = t0 + kC, te = min(tn + kC, T);
@@ -768,12 +776,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (*s_abort) { aborted = true; break; }
 
     // ---------------- B: epilogue of MMA1 -> [Bku;QU], QK (bf16); then MMA2, MMA5a (fast), QK*T
-    bool ok = warp_wait(bar_mma, ph_mma, lim, p.status);
-    ph_mma ^= 1;
-    if (tid == 0 && ok) {
-      mma_inflight = -1;
-      if (n + 1 < nchunks) load_q(t0 + kC);  // MMA1 and MMA3 have read Q
-    }
+    bool ok = warp_wait(bar_mma1, ph_mma1, lim, p.status);
+    ph_mma1 ^= 1;
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     float gl_next[4] = {1.f, 1.f, 0.f, 0.f};  // warp 2: next chunk's gates, scanned in step C
     if (warp == 2 && n + 1 < nchunks) gate_load(n + 1, gl_next);
@@ -787,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float rsu = fast ? (krow ? Bt[t] : 1.f) * __expf(Gt - G[63]) : 0.f;
       constexpr int NP = (64 + UR) / 16;  // 16-column pieces of R1
       constexpr int PQ = NP / 4;           // pieces of this thread's column quarter
-      constexpr int PB = PQ >= 2 ? 2 : 1;  // pieces per TMEM wait
+      constexpr int PB = PQ;               // pieces per TMEM wait: all of them
 #pragma unroll
       for (int pb = 0; pb < PQ; pb += PB) {
       uint32_t raw[PB][16];
@@ -840,6 +844,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       }
     }
+    if (ok && M > 0 && !fast) {
+      // exact path: U <- diag(c) U in place, so that MMA5a = P^T (diag(c) U) runs next to MMA2
+      // (both read the unscaled P); MMA1, the other reader of U, has completed
+      for (int e = tid; e < UR * D / 8; e += kThreads) {
+        const int r = e / (D / 8), c8 = (e % (D / 8)) * 8;
+        const uint32_t off = sw128_offset(r, c8, Ly::U_ATOM);
+        const uint4 u = *reinterpret_cast<const uint4*>(sU + off);
+        const float sc = sCdec[r & 63];
+        float f[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) f[k] = sc * bf16_at(u, k);
+        st_bf16x8(sU, off, f);
+      }
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -851,14 +869,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < UR / 16; ++kk)  // MMA2: (Bku P)^T | (QU P)^T
           mma_bf16(tmem + R1, mndesc(aP, kk, Ly::U_ATOM), kdesc(aBQ, kk, kAtom), idesc_bf16(128, 128, 1, 0),
                    kk > 0);
-        if (fast) {
-          // MMA5a (RS += P~^T U) needs only P~ (= P), U and the decayed RS: issued now, it
-          // completes before step E's wait, ahead of the next prologue overwriting P
+        // MMA5a: RS += P~^T U (fast path) or P^T (diag(c) U) (exact path); it completes before
+        // step E's wait, after which P's and U's buffers take the next chunk's tiles
 #pragma unroll
-          for (int kk = 0; kk < UR / 16; ++kk)
-            mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1),
-                     1);
-        }
+        for (int kk = 0; kk < UR / 16; ++kk)
+          mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
       }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)  // [T;QK] x T: rows 64..127 = QK T
@@ -871,6 +886,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the next prologue and the values of v it needs for X (their latency hides behind the MMAs)
     if (warp == 2 && n + 1 < nchunks) gate_scan(gl_next, cur ^ 1);
     const float tap_reg = (M > 0 && tap_thread) ? __ldg(cw_head + tid) : 0.f;
+    float al_next[NPASS][M1];  // alpha of the next chunk, for its prologue
     // (padded steps have beta = 0, so any in-range token may stand in for them)
     __nv_bfloat16 vraw16[16];  // converted where X is formed, so the loads are not waited on here
     {
@@ -887,8 +903,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     ph_mma ^= 1;
     if (tid == 0 && ok) {
       mma_inflight = -1;
-      if (fast && n + 1 < nchunks) load_u(t0 + kC);  // fast path: MMA5a (issued in C) has read U
+      if (n + 1 < nchunks) {  // MMA3, MMA2 and MMA5a, the last readers of Q, P, U and [Bku;QU], are done
+        load_q(t0 + kC);
+        load_u(t0 + kC);
+        if (M > 0) load_pre(n + 1);
+      }
     }
+    if (n + 1 < nchunks) load_alpha(n + 1, al_next);
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
     if (ok) {
@@ -898,23 +919,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(tl + R1 + 128 + 16 * cq, x);
         st_bf16x8(sTQ, sw128_offset(row, 16 * cq, kAtom), x);
         st_bf16x8(sTQ, sw128_offset(row, 16 * cq + 8, kAtom), x + 8);
-      }
-      if (M > 0 && !fast) {  // exact path: P~ = diag(c) P into the [Bku;QU] buffer
-        for (int e = tid; e < UR * D / 8; e += kThreads) {
-          const int r = e / (D / 8), c8 = (e % (D / 8)) * 8;
-          const uint32_t off = sw128_offset(r, c8, Ly::U_ATOM);
-          const float sc = sCdec[r & 63];
-          uint4 u = *reinterpret_cast<const uint4*>(sP + off);
-          __nv_bfloat162* hx = reinterpret_cast<__nv_bfloat162*>(&u);
-          float f[8];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float2 ff = __bfloat1622float2(hx[k]);
-            f[2 * k] = sc * ff.x;
-            f[2 * k + 1] = sc * ff.y;
-          }
-          st_bf16x8(sBQ, off, f);
-        }
       }
       if (srow) {  // state row c = row; tokens t = 16*cq + e
         const int tb = 16 * cq;
@@ -948,32 +952,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + R1 + 128, kdesc(aX, kk, kAtom), kdesc(aTQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
-      if (M > 0 && !fast) {  // exact path: P~ was copied into the [Bku;QU] buffer in this step
-#pragma unroll
-        for (int kk = 0; kk < UR / 16; ++kk)
-          mma_bf16(tmem + RS, mndesc(aBQ, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
-      }
       mma_commit(bar_mma);
       mma_inflight = (int)ph_mma;
     }
-
-    // ---------------- F: next chunk's prologue while MMA4 (and, on the exact path, MMA5a) run;
-    // P is no longer read: MMA2 and the fast-path MMA5a completed before step E's wait
-    if (n + 1 < nchunks) {
-      float* taps = reinterpret_cast<float*>(sDl);  // Delta~ is written only after MMA4 completes
-      if (M > 0 && tap_thread) taps[(tid % p.W) * D + tid / p.W] = tap_reg;
-      __syncthreads();
-      prologue(n + 1, cur ^ 1, taps);
-      __syncthreads();  // every thread is done with the staged taps before Delta~ overwrites them
-    }
-    fence_proxy_async_smem();
 
     // ---------------- G: Delta~^T -> SXA; o = O partial + (QKT X); issue MMA5b
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) {
       mma_inflight = -1;
-      if (!fast && n + 1 < nchunks) load_u(t0 + kC);  // exact path: MMA5a has read U
       if (n + 1 < nchunks) load_t(n + 1);              // MMA4, the last reader of TQ, has completed
     }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
@@ -1011,16 +998,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       bulk_commit_group();
     }
 
-    // ---------------- I: next chunk's loads; S_{n+1} -> bf16 SXA (and S_final)
-    ok = warp_wait(bar_mma, ph_mma, lim, p.status);
-    ph_mma ^= 1;
-    if (tid == 0) {
-      if (ok) mma_inflight = -1;
-      if (ok && n + 1 < nchunks) {
-        load_k_arrive(t0 + kC);  // MMA5b has read K
-        load_inflight = (int)ph_load;
+    // ---------------- F: next chunk's prologue while MMA5b runs.  Warp 0 first waits for MMA5b
+    // and requests the next chunk's K (MMA5b has read K), so that load overlaps the prologue.
+    bool ok5 = true;
+    if (warp == 0) {
+      ok5 = warp_wait(bar_mma, ph_mma, lim, p.status);
+      if (tid == 0 && ok5) {
+        mma_inflight = -1;
+        if (n + 1 < nchunks) {
+          load_k_arrive(t0 + kC);
+          load_inflight = (int)ph_load;
+        }
       }
+      if (!ok5 && lane == 0) atomicExch(s_abort, 1);
     }
+    if (n + 1 < nchunks) {
+      float* taps = reinterpret_cast<float*>(sBQ + NA * VT_ATOM);  // behind the v tile
+      if (M > 0 && tap_thread) taps[(tid % p.W) * D + tid / p.W] = tap_reg;
+      __syncthreads();
+      if (M > 0) {
+        const bool okp = warp_wait(bar_pre, ph_pre, lim, p.status);
+        if (okp) {
+          if (tid == 0) pre_inflight = -1;
+          prologue(n + 1, cur ^ 1, taps, al_next);
+        } else if (lane == 0) {
+          atomicExch(s_abort, 1);
+        }
+      }
+      ph_pre ^= 1;
+      // MMA1 of the next chunk (R1 is free since step G); it runs under the state pass below
+      if (tid == 0 && ok5 && !issue_mma1()) *s_abort = 1;
+      ph_load ^= 1;
+    }
+    fence_proxy_async_smem();
+
+    // ---------------- I: S_{n+1} -> bf16 SXA (and S_final)
+    ok = warp == 0 ? ok5 : warp_wait(bar_mma, ph_mma, lim, p.status);
+    ph_mma ^= 1;
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     if (tid == 0) bulk_wait_read_all();  // the o tile in SXA has been read by the TMA store
     __syncthreads();
@@ -1084,6 +1098,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (load_inflight >= 0) mbar_wait(bar_load, (uint32_t)load_inflight, kDrainLimit, p.status);
     if (mma_inflight >= 0) mbar_wait(bar_mma, (uint32_t)mma_inflight, kDrainLimit, p.status);
+    if (pre_inflight >= 0) mbar_wait(bar_pre, (uint32_t)pre_inflight, kDrainLimit, p.status);
     mma_commit(bar_drain);  // also covers MMAs issued after the last commit observed
     mbar_wait(bar_drain, 0u, kDrainLimit, p.status);
   }
@@ -1157,8 +1172,9 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
   const cuuint64_t dims4[4] = {(cuuint64_t)D, H, T, B};
   const cuuint64_t str4[3] = {(cuuint64_t)D * 2, H * D * 2, T * H * D * 2};
   const cuuint32_t box4[4] = {64, 1, 64, 1};
+  const cuuint32_t box_v[4] = {64, 1, 72, 1};  // a chunk's v rows and 8 rows of ShortConv history
   if (!encode(&mq, p.q, 4, dims4, str4, box4) || !encode(&mk, p.k, 4, dims4, str4, box4) ||
-      !encode(&mv, p.v, 4, dims4, str4, box4) || !encode(&mo, p.o, 4, dims4, str4, box4))
+      !encode(&mv, p.v, 4, dims4, str4, box_v) || !encode(&mo, p.o, 4, dims4, str4, box4))
     return cudaErrorInvalidValue;
   if (M > 0) {
     const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)M, H, T, B};

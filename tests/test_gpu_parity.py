@@ -220,3 +220,29 @@ def test_full_size_bitwise_deterministic():
     o3, S3 = gpu_run(inp, w)
     assert np.array_equal(o1, o2) and np.array_equal(o1, o3)
     assert np.array_equal(S1, S2) and np.array_equal(S1, S3)
+
+
+# ---------------------------------------------------------------- strongly decaying chunks
+@pytest.mark.parametrize("name", ["lm_130m", "recsys"])
+@pytest.mark.parametrize("chain", ["linear", "gelu"])
+def test_strongly_decaying_chunks(name, chain):
+    """Chunks whose total log-decay is below -60 take the exact path of the chunk
+    kernel (per-element e^{G_t - G_i}, the state-side decay applied to U instead of
+    P).  Row 0: every other chunk strongly decaying; row 1: all of them; the other
+    rows: the ordinary gates."""
+    w = {"lm_130m": W["lm_130m"].replace(B=3, T=300, H=2, with_s0=True),
+         "recsys": W["recsys"].replace(B=3, T=260, lengths_lo=None)}[name]
+    inp = synth.make_inputs(w)
+    g = inp["gamma"].clone()
+    strong = torch.full_like(g[0, :64], 0.38).to(torch.bfloat16).float()  # 64 log(0.38) = -62
+    for c0 in range(64, w.T, 128):
+        n = min(64, w.T - c0)
+        g[0, c0:c0 + n] = strong[:n]
+    g[1] = torch.full_like(g[1], 0.38).to(torch.bfloat16).float()
+    inp["gamma"] = g
+    import linear_attention_sequence_shortconv_b200 as prism
+    assert prism.uses_tensor_cores(w.d_k, w.d_v, w.L, w.W, w.chunk, prism.PRISM_BF16)
+    o, S = gpu_run(inp, w, chain=chain)
+    o_ref, S_ref = oracle_run(inp, w, chain=chain)
+    assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
