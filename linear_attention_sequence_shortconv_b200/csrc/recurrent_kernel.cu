@@ -93,7 +93,8 @@ int tile_tokens(int dk, int m, int rpb) {
   return 1;
 }
 
-template <typename T, int LPR, int EPL>
+// CH: residual chain step (PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU), fixed at compile time.
+template <typename T, int LPR, int EPL, int CH>
 __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, int TT) {
   constexpr int RPB = kBlock / LPR;  // rows per block
   extern __shared__ __align__(16) uint8_t smem[];
@@ -241,7 +242,7 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
       }
       // rank-m residual write
       for (int l = 0; l < m; ++l) {
-        r = chain_step(r, to_f<T>(sg_[(i * m + l) * RPB + cr]), p.chain);
+        r = chain_step(r, to_f<T>(sg_[(i * m + l) * RPB + cr]), CH);
         const float rho = sal[i * m + l] * r;
         const T* uu = su_ + ((size_t)i * m + l) * dk + EPL * j;
 #pragma unroll
@@ -275,17 +276,23 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   }
 }
 
-template <typename T, int LPR, int EPL>
-cudaError_t launch_shape(const ScanParams& p, cudaStream_t stream) {
+template <typename T, int LPR, int EPL, int CH>
+cudaError_t launch_chain(const ScanParams& p, cudaStream_t stream) {
   constexpr int RPB = kBlock / LPR;
   const int TT = tile_tokens<T>(p.d_k, p.L - 1, RPB);
   const int smem = 2 * TileLayout(TT, p.d_k, p.L - 1, RPB, sizeof(T)).bytes;
-  cudaError_t err =
-      cudaFuncSetAttribute(recurrent_scan_kernel<T, LPR, EPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t err = cudaFuncSetAttribute(recurrent_scan_kernel<T, LPR, EPL, CH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   dim3 grid((p.d_v + RPB - 1) / RPB, p.H, p.B);
-  recurrent_scan_kernel<T, LPR, EPL><<<grid, kBlock, smem, stream>>>(p, TT);
+  recurrent_scan_kernel<T, LPR, EPL, CH><<<grid, kBlock, smem, stream>>>(p, TT);
   return cudaGetLastError();
+}
+
+template <typename T, int LPR, int EPL>
+cudaError_t launch_shape(const ScanParams& p, cudaStream_t stream) {
+  if (p.chain == PRISM_CHAIN_GELU) return launch_chain<T, LPR, EPL, PRISM_CHAIN_GELU>(p, stream);
+  return launch_chain<T, LPR, EPL, PRISM_CHAIN_LINEAR>(p, stream);
 }
 
 template <typename T>
