@@ -356,8 +356,8 @@ __global__ void __launch_bounds__(kPrepThreads) prism_chunk_prep_kernel(const __
       *s_abort = 1;
     }
   }
-  __syncthreads();
-  if (*s_abort == 0 && warp < 2) {  // TMEM lanes 0..63 = token rows t
+  const bool load_failed = __syncthreads_or(*s_abort) != 0;  // uniform decision
+  if (!load_failed && warp < 2) {  // TMEM lanes 0..63 = token rows t
     const bool ok = warp_wait(bar_mma, 0, lim, p.status);
     if (ok) {
       tc_fence_after();
@@ -382,8 +382,8 @@ __global__ void __launch_bounds__(kPrepThreads) prism_chunk_prep_kernel(const __
     }
   }
   tc_fence_before();
-  __syncthreads();
-  if (*s_abort == 0) {
+  const bool failed = __syncthreads_or(*s_abort) != 0;  // uniform: the inverse synchronises internally
+  if (!failed) {
     invert_unit_lower64<LDA>(sA, sY, tid);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {  // T -> bf16 rows of 128 bytes, 16 bytes per thread and pass
@@ -772,8 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sEn[tid] = fast ? __expf(-G[tid]) : 0.f;
       sCdec[tid] = __expf(G[63] - G[tid]);
     }
-    __syncthreads();
-    if (*s_abort) { aborted = true; break; }
+    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
 
     // ---------------- B: epilogue of MMA1 -> [Bku;QU], QK (bf16); then MMA2, MMA5a (fast), QK*T
     bool ok = warp_wait(bar_mma1, ph_mma1, lim, p.status);
@@ -860,8 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) { aborted = true; break; }
+    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
     if (tid == 0) {
       tc_fence_after();
       if (M > 0) {
@@ -945,8 +943,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) { aborted = true; break; }
+    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -984,8 +981,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) { aborted = true; break; }
+    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -1067,8 +1063,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) { aborted = true; break; }
+    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
   }
 
   if (!aborted) {
