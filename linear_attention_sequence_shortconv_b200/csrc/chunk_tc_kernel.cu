@@ -130,6 +130,43 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// The scan kernel's CTA: kThreads worker threads (16 warps) and one MMA warp that issues
+// every tcgen05.mma.  A tcgen05.mma sequence holds its issuing thread for about its
+// execution time; in a warp of its own that no longer stalls the workers, who meet on
+// barrier 1 and hand operands over through mbarriers.
+constexpr int kMmaWarp = kThreads / 32;
+constexpr int kCtaThreads = kThreads + 32;
+
+__device__ __forceinline__ void worker_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
+// Barrier 1 with an OR over the workers' votes: every worker gets the same answer.
+__device__ __forceinline__ bool worker_sync_or(int v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q, p;\n\t"
+      "setp.ne.s32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(v), "n"(kThreads)
+      : "memory");
+  return r != 0;
+}
+
+// Bounded, warp-uniform wait of the MMA warp; also gives up once the abort flag is set.
+__device__ __forceinline__ bool mma_warp_wait(uint64_t* bar, uint32_t parity, long long limit, int* status,
+                                              const volatile int* abort_flag) {
+  bool ok = false;
+  if ((threadIdx.x & 31) == 0) {
+    const uint32_t hint = limit < 1024 ? 0u : 20000u;
+    for (long long i = 0; i < limit && !ok; ++i) {
+      if (mbar_try_wait_suspend(bar, parity, hint)) ok = true;
+      else if (*abort_flag) break;
+    }
+    if (!ok && !*abort_flag) record_status(status, PRISM_ERR_TIMEOUT);
+  }
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 __device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk, uint32_t atom_stride) {
   return sdesc_sw128(base + (uint32_t)(kk >> 2) * atom_stride + (uint32_t)(kk & 3) * 32u, 16, 1024);
 }
@@ -410,7 +447,7 @@ __global__ void __launch_bounds__(kPrepThreads) prism_chunk_prep_kernel(const __
 // CH: residual chain step (PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU), fixed at compile
 // time so the linear chain carries none of the GELU step's code or registers.
 template <int D, int M, int CH>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kCtaThreads, 1)
     prism_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                           const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_v,
                           const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_o,
@@ -437,6 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_drain = bar_load + 4;  // one commit on the abort path: every MMA issued has completed
   uint64_t* bar_pre = bar_load + 5;    // gain and v tiles of the next prologue
   uint64_t* bar_mma1 = bar_load + 6;   // MMA1 of a chunk (issued while the previous one finishes)
+  // worker -> MMA warp hand-overs, one arrival per chunk each: operands of MMA1 requested
+  // (F), S_n in bf16 (A), [Bku;QU] and QK written (B), X written (E), Delta~ written (G)
+  uint64_t* go_F = bar_load + 7;
+  uint64_t* go_A = bar_load + 8;
+  uint64_t* go_B = bar_load + 9;
+  uint64_t* go_E = bar_load + 10;
+  uint64_t* go_G = bar_load + 11;
   uint8_t* sX = sSXA;                          // X^T      bf16 [128][64] K-major
   uint8_t* sDl = sSXA + kAtom;                 // Delta~^T bf16 [128][64] K-major
 
@@ -456,6 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_drain, 1);
     mbar_init(bar_pre, 1);
     mbar_init(bar_mma1, 1);
+    mbar_init(go_F, 1);
+    mbar_init(go_A, 1);
+    mbar_init(go_B, 1);
+    mbar_init(go_E, 1);
+    mbar_init(go_G, 1);
     fence_mbar_init();
     *s_abort = 0;
     tma_prefetch_desc(&map_q);
@@ -483,8 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t aTQ = smem_u32(sTQ), aS = smem_u32(sSXA), aX = smem_u32(sX), aDl = smem_u32(sDl);
   uint32_t ph_load = 0, ph_mma = 0, ph_pre = 0, ph_mma1 = 0;
   int pre_inflight = -1;  // (thread 0) phase of the prologue tiles in flight, or -1
-  // (thread 0) phase of a TMA batch / MMA commit in flight and not yet observed, or -1
-  int load_inflight = -1, mma_inflight = -1;
+  int load_inflight = -1;  // (thread 0) parity of the last closed load phase (the MMA warp consumes it)
   bool load_open = false;  // (thread 0) next chunk's Q/U loads issued, closing arrival not yet made
 
   // The next chunk's tiles are loaded as soon as their buffers are free: Q once MMA1/MMA3 have
@@ -508,6 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   auto load_k_arrive = [&](int t0) {
     load_open = false;
+    load_inflight = (int)ph_load;
+    ph_load ^= 1;
     mbar_arrive_expect_tx(bar_load, NA * 8192);
 #pragma unroll
     for (int a = 0; a < NA; ++a) tma_load_4d(sKQ + a * kAtom, &map_k, bar_load, 64 * a, h, t0, b);
@@ -539,21 +589,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_5d(sP + a * Ly::U_ATOM + l * 8192, &map_g, bar_pre, 64 * a, l, h, tn, b);
     }
     pre_inflight = (int)ph_pre;
-  };
-  // (thread 0) MMA1 of the chunk whose K, Q, U, T tiles are in flight on bar_load: [K;Q] x [K;U]^T
-  // into R1.  Issued as soon as those tiles are in, while the previous chunk's state pass runs.
-  auto issue_mma1 = [&]() -> bool {
-    if (!mbar_wait(bar_load, ph_load, lim, p.status)) return false;
-    load_inflight = -1;
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < 4 * NA; ++kk) {
-      const uint64_t a = kdesc(aKQ, kk, kAtom);
-      mma_bf16(tmem + R1, a, a, idesc_bf16(128, 64, 0, 0), kk > 0);
-      if (M > 0) mma_bf16(tmem + R1 + 64, a, kdesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, UR, 0, 0), kk > 0);
-    }
-    mma_commit(bar_mma1);
-    return true;
   };
   constexpr int CPT = D / 8;           // threads per token in the prologue
   constexpr int TPP = kThreads / CPT;  // tokens per prologue pass
@@ -666,6 +701,95 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
+  if (warp == kMmaWarp) {
+    // ---- the MMA warp: lane 0 issues, in the order the workers hand the operands over
+    const volatile int* abort_flag = s_abort;
+    uint32_t pF = 0, pA = 0, pB = 0, pE = 0, pG = 0, pL = 0;
+    bool ok = true;
+    for (int n = 0; n < nchunks && ok; ++n) {
+      // MMA1: [K;Q] x [K;U]^T -> R1 once the chunk's K, Q, U, T are in
+      ok = mma_warp_wait(go_F, pF, lim, p.status, abort_flag) && mma_warp_wait(bar_load, pL, lim, p.status, abort_flag);
+      pF ^= 1;
+      pL ^= 1;
+      if (!ok) break;
+      if (lane == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4 * NA; ++kk) {
+          const uint64_t a = kdesc(aKQ, kk, kAtom);
+          mma_bf16(tmem + R1, a, a, idesc_bf16(128, 64, 0, 0), kk > 0);
+          if (M > 0) mma_bf16(tmem + R1 + 64, a, kdesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, UR, 0, 0), kk > 0);
+        }
+        mma_commit(bar_mma1);
+      }
+      __syncwarp();
+      // MMA3: S_n x [K;Q]^T -> D3, covered by the next commit (step E reads D3 after it)
+      ok = mma_warp_wait(go_A, pA, lim, p.status, abort_flag);
+      pA ^= 1;
+      if (!ok) break;
+      if (lane == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4 * NA; ++kk)
+          mma_bf16(tmem + D3, kdesc(aS, kk, kAtom), kdesc(aKQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
+      }
+      __syncwarp();
+      // MMA2: (Bku P)^T | (QU P)^T -> R1; MMA5a: P~^T U or P^T (diag(c) U) onto RS; [T;QK] x T
+      ok = mma_warp_wait(go_B, pB, lim, p.status, abort_flag);
+      pB ^= 1;
+      if (!ok) break;
+      if (lane == 0) {
+        tc_fence_after();
+        if (M > 0) {
+#pragma unroll
+          for (int kk = 0; kk < UR / 16; ++kk)
+            mma_bf16(tmem + R1, mndesc(aP, kk, Ly::U_ATOM), kdesc(aBQ, kk, kAtom), idesc_bf16(128, 128, 1, 0),
+                     kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < UR / 16; ++kk)
+            mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1),
+                     1);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + R1 + 128, kdesc(aTQ, kk, kAtom), mndesc(aTQ, kk, kAtom), idesc_bf16(128, 64, 0, 1),
+                   kk > 0);
+        mma_commit(bar_mma);
+      }
+      __syncwarp();
+      // MMA4: X^T x [T;QKT]^T -> Delta^T | (QKT X)^T in R1+128
+      ok = mma_warp_wait(go_E, pE, lim, p.status, abort_flag);
+      pE ^= 1;
+      if (!ok) break;
+      if (lane == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + R1 + 128, kdesc(aX, kk, kAtom), kdesc(aTQ, kk, kAtom), idesc_bf16(128, 128, 0, 0),
+                   kk > 0);
+        mma_commit(bar_mma);
+      }
+      __syncwarp();
+      // MMA5b: Delta~^T K onto RS
+      ok = mma_warp_wait(go_G, pG, lim, p.status, abort_flag);
+      pG ^= 1;
+      if (!ok) break;
+      if (lane == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + RS, kdesc(aDl, kk, kAtom), mndesc(aKQ, kk, kAtom), idesc_bf16(128, D, 0, 1), 1);
+        mma_commit(bar_mma);
+      }
+      __syncwarp();
+    }
+    if (!ok && lane == 0) atomicExch(s_abort, 1);
+    if (lane == 0) {  // every MMA issued has completed before the tensor memory is freed
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0u, kDrainLimit, p.status);
+    }
+    __syncwarp();
+  } else {
   // ---- initial state: RS <- S0 (or 0), bf16 copy -> SXA (A operand of MMA3); chunk 0 prologue
   if (srow) {
 #pragma unroll
@@ -688,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0 && nchunks > 0) {
     issue_loads(0);
-    load_inflight = (int)ph_load;
+    mbar_arrive(go_F);  // MMA1 of chunk 0 as soon as its tiles are in
     if (M > 0) load_pre(0);
   }
   float al0[NPASS][M1];
@@ -700,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gate_scan(gl, 0);
   }
   if (M > 0 && tap_thread) taps0[(tid % p.W) * D + tid / p.W] = __ldg(cw_head + tid);
-  __syncthreads();
+  worker_sync();
   if (srow) {  // RS <- exp(G_63 of chunk 0) S0 (undecayed S0 when there is no chunk: S_final)
     const float b0 = nchunks > 0 ? __expf(sG[63]) : 1.f;
 #pragma unroll
@@ -730,11 +854,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   ph_pre ^= 1;
-  if (tid == 0 && nchunks > 0 && !issue_mma1()) *s_abort = 1;
-  ph_load ^= 1;
   fence_proxy_async_smem();
   tc_fence_before();
-  __syncthreads();
+  worker_sync();
 
   bool aborted = false;
   for (int n = 0; n < nchunks && !aborted; ++n) {
@@ -746,13 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------- A: MMA3 (S_n x [K;Q]^T; MMA1 was issued at the end of the previous chunk);
     // per-chunk decay tables; L2 prefetch of the next chunk's gate lines
-    if (tid == 0) {
-      tc_fence_after();
-      // covered by the commit after MMA2 and QK*T (step E reads D3 after that one)
-#pragma unroll
-      for (int kk = 0; kk < 4 * NA; ++kk)
-        mma_bf16(tmem + D3, kdesc(aS, kk, kAtom), kdesc(aKQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
-    }
+    if (tid == 0) mbar_arrive(go_A);  // S_n (bf16) is in SXA: MMA3
     if (warp == 1 && n + 1 < nchunks) {
       // the next chunk's gates are token-major spans [b, t0+64 .. t0+128, :]: prefetch their L2 lines
       const int tn = t0 + kC, te = min(tn + kC, T);
@@ -772,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sEn[tid] = fast ? __expf(-G[tid]) : 0.f;
       sCdec[tid] = __expf(G[63] - G[tid]);
     }
-    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
+    if (worker_sync_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
 
     // ---------------- B: epilogue of MMA1 -> [Bku;QU], QK (bf16); then MMA2, MMA5a (fast), QK*T
     bool ok = warp_wait(bar_mma1, ph_mma1, lim, p.status);
@@ -790,7 +906,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float rsu = fast ? (krow ? Bt[t] : 1.f) * __expf(Gt - G[63]) : 0.f;
       constexpr int NP = (64 + UR) / 16;  // 16-column pieces of R1
       constexpr int PQ = NP / 4;           // pieces of this thread's column quarter
-      constexpr int PB = PQ;               // pieces per TMEM wait: all of them
+      constexpr int PB = PQ >= 2 ? 2 : 1;  // pieces per TMEM wait
 #pragma unroll
       for (int pb = 0; pb < PQ; pb += PB) {
       uint32_t raw[PB][16];
@@ -859,26 +975,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
-    if (tid == 0) {
-      tc_fence_after();
-      if (M > 0) {
-#pragma unroll
-        for (int kk = 0; kk < UR / 16; ++kk)  // MMA2: (Bku P)^T | (QU P)^T
-          mma_bf16(tmem + R1, mndesc(aP, kk, Ly::U_ATOM), kdesc(aBQ, kk, kAtom), idesc_bf16(128, 128, 1, 0),
-                   kk > 0);
-        // MMA5a: RS += P~^T U (fast path) or P^T (diag(c) U) (exact path); it completes before
-        // step E's wait, after which P's and U's buffers take the next chunk's tiles
-#pragma unroll
-        for (int kk = 0; kk < UR / 16; ++kk)
-          mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1), 1);
-      }
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)  // [T;QK] x T: rows 64..127 = QK T
-        mma_bf16(tmem + R1 + 128, kdesc(aTQ, kk, kAtom), mndesc(aTQ, kk, kAtom), idesc_bf16(128, 64, 0, 1), kk > 0);
-      mma_commit(bar_mma);
-      mma_inflight = (int)ph_mma;
-    }
+    if (worker_sync_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
+    if (tid == 0) mbar_arrive(go_B);  // MMA2, MMA5a, QK*T
 
     // ---------------- C: the next chunk's gate prefix; the tap element this thread stages for
     // the next prologue and the values of v it needs for X (their latency hides behind the MMAs)
@@ -900,7 +998,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) {
-      mma_inflight = -1;
       if (n + 1 < nchunks) {  // MMA3, MMA2 and MMA5a, the last readers of Q, P, U and [Bku;QU], are done
         load_q(t0 + kC);
         load_u(t0 + kC);
@@ -943,21 +1040,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + R1 + 128, kdesc(aX, kk, kAtom), kdesc(aTQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
-      mma_commit(bar_mma);
-      mma_inflight = (int)ph_mma;
-    }
+    if (worker_sync_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
+    if (tid == 0) mbar_arrive(go_E);  // MMA4
 
     // ---------------- G: Delta~^T -> SXA; o = O partial + (QKT X); issue MMA5b
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) {
-      mma_inflight = -1;
       if (n + 1 < nchunks) load_t(n + 1);              // MMA4, the last reader of TQ, has completed
     }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
@@ -981,14 +1070,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
+    if (worker_sync_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
     if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + RS, kdesc(aDl, kk, kAtom), mndesc(aKQ, kk, kAtom), idesc_bf16(128, D, 0, 1), 1);
-      mma_commit(bar_mma);
-      mma_inflight = (int)ph_mma;
+      mbar_arrive(go_G);  // MMA5b
 #pragma unroll
       for (int a = 0; a < NA; ++a) tma_store_4d(&map_o, sX + a * 8192, 64 * a, h, t0, b);
       bulk_commit_group();
@@ -999,19 +1083,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok5 = true;
     if (warp == 0) {
       ok5 = warp_wait(bar_mma, ph_mma, lim, p.status);
-      if (tid == 0 && ok5) {
-        mma_inflight = -1;
-        if (n + 1 < nchunks) {
-          load_k_arrive(t0 + kC);
-          load_inflight = (int)ph_load;
-        }
+      if (tid == 0 && ok5 && n + 1 < nchunks) {
+        load_k_arrive(t0 + kC);
+        mbar_arrive(go_F);  // MMA1 of the next chunk once its tiles are in (R1 is free)
       }
       if (!ok5 && lane == 0) atomicExch(s_abort, 1);
     }
     if (n + 1 < nchunks) {
       float* taps = reinterpret_cast<float*>(sBQ + NA * VT_ATOM);  // behind the v tile
       if (M > 0 && tap_thread) taps[(tid % p.W) * D + tid / p.W] = tap_reg;
-      __syncthreads();
+      worker_sync();
       if (M > 0) {
         const bool okp = warp_wait(bar_pre, ph_pre, lim, p.status);
         if (okp) {
@@ -1022,9 +1103,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ph_pre ^= 1;
-      // MMA1 of the next chunk (R1 is free since step G); it runs under the state pass below
-      if (tid == 0 && ok5 && !issue_mma1()) *s_abort = 1;
-      ph_load ^= 1;
     }
     fence_proxy_async_smem();
 
@@ -1033,7 +1111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ph_mma ^= 1;
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     if (tid == 0) bulk_wait_read_all();  // the o tile in SXA has been read by the TMA store
-    __syncthreads();
+    worker_sync();
     tc_fence_after();
     if (ok && srow) {
       // RS <- exp(G_63 of chunk n+1) S_{n+1}, the decayed state MMA5a / MMA5b of chunk n+1
@@ -1063,7 +1141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    if (__syncthreads_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
+    if (worker_sync_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
   }
 
   if (!aborted) {
@@ -1092,12 +1170,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_inflight = (int)ph_load;
     }
     if (load_inflight >= 0) mbar_wait(bar_load, (uint32_t)load_inflight, kDrainLimit, p.status);
-    if (mma_inflight >= 0) mbar_wait(bar_mma, (uint32_t)mma_inflight, kDrainLimit, p.status);
     if (pre_inflight >= 0) mbar_wait(bar_pre, (uint32_t)pre_inflight, kDrainLimit, p.status);
-    mma_commit(bar_drain);  // also covers MMAs issued after the last commit observed
-    mbar_wait(bar_drain, 0u, kDrainLimit, p.status);
   }
   if (tid == 0) bulk_wait_all();
+  }  // workers
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1192,7 +1268,7 @@ cudaError_t launch_dm(const ScanParams& p, cudaStream_t stream) {
            static_cast<const __nv_bfloat16*>(p.u), static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha,
            static_cast<const __nv_bfloat16*>(p.gain), p.conv_w, p.S0, p.lengths,
            static_cast<__nv_bfloat16*>(p.o), p.S_final, p.B, p.T, p.H, p.W, NC, p.status, p.spin_limit};
-  prism_chunk_tc_kernel<D, M, CH><<<p.B * p.H, kThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, mo, mt, a);
+  prism_chunk_tc_kernel<D, M, CH><<<p.B * p.H, kCtaThreads, Ly::SMEM_ALLOC, stream>>>(mq, mk, mu, mv, mg, mo, mt, a);
   return cudaGetLastError();
 }
 
