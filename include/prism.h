@@ -146,6 +146,39 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v,
 size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L,
                                      int W, int chunk, int dtype);
 
+/*
+ * prism_scan_bwd - gradients of the scan (the training pass): for the cotangents dO of o
+ * and (optionally) dS_final of S_final, the gradients of L = <o, dO> + <S_final, dS_final>
+ * with respect to every input of prism_scan_fwd_ex with the same arguments.  Reverse-mode
+ * differentiation of the recurrence defined above (ICML 2026 PRISM write-up, 核心迭代形式 /
+ * 架构形式; PRISM explainer 2.1-2.2).
+ *
+ * Inputs: as prism_scan_fwd_ex (q, k, v, gamma, beta, u, alpha, gain, conv_w, S0, lengths,
+ *   chain), plus dO [B,T,H,d_v] (dtype) and dS_final [B,H,d_v,d_k] fp32 or NULL (zero).
+ * Outputs (fp32, device, caller-owned, same shapes as the inputs): dq, dk [B,T,H,d_k];
+ *   dv [B,T,H,d_v]; dgamma, dbeta [B,T,H]; du [B,T,H,L-1,d_k], dalpha [B,T,H,L-1],
+ *   dgain [B,T,H,L-1,d_v] (all three NULL iff L == 1); dconv_w [H,d_v,W]; dS0 [B,H,d_v,d_k]
+ *   (the gradient with respect to the initial state, zeros or S0).  Padded steps get zero
+ *   gradients.
+ * workspace: prism_scan_bwd_workspace_size() bytes: every state S_t of the forward
+ *   (B*H*T*d_v*d_k fp32, recorded by a token-by-token forward launch) and per-(b, h)
+ *   partial sums of dconv_w.  Results are deterministic.
+ * Sizes as prism_scan_fwd; additionally (L + 1) * d_k * d_v * (d_k == 16 ? 4 : 8) / 8 bytes
+ * of per-token reduction space must fit in 227 KB (d = 128: L <= 13), else
+ * PRISM_ERR_UNSUPPORTED.  Three launches on `stream`; no synchronisation.
+ */
+size_t prism_scan_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int dtype);
+
+int prism_scan_bwd(const void* q, const void* k, const void* v,
+                   const float* gamma, const float* beta,
+                   const void* u, const float* alpha, const void* gain,
+                   const float* conv_w, const float* S0, const int32_t* lengths,
+                   const void* dO, const float* dS_final,
+                   int B, int T, int H, int d_k, int d_v, int L, int W, int dtype, int chain,
+                   float* dq, float* dk, float* dv, float* dgamma, float* dbeta,
+                   float* du, float* dalpha, float* dgain, float* dconv_w, float* dS0,
+                   void* workspace, size_t workspace_bytes, prism_stream_t stream);
+
 /* Size of the device-global scratch behind prism_scan_fwd_static. */
 #define PRISM_STATIC_WORKSPACE_BYTES (32u << 20)
 

@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     lib,
     decode_step,
     prologue_fwd,
+    scan_bwd,
     scan_fwd,
     scan_fwd_host,
     scan_fwd_static,

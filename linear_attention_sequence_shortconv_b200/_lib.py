@@ -39,6 +39,8 @@ EXPORTS = (
     "prism_prologue_fwd",
     "prism_prologue_fwd_ex",
     "prism_decode_step",
+    "prism_scan_bwd",
+    "prism_scan_bwd_workspace_size",
     "prism_scan_fwd_uses_tensor_cores",
     "prism_stream_status",
     "prism_set_spin_limit",
@@ -86,6 +88,10 @@ def lib() -> ctypes.CDLL:
     L.prism_prologue_fwd_ex.restype = ci
     L.prism_decode_step.argtypes = [vp] * 11 + [ci] * 8 + [vp, vp]
     L.prism_decode_step.restype = ci
+    L.prism_scan_bwd_workspace_size.argtypes = [ci] * 8
+    L.prism_scan_bwd_workspace_size.restype = cs
+    L.prism_scan_bwd.argtypes = [vp] * 13 + [ci] * 9 + [vp] * 11 + [cs, vp]
+    L.prism_scan_bwd.restype = ci
     L.prism_scan_fwd_uses_tensor_cores.argtypes = [ci] * 6
     L.prism_scan_fwd_uses_tensor_cores.restype = ci
     L.prism_stream_status.argtypes = [vp]
@@ -312,6 +318,51 @@ def decode_step(q, k, v, gamma, beta, u, alpha, gain, conv_w, conv_state, S, L: 
     if rc != 0:
         raise PrismError(rc, "prism_decode_step")
     return o
+
+
+def scan_bwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, dO, L: int, S0=None, lengths=None, dS_final=None,
+             workspace=None, stream=None, chain: str = "linear"):
+    """Gradients of <o, dO> + <S_final, dS_final> on CUDA tensors (fp32); returns a dict
+    with keys q, k, v, gamma, beta, conv_w, S0 and (L > 1) u, alpha, gain."""
+    chain_code = _chain_code(chain)
+    dt = q.dtype
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v), ("dO", dO)):
+        _check(t, name, dt)
+    for name, t in (("gamma", gamma), ("beta", beta), ("conv_w", conv_w)):
+        _check(t, name, torch.float32)
+    if L > 1:
+        _check(u, "u", dt)
+        _check(gain, "gain", dt)
+        _check(alpha, "alpha", torch.float32)
+    _check(S0, "S0", torch.float32, required=False)
+    _check(dS_final, "dS_final", torch.float32, required=False)
+    _check(lengths, "lengths", torch.int32, required=False)
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    W = conv_w.shape[-1]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"q": torch.empty(q.shape, **f32), "k": torch.empty(k.shape, **f32), "v": torch.empty(v.shape, **f32),
+         "gamma": torch.empty(gamma.shape, **f32), "beta": torch.empty(beta.shape, **f32),
+         "conv_w": torch.empty(conv_w.shape, **f32), "S0": torch.empty((B, H, d_v, d_k), **f32)}
+    if L > 1:
+        g["u"] = torch.empty(u.shape, **f32)
+        g["alpha"] = torch.empty(alpha.shape, **f32)
+        g["gain"] = torch.empty(gain.shape, **f32)
+    ws_bytes = int(lib().prism_scan_bwd_workspace_size(B, T, H, d_k, d_v, L, W, code))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    rc = lib().prism_scan_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+        _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
+        _ptr(conv_w), _ptr(S0), _ptr(lengths), _ptr(dO), _ptr(dS_final),
+        B, T, H, d_k, d_v, L, W, code, chain_code,
+        _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["gamma"]), _ptr(g["beta"]),
+        _ptr(g.get("u")), _ptr(g.get("alpha")), _ptr(g.get("gain")), _ptr(g["conv_w"]), _ptr(g["S0"]),
+        _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    if rc != 0:
+        raise PrismError(rc, "prism_scan_bwd")
+    return g
 
 
 def uses_tensor_cores(d_k, d_v, L, W, chunk, dtype_code) -> bool:

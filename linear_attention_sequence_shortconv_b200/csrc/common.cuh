@@ -29,6 +29,8 @@ struct ScanParams {
   long long spin_limit;   // bound of every device-side wait
   int chain;              // PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU
   void* workspace;        // prism_scan_fwd_workspace_size() bytes (NULL when that is 0)
+  float* states;          // token-by-token path only: S_t after every valid token,
+                          // [B, H, T, d_v, d_k] fp32 (NULL: not recorded)
 };
 
 // Pointers and sizes of one prism_decode_step call (device pointers).
@@ -46,6 +48,36 @@ struct DecodeParams {
   float* S;
   void* o;
   int B, H, d_k, d_v, L, W, chain;
+};
+
+// Pointers and sizes of one prism_scan_bwd call (device pointers).
+struct BwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* gamma;
+  const float* beta;
+  const void* u;
+  const float* alpha;
+  const void* gain;
+  const float* conv_w;
+  const float* S0;
+  const int32_t* lengths;
+  const void* dO;
+  const float* dS_final;
+  const float* states;  // [B, H, T, d_v, d_k]: S_t after every valid token
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dgamma;
+  float* dbeta;
+  float* du;
+  float* dalpha;
+  float* dgain;
+  float* dconv_part;  // [B, H, d_v, W] (workspace)
+  float* dconv_w;     // [H, d_v, W]
+  float* dS0;
+  int B, T, H, d_k, d_v, L, W, chain;
 };
 
 // One step of the residual chain.  Exact form (gist.science PRISM explainer, 2.2

@@ -14,6 +14,8 @@ bool chunk_tc_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
 cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream);
 size_t chunk_tc_workspace_bytes(int B, int T, int H);
 cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t stream);
+cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, cudaStream_t stream);
+size_t bwd_smem_bytes(int d_k, int d_v, int L);
 }  // namespace prism
 
 namespace {
@@ -293,6 +295,61 @@ int prism_decode_step(const void* q, const void* k, const void* v, const float* 
   prism::DecodeParams p{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr,
                         conv_w, W > 1 ? conv_state : nullptr, S, o, B, H, d_k, d_v, L, W, chain};
   cudaError_t err = prism::launch_decode_step(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+size_t prism_scan_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int dtype) {
+  if (check_sizes(B, T, H, d_k, d_v, L, W, 16, dtype) != PRISM_OK) return 0;
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return al((size_t)B * H * T * d_v * d_k * 4) + al((size_t)B * H * d_v * W * 4);
+}
+
+int prism_scan_bwd(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
+                   const void* u, const float* alpha, const void* gain, const float* conv_w, const float* S0,
+                   const int32_t* lengths, const void* dO, const float* dS_final, int B, int T, int H, int d_k,
+                   int d_v, int L, int W, int dtype, int chain, float* dq, float* dk, float* dv, float* dgamma,
+                   float* dbeta, float* du, float* dalpha, float* dgain, float* dconv_w, float* dS0,
+                   void* workspace, size_t workspace_bytes, prism_stream_t stream) {
+  if (chain != PRISM_CHAIN_LINEAR && chain != PRISM_CHAIN_GELU) return PRISM_ERR_INVALID_ARG;
+  int rc = check_sizes(B, T, H, d_k, d_v, L, W, 16, dtype);
+  if (rc != PRISM_OK) return rc;
+  if (!q || !k || !v || !gamma || !beta || !conv_w || !dO) return PRISM_ERR_INVALID_ARG;
+  if (!dq || !dk || !dv || !dgamma || !dbeta || !dconv_w || !dS0) return PRISM_ERR_INVALID_ARG;
+  if (L > 1 && (!u || !alpha || !gain || !du || !dalpha || !dgain)) return PRISM_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, gamma, beta, conv_w, S0, lengths, dO, dS_final, dq, dk, dv, dgamma, dbeta,
+                        dconv_w, dS0, workspace, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr,
+                        L > 1 ? gain : nullptr, L > 1 ? du : nullptr, L > 1 ? dalpha : nullptr,
+                        L > 1 ? dgain : nullptr};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return PRISM_ERR_UNSUPPORTED;
+  if (prism::bwd_smem_bytes(d_k, d_v, L) > 227u * 1024u) return PRISM_ERR_UNSUPPORTED;
+  const size_t need = prism_scan_bwd_workspace_size(B, T, H, d_k, d_v, L, W, dtype);
+  if (!workspace || workspace_bytes < need) return PRISM_ERR_WORKSPACE;
+  int* status = nullptr;
+  rc = device_setup(&status);
+  if (rc != PRISM_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t toks = (size_t)B * T * H, m = (size_t)(L - 1);
+  // gradients of padded steps stay zero
+  struct Z { void* p; size_t bytes; };
+  const Z zs[] = {{dq, toks * d_k * 4}, {dk, toks * d_k * 4}, {dv, toks * d_v * 4}, {dgamma, toks * 4},
+                  {dbeta, toks * 4}, {du, toks * m * d_k * 4}, {dalpha, toks * m * 4}, {dgain, toks * m * d_v * 4}};
+  for (const Z& z : zs)
+    if (z.p && z.bytes && cudaMemsetAsync(z.p, 0, z.bytes, s) != cudaSuccess) return PRISM_ERR_CUDA;
+  float* states = static_cast<float*>(workspace);
+  float* dconv_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                               (((size_t)B * H * T * d_v * d_k * 4 + 255) & ~(size_t)255));
+  // forward that records S_t after every valid token (no outputs)
+  prism::ScanParams fp{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr,
+                       conv_w, S0, lengths, nullptr, nullptr, B, T, H, d_k, d_v, L, W, 16, status,
+                       g_spin_limit.load(), chain, nullptr, states};
+  cudaError_t err = prism::launch_recurrent_scan(fp, dtype, s);
+  if (err != cudaSuccess) return PRISM_ERR_CUDA;
+  prism::BwdParams bp{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr,
+                      conv_w, S0, lengths, dO, dS_final, states, dq, dk, dv, dgamma, dbeta,
+                      L > 1 ? du : nullptr, L > 1 ? dalpha : nullptr, L > 1 ? dgain : nullptr, dconv_part, dconv_w,
+                      dS0, B, T, H, d_k, d_v, L, W, chain};
+  err = prism::launch_scan_bwd(bp, dtype, s);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 

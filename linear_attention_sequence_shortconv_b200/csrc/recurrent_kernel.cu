@@ -254,6 +254,12 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
           s[e + 3] += rho * f.w;
         }
       }
+      if (p.states && row_ok) {  // S_t of this row, for the backward pass
+        float* dst = p.states + ((((size_t)b * H + h) * T_ + t0 + i) * dv + c) * dk + EPL * j;
+#pragma unroll
+        for (int e = 0; e < EPL; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+      }
       const T* qq = sq_ + i * dk + EPL * j;
       float oq = 0.f;
 #pragma unroll
@@ -262,12 +268,12 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
         oq += s[e] * f.x + s[e + 1] * f.y + s[e + 2] * f.z + s[e + 3] * f.w;
       }
       oq = row_sum<LPR>(oq);
-      if (row_ok && j == 0) st1<T>(o + (((size_t)b * T_ + t0 + i) * H + h) * dv + c, oq);
+      if (o && row_ok && j == 0) st1<T>(o + (((size_t)b * T_ + t0 + i) * H + h) * dv + c, oq);
     }
     __syncthreads();  // the buffer is refilled next iteration
   }
   cp_async_wait_0();
-  if (row_ok && j == 0)
+  if (o && row_ok && j == 0)
     for (int t = len; t < T_; ++t) st1<T>(o + (((size_t)b * T_ + t) * H + h) * dv + c, 0.f);
   if (row_ok && p.S_final) {
 #pragma unroll

@@ -1,0 +1,82 @@
+"""Gradients of the scan on the GPU (prism_scan_bwd, through the C ABI) against the
+oracle's autograd gradients (oracle/prism_grad.py) on the same, already rounded
+inputs.  fp32 arithmetic on both the fp32 and the bf16 inputs, so one bar: 2e-4
+max-abs-relative per gradient tensor.
+"""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_sequence_shortconv_b200 import synth
+from oracle.prism_grad import prism_seq_grad
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-4
+
+CASES = {
+    "fp32_d32_L3": (synth.Workload("a", B=2, T=37, H=2, d_k=32, d_v=32, L=3, chunk=16, W=4, dtype="fp32",
+                                   lengths_lo=20, with_s0=True), "linear"),
+    "fp32_d16_L4_gelu": (synth.Workload("b", B=1, T=25, H=2, d_k=16, d_v=16, L=4, chunk=16, W=2, dtype="fp32",
+                                        with_s0=True), "gelu"),
+    "bf16_d128_L4": (synth.Workload("c", B=1, T=70, H=2, d_k=128, d_v=128, L=4, chunk=64, W=4, with_s0=True),
+                     "linear"),
+    "fp32_d64_L1": (synth.Workload("d", B=2, T=40, H=1, d_k=64, d_v=64, L=1, chunk=16, W=4, dtype="fp32"), "linear"),
+    "fp32_dk64_dv32_W1": (synth.Workload("e", B=1, T=30, H=3, d_k=64, d_v=32, L=2, chunk=16, W=1, dtype="fp32"),
+                          "linear"),
+}
+
+
+def _run(w, chain, seed=5):
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    inp = synth.make_inputs(w)
+    if chain == "gelu":
+        gg = torch.Generator().manual_seed(w.seed + 101)
+        inp["gain"] = (1.5 * torch.randn(inp["gain"].shape, generator=gg)).to(inp["gain"].dtype)
+    gen = torch.Generator().manual_seed(seed)
+    dO = torch.randn((w.B, w.T, w.H, w.d_v), generator=gen).to(inp["v"].dtype)
+    dSf = torch.randn((w.B, w.H, w.d_v, w.d_k), generator=gen)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    g = prism.scan_bwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"], d["conv_w"],
+                       dO.cuda(), L=w.L, S0=d["S0"], lengths=d["lengths"], dS_final=dSf.cuda(), chain=chain)
+    torch.cuda.synchronize()
+    return inp, dO, dSf, {n: t.cpu().numpy().astype(np.float64) for n, t in g.items()}
+
+
+def _rel(x, ref):
+    return float(np.abs(x - ref).max() / max(np.abs(ref).max(), 1e-6))
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_matches_oracle(name):
+    w, chain = CASES[name]
+    inp, dO, dSf, got = _run(w, chain)
+    x = synth.to_float64_numpy(inp)
+    if w.L == 1:
+        x["u"] = x["alpha"] = x["gain"] = None
+    ref = prism_seq_grad(**x, dO=dO.double().numpy(), dS_final=dSf.double().numpy(), chain=chain)
+    for n, r in ref.items():
+        assert n in got, n
+        assert got[n].shape == r.shape, (n, got[n].shape, r.shape)
+        assert _rel(got[n], r) <= TOL, (name, n, _rel(got[n], r))
+
+
+def test_backward_is_deterministic():
+    w, chain = CASES["bf16_d128_L4"]
+    _, _, _, g1 = _run(w, chain)
+    _, _, _, g2 = _run(w, chain)
+    for n in g1:
+        assert np.array_equal(g1[n], g2[n]), n
+
+
+def test_backward_rejects_what_it_cannot_hold():
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    w = synth.Workload("big", B=1, T=8, H=1, d_k=128, d_v=128, L=16, chunk=64, W=4)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in synth.make_inputs(w).items()}
+    dO = torch.zeros((1, 8, 1, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(prism.PrismError) as e:
+        prism.scan_bwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"], d["conv_w"],
+                       dO, L=w.L)
+    assert e.value.code == 2  # PRISM_ERR_UNSUPPORTED: per-token reduction space above 227 KB
