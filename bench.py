@@ -62,6 +62,21 @@ def algorithmic_work(w, lengths=None):
             "bytes": token_heads * per_th + state, "flops": token_heads * flops_th}
 
 
+def algorithmic_work_bwd(w, lengths=None):
+    """Algorithmic bytes of one backward pass over workload ``w``: the forward's
+    inputs and dO read once (as the forward's bytes with dO in place of o), the
+    gradients written once in fp32 (dq, dk, dv, dgamma, dbeta, du, dalpha, dgain per
+    token-head; dS0 per sequence-head; dS_final read per sequence-head)."""
+    es = 2 if w.dtype == "bf16" else 4
+    m = w.m
+    valid_tokens = int(lengths.sum()) if lengths is not None else w.B * w.T
+    token_heads = valid_tokens * w.H
+    reads = es * (2 * w.d_k + 2 * w.d_v) + es * m * (w.d_k + w.d_v) + 4 * (2 + m)
+    writes = 4 * (2 * w.d_k + w.d_v) + 4 * m * (w.d_k + w.d_v) + 4 * (2 + m)
+    state = w.B * w.H * w.d_v * w.d_k * 4 * (3 if w.with_s0 else 2)
+    return {"tokens": valid_tokens, "token_heads": token_heads, "bytes": token_heads * (reads + writes) + state}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -234,6 +249,84 @@ def workload_config(w, n):
 
 
 # ---------------------------------------------------------------- our arm
+def run_ours_bwd(args, w):
+    """The training pass: prism_scan_bwd (gradients of every input) on workload ``w``."""
+    import numpy as np
+    import torch
+
+    import linear_attention_sequence_shortconv_b200 as prism
+    from linear_attention_sequence_shortconv_b200 import synth
+
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("--pass bwd runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    host_inputs = synth.make_inputs(w)
+    d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in host_inputs.items()}
+    gen = torch.Generator().manual_seed(w.seed + 7)
+    io_dtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dO = torch.randn((w.B, w.T, w.H, w.d_v), generator=gen).to(io_dtype).to(dev)
+    dSf = torch.randn((w.B, w.H, w.d_v, w.d_k), generator=gen).to(dev)
+    code = prism.PRISM_BF16 if w.dtype == "bf16" else prism.PRISM_FP32
+    ws = torch.empty(int(prism.lib().prism_scan_bwd_workspace_size(w.B, w.T, w.H, w.d_k, w.d_v, w.L, w.W, code)),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return prism.scan_bwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"],
+                              d["conv_w"], dO, L=w.L, S0=d["S0"], lengths=d["lengths"], dS_final=dSf,
+                              workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if prism.stream_status() != 0:
+        raise SystemExit("device status word reports an error after warm-up")
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clocks:
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    work = algorithmic_work_bwd(w, host_inputs["lengths"].numpy() if host_inputs["lengths"] is not None else None)
+    peaks, peak_kind = load_peaks()
+    achieved = work["bytes"] / (ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "scan_bwd",
+                "timed": "step = recording forward + reverse kernel + dconv reduction",
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS hbm_gbs burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": work["bytes"]}
+    cpu_baseline = None
+    if not args.no_cpu_baseline:
+        from oracle.prism_grad import prism_seq_grad
+
+        tokens = min(w.T, 128)
+        sample = w.replace(B=1, T=tokens, lengths_lo=None)
+        xs = synth.to_float64_numpy(synth.make_inputs(sample))
+        if w.L == 1:
+            xs["u"] = xs["alpha"] = xs["gain"] = None
+        t0 = time.perf_counter()
+        prism_seq_grad(**xs, dO=np.ones((1, tokens, w.H, w.d_v)), dS_final=None)
+        sec = time.perf_counter() - t0
+        cpu_baseline = {"value": tokens / sec, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+                        "sample": f"autograd of the first {tokens} steps of 1 batch row x {w.H} heads of {w.name}",
+                        "seconds": sec}
+    line = {"metric": "PRISM scan bwd (all input gradients) tokens/s on 1 B200", "value": work["tokens"] / (ms / 1e3),
+            "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded)",
+            "config": workload_config(w, 1), "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": None,
+            "gpu_launches": 3 * K, "clocks": clocks.summary(), "impl": "ours", "pass": "bwd"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -382,6 +475,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=("fwd", "bwd"), default="fwd",
+                    help="fwd: the scan (the headline); bwd: prism_scan_bwd, one GPU")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -392,6 +487,8 @@ def main():
         w = w.replace(B=args.batch, name=f"{w.name}_b{args.batch}")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.pass_ == "bwd":
+        return run_ours_bwd(args, w)
     return run_ours(args, w)
 
 
