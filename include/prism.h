@@ -161,11 +161,13 @@ size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int 
  *   (the gradient with respect to the initial state, zeros or S0).  Padded steps get zero
  *   gradients.
  * workspace: prism_scan_bwd_workspace_size() bytes: every state S_t of the forward
- *   (B*H*T*d_v*d_k fp32, recorded by a token-by-token forward launch) and per-(b, h)
- *   partial sums of dconv_w.  Results are deterministic.
- * Sizes as prism_scan_fwd; additionally (L + 1) * d_k * d_v * (d_k == 16 ? 4 : 8) / 8 bytes
- * of per-token reduction space must fit in 227 KB (d = 128: L <= 13), else
- * PRISM_ERR_UNSUPPORTED.  Three launches on `stream`; no synchronisation.
+ *   (B*H*T*d_v*d_k fp32, recorded by a token-by-token forward launch) and partial sums.
+ *   Results are deterministic.
+ * workspace also holds per-token sums over row blocks (of 32 rows; 64 for d_k = 16) of the
+ * gradients that are sums over rows (dq, dk, du, dgamma, dbeta, dalpha).
+ * Sizes as prism_scan_fwd.  Four launches on `stream` (recording forward, reverse
+ * recurrence, two deterministic reductions) after memsets of the outputs; no
+ * synchronisation.
  */
 size_t prism_scan_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int dtype);
 

@@ -75,6 +75,7 @@ struct BwdParams {
   float* dalpha;
   float* dgain;
   float* dconv_part;  // [B, H, d_v, W] (workspace)
+  float* part;        // [B*T*H, row blocks, NV] per-token partial sums over a block's rows (workspace)
   float* dconv_w;     // [H, d_v, W]
   float* dS0;
   int B, T, H, d_k, d_v, L, W, chain;

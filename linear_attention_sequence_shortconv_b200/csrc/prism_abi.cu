@@ -16,6 +16,7 @@ size_t chunk_tc_workspace_bytes(int B, int T, int H);
 cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, cudaStream_t stream);
 size_t bwd_smem_bytes(int d_k, int d_v, int L);
+int bwd_row_blocks(int d_k, int d_v);
 }  // namespace prism
 
 namespace {
@@ -301,7 +302,9 @@ int prism_decode_step(const void* q, const void* k, const void* v, const float* 
 size_t prism_scan_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int dtype) {
   if (check_sizes(B, T, H, d_k, d_v, L, W, 16, dtype) != PRISM_OK) return 0;
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return al((size_t)B * H * T * d_v * d_k * 4) + al((size_t)B * H * d_v * W * 4);
+  const size_t nv = (size_t)(L + 1) * d_k + (L + 1);
+  return al((size_t)B * H * T * d_v * d_k * 4) + al((size_t)B * H * d_v * W * 4) +
+         al((size_t)B * T * H * prism::bwd_row_blocks(d_k, d_v) * nv * 4);
 }
 
 int prism_scan_bwd(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
@@ -337,8 +340,12 @@ int prism_scan_bwd(const void* q, const void* k, const void* v, const float* gam
   for (const Z& z : zs)
     if (z.p && z.bytes && cudaMemsetAsync(z.p, 0, z.bytes, s) != cudaSuccess) return PRISM_ERR_CUDA;
   float* states = static_cast<float*>(workspace);
-  float* dconv_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                               (((size_t)B * H * T * d_v * d_k * 4 + 255) & ~(size_t)255));
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* wsb = static_cast<char*>(workspace);
+  const size_t off_conv = al((size_t)B * H * T * d_v * d_k * 4);
+  const size_t off_part = off_conv + al((size_t)B * H * d_v * W * 4);
+  float* dconv_part = reinterpret_cast<float*>(wsb + off_conv);
+  float* part = reinterpret_cast<float*>(wsb + off_part);
   // forward that records S_t after every valid token (no outputs)
   prism::ScanParams fp{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr,
                        conv_w, S0, lengths, nullptr, nullptr, B, T, H, d_k, d_v, L, W, 16, status,
@@ -347,8 +354,8 @@ int prism_scan_bwd(const void* q, const void* k, const void* v, const float* gam
   if (err != cudaSuccess) return PRISM_ERR_CUDA;
   prism::BwdParams bp{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr,
                       conv_w, S0, lengths, dO, dS_final, states, dq, dk, dv, dgamma, dbeta,
-                      L > 1 ? du : nullptr, L > 1 ? dalpha : nullptr, L > 1 ? dgain : nullptr, dconv_part, dconv_w,
-                      dS0, B, T, H, d_k, d_v, L, W, chain};
+                      L > 1 ? du : nullptr, L > 1 ? dalpha : nullptr, L > 1 ? dgain : nullptr, dconv_part, part,
+                      dconv_w, dS0, B, T, H, d_k, d_v, L, W, chain};
   err = prism::launch_scan_bwd(bp, dtype, s);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }

@@ -70,13 +70,11 @@ def test_backward_is_deterministic():
         assert np.array_equal(g1[n], g2[n]), n
 
 
-def test_backward_rejects_what_it_cannot_hold():
-    import linear_attention_sequence_shortconv_b200 as prism
-
-    w = synth.Workload("big", B=1, T=8, H=1, d_k=128, d_v=128, L=16, chunk=64, W=4)
-    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in synth.make_inputs(w).items()}
-    dO = torch.zeros((1, 8, 1, 128), dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(prism.PrismError) as e:
-        prism.scan_bwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"], d["conv_w"],
-                       dO, L=w.L)
-    assert e.value.code == 2  # PRISM_ERR_UNSUPPORTED: per-token reduction space above 227 KB
+def test_backward_long_chain_full_width():
+    """L = 16 (fifteen residual directions) at d = 128: the largest per-token reduction."""
+    w = synth.Workload("long_chain", B=1, T=12, H=1, d_k=128, d_v=128, L=16, chunk=64, W=4, with_s0=True)
+    inp, dO, dSf, got = _run(w, "linear")
+    x = synth.to_float64_numpy(inp)
+    ref = prism_seq_grad(**x, dO=dO.double().numpy(), dS_final=dSf.double().numpy())
+    for n, r in ref.items():
+        assert _rel(got[n], r) <= TOL, (n, _rel(got[n], r))
