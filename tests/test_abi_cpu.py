@@ -140,3 +140,29 @@ def test_decode_optional_inputs(L):
     # W = 1 needs no history and L = 1 no residual inputs: with those NULL the only
     # error left is the size error planted here.
     assert decode_call(L, W=1, conv_state=None, L=1, u=None, alpha=None, gain=None, B=0) == 1
+
+
+def bwd_call(lib_, ws_ok=True, **kw):
+    a = dict(B=2, T=8, H=2, d_k=64, d_v=64, L=4, W=4, dtype=0, chain=0, q=FAKE, dO=FAKE, dq=FAKE, du=FAKE)
+    a.update(kw)
+    ws, wsb = (FAKE, 1 << 40) if ws_ok else (None, 0)
+    return lib_.prism_scan_bwd(a["q"], FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, a["dO"], None,
+                               a["B"], a["T"], a["H"], a["d_k"], a["d_v"], a["L"], a["W"], a["dtype"], a["chain"],
+                               a["dq"], FAKE, FAKE, FAKE, FAKE, a["du"], FAKE, FAKE, FAKE, FAKE, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), 1), (dict(L=0), 1), (dict(chain=3), 1), (dict(dtype=5), 1), (dict(dO=None), 1), (dict(dq=None), 1),
+    (dict(du=None), 1), (dict(d_k=48), 2), (dict(L=17), 2), (dict(q=FAKE + 4), 2), (dict(ws_ok=False), 3),
+])
+def test_backward_invalid_arguments(L, kw, code):
+    assert bwd_call(L, **kw) == code
+
+
+def test_backward_workspace_size(L):
+    # every state S_t (fp32) + dconv_w partials + per-token row-block sums, each 256-byte aligned
+    B, T, H, d, Lc, W = 2, 10, 3, 64, 4, 4
+    al = lambda x: (x + 255) // 256 * 256
+    nv = (Lc + 1) * d + (Lc + 1)
+    expect = al(B * H * T * d * d * 4) + al(B * H * d * W * 4) + al(B * T * H * 2 * nv * 4)
+    assert prism.lib().prism_scan_bwd_workspace_size(B, T, H, d, d, Lc, W, 0) == expect
