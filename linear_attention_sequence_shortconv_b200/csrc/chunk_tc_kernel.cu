@@ -734,7 +734,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
           mma_bf16(tmem + D3, kdesc(aS, kk, kAtom), kdesc(aKQ, kk, kAtom), idesc_bf16(128, 128, 0, 0), kk > 0);
       }
       __syncwarp();
-      // MMA2: (Bku P)^T | (QU P)^T -> R1; MMA5a: P~^T U or P^T (diag(c) U) onto RS; [T;QK] x T
+      // MMA2: (Bku P)^T | (QU P)^T -> R1 and [T;QK] x T, committed for step E; then MMA5a:
+      // P~^T U or P^T (diag(c) U) onto RS, which only the state pass needs (covered by the
+      // commit after MMA4)
       ok = mma_warp_wait(go_B, pB, lim, p.status, abort_flag);
       pB ^= 1;
       if (!ok) break;
@@ -745,16 +747,18 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
           for (int kk = 0; kk < UR / 16; ++kk)
             mma_bf16(tmem + R1, mndesc(aP, kk, Ly::U_ATOM), kdesc(aBQ, kk, kAtom), idesc_bf16(128, 128, 1, 0),
                      kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < UR / 16; ++kk)
-            mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1),
-                     1);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + R1 + 128, kdesc(aTQ, kk, kAtom), mndesc(aTQ, kk, kAtom), idesc_bf16(128, 64, 0, 1),
                    kk > 0);
         mma_commit(bar_mma);
+        if (M > 0) {
+#pragma unroll
+          for (int kk = 0; kk < UR / 16; ++kk)
+            mma_bf16(tmem + RS, mndesc(aP, kk, Ly::U_ATOM), mndesc(aU, kk, Ly::U_ATOM), idesc_bf16(128, D, 1, 1),
+                     1);
+        }
       }
       __syncwarp();
       // MMA4: X^T x [T;QKT]^T -> Delta^T | (QKT X)^T in R1+128
@@ -998,11 +1002,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) {
-      if (n + 1 < nchunks) {  // MMA3, MMA2 and MMA5a, the last readers of Q, P, U and [Bku;QU], are done
-        load_q(t0 + kC);
-        load_u(t0 + kC);
-        if (M > 0) load_pre(n + 1);
-      }
+      if (n + 1 < nchunks) load_q(t0 + kC);  // MMA1 and MMA3, the readers of Q, are done
     }
     if (n + 1 < nchunks) load_alpha(n + 1, al_next);
     if (!ok && lane == 0) atomicExch(s_abort, 1);
@@ -1047,7 +1047,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) {
-      if (n + 1 < nchunks) load_t(n + 1);              // MMA4, the last reader of TQ, has completed
+      if (n + 1 < nchunks) {  // MMA4 (last reader of TQ) and MMA5a (last of P, U) have completed
+        load_t(n + 1);
+        load_u(t0 + kC);
+        if (M > 0) load_pre(n + 1);
+      }
     }
     if (!ok && lane == 0) atomicExch(s_abort, 1);
     tc_fence_after();
