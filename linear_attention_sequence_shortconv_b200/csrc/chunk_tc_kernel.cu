@@ -309,7 +309,7 @@ struct PrepLayout {
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_A = NA * kPrepAtom;             // [64][kPrepLDA] fp32
   static constexpr uint32_t OFF_Y = OFF_A + 64 * kPrepLDA * 4;  // 1024 fp32 inverse scratch
-  static constexpr uint32_t OFF_SMALL = OFF_Y + 4096;           // G, beta [64] each; barriers
+  static constexpr uint32_t OFF_SMALL = OFF_Y + 4096;           // G, beta, e^{-G} [64] each; barriers
   static constexpr uint32_t BYTES = OFF_SMALL + 1024;
   static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;  // + alignment slack
 };
@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(kPrepThreads) prism_chunk_prep_kernel(const __
   float* sY = reinterpret_cast<float*>(sm + Ly::OFF_Y);
   float* sG = reinterpret_cast<float*>(sm + Ly::OFF_SMALL);
   float* sBeta = sG + 64;
+  float* sEn = sG + 192;  // e^{-G_i} (chunks with log-decay >= -60)
   uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + Ly::OFF_SMALL + 512);
   uint64_t* bar_mma = bar_load + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_load + 2);
@@ -373,6 +374,10 @@ __global__ void __launch_bounds__(kPrepThreads) prism_chunk_prep_kernel(const __
     sG[2 * lane + 1] = x;
     sBeta[2 * lane] = bl[0];
     sBeta[2 * lane + 1] = bl[1];
+    if (__shfl_sync(0xffffffffu, x, 31) >= -60.f) {  // e^{-G} stays finite: factor the decays
+      sEn[2 * lane] = __expf(lg1 - x);
+      sEn[2 * lane + 1] = __expf(-x);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -400,15 +405,25 @@ __global__ void __launch_bounds__(kPrepThreads) prism_chunk_prep_kernel(const __
       tc_fence_after();
       const int t = 32 * warp + lane;
       const float Gt = sG[t], bt = sBeta[t];
+      const bool fast = sG[63] >= -60.f;  // as decided where sEn was written
+      const float rs = fast ? bt * __expf(Gt) : 0.f;
       const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
       for (int pc = 0; pc < 4; ++pc) {
         float x[16];
         tmem_ld16(tl + 16 * pc, x);
+        if (fast) {  // e^{G_t - G_i} = e^{G_t} e^{-G_i}
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i = 16 * pc + e;
-          x[e] = (i < t) ? bt * __expf(Gt - sG[i]) * x[e] : 0.f;
+          for (int e = 0; e < 16; ++e) {
+            const int i = 16 * pc + e;
+            x[e] = (i < t) ? rs * sEn[i] * x[e] : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int i = 16 * pc + e;
+            x[e] = (i < t) ? bt * __expf(Gt - sG[i]) * x[e] : 0.f;
+          }
         }
         float4* dst = reinterpret_cast<float4*>(sA + t * LDA + 16 * pc);
 #pragma unroll
