@@ -842,6 +842,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     gate_load(0, gl);
     gate_scan(gl, 0);
   }
+  // warp 2 holds the gates of the chunk after the current one in registers, requested a
+  // whole chunk before its scan (step C) needs them
+  float gl_next[4] = {1.f, 1.f, 0.f, 0.f};
+  if (warp == 2 && nchunks > 1) gate_load(1, gl_next);
   if (M > 0 && tap_thread) taps0[(tid % p.W) * D + tid / p.W] = __ldg(cw_head + tid);
   worker_sync();
   if (srow) {  // RS <- exp(G_63 of chunk 0) S0 (undecayed S0 when there is no chunk: S_final)
@@ -886,21 +890,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     const float* Bt = sBeta + cur * 64;
 
     // ---------------- A: MMA3 (S_n x [K;Q]^T; MMA1 was issued at the end of the previous chunk);
-    // per-chunk decay tables; L2 prefetch of the next chunk's gate lines
+    // per-chunk decay tables
     if (tid == 0) mbar_arrive(go_A);  // S_n (bf16) is in SXA: MMA3
-    if (warp == 1 && n + 1 < nchunks) {
-      // the next chunk's gates are token-major spans [b, t0+64 .. t0+128, :]: prefetch their L2 lines
-      const int tn = t0 + kC, te = min(tn + kC, T);
-      const char* g0 = reinterpret_cast<const char*>(p.gamma + ((size_t)b * T + tn) * H);
-      const char* b0 = reinterpret_cast<const char*>(p.beta + ((size_t)b * T + tn) * H);
-      const char* a0 = reinterpret_cast<const char*>(p.alpha + ((size_t)b * T + tn) * H * (M > 0 ? M : 1));
-      const int gbytes = (te - tn) * H * 4, abytes = M > 0 ? gbytes * M : 0;
-      for (int off = lane * 128; off < gbytes; off += 32 * 128) {
-        prefetch_l2(g0 + off);
-        prefetch_l2(b0 + off);
-      }
-      for (int off = lane * 128; off < abytes; off += 32 * 128) prefetch_l2(a0 + off);
-    }
     const bool fast = G[63] >= -60.f;  // exp(-G) stays finite: factor D[t,i] = e^{G_t} e^{-G_i}
     if (tid < 64) {
       sEp[tid] = __expf(G[tid]);
@@ -913,8 +904,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     bool ok = warp_wait(bar_mma1, ph_mma1, lim, p.status);
     ph_mma1 ^= 1;
     if (!ok && lane == 0) atomicExch(s_abort, 1);
-    float gl_next[4] = {1.f, 1.f, 0.f, 0.f};  // warp 2: next chunk's gates, scanned in step C
-    if (warp == 2 && n + 1 < nchunks) gate_load(n + 1, gl_next);
+    float gl_after[4] = {1.f, 1.f, 0.f, 0.f};  // warp 2: gates of chunk n+2
+    if (warp == 2 && n + 2 < nchunks) gate_load(n + 2, gl_after);
     tc_fence_after();
     if (ok) {
       const bool krow = row < 64;
@@ -1000,6 +991,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     // ---------------- C: the next chunk's gate prefix; the tap element this thread stages for
     // the next prologue and the values of v it needs for X (their latency hides behind the MMAs)
     if (warp == 2 && n + 1 < nchunks) gate_scan(gl_next, cur ^ 1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) gl_next[e] = gl_after[e];
     const float tap_reg = (M > 0 && tap_thread) ? __ldg(cw_head + tid) : 0.f;
     float al_next[NPASS][M1];  // alpha of the next chunk, for its prologue
     // (padded steps have beta = 0, so any in-range token may stand in for them)
