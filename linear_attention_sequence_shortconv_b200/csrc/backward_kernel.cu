@@ -101,21 +101,30 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(BwdParams p) {
 #pragma unroll
   for (int i = 0; i < MW; ++i) da_later[i] = dw[i] = 0.f;
 
-  // S_t of the token being processed (loaded one token ahead)
-  float st[EPL];
-  if (len > 0) ld_slice<float, EPL>(p.states + (((size_t)bh * T_ + len - 1) * dv + c) * dk + EPL * j, st);
+  // state slices: S_t of the token being processed and S_{t-1}, each requested one token
+  // ahead (S_{t-2} is in flight while token t is processed)
+  auto load_state = [&](int tt, float* dst) {  // S_tt; tt = -1 is the initial state
+    if (tt >= 0) {
+      ld_slice<float, EPL>(p.states + (((size_t)bh * T_ + tt) * dv + c) * dk + EPL * j, dst);
+    } else if (p.S0) {
+      ld_slice<float, EPL>(p.S0 + ((size_t)bh * dv + c) * dk + EPL * j, dst);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) dst[e] = 0.f;
+    }
+  };
+  float st[EPL], sp_next[EPL];
+  if (len > 0) {
+    load_state(len - 1, st);
+    load_state(len - 2, sp_next);
+  }
 
   for (int t = len - 1; t >= 0; --t) {
     const size_t th = ((size_t)b * T_ + t) * H + h;
     float sp[EPL];  // S_{t-1}
-    if (t > 0) {
-      ld_slice<float, EPL>(p.states + (((size_t)bh * T_ + t - 1) * dv + c) * dk + EPL * j, sp);
-    } else if (p.S0) {
-      ld_slice<float, EPL>(p.S0 + ((size_t)bh * dv + c) * dk + EPL * j, sp);
-    } else {
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) sp[e] = 0.f;
-    }
+    for (int e = 0; e < EPL; ++e) sp[e] = sp_next[e];
+    if (t >= 1) load_state(t - 2, sp_next);  // for the next token
     float qv[EPL], kv[EPL];
     ld_slice<T, EPL>(q + th * dk + EPL * j, qv);
     ld_slice<T, EPL>(k + th * dk + EPL * j, kv);
