@@ -889,8 +889,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     const float* G = sG + cur * 64;
     const float* Bt = sBeta + cur * 64;
 
-    // ---------------- A: MMA3 (S_n x [K;Q]^T; MMA1 was issued at the end of the previous chunk);
-    // per-chunk decay tables
+    // ---------------- A: hand S_n (bf16) to the MMA warp for MMA3 (S_n x [K;Q]^T; MMA1 of this
+    // chunk was issued during the previous one); per-chunk decay tables
     if (tid == 0) mbar_arrive(go_A);  // S_n (bf16) is in SXA: MMA3
     const bool fast = G[63] >= -60.f;  // exp(-G) stays finite: factor D[t,i] = e^{G_t} e^{-G_i}
     if (tid < 64) {
@@ -900,7 +900,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     }
     if (worker_sync_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
 
-    // ---------------- B: epilogue of MMA1 -> [Bku;QU], QK (bf16); then MMA2, MMA5a (fast), QK*T
+    // ---------------- B: epilogue of MMA1 -> [Bku;QU], QK (bf16) (exact path: U <- diag(c) U);
+    // then the MMA warp issues MMA2 and QK*T (committed for step E) and MMA5a
     bool ok = warp_wait(bar_mma1, ph_mma1, lim, p.status);
     ph_mma1 ^= 1;
     if (!ok && lane == 0) atomicExch(s_abort, 1);
@@ -1006,7 +1007,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
         vraw16[e] = p.v[(((size_t)b * T + t) * H + h) * D + rr];
       }
     }
-    // ---------------- E: QKT -> TQ rows 64..127; P~ = diag(c) P -> BQ; X^T -> SXA; O partial
+    // ---------------- E: QKT -> TQ rows 64..127; X^T -> SXA; O partial parked in TMEM; the next
+    // chunk's Q requested; then MMA4
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) {
@@ -1051,7 +1053,8 @@ __global__ void __launch_bounds__(kCtaThreads, 1)
     if (worker_sync_or(*s_abort)) { aborted = true; break; }  // uniform: every setter votes
     if (tid == 0) mbar_arrive(go_E);  // MMA4
 
-    // ---------------- G: Delta~^T -> SXA; o = O partial + (QKT X); issue MMA5b
+    // ---------------- G: the next chunk's T, U, gain and v tiles requested (MMA4 and MMA5a are
+    // done); Delta~^T -> SXA; o = O partial + (QKT X) -> TMA store; then MMA5b
     ok = warp_wait(bar_mma, ph_mma, lim, p.status);
     ph_mma ^= 1;
     if (tid == 0 && ok) {
