@@ -1,0 +1,809 @@
+// Chunked backward of the PRISM scan (fp32 arithmetic, fp32 or bf16 inputs).
+//
+// The gradient of L = <o, dO> + <S_final, dS_final> through the recurrence
+// (ICML 2026 PRISM write-up, 核心迭代形式 / 架构形式; PRISM explainer 2.1-2.2)
+//
+//   S_t = gamma_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T + sum_l alpha_l r_l u_l^T,  o_t = S_t q_t
+//
+// is taken in three passes instead of one token-by-token walk over recorded states:
+//
+//  1. the forward token kernel records S at every 64-token chunk boundary and
+//     psi_t = v_t - gamma_t S_{t-1} k_t (so delta_t = beta_t psi_t is the delta-rule
+//     write of token t);
+//  2. adjoint_scan_kernel (here) runs the adjoint recurrence in reverse,
+//        G_t = dO_t q_t^T + gamma_{t+1} G_{t+1} (I - beta_{t+1} k_{t+1} k_{t+1}^T),
+//     with G_T = dS_final, and records per token gk_t = G_t k_t and gu_{t,l} = G_t u_{t,l},
+//     at every chunk end the gradient H_n flowing into it from later chunks, and
+//     <H_n, S_{n+1}>; G before the first token is dS0;
+//  3. chunk_grad_kernel (here) forms every input gradient of one chunk from those
+//     records with no sequential dependence between chunks.  With c_t the cumulative
+//     log gate inside the chunk, D_{ti} = e^{c_t - c_i}, and the chunk's writes
+//     x_{t,0} = delta_t, y_{t,0} = k_t, x_{t,l} = alpha_l r_l, y_{t,l} = u_l:
+//
+//        S_t = e^{c_t} S_n + sum_{i<=t} D_{ti} sum_a x_{i,a} y_{i,a}^T
+//        G_t = e^{c_C - c_t} H_n + sum_{j>=t} D_{jt} dO_j q_j^T - sum_{j>t} D_{jt} beta_j gk_j k_j^T
+//
+//     so that, with M_a = tril(D o (dO X_a^T)) and N_a = strict tril(D o (Gk X_a^T)):
+//
+//        dq   = diag(e^c) dO S_n + sum_a M_a Y_a                       (S_t^T dO_t)
+//        F    = diag(e^c) Gk S_n + sum_a N_a Y_a                       (gamma_t S_{t-1}^T gk_t)
+//        Gx_a = diag(e^{c_C - c}) X_a H_n + M_a^T Q - (diag(beta) N_a)^T K   (G_t^T x_{t,a})
+//        dk   = Gx_0 - diag(beta) F,   du_l = Gx_l,   dbeta_t = gk_t . psi_t,
+//        dalpha_{t,l} = r_{t,l} . gu_{t,l},   dr_{t,l} = alpha_l gu_{t,l} (then the chain backwards),
+//        gamma_t dgamma_t = <H_n, S_{n+1}> + sum_{j>=t in chunk} (q_j . dq_j - w_j),
+//        w_j = <G_j, W_j> = beta_j v_j . gk_j + sum_l alpha_l r_{j,l} . gu_{j,l}.
+//
+//     The last identity is the chunk form of gamma_t dgamma_t = <G_t, S_t> - <G_t, W_t>
+//     together with <G_{t-1}, S_{t-1}> = gamma_t dgamma_t + dO_{t-1} . o_{t-1} and
+//     dO_j . o_j = q_j . dq_j.
+#include "common.cuh"
+
+namespace prism {
+namespace {
+
+constexpr int kAdjBlock = 64;
+constexpr int kAdjTileBytes = 8 * 1024;  // per buffer (small tiles: every row block resident at once)
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+template <typename T>
+__device__ __forceinline__ float4 lds4(const T* p);
+template <>
+__device__ __forceinline__ float4 lds4<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
+template <>
+__device__ __forceinline__ float4 lds4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+template <typename T>
+__device__ __forceinline__ float lds1(const T* p);
+template <>
+__device__ __forceinline__ float lds1<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float lds1<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+template <int LPR>
+__device__ __forceinline__ float row_sum(float x) {
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// d/dx of x Phi(x): Phi(x) + x phi(x)
+__device__ __forceinline__ float gelu_grad(float x) {
+  return 0.5f * (1.f + erff(x * 0.7071067811865476f)) + x * 0.3989422804014327f * __expf(-0.5f * x * x);
+}
+
+// ------------------------------------------------------------------ adjoint pass
+
+// Shared-memory tile of TT tokens for the adjoint pass (byte offsets, 16-byte aligned).
+struct AdjLayout {
+  int off_k, off_q, off_u, off_do, off_gam, off_bet, bytes;
+  __host__ __device__ AdjLayout(int TT, int dk, int m, int rpb, int es) {
+    auto al16 = [](int x) { return (x + 15) & ~15; };
+    off_k = 0;
+    off_q = al16(off_k + TT * dk * es);
+    off_u = al16(off_q + TT * dk * es);
+    off_do = al16(off_u + TT * m * dk * es);
+    off_gam = al16(off_do + TT * rpb * es);
+    off_bet = al16(off_gam + TT * 4);
+    bytes = al16(off_bet + TT * 4);
+  }
+};
+
+template <typename T>
+int adj_tile_tokens(int dk, int m, int rpb) {
+  for (int TT = 32; TT > 1; TT >>= 1)
+    if (AdjLayout(TT, dk, m, rpb, sizeof(T)).bytes <= kAdjTileBytes) return TT;
+  return 1;
+}
+
+// One block: kAdjBlock / LPR rows of G for one (batch, head).  Rows of G are
+// independent (G is multiplied from the right by the transition), so row c only
+// needs the dot products (G k)_c and (G u_l)_c inside the row, over its LPR lanes.
+// Tokens are walked from the last valid one down to 0, tiles streamed in reverse.
+template <typename T, int LPR, int EPL>
+__global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams p, int TT) {
+  constexpr int RPB = kAdjBlock / LPR;
+  constexpr int C = kBwdChunk;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int tid = threadIdx.x;
+  const int j = tid % LPR;
+  const int lrow = tid / LPR;
+  const int row0 = blockIdx.x * RPB;
+  const int row = row0 + lrow;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T_ = p.T, H = p.H, dk = p.d, dv = p.d, m = p.L - 1;
+  const bool row_ok = row < dv;
+  const int c = row_ok ? row : dv - 1;
+  const int cr = row_ok ? lrow : 0;
+  const int len = p.lengths ? min(max(p.lengths[b], 0), T_) : T_;
+  const int NC = (T_ + C - 1) / C;
+  const int ncb = (len + C - 1) / C;
+  const AdjLayout L(TT, dk, m, RPB, (int)sizeof(T));
+  const int nrows = min(RPB, dv - row0);
+  const size_t bh = (size_t)b * H + h;
+
+  const T* q = static_cast<const T*>(p.q);
+  const T* k = static_cast<const T*>(p.k);
+  const T* u = static_cast<const T*>(p.u);
+  const T* dO = static_cast<const T*>(p.dO);
+
+  auto load_tile = [&](int ti, int buf) {
+    uint8_t* base = smem + buf * L.bytes;
+    const int t0 = ti * TT, nt = min(TT, len - t0);
+    const int vec = 16 / (int)sizeof(T);
+    const int kchunks = dk / vec;
+    for (int e = tid; e < nt * kchunks; e += kAdjBlock) {
+      const int i = e / kchunks, cc = e % kchunks;
+      const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+      cp_async16(base + L.off_k + (i * dk + cc * vec) * sizeof(T), k + tok * dk + cc * vec);
+      cp_async16(base + L.off_q + (i * dk + cc * vec) * sizeof(T), q + tok * dk + cc * vec);
+    }
+    for (int e = tid; e < nt * m * kchunks; e += kAdjBlock) {
+      const int i = e / (m * kchunks), r = e % (m * kchunks);
+      const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+      cp_async16(base + L.off_u + ((size_t)i * m * dk + r * vec) * sizeof(T), u + tok * m * dk + r * vec);
+    }
+    const int rbytes = RPB * (int)sizeof(T);
+    if (nrows == RPB && rbytes % 16 == 0) {
+      const int rch = rbytes / 16;
+      for (int e = tid; e < nt * rch; e += kAdjBlock) {
+        const int i = e / rch, cc = e % rch;
+        const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+        cp_async16(base + L.off_do + i * rbytes + cc * 16, dO + tok * dv + row0 + cc * (16 / (int)sizeof(T)));
+      }
+    } else {
+      for (int e = tid; e < nt * nrows; e += kAdjBlock) {
+        const int i = e / nrows, rr = e % nrows;
+        const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+        T* dst = reinterpret_cast<T*>(base + L.off_do) + i * RPB + rr;
+        if (sizeof(T) == 4)
+          cp_async4(dst, dO + tok * dv + row0 + rr);
+        else
+          *dst = dO[tok * dv + row0 + rr];
+      }
+    }
+    for (int e = tid; e < nt * 2; e += kAdjBlock) {
+      const int i = e / 2, r = e % 2;
+      const size_t tok = ((size_t)b * T_ + t0 + i) * H + h;
+      float* dst = reinterpret_cast<float*>(base + (r == 0 ? L.off_gam : L.off_bet)) + i;
+      cp_async4(dst, r == 0 ? p.gamma + tok : p.beta + tok);
+    }
+  };
+
+  float g[EPL];
+  const size_t gbase = (bh * dv + c) * dk + EPL * j;
+#pragma unroll
+  for (int e = 0; e < EPL; e += 4) {
+    const float4 f = p.dS_final ? __ldg(reinterpret_cast<const float4*>(p.dS_final + gbase + e))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    g[e] = f.x; g[e + 1] = f.y; g[e + 2] = f.z; g[e + 3] = f.w;
+  }
+  // H_n (the gradient flowing into the end of chunk n from later tokens) and <H_n, S_{n+1}>
+  auto record_boundary = [&](int n) {
+    const float* st = p.states + ((bh * (NC + 1) + n + 1) * dv + c) * dk + EPL * j;
+    float* hn = p.Hn + ((bh * NC + n) * dv + c) * dk + EPL * j;
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; e += 4) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(st + e));
+      dot += g[e] * f.x + g[e + 1] * f.y + g[e + 2] * f.z + g[e + 3] * f.w;
+      if (row_ok) *reinterpret_cast<float4*>(hn + e) = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
+    }
+    dot = row_sum<LPR>(dot);
+    if (row_ok && j == 0) p.hs[(bh * NC + n) * dv + c] = dot;
+  };
+  if (ncb > 0) record_boundary(ncb - 1);
+
+  const int ntiles = (len + TT - 1) / TT;
+  if (ntiles > 0) load_tile(ntiles - 1, 0);
+  cp_async_commit();
+  for (int it = 0; it < ntiles; ++it) {
+    const int ti = ntiles - 1 - it, buf = it & 1;
+    if (ti > 0) load_tile(ti - 1, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait_1();
+    __syncthreads();
+    const uint8_t* base = smem + buf * L.bytes;
+    const T* sk_ = reinterpret_cast<const T*>(base + L.off_k);
+    const T* sq_ = reinterpret_cast<const T*>(base + L.off_q);
+    const T* su_ = reinterpret_cast<const T*>(base + L.off_u);
+    const T* sdo = reinterpret_cast<const T*>(base + L.off_do);
+    const float* sgam = reinterpret_cast<const float*>(base + L.off_gam);
+    const float* sbet = reinterpret_cast<const float*>(base + L.off_bet);
+    const int t0 = ti * TT, nt = min(TT, len - t0);
+    for (int i = nt - 1; i >= 0; --i) {
+      const int t = t0 + i;
+      const size_t tok = ((size_t)b * T_ + t) * H + h;
+      // G_t = (carry) + dO_t q_t^T
+      const float dot_ = lds1<T>(sdo + i * RPB + cr);
+      const T* qq = sq_ + i * dk + EPL * j;
+#pragma unroll
+      for (int e = 0; e < EPL; e += 4) {
+        const float4 f = lds4<T>(qq + e);
+        g[e] += dot_ * f.x; g[e + 1] += dot_ * f.y; g[e + 2] += dot_ * f.z; g[e + 3] += dot_ * f.w;
+      }
+      const T* kk = sk_ + i * dk + EPL * j;
+      float gk = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; e += 4) {
+        const float4 f = lds4<T>(kk + e);
+        gk += g[e] * f.x + g[e + 1] * f.y + g[e + 2] * f.z + g[e + 3] * f.w;
+      }
+      gk = row_sum<LPR>(gk);
+      if (row_ok && j == 0) p.gk[tok * dv + c] = gk;
+      for (int l = 0; l < m; ++l) {
+        const T* uu = su_ + ((size_t)i * m + l) * dk + EPL * j;
+        float gu = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; e += 4) {
+          const float4 f = lds4<T>(uu + e);
+          gu += g[e] * f.x + g[e + 1] * f.y + g[e + 2] * f.z + g[e + 3] * f.w;
+        }
+        gu = row_sum<LPR>(gu);
+        if (row_ok && j == 0) p.gu[(tok * m + l) * dv + c] = gu;
+      }
+      // carry into token t - 1: gamma_t (G_t - beta_t (G_t k_t) k_t^T)
+      const float gam = sgam[i], bg = sbet[i] * gk;
+#pragma unroll
+      for (int e = 0; e < EPL; e += 4) {
+        const float4 f = lds4<T>(kk + e);
+        g[e] = gam * (g[e] - bg * f.x);
+        g[e + 1] = gam * (g[e + 1] - bg * f.y);
+        g[e + 2] = gam * (g[e + 2] - bg * f.z);
+        g[e + 3] = gam * (g[e + 3] - bg * f.w);
+      }
+      if (t > 0 && t % C == 0) record_boundary(t / C - 1);
+    }
+    __syncthreads();  // the buffer is refilled next iteration
+  }
+  cp_async_wait_0();
+  if (row_ok) {
+#pragma unroll
+    for (int e = 0; e < EPL; e += 4)
+      *reinterpret_cast<float4*>(p.dS0 + gbase + e) = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
+  }
+}
+
+// ------------------------------------------------------------------ per-chunk gradients
+
+constexpr int kGradThreads = 256;  // 16 x 16 thread grid over every tile
+constexpr int kHalo = PRISM_MAX_W - 1;
+
+// Shared-memory layout of chunk_grad_kernel (float offsets).  Rows are padded by 4
+// floats so that float4 reads of 16 different rows hit different banks.
+template <int D>
+struct GradLayout {
+  static constexpr int C = kBwdChunk;
+  static constexpr int LDD = D + 4;  // row stride of the C x D tiles
+  static constexpr int LDC = C + 4;  // row stride of the C x C tiles
+  static constexpr int VROWS = C + 2 * kHalo;
+  static constexpr int DO = 0;                      // dO, later dr_0 of the chunk's tokens
+  static constexpr int GK = DO + C * LDD;           // gk
+  static constexpr int X = GK + C * LDD;            // X_a
+  static constexpr int V = X + C * LDD;             // v of tokens t0 - kHalo .. t0 + C + kHalo - 1
+  static constexpr int M = V + VROWS * LDD;         // M_a, later dr_0 of the halo tokens
+  static constexpr int N = M + C * LDC;             // N_a
+  static constexpr int WC = N + C * LDC;            // conv taps [W][D]
+  static constexpr int SC = WC + PRISM_MAX_W * D;   // c_t
+  static constexpr int EC = SC + C;                 // e^{c_t}
+  static constexpr int ECC = EC + C;                // e^{c_C - c_t}
+  static constexpr int BE = ECC + C;                // beta (0 past the last valid token)
+  static constexpr int QDQ = BE + C;                // q_t . dq_t
+  static constexpr int WT = QDQ + C;                // w_t
+  static constexpr int RED = WT + C;                // scratch for reductions
+  static constexpr int FLOATS = RED + 32;
+  static constexpr size_t BYTES = (size_t)FLOATS * 4;
+};
+
+// acc[r][s4*4 + e] += sum_k A(row_r, k) * B(k, col), rows ty + 16 r, columns
+// 4 tx + 64 s4 + e.  A is a C x K tile in shared memory (row stride lda) read
+// four k at a time, B a K x D row-major matrix in global fp32 memory.
+template <int D>
+__device__ __forceinline__ void gemm_smemA_globalB(float (&acc)[4][D / 16], const float* sA, int lda,
+                                                   const float* gB, int K, int ty, int tx) {
+  for (int k = 0; k < K; k += 4) {
+    float4 a[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) a[r] = *reinterpret_cast<const float4*>(sA + (ty + 16 * r) * lda + k);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+      for (int s4 = 0; s4 < D / 64; ++s4) {
+        const float4 bv = __ldg(reinterpret_cast<const float4*>(gB + (size_t)(k + kk) * D + 4 * tx + 64 * s4));
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float av = kk == 0 ? a[r].x : (kk == 1 ? a[r].y : (kk == 2 ? a[r].z : a[r].w));
+          acc[r][4 * s4] += av * bv.x;
+          acc[r][4 * s4 + 1] += av * bv.y;
+          acc[r][4 * s4 + 2] += av * bv.z;
+          acc[r][4 * s4 + 3] += av * bv.w;
+        }
+      }
+    }
+  }
+}
+
+template <typename T, int D, int M, int CH>
+__global__ void __launch_bounds__(kGradThreads) chunk_grad_kernel(ChunkBwdParams p) {
+  using Ly = GradLayout<D>;
+  constexpr int C = kBwdChunk, LDD = Ly::LDD, LDC = Ly::LDC, TN = D / 16;
+  extern __shared__ __align__(16) float sm[];
+  float* sDO = sm + Ly::DO;
+  float* sGK = sm + Ly::GK;
+  float* sX = sm + Ly::X;
+  float* sV = sm + Ly::V;
+  float* sM = sm + Ly::M;
+  float* sN = sm + Ly::N;
+  float* sWc = sm + Ly::WC;
+  float* sc = sm + Ly::SC;
+  float* sec = sm + Ly::EC;
+  float* secc = sm + Ly::ECC;
+  float* sbe = sm + Ly::BE;
+  float* sqdq = sm + Ly::QDQ;
+  float* swt = sm + Ly::WT;
+  float* sred = sm + Ly::RED;
+
+  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int T_ = p.T, H = p.H, W = p.W;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15, warp = tid >> 5, lane = tid & 31;
+  const int len = p.lengths ? min(max(p.lengths[b], 0), T_) : T_;
+  const int NC = (T_ + C - 1) / C;
+  const int t0 = n * C;
+  const size_t bh = (size_t)b * H + h;
+  float* part = p.dconv_part + (((size_t)b * NC + n) * H + h) * D * W;
+  if (t0 >= len) {  // a chunk past the last valid token: its dconv partial is zero
+    for (int e = tid; e < D * W; e += kGradThreads) part[e] = 0.f;
+    return;
+  }
+  const int nt = min(C, len - t0);                // valid tokens of the chunk
+  const int nh = min(C + W - 1, len - t0);        // ... and of the forward halo (dr_0 of later tokens)
+  const T* q = static_cast<const T*>(p.q);
+  const T* k = static_cast<const T*>(p.k);
+  const T* v = static_cast<const T*>(p.v);
+  const T* u = static_cast<const T*>(p.u);
+  const T* gain = static_cast<const T*>(p.gain);
+  const T* dO = static_cast<const T*>(p.dO);
+  auto tokidx = [&](int t) { return ((size_t)b * T_ + t0 + t) * H + h; };  // t relative to the chunk
+
+  // ---- gates: c_t (cumulative log gate inside the chunk; 0 past the last valid token)
+  if (tid < C) {
+    const bool ok = tid < nt;
+    const float gm = ok ? __ldg(p.gamma + tokidx(tid)) : 1.f;
+    sbe[tid] = ok ? __ldg(p.beta + tokidx(tid)) : 0.f;
+    float x = ok ? logf(gm) : 0.f;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    sc[tid] = x;
+  }
+  // conv taps of the head, [W][D]
+  for (int e = tid; e < W * D; e += kGradThreads) {
+    const int i = e / D, cc = e % D;
+    sWc[e] = __ldg(p.conv_w + ((size_t)h * D + cc) * W + i);
+  }
+  // hs = <H_n, S_{n+1}> (row partials of the adjoint pass)
+  if (warp == 0) {
+    float x = 0.f;
+    for (int cc = lane; cc < D; cc += 32) x += __ldg(p.hs + (bh * NC + n) * D + cc);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if (lane == 0) sred[0] = x;
+  }
+  // dO and gk of the chunk (zero rows past the last valid token)
+  for (int e = tid; e < C * (D / 4); e += kGradThreads) {
+    const int t = e / (D / 4), c4 = 4 * (e % (D / 4));
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), g = a;
+    if (t < nt) {
+      a = ld4<T>(dO + tokidx(t) * D + c4);
+      g = __ldg(reinterpret_cast<const float4*>(p.gk + tokidx(t) * D + c4));
+    }
+    *reinterpret_cast<float4*>(sDO + t * LDD + c4) = a;
+    *reinterpret_cast<float4*>(sGK + t * LDD + c4) = g;
+  }
+  // v of tokens t0 - kHalo .. t0 + C + kHalo - 1 (zero outside 0 .. len - 1)
+  for (int e = tid; e < Ly::VROWS * (D / 4); e += kGradThreads) {
+    const int rr = e / (D / 4), c4 = 4 * (e % (D / 4));
+    const int t = rr - kHalo;  // relative to the chunk
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t0 + t >= 0 && t0 + t < len) a = ld4<T>(v + tokidx(t) * D + c4);
+    *reinterpret_cast<float4*>(sV + rr * LDD + c4) = a;
+  }
+  __syncthreads();
+  if (tid >= 32 && tid < C) sc[tid] += sc[31];
+  __syncthreads();
+  if (tid < C) {
+    sec[tid] = __expf(sc[tid]);
+    secc[tid] = __expf(sc[C - 1] - sc[tid]);
+  }
+  __syncthreads();
+  const float hs = sred[0];
+
+  // residual r_l of channel cc at chunk-relative token t (l <= M)
+  auto residual = [&](int t, int cc, int l) {
+    const float* vr = sV + (t + kHalo) * LDD + cc;
+    float a = 0.f;
+    for (int i = 0; i < W; ++i) a += sWc[i * D + cc] * vr[-i * LDD];
+    float r = vr[0] - a;
+    for (int z = 0; z < l; ++z) r = chain_step(r, ld1<T>(gain + (tokidx(t) * M + z) * D + cc), CH);
+    return r;
+  };
+
+  // ---- dq = diag(e^c) dO S_n + ..., F = diag(e^c) gk S_n + ...
+  float adq[4][TN], aF[4][TN];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int e = 0; e < TN; ++e) adq[r][e] = aF[r][e] = 0.f;
+  const float* Sn = p.states + (bh * (NC + 1) + n) * D * D;
+  const float* Hn = p.Hn + (bh * NC + n) * D * D;
+  gemm_smemA_globalB<D>(adq, sDO, LDD, Sn, D, ty, tx);
+  gemm_smemA_globalB<D>(aF, sGK, LDD, Sn, D, ty, tx);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float ec = sec[ty + 16 * r];
+#pragma unroll
+    for (int e = 0; e < TN; ++e) { adq[r][e] *= ec; aF[r][e] *= ec; }
+  }
+
+  for (int a = 0; a <= M; ++a) {
+    // X_a: a = 0 delta_t = beta_t psi_t; a = l alpha_{t,l} r_{t,l}
+    for (int e = tid; e < C * (D / 4); e += kGradThreads) {
+      const int t = e / (D / 4), c4 = 4 * (e % (D / 4));
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < nt) {
+        if (a == 0) {
+          const float4 ps = __ldg(reinterpret_cast<const float4*>(p.psi + tokidx(t) * D + c4));
+          const float be = sbe[t];
+          x = make_float4(be * ps.x, be * ps.y, be * ps.z, be * ps.w);
+        } else {
+          const float al = __ldg(p.alpha + tokidx(t) * M + a - 1);
+          x = make_float4(al * residual(t, c4, a), al * residual(t, c4 + 1, a), al * residual(t, c4 + 2, a),
+                          al * residual(t, c4 + 3, a));
+        }
+      }
+      *reinterpret_cast<float4*>(sX + t * LDD + c4) = x;
+    }
+    __syncthreads();
+    // Grams P = dO X_a^T, Pf = gk X_a^T (C x C over D), masked and decayed into M_a, N_a
+    {
+      float gp[4][4], gf[4][4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int s = 0; s < 4; ++s) gp[r][s] = gf[r][s] = 0.f;
+      for (int kc = 0; kc < D; kc += 4) {
+        float4 ad[4], ag[4], bx[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          ad[r] = *reinterpret_cast<const float4*>(sDO + (ty + 16 * r) * LDD + kc);
+          ag[r] = *reinterpret_cast<const float4*>(sGK + (ty + 16 * r) * LDD + kc);
+        }
+#pragma unroll
+        for (int s = 0; s < 4; ++s) bx[s] = *reinterpret_cast<const float4*>(sX + (tx + 16 * s) * LDD + kc);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            gp[r][s] += ad[r].x * bx[s].x + ad[r].y * bx[s].y + ad[r].z * bx[s].z + ad[r].w * bx[s].w;
+            gf[r][s] += ag[r].x * bx[s].x + ag[r].y * bx[s].y + ag[r].z * bx[s].z + ag[r].w * bx[s].w;
+          }
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int t = ty + 16 * r;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const int i = tx + 16 * s;
+          const float dd = i <= t ? __expf(sc[t] - sc[i]) : 0.f;
+          sM[t * LDC + i] = dd * gp[r][s];
+          sN[t * LDC + i] = i < t ? dd * gf[r][s] : 0.f;
+        }
+      }
+    }
+    __syncthreads();
+    // dq += M_a Y_a, F += N_a Y_a  (Y_0 = K, Y_l = U_l; rows past nt never read)
+    const T* Y = a == 0 ? k : u;
+    const size_t ystride = a == 0 ? (size_t)H * D : (size_t)H * M * D;
+    const T* Y0 = a == 0 ? k + tokidx(0) * D : u + (tokidx(0) * M + (a - 1)) * D;
+    (void)Y;
+    for (int i = 0; i < nt; ++i) {
+      float am[4], an[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        am[r] = sM[(ty + 16 * r) * LDC + i];
+        an[r] = sN[(ty + 16 * r) * LDC + i];
+      }
+#pragma unroll
+      for (int s4 = 0; s4 < D / 64; ++s4) {
+        const float4 bv = ld4<T>(Y0 + i * ystride + 4 * tx + 64 * s4);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          adq[r][4 * s4] += am[r] * bv.x; adq[r][4 * s4 + 1] += am[r] * bv.y;
+          adq[r][4 * s4 + 2] += am[r] * bv.z; adq[r][4 * s4 + 3] += am[r] * bv.w;
+          aF[r][4 * s4] += an[r] * bv.x; aF[r][4 * s4 + 1] += an[r] * bv.y;
+          aF[r][4 * s4 + 2] += an[r] * bv.z; aF[r][4 * s4 + 3] += an[r] * bv.w;
+        }
+      }
+    }
+    // Gx_a = diag(e^{c_C - c}) X_a H_n + M_a^T Q - (diag(beta) N_a)^T K
+    {
+      float ag[4][TN];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int e = 0; e < TN; ++e) ag[r][e] = 0.f;
+      gemm_smemA_globalB<D>(ag, sX, LDD, Hn, D, ty, tx);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float ec = secc[ty + 16 * r];
+#pragma unroll
+        for (int e = 0; e < TN; ++e) ag[r][e] *= ec;
+      }
+      const T* Q0 = q + tokidx(0) * D;
+      const T* K0 = k + tokidx(0) * D;
+      const size_t qs = (size_t)H * D;
+      for (int jj = 0; jj < nt; ++jj) {
+        float am[4], an[4];
+        const float be = sbe[jj];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          am[r] = sM[jj * LDC + ty + 16 * r];
+          an[r] = -be * sN[jj * LDC + ty + 16 * r];
+        }
+#pragma unroll
+        for (int s4 = 0; s4 < D / 64; ++s4) {
+          const float4 qv = ld4<T>(Q0 + jj * qs + 4 * tx + 64 * s4);
+          const float4 kv = ld4<T>(K0 + jj * qs + 4 * tx + 64 * s4);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            ag[r][4 * s4] += am[r] * qv.x + an[r] * kv.x;
+            ag[r][4 * s4 + 1] += am[r] * qv.y + an[r] * kv.y;
+            ag[r][4 * s4 + 2] += am[r] * qv.z + an[r] * kv.z;
+            ag[r][4 * s4 + 3] += am[r] * qv.w + an[r] * kv.w;
+          }
+        }
+      }
+      // a = 0: G_t^T delta_t, kept in dk until F is complete; a = l: du_l
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int t = ty + 16 * r;
+        if (t >= nt) continue;
+#pragma unroll
+        for (int s4 = 0; s4 < D / 64; ++s4) {
+          float* dst = a == 0 ? p.dk + tokidx(t) * D : p.du + (tokidx(t) * M + (a - 1)) * D;
+          *reinterpret_cast<float4*>(dst + 4 * tx + 64 * s4) =
+              make_float4(ag[r][4 * s4], ag[r][4 * s4 + 1], ag[r][4 * s4 + 2], ag[r][4 * s4 + 3]);
+        }
+      }
+    }
+    __syncthreads();  // sX, sM, sN are rewritten by the next a
+  }
+
+  // ---- dq, dk = G^T delta - diag(beta) F, q_t . dq_t
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int t = ty + 16 * r;
+    float qd = 0.f;
+    if (t < nt) {
+      const float be = sbe[t];
+#pragma unroll
+      for (int s4 = 0; s4 < D / 64; ++s4) {
+        const int col = 4 * tx + 64 * s4;
+        const float4 qv = ld4<T>(q + tokidx(t) * D + col);
+        qd += qv.x * adq[r][4 * s4] + qv.y * adq[r][4 * s4 + 1] + qv.z * adq[r][4 * s4 + 2] +
+              qv.w * adq[r][4 * s4 + 3];
+        *reinterpret_cast<float4*>(p.dq + tokidx(t) * D + col) =
+            make_float4(adq[r][4 * s4], adq[r][4 * s4 + 1], adq[r][4 * s4 + 2], adq[r][4 * s4 + 3]);
+        float4* dk4 = reinterpret_cast<float4*>(p.dk + tokidx(t) * D + col);
+        const float4 gx = *dk4;  // this thread's own store above
+        *dk4 = make_float4(gx.x - be * aF[r][4 * s4], gx.y - be * aF[r][4 * s4 + 1], gx.z - be * aF[r][4 * s4 + 2],
+                           gx.w - be * aF[r][4 * s4 + 3]);
+      }
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) qd += __shfl_xor_sync(0xffffffffu, qd, off);
+    if (tx == 0) sqdq[t] = qd;
+  }
+
+  // ---- per token (one warp each): dbeta, dalpha, w_t, the chain backwards -> dr_0, dgain
+  // dr_0 of chunk token t goes to sDO row t (dO is no longer needed), of halo token
+  // C + z to sM row z.
+  for (int t = warp; t < nh; t += kGradThreads / 32) {
+    const size_t tok = tokidx(t);
+    const bool own = t < nt;
+    const float be = own ? sbe[t] : __ldg(p.beta + tok);
+    float db = 0.f, wsum = 0.f, dal[M > 0 ? M : 1];
+#pragma unroll
+    for (int l = 0; l < M; ++l) dal[l] = 0.f;
+    float* drow = t < C ? sDO + t * LDD : sM + (t - C) * LDD;
+    for (int cc = lane; cc < D; cc += 32) {
+      const float gkc = own ? sGK[t * LDD + cc] : __ldg(p.gk + tok * D + cc);
+      float rr[M + 1];
+      {
+        const float* vr = sV + (t + kHalo) * LDD + cc;
+        float an = 0.f;
+        for (int i = 0; i < W; ++i) an += sWc[i * D + cc] * vr[-i * LDD];
+        rr[0] = vr[0] - an;
+#pragma unroll
+        for (int l = 0; l < M; ++l) rr[l + 1] = chain_step(rr[l], ld1<T>(gain + (tok * M + l) * D + cc), CH);
+      }
+      if (own) {
+        db += gkc * __ldg(p.psi + tok * D + cc);
+        wsum += be * sV[(t + kHalo) * LDD + cc] * gkc;
+      }
+      float dr = 0.f;
+#pragma unroll
+      for (int l = M; l >= 1; --l) {
+        const float al = __ldg(p.alpha + tok * M + l - 1);
+        const float gu = __ldg(p.gu + (tok * M + l - 1) * D + cc);
+        if (own) {
+          dal[l - 1] += rr[l] * gu;
+          wsum += al * rr[l] * gu;
+        }
+        dr += al * gu;
+        const float gl = ld1<T>(gain + (tok * M + l - 1) * D + cc);
+        const float rp = rr[l - 1];
+        float dg;
+        if (CH == PRISM_CHAIN_GELU) {
+          const float gp = gelu_grad(gl * rp);
+          dg = -rp * gp * dr;
+          dr *= 1.f - gl * gp;
+        } else {
+          dg = -rp * dr;
+          dr *= 1.f - gl;
+        }
+        if (own) p.dgain[(tok * M + l - 1) * D + cc] = dg;
+      }
+      drow[cc] = dr;
+    }
+    if (own) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        db += __shfl_xor_sync(0xffffffffu, db, off);
+        wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+      }
+#pragma unroll
+      for (int l = 0; l < M; ++l)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dal[l] += __shfl_xor_sync(0xffffffffu, dal[l], off);
+      if (lane == 0) {
+        p.dbeta[tok] = db;
+        swt[t] = wsum;
+#pragma unroll
+        for (int l = 0; l < M; ++l) p.dalpha[tok * M + l] = dal[l];
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- gamma_t dgamma_t = hs + sum_{j >= t} (q_j . dq_j - w_j): a suffix sum over the chunk
+  if (warp == 0) {
+    const int ta = 2 * lane, tb = 2 * lane + 1;
+    const float xa = ta < nt ? sqdq[ta] - swt[ta] : 0.f;
+    const float xb = tb < nt ? sqdq[tb] - swt[tb] : 0.f;
+    float x = xa + xb;  // pair sum; suffix-scan the pairs
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_down_sync(0xffffffffu, x, off);
+      if (lane + off < 32) x += y;
+    }
+    // x = sum over pairs lane.. = sum_{j >= ta}
+    if (ta < nt) p.dgamma[tokidx(ta)] = (hs + x) / __ldg(p.gamma + tokidx(ta));
+    if (tb < nt) p.dgamma[tokidx(tb)] = (hs + x - xa) / __ldg(p.gamma + tokidx(tb));
+  }
+
+  // ---- dv_t = beta_t gk_t + dr_0,t - sum_i w_i dr_0,t+i  (ShortConv transpose, within len)
+  auto dr0 = [&](int t, int cc) { return t < C ? sDO[t * LDD + cc] : sM[(t - C) * LDD + cc]; };
+  for (int e = tid; e < nt * D; e += kGradThreads) {
+    const int t = e / D, cc = e % D;
+    float dvv = sbe[t] * sGK[t * LDD + cc] + dr0(t, cc);
+    for (int i = 0; i < W; ++i)
+      if (t + i < nh) dvv -= sWc[i * D + cc] * dr0(t + i, cc);
+    p.dv[tokidx(t) * D + cc] = dvv;
+  }
+  // ---- dconv partial of this chunk: -sum_t dr_0,t v_{t-i}
+  for (int e = tid; e < D * W; e += kGradThreads) {
+    const int cc = e / W, i = e % W;
+    float s = 0.f;
+    for (int t = 0; t < nt; ++t) s -= dr0(t, cc) * sV[(t + kHalo - i) * LDD + cc];
+    part[e] = s;
+  }
+}
+
+// dconv_w[h, c, i] = sum over (batch, chunk) of the partials, in a fixed order
+__global__ void chunk_dconv_reduce_kernel(const float* part, float* dconv_w, int nparts, int n) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n) return;
+  float s = 0.f;
+  for (int b = 0; b < nparts; ++b) s += part[(size_t)b * n + idx];
+  dconv_w[idx] = s;
+}
+
+template <typename T, int D, int M, int CH>
+cudaError_t launch_grad(const ChunkBwdParams& p, cudaStream_t stream) {
+  const size_t smem = GradLayout<D>::BYTES;
+  cudaError_t err = cudaFuncSetAttribute(chunk_grad_kernel<T, D, M, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  if (err != cudaSuccess) return err;
+  const int NC = (p.T + kBwdChunk - 1) / kBwdChunk;
+  chunk_grad_kernel<T, D, M, CH><<<dim3(NC, p.H, p.B), kGradThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int CH>
+cudaError_t launch_grad_m(const ChunkBwdParams& p, cudaStream_t stream) {
+  switch (p.L - 1) {
+    case 0: return launch_grad<T, D, 0, CH>(p, stream);
+    case 1: return launch_grad<T, D, 1, CH>(p, stream);
+    case 2: return launch_grad<T, D, 2, CH>(p, stream);
+    case 3: return launch_grad<T, D, 3, CH>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename T>
+cudaError_t launch_chunk_bwd_t(const ChunkBwdParams& p, cudaStream_t stream) {
+  // adjoint pass: 8 lanes per row as in the forward token kernel
+  constexpr int LPR = 8;
+  constexpr int RPB = kAdjBlock / LPR;
+  const int TT = adj_tile_tokens<T>(p.d, p.L - 1, RPB);
+  const int smem = 2 * AdjLayout(TT, p.d, p.L - 1, RPB, sizeof(T)).bytes;
+  const dim3 grid((p.d + RPB - 1) / RPB, p.H, p.B);
+  cudaError_t err;
+  if (p.d == 64) {
+    err = cudaFuncSetAttribute(adjoint_scan_kernel<T, LPR, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    adjoint_scan_kernel<T, LPR, 8><<<grid, kAdjBlock, smem, stream>>>(p, TT);
+  } else {
+    err = cudaFuncSetAttribute(adjoint_scan_kernel<T, LPR, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    adjoint_scan_kernel<T, LPR, 16><<<grid, kAdjBlock, smem, stream>>>(p, TT);
+  }
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  if (p.d == 64)
+    err = p.chain == PRISM_CHAIN_GELU ? launch_grad_m<T, 64, PRISM_CHAIN_GELU>(p, stream)
+                                      : launch_grad_m<T, 64, PRISM_CHAIN_LINEAR>(p, stream);
+  else
+    err = p.chain == PRISM_CHAIN_GELU ? launch_grad_m<T, 128, PRISM_CHAIN_GELU>(p, stream)
+                                      : launch_grad_m<T, 128, PRISM_CHAIN_LINEAR>(p, stream);
+  if (err != cudaSuccess) return err;
+  const int NC = (p.T + kBwdChunk - 1) / kBwdChunk;
+  const int n = p.H * p.d * p.W;
+  chunk_dconv_reduce_kernel<<<(n + 255) / 256, 256, 0, stream>>>(p.dconv_part, p.dconv_w, p.B * NC, n);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_bwd_supported(int d_k, int d_v, int L) {
+  return d_k == d_v && (d_k == 64 || d_k == 128) && L >= 1 && L <= 4;
+}
+
+size_t chunk_bwd_smem_bytes(int d) { return d == 64 ? GradLayout<64>::BYTES : GradLayout<128>::BYTES; }
+
+cudaError_t launch_chunk_bwd(const ChunkBwdParams& p, int dtype, cudaStream_t stream) {
+  if (!chunk_bwd_supported(p.d, p.d, p.L)) return cudaErrorInvalidValue;
+  if (dtype == PRISM_FP32) return launch_chunk_bwd_t<float>(p, stream);
+  return launch_chunk_bwd_t<__nv_bfloat16>(p, stream);
+}
+
+}  // namespace prism

@@ -31,7 +31,15 @@ struct ScanParams {
   void* workspace;        // prism_scan_fwd_workspace_size() bytes (NULL when that is 0)
   float* states;          // token-by-token path only: S_t after every valid token,
                           // [B, H, T, d_v, d_k] fp32 (NULL: not recorded)
+  // records for the chunked backward (token-by-token path; NULL: not recorded)
+  float* rec_states;      // S at every 64-token chunk boundary, [B, H, NC + 1, d_v, d_k] fp32:
+                          // slot 0 the initial state, slot n the state after token 64 n - 1,
+                          // slot ceil(len / 64) the state after the last valid token
+  float* rec_psi;         // v_t - gamma_t S_{t-1} k_t per valid token, [B, T, H, d_v] fp32
 };
+
+// Tokens per chunk of the chunked backward.
+constexpr int kBwdChunk = 64;
 
 // Pointers and sizes of one prism_decode_step call (device pointers).
 struct DecodeParams {
@@ -79,6 +87,41 @@ struct BwdParams {
   float* dconv_w;     // [H, d_v, W]
   float* dS0;
   int B, T, H, d_k, d_v, L, W, chain;
+};
+
+// Pointers and sizes of the chunked backward (d_k = d_v = d; device pointers).
+// NC = ceil(T / kBwdChunk).  The records are fp32 and live in the workspace.
+struct ChunkBwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* gamma;
+  const float* beta;
+  const void* u;
+  const float* alpha;
+  const void* gain;
+  const float* conv_w;
+  const int32_t* lengths;
+  const void* dO;
+  const float* dS_final;
+  const float* states;  // [B, H, NC + 1, d, d]: S at the chunk boundaries (forward record)
+  const float* psi;     // [B, T, H, d]: v_t - gamma_t S_{t-1} k_t (forward record)
+  float* Hn;            // [B, H, NC, d, d]: gradient flowing into the end of chunk n from later tokens
+  float* gk;            // [B, T, H, d]: G_t k_t
+  float* gu;            // [B, T, H, L - 1, d]: G_t u_{t,l}
+  float* hs;            // [B, H, NC, d]: row partials of <H_n, S_{n+1}>
+  float* dconv_part;    // [B, NC, H, d, W]: per-chunk dconv_w partials
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dgamma;
+  float* dbeta;
+  float* du;
+  float* dalpha;
+  float* dgain;
+  float* dconv_w;
+  float* dS0;
+  int B, T, H, d, L, W, chain;
 };
 
 // One step of the residual chain.  Exact form (gist.science PRISM explainer, 2.2

@@ -17,6 +17,9 @@ cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t st
 cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, cudaStream_t stream);
 size_t bwd_smem_bytes(int d_k, int d_v, int L);
 int bwd_row_blocks(int d_k, int d_v);
+bool chunk_bwd_supported(int d_k, int d_v, int L);
+size_t chunk_bwd_smem_bytes(int d);
+cudaError_t launch_chunk_bwd(const ChunkBwdParams& p, int dtype, cudaStream_t stream);
 }  // namespace prism
 
 namespace {
@@ -299,8 +302,32 @@ int prism_decode_step(const void* q, const void* k, const void* v, const float* 
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
+namespace {
+
+// Workspace of the chunked backward: the forward and adjoint records (fp32).
+struct ChunkBwdWs {
+  size_t states, psi, Hn, gk, gu, hs, part, total;
+  ChunkBwdWs(int B, int T, int H, int d, int L, int W) {
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t NC = (size_t)(T + prism::kBwdChunk - 1) / prism::kBwdChunk;
+    const size_t tok = (size_t)B * T * H;
+    size_t o = 0;
+    states = o; o += al((size_t)B * H * (NC + 1) * d * d * 4);
+    Hn = o;     o += al((size_t)B * H * NC * d * d * 4);
+    psi = o;    o += al(tok * d * 4);
+    gk = o;     o += al(tok * d * 4);
+    gu = o;     o += al(tok * (size_t)(L - 1) * d * 4);
+    hs = o;     o += al((size_t)B * H * NC * d * 4);
+    part = o;   o += al((size_t)B * NC * H * d * W * 4);
+    total = o;
+  }
+};
+
+}  // namespace
+
 size_t prism_scan_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int dtype) {
   if (check_sizes(B, T, H, d_k, d_v, L, W, 16, dtype) != PRISM_OK) return 0;
+  if (prism::chunk_bwd_supported(d_k, d_v, L)) return ChunkBwdWs(B, T, H, d_k, L, W).total;
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t nv = (size_t)(L + 1) * d_k + (L + 1);
   return al((size_t)B * H * T * d_v * d_k * 4) + al((size_t)B * H * d_v * W * 4) +
@@ -325,7 +352,8 @@ int prism_scan_bwd(const void* q, const void* k, const void* v, const float* gam
                         L > 1 ? dgain : nullptr};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return PRISM_ERR_UNSUPPORTED;
-  if (prism::bwd_smem_bytes(d_k, d_v, L) > 227u * 1024u) return PRISM_ERR_UNSUPPORTED;
+  if (!prism::chunk_bwd_supported(d_k, d_v, L) && prism::bwd_smem_bytes(d_k, d_v, L) > 227u * 1024u)
+    return PRISM_ERR_UNSUPPORTED;
   const size_t need = prism_scan_bwd_workspace_size(B, T, H, d_k, d_v, L, W, dtype);
   if (!workspace || workspace_bytes < need) return PRISM_ERR_WORKSPACE;
   int* status = nullptr;
@@ -339,6 +367,28 @@ int prism_scan_bwd(const void* q, const void* k, const void* v, const float* gam
                   {dbeta, toks * 4}, {du, toks * m * d_k * 4}, {dalpha, toks * m * 4}, {dgain, toks * m * d_v * 4}};
   for (const Z& z : zs)
     if (z.p && z.bytes && cudaMemsetAsync(z.p, 0, z.bytes, s) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (prism::chunk_bwd_supported(d_k, d_v, L)) {
+    // chunked backward: forward records at chunk boundaries, the adjoint pass, then
+    // every chunk's gradients in parallel
+    const ChunkBwdWs ws(B, T, H, d_k, L, W);
+    char* wsb = static_cast<char*>(workspace);
+    float* rec_states = reinterpret_cast<float*>(wsb + ws.states);
+    float* rec_psi = reinterpret_cast<float*>(wsb + ws.psi);
+    prism::ScanParams fp{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr,
+                         L > 1 ? gain : nullptr, conv_w, S0, lengths, nullptr, nullptr, B, T, H, d_k, d_v, L, W, 16,
+                         status, g_spin_limit.load(), chain, nullptr, nullptr, rec_states, rec_psi};
+    cudaError_t err = prism::launch_recurrent_scan(fp, dtype, s);
+    if (err != cudaSuccess) return PRISM_ERR_CUDA;
+    prism::ChunkBwdParams cp{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr,
+                             L > 1 ? gain : nullptr, conv_w, lengths, dO, dS_final, rec_states, rec_psi,
+                             reinterpret_cast<float*>(wsb + ws.Hn), reinterpret_cast<float*>(wsb + ws.gk),
+                             reinterpret_cast<float*>(wsb + ws.gu), reinterpret_cast<float*>(wsb + ws.hs),
+                             reinterpret_cast<float*>(wsb + ws.part), dq, dk, dv, dgamma, dbeta,
+                             L > 1 ? du : nullptr, L > 1 ? dalpha : nullptr, L > 1 ? dgain : nullptr, dconv_w, dS0,
+                             B, T, H, d_k, L, W, chain};
+    err = prism::launch_chunk_bwd(cp, dtype, s);
+    return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+  }
   float* states = static_cast<float*>(workspace);
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   char* wsb = static_cast<char*>(workspace);

@@ -24,7 +24,8 @@ namespace prism {
 namespace {
 
 constexpr int kBlock = 64;
-constexpr int kTileBytes = 48 * 1024;  // per buffer
+constexpr int kTileBytes = 48 * 1024;    // per buffer
+constexpr int kRecTileBytes = 8 * 1024;  // per buffer, recording launches of the chunked backward
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
@@ -87,9 +88,9 @@ struct TileLayout {
 };
 
 template <typename T>
-int tile_tokens(int dk, int m, int rpb) {
+int tile_tokens(int dk, int m, int rpb, int budget) {
   for (int TT = 32; TT > 1; TT >>= 1)
-    if (TileLayout(TT, dk, m, rpb, sizeof(T)).bytes <= kTileBytes) return TT;
+    if (TileLayout(TT, dk, m, rpb, sizeof(T)).bytes <= budget) return TT;
   return 1;
 }
 
@@ -189,6 +190,14 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
     s[e] = f.x; s[e + 1] = f.y; s[e + 2] = f.z; s[e + 3] = f.w;
   }
 
+  const int NCr = (T_ + kBwdChunk - 1) / kBwdChunk;  // chunk-boundary record slots: NCr + 1
+  float* rec_row = p.rec_states ? p.rec_states + (((size_t)b * H + h) * (NCr + 1) * dv + c) * dk + EPL * j : nullptr;
+  if (rec_row && row_ok) {
+#pragma unroll
+    for (int e = 0; e < EPL; e += 4)
+      *reinterpret_cast<float4*>(rec_row + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+  }
+
   const int ntiles = (len + TT - 1) / TT;
   if (ntiles > 0) load_tile(0, 0);
   cp_async_commit();
@@ -231,7 +240,9 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
 
       // gated delta write: gamma S (I - beta k k^T) + beta v k^T
       const float gam = sgam[i];
-      const float coef = sbet[i] * (vt - gam * sk);
+      const float psi = vt - gam * sk;
+      const float coef = sbet[i] * psi;
+      if (p.rec_psi && row_ok && j == 0) p.rec_psi[(((size_t)b * T_ + t0 + i) * H + h) * dv + c] = psi;
 #pragma unroll
       for (int e = 0; e < EPL; e += 4) {
         const float4 f = ld4_smem<T>(kk + e);
@@ -253,6 +264,13 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
           s[e + 2] += rho * f.z;
           s[e + 3] += rho * f.w;
         }
+      }
+      const int tn = t0 + i + 1;  // tokens done
+      if (rec_row && row_ok && (tn % kBwdChunk == 0 || tn == len)) {  // a chunk boundary
+        float* dst = rec_row + (size_t)((tn + kBwdChunk - 1) / kBwdChunk) * dv * dk;
+#pragma unroll
+        for (int e = 0; e < EPL; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
       }
       if (p.states && row_ok) {  // S_t of this row, for the backward pass
         float* dst = p.states + ((((size_t)b * H + h) * T_ + t0 + i) * dv + c) * dk + EPL * j;
@@ -285,7 +303,9 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
 template <typename T, int LPR, int EPL, int CH>
 cudaError_t launch_chain(const ScanParams& p, cudaStream_t stream) {
   constexpr int RPB = kBlock / LPR;
-  const int TT = tile_tokens<T>(p.d_k, p.L - 1, RPB);
+  // the chunked backward launches this kernel over every (batch, head) row block at
+  // once: small tiles keep all of them resident (one wave)
+  const int TT = tile_tokens<T>(p.d_k, p.L - 1, RPB, p.rec_states ? kRecTileBytes : kTileBytes);
   const int smem = 2 * TileLayout(TT, p.d_k, p.L - 1, RPB, sizeof(T)).bytes;
   cudaError_t err = cudaFuncSetAttribute(recurrent_scan_kernel<T, LPR, EPL, CH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

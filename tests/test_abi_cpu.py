@@ -160,9 +160,19 @@ def test_backward_invalid_arguments(L, kw, code):
 
 
 def test_backward_workspace_size(L):
-    # every state S_t (fp32) + dconv_w partials + per-token row-block sums, each 256-byte aligned
-    B, T, H, d, Lc, W = 2, 10, 3, 64, 4, 4
     al = lambda x: (x + 255) // 256 * 256
-    nv = (Lc + 1) * d + (Lc + 1)
-    expect = al(B * H * T * d * d * 4) + al(B * H * d * W * 4) + al(B * T * H * 2 * nv * 4)
+    # token-by-token path (d_k != d_v here): every state S_t (fp32) + dconv_w partials +
+    # per-token row-block sums, each 256-byte aligned
+    B, T, H, dk, dv, Lc, W = 2, 10, 3, 64, 32, 4, 4
+    nv = (Lc + 1) * dk + (Lc + 1)
+    expect = al(B * H * T * dv * dk * 4) + al(B * H * dv * W * 4) + al(B * T * H * 1 * nv * 4)
+    assert prism.lib().prism_scan_bwd_workspace_size(B, T, H, dk, dv, Lc, W, 0) == expect
+    # chunked path (d_k = d_v = 64, L <= 4): boundary states (NC + 1 per chain), H_n (NC per
+    # chain), psi, gk, gu per token, <H_n, S_{n+1}> row partials, per-chunk dconv partials
+    B, T, H, d, Lc, W = 2, 130, 3, 64, 4, 4
+    NC = 3
+    expect = (al(B * H * (NC + 1) * d * d * 4) + al(B * H * NC * d * d * 4) + al(B * T * H * d * 4) * 2 +
+              al(B * T * H * (Lc - 1) * d * 4) + al(B * H * NC * d * 4) + al(B * NC * H * d * W * 4))
     assert prism.lib().prism_scan_bwd_workspace_size(B, T, H, d, d, Lc, W, 0) == expect
+    # far smaller than recording every state: 9.6 MB against 134 MB at T = 2048, B = H = 1, d = 128
+    assert prism.lib().prism_scan_bwd_workspace_size(1, 2048, 1, 128, 128, 4, 4, 0) < 10_000_000

@@ -27,7 +27,24 @@ CASES = {
 }
 
 
-def _run(w, chain, seed=5):
+# d_k = d_v in {64, 128} and L <= 4 take the chunked backward (64-token chunks):
+# several chunks, a ragged last chunk, lengths ending mid-chunk, on a chunk edge, and
+# sequences shorter than the ShortConv window behind a chunk start.
+CHUNKED = {
+    "chunked_bf16_d128_L4": (synth.Workload("f", B=2, T=200, H=2, d_k=128, d_v=128, L=4, chunk=64, W=4,
+                                            lengths_lo=60, with_s0=True, seed=21), "linear"),
+    "chunked_fp32_d64_L3_gelu": (synth.Workload("g", B=3, T=150, H=2, d_k=64, d_v=64, L=3, chunk=64, W=8,
+                                                dtype="fp32", lengths_lo=1, with_s0=True, seed=22), "gelu"),
+    "chunked_bf16_d64_L1": (synth.Workload("h", B=2, T=129, H=3, d_k=64, d_v=64, L=1, chunk=64, W=3,
+                                           seed=23), "linear"),
+    "chunked_fp32_d128_L2_W1": (synth.Workload("i", B=1, T=256, H=1, d_k=128, d_v=128, L=2, chunk=64, W=1,
+                                               dtype="fp32", seed=24), "linear"),
+    "chunked_bf16_d128_L3_gelu_edges": (synth.Workload("j", B=4, T=192, H=1, d_k=128, d_v=128, L=3, chunk=64,
+                                                       W=4, lengths_lo=64, with_s0=True, seed=25), "gelu"),
+}
+
+
+def _run(w, chain, seed=5, lengths=None):
     import linear_attention_sequence_shortconv_b200 as prism
 
     inp = synth.make_inputs(w)
@@ -37,6 +54,8 @@ def _run(w, chain, seed=5):
     gen = torch.Generator().manual_seed(seed)
     dO = torch.randn((w.B, w.T, w.H, w.d_v), generator=gen).to(inp["v"].dtype)
     dSf = torch.randn((w.B, w.H, w.d_v, w.d_k), generator=gen)
+    if lengths is not None:
+        inp["lengths"] = torch.tensor(lengths, dtype=torch.int32)
     d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
     g = prism.scan_bwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"], d["conv_w"],
                        dO.cuda(), L=w.L, S0=d["S0"], lengths=d["lengths"], dS_final=dSf.cuda(), chain=chain)
@@ -78,3 +97,41 @@ def test_backward_long_chain_full_width():
     ref = prism_seq_grad(**x, dO=dO.double().numpy(), dS_final=dSf.double().numpy())
     for n, r in ref.items():
         assert _rel(got[n], r) <= TOL, (n, _rel(got[n], r))
+
+
+# lengths on a chunk edge (64, 128), one token into a chunk (65), one short of it (127)
+EDGE_LENGTHS = {"chunked_bf16_d128_L3_gelu_edges": [64, 65, 127, 128]}
+
+
+@pytest.mark.parametrize("name", list(CHUNKED))
+def test_chunked_backward_matches_oracle(name):
+    w, chain = CHUNKED[name]
+    inp, dO, dSf, got = _run(w, chain, lengths=EDGE_LENGTHS.get(name))
+    x = synth.to_float64_numpy(inp)
+    if w.L == 1:
+        x["u"] = x["alpha"] = x["gain"] = None
+    ref = prism_seq_grad(**x, dO=dO.double().numpy(), dS_final=dSf.double().numpy(), chain=chain)
+    for n, r in ref.items():
+        assert got[n].shape == r.shape, (n, got[n].shape, r.shape)
+        assert _rel(got[n], r) <= TOL, (name, n, _rel(got[n], r))
+
+
+def test_chunked_backward_strong_decay():
+    """gamma around 0.3: dgamma comes out of gamma_t dgamma_t divided by gamma_t."""
+    w = synth.Workload("k", B=1, T=130, H=2, d_k=64, d_v=64, L=3, chunk=64, W=4, dtype="fp32", with_s0=True,
+                       seed=26)
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    inp = synth.make_inputs(w)
+    gg = torch.Generator().manual_seed(27)
+    inp["gamma"] = torch.sigmoid(torch.randn(inp["gamma"].shape, generator=gg) - 1.0)
+    gen = torch.Generator().manual_seed(5)
+    dO = torch.randn((w.B, w.T, w.H, w.d_v), generator=gen)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    g = prism.scan_bwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"], d["conv_w"],
+                       dO.cuda(), L=w.L, S0=d["S0"], lengths=d["lengths"])
+    torch.cuda.synchronize()
+    x = synth.to_float64_numpy(inp)
+    ref = prism_seq_grad(**x, dO=dO.double().numpy())
+    for n, r in ref.items():
+        assert _rel(g[n].cpu().numpy().astype(np.float64), r) <= TOL, (n,)
