@@ -296,11 +296,16 @@ def run_ours_bwd(args, w):
         torch.cuda.synchronize()
     ms = sum(a.elapsed_time(b) for a, b in ev) / K
     work = algorithmic_work_bwd(w, host_inputs["lengths"].numpy() if host_inputs["lengths"] is not None else None)
+    # d_k = d_v in {64, 128}, L <= 4: the chunked backward; otherwise the token-by-token one
+    chunked = w.d_k == w.d_v and w.d_k in (64, 128) and w.L <= 4
+    bwd_kernel = "chunk_grad" if chunked else "scan_bwd"
+    bwd_timed = ("step = forward recording chunk-boundary states + adjoint pass + per-chunk gradients "
+                 "+ dconv_w reduction" if chunked else "step = recording forward + reverse kernel + two reductions")
     peaks, peak_kind = load_peaks()
     achieved = work["bytes"] / (ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "scan_bwd",
-                "timed": "step = recording forward + reverse kernel + two reductions",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": bwd_kernel,
+                "timed": bwd_timed,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS hbm_gbs burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_launch": work["bytes"]}
     cpu_baseline = None

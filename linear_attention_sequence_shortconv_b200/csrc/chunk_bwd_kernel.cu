@@ -282,8 +282,9 @@ __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams 
 
 // ------------------------------------------------------------------ per-chunk gradients
 
-constexpr int kGradThreads = 256;  // 16 x 16 thread grid over every tile
+constexpr int kGradThreads = 256;  // 8 warps
 constexpr int kHalo = PRISM_MAX_W - 1;
+constexpr int kStageRows = 16;     // rows of a B operand per stage of the cp.async ring
 
 // Shared-memory layout of chunk_grad_kernel (float offsets).  Rows are padded by 4
 // floats so that float4 reads of 16 different rows hit different banks.
@@ -307,36 +308,87 @@ struct GradLayout {
   static constexpr int QDQ = BE + C;                // q_t . dq_t
   static constexpr int WT = QDQ + C;                // w_t
   static constexpr int RED = WT + C;                // scratch for reductions
-  static constexpr int FLOATS = RED + 32;
+  static constexpr int STAGE = RED + 32;            // B-operand ring: 2 stages x 2 sources x kStageRows x D
+  static constexpr int FLOATS = STAGE + 2 * 2 * kStageRows * D;
   static constexpr size_t BYTES = (size_t)FLOATS * 4;
 };
 
-// acc[r][s4*4 + e] += sum_k A(row_r, k) * B(k, col), rows ty + 16 r, columns
-// 4 tx + 64 s4 + e.  A is a C x K tile in shared memory (row stride lda) read
-// four k at a time, B a K x D row-major matrix in global fp32 memory.
+// Thread mapping of the C x D products: lane % (D / 4) owns columns 4 cg .. 4 cg + 3,
+// the warp (and, for D = 64, lane / 16) owns rows r0 + 8 NRW r; A values are then
+// shared by the whole row group and each stage row of B is read once per warp,
+// conflict-free.
 template <int D>
-__device__ __forceinline__ void gemm_smemA_globalB(float (&acc)[4][D / 16], const float* sA, int lda,
-                                                   const float* gB, int K, int ty, int tx) {
-  for (int k = 0; k < K; k += 4) {
-    float4 a[4];
+struct RowMap {
+  static constexpr int NRW = 128 / D;        // row groups per warp
+  static constexpr int RT = kBwdChunk / (8 * NRW);  // rows per thread
+  int cg, r0;
+  __device__ RowMap(int warp, int lane) : cg(lane % (D / 4)), r0(warp * NRW + lane / (D / 4)) {}
+  __device__ int row(int r) const { return r0 + 8 * NRW * r; }
+};
+
+// Copy rows [st * kStageRows, +kStageRows) of a K x D row-major matrix (row stride ldb,
+// element type TB) into one stage of the ring; rows at or past K are zero-filled.
+template <int D, typename TB>
+__device__ __forceinline__ void stage_rows(TB* dst, const TB* src, size_t ldb, int st, int K, int tid) {
+  constexpr int V = 16 / (int)sizeof(TB);
+  const int r0 = st * kStageRows;
+  for (int e = tid; e < kStageRows * (D / V); e += kGradThreads) {
+    const int rr = e / (D / V), cc = (e % (D / V)) * V;
+    TB* d = dst + rr * D + cc;
+    if (r0 + rr < K)
+      cp_async16(d, src + (size_t)(r0 + rr) * ldb + cc);
+    else
+      *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// acc_s[r][e] += sum_{k < K} A_s(row r, k) B_s[k][4 cg + e] for NS = 1 or 2 products
+// that share the k loop, with NB = 1 (one B for all) or NB = NS B operands.  B is in
+// global memory and streams through a two-stage cp.async ring in shared memory
+// (kStageRows rows per stage); A_s is read from shared memory by `a(s, r, k)`.  K
+// may be any value <= the rows of B (the rest of the last stage is zero).  Every
+// thread of the block must call it.
+template <int D, int NS, int NB, typename TB, class AF>
+__device__ __forceinline__ void staged_gemm(float (&acc)[NS][RowMap<D>::RT][4], const AF& a, const TB* gB0,
+                                            const TB* gB1, size_t ldb, int K, TB* ring, const RowMap<D>& rm,
+                                            int tid) {
+  static_assert(NB == 1 || NB == NS, "one B operand, or one per product");
+  constexpr int RT = RowMap<D>::RT;
+  constexpr int SZ = kStageRows * D;  // elements per source per stage
+  const int nst = (K + kStageRows - 1) / kStageRows;
+  auto issue = [&](int st) {
+    TB* base = ring + (st & 1) * NB * SZ;
+    stage_rows<D, TB>(base, gB0, ldb, st, K, tid);
+    if (NB == 2) stage_rows<D, TB>(base + SZ, gB1, ldb, st, K, tid);
+  };
+  issue(0);
+  cp_async_commit();
+  for (int st = 0; st < nst; ++st) {
+    if (st + 1 < nst) issue(st + 1);
+    cp_async_commit();
+    cp_async_wait_1();
+    __syncthreads();
+    const TB* base = ring + (st & 1) * NB * SZ;
+#pragma unroll 4
+    for (int kk = 0; kk < kStageRows; ++kk) {
+      const int k = st * kStageRows + kk;
+      const float4 b0 = lds4<TB>(base + kk * D + 4 * rm.cg);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) a[r] = *reinterpret_cast<const float4*>(sA + (ty + 16 * r) * lda + k);
+      for (int s = 0; s < NS; ++s) {
+        const float4 bv = (NB == 1 || s == 0) ? b0 : lds4<TB>(base + SZ + kk * D + 4 * rm.cg);
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-      for (int s4 = 0; s4 < D / 64; ++s4) {
-        const float4 bv = __ldg(reinterpret_cast<const float4*>(gB + (size_t)(k + kk) * D + 4 * tx + 64 * s4));
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const float av = kk == 0 ? a[r].x : (kk == 1 ? a[r].y : (kk == 2 ? a[r].z : a[r].w));
-          acc[r][4 * s4] += av * bv.x;
-          acc[r][4 * s4 + 1] += av * bv.y;
-          acc[r][4 * s4 + 2] += av * bv.z;
-          acc[r][4 * s4 + 3] += av * bv.w;
+        for (int r = 0; r < RT; ++r) {
+          const float av = a(s, r, k);
+          acc[s][r][0] += av * bv.x;
+          acc[s][r][1] += av * bv.y;
+          acc[s][r][2] += av * bv.z;
+          acc[s][r][3] += av * bv.w;
         }
       }
     }
+    __syncthreads();  // this stage is refilled two stages on
   }
+  cp_async_wait_0();
 }
 
 template <typename T, int D, int M, int CH>
@@ -447,20 +499,32 @@ __global__ void __launch_bounds__(kGradThreads) chunk_grad_kernel(ChunkBwdParams
   };
 
   // ---- dq = diag(e^c) dO S_n + ..., F = diag(e^c) gk S_n + ...
-  float adq[4][TN], aF[4][TN];
+  const RowMap<D> rm(warp, lane);
+  constexpr int RT = RowMap<D>::RT;
+  float acc[2][RT][4];  // [0] dq, [1] F
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+  for (int s = 0; s < 2; ++s)
 #pragma unroll
-    for (int e = 0; e < TN; ++e) adq[r][e] = aF[r][e] = 0.f;
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[s][r][e] = 0.f;
   const float* Sn = p.states + (bh * (NC + 1) + n) * D * D;
   const float* Hn = p.Hn + (bh * NC + n) * D * D;
-  gemm_smemA_globalB<D>(adq, sDO, LDD, Sn, D, ty, tx);
-  gemm_smemA_globalB<D>(aF, sGK, LDD, Sn, D, ty, tx);
+  float* ringf = sm + Ly::STAGE;
+  T* ringt = reinterpret_cast<T*>(sm + Ly::STAGE);
+  {
+    // both products share B = S_n
+    auto aSn = [&](int s, int r, int kx) { return (s == 0 ? sDO : sGK)[rm.row(r) * LDD + kx]; };
+    staged_gemm<D, 2, 1, float>(acc, aSn, Sn, Sn, D, D, ringf, rm, tid);
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const float ec = sec[ty + 16 * r];
+    for (int r = 0; r < RT; ++r) {
+      const float ec = sec[rm.row(r)];
 #pragma unroll
-    for (int e = 0; e < TN; ++e) { adq[r][e] *= ec; aF[r][e] *= ec; }
+      for (int e = 0; e < 4; ++e) {
+        acc[0][r][e] *= ec;
+        acc[1][r][e] *= ec;
+      }
+    }
   }
 
   for (int a = 0; a <= M; ++a) {
@@ -482,7 +546,8 @@ __global__ void __launch_bounds__(kGradThreads) chunk_grad_kernel(ChunkBwdParams
       *reinterpret_cast<float4*>(sX + t * LDD + c4) = x;
     }
     __syncthreads();
-    // Grams P = dO X_a^T, Pf = gk X_a^T (C x C over D), masked and decayed into M_a, N_a
+    // Grams P = dO X_a^T, Pf = gk X_a^T (C x C over D), masked and decayed into M_a, N_a;
+    // 16 x 16 threads, rows ty + 16 r and columns tx + 16 s
     {
       float gp[4][4], gf[4][4];
 #pragma unroll
@@ -519,108 +584,75 @@ __global__ void __launch_bounds__(kGradThreads) chunk_grad_kernel(ChunkBwdParams
       }
     }
     __syncthreads();
-    // dq += M_a Y_a, F += N_a Y_a  (Y_0 = K, Y_l = U_l; rows past nt never read)
-    const T* Y = a == 0 ? k : u;
-    const size_t ystride = a == 0 ? (size_t)H * D : (size_t)H * M * D;
-    const T* Y0 = a == 0 ? k + tokidx(0) * D : u + (tokidx(0) * M + (a - 1)) * D;
-    (void)Y;
-    for (int i = 0; i < nt; ++i) {
-      float am[4], an[4];
+    // dq += M_a Y_a, F += N_a Y_a  (Y_0 = K, Y_l = U_l; B rows past nt are zero-filled)
+    {
+      const size_t ystride = a == 0 ? (size_t)H * D : (size_t)H * M * D;
+      const T* Y0 = a == 0 ? k + tokidx(0) * D : u + (tokidx(0) * M + (a - 1)) * D;
+      auto aMN = [&](int s, int r, int i) { return (s == 0 ? sM : sN)[rm.row(r) * LDC + i]; };
+      float t2[2][RT][4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        am[r] = sM[(ty + 16 * r) * LDC + i];
-        an[r] = sN[(ty + 16 * r) * LDC + i];
-      }
+      for (int s = 0; s < 2; ++s)
 #pragma unroll
-      for (int s4 = 0; s4 < D / 64; ++s4) {
-        const float4 bv = ld4<T>(Y0 + i * ystride + 4 * tx + 64 * s4);
+        for (int r = 0; r < RT; ++r)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          adq[r][4 * s4] += am[r] * bv.x; adq[r][4 * s4 + 1] += am[r] * bv.y;
-          adq[r][4 * s4 + 2] += am[r] * bv.z; adq[r][4 * s4 + 3] += am[r] * bv.w;
-          aF[r][4 * s4] += an[r] * bv.x; aF[r][4 * s4 + 1] += an[r] * bv.y;
-          aF[r][4 * s4 + 2] += an[r] * bv.z; aF[r][4 * s4 + 3] += an[r] * bv.w;
-        }
-      }
+          for (int e = 0; e < 4; ++e) t2[s][r][e] = 0.f;
+      staged_gemm<D, 2, 1, T>(t2, aMN, Y0, Y0, ystride, nt, ringt, rm, tid);
+#pragma unroll
+      for (int s = 0; s < 2; ++s)
+#pragma unroll
+        for (int r = 0; r < RT; ++r)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[s][r][e] += t2[s][r][e];
     }
     // Gx_a = diag(e^{c_C - c}) X_a H_n + M_a^T Q - (diag(beta) N_a)^T K
     {
-      float ag[4][TN];
+      float gx[1][RT][4], t2[2][RT][4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < RT; ++r)
 #pragma unroll
-        for (int e = 0; e < TN; ++e) ag[r][e] = 0.f;
-      gemm_smemA_globalB<D>(ag, sX, LDD, Hn, D, ty, tx);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float ec = secc[ty + 16 * r];
-#pragma unroll
-        for (int e = 0; e < TN; ++e) ag[r][e] *= ec;
-      }
-      const T* Q0 = q + tokidx(0) * D;
-      const T* K0 = k + tokidx(0) * D;
-      const size_t qs = (size_t)H * D;
-      for (int jj = 0; jj < nt; ++jj) {
-        float am[4], an[4];
-        const float be = sbe[jj];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          am[r] = sM[jj * LDC + ty + 16 * r];
-          an[r] = -be * sN[jj * LDC + ty + 16 * r];
-        }
-#pragma unroll
-        for (int s4 = 0; s4 < D / 64; ++s4) {
-          const float4 qv = ld4<T>(Q0 + jj * qs + 4 * tx + 64 * s4);
-          const float4 kv = ld4<T>(K0 + jj * qs + 4 * tx + 64 * s4);
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            ag[r][4 * s4] += am[r] * qv.x + an[r] * kv.x;
-            ag[r][4 * s4 + 1] += am[r] * qv.y + an[r] * kv.y;
-            ag[r][4 * s4 + 2] += am[r] * qv.z + an[r] * kv.z;
-            ag[r][4 * s4 + 3] += am[r] * qv.w + an[r] * kv.w;
-          }
-        }
-      }
+        for (int e = 0; e < 4; ++e) gx[0][r][e] = t2[0][r][e] = t2[1][r][e] = 0.f;
+      auto aX = [&](int, int r, int kx) { return sX[rm.row(r) * LDD + kx]; };
+      staged_gemm<D, 1, 1, float>(gx, aX, Hn, Hn, D, D, ringf, rm, tid);
+      auto aT = [&](int s, int r, int j) {
+        return s == 0 ? sM[j * LDC + rm.row(r)] : -sbe[j] * sN[j * LDC + rm.row(r)];
+      };
+      staged_gemm<D, 2, 2, T>(t2, aT, q + tokidx(0) * D, k + tokidx(0) * D, (size_t)H * D, nt, ringt, rm, tid);
       // a = 0: G_t^T delta_t, kept in dk until F is complete; a = l: du_l
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int t = ty + 16 * r;
-        if (t >= nt) continue;
-#pragma unroll
-        for (int s4 = 0; s4 < D / 64; ++s4) {
-          float* dst = a == 0 ? p.dk + tokidx(t) * D : p.du + (tokidx(t) * M + (a - 1)) * D;
-          *reinterpret_cast<float4*>(dst + 4 * tx + 64 * s4) =
-              make_float4(ag[r][4 * s4], ag[r][4 * s4 + 1], ag[r][4 * s4 + 2], ag[r][4 * s4 + 3]);
+      for (int r = 0; r < RT; ++r) {
+        const int t = rm.row(r);
+        const float ec = secc[t];
+        if (t < nt) {
+          float* dst = (a == 0 ? p.dk + tokidx(t) * D : p.du + (tokidx(t) * M + (a - 1)) * D) + 4 * rm.cg;
+          *reinterpret_cast<float4*>(dst) =
+              make_float4(ec * gx[0][r][0] + t2[0][r][0] + t2[1][r][0], ec * gx[0][r][1] + t2[0][r][1] + t2[1][r][1],
+                          ec * gx[0][r][2] + t2[0][r][2] + t2[1][r][2], ec * gx[0][r][3] + t2[0][r][3] + t2[1][r][3]);
         }
       }
     }
     __syncthreads();  // sX, sM, sN are rewritten by the next a
   }
 
-  // ---- dq, dk = G^T delta - diag(beta) F, q_t . dq_t
+  // ---- dq, dk = G^T delta - diag(beta) F, q_t . dq_t (row sums over the D / 4 lanes of a row)
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int t = ty + 16 * r;
+  for (int r = 0; r < RT; ++r) {
+    const int t = rm.row(r);
     float qd = 0.f;
     if (t < nt) {
       const float be = sbe[t];
-#pragma unroll
-      for (int s4 = 0; s4 < D / 64; ++s4) {
-        const int col = 4 * tx + 64 * s4;
-        const float4 qv = ld4<T>(q + tokidx(t) * D + col);
-        qd += qv.x * adq[r][4 * s4] + qv.y * adq[r][4 * s4 + 1] + qv.z * adq[r][4 * s4 + 2] +
-              qv.w * adq[r][4 * s4 + 3];
-        *reinterpret_cast<float4*>(p.dq + tokidx(t) * D + col) =
-            make_float4(adq[r][4 * s4], adq[r][4 * s4 + 1], adq[r][4 * s4 + 2], adq[r][4 * s4 + 3]);
-        float4* dk4 = reinterpret_cast<float4*>(p.dk + tokidx(t) * D + col);
-        const float4 gx = *dk4;  // this thread's own store above
-        *dk4 = make_float4(gx.x - be * aF[r][4 * s4], gx.y - be * aF[r][4 * s4 + 1], gx.z - be * aF[r][4 * s4 + 2],
-                           gx.w - be * aF[r][4 * s4 + 3]);
-      }
+      const int col = 4 * rm.cg;
+      const float4 qv = ld4<T>(q + tokidx(t) * D + col);
+      qd = qv.x * acc[0][r][0] + qv.y * acc[0][r][1] + qv.z * acc[0][r][2] + qv.w * acc[0][r][3];
+      *reinterpret_cast<float4*>(p.dq + tokidx(t) * D + col) =
+          make_float4(acc[0][r][0], acc[0][r][1], acc[0][r][2], acc[0][r][3]);
+      float4* dk4 = reinterpret_cast<float4*>(p.dk + tokidx(t) * D + col);
+      const float4 gx = *dk4;  // this thread's own store above
+      *dk4 = make_float4(gx.x - be * acc[1][r][0], gx.y - be * acc[1][r][1], gx.z - be * acc[1][r][2],
+                         gx.w - be * acc[1][r][3]);
     }
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) qd += __shfl_xor_sync(0xffffffffu, qd, off);
-    if (tx == 0) sqdq[t] = qd;
+    for (int off = D / 8; off > 0; off >>= 1) qd += __shfl_xor_sync(0xffffffffu, qd, off);
+    if (rm.cg == 0) sqdq[t] = qd;
   }
 
   // ---- per token (one warp each): dbeta, dalpha, w_t, the chain backwards -> dr_0, dgain

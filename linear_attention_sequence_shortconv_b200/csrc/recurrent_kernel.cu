@@ -278,15 +278,17 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
         for (int e = 0; e < EPL; e += 4)
           *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
       }
-      const T* qq = sq_ + i * dk + EPL * j;
-      float oq = 0.f;
+      if (o) {  // no readout in the recording launches of the backward
+        const T* qq = sq_ + i * dk + EPL * j;
+        float oq = 0.f;
 #pragma unroll
-      for (int e = 0; e < EPL; e += 4) {
-        const float4 f = ld4_smem<T>(qq + e);
-        oq += s[e] * f.x + s[e + 1] * f.y + s[e + 2] * f.z + s[e + 3] * f.w;
+        for (int e = 0; e < EPL; e += 4) {
+          const float4 f = ld4_smem<T>(qq + e);
+          oq += s[e] * f.x + s[e + 1] * f.y + s[e + 2] * f.z + s[e + 3] * f.w;
+        }
+        oq = row_sum<LPR>(oq);
+        if (row_ok && j == 0) st1<T>(o + (((size_t)b * T_ + t0 + i) * H + h) * dv + c, oq);
       }
-      oq = row_sum<LPR>(oq);
-      if (o && row_ok && j == 0) st1<T>(o + (((size_t)b * T_ + t0 + i) * H + h) * dv + c, oq);
     }
     __syncthreads();  // the buffer is refilled next iteration
   }
