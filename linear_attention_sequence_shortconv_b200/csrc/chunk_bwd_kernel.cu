@@ -114,7 +114,9 @@ int adj_tile_tokens(int dk, int m, int rpb) {
 
 // One block: kAdjBlock / LPR rows of G for one (batch, head).  Rows of G are
 // independent (G is multiplied from the right by the transition), so row c only
-// needs the dot products (G k)_c and (G u_l)_c inside the row, over its LPR lanes.
+// needs the dot products (G k)_c and (G u_l)_c inside the row, over its LPR lanes;
+// lane j holds the columns 4 j + 4 LPR g + (0..3) (interleaved, so that the LPR lanes
+// of a row read one contiguous span of shared memory).
 // Tokens are walked from the last valid one down to 0, tiles streamed in reverse.
 template <typename T, int LPR, int EPL>
 __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams p, int TT) {
@@ -187,23 +189,23 @@ __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams 
   };
 
   float g[EPL];
-  const size_t gbase = (bh * dv + c) * dk + EPL * j;
+  const size_t gbase = (bh * dv + c) * dk + 4 * j;
 #pragma unroll
   for (int e = 0; e < EPL; e += 4) {
-    const float4 f = p.dS_final ? __ldg(reinterpret_cast<const float4*>(p.dS_final + gbase + e))
+    const float4 f = p.dS_final ? __ldg(reinterpret_cast<const float4*>(p.dS_final + gbase + e * LPR))
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
     g[e] = f.x; g[e + 1] = f.y; g[e + 2] = f.z; g[e + 3] = f.w;
   }
   // H_n (the gradient flowing into the end of chunk n from later tokens) and <H_n, S_{n+1}>
   auto record_boundary = [&](int n) {
-    const float* st = p.states + ((bh * (NC + 1) + n + 1) * dv + c) * dk + EPL * j;
-    float* hn = p.Hn + ((bh * NC + n) * dv + c) * dk + EPL * j;
+    const float* st = p.states + ((bh * (NC + 1) + n + 1) * dv + c) * dk + 4 * j;
+    float* hn = p.Hn + ((bh * NC + n) * dv + c) * dk + 4 * j;
     float dot = 0.f;
 #pragma unroll
     for (int e = 0; e < EPL; e += 4) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(st + e));
+      const float4 f = __ldg(reinterpret_cast<const float4*>(st + e * LPR));
       dot += g[e] * f.x + g[e + 1] * f.y + g[e + 2] * f.z + g[e + 3] * f.w;
-      if (row_ok) *reinterpret_cast<float4*>(hn + e) = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
+      if (row_ok) *reinterpret_cast<float4*>(hn + e * LPR) = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
     }
     dot = row_sum<LPR>(dot);
     if (row_ok && j == 0) p.hs[(bh * NC + n) * dv + c] = dot;
@@ -232,27 +234,27 @@ __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams 
       const size_t tok = ((size_t)b * T_ + t) * H + h;
       // G_t = (carry) + dO_t q_t^T
       const float dot_ = lds1<T>(sdo + i * RPB + cr);
-      const T* qq = sq_ + i * dk + EPL * j;
+      const T* qq = sq_ + i * dk + 4 * j;
 #pragma unroll
       for (int e = 0; e < EPL; e += 4) {
-        const float4 f = lds4<T>(qq + e);
+        const float4 f = lds4<T>(qq + e * LPR);
         g[e] += dot_ * f.x; g[e + 1] += dot_ * f.y; g[e + 2] += dot_ * f.z; g[e + 3] += dot_ * f.w;
       }
-      const T* kk = sk_ + i * dk + EPL * j;
+      const T* kk = sk_ + i * dk + 4 * j;
       float gk = 0.f;
 #pragma unroll
       for (int e = 0; e < EPL; e += 4) {
-        const float4 f = lds4<T>(kk + e);
+        const float4 f = lds4<T>(kk + e * LPR);
         gk += g[e] * f.x + g[e + 1] * f.y + g[e + 2] * f.z + g[e + 3] * f.w;
       }
       gk = row_sum<LPR>(gk);
       if (row_ok && j == 0) p.gk[tok * dv + c] = gk;
       for (int l = 0; l < m; ++l) {
-        const T* uu = su_ + ((size_t)i * m + l) * dk + EPL * j;
+        const T* uu = su_ + ((size_t)i * m + l) * dk + 4 * j;
         float gu = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; e += 4) {
-          const float4 f = lds4<T>(uu + e);
+          const float4 f = lds4<T>(uu + e * LPR);
           gu += g[e] * f.x + g[e + 1] * f.y + g[e + 2] * f.z + g[e + 3] * f.w;
         }
         gu = row_sum<LPR>(gu);
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams 
       const float gam = sgam[i], bg = sbet[i] * gk;
 #pragma unroll
       for (int e = 0; e < EPL; e += 4) {
-        const float4 f = lds4<T>(kk + e);
+        const float4 f = lds4<T>(kk + e * LPR);
         g[e] = gam * (g[e] - bg * f.x);
         g[e + 1] = gam * (g[e + 1] - bg * f.y);
         g[e + 2] = gam * (g[e + 2] - bg * f.z);
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams 
   if (row_ok) {
 #pragma unroll
     for (int e = 0; e < EPL; e += 4)
-      *reinterpret_cast<float4*>(p.dS0 + gbase + e) = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
+      *reinterpret_cast<float4*>(p.dS0 + gbase + e * LPR) = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
   }
 }
 

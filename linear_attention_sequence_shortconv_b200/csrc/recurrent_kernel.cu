@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   constexpr int RPB = kBlock / LPR;  // rows per block
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x;
-  const int j = tid % LPR;  // lane within the row: owns d_k elements EPL*j .. EPL*j+EPL-1
+  const int j = tid % LPR;  // lane within the row: owns d_k elements 4 j + 4 LPR g + (0..3), g < EPL / 4
   const int lrow = tid / LPR;
   const int row0 = blockIdx.x * RPB;
   const int row = row0 + lrow;
@@ -182,20 +182,20 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   for (int i = 0; i < PRISM_MAX_W; ++i) hist[i] = 0.f;
 
   float s[EPL];
-  const size_t sbase = (((size_t)b * H + h) * dv + c) * dk + EPL * j;
+  const size_t sbase = (((size_t)b * H + h) * dv + c) * dk + 4 * j;
 #pragma unroll
   for (int e = 0; e < EPL; e += 4) {
     const float4 f =
-        p.S0 ? __ldg(reinterpret_cast<const float4*>(p.S0 + sbase + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        p.S0 ? __ldg(reinterpret_cast<const float4*>(p.S0 + sbase + e * LPR)) : make_float4(0.f, 0.f, 0.f, 0.f);
     s[e] = f.x; s[e + 1] = f.y; s[e + 2] = f.z; s[e + 3] = f.w;
   }
 
   const int NCr = (T_ + kBwdChunk - 1) / kBwdChunk;  // chunk-boundary record slots: NCr + 1
-  float* rec_row = p.rec_states ? p.rec_states + (((size_t)b * H + h) * (NCr + 1) * dv + c) * dk + EPL * j : nullptr;
+  float* rec_row = p.rec_states ? p.rec_states + (((size_t)b * H + h) * (NCr + 1) * dv + c) * dk + 4 * j : nullptr;
   if (rec_row && row_ok) {
 #pragma unroll
     for (int e = 0; e < EPL; e += 4)
-      *reinterpret_cast<float4*>(rec_row + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+      *reinterpret_cast<float4*>(rec_row + e * LPR) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
   }
 
   const int ntiles = (len + TT - 1) / TT;
@@ -219,11 +219,11 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
     const int t0 = ti * TT, nt = min(TT, len - t0);
     const int cr = row_ok ? lrow : 0;
     for (int i = 0; i < nt; ++i) {
-      const T* kk = sk_ + i * dk + EPL * j;
+      const T* kk = sk_ + i * dk + 4 * j;
       float sk = 0.f;
 #pragma unroll
       for (int e = 0; e < EPL; e += 4) {
-        const float4 f = ld4_smem<T>(kk + e);
+        const float4 f = ld4_smem<T>(kk + e * LPR);
         sk += s[e] * f.x + s[e + 1] * f.y + s[e + 2] * f.z + s[e + 3] * f.w;
       }
       sk = row_sum<LPR>(sk);
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
       if (p.rec_psi && row_ok && j == 0) p.rec_psi[(((size_t)b * T_ + t0 + i) * H + h) * dv + c] = psi;
 #pragma unroll
       for (int e = 0; e < EPL; e += 4) {
-        const float4 f = ld4_smem<T>(kk + e);
+        const float4 f = ld4_smem<T>(kk + e * LPR);
         s[e] = gam * s[e] + coef * f.x;
         s[e + 1] = gam * s[e + 1] + coef * f.y;
         s[e + 2] = gam * s[e + 2] + coef * f.z;
@@ -255,10 +255,10 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
       for (int l = 0; l < m; ++l) {
         r = chain_step(r, to_f<T>(sg_[(i * m + l) * RPB + cr]), CH);
         const float rho = sal[i * m + l] * r;
-        const T* uu = su_ + ((size_t)i * m + l) * dk + EPL * j;
+        const T* uu = su_ + ((size_t)i * m + l) * dk + 4 * j;
 #pragma unroll
         for (int e = 0; e < EPL; e += 4) {
-          const float4 f = ld4_smem<T>(uu + e);
+          const float4 f = ld4_smem<T>(uu + e * LPR);
           s[e] += rho * f.x;
           s[e + 1] += rho * f.y;
           s[e + 2] += rho * f.z;
@@ -270,20 +270,20 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
         float* dst = rec_row + (size_t)((tn + kBwdChunk - 1) / kBwdChunk) * dv * dk;
 #pragma unroll
         for (int e = 0; e < EPL; e += 4)
-          *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+          *reinterpret_cast<float4*>(dst + e * LPR) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
       }
       if (p.states && row_ok) {  // S_t of this row, for the backward pass
-        float* dst = p.states + ((((size_t)b * H + h) * T_ + t0 + i) * dv + c) * dk + EPL * j;
+        float* dst = p.states + ((((size_t)b * H + h) * T_ + t0 + i) * dv + c) * dk + 4 * j;
 #pragma unroll
         for (int e = 0; e < EPL; e += 4)
-          *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+          *reinterpret_cast<float4*>(dst + e * LPR) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
       }
       if (o) {  // no readout in the recording launches of the backward
-        const T* qq = sq_ + i * dk + EPL * j;
+        const T* qq = sq_ + i * dk + 4 * j;
         float oq = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; e += 4) {
-          const float4 f = ld4_smem<T>(qq + e);
+          const float4 f = ld4_smem<T>(qq + e * LPR);
           oq += s[e] * f.x + s[e + 1] * f.y + s[e + 2] * f.z + s[e + 3] * f.w;
         }
         oq = row_sum<LPR>(oq);
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   if (row_ok && p.S_final) {
 #pragma unroll
     for (int e = 0; e < EPL; e += 4)
-      *reinterpret_cast<float4*>(p.S_final + sbase + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+      *reinterpret_cast<float4*>(p.S_final + sbase + e * LPR) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
   }
 }
 
