@@ -160,13 +160,23 @@ size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int 
  *   dgain [B,T,H,L-1,d_v] (all three NULL iff L == 1); dconv_w [H,d_v,W]; dS0 [B,H,d_v,d_k]
  *   (the gradient with respect to the initial state, zeros or S0).  Padded steps get zero
  *   gradients.
- * workspace: prism_scan_bwd_workspace_size() bytes: every state S_t of the forward
- *   (B*H*T*d_v*d_k fp32, recorded by a token-by-token forward launch) and partial sums.
- *   Results are deterministic.
- * workspace also holds per-token sums over row blocks (of 32 rows; 64 for d_k = 16) of the
- * gradients that are sums over rows (dq, dk, du, dgamma, dbeta, dalpha).
- * Sizes as prism_scan_fwd.  Four launches on `stream` (recording forward, reverse
- * recurrence, two deterministic reductions) after memsets of the outputs; no
+ * Two algorithms, chosen by shape; both compute in fp32 and are deterministic:
+ *   chunked (d_k = d_v in {64, 128}, L <= 4): a token-by-token forward records S at every
+ *     64-token chunk boundary and v_t - gamma_t S_{t-1} k_t; a reverse token-by-token
+ *     launch runs the adjoint recurrence G_t = dO_t q_t^T + gamma_{t+1} G_{t+1}
+ *     (I - beta_{t+1} k_{t+1} k_{t+1}^T) and records G_t k_t, G_t u_{t,l}, the gradient
+ *     entering every chunk end and its inner product with the state there; one launch
+ *     per chunk then forms every gradient of the chunk's tokens from those records; a
+ *     last launch adds the per-chunk dconv_w partials in a fixed order.  Workspace
+ *     (fp32): B*H*(2*NC+1)*d*d for the boundary states and gradients (NC = ceil(T/64)),
+ *     B*T*H*(L+1)*d for the per-token records, plus small per-chunk partials.
+ *   token-by-token (every other shape): a forward records every state S_t
+ *     (B*H*T*d_v*d_k fp32), a reverse launch walks the tokens, two launches reduce the
+ *     per-row-block partial sums (of 32 rows; 64 for d_k = 16) of the gradients that
+ *     are sums over rows (dq, dk, du, dgamma, dbeta, dalpha) and dconv_w.
+ * workspace: prism_scan_bwd_workspace_size() bytes (the chunked form: 0.54 GB for the
+ *   130M-LM layer, B=16 T=2048 H=6 d=128 L=4, against 12.9 GB token by token).
+ * Sizes as prism_scan_fwd.  Four launches on `stream` after memsets of the outputs; no
  * synchronisation.
  */
 size_t prism_scan_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int dtype);
