@@ -99,8 +99,20 @@ def test_backward_long_chain_full_width():
         assert _rel(got[n], r) <= TOL, (n, _rel(got[n], r))
 
 
-# lengths on a chunk edge (64, 128), one token into a chunk (65), one short of it (127)
-EDGE_LENGTHS = {"chunked_bf16_d128_L3_gelu_edges": [64, 65, 127, 128]}
+CHUNKED.update({
+    # an empty row, one token, a chunk and one more, and shorter than one chunk
+    "chunked_fp32_d64_L4_empty_rows": (synth.Workload("l", B=4, T=65, H=2, d_k=64, d_v=64, L=4, chunk=64, W=8,
+                                                      dtype="fp32", with_s0=True, seed=28), "linear"),
+    "chunked_bf16_d128_L2_T1": (synth.Workload("m", B=2, T=1, H=2, d_k=128, d_v=128, L=2, chunk=64, W=4,
+                                               with_s0=True, seed=29), "gelu"),
+    "chunked_bf16_d64_L3_T40": (synth.Workload("n", B=1, T=40, H=3, d_k=64, d_v=64, L=3, chunk=64, W=2,
+                                               seed=30), "linear"),
+})
+
+# lengths on a chunk edge (64, 128), one token into a chunk (65), one short of it (127);
+# an empty row (0), a single token (1)
+EDGE_LENGTHS = {"chunked_bf16_d128_L3_gelu_edges": [64, 65, 127, 128],
+                "chunked_fp32_d64_L4_empty_rows": [0, 1, 64, 65]}
 
 
 @pytest.mark.parametrize("name", list(CHUNKED))
