@@ -232,20 +232,19 @@ __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams 
     for (int i = nt - 1; i >= 0; --i) {
       const int t = t0 + i;
       const size_t tok = ((size_t)b * T_ + t) * H + h;
-      // G_t = (carry) + dO_t q_t^T
+      // G_t = (carry) + dO_t q_t^T, and gk = G_t k_t in the same pass (k kept for the carry)
       const float dot_ = lds1<T>(sdo + i * RPB + cr);
       const T* qq = sq_ + i * dk + 4 * j;
-#pragma unroll
-      for (int e = 0; e < EPL; e += 4) {
-        const float4 f = lds4<T>(qq + e * LPR);
-        g[e] += dot_ * f.x; g[e + 1] += dot_ * f.y; g[e + 2] += dot_ * f.z; g[e + 3] += dot_ * f.w;
-      }
       const T* kk = sk_ + i * dk + 4 * j;
+      float kr[EPL];
       float gk = 0.f;
 #pragma unroll
       for (int e = 0; e < EPL; e += 4) {
-        const float4 f = lds4<T>(kk + e * LPR);
-        gk += g[e] * f.x + g[e + 1] * f.y + g[e + 2] * f.z + g[e + 3] * f.w;
+        const float4 fq = lds4<T>(qq + e * LPR);
+        const float4 fk = lds4<T>(kk + e * LPR);
+        g[e] += dot_ * fq.x; g[e + 1] += dot_ * fq.y; g[e + 2] += dot_ * fq.z; g[e + 3] += dot_ * fq.w;
+        kr[e] = fk.x; kr[e + 1] = fk.y; kr[e + 2] = fk.z; kr[e + 3] = fk.w;
+        gk += g[e] * fk.x + g[e + 1] * fk.y + g[e + 2] * fk.z + g[e + 3] * fk.w;
       }
       gk = row_sum<LPR>(gk);
       if (row_ok && j == 0) p.gk[tok * dv + c] = gk;
@@ -263,13 +262,7 @@ __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams 
       // carry into token t - 1: gamma_t (G_t - beta_t (G_t k_t) k_t^T)
       const float gam = sgam[i], bg = sbet[i] * gk;
 #pragma unroll
-      for (int e = 0; e < EPL; e += 4) {
-        const float4 f = lds4<T>(kk + e * LPR);
-        g[e] = gam * (g[e] - bg * f.x);
-        g[e + 1] = gam * (g[e + 1] - bg * f.y);
-        g[e + 2] = gam * (g[e + 2] - bg * f.z);
-        g[e + 3] = gam * (g[e + 3] - bg * f.w);
-      }
+      for (int e = 0; e < EPL; ++e) g[e] = gam * (g[e] - bg * kr[e]);
       if (t > 0 && t % C == 0) record_boundary(t / C - 1);
     }
     __syncthreads();  // the buffer is refilled next iteration
