@@ -18,14 +18,15 @@
 // to them: tiles of TT tokens (k, q, u of the head; v and gains of the block's
 // rows; gamma, beta, alpha) stream into double-buffered shared memory with
 // cp.async while the previous tile is being scanned.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace prism {
 namespace {
 
 constexpr int kBlock = 64;
-constexpr int kTileBytes = 48 * 1024;    // per buffer
-constexpr int kRecTileBytes = 8 * 1024;  // per buffer, recording launches of the chunked backward
+constexpr int kTileBytes = 48 * 1024;  // per buffer, at most
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
@@ -302,17 +303,31 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   }
 }
 
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n = 148;
+  }
+  return n;
+}
+
 template <typename T, int LPR, int EPL, int CH>
 cudaError_t launch_chain(const ScanParams& p, cudaStream_t stream) {
   constexpr int RPB = kBlock / LPR;
-  // the chunked backward launches this kernel over every (batch, head) row block at
-  // once: small tiles keep all of them resident (one wave)
-  const int TT = tile_tokens<T>(p.d_k, p.L - 1, RPB, p.rec_states ? kRecTileBytes : kTileBytes);
+  // Every block walks the whole sequence, so all of them must be resident at once (a
+  // second wave would double the time): the double-buffered tile shrinks with the
+  // blocks each SM has to hold (about 200 KB of shared memory per SM in all).
+  dim3 grid((p.d_v + RPB - 1) / RPB, p.H, p.B);
+  const long long nblocks = (long long)grid.x * grid.y * grid.z;
+  const long long per_sm = (nblocks + sm_count() - 1) / sm_count();
+  const int budget = (int)std::min<long long>(kTileBytes, (200 * 1024) / (2 * std::max<long long>(per_sm, 1)));
+  const int TT = tile_tokens<T>(p.d_k, p.L - 1, RPB, budget);
   const int smem = 2 * TileLayout(TT, p.d_k, p.L - 1, RPB, sizeof(T)).bytes;
   cudaError_t err = cudaFuncSetAttribute(recurrent_scan_kernel<T, LPR, EPL, CH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  dim3 grid((p.d_v + RPB - 1) / RPB, p.H, p.B);
   recurrent_scan_kernel<T, LPR, EPL, CH><<<grid, kBlock, smem, stream>>>(p, TT);
   return cudaGetLastError();
 }
