@@ -381,7 +381,7 @@ __device__ __forceinline__ void staged_gemm(float (&acc)[NS][RowMap<D>::RT][4], 
         }
       }
     }
-    __syncthreads();  // this stage is refilled two stages on
+    __syncthreads();  // the next iteration refills this buffer with stage st + 2
   }
   cp_async_wait_0();
 }
@@ -389,7 +389,7 @@ __device__ __forceinline__ void staged_gemm(float (&acc)[NS][RowMap<D>::RT][4], 
 template <typename T, int D, int M, int CH>
 __global__ void __launch_bounds__(kGradThreads) chunk_grad_kernel(ChunkBwdParams p) {
   using Ly = GradLayout<D>;
-  constexpr int C = kBwdChunk, LDD = Ly::LDD, LDC = Ly::LDC, TN = D / 16;
+  constexpr int C = kBwdChunk, LDD = Ly::LDD, LDC = Ly::LDC;
   extern __shared__ __align__(16) float sm[];
   float* sDO = sm + Ly::DO;
   float* sGK = sm + Ly::GK;
