@@ -147,3 +147,42 @@ def test_chunked_backward_strong_decay():
     ref = prism_seq_grad(**x, dO=dO.double().numpy())
     for n, r in ref.items():
         assert _rel(g[n].cpu().numpy().astype(np.float64), r) <= TOL, (n,)
+
+
+def test_full_size_lm_layer_sampled_chains():
+    """The backward at the benchmarked size and launch configuration (130M-LM layer,
+    B=16 T=2048 H=6 d=128 L=4, bf16), checked on two sampled (b, h) chains: each
+    chain's gradients depend on that chain's inputs only, so the oracle (about 15 s a
+    chain) runs on the chain alone.  dconv_w sums over the batch and is left to the
+    smaller cases above (the oracle would need all 16 rows of a head, minutes)."""
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    w = synth.WORKLOADS["lm_130m"].replace(with_s0=True)
+    inp = synth.make_inputs(w)
+    gen = torch.Generator().manual_seed(31)
+    dO = torch.randn((w.B, w.T, w.H, w.d_v), generator=gen).to(torch.bfloat16)
+    dSf = torch.randn((w.B, w.H, w.d_v, w.d_k), generator=gen)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    g = prism.scan_bwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"], d["conv_w"],
+                       dO.cuda(), L=w.L, S0=d["S0"], lengths=d["lengths"], dS_final=dSf.cuda())
+    torch.cuda.synchronize()
+    assert prism.stream_status() == 0
+    got = {n: t.cpu().numpy().astype(np.float64) for n, t in g.items()}
+    x = synth.to_float64_numpy(inp)
+    dO64, dSf64 = dO.double().numpy(), dSf.double().numpy()
+
+    def chain_inputs(bs, h):
+        c = {n: x[n][bs][:, :, h:h + 1] for n in ("q", "k", "v", "gamma", "beta", "u", "alpha", "gain")}
+        c["conv_w"] = x["conv_w"][h:h + 1]
+        c["S0"] = x["S0"][bs][:, h:h + 1]
+        c["lengths"] = None if x["lengths"] is None else x["lengths"][bs]
+        return c
+
+    for b, h in ((0, 0), (15, 5)):
+        ref = prism_seq_grad(**chain_inputs(slice(b, b + 1), h), dO=dO64[b:b + 1, :, h:h + 1],
+                             dS_final=dSf64[b:b + 1, h:h + 1])
+        for n, r in ref.items():
+            if n == "conv_w":
+                continue
+            mine = got[n][b:b + 1, h:h + 1] if n == "S0" else got[n][b:b + 1, :, h:h + 1]
+            assert _rel(mine, r) <= TOL, ((b, h), n, _rel(mine, r))
