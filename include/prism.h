@@ -191,6 +191,22 @@ int prism_scan_bwd(const void* q, const void* k, const void* v,
                    float* du, float* dalpha, float* dgain, float* dconv_w, float* dS0,
                    void* workspace, size_t workspace_bytes, prism_stream_t stream);
 
+/*
+ * prism_state_affine - out = S M + N for every (batch, head): the composition step of
+ * per-segment state maps.  The state update is affine in the state (see the recurrence
+ * above), so a run over a segment of tokens maps a start state S to S M + N, with
+ * M [d_k, d_k] the ordered product of the transitions gamma_t (I - beta_t k_t k_t^T) and
+ * N [d_v, d_k] the segment's end state from a zero start.  Sequence sharding folds the
+ * maps of earlier segments into a segment's start state with this call.
+ *
+ * S, N, out: [BH, d_v, d_k] fp32; M: [BH, d_k, d_k] fp32; device, caller-owned.  N may
+ * be NULL (zero).  out may alias S or N but not M (PRISM_ERR_INVALID_ARG).  d_k, d_v in
+ * {16, 32, 64, 128}; 1 <= BH <= 65535.  fp32, fixed summation order (deterministic).
+ * One launch on `stream`, no synchronisation.
+ */
+int prism_state_affine(const float* S, const float* M, const float* N, float* out, int BH, int d_v, int d_k,
+                       prism_stream_t stream);
+
 /* Size of the device-global scratch behind prism_scan_fwd_static. */
 #define PRISM_STATIC_WORKSPACE_BYTES (32u << 20)
 

@@ -20,6 +20,7 @@ from ._lib import (  # noqa: F401
     scan_fwd_host,
     scan_fwd_static,
     set_spin_limit,
+    state_affine,
     status_string,
     stream_status,
     uses_tensor_cores,

@@ -41,6 +41,7 @@ EXPORTS = (
     "prism_decode_step",
     "prism_scan_bwd",
     "prism_scan_bwd_workspace_size",
+    "prism_state_affine",
     "prism_scan_fwd_uses_tensor_cores",
     "prism_stream_status",
     "prism_set_spin_limit",
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
     L.prism_scan_bwd_workspace_size.restype = cs
     L.prism_scan_bwd.argtypes = [vp] * 13 + [ci] * 9 + [vp] * 11 + [cs, vp]
     L.prism_scan_bwd.restype = ci
+    L.prism_state_affine.argtypes = [fp, fp, fp, fp, ci, ci, ci, vp]
+    L.prism_state_affine.restype = ci
     L.prism_scan_fwd_uses_tensor_cores.argtypes = [ci] * 6
     L.prism_scan_fwd_uses_tensor_cores.restype = ci
     L.prism_stream_status.argtypes = [vp]
@@ -318,6 +321,31 @@ def decode_step(q, k, v, gamma, beta, u, alpha, gain, conv_w, conv_state, S, L: 
     if rc != 0:
         raise PrismError(rc, "prism_decode_step")
     return o
+
+
+def state_affine(S, M, N=None, out=None, stream=None):
+    """out = S M + N per (batch, head) on CUDA fp32 tensors: S, N [..., d_v, d_k], M
+    [..., d_k, d_k] with the same leading dimensions (the composition step of per-segment
+    state maps).  N may be None (zero); out may be S or N."""
+    _check(S, "S", torch.float32)
+    _check(M, "M", torch.float32)
+    _check(N, "N", torch.float32, required=False)
+    d_v, d_k = S.shape[-2], S.shape[-1]
+    if tuple(M.shape) != tuple(S.shape[:-2]) + (d_k, d_k):
+        raise ValueError(f"M must be {tuple(S.shape[:-2]) + (d_k, d_k)}, got {tuple(M.shape)}")
+    if N is not None and tuple(N.shape) != tuple(S.shape):
+        raise ValueError(f"N must be {tuple(S.shape)}, got {tuple(N.shape)}")
+    if out is None:
+        out = torch.empty_like(S)
+    else:
+        _check(out, "out", torch.float32)
+        if tuple(out.shape) != tuple(S.shape):
+            raise ValueError(f"out must be {tuple(S.shape)}, got {tuple(out.shape)}")
+    BH = S.numel() // (d_v * d_k)
+    rc = lib().prism_state_affine(_ptr(S), _ptr(M), _ptr(N), _ptr(out), BH, d_v, d_k, _stream_handle(stream))
+    if rc != 0:
+        raise PrismError(rc, "prism_state_affine")
+    return out
 
 
 def scan_bwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, dO, L: int, S0=None, lengths=None, dS_final=None,

@@ -20,6 +20,8 @@ int bwd_row_blocks(int d_k, int d_v);
 bool chunk_bwd_supported(int d_k, int d_v, int L);
 size_t chunk_bwd_smem_bytes(int d);
 cudaError_t launch_chunk_bwd(const ChunkBwdParams& p, int dtype, cudaStream_t stream);
+cudaError_t launch_state_affine(const float* S, const float* M, const float* N, float* out, int BH, int d_v, int d_k,
+                                cudaStream_t stream);
 }  // namespace prism
 
 namespace {
@@ -278,6 +280,19 @@ int prism_stream_status(prism_stream_t stream) {
   if (value != PRISM_OK && cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return PRISM_ERR_CUDA;
   return value;
+}
+
+int prism_state_affine(const float* S, const float* M, const float* N, float* out, int BH, int d_v, int d_k,
+                       prism_stream_t stream) {
+  if (!S || !M || !out || BH < 1 || d_v < 1 || d_k < 1) return PRISM_ERR_INVALID_ARG;
+  if (M == out) return PRISM_ERR_INVALID_ARG;  // out may alias S or N, not M
+  if (!head_dim_ok(d_k) || !head_dim_ok(d_v) || BH > 65535) return PRISM_ERR_UNSUPPORTED;
+  int* status = nullptr;
+  const int rc = device_setup(&status);
+  if (rc != PRISM_OK) return rc;
+  const cudaError_t err =
+      prism::launch_state_affine(S, M, N, out, BH, d_v, d_k, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
 int prism_decode_step(const void* q, const void* k, const void* v, const float* gamma, const float* beta,

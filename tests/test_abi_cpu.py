@@ -176,3 +176,15 @@ def test_backward_workspace_size(L):
     assert prism.lib().prism_scan_bwd_workspace_size(B, T, H, d, d, Lc, W, 0) == expect
     # far smaller than recording every state: 9.6 MB against 134 MB at T = 2048, B = H = 1, d = 128
     assert prism.lib().prism_scan_bwd_workspace_size(1, 2048, 1, 128, 128, 4, 4, 0) < 10_000_000
+
+
+def test_state_affine_rejects_bad_arguments_before_any_launch(L):
+    F = 0x10000  # never dereferenced: every call below fails before a CUDA call
+    f = L.prism_state_affine
+    assert f(None, F, F, F, 4, 64, 64, None) == 1          # S missing
+    assert f(F, None, F, F, 4, 64, 64, None) == 1          # M missing
+    assert f(F, F, F, None, 4, 64, 64, None) == 1          # out missing
+    assert f(F, F, F, F, 0, 64, 64, None) == 1             # no (batch, head)
+    assert f(F, F + 64, F, F + 64, 4, 64, 64, None) == 1   # out aliases M
+    assert f(F, F, F, F + 64, 4, 48, 64, None) == 2        # d_v not a supported head size
+    assert f(F, F, F, F + 64, 70000, 64, 64, None) == 2    # more (batch, head) pairs than one grid axis

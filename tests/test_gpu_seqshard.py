@@ -1,0 +1,76 @@
+"""Sequence sharding on the GPU, one process: prism_state_affine against an fp64
+matmul, and the phases of seqshard.py run for every segment in turn on the library's
+kernels (the all-gathers become lists), against the oracle's scan of the whole,
+unsharded sequence at the forward bars (2e-2 bf16, 1e-4 fp32)."""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_sequence_shortconv_b200 as prism
+from linear_attention_sequence_shortconv_b200 import seqshard, synth
+from oracle import prism_seq
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("d_v,d_k", [(64, 128), (128, 128), (32, 16)])
+def test_state_affine_matches_fp64(d_v, d_k):
+    g = torch.Generator().manual_seed(d_v + d_k)
+    S = torch.randn(3, 4, d_v, d_k, generator=g)
+    M = torch.randn(3, 4, d_k, d_k, generator=g) / d_k ** 0.5
+    N = torch.randn(3, 4, d_v, d_k, generator=g)
+    ref = S.double() @ M.double() + N.double()
+    Sd, Md, Nd = S.cuda(), M.cuda(), N.cuda()
+    out = prism.state_affine(Sd, Md, Nd)
+    no_n = prism.state_affine(Sd, Md)
+    prism.state_affine(Sd, Md, Nd, out=Sd)  # in place over S
+    torch.cuda.synchronize()
+    err = (out.cpu().double() - ref).abs().max().item() / ref.abs().max().item()
+    assert err < 1e-5
+    assert torch.equal(out, Sd)  # same arithmetic, same order
+    assert (no_n.cpu().double() - (S.double() @ M.double())).abs().max().item() < 1e-4
+
+
+def _sharded_on_gpu(w, bounds, chain="linear"):
+    inp = synth.make_inputs(w)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    W = w.W
+    names = ("q", "k", "v", "gamma", "beta", "u", "alpha", "gain")
+    segs = [seqshard.Segment(**{n: d[n][:, s:e].contiguous() for n in names}, start=s)
+            for s, e in zip(bounds[:-1], bounds[1:])]
+    ops = seqshard.LibraryOps()
+    halos = [seqshard.halo_rows(s.v, W) for s in segs]
+    exts = [seqshard.extend(s, halos[i - 1] if i else torch.zeros_like(halos[0])) for i, s in enumerate(segs)]
+    lens = [seqshard.local_lengths(d["lengths"], e, s.v.shape[1], W - 1) for e, s in zip(exts, segs)]
+    maps = [seqshard.segment_map(e, d["conv_w"], w.L, ln, chain, w.chunk, ops) for e, ln in zip(exts, lens)]
+    outs, S_end = [], None
+    for r, (e, ln) in enumerate(zip(exts, lens)):
+        S_start = seqshard.start_state(d["S0"], maps[:r], maps[0][1], ops)
+        o, S_end = seqshard.scan_segment(e, d["conv_w"], w.L, ln, chain, w.chunk, S_start, W - 1, ops)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert prism.stream_status() == 0
+    x = synth.to_float64_numpy(inp)
+    o_ref, S_ref = prism_seq(**x, chain=chain)
+    return torch.cat(outs, 1).float().cpu().numpy(), S_end.cpu().numpy(), o_ref, S_ref
+
+
+def _rel(x, ref):
+    return float(np.abs(x - ref).max() / max(np.abs(ref).max(), 1e-6))
+
+
+def test_sharded_bf16_tensor_core_segments():
+    """Four segments of an LM-shaped head (d = 128, L = 4, W = 4, bf16: the tensor-core
+    scan), segments of 128 tokens plus 3 history tokens (a ragged last chunk)."""
+    w = synth.WORKLOADS["lm_130m"].replace(B=2, T=512, H=2, with_s0=True, seed=41)
+    o, S, o_ref, S_ref = _sharded_on_gpu(w, [0, 128, 256, 384, 512])
+    assert _rel(o, o_ref) <= 2e-2
+    assert _rel(S, S_ref) <= 2e-2
+
+
+def test_sharded_fp32_uneven_segments_ragged_lengths():
+    w = synth.Workload("shard_fp32", B=3, T=150, H=2, d_k=64, d_v=64, L=3, chunk=64, W=4, dtype="fp32",
+                       lengths_lo=40, with_s0=True, seed=42)
+    o, S, o_ref, S_ref = _sharded_on_gpu(w, [0, 37, 100, 150], chain="gelu")
+    assert _rel(o, o_ref) <= 1e-4
+    assert _rel(S, S_ref) <= 1e-4

@@ -1,0 +1,145 @@
+"""Sequence sharding (seqshard.py) on CPU: gloo ranks each scan one segment of every
+sequence, exchange the ShortConv history and the segment maps with all-gathers, and
+rescan from their exact start state.  The two library operations (the scan and the
+affine step S M + N) are supplied here by the fp64 oracle and numpy; the checks are
+the host logic and the exchange: each rank's outputs and end state must equal the
+oracle's scan of the whole, unsharded sequence to 1e-10."""
+import datetime
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class OracleOps:
+    """The library's two operations, restated by the oracle (fp64, CPU)."""
+
+    def scan(self, q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, chain, chunk):
+        from oracle import prism_seq
+
+        n = lambda t: None if t is None else t.double().numpy()
+        o, S = prism_seq(n(q), n(k), n(v), n(gamma), n(beta), n(u) if L > 1 else None, n(alpha) if L > 1 else None,
+                         n(gain) if L > 1 else None, n(conv_w), S0=n(S0), lengths=n(lengths), chain=chain)
+        return torch.from_numpy(o), torch.from_numpy(S)
+
+    def affine(self, S, M, N):
+        return torch.from_numpy(np.einsum("bhij,bhjk->bhik", S.double().numpy(), M.double().numpy())
+                                + N.double().numpy())
+
+
+def _problem(seed, B, T, H, dk, dv, L, W):
+    g = torch.Generator().manual_seed(seed)
+    r = lambda *s: torch.randn(*s, generator=g, dtype=torch.float64)
+    k = r(B, T, H, dk)
+    k = k / k.norm(dim=-1, keepdim=True)
+    m = L - 1
+    return dict(q=0.5 * r(B, T, H, dk), k=k, v=r(B, T, H, dv),
+                gamma=torch.sigmoid(r(B, T, H) + 2.0), beta=torch.sigmoid(r(B, T, H)),
+                u=0.3 * r(B, T, H, m, dk), alpha=torch.sigmoid(r(B, T, H, m)),
+                gain=torch.sigmoid(r(B, T, H, m, dv)), conv_w=0.5 * r(H, dv, W), S0=0.3 * r(B, H, dv, dk))
+
+
+def _worker(rank, world, port, out_dir, case):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from linear_attention_sequence_shortconv_b200 import seqshard
+    from test_seqshard_cpu import OracleOps, _problem
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        p = _problem(**case["shape"])
+        bounds = case["bounds"]  # segment starts, then T
+        s, e = bounds[rank], bounds[rank + 1]
+        seg = seqshard.Segment(**{n: p[n][:, s:e].contiguous() for n in ("q", "k", "v", "gamma", "beta", "u", "alpha",
+                                                                         "gain")}, start=s)
+        lengths = None if case["lengths"] is None else torch.tensor(case["lengths"], dtype=torch.int32)
+        o, S_end = seqshard.scan_fwd_sequence_sharded(seg, p["conv_w"], case["shape"]["L"], S0=p["S0"],
+                                                      lengths=lengths, chain=case["chain"], ops=OracleOps())
+        np.save(os.path.join(out_dir, f"o_{rank}.npy"), o.numpy())
+        np.save(os.path.join(out_dir, f"S_{rank}.npy"), S_end.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+CASES = {
+    # two ranks, equal segments, ragged lengths (one ends inside rank 0's segment)
+    "two_ranks": dict(shape=dict(seed=1, B=3, T=24, H=2, dk=6, dv=5, L=3, W=4), bounds=[0, 12, 24],
+                      lengths=[24, 17, 9], chain="linear"),
+    # three uneven segments, the exact GELU chain, W = 3
+    "three_ranks_gelu": dict(shape=dict(seed=2, B=2, T=23, H=1, dk=4, dv=4, L=4, W=3), bounds=[0, 7, 16, 23],
+                             lengths=None, chain="gelu"),
+    # W = 1 (no history to exchange), L = 1 (plain gated delta rule)
+    "no_history_gdn": dict(shape=dict(seed=3, B=2, T=10, H=2, dk=4, dv=3, L=1, W=1), bounds=[0, 5, 10],
+                           lengths=[10, 3], chain="linear"),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_sharded_scan_equals_whole_sequence(name, tmp_path):
+    case = CASES[name]
+    world = len(case["bounds"]) - 1
+    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path), case), nprocs=world, join=True,
+                       start_method="spawn")
+    sys.path.insert(0, ROOT)
+    from oracle import prism_seq
+
+    p = _problem(**case["shape"])
+    L = case["shape"]["L"]
+    n = lambda t: t.numpy()
+    lengths = None if case["lengths"] is None else np.array(case["lengths"])
+    o_ref, S_ref = prism_seq(n(p["q"]), n(p["k"]), n(p["v"]), n(p["gamma"]), n(p["beta"]),
+                             n(p["u"]) if L > 1 else None, n(p["alpha"]) if L > 1 else None,
+                             n(p["gain"]) if L > 1 else None, n(p["conv_w"]), S0=n(p["S0"]), lengths=lengths,
+                             chain=case["chain"])
+    o = np.concatenate([np.load(tmp_path / f"o_{r}.npy") for r in range(world)], axis=1)
+    assert o.shape == o_ref.shape
+    assert np.abs(o - o_ref).max() <= 1e-10 * max(1.0, np.abs(o_ref).max())
+    S_last = np.load(tmp_path / f"S_{world - 1}.npy")
+    assert np.abs(S_last - S_ref).max() <= 1e-10 * max(1.0, np.abs(S_ref).max())
+
+
+def test_phases_without_collectives():
+    """One process running every segment in turn (the gathers become lists): the same
+    phases, the same answer; and a segment shorter than the history is rejected."""
+    sys.path.insert(0, ROOT)
+    from linear_attention_sequence_shortconv_b200 import seqshard
+    from oracle import prism_seq
+
+    ops = OracleOps()
+    L, W, T = 3, 4, 20
+    p = _problem(seed=4, B=2, T=T, H=1, dk=4, dv=4, L=L, W=W)
+    bounds = [0, 6, 13, 20]
+    segs = [seqshard.Segment(**{n: p[n][:, s:e].contiguous() for n in ("q", "k", "v", "gamma", "beta", "u", "alpha",
+                                                                      "gain")}, start=s)
+            for s, e in zip(bounds[:-1], bounds[1:])]
+    halos = [seqshard.halo_rows(s.v, W) for s in segs]
+    exts = [seqshard.extend(s, halos[i - 1] if i else torch.zeros_like(halos[0])) for i, s in enumerate(segs)]
+    lens = [seqshard.local_lengths(None, e, s.v.shape[1], W - 1) for e, s in zip(exts, segs)]
+    maps = [seqshard.segment_map(e, p["conv_w"], L, ln, "linear", 64, ops) for e, ln in zip(exts, lens)]
+    outs = []
+    for r, (e, ln) in enumerate(zip(exts, lens)):
+        S_start = seqshard.start_state(p["S0"], maps[:r], maps[0][1], ops)
+        o, S_end = seqshard.scan_segment(e, p["conv_w"], L, ln, "linear", 64, S_start, W - 1, ops)
+        outs.append(o.numpy())
+    n = lambda t: t.numpy()
+    o_ref, S_ref = prism_seq(n(p["q"]), n(p["k"]), n(p["v"]), n(p["gamma"]), n(p["beta"]), n(p["u"]), n(p["alpha"]),
+                             n(p["gain"]), n(p["conv_w"]), S0=n(p["S0"]))
+    assert np.abs(np.concatenate(outs, 1) - o_ref).max() < 1e-10
+    assert np.abs(S_end.numpy() - S_ref).max() < 1e-10
+    with pytest.raises(ValueError):
+        seqshard.halo_rows(p["v"][:, :2], W)
