@@ -9,6 +9,8 @@ is affine in the state, so a run over a segment maps its start state S to S M + 
 M (d_k x d_k) is the ordered product of the transitions and N the segment's end
 state from a zero start.  Each rank
 
+  0. all-gathers the segment lengths (a segment shorter than the W - 1 history rows
+     makes every rank raise, not only its own);
   1. all-gathers the last W - 1 rows of v of every segment: the ShortConv history
      of the segment after it;
   2. scans its segment from a zero state (N) and, with the writes switched off, from
@@ -134,6 +136,13 @@ def scan_fwd_sequence_sharded(seg: Segment, conv_w, L: int, S0=None, lengths=Non
     rank, P = dist.get_rank(group), dist.get_world_size(group)
     W = conv_w.shape[-1]
     n_tokens = seg.v.shape[1]
+    # 0. every rank checks every segment's length, so that all of them raise together
+    #    instead of some waiting in a collective that the others never reach
+    sizes = [torch.zeros(1, dtype=torch.int64, device=seg.v.device) for _ in range(P)]
+    dist.all_gather(sizes, torch.tensor([n_tokens], dtype=torch.int64, device=seg.v.device), group=group)
+    if min(int(x.item()) for x in sizes) < W - 1:
+        raise ValueError(f"every segment needs at least W - 1 = {W - 1} tokens; segment lengths "
+                         f"{[int(x.item()) for x in sizes]}")
     # 1. ShortConv history of every segment
     mine = halo_rows(seg.v, W)
     halos = [torch.empty_like(mine) for _ in range(P)]

@@ -67,8 +67,14 @@ def _worker(rank, world, port, out_dir, case):
         seg = seqshard.Segment(**{n: p[n][:, s:e].contiguous() for n in ("q", "k", "v", "gamma", "beta", "u", "alpha",
                                                                          "gain")}, start=s)
         lengths = None if case["lengths"] is None else torch.tensor(case["lengths"], dtype=torch.int32)
-        o, S_end = seqshard.scan_fwd_sequence_sharded(seg, p["conv_w"], case["shape"]["L"], S0=p["S0"],
-                                                      lengths=lengths, chain=case["chain"], ops=OracleOps())
+        try:
+            o, S_end = seqshard.scan_fwd_sequence_sharded(seg, p["conv_w"], case["shape"]["L"], S0=p["S0"],
+                                                          lengths=lengths, chain=case["chain"], ops=OracleOps())
+        except ValueError as e:  # a segment shorter than the history: every rank must see it
+            np.save(os.path.join(out_dir, f"err_{rank}.npy"), np.array([1]))
+            assert "W - 1" in str(e)
+            dist.barrier()
+            return
         np.save(os.path.join(out_dir, f"o_{rank}.npy"), o.numpy())
         np.save(os.path.join(out_dir, f"S_{rank}.npy"), S_end.numpy())
         dist.barrier()
@@ -87,6 +93,16 @@ CASES = {
     "no_history_gdn": dict(shape=dict(seed=3, B=2, T=10, H=2, dk=4, dv=3, L=1, W=1), bounds=[0, 5, 10],
                            lengths=[10, 3], chain="linear"),
 }
+
+
+def test_short_segment_fails_on_every_rank(tmp_path):
+    """Rank 1's segment (2 tokens) is shorter than the W - 1 = 3 history rows: both
+    ranks raise together, none waits in a collective."""
+    case = dict(shape=dict(seed=5, B=1, T=12, H=1, dk=4, dv=4, L=2, W=4), bounds=[0, 10, 12], lengths=None,
+                chain="linear")
+    mp.start_processes(_worker, args=(2, _free_port(), str(tmp_path), case), nprocs=2, join=True,
+                       start_method="spawn")
+    assert (tmp_path / "err_0.npy").exists() and (tmp_path / "err_1.npy").exists()
 
 
 @pytest.mark.parametrize("name", list(CASES))
