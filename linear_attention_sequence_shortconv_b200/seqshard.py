@@ -161,3 +161,50 @@ def scan_fwd_sequence_sharded(seg: Segment, conv_w, L: int, S0=None, lengths=Non
     S_start = start_state(S0, list(zip(Ms[:rank], Ns[:rank])), N, ops)
     # 4. the exact pass
     return scan_segment(ext, conv_w, L, lens, chain, chunk, S_start, W - 1, ops)
+
+
+def scan_fwd_segmented(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, P: int, S0=None, lengths=None,
+                       chain: str = "linear", chunk: int = 64, ops=None):
+    """The whole scan on one device with each sequence cut into P segments that run
+    side by side: the segments are stacked along the batch axis (P x B sequences of
+    ceil(T / P) + W - 1 tokens), so each of the three scans has P times the
+    parallelism at 1/P of the length; the maps are folded in P - 1 affine steps.
+    Returns (o [B, T, H, d_v], S_final) as scan_fwd."""
+    ops = ops or LibraryOps()
+    B, T, H, _ = q.shape
+    W = conv_w.shape[-1]
+    Ts = -(-T // P)
+    if Ts < W - 1:
+        raise ValueError(f"segments of {Ts} tokens are shorter than the W - 1 = {W - 1} history rows")
+    pad = P * Ts - T
+
+    def padded(x):  # [B, P*Ts, ...]: the tail past T is never a valid token
+        if x is None or pad == 0:
+            return x
+        return torch.cat([x, torch.zeros((B, pad) + tuple(x.shape[2:]), dtype=x.dtype, device=x.device)], 1)
+
+    full = {n: padded(x) for n, x in dict(q=q, k=k, v=v, gamma=gamma, beta=beta, u=u, alpha=alpha,
+                                          gain=gain).items()}
+    if lengths is None:
+        lengths = torch.full((B,), T, dtype=torch.int32, device=q.device)
+    exts, lens = [], []
+    for r in range(P):
+        seg = Segment(**{n: None if x is None else x[:, r * Ts:(r + 1) * Ts] for n, x in full.items()},
+                      start=r * Ts)
+        halo = (full["v"][:, r * Ts - (W - 1):r * Ts] if r > 0 else
+                torch.zeros((B, W - 1) + tuple(v.shape[2:]), dtype=v.dtype, device=v.device))
+        ext = extend(seg, halo)
+        exts.append(ext)
+        lens.append(local_lengths(lengths, ext, Ts, W - 1))
+    # every segment side by side: batch index r * B + b
+    cat = lambda xs: None if xs[0] is None else torch.cat(xs, 0).contiguous()
+    stacked = Segment(**{n: cat([getattr(e, n) for e in exts]) for n in full}, start=0)
+    lens_all = torch.cat(lens, 0).contiguous()
+    M, N = segment_map(stacked, conv_w, L, lens_all, chain, chunk, ops)
+    Ms, Ns = M.view(P, B, *M.shape[1:]), N.view(P, B, *N.shape[1:])
+    starts = [torch.zeros_like(Ns[0]) if S0 is None else S0]
+    for r in range(1, P):
+        starts.append(ops.affine(starts[-1].contiguous(), Ms[r - 1].contiguous(), Ns[r - 1].contiguous()))
+    o, S_end = scan_segment(stacked, conv_w, L, lens_all, chain, chunk, torch.cat(starts, 0), W - 1, ops)
+    o = o.reshape(P, B, Ts, *o.shape[2:]).permute(1, 0, 2, 3, 4).reshape(B, P * Ts, *o.shape[2:])
+    return o[:, :T], S_end.view(P, B, *S_end.shape[1:])[P - 1]

@@ -159,3 +159,30 @@ def test_phases_without_collectives():
     assert np.abs(S_end.numpy() - S_ref).max() < 1e-10
     with pytest.raises(ValueError):
         seqshard.halo_rows(p["v"][:, :2], W)
+
+
+@pytest.mark.parametrize("P,T,W,L,chain,lengths", [
+    (4, 26, 4, 3, "linear", [26, 11]),   # uneven: the last segment is padded
+    (3, 18, 3, 4, "gelu", None),
+    (2, 9, 1, 1, "linear", [9, 0]),      # no history, plain gated delta rule, an empty row
+])
+def test_segmented_single_device_equals_whole_sequence(P, T, W, L, chain, lengths):
+    """scan_fwd_segmented: the segments of every sequence stacked along the batch axis
+    in one process, against the oracle's scan of the whole sequence."""
+    sys.path.insert(0, ROOT)
+    from linear_attention_sequence_shortconv_b200 import seqshard
+    from oracle import prism_seq
+
+    p = _problem(seed=P * 10 + T, B=2, T=T, H=2, dk=4, dv=3, L=L, W=W)
+    lens = None if lengths is None else torch.tensor(lengths, dtype=torch.int32)
+    o, S = seqshard.scan_fwd_segmented(p["q"], p["k"], p["v"], p["gamma"], p["beta"], p["u"], p["alpha"],
+                                       p["gain"], p["conv_w"], L, P, S0=p["S0"], lengths=lens, chain=chain,
+                                       ops=OracleOps())
+    n = lambda t: t.numpy()
+    o_ref, S_ref = prism_seq(n(p["q"]), n(p["k"]), n(p["v"]), n(p["gamma"]), n(p["beta"]),
+                             n(p["u"]) if L > 1 else None, n(p["alpha"]) if L > 1 else None,
+                             n(p["gain"]) if L > 1 else None, n(p["conv_w"]), S0=n(p["S0"]),
+                             lengths=None if lengths is None else np.array(lengths), chain=chain)
+    assert o.shape == o_ref.shape
+    assert np.abs(o.numpy() - o_ref).max() < 1e-10
+    assert np.abs(S.numpy() - S_ref).max() < 1e-10
