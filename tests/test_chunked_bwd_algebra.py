@@ -163,3 +163,111 @@ def test_chunked_formulas_match_autograd(chain, L, W, C, T, lengths):
     for n, r in ref.items():
         err = np.abs(got[n] - r).max() / max(np.abs(r).max(), 1e-12)
         assert err < 1e-10, (n, err)
+
+
+def chunk_boundary_passes(q, k, v, gamma, beta, u, alpha, gain, conv_w, dO, S0, dSf, chain, C):
+    """The two boundary passes in chunk (GEMM) form, one sequence (B = H = 1, full
+    length): the forward carry S_n -> S_{n+1} through T = (I + A)^{-1}, and the
+    adjoint carry H_n -> H_{n-1} through T^T, with the per-token records psi and gk
+    they produce.  Returns (states [NC+1], psi [T], Hn [NC], gk [T])."""
+    T_, dk = k.shape[1], k.shape[-1]
+    dv, W, m = v.shape[-1], conv_w.shape[-1], u.shape[3]
+    NC = (T_ + C - 1) // C
+    w = conv_w[0]
+
+    def resid(t):
+        rs = [v[0, t, 0] - sum(w[:, i] * v[0, t - i, 0] for i in range(W) if t - i >= 0)]
+        for l in range(m):
+            r = rs[-1]
+            rs.append((1 - gain[0, t, 0, l]) * r if chain == "linear" else r - _gelu(gain[0, t, 0, l] * r))
+        return rs
+
+    chunks = []
+    for n in range(NC):
+        ii = np.arange(n * C, min(T_, n * C + C))
+        c = np.cumsum(np.log(gamma[0, ii, 0]))
+        Dm = np.tril(np.exp(c[:, None] - c[None, :]))
+        Dms = Dm - np.diag(np.diag(Dm))
+        K, Q, V, be = k[0, ii, 0], q[0, ii, 0], v[0, ii, 0], beta[0, ii, 0]
+        R = [resid(t) for t in ii]
+        Rt = [alpha[0, ii, 0, l][:, None] * np.array([r[l + 1] for r in R]) for l in range(m)]
+        U = [u[0, ii, 0, l] for l in range(m)]
+        A = be[:, None] * Dms * (K @ K.T)
+        Tinv = np.linalg.inv(np.eye(len(ii)) + A)
+        chunks.append((ii, c, Dm, Dms, K, Q, V, be, Rt, U, Tinv))
+    # forward carry: X = diag(beta)(V - P'), Delta = T X, psi = V - P' - Kp_0 Delta
+    S = S0[0, 0].copy()
+    states, psi = [S.copy()], np.zeros((T_, dv))
+    for ii, c, Dm, Dms, K, Q, V, be, Rt, U, Tinv in chunks:
+        Pp = np.exp(c)[:, None] * (K @ S.T) + sum((Dms * (K @ U[l].T)) @ Rt[l] for l in range(m))
+        Delta = Tinv @ (be[:, None] * (V - Pp))
+        psi[ii] = V - Pp - (Dms * (K @ K.T)) @ Delta
+        dec = np.exp(c[-1] - c)[:, None]
+        S = np.exp(c[-1]) * S + (dec * Delta).T @ K + sum((dec * Rt[l]).T @ U[l] for l in range(m))
+        states.append(S.copy())
+    # adjoint carry: Y = diag(e^{c_C - c}) K H^T + (D o Q K^T)^T dO, gk = T^T Y
+    H = dSf[0, 0].copy()
+    Hn, gk = [None] * NC, np.zeros((T_, dv))
+    for n in range(NC - 1, -1, -1):
+        ii, c, Dm, Dms, K, Q, V, be, Rt, U, Tinv = chunks[n]
+        Hn[n] = H.copy()
+        DO = dO[0, ii, 0]
+        Y = np.exp(c[-1] - c)[:, None] * (K @ H.T) + (Dm * (Q @ K.T)).T @ DO
+        G = Tinv.T @ Y
+        gk[ii] = G
+        E = be[:, None] * G
+        H = np.exp(c[-1]) * H + DO.T @ (np.exp(c)[:, None] * Q) - E.T @ (np.exp(c)[:, None] * K)
+    return states, psi, Hn, gk, H
+
+
+@pytest.mark.parametrize("chain,L,C,T", [("linear", 3, 8, 29), ("gelu", 4, 4, 16), ("linear", 1, 8, 8)])
+def test_chunk_form_boundary_passes_equal_token_records(chain, L, C, T):
+    """The boundary passes in chunk form (serial over chunks, GEMM-shaped) reproduce
+    the token-by-token records: the states at every chunk boundary, psi, the adjoint
+    H_n at every chunk end, gk, and dS0."""
+    rng = np.random.default_rng(7 + L + C)
+    dk, dv, W, m = 6, 5, 3, L - 1
+    k = rng.standard_normal((1, T, 1, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    x = dict(q=0.5 * rng.standard_normal((1, T, 1, dk)), k=k, v=rng.standard_normal((1, T, 1, dv)),
+             gamma=rng.uniform(0.5, 1.0, (1, T, 1)), beta=rng.uniform(0.1, 1.0, (1, T, 1)),
+             u=0.3 * rng.standard_normal((1, T, 1, m, dk)), alpha=rng.uniform(0.0, 0.5, (1, T, 1, m)),
+             gain=0.5 * rng.standard_normal((1, T, 1, m, dv)), conv_w=0.3 * rng.standard_normal((1, dv, W)))
+    dO = rng.standard_normal((1, T, 1, dv))
+    S0 = 0.3 * rng.standard_normal((1, 1, dv, dk))
+    dSf = rng.standard_normal((1, 1, dv, dk))
+    states, psi, Hn, gk, dS0 = chunk_boundary_passes(**x, dO=dO, S0=S0, dSf=dSf, chain=chain, C=C)
+    # the token-by-token records, written out directly
+    NC = (T + C - 1) // C
+    S, ref_states, ref_psi = S0[0, 0].copy(), [S0[0, 0].copy()], np.zeros((T, dv))
+    w = x["conv_w"][0]
+    for t in range(T):
+        rs = [x["v"][0, t, 0] - sum(w[:, i] * x["v"][0, t - i, 0] for i in range(W) if t - i >= 0)]
+        for l in range(m):
+            r = rs[-1]
+            g = x["gain"][0, t, 0, l]
+            rs.append((1 - g) * r if chain == "linear" else r - _gelu(g * r))
+        kt, gm, bt = x["k"][0, t, 0], x["gamma"][0, t, 0], x["beta"][0, t, 0]
+        sk = S @ kt
+        ref_psi[t] = x["v"][0, t, 0] - gm * sk
+        S = gm * (S - bt * np.outer(sk, kt)) + bt * np.outer(x["v"][0, t, 0], kt)
+        for l in range(m):
+            S = S + x["alpha"][0, t, 0, l] * np.outer(rs[l + 1], x["u"][0, t, 0, l])
+        if (t + 1) % C == 0 or t + 1 == T:
+            ref_states.append(S.copy())
+    G, ref_Hn, ref_gk = dSf[0, 0].copy(), [None] * NC, np.zeros((T, dv))
+    ref_Hn[NC - 1] = G.copy()
+    for t in range(T - 1, -1, -1):
+        G = G + np.outer(dO[0, t, 0], x["q"][0, t, 0])
+        kt = x["k"][0, t, 0]
+        ref_gk[t] = G @ kt
+        G = x["gamma"][0, t, 0] * (G - x["beta"][0, t, 0] * np.outer(ref_gk[t], kt))
+        if t % C == 0 and t > 0:
+            ref_Hn[t // C - 1] = G.copy()
+    for a, b in zip(states, ref_states):
+        assert np.abs(a - b).max() < 1e-10
+    assert np.abs(psi - ref_psi).max() < 1e-10
+    for a, b in zip(Hn, ref_Hn):
+        assert np.abs(a - b).max() < 1e-10
+    assert np.abs(gk - ref_gk).max() < 1e-10
+    assert np.abs(dS0 - G).max() < 1e-10
