@@ -196,13 +196,20 @@ def time_oracle(w, budget_s, rows=None, tokens=None):
     x = synth.to_float64_numpy(synth.make_inputs(sample))
     if w.L == 1:
         x["u"] = x["alpha"] = x["gain"] = None
-    wall0, cpu0 = time.perf_counter(), time.process_time()
-    prism_seq(**x)
-    wall = time.perf_counter() - wall0
-    cpu = time.process_time() - cpu0
-    cores = max(1, round(cpu / wall)) if wall > 0 else 1
-    return {"tokens": rows * tokens, "seconds": wall, "cores": cores,
-            "sample": f"first {tokens} steps of {rows} batch row(s) x {w.H} heads of {w.name}"}
+    # every core this process may run on is offered to the BLAS and torch thread pools
+    import torch
+
+    avail = len(os.sched_getaffinity(0))
+    torch.set_num_threads(avail)
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=avail):
+        wall0, cpu0 = time.perf_counter(), time.process_time()
+        prism_seq(**x)
+        wall = time.perf_counter() - wall0
+        cpu = time.process_time() - cpu0
+    used = max(1, round(cpu / wall)) if wall > 0 else 1  # cores the oracle actually kept busy
+    return {"tokens": rows * tokens, "seconds": wall, "cores": used, "cores_available": avail,
+            "threads": avail, "sample": f"first {tokens} steps of {rows} batch row(s) x {w.H} heads of {w.name}"}
 
 
 def calibrate_oracle_tokens(w, target_s):
@@ -220,12 +227,12 @@ def run_reference(args, w):
     tokens = calibrate_oracle_tokens(w, budget / max(1, steps + warmup))
     for _ in range(warmup):
         time_oracle(w, 0, rows=1, tokens=tokens)
-    times, cores, sample = [], 1, ""
+    times, cores, sample, avail = [], 1, "", 1
     for _ in range(steps):
         r = time_oracle(w, 0, rows=1, tokens=tokens)
         times.append(r["seconds"])
         cores = max(cores, r["cores"])
-        sample = r["sample"]
+        sample, avail = r["sample"], r["cores_available"]
     ms = 1e3 * sum(times) / len(times)
     value = tokens / (ms / 1e3)
     line = {
@@ -233,7 +240,8 @@ def run_reference(args, w):
         "steps": steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "cores_available": avail, "threads": avail,
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -317,10 +325,14 @@ def run_ours_bwd(args, w):
         xs = synth.to_float64_numpy(synth.make_inputs(sample))
         if w.L == 1:
             xs["u"] = xs["alpha"] = xs["gain"] = None
-        t0 = time.perf_counter()
+        avail = len(os.sched_getaffinity(0))
+        torch.set_num_threads(avail)
+        t0, c0 = time.perf_counter(), time.process_time()
         prism_seq_grad(**xs, dO=np.ones((1, tokens, w.H, w.d_v)), dS_final=None)
         sec = time.perf_counter() - t0
-        cpu_baseline = {"value": tokens / sec, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+        used = max(1, round((time.process_time() - c0) / sec)) if sec > 0 else 1
+        cpu_baseline = {"value": tokens / sec, "unit": UNIT, "cores": used, "cores_available": avail,
+                        "threads": avail, "kind": "oracle",
                         "sample": f"autograd of the first {tokens} steps of 1 batch row x {w.H} heads of {w.name}",
                         "seconds": sec}
     line = {"metric": "PRISM scan bwd (all input gradients) tokens/s on 1 B200", "value": work["tokens"] / (ms / 1e3),
@@ -459,7 +471,8 @@ def run_ours(args, w):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = 4 if w.T >= 1024 else 16
         r = time_oracle(w, 0, rows=min(rows, w.B), tokens=min(w.T, 2048))
-        cpu_baseline = {"value": r["tokens"] / r["seconds"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+        cpu_baseline = {"value": r["tokens"] / r["seconds"], "unit": UNIT, "cores": r["cores"],
+                        "cores_available": r["cores_available"], "threads": r["threads"], "kind": "oracle",
                         "sample": r["sample"], "seconds": r["seconds"]}
 
     clk = clocks.summary()

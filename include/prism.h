@@ -200,7 +200,8 @@ int prism_scan_bwd(const void* q, const void* k, const void* v,
  * maps of earlier segments into a segment's start state with this call.
  *
  * S, N, out: [BH, d_v, d_k] fp32; M: [BH, d_k, d_k] fp32; device, caller-owned.  N may
- * be NULL (zero).  out may alias S or N but not M (PRISM_ERR_INVALID_ARG).  d_k, d_v in
+ * be NULL (zero).  out may be exactly S or exactly N; any other overlap of out with S, M
+ * or N returns PRISM_ERR_INVALID_ARG before any launch.  d_k, d_v in
  * {16, 32, 64, 128}; 1 <= BH <= 65535.  fp32, fixed summation order (deterministic).
  * One launch on `stream`, no synchronisation.
  */
@@ -214,8 +215,13 @@ int prism_state_affine(const float* S, const float* M, const float* N, float* ou
  * prism_scan_fwd_static - prism_scan_fwd_ex without a caller-supplied workspace and
  * without any allocation: the scratch is a file-scope device array of
  * PRISM_STATIC_WORKSPACE_BYTES (32 MiB, 256-byte aligned) inside the library, one per
- * device, located once per device with cudaGetSymbolAddress.  Results are bit-for-bit
- * those of prism_scan_fwd_ex with a workspace.  Sizes whose
+ * device.  The first call on a device looks its address up with cudaGetSymbolAddress
+ * (make that first call before any stream capture); later calls reuse it.  The array
+ * sits in a module of its own: with lazy module loading (the default of CUDA 12, and
+ * what PyTorch sets) it is held, until the process exits, on each device where this
+ * entry point has run; with CUDA_MODULE_LOADING=EAGER, on every device where the
+ * library is loaded.  Results are bit-for-bit those of prism_scan_fwd_ex with a
+ * workspace.  Sizes whose
  * prism_scan_fwd_workspace_size() exceeds PRISM_STATIC_WORKSPACE_BYTES return
  * PRISM_ERR_WORKSPACE before any launch (the 130M-LM layer, B=16 T=2048 H=6 d=128,
  * needs 24 MiB).  Because the scratch is shared, calls on one device must not overlap

@@ -144,21 +144,76 @@ def _chain_code(chain: str) -> int:
     return CHAINS[chain]
 
 
-def _check(t: Optional[torch.Tensor], name: str, dtype=None, required=True):
+def _check(t: Optional[torch.Tensor], name: str, dtype=None, required=True, shape=None, device=None):
+    """Validate one tensor argument: CUDA, contiguous, dtype, and (when given) the exact
+    shape and the device every other argument of the call is on."""
     if t is None:
         if required:
             raise ValueError(f"{name} is required")
         return
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, but the call's tensors are on {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _call_device(first: torch.Tensor, stream) -> torch.device:
+    """The device a call runs on: that of its first tensor argument.  The library launches
+    on the current CUDA device, so every entry point below runs inside
+    ``torch.cuda.device(dev)``; a stream passed in must belong to the same device."""
+    if not isinstance(first, torch.Tensor) or not first.is_cuda:
+        raise ValueError("the first tensor argument must be a CUDA tensor (the library has no CPU path)")
+    dev = first.device
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"stream belongs to {stream.device}, but the call's tensors are on {dev}")
+    return dev
 
 
 def workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype_code) -> int:
     return int(lib().prism_scan_fwd_workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype_code))
+
+
+def _scan_checks(q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o, S_final, want_state,
+                 stream):
+    """Argument checks shared by scan_fwd and scan_fwd_static; returns the sizes, the
+    device and the (allocated when missing) outputs."""
+    dev = _call_device(q, stream)
+    dt = q.dtype
+    code = _dtype_code(q)
+    if q.dim() != 4 or v.dim() != 4 or conv_w.dim() != 3:
+        raise ValueError("q, k, v must be [B, T, H, d] and conv_w [H, d_v, W]")
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    W = conv_w.shape[-1]
+    m = L - 1
+    _check(q, "q", dt, device=dev)
+    _check(k, "k", dt, shape=(B, T, H, d_k), device=dev)
+    _check(v, "v", dt, shape=(B, T, H, d_v), device=dev)
+    _check(gamma, "gamma", torch.float32, shape=(B, T, H), device=dev)
+    _check(beta, "beta", torch.float32, shape=(B, T, H), device=dev)
+    _check(conv_w, "conv_w", torch.float32, shape=(H, d_v, W), device=dev)
+    if L > 1:
+        _check(u, "u", dt, shape=(B, T, H, m, d_k), device=dev)
+        _check(gain, "gain", dt, shape=(B, T, H, m, d_v), device=dev)
+        _check(alpha, "alpha", torch.float32, shape=(B, T, H, m), device=dev)
+    _check(S0, "S0", torch.float32, required=False, shape=(B, H, d_v, d_k), device=dev)
+    _check(lengths, "lengths", torch.int32, required=False, shape=(B,), device=dev)
+    if o is None:
+        o = torch.empty((B, T, H, d_v), dtype=dt, device=dev)
+    else:
+        _check(o, "o", dt, shape=(B, T, H, d_v), device=dev)
+    if want_state:
+        if S_final is None:
+            S_final = torch.empty((B, H, d_v, d_k), dtype=torch.float32, device=dev)
+        else:
+            _check(S_final, "S_final", torch.float32, shape=(B, H, d_v, d_k), device=dev)
+    return (B, T, H, d_k, d_v, W, code), dev, o, S_final
 
 
 def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 64,
@@ -172,37 +227,25 @@ def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 
     Shapes as in include/prism.h: q, k [B,T,H,d_k]; v [B,T,H,d_v]; gamma, beta
     [B,T,H] fp32; u [B,T,H,L-1,d_k]; alpha [B,T,H,L-1] fp32; gain [B,T,H,L-1,d_v];
     conv_w [H,d_v,W] fp32; S0 [B,H,d_v,d_k] fp32 or None; lengths [B] int32 or None.
+    Every tensor must be on one CUDA device; the call runs on that device.
     """
-    dt = q.dtype
-    code = _dtype_code(q)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _check(t, name, dt)
-    for name, t in (("gamma", gamma), ("beta", beta), ("conv_w", conv_w)):
-        _check(t, name, torch.float32)
-    if L > 1:
-        _check(u, "u", dt)
-        _check(gain, "gain", dt)
-        _check(alpha, "alpha", torch.float32)
-    _check(S0, "S0", torch.float32, required=False)
-    _check(lengths, "lengths", torch.int32, required=False)
-    B, T, H, d_k = q.shape
-    d_v = v.shape[-1]
-    W = conv_w.shape[-1]
-    if o is None:
-        o = torch.empty((B, T, H, d_v), dtype=dt, device=q.device)
-    if want_state and S_final is None:
-        S_final = torch.empty((B, H, d_v, d_k), dtype=torch.float32, device=q.device)
-    ws_bytes = workspace_size(B, T, H, d_k, d_v, L, W, chunk, code)
-    if ws_bytes and workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     chain_code = _chain_code(chain)
-    rc = lib().prism_scan_fwd_ex(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
-        _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
-        _ptr(conv_w), _ptr(S0), _ptr(lengths),
-        B, T, H, d_k, d_v, L, W, chunk, code,
-        _ptr(o), _ptr(S_final if want_state else None),
-        _ptr(workspace), ws_bytes if workspace is not None else 0, _stream_handle(stream), chain_code)
+    (B, T, H, d_k, d_v, W, code), dev, o, S_final = _scan_checks(
+        q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o, S_final, want_state, stream)
+    with torch.cuda.device(dev):
+        ws_bytes = workspace_size(B, T, H, d_k, d_v, L, W, chunk, code)
+        if ws_bytes and workspace is None:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        if workspace is not None:
+            _check(workspace, "workspace", torch.uint8, device=dev)
+        rc = lib().prism_scan_fwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+            _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
+            _ptr(conv_w), _ptr(S0), _ptr(lengths),
+            B, T, H, d_k, d_v, L, W, chunk, code,
+            _ptr(o), _ptr(S_final if want_state else None),
+            _ptr(workspace), workspace.numel() if workspace is not None else 0, _stream_handle(stream),
+            chain_code)
     if rc != 0:
         raise PrismError(rc, "prism_scan_fwd_ex")
     return o, (S_final if want_state else None)
@@ -214,31 +257,15 @@ def scan_fwd_static(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk:
     """scan_fwd through prism_scan_fwd_static: no workspace argument, and the library
     allocates nothing (its scratch is a device-global array); returns (o, S_final)."""
     chain_code = _chain_code(chain)
-    dt = q.dtype
-    code = _dtype_code(q)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _check(t, name, dt)
-    for name, t in (("gamma", gamma), ("beta", beta), ("conv_w", conv_w)):
-        _check(t, name, torch.float32)
-    if L > 1:
-        _check(u, "u", dt)
-        _check(gain, "gain", dt)
-        _check(alpha, "alpha", torch.float32)
-    _check(S0, "S0", torch.float32, required=False)
-    _check(lengths, "lengths", torch.int32, required=False)
-    B, T, H, d_k = q.shape
-    d_v = v.shape[-1]
-    W = conv_w.shape[-1]
-    if o is None:
-        o = torch.empty((B, T, H, d_v), dtype=dt, device=q.device)
-    if want_state and S_final is None:
-        S_final = torch.empty((B, H, d_v, d_k), dtype=torch.float32, device=q.device)
-    rc = lib().prism_scan_fwd_static(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
-        _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
-        _ptr(conv_w), _ptr(S0), _ptr(lengths),
-        B, T, H, d_k, d_v, L, W, chunk, code,
-        _ptr(o), _ptr(S_final if want_state else None), _stream_handle(stream), chain_code)
+    (B, T, H, d_k, d_v, W, code), dev, o, S_final = _scan_checks(
+        q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o, S_final, want_state, stream)
+    with torch.cuda.device(dev):
+        rc = lib().prism_scan_fwd_static(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+            _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
+            _ptr(conv_w), _ptr(S0), _ptr(lengths),
+            B, T, H, d_k, d_v, L, W, chunk, code,
+            _ptr(o), _ptr(S_final if want_state else None), _stream_handle(stream), chain_code)
     if rc != 0:
         raise PrismError(rc, "prism_scan_fwd_static")
     return o, (S_final if want_state else None)
@@ -255,15 +282,27 @@ def scan_fwd_host(host: dict, dev: dict, L: int, chunk: int = 64, stream=None):
     d_v = host["v"].shape[-1]
     W = host["conv_w"].shape[-1]
     code = _dtype_code(q)
+    device = _call_device(dev["o"], stream)
+    for n in names + ("o", "S_final"):
+        h = host.get(n)
+        if h is None:
+            continue
+        if h.is_cuda or not h.is_contiguous():
+            raise ValueError(f"host[{n!r}] must be a contiguous CPU tensor (pinned for asynchronous copies)")
+        _check(dev.get(n), f"dev[{n!r}]", h.dtype, shape=h.shape, device=device)
     ws_bytes = workspace_size(B, T, H, d_k, d_v, L, W, chunk, code)
     ws = dev.get("workspace")
-    if ws_bytes and ws is None:
-        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev["o"].device)
-    rc = lib().prism_scan_fwd_host(
-        *[_ptr(host.get(n)) for n in names], *[_ptr(dev.get(n) if host.get(n) is not None else None) for n in names],
-        B, T, H, d_k, d_v, L, W, chunk, code,
-        _ptr(dev["o"]), _ptr(dev.get("S_final")), _ptr(host["o"]), _ptr(host.get("S_final")),
-        _ptr(ws), ws_bytes if ws is not None else 0, _stream_handle(stream))
+    with torch.cuda.device(device):
+        if ws_bytes and ws is None:
+            ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+        if ws is not None:
+            _check(ws, "dev['workspace']", torch.uint8, device=device)
+        rc = lib().prism_scan_fwd_host(
+            *[_ptr(host.get(n)) for n in names],
+            *[_ptr(dev.get(n) if host.get(n) is not None else None) for n in names],
+            B, T, H, d_k, d_v, L, W, chunk, code,
+            _ptr(dev["o"]), _ptr(dev.get("S_final")), _ptr(host["o"]), _ptr(host.get("S_final")),
+            _ptr(ws), ws.numel() if ws is not None else 0, _stream_handle(stream))
     if rc != 0:
         raise PrismError(rc, "prism_scan_fwd_host")
 
@@ -271,17 +310,19 @@ def scan_fwd_host(host: dict, dev: dict, L: int, chunk: int = 64, stream=None):
 def prologue_fwd(v, alpha, gain, conv_w, L: int, lengths=None, stream=None, chain: str = "linear"):
     """rho_{t,l} = alpha_{t,l} r_{t,l} as [B,T,H,L-1,d_v] fp32 (CUDA)."""
     chain_code = _chain_code(chain)
+    dev = _call_device(v, stream)
     code = _dtype_code(v)
-    _check(v, "v")
-    _check(gain, "gain", v.dtype)
-    _check(alpha, "alpha", torch.float32)
-    _check(conv_w, "conv_w", torch.float32)
-    _check(lengths, "lengths", torch.int32, required=False)
+    _check(v, "v", device=dev)
     B, T, H, d_v = v.shape
-    rho = torch.empty((B, T, H, L - 1, d_v), dtype=torch.float32, device=v.device)
-    rc = lib().prism_prologue_fwd_ex(_ptr(v), _ptr(alpha), _ptr(gain), _ptr(conv_w), _ptr(lengths),
-                                     B, T, H, d_v, L, conv_w.shape[-1], code, _ptr(rho),
-                                     _stream_handle(stream), chain_code)
+    W = conv_w.shape[-1]
+    _check(gain, "gain", v.dtype, shape=(B, T, H, L - 1, d_v), device=dev)
+    _check(alpha, "alpha", torch.float32, shape=(B, T, H, L - 1), device=dev)
+    _check(conv_w, "conv_w", torch.float32, shape=(H, d_v, W), device=dev)
+    _check(lengths, "lengths", torch.int32, required=False, shape=(B,), device=dev)
+    rho = torch.empty((B, T, H, L - 1, d_v), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib().prism_prologue_fwd_ex(_ptr(v), _ptr(alpha), _ptr(gain), _ptr(conv_w), _ptr(lengths),
+                                         B, T, H, d_v, L, W, code, _ptr(rho), _stream_handle(stream), chain_code)
     if rc != 0:
         raise PrismError(rc, "prism_prologue_fwd_ex")
     return rho
@@ -297,27 +338,35 @@ def decode_step(q, k, v, gamma, beta, u, alpha, gain, conv_w, conv_state, S, L: 
     updated in place.
     """
     chain_code = _chain_code(chain)
+    dev = _call_device(q, stream)
     dt = q.dtype
     code = _dtype_code(q)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _check(t, name, dt)
-    for name, t in (("gamma", gamma), ("beta", beta), ("conv_w", conv_w), ("S", S)):
-        _check(t, name, torch.float32)
-    if L > 1:
-        _check(u, "u", dt)
-        _check(gain, "gain", dt)
-        _check(alpha, "alpha", torch.float32)
-    W = conv_w.shape[-1]
-    _check(conv_state, "conv_state", dt, required=W > 1)
     B, H, d_k = q.shape
     d_v = v.shape[-1]
+    W = conv_w.shape[-1]
+    m = L - 1
+    _check(q, "q", dt, device=dev)
+    _check(k, "k", dt, shape=(B, H, d_k), device=dev)
+    _check(v, "v", dt, shape=(B, H, d_v), device=dev)
+    _check(gamma, "gamma", torch.float32, shape=(B, H), device=dev)
+    _check(beta, "beta", torch.float32, shape=(B, H), device=dev)
+    _check(conv_w, "conv_w", torch.float32, shape=(H, d_v, W), device=dev)
+    _check(S, "S", torch.float32, shape=(B, H, d_v, d_k), device=dev)
+    if L > 1:
+        _check(u, "u", dt, shape=(B, H, m, d_k), device=dev)
+        _check(gain, "gain", dt, shape=(B, H, m, d_v), device=dev)
+        _check(alpha, "alpha", torch.float32, shape=(B, H, m), device=dev)
+    _check(conv_state, "conv_state", dt, required=W > 1, shape=(B, H, W - 1, d_v), device=dev)
     if o is None:
-        o = torch.empty((B, H, d_v), dtype=dt, device=q.device)
-    rc = lib().prism_decode_step(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
-        _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
-        _ptr(conv_w), _ptr(conv_state if W > 1 else None), _ptr(S),
-        B, H, d_k, d_v, L, W, code, chain_code, _ptr(o), _stream_handle(stream))
+        o = torch.empty((B, H, d_v), dtype=dt, device=dev)
+    else:
+        _check(o, "o", dt, shape=(B, H, d_v), device=dev)
+    with torch.cuda.device(dev):
+        rc = lib().prism_decode_step(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+            _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
+            _ptr(conv_w), _ptr(conv_state if W > 1 else None), _ptr(S),
+            B, H, d_k, d_v, L, W, code, chain_code, _ptr(o), _stream_handle(stream))
     if rc != 0:
         raise PrismError(rc, "prism_decode_step")
     return o
@@ -327,9 +376,10 @@ def state_affine(S, M, N=None, out=None, stream=None):
     """out = S M + N per (batch, head) on CUDA fp32 tensors: S, N [..., d_v, d_k], M
     [..., d_k, d_k] with the same leading dimensions (the composition step of per-segment
     state maps).  N may be None (zero); out may be S or N."""
-    _check(S, "S", torch.float32)
-    _check(M, "M", torch.float32)
-    _check(N, "N", torch.float32, required=False)
+    dev = _call_device(S, stream)
+    _check(S, "S", torch.float32, device=dev)
+    _check(M, "M", torch.float32, device=dev)
+    _check(N, "N", torch.float32, required=False, device=dev)
     d_v, d_k = S.shape[-2], S.shape[-1]
     if tuple(M.shape) != tuple(S.shape[:-2]) + (d_k, d_k):
         raise ValueError(f"M must be {tuple(S.shape[:-2]) + (d_k, d_k)}, got {tuple(M.shape)}")
@@ -338,11 +388,10 @@ def state_affine(S, M, N=None, out=None, stream=None):
     if out is None:
         out = torch.empty_like(S)
     else:
-        _check(out, "out", torch.float32)
-        if tuple(out.shape) != tuple(S.shape):
-            raise ValueError(f"out must be {tuple(S.shape)}, got {tuple(out.shape)}")
+        _check(out, "out", torch.float32, shape=S.shape, device=dev)
     BH = S.numel() // (d_v * d_k)
-    rc = lib().prism_state_affine(_ptr(S), _ptr(M), _ptr(N), _ptr(out), BH, d_v, d_k, _stream_handle(stream))
+    with torch.cuda.device(dev):
+        rc = lib().prism_state_affine(_ptr(S), _ptr(M), _ptr(N), _ptr(out), BH, d_v, d_k, _stream_handle(stream))
     if rc != 0:
         raise PrismError(rc, "prism_state_affine")
     return out
@@ -353,23 +402,10 @@ def scan_bwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, dO, L: int, S0=None, 
     """Gradients of <o, dO> + <S_final, dS_final> on CUDA tensors (fp32); returns a dict
     with keys q, k, v, gamma, beta, conv_w, S0 and (L > 1) u, alpha, gain."""
     chain_code = _chain_code(chain)
-    dt = q.dtype
-    code = _dtype_code(q)
-    for name, t in (("q", q), ("k", k), ("v", v), ("dO", dO)):
-        _check(t, name, dt)
-    for name, t in (("gamma", gamma), ("beta", beta), ("conv_w", conv_w)):
-        _check(t, name, torch.float32)
-    if L > 1:
-        _check(u, "u", dt)
-        _check(gain, "gain", dt)
-        _check(alpha, "alpha", torch.float32)
-    _check(S0, "S0", torch.float32, required=False)
-    _check(dS_final, "dS_final", torch.float32, required=False)
-    _check(lengths, "lengths", torch.int32, required=False)
-    B, T, H, d_k = q.shape
-    d_v = v.shape[-1]
-    W = conv_w.shape[-1]
-    f32 = dict(dtype=torch.float32, device=q.device)
+    (B, T, H, d_k, d_v, W, code), dev, _, _ = _scan_checks(
+        q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, dO, None, False, stream)
+    _check(dS_final, "dS_final", torch.float32, required=False, shape=(B, H, d_v, d_k), device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
     g = {"q": torch.empty(q.shape, **f32), "k": torch.empty(k.shape, **f32), "v": torch.empty(v.shape, **f32),
          "gamma": torch.empty(gamma.shape, **f32), "beta": torch.empty(beta.shape, **f32),
          "conv_w": torch.empty(conv_w.shape, **f32), "S0": torch.empty((B, H, d_v, d_k), **f32)}
@@ -379,15 +415,18 @@ def scan_bwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, dO, L: int, S0=None, 
         g["gain"] = torch.empty(gain.shape, **f32)
     ws_bytes = int(lib().prism_scan_bwd_workspace_size(B, T, H, d_k, d_v, L, W, code))
     if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
-    rc = lib().prism_scan_bwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
-        _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
-        _ptr(conv_w), _ptr(S0), _ptr(lengths), _ptr(dO), _ptr(dS_final),
-        B, T, H, d_k, d_v, L, W, code, chain_code,
-        _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["gamma"]), _ptr(g["beta"]),
-        _ptr(g.get("u")), _ptr(g.get("alpha")), _ptr(g.get("gain")), _ptr(g["conv_w"]), _ptr(g["S0"]),
-        _ptr(workspace), workspace.numel(), _stream_handle(stream))
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    else:
+        _check(workspace, "workspace", torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib().prism_scan_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
+            _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
+            _ptr(conv_w), _ptr(S0), _ptr(lengths), _ptr(dO), _ptr(dS_final),
+            B, T, H, d_k, d_v, L, W, code, chain_code,
+            _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["gamma"]), _ptr(g["beta"]),
+            _ptr(g.get("u")), _ptr(g.get("alpha")), _ptr(g.get("gain")), _ptr(g["conv_w"]), _ptr(g["S0"]),
+            _ptr(workspace), workspace.numel(), _stream_handle(stream))
     if rc != 0:
         raise PrismError(rc, "prism_scan_bwd")
     return g

@@ -37,15 +37,16 @@ int g_arch_ok[kMaxDevices] = {};  // 0 unknown, 1 sm_100, -1 other
 constexpr long long kDefaultSpinLimit = 1ll << 18;  // polls; each may suspend up to 20 us
 std::atomic<long long> g_spin_limit{kDefaultSpinLimit};
 
-// Scratch of prism_scan_fwd_static: a device-global array, so that entry point allocates
-// nothing.  Its address is looked up once per device.
-constexpr size_t kStaticWorkspaceBytes = (size_t)PRISM_STATIC_WORKSPACE_BYTES;
-static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
-void* g_static_ws_ptr[kMaxDevices] = {};
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ranges_overlap(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + b_bytes && y < x + a_bytes;
+}
 bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
+}  // namespace
+
+namespace prism {
 // Device-side status word address and architecture check for the current device.
 int device_setup(int** status_out) {
   int dev = 0;
@@ -69,21 +70,6 @@ int device_setup(int** status_out) {
   return PRISM_OK;
 }
 
-// Device address of g_static_workspace on the current device.
-int static_workspace(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return PRISM_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_static_ws_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_static_workspace) != cudaSuccess || !ptr) return PRISM_ERR_CUDA;
-    g_static_ws_ptr[dev] = ptr;
-  }
-  *out = g_static_ws_ptr[dev];
-  return PRISM_OK;
-}
-
 int check_sizes(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype) {
   if (B < 1 || T < 1 || H < 1 || d_k < 1 || d_v < 1 || L < 1 || W < 1 || chunk < 1)
     return PRISM_ERR_INVALID_ARG;
@@ -96,6 +82,11 @@ int check_sizes(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, 
   if (elems > 9.0e15) return PRISM_ERR_UNSUPPORTED;
   return PRISM_OK;
 }
+}  // namespace prism
+
+namespace {
+using prism::check_sizes;
+using prism::device_setup;
 
 }  // namespace
 
@@ -169,28 +160,6 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* 
   else
     err = prism::launch_recurrent_scan(p, dtype, s);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
-}
-
-int prism_scan_fwd_static(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
-                          const void* u, const float* alpha, const void* gain, const float* conv_w,
-                          const float* S0, const int32_t* lengths, int B, int T, int H, int d_k, int d_v,
-                          int L, int W, int chunk, int dtype, void* o, float* S_final, prism_stream_t stream,
-                          int chain) {
-  if (chain != PRISM_CHAIN_LINEAR && chain != PRISM_CHAIN_GELU) return PRISM_ERR_INVALID_ARG;
-  int rc = check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype);
-  if (rc != PRISM_OK) return rc;
-  const size_t need = prism_scan_fwd_workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype);
-  if (need > kStaticWorkspaceBytes) return PRISM_ERR_WORKSPACE;
-  void* ws = nullptr;
-  if (need > 0) {
-    int* status = nullptr;
-    rc = device_setup(&status);  // architecture check before the module's symbol is touched
-    if (rc != PRISM_OK) return rc;
-    rc = static_workspace(&ws);
-    if (rc != PRISM_OK) return rc;
-  }
-  return prism_scan_fwd_ex(q, k, v, gamma, beta, u, alpha, gain, conv_w, S0, lengths, B, T, H, d_k, d_v, L, W,
-                           chunk, dtype, o, S_final, ws, need > 0 ? kStaticWorkspaceBytes : 0, stream, chain);
 }
 
 int prism_scan_fwd_host(const void* host_q, const void* host_k, const void* host_v, const float* host_gamma,
@@ -285,8 +254,13 @@ int prism_stream_status(prism_stream_t stream) {
 int prism_state_affine(const float* S, const float* M, const float* N, float* out, int BH, int d_v, int d_k,
                        prism_stream_t stream) {
   if (!S || !M || !out || BH < 1 || d_v < 1 || d_k < 1) return PRISM_ERR_INVALID_ARG;
-  if (M == out) return PRISM_ERR_INVALID_ARG;  // out may alias S or N, not M
   if (!head_dim_ok(d_k) || !head_dim_ok(d_v) || BH > 65535) return PRISM_ERR_UNSUPPORTED;
+  // out may be S or N exactly (every element is read by the thread that writes it, after
+  // its row has been staged); any other overlap with S, M or N would be read after write
+  const size_t sn_bytes = (size_t)BH * d_v * d_k * sizeof(float), m_bytes = (size_t)BH * d_k * d_k * sizeof(float);
+  if (ranges_overlap(out, sn_bytes, M, m_bytes)) return PRISM_ERR_INVALID_ARG;
+  if (out != S && ranges_overlap(out, sn_bytes, S, sn_bytes)) return PRISM_ERR_INVALID_ARG;
+  if (N && out != N && ranges_overlap(out, sn_bytes, N, sn_bytes)) return PRISM_ERR_INVALID_ARG;
   int* status = nullptr;
   const int rc = device_setup(&status);
   if (rc != PRISM_OK) return rc;

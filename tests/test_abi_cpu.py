@@ -188,3 +188,9 @@ def test_state_affine_rejects_bad_arguments_before_any_launch(L):
     assert f(F, F + 64, F, F + 64, 4, 64, 64, None) == 1   # out aliases M
     assert f(F, F, F, F + 64, 4, 48, 64, None) == 2        # d_v not a supported head size
     assert f(F, F, F, F + 64, 70000, 64, 64, None) == 2    # more (batch, head) pairs than one grid axis
+    # out overlapping an input anywhere but exactly at S or N: read after write, rejected
+    S, M, N = 0x100000, 0x200000, 0x300000  # 64 KB regions: BH = 1, d = 128, fp32
+    assert f(S, M, N, S + 256, 1, 128, 128, None) == 1      # out inside S at an offset
+    assert f(S, M, N, N + 64, 1, 128, 128, None) == 1       # out inside N at an offset
+    assert f(S, M, N, M - 4096, 1, 128, 128, None) == 1     # out's tail covers the start of M
+    assert f(S, M, None, S - 65536 + 16, 1, 128, 128, None) == 1  # out's tail covers the start of S

@@ -8,7 +8,7 @@ import torch
 
 import linear_attention_sequence_shortconv_b200 as prism
 from linear_attention_sequence_shortconv_b200 import seqshard, synth
-from oracle import prism_seq
+from oracle import max_abs_rel_err, prism_seq
 
 pytestmark = pytest.mark.gpu
 
@@ -55,8 +55,15 @@ def _sharded_on_gpu(w, bounds, chain="linear"):
     return torch.cat(outs, 1).float().cpu().numpy(), S_end.cpu().numpy(), o_ref, S_ref
 
 
-def _rel(x, ref):
-    return float(np.abs(x - ref).max() / max(np.abs(ref).max(), 1e-6))
+def _rel_o(o, o_ref):
+    """The forward bars' metric on outputs [B, T, H, d_v]: max-abs-relative error per
+    (batch, head) slice, the largest over slices."""
+    return max_abs_rel_err(o, o_ref)
+
+
+def _rel_S(S, S_ref):
+    """The same metric on states [B, H, d_v, d_k], one slice per (batch, head)."""
+    return max_abs_rel_err(S, S_ref, slice_axes=(0, 1))
 
 
 def test_sharded_bf16_tensor_core_segments():
@@ -64,13 +71,52 @@ def test_sharded_bf16_tensor_core_segments():
     scan), segments of 128 tokens plus 3 history tokens (a ragged last chunk)."""
     w = synth.WORKLOADS["lm_130m"].replace(B=2, T=512, H=2, with_s0=True, seed=41)
     o, S, o_ref, S_ref = _sharded_on_gpu(w, [0, 128, 256, 384, 512])
-    assert _rel(o, o_ref) <= 2e-2
-    assert _rel(S, S_ref) <= 2e-2
+    assert _rel_o(o, o_ref) <= 2e-2
+    assert _rel_S(S, S_ref) <= 2e-2
 
 
 def test_sharded_fp32_uneven_segments_ragged_lengths():
     w = synth.Workload("shard_fp32", B=3, T=150, H=2, d_k=64, d_v=64, L=3, chunk=64, W=4, dtype="fp32",
                        lengths_lo=40, with_s0=True, seed=42)
     o, S, o_ref, S_ref = _sharded_on_gpu(w, [0, 37, 100, 150], chain="gelu")
-    assert _rel(o, o_ref) <= 1e-4
-    assert _rel(S, S_ref) <= 1e-4
+    assert _rel_o(o, o_ref) <= 1e-4
+    assert _rel_S(S, S_ref) <= 1e-4
+
+
+@pytest.mark.parametrize("P", [4, 8])
+def test_segmented_bf16_tensor_core_segments(P):
+    """scan_fwd_segmented on one device: each sequence cut into P segments that run side
+    by side on the tensor-core scan (d = 128, L = 4, bf16), with S0 and ragged lengths,
+    against the oracle's scan of the whole sequence."""
+    w = synth.WORKLOADS["lm_130m"].replace(B=2, T=700, H=2, with_s0=True, lengths_lo=300, seed=43)
+    inp = synth.make_inputs(w)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    o, S = seqshard.scan_fwd_segmented(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"],
+                                       d["gain"], d["conv_w"], w.L, P, S0=d["S0"], lengths=d["lengths"])
+    torch.cuda.synchronize()
+    assert prism.stream_status() == 0
+    o_ref, S_ref = prism_seq(**synth.to_float64_numpy(inp))
+    o = o.float().cpu().numpy()
+    assert _rel_o(o, o_ref) <= 2e-2
+    assert _rel_S(S.cpu().numpy(), S_ref) <= 2e-2
+    lens = inp["lengths"].numpy()
+    for b, n in enumerate(lens):
+        assert np.all(o[b, n:] == 0)
+
+
+@pytest.mark.parametrize("P", [4, 8])
+def test_segmented_fp32_gelu_ragged(P):
+    """The same on the fp32 build with the exact GELU chain (1e-4 bar), T not a multiple
+    of P, and lengths that end inside early segments."""
+    w = synth.Workload("seg_fp32", B=3, T=203, H=2, d_k=64, d_v=64, L=3, chunk=64, W=4, dtype="fp32",
+                       lengths_lo=20, with_s0=True, seed=44)
+    inp = synth.make_inputs(w)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    o, S = seqshard.scan_fwd_segmented(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"],
+                                       d["gain"], d["conv_w"], w.L, P, S0=d["S0"], lengths=d["lengths"],
+                                       chain="gelu")
+    torch.cuda.synchronize()
+    assert prism.stream_status() == 0
+    o_ref, S_ref = prism_seq(**synth.to_float64_numpy(inp), chain="gelu")
+    assert _rel_o(o.cpu().numpy(), o_ref) <= 1e-4
+    assert _rel_S(S.cpu().numpy(), S_ref) <= 1e-4

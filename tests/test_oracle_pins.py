@@ -123,6 +123,47 @@ def test_rank_of_residual_and_total_write():
             assert int((s > 1e-10 * s[0]).sum()) == L
 
 
+def test_affine_transition_eigenstructure_and_gdn_product():
+    """The transition half of affine_maps, A_t = gamma_t (I - beta_t k_t k_t^T)
+    ([summary] sec. 2.1: the forgetting path is the rank-1 gated-delta transition),
+    pinned without the oracle's own scan.  Textbook facts of a rank-1 update of the
+    identity with a unit vector k: A_t is symmetric, k_t is an eigenvector with
+    eigenvalue gamma_t (1 - beta_t), every vector orthogonal to k_t has eigenvalue
+    gamma_t; padded steps give the identity.  And with the writes off (v = 0), the
+    ordered product S0 A_1 A_2 ... A_T is the final state of the separately written
+    gated-delta recurrence gdn_seq started from S0.  Dropping gamma or beta, or a
+    transposed or reversed product, fails one of these."""
+    rng = np.random.default_rng(11)
+    B, T, H, dk, dv = 2, 9, 2, 6, 5
+    d = rand_inputs(rng, B=B, T=T, H=H, dk=dk, dv=dv, L=3)
+    d["gamma"] = rng.uniform(0.3, 0.9, (B, T, H))   # both well away from 1 and 0
+    d["beta"] = rng.uniform(0.2, 0.8, (B, T, H))
+    lengths = np.array([T, T - 3])
+    A, _ = affine_maps(d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"], d["conv_w"],
+                       lengths=lengths)
+    for b in range(B):
+        for t in range(T):
+            for h in range(H):
+                a = A[b, t, h]
+                if t >= lengths[b]:
+                    np.testing.assert_array_equal(a, np.eye(dk))
+                    continue
+                k, g, be = d["k"][b, t, h], d["gamma"][b, t, h], d["beta"][b, t, h]
+                np.testing.assert_allclose(a, a.T, rtol=0, atol=1e-15)
+                np.testing.assert_allclose(a @ k, g * (1 - be) * k, rtol=0, atol=1e-14)
+                x = rng.standard_normal(dk)
+                x -= (x @ k) * k  # orthogonal to the unit key
+                np.testing.assert_allclose(a @ x, g * x, rtol=0, atol=1e-14)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    _, S_ref = gdn_seq(d["q"], d["k"], np.zeros((B, T, H, dv)), d["gamma"], d["beta"], S0=S0, lengths=lengths)
+    for b in range(B):
+        for h in range(H):
+            S = S0[b, h]
+            for t in range(T):
+                S = S @ A[b, t, h]
+            np.testing.assert_allclose(S, S_ref[b, h], rtol=0, atol=1e-13)
+
+
 def test_gain_extremes():
     """g = 0: every step keeps r_0, so dS_res = r_0 (sum_l alpha_l u_l)^T (rank 1).
     g = 1: the first step removes the whole residual, dS_res = 0 and PRISM = GDN."""
