@@ -1,0 +1,1254 @@
+// Chunkwise-parallel PRISM scan on the 5th-generation tensor cores (tcgen05), one launch.
+//
+// One CTA owns one (batch row, head) chain and walks its chunks of C = 64 tokens in
+// order; the fp32 state S (d_v x d_k) stays in tensor memory for the whole sequence.
+// Sources: ICML 2026 PRISM write-up (核心迭代形式, 消除 Token 间串行, 消除 Step 间串行,
+// 架构形式) and the PRISM technical summary (2.1, 2.2), which fix the recurrence; the
+// chunk form below is derived from it.
+//
+// Chunk algebra (token-local t, i in [0, 64); S_n = state before the chunk; G_t =
+// sum_{j<=t} log gamma_j; e_t = e^{G_t}; D[t,i] = e^{G_t - G_i}; c_i = e^{G_63 - G_i};
+// rho_{i,l} = alpha_{i,l} r_{i,l}; P_l stacks rho_{.,l} over tokens, U_l stacks u_{.,l}):
+//
+//   A[t,i]     = beta_t D[t,i] k_t.k_i        (i < t)      T = (I + A)^{-1}
+//   Bku_l[t,i] = beta_t D[t,i] k_t.u_{i,l}    (i < t)
+//   Mqk[t,i]   = D[t,i] q_t.k_i               (i <= t)     Mqu_l[t,i] = D[t,i] q_t.u_{i,l}  (i <= t)
+//   X0  = diag(beta) V - sum_l Bku_l P_l
+//   U'  = T X0,                 W' = T diag(beta e) K
+//   O_0 = Mqk U' + sum_l Mqu_l P_l,  Q' = diag(e) Q - Mqk W'
+//   Delta = U' - W' S_n^T  (the delta-rule corrections beta_t (v_t - gamma_t S_{t-1} k_t))
+//   O     = O_0 + Q' S_n^T
+//   S_{n+1} = e^{G_63} S_n + Delta^T diag(c) K + sum_l P_l^T diag(c) U_l
+//
+// Everything but the last three lines is independent of the state, so the state-dependent
+// chain of a chunk is two MMAs (Q'/W' against S_n, Delta~ against K) and two short
+// tensor-memory epilogues; the rest (the residual chain, the masked Gram products, the
+// inverse, W', Q', U', O_0 and the residual state write) is worked off by other warps.
+//
+// Tensor-core products (bf16 operands, fp32 accumulators in TMEM, M = 128, one issuing
+// thread each; "x^T" operands come from TMEM or MN-major shared memory):
+//   key     [K;Q] x K^T                     -> RKQ (token rows: A | Mqk)
+//   MqkT    [T;Mqk] x T                     -> RKQ (rows 64..127: Mqk T)
+//   a_l     [K;Q] x U_l^T                   -> RU[s] (token rows: Bku_l | Mqu_l)
+//   b_l     P~_l^T x [Bku_l;Mqu_l]^T        -> ACC  (state rows: (Bku P)^T | (Mqu P)^T)
+//   e_l     P~_l^T x U~_l                   -> RS   (the residual write of the chunk)
+//   d       [T;MqkT] x (diag(beta e) K)     -> RW   ([W'; Mqk W'])
+//   c       X0^T x [T;MqkT]^T               -> ACC  ([U'^T | O_0^T])
+//   one     S_n (TMEM) x [-W';Q']^T         -> ACC  ([Delta^T | O^T])
+//   two     Delta~^T (TMEM) x K             -> RS   (S_{n+1})
+// "Fast" chunks (G_63 >= -60) factor the decay as e^{G_t - G_63} c_i: the prologue writes
+// P~ = diag(c) P and U~ = U; other chunks use e^{G_t - G_i} per element, P~ = P and
+// U~ = diag(c) U (scaled in place).
+//
+// Warp roles (448 threads): warps 0-7 the epilogue group EG (prologue, Bku/Mqu epilogues,
+// X0, the state epilogues, o), warps 8-11 the key group KG (gate prefix, A and Mqk, the
+// inverse, Mqk T, K^, W'/Q'; issues its own MMAs), warp 12 the MMA warp (every other MMA),
+// warp 13 the TMA warp.  Hand-overs go through mbarriers; every wait is bounded and gives
+// up once another agent has set the abort flag, so a missed arrival records
+// PRISM_ERR_TIMEOUT instead of hanging the GPU.
+#include <cuda.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace prism {
+namespace {
+
+using namespace sm100;
+
+constexpr int kC = 64;            // chunk length
+constexpr int kEG = 256;          // epilogue group threads (warps 0-7)
+constexpr int kKG = 128;          // key group threads (warps 8-11)
+constexpr int kMW = 12;           // MMA warp
+constexpr int kTW = 13;           // TMA warp
+constexpr int kThreads = 448;
+constexpr uint32_t kAtom128 = 16384;  // one 128-row, 128-byte-wide swizzle atom column
+constexpr uint32_t kAtom64 = 8192;    // the same with 64 rows
+constexpr uint32_t kAtomV = 9216;     // 72 rows of v: 8 of ShortConv history, then the chunk
+constexpr long long kDrainLimit = 1ll << 18;
+constexpr int kWsLd = 68;  // fp32 row stride of the inverse's scratch (bank padding)
+
+// TMEM columns
+constexpr uint32_t kRS = 0, kACC = 128, kSB = 256, kRKQ = 320, kRU = 384, kRW = 384;
+
+template <int D>
+struct Lay {
+  static constexpr int NA = D / 64;
+  static constexpr uint32_t KQ = 0;                          // [K;Q] per atom column
+  static constexpr uint32_t KB = KQ + NA * kAtom128;         // K for the state update
+  static constexpr uint32_t UB = KB + NA * kAtom64;          // U_l, two slots
+  static constexpr uint32_t PB = UB + 2 * NA * kAtom64;      // gain -> P~_l, two slots
+  static constexpr uint32_t BQ = PB + 2 * NA * kAtom64;      // [Bku_l;Mqu_l], two slots; slot 0 also X0^T
+  static constexpr uint32_t VB = BQ + 2 * kAtom128;          // v, 72 rows
+  static constexpr uint32_t ZB = VB + NA * kAtomV;           // [T; Mqk | MqkT]
+  static constexpr uint32_t WQ = ZB + kAtom128;              // [-W'; Q']
+  static constexpr uint32_t WS_BYTES = 64 * kWsLd * 4 + 4096;
+  // the inverse's scratch lives in WQ when it fits (WQ is free while the inverse runs)
+  static constexpr uint32_t WS = (NA * kAtom128 >= WS_BYTES) ? WQ : WQ + NA * kAtom128;
+  static constexpr uint32_t TAPS = (WS == WQ) ? WQ + NA * kAtom128 : WS + ((WS_BYTES + 1023) / 1024) * 1024;
+  static constexpr uint32_t SMALL = TAPS + D * PRISM_MAX_W * 4;
+  static constexpr uint32_t BYTES = SMALL + 4096;
+  static constexpr uint32_t ALLOC = BYTES + 1024;
+  static_assert(ALLOC <= 232448, "exceeds the 227 KB opt-in shared memory of sm_100");
+};
+
+// One launch of the scan kernel.  A sequence may be cut into P segments of Ts tokens
+// (Ts a multiple of 64), one CTA each; CTA (b, h, p) scans tokens [p Ts, min((p+1) Ts, len)).
+// Its start state is S0 (p = 0), else the identity (s_in_identity), else S_in[b, h, p],
+// else zero; its end state goes to S_out[b, h, p] when S_out is set, else to S_final from
+// the last segment.  writes_off treats v and the residual writes as zero (the transitions
+// alone); write_o = 0 skips the outputs.
+struct ScanArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* gamma;
+  const float* beta;
+  const float* alpha;
+  const float* conv_w;
+  const float* S0;
+  const int32_t* lengths;
+  __nv_bfloat16* o;
+  float* S_final;
+  const float* S_in;   // [B, H, P, D, D] or NULL
+  float* S_out;        // [B, H, P, D, D] or NULL
+  int B, T, H, W, m;   // m: residual directions of this launch (0 when writes are off)
+  int P, Ts;
+  int s_in_identity, write_o, writes_off;
+  int* status;
+  long long spin_limit;
+};
+
+// Per-chunk gate tables (two slots: chunk n uses slot n & 1).
+struct Gates {
+  float G[64], beta[64], e[64], en[64], c[64], rr[64];
+  int fast, nv, pad0, pad1;
+};
+
+// Barriers (one 8-byte word each, in shared memory).
+enum Bar {
+  kKqFull, kKqFree, kKbFull, kVFull, kVFree, kUgFull0, kUgFull1, kSlotFree0, kSlotFree1, kRuFull0, kRuFull1,
+  kEpiDone0, kEpiDone1, kE1Done, kKqkFree, kBkupDone, kX0Ready, kZReady, kWqReady, kAccFull, kDlReady, kRsFull,
+  kGates0, kGates1, kGFree0, kGFree1, kKgMma, kDrain, kKgDrain, kNumBars
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ void st_bf16x8(uint8_t* base, uint32_t off, const float* x) {
+  uint4 u;
+  u.x = pack_bf16x2(x[0], x[1]);
+  u.y = pack_bf16x2(x[2], x[3]);
+  u.z = pack_bf16x2(x[4], x[5]);
+  u.w = pack_bf16x2(x[6], x[7]);
+  *reinterpret_cast<uint4*>(base + off) = u;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+  f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+}
+
+// ---------------------------------------------------------------- TMEM helpers
+__device__ __forceinline__ void tmem_ld32_raw(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32_raw(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+      "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]),
+      "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16_raw(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T: the A operand from tensor memory (lane = row of A,
+// bf16 pairs packed per 32-bit column).
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk, uint32_t atom_stride) {
+  return sdesc_sw128(base + (uint32_t)(kk >> 2) * atom_stride + (uint32_t)(kk & 3) * 32u, 16, 1024);
+}
+__device__ __forceinline__ uint64_t mndesc(uint32_t base, int kk, uint32_t lbo) {
+  return sdesc_sw128(base + (uint32_t)kk * 2048u, lbo, 1024);
+}
+
+// ---------------------------------------------------------------- barriers and waits
+__device__ __forceinline__ void eg_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool eg_sync_or(int v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q, p;\n\tsetp.ne.s32 q, %1, 0;\n\tbar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(v)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void kg_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ bool kg_sync_or(int v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q, p;\n\tsetp.ne.s32 q, %1, 0;\n\tbar.red.or.pred p, 2, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(v)
+      : "memory");
+  return r != 0;
+}
+
+// Bounded wait for the phase of parity `par`: false once the abort flag is set, or after
+// `limit` polls (then PRISM_ERR_TIMEOUT is recorded and the abort flag set).
+__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t par, long long limit, int* status,
+                                      volatile int* abort_flag) {
+  const uint32_t hint = limit < 1024 ? 0u : 20000u;
+  for (long long i = 0; i < limit; ++i) {
+    if (mbar_try_wait_suspend(bar, par, hint)) return true;
+    if (*abort_flag) return false;
+  }
+  record_status(status, PRISM_ERR_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+// The same for a whole warp: lane 0 waits, the answer is broadcast.
+__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t par, long long limit, int* status,
+                                      volatile int* abort_flag) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = bwait(bar, par, limit, status, abort_flag) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// T = (I + A)^{-1} in place for a strictly lower-triangular 64 x 64 fp32 A (row stride
+// kWsLd, zeros on and above the diagonal) by blocked forward substitution: the four
+// 16 x 16 diagonal blocks column by column, then the 16 -> 32 and 32 -> 64 merges
+// T_21 = -T_22 A_21 T_11.  Called by the key group's 128 threads (tid 0..127); sY holds
+// 1024 fp32 of scratch.
+__device__ __forceinline__ void invert_unit_lower64(float* sA, float* sY, int tid) {
+  constexpr int LDA = kWsLd;
+  {
+    float xcol[16];
+    const int blk = tid >> 4, j = tid & 15;
+    if (tid < 64) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        float acc = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < r; ++s2) acc += sA[(16 * blk + r) * LDA + 16 * blk + s2] * xcol[s2];
+        xcol[r] = (r < j) ? 0.f : (r == j ? 1.f : -acc);
+      }
+    }
+    kg_sync();
+    if (tid < 64) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) sA[(16 * blk + r) * LDA + 16 * blk + j] = xcol[r];
+    }
+    kg_sync();
+  }
+  {
+    const int pr = tid >> 6, r = (tid >> 2) & 15, c0 = (tid & 3) * 4;
+    const int I = 2 * pr + 1, J = 2 * pr;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const float a = sA[(16 * I + r) * LDA + 16 * J + u];
+      const float4 t = *reinterpret_cast<const float4*>(sA + (16 * J + u) * LDA + 16 * J + c0);
+      acc[0] += a * t.x;
+      acc[1] += a * t.y;
+      acc[2] += a * t.z;
+      acc[3] += a * t.w;
+    }
+    *reinterpret_cast<float4*>(sY + pr * 256 + r * 16 + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    kg_sync();
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      if (u <= r) {
+        const float a = sA[(16 * I + r) * LDA + 16 * I + u];
+        const float4 y = *reinterpret_cast<const float4*>(sY + pr * 256 + u * 16 + c0);
+        acc[0] += a * y.x;
+        acc[1] += a * y.y;
+        acc[2] += a * y.z;
+        acc[3] += a * y.w;
+      }
+    }
+    *reinterpret_cast<float4*>(sA + (16 * I + r) * LDA + 16 * J + c0) =
+        make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+    kg_sync();
+  }
+  {
+    const int r0 = (tid >> 3) * 2, c0 = (tid & 7) * 4;
+    float acc[2][4] = {};
+#pragma unroll 8
+    for (int u = 0; u < 32; ++u) {
+      const float4 t = *reinterpret_cast<const float4*>(sA + u * LDA + c0);
+#pragma unroll
+      for (int i2 = 0; i2 < 2; ++i2) {
+        const float a = sA[(32 + r0 + i2) * LDA + u];
+        acc[i2][0] += a * t.x;
+        acc[i2][1] += a * t.y;
+        acc[i2][2] += a * t.z;
+        acc[i2][3] += a * t.w;
+      }
+    }
+#pragma unroll
+    for (int i2 = 0; i2 < 2; ++i2)
+      *reinterpret_cast<float4*>(sY + (r0 + i2) * 32 + c0) = make_float4(acc[i2][0], acc[i2][1], acc[i2][2], acc[i2][3]);
+    kg_sync();
+#pragma unroll
+    for (int i2 = 0; i2 < 2; ++i2) acc[i2][0] = acc[i2][1] = acc[i2][2] = acc[i2][3] = 0.f;
+    const int ulim = r0 + 2;
+#pragma unroll 8
+    for (int u = 0; u < ulim; ++u) {
+      const float4 y = *reinterpret_cast<const float4*>(sY + u * 32 + c0);
+#pragma unroll
+      for (int i2 = 0; i2 < 2; ++i2) {
+        const float a = sA[(32 + r0 + i2) * LDA + 32 + u];
+        acc[i2][0] += a * y.x;
+        acc[i2][1] += a * y.y;
+        acc[i2][2] += a * y.z;
+        acc[i2][3] += a * y.w;
+      }
+    }
+#pragma unroll
+    for (int i2 = 0; i2 < 2; ++i2)
+      *reinterpret_cast<float4*>(sA + (32 + r0 + i2) * LDA + c0) =
+          make_float4(-acc[i2][0], -acc[i2][1], -acc[i2][2], -acc[i2][3]);
+    kg_sync();
+  }
+}
+
+// ---------------------------------------------------------------- the kernel
+template <int D, int CH>
+__global__ void __launch_bounds__(kThreads, 1)
+    prism_scan_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_v,
+                      const __grid_constant__ CUtensorMap map_g, ScanArgs p) {
+  using Ly = Lay<D>;
+  constexpr int NA = Ly::NA;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sKQ = sm + Ly::KQ;
+  uint8_t* sKB = sm + Ly::KB;
+  uint8_t* sBQ0 = sm + Ly::BQ;
+  uint8_t* sVB = sm + Ly::VB;
+  uint8_t* sZB = sm + Ly::ZB;
+  uint8_t* sWQ = sm + Ly::WQ;
+  float* sWS = reinterpret_cast<float*>(sm + Ly::WS);
+  float* sTaps = reinterpret_cast<float*>(sm + Ly::TAPS);  // [w][c]
+  Gates* sGates = reinterpret_cast<Gates*>(sm + Ly::SMALL);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::SMALL + 2 * sizeof(Gates));
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  static_assert(2 * sizeof(Gates) + 8 * kNumBars + 8 <= 4096, "small region");
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P, b = bh / p.H, h = bh % p.H;
+  const int T = p.T, H = p.H, m = p.m;
+  const int len = p.lengths ? min(max(p.lengths[b], 0), T) : T;
+  const int tok0 = seg * p.Ts;                         // first token of this CTA's segment
+  const int seg_end = min(tok0 + p.Ts, T);             // end of the segment
+  const int vend = min(len, seg_end);                  // end of its valid tokens
+  const int nchunks = vend > tok0 ? (vend - tok0 + kC - 1) / kC : 0;
+  const long long lim = p.spin_limit;
+  int* status = p.status;
+  const size_t DD = (size_t)D * D;
+  const float* S_start = seg == 0 ? (p.S0 ? p.S0 + (size_t)bh * DD : nullptr)
+                                  : (p.S_in ? p.S_in + ((size_t)bh * p.P + seg) * DD : nullptr);
+  const bool start_identity = seg > 0 && p.s_in_identity;
+  float* S_end = p.S_out ? p.S_out + ((size_t)bh * p.P + seg) * DD
+                         : (seg == p.P - 1 && p.S_final ? p.S_final + (size_t)bh * DD : nullptr);
+
+  if (tid == 0) {
+    // one arrival each, but the Delta hand-over: one per warp of the epilogue group's Delta half
+    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], i == kDlReady ? 4 : 1);
+    fence_mbar_init();
+    *s_abort = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  const uint32_t aKQ = smem_u32(sKQ), aKB = smem_u32(sKB), aZB = smem_u32(sZB), aWQ = smem_u32(sWQ);
+  const uint32_t aUB0 = smem_u32(sm + Ly::UB), aPB0 = smem_u32(sm + Ly::PB), aBQ0 = smem_u32(sBQ0);
+
+  if (warp == kTW) {
+    // ================================================================ TMA warp
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      if (m > 0) {
+        tma_prefetch_desc(&map_u);
+        tma_prefetch_desc(&map_g);
+      }
+    }
+    const int nug = nchunks * m;
+    int n_kq = 0, n_v = p.writes_off ? nchunks : 0, n_kb = 0, j_ug = 0;
+    bool ok = true;
+    long long idle = 0;
+    auto prefetch = [&](int n) {  // every tile of chunk n into L2
+      const int t0 = tok0 + n * kC;
+      for (int a = 0; a < NA; ++a) {
+        tma_prefetch_l2_4d(&map_k, 64 * a, h, t0, b);
+        tma_prefetch_l2_4d(&map_q, 64 * a, h, t0, b);
+        if (!p.writes_off) tma_prefetch_l2_4d(&map_v, 64 * a, h, t0 - 8, b);
+        for (int l = 0; l < m; ++l) {
+          tma_prefetch_l2_5d(&map_u, 64 * a, l, h, t0, b);
+          tma_prefetch_l2_5d(&map_g, 64 * a, l, h, t0, b);
+        }
+      }
+    };
+    while (ok && (n_kq < nchunks || n_v < nchunks || n_kb < nchunks || j_ug < nug)) {
+      bool issued = false;
+      if (lane == 0) {
+        // U_l and gain_l of direction j (slot j & 1)
+        if (j_ug < nug) {
+          const int s = j_ug & 1;
+          if (j_ug < 2 || mbar_try_wait(&bars[kSlotFree0 + s], ((j_ug >> 1) - 1) & 1)) {
+            const int n = j_ug / m, l = j_ug % m, t0 = tok0 + n * kC;
+            mbar_arrive_expect_tx(&bars[kUgFull0 + s], 2 * NA * kAtom64);
+            for (int a = 0; a < NA; ++a) {
+              tma_load_5d(sm + Ly::UB + (s * NA + a) * kAtom64, &map_u, &bars[kUgFull0 + s], 64 * a, l, h, t0, b);
+              tma_load_5d(sm + Ly::PB + (s * NA + a) * kAtom64, &map_g, &bars[kUgFull0 + s], 64 * a, l, h, t0, b);
+            }
+            ++j_ug;
+            issued = true;
+          }
+        }
+        if (n_kq < nchunks && (n_kq == 0 || mbar_try_wait(&bars[kKqFree], (n_kq - 1) & 1))) {
+          const int t0 = tok0 + n_kq * kC;
+          mbar_arrive_expect_tx(&bars[kKqFull], 2 * NA * kAtom64);
+          for (int a = 0; a < NA; ++a) {
+            tma_load_4d(sKQ + a * kAtom128, &map_k, &bars[kKqFull], 64 * a, h, t0, b);
+            tma_load_4d(sKQ + a * kAtom128 + kAtom64, &map_q, &bars[kKqFull], 64 * a, h, t0, b);
+          }
+          if (n_kq + 2 < nchunks) prefetch(n_kq + 2);
+          ++n_kq;
+          issued = true;
+        }
+        if (n_v < nchunks && (n_v == 0 || mbar_try_wait(&bars[kVFree], (n_v - 1) & 1))) {
+          mbar_arrive_expect_tx(&bars[kVFull], NA * kAtomV);
+          for (int a = 0; a < NA; ++a)
+            tma_load_4d(sVB + a * kAtomV, &map_v, &bars[kVFull], 64 * a, h, tok0 + n_v * kC - 8, b);
+          ++n_v;
+          issued = true;
+        }
+        if (n_kb < nchunks && (n_kb == 0 || mbar_try_wait(&bars[kRsFull], (n_kb - 1) & 1))) {
+          mbar_arrive_expect_tx(&bars[kKbFull], NA * kAtom64);
+          for (int a = 0; a < NA; ++a)
+            tma_load_4d(sKB + a * kAtom64, &map_k, &bars[kKbFull], 64 * a, h, tok0 + n_kb * kC, b);
+          ++n_kb;
+          issued = true;
+        }
+        if (issued) {
+          idle = 0;
+        } else {
+          if (++idle > lim * 64) {  // nothing could be issued for far longer than any wait may take
+            record_status(status, PRISM_ERR_TIMEOUT);
+            *s_abort = 1;
+          }
+          __nanosleep(200);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, *s_abort ? 0 : 1, 0) != 0;
+      n_kq = __shfl_sync(0xffffffffu, n_kq, 0);
+      n_v = __shfl_sync(0xffffffffu, n_v, 0);
+      n_kb = __shfl_sync(0xffffffffu, n_kb, 0);
+      j_ug = __shfl_sync(0xffffffffu, j_ug, 0);
+    }
+    // drain: the last phase of every barrier a load was issued on has completed
+    if (lane == 0 && *s_abort) {
+      if (n_kq > 0) mbar_wait(&bars[kKqFull], (n_kq - 1) & 1, kDrainLimit, status);
+      if (n_v > 0) mbar_wait(&bars[kVFull], (n_v - 1) & 1, kDrainLimit, status);
+      if (n_kb > 0) mbar_wait(&bars[kKbFull], (n_kb - 1) & 1, kDrainLimit, status);
+      for (int s = 0; s < 2; ++s) {
+        const int uses = (j_ug + 1 - s) / 2;  // loads issued on slot s
+        if (uses > 0) mbar_wait(&bars[kUgFull0 + s], (uses - 1) & 1, kDrainLimit, status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMW) {
+    // ================================================================ MMA warp
+    bool ok = true;
+    int j = 0;
+    auto do_be = [&](int n, int jj, int l) -> bool {  // MMA-b and MMA-e of direction jj (l of chunk n)
+      const int s = jj & 1;
+      if (!wwait(&bars[kEpiDone0 + s], (jj >> 1) & 1, lim, status, s_abort)) return false;
+      if (l == 0 && !wwait(&bars[kE1Done], n & 1, lim, status, s_abort)) return false;
+      if (lane == 0) {
+        tc_fence_after();
+        const uint32_t aP = aPB0 + s * NA * kAtom64, aU = aUB0 + s * NA * kAtom64, aB = aBQ0 + s * kAtom128;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kACC, mndesc(aP, kk, kAtom64), kdesc(aB, kk, kAtom128), idesc_bf16(128, 128, 1, 0),
+                   (l > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kRS, mndesc(aP, kk, kAtom64), mndesc(aU, kk, kAtom64), idesc_bf16(128, D, 1, 1), 1);
+        mma_commit(&bars[kSlotFree0 + s]);
+        if (l == m - 1) mma_commit(&bars[kBkupDone]);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int n = 0; n < nchunks && ok; ++n) {
+      if (m > 0) {
+        ok = wwait(&bars[kKqFull], n & 1, lim, status, s_abort);
+        for (int l = 0; l < m && ok; ++l) {
+          const int jj = j + l, s = jj & 1;
+          ok = wwait(&bars[kUgFull0 + s], (jj >> 1) & 1, lim, status, s_abort);
+          if (!ok) break;
+          if (lane == 0) {
+            tc_fence_after();
+            const uint32_t aU = aUB0 + s * NA * kAtom64;
+#pragma unroll
+            for (int kk = 0; kk < 4 * NA; ++kk)
+              mma_bf16(tmem + kRU + 64 * s, kdesc(aKQ, kk, kAtom128), kdesc(aU, kk, kAtom64),
+                       idesc_bf16(128, 64, 0, 0), kk > 0);
+            mma_commit(&bars[kRuFull0 + s]);
+            if (l == m - 1) mma_commit(&bars[kKqkFree]);
+          }
+          __syncwarp();
+          if (l >= 1) ok = do_be(n, jj - 1, l - 1);
+        }
+        if (ok) ok = do_be(n, j + m - 1, m - 1);
+        j += m;
+      } else {
+        ok = wwait(&bars[kE1Done], n & 1, lim, status, s_abort);
+      }
+      // MMA-c: [U'^T | O_0^T] onto ACC (nothing to add when the writes are off)
+      if (ok && !p.writes_off)
+        ok = wwait(&bars[kX0Ready], n & 1, lim, status, s_abort) && wwait(&bars[kZReady], n & 1, lim, status, s_abort);
+      if (ok && lane == 0 && !p.writes_off) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kACC, kdesc(aBQ0, kk, kAtom128), kdesc(aZB, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
+                   (m > 0 || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+      // MMA1: S_n x [-W';Q']^T onto ACC
+      if (ok) ok = wwait(&bars[kWqReady], n & 1, lim, status, s_abort);
+      if (ok && lane == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4 * NA; ++kk)
+          mma_ts(tmem + kACC, tmem + kSB + 8 * kk, kdesc(aWQ, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
+                 (!p.writes_off || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[kAccFull]);
+      }
+      __syncwarp();
+      // MMA2: Delta~^T x K onto RS
+      if (ok) ok = wwait(&bars[kDlReady], n & 1, lim, status, s_abort) && wwait(&bars[kKbFull], n & 1, lim, status, s_abort);
+      if (ok && lane == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + kRS, tmem + kSB + 8 * kk, mndesc(aKB, kk, kAtom64), idesc_bf16(128, D, 0, 1), 1);
+        mma_commit(&bars[kRsFull]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {  // every MMA this warp issued has completed before TMEM is freed
+      mma_commit(&bars[kDrain]);
+      mbar_wait(&bars[kDrain], 0, kDrainLimit, status);
+    }
+    __syncwarp();
+  } else if (warp >= 8) {
+    // ================================================================ key group
+    const int kt = tid - kEG;  // 0..127
+    const int q4 = warp & 3;
+    const int row = 32 * q4 + lane;  // TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
+    uint32_t ph_kg = 0;
+    bool ok = true;
+    auto kg_mma_wait = [&]() -> bool {
+      const bool r = bwait(&bars[kKgMma], ph_kg, lim, status, s_abort);
+      ph_kg ^= 1;
+      return r;
+    };
+    for (int n = 0; n < nchunks; ++n) {
+      const int g = n & 1;
+      Gates& gt = sGates[g];
+      const int t0 = tok0 + n * kC;
+      // ---- gate prefix of chunk n (warp 8)
+      bool fail = false;
+      if (n >= 2) fail = !bwait(&bars[kGFree0 + g], ((n - 2) >> 1) & 1, lim, status, s_abort);
+      if (kg_sync_or(fail)) break;
+      if (warp == 8) {
+        const int nv = min(kC, vend - t0);
+        float gl[2], bl[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          const bool valid = t < nv;
+          const size_t th = ((size_t)b * T + min(t0 + t, T - 1)) * H + h;
+          gl[e] = valid ? __ldg(p.gamma + th) : 1.f;
+          bl[e] = valid ? __ldg(p.beta + th) : 0.f;
+        }
+        const float lg0 = __logf(gl[0]), lg1 = __logf(gl[1]);
+        float x = lg0 + lg1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, x, off);
+          if (lane >= off) x += y;
+        }
+        const float G63 = __shfl_sync(0xffffffffu, x, 31);
+        const bool fast = G63 >= -60.f;
+        const float Gv[2] = {x - lg1, x};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * lane + e;
+          gt.G[t] = Gv[e];
+          gt.beta[t] = bl[e];
+          gt.e[t] = __expf(Gv[e]);
+          gt.en[t] = fast ? __expf(-Gv[e]) : 0.f;
+          gt.c[t] = __expf(G63 - Gv[e]);
+          gt.rr[t] = fast ? __expf(Gv[e] - G63) : 0.f;
+        }
+        if (lane == 0) {
+          gt.fast = fast ? 1 : 0;
+          gt.nv = nv;
+        }
+      }
+      kg_sync();
+      if (kt == 0) mbar_arrive(&bars[kGates0 + g]);
+      const bool fast = gt.fast != 0;
+      // ---- key product [K;Q] K^T
+      fail = !bwait(&bars[kKqFull], n & 1, lim, status, s_abort);
+      if (kg_sync_or(fail)) break;
+      if (kt == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4 * NA; ++kk) {
+          const uint64_t a = kdesc(aKQ, kk, kAtom128);
+          mma_bf16(tmem + kRKQ, a, a, idesc_bf16(128, 64, 0, 0), kk > 0);
+        }
+        mma_commit(&bars[kKgMma]);
+      }
+      fail = !kg_mma_wait();
+      // the inverse's scratch and ZB are free once MMA-c and MMA1 of the previous chunk are done
+      if (!fail && n >= 1) fail = !bwait(&bars[kAccFull], (n - 1) & 1, lim, status, s_abort);
+      if (kg_sync_or(fail)) break;
+      tc_fence_after();
+      {  // A (token rows 0..63, fp32 into the inverse's scratch) and Mqk (rows 64..127, bf16 into ZB)
+        const bool krow = row < 64;
+        const int t = krow ? row : row - 64;
+        const float bt = krow ? gt.beta[t] : 1.f;
+        const float et = gt.e[t], Gt = gt.G[t];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t raw[32];
+          tmem_ld32_raw(tl + kRKQ + 32 * half, raw);
+          tmem_wait_ld();
+          float x[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int i = 32 * half + e;
+            const bool keep = krow ? (i < t) : (i <= t);
+            const float dti = fast ? et * gt.en[i] : __expf(Gt - gt.G[i]);
+            x[e] = keep ? bt * dti * __uint_as_float(raw[e]) : 0.f;
+          }
+          if (krow) {
+            float4* dst = reinterpret_cast<float4*>(sWS + t * kWsLd + 32 * half);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+          } else {
+#pragma unroll
+            for (int c8 = 0; c8 < 32; c8 += 8) st_bf16x8(sZB, sw128_offset(row, 32 * half + c8, kAtom128), x + c8);
+          }
+        }
+      }
+      kg_sync();
+      invert_unit_lower64(sWS, sWS + 64 * kWsLd, kt);
+      // T -> rows 0..63 of ZB (bf16)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = q * kKG + kt, t = e >> 3, c8 = (e & 7) * 8;
+        float f[8];
+        const float4 lo = *reinterpret_cast<const float4*>(sWS + t * kWsLd + c8);
+        const float4 hi = *reinterpret_cast<const float4*>(sWS + t * kWsLd + c8 + 4);
+        f[0] = lo.x; f[1] = lo.y; f[2] = lo.z; f[3] = lo.w; f[4] = hi.x; f[5] = hi.y; f[6] = hi.z; f[7] = hi.w;
+        st_bf16x8(sZB, sw128_offset(t, c8, kAtom128), f);
+      }
+      fence_proxy_async_smem();
+      kg_sync();
+      // ---- Mqk T
+      if (kt == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kRKQ, kdesc(aZB, kk, kAtom128), mndesc(aZB, kk, kAtom128), idesc_bf16(128, 64, 0, 1),
+                   kk > 0);
+        mma_commit(&bars[kKgMma]);
+      }
+      fail = !kg_mma_wait();
+      if (kg_sync_or(fail)) break;
+      tc_fence_after();
+      if (row >= 64) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t raw[32];
+          tmem_ld32_raw(tl + kRKQ + 32 * half, raw);
+          tmem_wait_ld();
+          float x[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(raw[e]);
+#pragma unroll
+          for (int c8 = 0; c8 < 32; c8 += 8) st_bf16x8(sZB, sw128_offset(row, 32 * half + c8, kAtom128), x + c8);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      kg_sync();
+      if (kt == 0) mbar_arrive(&bars[kZReady]);
+      // ---- K^ = diag(beta e) K in place (rows 0..63 of KQ) once the direction loop is done with K
+      if (m > 0) fail = !bwait(&bars[kKqkFree], n & 1, lim, status, s_abort);
+      if (kg_sync_or(fail)) break;
+      for (int e = kt; e < 64 * (D / 8); e += kKG) {
+        const int t = e / (D / 8), c8 = (e % (D / 8)) * 8;
+        const uint32_t off = sw128_offset(t, c8, kAtom128);
+        const float sc = gt.beta[t] * gt.e[t];
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4*>(sKQ + off), f);
+#pragma unroll
+        for (int k2 = 0; k2 < 8; ++k2) f[k2] *= sc;
+        st_bf16x8(sKQ, off, f);
+      }
+      fence_proxy_async_smem();
+      // RW shares columns with RU: free once the direction loop's MMAs are done
+      if (m > 0) fail = !bwait(&bars[kBkupDone], n & 1, lim, status, s_abort);
+      if (kg_sync_or(fail)) break;
+      // ---- [W'; Mqk W'] = [T; MqkT] K^
+      if (kt == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kRW, kdesc(aZB, kk, kAtom128), mndesc(aKQ, kk, kAtom128), idesc_bf16(128, D, 0, 1),
+                   kk > 0);
+        mma_commit(&bars[kKgMma]);
+      }
+      fail = !kg_mma_wait();
+      if (kg_sync_or(fail)) break;
+      tc_fence_after();
+      // ---- [-W'; Q'] -> WQ (Q' = e Q - Mqk W')
+      {
+        const bool wrow = row < 64;
+        const int t = wrow ? row : row - 64;
+        const float et = gt.e[t];
+#pragma unroll
+        for (int pc = 0; pc < D / 32; ++pc) {
+          uint32_t raw[32];
+          tmem_ld32_raw(tl + kRW + 32 * pc, raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c8 = 0; c8 < 32; c8 += 8) {
+            const int d0 = 32 * pc + c8;
+            float f[8];
+            if (wrow) {
+#pragma unroll
+              for (int k2 = 0; k2 < 8; ++k2) f[k2] = -__uint_as_float(raw[c8 + k2]);
+            } else {
+              float qv[8];
+              unpack8(*reinterpret_cast<const uint4*>(sKQ + sw128_offset(64 + t, d0, kAtom128)), qv);
+#pragma unroll
+              for (int k2 = 0; k2 < 8; ++k2) f[k2] = et * qv[k2] - __uint_as_float(raw[c8 + k2]);
+            }
+            st_bf16x8(sWQ, sw128_offset(row, d0, kAtom128), f);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      kg_sync();
+      if (kt == 0) {
+        mbar_arrive(&bars[kWqReady]);
+        mbar_arrive(&bars[kKqFree]);
+      }
+      ok = true;
+    }
+    (void)ok;
+    if (kt == 0) {  // the group's own MMAs have completed before TMEM is freed
+      mma_commit(&bars[kKgDrain]);
+      mbar_wait(&bars[kKgDrain], 0, kDrainLimit, status);
+    }
+  } else {
+    // ================================================================ epilogue group
+    const int q4 = warp & 3, ch = warp >> 2;
+    const int row = 32 * q4 + lane;  // TMEM lane: state row c, or token row
+    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
+    const bool srow = row < D;
+    constexpr int CPT = D / 8;          // prologue threads per token
+    constexpr int TPP = kEG / CPT;      // tokens per prologue pass
+    constexpr int NPASS = kC / TPP;
+    const int pc8 = (tid % CPT) * 8;    // this thread's 8 prologue channels
+    const float* cw_head = p.conv_w + (size_t)h * D * p.W;
+    for (int e = tid; e < D * p.W; e += kEG) sTaps[(e % p.W) * D + e / p.W] = __ldg(cw_head + e);
+    eg_sync();
+    float r[NPASS][8];  // the running residual of the prologue's tokens
+    bool aborted = false;
+    int j = 0;
+    for (int n = 0; n < nchunks; ++n) {
+      const int g = n & 1;
+      Gates& gt = sGates[g];
+      const int t0 = tok0 + n * kC;
+      bool fail = !bwait(&bars[kGates0 + g], (n >> 1) & 1, lim, status, s_abort);
+      // ---- E1: S_n -> bf16 into SB (A operand of MMA1), RS <- e^{G_63} S_n
+      if (!fail && n >= 1) fail = !bwait(&bars[kRsFull], (n - 1) & 1, lim, status, s_abort);
+      if (eg_sync_or(fail)) { aborted = true; break; }
+      if (n >= 1 && tid == 0) mbar_arrive(&bars[kGFree0 + (g ^ 1)]);  // done with chunk n-1's gates
+      tc_fence_after();
+      if (srow) {  // this thread: state row c = row, columns [ch*D/2, ch*D/2 + D/2), 32 at a time
+        const float e63 = gt.e[63];
+#pragma unroll
+        for (int pc = 0; pc < D / 64; ++pc) {
+          const int c0 = ch * (D / 2) + 32 * pc;
+          uint32_t raw[32];
+          if (n == 0) {  // the segment's start state: S0, the identity, a folded state or zero
+            const float4* src = reinterpret_cast<const float4*>(S_start + (size_t)row * D + c0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float4 f = S_start ? __ldg(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+              raw[4 * e] = __float_as_uint(f.x);
+              raw[4 * e + 1] = __float_as_uint(f.y);
+              raw[4 * e + 2] = __float_as_uint(f.z);
+              raw[4 * e + 3] = __float_as_uint(f.w);
+            }
+            if (start_identity) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(c0 + e == row ? 1.f : 0.f);
+            }
+          } else {
+            tmem_ld32_raw(tl + kRS + c0, raw);
+            tmem_wait_ld();
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(__uint_as_float(raw[2 * c]), __uint_as_float(raw[2 * c + 1]));
+          tmem_st16_raw(tl + kSB + c0 / 2, pk);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(e63 * __uint_as_float(raw[c]));
+          tmem_st32_raw(tl + kRS + c0, raw);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      eg_sync();
+      if (tid == 0) mbar_arrive(&bars[kE1Done]);
+      const bool fast = gt.fast != 0;
+      const int nv = gt.nv;
+      // ---- direction loop: prologue (P~_l) and epilogue ([Bku_l; Mqu_l]) of every direction
+      for (int l = 0; l < m; ++l, ++j) {
+        const int s = j & 1;
+        uint8_t* sP = sm + Ly::PB + s * NA * kAtom64;
+        uint8_t* sU = sm + Ly::UB + s * NA * kAtom64;
+        uint8_t* sB = sBQ0 + s * kAtom128;
+        fail = !bwait(&bars[kUgFull0 + s], (j >> 1) & 1, lim, status, s_abort);
+        if (!fail && l == 0) fail = !bwait(&bars[kVFull], n & 1, lim, status, s_abort);
+        if (eg_sync_or(fail)) { aborted = true; break; }
+        // prologue: r_0 = v - anchor (l = 0), r_l = chain step, P~_l = (c_i or 1) alpha_{i,l} r_l
+#pragma unroll
+        for (int ps = 0; ps < NPASS; ++ps) {
+          const int i = ps * TPP + tid / CPT;
+          const bool valid = i < nv;
+          if (l == 0) {
+            float v0[8];
+            unpack8(*reinterpret_cast<const uint4*>(sVB + sw128_offset(8 + i, pc8 & 63, kAtomV) + (pc8 >> 6) * kAtomV), v0);
+            float a[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a[e] = sTaps[pc8 + e] * v0[e];
+            for (int w = 1; w < p.W; ++w) {
+              float vw[8];
+              unpack8(*reinterpret_cast<const uint4*>(sVB + sw128_offset(8 + i - w, pc8 & 63, kAtomV) + (pc8 >> 6) * kAtomV), vw);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) a[e] += sTaps[w * D + pc8 + e] * vw[e];
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[ps][e] = v0[e] - a[e];
+          }
+          const uint32_t off = sw128_offset(i, pc8 & 63, kAtom64) + (pc8 >> 6) * kAtom64;
+          float gv[8];
+          unpack8(*reinterpret_cast<const uint4*>(sP + off), gv);
+          const float al = valid ? __ldg(p.alpha + (((size_t)b * T + t0 + i) * H + h) * m + l) : 0.f;
+          const float sc = valid ? (fast ? al * gt.c[i] : al) : 0.f;
+          float rho[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            r[ps][e] = chain_step(r[ps][e], gv[e], CH);
+            rho[e] = sc * r[ps][e];
+          }
+          st_bf16x8(sP, off, rho);
+        }
+        fail = !bwait(&bars[kRuFull0 + s], (j >> 1) & 1, lim, status, s_abort);
+        if (eg_sync_or(fail)) { aborted = true; break; }
+        tc_fence_after();
+        // epilogue: RU[s] (token rows) -> [Bku_l; Mqu_l] bf16 in BQ[s]
+        {
+          const bool krow = row < 64;
+          const int t = krow ? row : row - 64;
+          const float bt = krow ? gt.beta[t] : 1.f;
+          uint32_t raw[32];
+          tmem_ld32_raw(tl + kRU + 64 * s + 32 * ch, raw);
+          tmem_wait_ld();
+          float x[32];
+          if (fast) {
+            const float f = bt * gt.rr[t];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int i = 32 * ch + e;
+              x[e] = (krow ? i < t : i <= t) ? f * __uint_as_float(raw[e]) : 0.f;
+            }
+          } else {
+            const float Gt = gt.G[t];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int i = 32 * ch + e;
+              x[e] = (krow ? i < t : i <= t) ? bt * __expf(Gt - gt.G[i]) * __uint_as_float(raw[e]) : 0.f;
+            }
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < 32; c8 += 8) st_bf16x8(sB, sw128_offset(row, 32 * ch + c8, kAtom128), x + c8);
+        }
+        if (!fast) {  // U~ = diag(c) U in place (MMA-a, its other reader, has completed)
+          for (int e = tid; e < 64 * (D / 8); e += kEG) {
+            const int i = e / (D / 8), c8 = (e % (D / 8)) * 8;
+            const uint32_t off = sw128_offset(i, c8 & 63, kAtom64) + (c8 >> 6) * kAtom64;
+            float f[8];
+            unpack8(*reinterpret_cast<const uint4*>(sU + off), f);
+            const float ci = gt.c[i];
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) f[k2] *= ci;
+            st_bf16x8(sU, off, f);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        eg_sync();
+        if (tid == 0) mbar_arrive(&bars[kEpiDone0 + s]);
+      }
+      if (aborted) break;
+      // ---- X0^T = beta V - (Bku P)^T -> BQ slot 0 (K-major rows c); ACC's Delta half zeroed
+      if (!p.writes_off) {
+      fail = m > 0 ? !bwait(&bars[kBkupDone], n & 1, lim, status, s_abort)
+                   : !bwait(&bars[kVFull], n & 1, lim, status, s_abort);
+      if (eg_sync_or(fail)) { aborted = true; break; }
+      tc_fence_after();
+      if (srow) {
+        float x[32];
+        if (m > 0) {
+          uint32_t raw[32];
+          tmem_ld32_raw(tl + kACC + 32 * ch, raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = -__uint_as_float(raw[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = 0.f;
+        }
+        const uint8_t* vcol = sVB + (row >> 6) * kAtomV;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int t = 32 * ch + e;
+          const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vcol + sw128_offset(8 + t, row & 63, kAtomV)));
+          x[e] += gt.beta[t] * vv;
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < 32; c8 += 8) st_bf16x8(sBQ0, sw128_offset(row, 32 * ch + c8, kAtom128), x + c8);
+        if (m > 0) {
+          uint32_t z[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) z[e] = 0u;
+          tmem_st32_raw(tl + kACC + 32 * ch, z);
+          tmem_wait_st();
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      eg_sync();
+      if (tid == 0) {
+        mbar_arrive(&bars[kX0Ready]);
+        mbar_arrive(&bars[kVFree]);
+      }
+      }
+      // ---- E2: Delta~^T -> SB (bf16, TMEM); O^T -> o
+      fail = !bwait(&bars[kAccFull], n & 1, lim, status, s_abort);
+      if (eg_sync_or(fail)) { aborted = true; break; }
+      tc_fence_after();
+      if (ch == 0) {  // Delta~^T[c, t] = c_t Delta^T[c, t] -> bf16 into SB (A operand of MMA2)
+        if (srow) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t raw[32];
+            tmem_ld32_raw(tl + kACC + 32 * half, raw);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int t = 32 * half + 2 * e;
+              pk[e] = pack_bf16x2(gt.c[t] * __uint_as_float(raw[2 * e]), gt.c[t + 1] * __uint_as_float(raw[2 * e + 1]));
+            }
+            tmem_st16_raw(tl + kSB + 16 * half, pk);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kDlReady]);
+      } else if (srow && p.write_o) {  // o[t0 + t, c] = O^T[c, t]; zero past the sequence's length
+        __nv_bfloat16* op = p.o + (((size_t)b * T + t0) * H + h) * D + row;
+        const int tmax = min(kC, seg_end - t0);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t raw[32];
+          tmem_ld32_raw(tl + kACC + 64 + 32 * half, raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int t = 32 * half + e;
+            if (t < tmax) op[(size_t)t * H * D] = __float2bfloat16_rn(t < nv ? __uint_as_float(raw[e]) : 0.f);
+          }
+        }
+      }
+    }
+    // ---- the final state, and o past the last chunk
+    if (!aborted && nchunks > 0) {
+      const bool okf = bwait(&bars[kRsFull], (nchunks - 1) & 1, lim, status, s_abort);
+      if (!eg_sync_or(!okf)) {
+        tc_fence_after();
+        if (srow && S_end) {
+#pragma unroll
+          for (int pc = 0; pc < D / 64; ++pc) {
+            const int c0 = ch * (D / 2) + 32 * pc;
+            uint32_t raw[32];
+            tmem_ld32_raw(tl + kRS + c0, raw);
+            tmem_wait_ld();
+            float4* dst = reinterpret_cast<float4*>(S_end + (size_t)row * D + c0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(raw[4 * e]), __uint_as_float(raw[4 * e + 1]),
+                                   __uint_as_float(raw[4 * e + 2]), __uint_as_float(raw[4 * e + 3]));
+          }
+        }
+      } else {
+        aborted = true;
+      }
+    }
+    if (!aborted) {
+      if (nchunks == 0 && S_end) {  // no valid token: the end state is the start state
+        for (int e = tid; e < D * D; e += kEG)
+          S_end[e] = start_identity ? (e / D == e % D ? 1.f : 0.f) : (S_start ? S_start[e] : 0.f);
+      }
+      if (p.write_o) {  // o = 0 for the segment's tokens past its last chunk
+        const int tz = tok0 + nchunks * kC;
+        const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+        for (size_t e = tid; e < (size_t)max(seg_end - tz, 0) * D; e += kEG) {
+          const int t = tz + (int)(e / D), c = (int)(e % D);
+          p.o[(((size_t)b * T + t) * H + h) * D + c] = zero;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- segment fold
+// The start states of the segments of a cut sequence.  A segment maps its start state S
+// to S M_p + N_p (M_p: the scan of the segment from the identity with the writes off;
+// N_p: from a zero start, or from S0 for the first segment, whose N is therefore already
+// its exact end state).  Sst[1] = N_0, Sst[p] = Sst[p-1] M_{p-1} + N_{p-1}.  Rows of the
+// state are independent, so one block carries one row through all segments.
+template <int D>
+__global__ void __launch_bounds__(D) segment_fold_kernel(const float* N, const float* M, float* Sst, int P) {
+  __shared__ float srow[D];
+  const int c = blockIdx.x, j = threadIdx.x;
+  const size_t bh = blockIdx.y, DD = (size_t)D * D;
+  float x = N[(bh * P) * DD + (size_t)c * D + j];
+  Sst[(bh * P + 1) * DD + (size_t)c * D + j] = x;
+  for (int q = 2; q < P; ++q) {
+    srow[j] = x;
+    __syncthreads();
+    const float* m = M + (bh * P + q - 1) * DD;
+    float acc = N[(bh * P + q - 1) * DD + (size_t)c * D + j];
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) acc += srow[i] * m[(size_t)i * D + j];
+    __syncthreads();
+    x = acc;
+    Sst[(bh * P + q) * DD + (size_t)c * D + j] = x;
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* map, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Segments of a long sequence over few chains: planned for the 148 SMs of a B200 on every
+// device, so that the plan (and with it the rounding of the results and the workspace size)
+// is a function of the sizes alone.  A plan cuts only sequences of at least 32 chunks whose
+// chains fill under half of those SMs, into segments of at least 16 chunks.
+constexpr int kPlanSMs = 148;
+struct SegPlan {
+  int P, Ts;
+};
+SegPlan plan_segments(int B, int T, int H) {
+  const int nc = (T + kC - 1) / kC, chains = B * H;
+  if (2 * chains > kPlanSMs || nc < 32) return {1, nc * kC};
+  const int P = std::min(kPlanSMs / chains, nc / 16);
+  if (P < 2) return {1, nc * kC};
+  const int cps = (nc + P - 1) / P;  // chunks per segment
+  return {(nc + cps - 1) / cps, cps * kC};
+}
+
+template <int D, int CH>
+cudaError_t set_smem_attr() {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(prism_scan_kernel<D, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Lay<D>::ALLOC);
+  });
+  return attr_err;
+}
+
+template <int D, int CH>
+cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
+  using Ly = Lay<D>;
+  cudaError_t attr_err = set_smem_attr<D, CH>();
+  if (attr_err == cudaSuccess && CH != PRISM_CHAIN_LINEAR) attr_err = set_smem_attr<D, PRISM_CHAIN_LINEAR>();
+  if (attr_err != cudaSuccess) return attr_err;
+  const cuuint64_t B = p.B, T = p.T, H = p.H;
+  const int m = p.L - 1;
+  CUtensorMap mq, mk, mu, mv, mg;
+  const cuuint64_t dims4[4] = {(cuuint64_t)D, H, T, B};
+  const cuuint64_t str4[3] = {(cuuint64_t)D * 2, H * D * 2, T * H * D * 2};
+  const cuuint32_t box4[4] = {64, 1, 64, 1};
+  const cuuint32_t box_v[4] = {64, 1, 72, 1};  // a chunk's v rows and 8 rows of ShortConv history
+  if (!encode(&mq, p.q, 4, dims4, str4, box4) || !encode(&mk, p.k, 4, dims4, str4, box4) ||
+      !encode(&mv, p.v, 4, dims4, str4, box_v))
+    return cudaErrorInvalidValue;
+  if (m > 0) {
+    const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)m, H, T, B};
+    const cuuint64_t str5[4] = {(cuuint64_t)D * 2, (cuuint64_t)m * D * 2, H * m * D * 2, T * H * m * D * 2};
+    const cuuint32_t box5[5] = {64, 1, 1, 64, 1};
+    if (!encode(&mu, p.u, 5, dims5, str5, box5) || !encode(&mg, p.gain, 5, dims5, str5, box5))
+      return cudaErrorInvalidValue;
+  } else {
+    mu = mk;
+    mg = mk;
+  }
+  const SegPlan plan = plan_segments(p.B, p.T, p.H);
+  ScanArgs a{static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
+             static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha, p.conv_w, p.S0, p.lengths,
+             static_cast<__nv_bfloat16*>(p.o), p.S_final, nullptr, nullptr, p.B, p.T, p.H, p.W, m,
+             plan.P, plan.Ts, 0, 1, 0, p.status, p.spin_limit};
+  const int grid = p.B * p.H * plan.P;
+  if (plan.P == 1) {
+    prism_scan_kernel<D, CH><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, a);
+    return cudaGetLastError();
+  }
+  // a long sequence over few chains: P segments side by side, three scans and a fold
+  const size_t seg_states = (size_t)p.B * p.H * plan.P * D * D;
+  float* wsN = static_cast<float*>(p.workspace);
+  float* wsM = wsN + seg_states;
+  float* wsS = wsM + seg_states;
+  ScanArgs aN = a;  // each segment from a zero start (the first from S0): N_p
+  aN.S_out = wsN;
+  aN.write_o = 0;
+  aN.S_final = nullptr;
+  prism_scan_kernel<D, CH><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aN);
+  ScanArgs aM = aN;  // the transitions alone from the identity: M_p
+  aM.S_out = wsM;
+  aM.s_in_identity = 1;
+  aM.writes_off = 1;
+  aM.m = 0;
+  prism_scan_kernel<D, PRISM_CHAIN_LINEAR><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aM);
+  segment_fold_kernel<D><<<dim3(D, p.B * p.H), D, 0, stream>>>(wsN, wsM, wsS, plan.P);
+  ScanArgs aF = a;  // every segment again from its exact start state: o and S_final
+  aF.S_in = wsS;
+  prism_scan_kernel<D, CH><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aF);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const ScanParams& p, cudaStream_t stream) {
+  if (p.L > 1 && p.chain == PRISM_CHAIN_GELU) return launch_dc<D, PRISM_CHAIN_GELU>(p, stream);
+  return launch_dc<D, PRISM_CHAIN_LINEAR>(p, stream);
+}
+
+}  // namespace
+
+bool chunk_scan_supported(int d_k, int d_v, int L, int W, int chunk, int dtype) {
+  return dtype == PRISM_BF16 && chunk == kC && d_k == d_v && (d_k == 64 || d_k == 128) && L >= 1 &&
+         L <= PRISM_MAX_L && W >= 1 && W <= PRISM_MAX_W;
+}
+
+size_t chunk_scan_workspace_bytes(int B, int T, int H, int D) {
+  const SegPlan plan = plan_segments(B, T, H);
+  return plan.P == 1 ? 0 : 3 * (size_t)B * H * plan.P * D * D * sizeof(float);
+}
+
+cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream) {
+  if (p.d_k == 128) return launch_d<128>(p, stream);
+  if (p.d_k == 64) return launch_d<64>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace prism

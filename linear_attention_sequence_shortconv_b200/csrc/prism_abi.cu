@@ -10,9 +10,9 @@ cudaError_t launch_recurrent_scan(const ScanParams& p, int dtype, cudaStream_t s
 cudaError_t launch_prologue(const void* v, const float* alpha, const void* gain, const float* conv_w,
                             const int32_t* lengths, int B, int T, int H, int d_v, int L, int W,
                             int dtype, float* rho, cudaStream_t stream, int chain);
-bool chunk_tc_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
-cudaError_t launch_chunk_tc(const ScanParams& p, cudaStream_t stream);
-size_t chunk_tc_workspace_bytes(int B, int T, int H);
+bool chunk_scan_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
+cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream);
+size_t chunk_scan_workspace_bytes(int B, int T, int H, int D);
 cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, cudaStream_t stream);
 size_t bwd_smem_bytes(int d_k, int d_v, int L);
@@ -115,8 +115,10 @@ void prism_set_spin_limit(long long limit) {
 size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
                                      int dtype) {
   if (check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype) != PRISM_OK) return 0;
-  // the tensor-core path keeps the inverse T of every chunk (bf16 64 x 64) in the workspace
-  if (prism::chunk_tc_supported(d_k, d_v, L, W, chunk, dtype)) return prism::chunk_tc_workspace_bytes(B, T, H);
+  // the tensor-core scan cuts long sequences over few chains into segments: three fp32
+  // states per segment (its maps from zero and from the identity, and its start state)
+  if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype))
+    return prism::chunk_scan_workspace_bytes(B, T, H, d_k);
   return 0;
 }
 
@@ -155,8 +157,8 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* 
                       need > 0 ? workspace : nullptr};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t err;
-  if (prism::chunk_tc_supported(d_k, d_v, L, W, chunk, dtype))
-    err = prism::launch_chunk_tc(p, s);
+  if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype))
+    err = prism::launch_chunk_scan(p, s);
   else
     err = prism::launch_recurrent_scan(p, dtype, s);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
@@ -236,7 +238,7 @@ int prism_prologue_fwd_ex(const void* v, const float* alpha, const void* gain, c
 
 int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype) {
   if (check_sizes(1, 1, 1, d_k, d_v, L, W, chunk, dtype) != PRISM_OK) return 0;
-  return prism::chunk_tc_supported(d_k, d_v, L, W, chunk, dtype) ? 1 : 0;
+  return prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype) ? 1 : 0;
 }
 
 int prism_stream_status(prism_stream_t stream) {

@@ -77,18 +77,46 @@ def test_L1_needs_no_residual_inputs(L):
     assert call(L, L=1, u=None, alpha=None, gain=None, B=0) == 1
 
 
+def _segments(B, T, H):
+    """Segments per sequence of the tensor-core scan: long sequences (>= 32 chunks of 64)
+    whose chains fill under half of a B200's 148 SMs are cut into segments of >= 16 chunks."""
+    nc, chains = -(-T // 64), B * H
+    if 2 * chains > 148 or nc < 32:
+        return 1
+    P = min(148 // chains, nc // 16)
+    if P < 2:
+        return 1
+    cps = -(-nc // P)
+    return -(-nc // cps)
+
+
 def test_workspace_size_query(L):
-    # tensor-core path: one bf16 64 x 64 inverse per (b, h, chunk); other paths need none
-    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) == 16 * 6 * 32 * 64 * 64 * 2
-    assert prism.workspace_size(2, 100, 3, 64, 64, 2, 4, 64, 0) == 2 * 3 * 2 * 8192
+    # the single-launch scan keeps everything on chip; only a cut sequence needs three fp32
+    # states per segment (its two maps and its start state)
+    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) == 0     # the 130M-LM layer
+    assert prism.workspace_size(128, 1024, 2, 64, 64, 4, 4, 64, 0) == 0     # recsys
+    P = _segments(1, 65536, 8)
+    assert P == 18
+    assert prism.workspace_size(1, 65536, 8, 128, 128, 8, 4, 64, 0) == 3 * 8 * P * 128 * 128 * 4
+    assert prism.workspace_size(2, 4096, 1, 64, 64, 2, 4, 64, 0) == 3 * 2 * _segments(2, 4096, 1) * 64 * 64 * 4
     assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 1) == 0   # fp32: token-by-token kernel
-    assert prism.workspace_size(1, 64, 8, 128, 128, 8, 4, 64, 0) == 0       # L = 8: token-by-token kernel
     assert prism.workspace_size(0, 64, 8, 128, 128, 4, 4, 64, 0) == 0       # invalid sizes
 
 
+def test_workspace_never_exceeds_the_static_scratch(L):
+    # chains x segments never exceeds 148, so no shape needs more than 3 x 148 x 128^2 fp32
+    worst = 0
+    for B in (1, 2, 3, 5, 8, 37, 74):
+        for H in (1, 2, 4, 8):
+            for T in (64, 2047, 2048, 65536, 1 << 20):
+                worst = max(worst, prism.workspace_size(B, T, H, 128, 128, 8, 4, 64, 0))
+    assert 0 < worst <= 3 * 148 * 128 * 128 * 4 <= 32 << 20
+
+
 def test_missing_workspace_is_rejected_before_launch(L):
-    # the tensor-core shapes need a workspace; without one the call fails before any launch
-    assert call(L, workspace_ok=False) == 3
+    # a cut sequence needs a workspace; without one the call fails before any launch
+    assert L.prism_scan_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                            1, 65536, 8, 128, 128, 8, 4, 64, 0, FAKE, None, None, 0, None) == 3
 
 
 def test_prologue_invalid_arguments(L):

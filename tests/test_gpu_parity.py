@@ -85,6 +85,38 @@ def test_long_context_full_size_final_state_sampled():
     assert rel_err(S[0, 5], states[0]) <= TOL["bf16"]
 
 
+# ---------------------------------------------------------------- cut sequences
+SEGMENTED = {
+    # 33 chunks over 2 chains: two segments, a ragged last chunk, S0, L = 8
+    "two_segments": synth.Workload("seg2", B=1, T=2100, H=2, d_k=128, d_v=128, L=8, chunk=64, with_s0=True, seed=5),
+    # two segments per row; row 0 ends inside the first one, so its second segment is empty
+    "ragged": synth.Workload("segr", B=2, T=2600, H=1, d_k=128, d_v=128, L=4, chunk=64, with_s0=True, seed=6),
+    # d = 64, one chain cut into four segments, the exact GELU chain
+    "d64": synth.Workload("seg64", B=1, T=4096, H=1, d_k=64, d_v=64, L=3, chunk=64, seed=7),
+}
+
+
+@pytest.mark.parametrize("name", list(SEGMENTED))
+def test_segmented_long_sequences(name):
+    """Long sequences over few chains run as segments side by side (three scans and a fold
+    of the per-segment state maps); outputs and final states against the token loop."""
+    import linear_attention_sequence_shortconv_b200 as prism
+
+    w = SEGMENTED[name]
+    assert prism.workspace_size(w.B, w.T, w.H, w.d_k, w.d_v, w.L, w.W, w.chunk, 0) > 0  # the cut path
+    inp = synth.make_inputs(w)
+    if name == "ragged":
+        inp["lengths"] = torch.tensor([700, 2600], dtype=torch.int32)
+    chain = "gelu" if name == "d64" else "linear"
+    o, S = gpu_run(inp, w, chain=chain)
+    assert prism.stream_status() == 0
+    o_ref, S_ref = oracle_run(inp, w, chain=chain)
+    assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
+    if name == "ragged":
+        assert np.all(o[0, 700:] == 0)
+
+
 # ---------------------------------------------------------------- edge cases
 @pytest.mark.parametrize("T", [1, 2, 3, 63, 64, 65])
 def test_short_and_boundary_lengths(T):
