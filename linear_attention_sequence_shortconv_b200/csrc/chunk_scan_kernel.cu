@@ -90,7 +90,8 @@ struct Lay {
   static constexpr uint32_t WS = (NA * kAtom128 >= WS_BYTES) ? WQ : WQ + NA * kAtom128;
   static constexpr uint32_t TAPS = (WS == WQ) ? WQ + NA * kAtom128 : WS + ((WS_BYTES + 1023) / 1024) * 1024;
   static constexpr uint32_t SMALL = TAPS + D * PRISM_MAX_W * 4;
-  static constexpr uint32_t BYTES = SMALL + 4096;
+  static constexpr uint32_t ALPHA = SMALL + 4096;  // [2][64][PRISM_MAX_L - 1] fp32 step sizes
+  static constexpr uint32_t BYTES = ALPHA + 2 * 64 * (PRISM_MAX_L - 1) * 4;
   static constexpr uint32_t ALLOC = BYTES + 1024;
   static_assert(ALLOC <= 232448, "exceeds the 227 KB opt-in shared memory of sm_100");
 };
@@ -132,7 +133,7 @@ struct Gates {
 enum Bar {
   kKqFull, kKqFree, kKbFull, kVFull, kVFree, kUgFull0, kUgFull1, kSlotFree0, kSlotFree1, kRuFull0, kRuFull1,
   kEpiDone0, kEpiDone1, kE1Done, kKqkFree, kBkupDone, kX0Ready, kZReady, kWqReady, kAccFull, kDlReady, kRsFull,
-  kGates0, kGates1, kGFree0, kGFree1, kKgMma, kDrain, kKgDrain, kNumBars
+  kGates0, kGates1, kGFree0, kGFree1, kKgMma, kDrain, kKgDrain, kRwFull, kNumBars
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -363,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sWQ = sm + Ly::WQ;
   float* sWS = reinterpret_cast<float*>(sm + Ly::WS);
   float* sTaps = reinterpret_cast<float*>(sm + Ly::TAPS);  // [w][c]
+  float* sAlpha = reinterpret_cast<float*>(sm + Ly::ALPHA);  // [slot][t][l]
   Gates* sGates = reinterpret_cast<Gates*>(sm + Ly::SMALL);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::SMALL + 2 * sizeof(Gates));
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + kNumBars);
@@ -387,8 +389,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                          : (seg == p.P - 1 && p.S_final ? p.S_final + (size_t)bh * DD : nullptr);
 
   if (tid == 0) {
-    // one arrival each, but the Delta hand-over: one per warp of the epilogue group's Delta half
-    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], i == kDlReady ? 4 : 1);
+    // one arrival each, except the epilogue group's hand-overs: one per warp (8, or the 4
+    // warps of the Delta half), so that its warps never wait for one another
+    for (int i = 0; i < kNumBars; ++i) {
+      const bool eg8 = i == kE1Done || i == kEpiDone0 || i == kEpiDone1 || i == kX0Ready || i == kVFree ||
+                       i == kWqReady || i == kKqFree || i == kGFree0 || i == kGFree1;
+      mbar_init(&bars[i], i == kDlReady ? 4 : eg8 ? 8 : 1);
+    }
     fence_mbar_init();
     *s_abort = 0;
   }
@@ -406,109 +413,107 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTW) {
     // ================================================================ TMA warp
+    // Lane 0 issues every load in one fixed order that follows their consumption, waiting
+    // (bounded) for each buffer to be released: chunk n's directions from the third on,
+    // then the next chunk's first two directions, its v, [K;Q] and K.  Every wait is on a
+    // release that needs only loads issued before it, so the order cannot deadlock.
     if (lane == 0) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
-      if (m > 0) {
-        tma_prefetch_desc(&map_u);
-        tma_prefetch_desc(&map_g);
-      }
-    }
-    const int nug = nchunks * m;
-    int n_kq = 0, n_v = p.writes_off ? nchunks : 0, n_kb = 0, j_ug = 0;
-    bool ok = true;
-    long long idle = 0;
-    auto prefetch = [&](int n) {  // every tile of chunk n into L2
-      const int t0 = tok0 + n * kC;
-      for (int a = 0; a < NA; ++a) {
-        tma_prefetch_l2_4d(&map_k, 64 * a, h, t0, b);
-        tma_prefetch_l2_4d(&map_q, 64 * a, h, t0, b);
-        if (!p.writes_off) tma_prefetch_l2_4d(&map_v, 64 * a, h, t0 - 8, b);
-        for (int l = 0; l < m; ++l) {
-          tma_prefetch_l2_5d(&map_u, 64 * a, l, h, t0, b);
-          tma_prefetch_l2_5d(&map_g, 64 * a, l, h, t0, b);
-        }
-      }
-    };
-    while (ok && (n_kq < nchunks || n_v < nchunks || n_kb < nchunks || j_ug < nug)) {
-      bool issued = false;
-      if (lane == 0) {
-        // U_l and gain_l of direction j (slot j & 1)
-        if (j_ug < nug) {
-          const int s = j_ug & 1;
-          if (j_ug < 2 || mbar_try_wait(&bars[kSlotFree0 + s], ((j_ug >> 1) - 1) & 1)) {
-            const int n = j_ug / m, l = j_ug % m, t0 = tok0 + n * kC;
-            mbar_arrive_expect_tx(&bars[kUgFull0 + s], 2 * NA * kAtom64);
-            for (int a = 0; a < NA; ++a) {
-              tma_load_5d(sm + Ly::UB + (s * NA + a) * kAtom64, &map_u, &bars[kUgFull0 + s], 64 * a, l, h, t0, b);
-              tma_load_5d(sm + Ly::PB + (s * NA + a) * kAtom64, &map_g, &bars[kUgFull0 + s], 64 * a, l, h, t0, b);
-            }
-            ++j_ug;
-            issued = true;
+      int n_kq = 0, n_v = 0, n_kb = 0, j_ug = 0;  // loads issued per stream
+      auto prefetch = [&](int n) {  // every tile of chunk n into L2
+        const int t0 = tok0 + n * kC;
+        for (int a = 0; a < NA; ++a) {
+          tma_prefetch_l2_4d(&map_k, 64 * a, h, t0, b);
+          tma_prefetch_l2_4d(&map_q, 64 * a, h, t0, b);
+          if (!p.writes_off) tma_prefetch_l2_4d(&map_v, 64 * a, h, t0 - 8, b);
+          for (int l = 0; l < m; ++l) {
+            tma_prefetch_l2_5d(&map_u, 64 * a, l, h, t0, b);
+            tma_prefetch_l2_5d(&map_g, 64 * a, l, h, t0, b);
           }
         }
-        if (n_kq < nchunks && (n_kq == 0 || mbar_try_wait(&bars[kKqFree], (n_kq - 1) & 1))) {
-          const int t0 = tok0 + n_kq * kC;
-          mbar_arrive_expect_tx(&bars[kKqFull], 2 * NA * kAtom64);
-          for (int a = 0; a < NA; ++a) {
-            tma_load_4d(sKQ + a * kAtom128, &map_k, &bars[kKqFull], 64 * a, h, t0, b);
-            tma_load_4d(sKQ + a * kAtom128 + kAtom64, &map_q, &bars[kKqFull], 64 * a, h, t0, b);
-          }
-          if (n_kq + 2 < nchunks) prefetch(n_kq + 2);
-          ++n_kq;
-          issued = true;
+      };
+      auto ld_ug = [&](int j) -> bool {  // U_l and gain_l of direction j into slot j & 1
+        const int s = j & 1;
+        if (j >= 2 && !bwait(&bars[kSlotFree0 + s], ((j >> 1) - 1) & 1, lim, status, s_abort)) return false;
+        const int t0 = tok0 + (j / m) * kC, l = j % m;
+        mbar_arrive_expect_tx(&bars[kUgFull0 + s], 2 * NA * kAtom64);
+        for (int a = 0; a < NA; ++a) {
+          tma_load_5d(sm + Ly::UB + (s * NA + a) * kAtom64, &map_u, &bars[kUgFull0 + s], 64 * a, l, h, t0, b);
+          tma_load_5d(sm + Ly::PB + (s * NA + a) * kAtom64, &map_g, &bars[kUgFull0 + s], 64 * a, l, h, t0, b);
         }
-        if (n_v < nchunks && (n_v == 0 || mbar_try_wait(&bars[kVFree], (n_v - 1) & 1))) {
-          mbar_arrive_expect_tx(&bars[kVFull], NA * kAtomV);
-          for (int a = 0; a < NA; ++a)
-            tma_load_4d(sVB + a * kAtomV, &map_v, &bars[kVFull], 64 * a, h, tok0 + n_v * kC - 8, b);
-          ++n_v;
-          issued = true;
+        ++j_ug;
+        return true;
+      };
+      auto ld_kq = [&](int n) -> bool {
+        if (n >= 1 && !bwait(&bars[kKqFree], (n - 1) & 1, lim, status, s_abort)) return false;
+        const int t0 = tok0 + n * kC;
+        mbar_arrive_expect_tx(&bars[kKqFull], 2 * NA * kAtom64);
+        for (int a = 0; a < NA; ++a) {
+          tma_load_4d(sKQ + a * kAtom128, &map_k, &bars[kKqFull], 64 * a, h, t0, b);
+          tma_load_4d(sKQ + a * kAtom128 + kAtom64, &map_q, &bars[kKqFull], 64 * a, h, t0, b);
         }
-        if (n_kb < nchunks && (n_kb == 0 || mbar_try_wait(&bars[kRsFull], (n_kb - 1) & 1))) {
-          mbar_arrive_expect_tx(&bars[kKbFull], NA * kAtom64);
-          for (int a = 0; a < NA; ++a)
-            tma_load_4d(sKB + a * kAtom64, &map_k, &bars[kKbFull], 64 * a, h, tok0 + n_kb * kC, b);
-          ++n_kb;
-          issued = true;
+        if (n + 2 < nchunks) prefetch(n + 2);
+        ++n_kq;
+        return true;
+      };
+      auto ld_v = [&](int n) -> bool {
+        if (p.writes_off) return true;
+        if (n >= 1 && !bwait(&bars[kVFree], (n - 1) & 1, lim, status, s_abort)) return false;
+        mbar_arrive_expect_tx(&bars[kVFull], NA * kAtomV);
+        for (int a = 0; a < NA; ++a)
+          tma_load_4d(sVB + a * kAtomV, &map_v, &bars[kVFull], 64 * a, h, tok0 + n * kC - 8, b);
+        ++n_v;
+        return true;
+      };
+      auto ld_kb = [&](int n) -> bool {
+        if (n >= 1 && !bwait(&bars[kRsFull], (n - 1) & 1, lim, status, s_abort)) return false;
+        mbar_arrive_expect_tx(&bars[kKbFull], NA * kAtom64);
+        for (int a = 0; a < NA; ++a)
+          tma_load_4d(sKB + a * kAtom64, &map_k, &bars[kKbFull], 64 * a, h, tok0 + n * kC, b);
+        ++n_kb;
+        return true;
+      };
+      bool ok = true;
+      if (nchunks > 0) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_k);
+        tma_prefetch_desc(&map_v);
+        if (m > 0) {
+          tma_prefetch_desc(&map_u);
+          tma_prefetch_desc(&map_g);
         }
-        if (issued) {
-          idle = 0;
-        } else {
-          if (++idle > lim * 64) {  // nothing could be issued for far longer than any wait may take
-            record_status(status, PRISM_ERR_TIMEOUT);
-            *s_abort = 1;
-          }
-          __nanosleep(200);
+        if (nchunks > 1) prefetch(1);
+        ok = ld_kq(0) && ld_v(0) && ld_kb(0);
+        for (int l = 0; l < min(m, 2) && ok; ++l) ok = ld_ug(l);
+      }
+      for (int n = 0; n < nchunks && ok; ++n) {
+        for (int l = 2; l < m && ok; ++l) ok = ld_ug(n * m + l);
+        if (n + 1 < nchunks && ok) {
+          for (int l = 0; l < min(m, 2) && ok; ++l) ok = ld_ug((n + 1) * m + l);
+          ok = ok && ld_v(n + 1) && ld_kq(n + 1) && ld_kb(n + 1);
         }
       }
-      ok = __shfl_sync(0xffffffffu, *s_abort ? 0 : 1, 0) != 0;
-      n_kq = __shfl_sync(0xffffffffu, n_kq, 0);
-      n_v = __shfl_sync(0xffffffffu, n_v, 0);
-      n_kb = __shfl_sync(0xffffffffu, n_kb, 0);
-      j_ug = __shfl_sync(0xffffffffu, j_ug, 0);
-    }
-    // drain: the last phase of every barrier a load was issued on has completed
-    if (lane == 0 && *s_abort) {
-      if (n_kq > 0) mbar_wait(&bars[kKqFull], (n_kq - 1) & 1, kDrainLimit, status);
-      if (n_v > 0) mbar_wait(&bars[kVFull], (n_v - 1) & 1, kDrainLimit, status);
-      if (n_kb > 0) mbar_wait(&bars[kKbFull], (n_kb - 1) & 1, kDrainLimit, status);
-      for (int s = 0; s < 2; ++s) {
-        const int uses = (j_ug + 1 - s) / 2;  // loads issued on slot s
-        if (uses > 0) mbar_wait(&bars[kUgFull0 + s], (uses - 1) & 1, kDrainLimit, status);
+      // drain on an abort: the last phase of every barrier a load was issued on has completed
+      if (*s_abort) {
+        if (n_kq > 0) mbar_wait(&bars[kKqFull], (n_kq - 1) & 1, kDrainLimit, status);
+        if (n_v > 0) mbar_wait(&bars[kVFull], (n_v - 1) & 1, kDrainLimit, status);
+        if (n_kb > 0) mbar_wait(&bars[kKbFull], (n_kb - 1) & 1, kDrainLimit, status);
+        for (int s2 = 0; s2 < 2; ++s2) {
+          const int uses = (j_ug + 1 - s2) / 2;  // loads issued on slot s2
+          if (uses > 0) mbar_wait(&bars[kUgFull0 + s2], (uses - 1) & 1, kDrainLimit, status);
+        }
       }
     }
     __syncwarp();
   } else if (warp == kMW) {
-    // ================================================================ MMA warp
-    bool ok = true;
-    int j = 0;
-    auto do_be = [&](int n, int jj, int l) -> bool {  // MMA-b and MMA-e of direction jj (l of chunk n)
-      const int s = jj & 1;
-      if (!wwait(&bars[kEpiDone0 + s], (jj >> 1) & 1, lim, status, s_abort)) return false;
-      if (l == 0 && !wwait(&bars[kE1Done], n & 1, lim, status, s_abort)) return false;
-      if (lane == 0) {
+    // ================================================================ MMA warp (lane 0 issues)
+    if (lane == 0) {
+      bool ok = true;
+      int j = 0;
+      // MMA-b and MMA-e of direction jj (direction l of chunk n)
+      auto do_be = [&](int n, int jj, int l) -> bool {
+        const int s = jj & 1;
+        if (!bwait(&bars[kEpiDone0 + s], (jj >> 1) & 1, lim, status, s_abort)) return false;
+        if (l == 0 && !bwait(&bars[kE1Done], n & 1, lim, status, s_abort)) return false;
         tc_fence_after();
         const uint32_t aP = aPB0 + s * NA * kAtom64, aU = aUB0 + s * NA * kAtom64, aB = aBQ0 + s * kAtom128;
 #pragma unroll
@@ -520,18 +525,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16(tmem + kRS, mndesc(aP, kk, kAtom64), mndesc(aU, kk, kAtom64), idesc_bf16(128, D, 1, 1), 1);
         mma_commit(&bars[kSlotFree0 + s]);
         if (l == m - 1) mma_commit(&bars[kBkupDone]);
-      }
-      __syncwarp();
-      return true;
-    };
-    for (int n = 0; n < nchunks && ok; ++n) {
-      if (m > 0) {
-        ok = wwait(&bars[kKqFull], n & 1, lim, status, s_abort);
-        for (int l = 0; l < m && ok; ++l) {
-          const int jj = j + l, s = jj & 1;
-          ok = wwait(&bars[kUgFull0 + s], (jj >> 1) & 1, lim, status, s_abort);
-          if (!ok) break;
-          if (lane == 0) {
+        return true;
+      };
+      for (int n = 0; n < nchunks && ok; ++n) {
+        if (m > 0) {
+          // MMA-a of every direction, each followed by MMA-b/e of the direction before it
+          ok = bwait(&bars[kKqFull], n & 1, lim, status, s_abort);
+          for (int l = 0; l < m && ok; ++l) {
+            const int jj = j + l, s = jj & 1;
+            ok = bwait(&bars[kUgFull0 + s], (jj >> 1) & 1, lim, status, s_abort);
+            if (!ok) break;
             tc_fence_after();
             const uint32_t aU = aUB0 + s * NA * kAtom64;
 #pragma unroll
@@ -540,49 +543,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                        idesc_bf16(128, 64, 0, 0), kk > 0);
             mma_commit(&bars[kRuFull0 + s]);
             if (l == m - 1) mma_commit(&bars[kKqkFree]);
+            if (l >= 1) ok = do_be(n, jj - 1, l - 1);
           }
-          __syncwarp();
-          if (l >= 1) ok = do_be(n, jj - 1, l - 1);
+          if (ok) ok = do_be(n, j + m - 1, m - 1);
+          j += m;
+        } else {
+          ok = bwait(&bars[kE1Done], n & 1, lim, status, s_abort);
         }
-        if (ok) ok = do_be(n, j + m - 1, m - 1);
-        j += m;
-      } else {
-        ok = wwait(&bars[kE1Done], n & 1, lim, status, s_abort);
-      }
-      // MMA-c: [U'^T | O_0^T] onto ACC (nothing to add when the writes are off)
-      if (ok && !p.writes_off)
-        ok = wwait(&bars[kX0Ready], n & 1, lim, status, s_abort) && wwait(&bars[kZReady], n & 1, lim, status, s_abort);
-      if (ok && lane == 0 && !p.writes_off) {
-        tc_fence_after();
+        // MMA-c: [U'^T | O_0^T] onto ACC (nothing to add when the writes are off)
+        if (ok && !p.writes_off) {
+          ok = bwait(&bars[kX0Ready], n & 1, lim, status, s_abort) && bwait(&bars[kZReady], n & 1, lim, status, s_abort);
+          if (ok) {
+            tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kACC, kdesc(aBQ0, kk, kAtom128), kdesc(aZB, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
-                   (m > 0 || kk > 0) ? 1u : 0u);
-      }
-      __syncwarp();
-      // MMA1: S_n x [-W';Q']^T onto ACC
-      if (ok) ok = wwait(&bars[kWqReady], n & 1, lim, status, s_abort);
-      if (ok && lane == 0) {
-        tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + kACC, kdesc(aBQ0, kk, kAtom128), kdesc(aZB, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
+                       (m > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        // MMA1: S_n x [-W';Q']^T onto ACC
+        if (ok) ok = bwait(&bars[kWqReady], n & 1, lim, status, s_abort);
+        if (ok) {
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4 * NA; ++kk)
-          mma_ts(tmem + kACC, tmem + kSB + 8 * kk, kdesc(aWQ, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
-                 (!p.writes_off || kk > 0) ? 1u : 0u);
-        mma_commit(&bars[kAccFull]);
-      }
-      __syncwarp();
-      // MMA2: Delta~^T x K onto RS
-      if (ok) ok = wwait(&bars[kDlReady], n & 1, lim, status, s_abort) && wwait(&bars[kKbFull], n & 1, lim, status, s_abort);
-      if (ok && lane == 0) {
-        tc_fence_after();
+          for (int kk = 0; kk < 4 * NA; ++kk)
+            mma_ts(tmem + kACC, tmem + kSB + 8 * kk, kdesc(aWQ, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
+                   (!p.writes_off || kk > 0) ? 1u : 0u);
+          mma_commit(&bars[kAccFull]);
+        }
+        // MMA2: Delta~^T x K onto RS
+        if (ok) ok = bwait(&bars[kDlReady], n & 1, lim, status, s_abort) && bwait(&bars[kKbFull], n & 1, lim, status, s_abort);
+        if (ok) {
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kRS, tmem + kSB + 8 * kk, mndesc(aKB, kk, kAtom64), idesc_bf16(128, D, 0, 1), 1);
-        mma_commit(&bars[kRsFull]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tmem + kRS, tmem + kSB + 8 * kk, mndesc(aKB, kk, kAtom64), idesc_bf16(128, D, 0, 1), 1);
+          mma_commit(&bars[kRsFull]);
+        }
       }
-      __syncwarp();
-    }
-    if (lane == 0) {  // every MMA this warp issued has completed before TMEM is freed
+      // every MMA this thread issued has completed before TMEM is freed
       mma_commit(&bars[kDrain]);
       mbar_wait(&bars[kDrain], 0, kDrainLimit, status);
     }
@@ -596,59 +595,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph_kg = 0;
     bool ok = true;
     auto kg_mma_wait = [&]() -> bool {
-      const bool r = bwait(&bars[kKgMma], ph_kg, lim, status, s_abort);
+      const bool r = wwait(&bars[kKgMma], ph_kg, lim, status, s_abort);
       ph_kg ^= 1;
       return r;
     };
+    // gate prefix, decay tables and step sizes of chunk n into slot n & 1 (warp 8; the key
+    // group meets on its barrier afterwards)
+    auto gates = [&](int n) {
+      if (warp != 8) return;
+      Gates& gq = sGates[n & 1];
+      float* al = sAlpha + (n & 1) * 64 * (PRISM_MAX_L - 1);
+      const int t0 = tok0 + n * kC;
+      const int nv = min(kC, vend - t0);
+      float gl[2], bl[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        const bool valid = t < nv;
+        const size_t th = ((size_t)b * T + min(t0 + t, T - 1)) * H + h;
+        gl[e] = valid ? __ldg(p.gamma + th) : 1.f;
+        bl[e] = valid ? __ldg(p.beta + th) : 0.f;
+        for (int l = 0; l < m; ++l) al[t * (PRISM_MAX_L - 1) + l] = valid ? __ldg(p.alpha + th * m + l) : 0.f;
+      }
+      const float lg0 = __logf(gl[0]), lg1 = __logf(gl[1]);
+      float x = lg0 + lg1;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+      }
+      const float G63 = __shfl_sync(0xffffffffu, x, 31);
+      const bool fast = G63 >= -60.f;
+      const float Gv[2] = {x - lg1, x};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        gq.G[t] = Gv[e];
+        gq.beta[t] = bl[e];
+        gq.e[t] = __expf(Gv[e]);
+        gq.en[t] = fast ? __expf(-Gv[e]) : 0.f;
+        gq.c[t] = __expf(G63 - Gv[e]);
+        gq.rr[t] = fast ? __expf(Gv[e] - G63) : 0.f;
+      }
+      if (lane == 0) {
+        gq.fast = fast ? 1 : 0;
+        gq.nv = nv;
+      }
+    };
+    if (nchunks > 0) {
+      gates(0);
+      kg_sync();
+      if (kt == 0) mbar_arrive(&bars[kGates0]);
+    }
     for (int n = 0; n < nchunks; ++n) {
       const int g = n & 1;
       Gates& gt = sGates[g];
-      const int t0 = tok0 + n * kC;
-      // ---- gate prefix of chunk n (warp 8)
       bool fail = false;
-      if (n >= 2) fail = !bwait(&bars[kGFree0 + g], ((n - 2) >> 1) & 1, lim, status, s_abort);
-      if (kg_sync_or(fail)) break;
-      if (warp == 8) {
-        const int nv = min(kC, vend - t0);
-        float gl[2], bl[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          const bool valid = t < nv;
-          const size_t th = ((size_t)b * T + min(t0 + t, T - 1)) * H + h;
-          gl[e] = valid ? __ldg(p.gamma + th) : 1.f;
-          bl[e] = valid ? __ldg(p.beta + th) : 0.f;
-        }
-        const float lg0 = __logf(gl[0]), lg1 = __logf(gl[1]);
-        float x = lg0 + lg1;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, x, off);
-          if (lane >= off) x += y;
-        }
-        const float G63 = __shfl_sync(0xffffffffu, x, 31);
-        const bool fast = G63 >= -60.f;
-        const float Gv[2] = {x - lg1, x};
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 2 * lane + e;
-          gt.G[t] = Gv[e];
-          gt.beta[t] = bl[e];
-          gt.e[t] = __expf(Gv[e]);
-          gt.en[t] = fast ? __expf(-Gv[e]) : 0.f;
-          gt.c[t] = __expf(G63 - Gv[e]);
-          gt.rr[t] = fast ? __expf(Gv[e] - G63) : 0.f;
-        }
-        if (lane == 0) {
-          gt.fast = fast ? 1 : 0;
-          gt.nv = nv;
-        }
-      }
-      kg_sync();
-      if (kt == 0) mbar_arrive(&bars[kGates0 + g]);
       const bool fast = gt.fast != 0;
       // ---- key product [K;Q] K^T
-      fail = !bwait(&bars[kKqFull], n & 1, lim, status, s_abort);
+      fail = !wwait(&bars[kKqFull], n & 1, lim, status, s_abort);
+      // the inverse's scratch and ZB are free once MMA-c and MMA1 of the previous chunk are
+      // done; the key product waits for them too, so it does not hold up MMA1 on the tensor pipe
+      if (!fail && n >= 1) fail = !wwait(&bars[kAccFull], (n - 1) & 1, lim, status, s_abort);
       if (kg_sync_or(fail)) break;
       if (kt == 0) {
         tc_fence_after();
@@ -660,8 +668,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars[kKgMma]);
       }
       fail = !kg_mma_wait();
-      // the inverse's scratch and ZB are free once MMA-c and MMA1 of the previous chunk are done
-      if (!fail && n >= 1) fail = !bwait(&bars[kAccFull], (n - 1) & 1, lim, status, s_abort);
       if (kg_sync_or(fail)) break;
       tc_fence_after();
       {  // A (token rows 0..63, fp32 into the inverse's scratch) and Mqk (rows 64..127, bf16 into ZB)
@@ -675,12 +681,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32_raw(tl + kRKQ + 32 * half, raw);
           tmem_wait_ld();
           float x[32];
+          const int tlim = krow ? t : t + 1;  // keep columns i < tlim
+          if (fast) {  // D[t,i] = e^{G_t} e^{-G_i}
+            const float rt = bt * et;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = 32 * half + e;
-            const bool keep = krow ? (i < t) : (i <= t);
-            const float dti = fast ? et * gt.en[i] : __expf(Gt - gt.G[i]);
-            x[e] = keep ? bt * dti * __uint_as_float(raw[e]) : 0.f;
+            for (int e4 = 0; e4 < 32; e4 += 4) {
+              const float4 en = *reinterpret_cast<const float4*>(gt.en + 32 * half + e4);
+              const float f[4] = {en.x, en.y, en.z, en.w};
+#pragma unroll
+              for (int k2 = 0; k2 < 4; ++k2) {
+                const int e = e4 + k2;
+                x[e] = (32 * half + e < tlim) ? rt * f[k2] * __uint_as_float(raw[e]) : 0.f;
+              }
+            }
+          } else {  // strongly decaying chunk: e^{G_t - G_i} per element
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int i = 32 * half + e;
+              x[e] = (i < tlim) ? bt * __expf(Gt - gt.G[i]) * __uint_as_float(raw[e]) : 0.f;
+            }
           }
           if (krow) {
             float4* dst = reinterpret_cast<float4*>(sWS + t * kWsLd + 32 * half);
@@ -736,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       kg_sync();
       if (kt == 0) mbar_arrive(&bars[kZReady]);
       // ---- K^ = diag(beta e) K in place (rows 0..63 of KQ) once the direction loop is done with K
-      if (m > 0) fail = !bwait(&bars[kKqkFree], n & 1, lim, status, s_abort);
+      if (m > 0) fail = !wwait(&bars[kKqkFree], n & 1, lim, status, s_abort);
       if (kg_sync_or(fail)) break;
       for (int e = kt; e < 64 * (D / 8); e += kKG) {
         const int t = e / (D / 8), c8 = (e % (D / 8)) * 8;
@@ -750,53 +769,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       // RW shares columns with RU: free once the direction loop's MMAs are done
-      if (m > 0) fail = !bwait(&bars[kBkupDone], n & 1, lim, status, s_abort);
+      if (m > 0) fail = !wwait(&bars[kBkupDone], n & 1, lim, status, s_abort);
       if (kg_sync_or(fail)) break;
-      // ---- [W'; Mqk W'] = [T; MqkT] K^
+      // ---- [W'; Mqk W'] = [T; MqkT] K^ into RW; the epilogue group turns it into [-W'; Q']
       if (kt == 0) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + kRW, kdesc(aZB, kk, kAtom128), mndesc(aKQ, kk, kAtom128), idesc_bf16(128, D, 0, 1),
                    kk > 0);
-        mma_commit(&bars[kKgMma]);
+        mma_commit(&bars[kRwFull]);
       }
-      fail = !kg_mma_wait();
-      if (kg_sync_or(fail)) break;
-      tc_fence_after();
-      // ---- [-W'; Q'] -> WQ (Q' = e Q - Mqk W')
-      {
-        const bool wrow = row < 64;
-        const int t = wrow ? row : row - 64;
-        const float et = gt.e[t];
-#pragma unroll
-        for (int pc = 0; pc < D / 32; ++pc) {
-          uint32_t raw[32];
-          tmem_ld32_raw(tl + kRW + 32 * pc, raw);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c8 = 0; c8 < 32; c8 += 8) {
-            const int d0 = 32 * pc + c8;
-            float f[8];
-            if (wrow) {
-#pragma unroll
-              for (int k2 = 0; k2 < 8; ++k2) f[k2] = -__uint_as_float(raw[c8 + k2]);
-            } else {
-              float qv[8];
-              unpack8(*reinterpret_cast<const uint4*>(sKQ + sw128_offset(64 + t, d0, kAtom128)), qv);
-#pragma unroll
-              for (int k2 = 0; k2 < 8; ++k2) f[k2] = et * qv[k2] - __uint_as_float(raw[c8 + k2]);
-            }
-            st_bf16x8(sWQ, sw128_offset(row, d0, kAtom128), f);
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      kg_sync();
-      if (kt == 0) {
-        mbar_arrive(&bars[kWqReady]);
-        mbar_arrive(&bars[kKqFree]);
+      // ---- gates of the next chunk, into the slot chunk n - 1 used (free once the epilogue
+      // group has started chunk n)
+      if (n + 1 < nchunks) {
+        if (n >= 1) fail = !wwait(&bars[kGFree0 + (g ^ 1)], ((n - 1) >> 1) & 1, lim, status, s_abort);
+        if (kg_sync_or(fail)) break;
+        gates(n + 1);
+        kg_sync();
+        if (kt == 0) mbar_arrive(&bars[kGates0 + (g ^ 1)]);
       }
       ok = true;
     }
@@ -817,19 +808,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pc8 = (tid % CPT) * 8;    // this thread's 8 prologue channels
     const float* cw_head = p.conv_w + (size_t)h * D * p.W;
     for (int e = tid; e < D * p.W; e += kEG) sTaps[(e % p.W) * D + e / p.W] = __ldg(cw_head + e);
+    for (int e = D * p.W + tid; e < D * 4; e += kEG) sTaps[e] = 0.f;  // taps W..3 are zero
     eg_sync();
     float r[NPASS][8];  // the running residual of the prologue's tokens
+    // r <- r_0 = v - ShortConv anchor of the chunk whose v tile is in VB (its 64 tokens after
+    // 8 rows of history)
+    auto anchor = [&](int ps0, int ps1) {
+#pragma unroll
+      for (int ps = 0; ps < NPASS; ++ps) {
+        if (ps < ps0 || ps >= ps1) continue;
+        const int i = ps * TPP + tid / CPT;
+        const uint8_t* vb = sVB + (pc8 >> 6) * kAtomV;
+        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, v0[8];
+        auto tap = [&](int w, float* vw) {
+          const float4 lo = *reinterpret_cast<const float4*>(sTaps + w * D + pc8);
+          const float4 hi = *reinterpret_cast<const float4*>(sTaps + w * D + pc8 + 4);
+          const float tw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a[e] += tw[e] * vw[e];
+        };
+        if (p.W <= 4) {  // taps W..3 are zero: one unrolled body, every load issued first
+          uint4 raw[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) raw[w] = *reinterpret_cast<const uint4*>(vb + sw128_offset(8 + i - w, pc8 & 63, kAtomV));
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            float vw[8];
+            unpack8(raw[w], vw);
+            if (w == 0) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v0[e] = vw[e];
+            }
+            tap(w, vw);
+          }
+        } else {
+          unpack8(*reinterpret_cast<const uint4*>(vb + sw128_offset(8 + i, pc8 & 63, kAtomV)), v0);
+          tap(0, v0);
+          for (int w = 1; w < p.W; ++w) {
+            float vw[8];
+            unpack8(*reinterpret_cast<const uint4*>(vb + sw128_offset(8 + i - w, pc8 & 63, kAtomV)), vw);
+            tap(w, vw);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[ps][e] = v0[e] - a[e];
+      }
+    };
     bool aborted = false;
     int j = 0;
-    for (int n = 0; n < nchunks; ++n) {
+    // chunk 0's v tile and anchor (later chunks get theirs while the state MMAs of the
+    // chunk before run)
+    if (nchunks > 0 && !p.writes_off) {
+      const bool okv = wwait(&bars[kVFull], 0, lim, status, s_abort);
+      if (!okv) aborted = true;
+      else if (m > 0) anchor(0, NPASS);
+    }
+    for (int n = 0; n < nchunks && !aborted; ++n) {
       const int g = n & 1;
       Gates& gt = sGates[g];
       const int t0 = tok0 + n * kC;
-      bool fail = !bwait(&bars[kGates0 + g], (n >> 1) & 1, lim, status, s_abort);
+      bool fail = !wwait(&bars[kGates0 + g], (n >> 1) & 1, lim, status, s_abort);
       // ---- E1: S_n -> bf16 into SB (A operand of MMA1), RS <- e^{G_63} S_n
-      if (!fail && n >= 1) fail = !bwait(&bars[kRsFull], (n - 1) & 1, lim, status, s_abort);
-      if (eg_sync_or(fail)) { aborted = true; break; }
-      if (n >= 1 && tid == 0) mbar_arrive(&bars[kGFree0 + (g ^ 1)]);  // done with chunk n-1's gates
+      if (!fail && n >= 1) fail = !wwait(&bars[kRsFull], (n - 1) & 1, lim, status, s_abort);
+      if (fail) { aborted = true; break; }
+      if (n >= 1 && lane == 0) mbar_arrive(&bars[kGFree0 + (g ^ 1)]);  // this warp is done with chunk n-1's gates
       tc_fence_after();
       if (srow) {  // this thread: state row c = row, columns [ch*D/2, ch*D/2 + D/2), 32 at a time
         const float e63 = gt.e[63];
@@ -866,8 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       tc_fence_before();
-      eg_sync();
-      if (tid == 0) mbar_arrive(&bars[kE1Done]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kE1Done]);
       const bool fast = gt.fast != 0;
       const int nv = gt.nv;
       // ---- direction loop: prologue (P~_l) and epilogue ([Bku_l; Mqu_l]) of every direction
@@ -876,44 +918,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sP = sm + Ly::PB + s * NA * kAtom64;
         uint8_t* sU = sm + Ly::UB + s * NA * kAtom64;
         uint8_t* sB = sBQ0 + s * kAtom128;
-        fail = !bwait(&bars[kUgFull0 + s], (j >> 1) & 1, lim, status, s_abort);
-        if (!fail && l == 0) fail = !bwait(&bars[kVFull], n & 1, lim, status, s_abort);
-        if (eg_sync_or(fail)) { aborted = true; break; }
-        // prologue: r_0 = v - anchor (l = 0), r_l = chain step, P~_l = (c_i or 1) alpha_{i,l} r_l
+        fail = !wwait(&bars[kUgFull0 + s], (j >> 1) & 1, lim, status, s_abort);
+        if (fail) { aborted = true; break; }
+        // prologue: r_l = chain step of r_{l-1}, P~_l = (c_i or 1) alpha_{i,l} r_l.  Every load
+        // first (the gain rows are then overwritten in place by P~)
+        {
+          uint4 graw[NPASS];
+          float sc[NPASS];
 #pragma unroll
-        for (int ps = 0; ps < NPASS; ++ps) {
-          const int i = ps * TPP + tid / CPT;
-          const bool valid = i < nv;
-          if (l == 0) {
-            float v0[8];
-            unpack8(*reinterpret_cast<const uint4*>(sVB + sw128_offset(8 + i, pc8 & 63, kAtomV) + (pc8 >> 6) * kAtomV), v0);
-            float a[8];
+          for (int ps = 0; ps < NPASS; ++ps) {
+            const int i = ps * TPP + tid / CPT;
+            graw[ps] = *reinterpret_cast<const uint4*>(sP + sw128_offset(i, pc8 & 63, kAtom64) + (pc8 >> 6) * kAtom64);
+            const float al = sAlpha[(g * 64 + i) * (PRISM_MAX_L - 1) + l];  // 0 past the valid tokens
+            sc[ps] = fast ? al * gt.c[i] : al;
+          }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = sTaps[pc8 + e] * v0[e];
-            for (int w = 1; w < p.W; ++w) {
-              float vw[8];
-              unpack8(*reinterpret_cast<const uint4*>(sVB + sw128_offset(8 + i - w, pc8 & 63, kAtomV) + (pc8 >> 6) * kAtomV), vw);
+          for (int ps = 0; ps < NPASS; ++ps) {
+            const int i = ps * TPP + tid / CPT;
+            float gv[8], rho[8];
+            unpack8(graw[ps], gv);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) a[e] += sTaps[w * D + pc8 + e] * vw[e];
+            for (int e = 0; e < 8; ++e) {
+              r[ps][e] = chain_step(r[ps][e], gv[e], CH);
+              rho[e] = sc[ps] * r[ps][e];
             }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) r[ps][e] = v0[e] - a[e];
+            st_bf16x8(sP, sw128_offset(i, pc8 & 63, kAtom64) + (pc8 >> 6) * kAtom64, rho);
           }
-          const uint32_t off = sw128_offset(i, pc8 & 63, kAtom64) + (pc8 >> 6) * kAtom64;
-          float gv[8];
-          unpack8(*reinterpret_cast<const uint4*>(sP + off), gv);
-          const float al = valid ? __ldg(p.alpha + (((size_t)b * T + t0 + i) * H + h) * m + l) : 0.f;
-          const float sc = valid ? (fast ? al * gt.c[i] : al) : 0.f;
-          float rho[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            r[ps][e] = chain_step(r[ps][e], gv[e], CH);
-            rho[e] = sc * r[ps][e];
-          }
-          st_bf16x8(sP, off, rho);
         }
-        fail = !bwait(&bars[kRuFull0 + s], (j >> 1) & 1, lim, status, s_abort);
-        if (eg_sync_or(fail)) { aborted = true; break; }
+        fail = !wwait(&bars[kRuFull0 + s], (j >> 1) & 1, lim, status, s_abort);
+        if (fail) { aborted = true; break; }
         tc_fence_after();
         // epilogue: RU[s] (token rows) -> [Bku_l; Mqu_l] bf16 in BQ[s]
         {
@@ -956,34 +989,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        eg_sync();
-        if (tid == 0) mbar_arrive(&bars[kEpiDone0 + s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kEpiDone0 + s]);
       }
       if (aborted) break;
       // ---- X0^T = beta V - (Bku P)^T -> BQ slot 0 (K-major rows c); ACC's Delta half zeroed
       if (!p.writes_off) {
-      fail = m > 0 ? !bwait(&bars[kBkupDone], n & 1, lim, status, s_abort)
-                   : !bwait(&bars[kVFull], n & 1, lim, status, s_abort);
-      if (eg_sync_or(fail)) { aborted = true; break; }
+      float x[32];  // beta_t v_t[c], read while the last direction's MMAs finish
+      if (srow) {
+        const uint8_t* vcol = sVB + (row >> 6) * kAtomV;
+#pragma unroll
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          const float4 b4 = *reinterpret_cast<const float4*>(gt.beta + 32 * ch + e4);
+          const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
+            const int t = 32 * ch + e4 + k2;
+            const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vcol + sw128_offset(8 + t, row & 63, kAtomV)));
+            x[e4 + k2] = bb[k2] * vv;
+          }
+        }
+      }
+      if (m > 0) fail = !wwait(&bars[kBkupDone], n & 1, lim, status, s_abort);
+      if (fail) { aborted = true; break; }
       tc_fence_after();
       if (srow) {
-        float x[32];
         if (m > 0) {
           uint32_t raw[32];
           tmem_ld32_raw(tl + kACC + 32 * ch, raw);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = -__uint_as_float(raw[e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = 0.f;
-        }
-        const uint8_t* vcol = sVB + (row >> 6) * kAtomV;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int t = 32 * ch + e;
-          const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vcol + sw128_offset(8 + t, row & 63, kAtomV)));
-          x[e] += gt.beta[t] * vv;
+          for (int e = 0; e < 32; ++e) x[e] -= __uint_as_float(raw[e]);
         }
 #pragma unroll
         for (int c8 = 0; c8 < 32; c8 += 8) st_bf16x8(sBQ0, sw128_offset(row, 32 * ch + c8, kAtom128), x + c8);
@@ -997,15 +1033,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      eg_sync();
-      if (tid == 0) {
+      __syncwarp();
+      if (lane == 0) {
         mbar_arrive(&bars[kX0Ready]);
         mbar_arrive(&bars[kVFree]);
       }
       }
+      // ---- [-W'; Q'] -> WQ (Q' = e Q - Mqk W'): token rows, this warp's half of the columns
+      fail = !wwait(&bars[kRwFull], n & 1, lim, status, s_abort);
+      if (fail) { aborted = true; break; }
+      tc_fence_after();
+      {
+        const bool wrow = row < 64;
+        const int t = wrow ? row : row - 64;
+        const float et = gt.e[t];
+#pragma unroll
+        for (int pc = 0; pc < D / 64; ++pc) {
+          const int c0 = ch * (D / 2) + 32 * pc;
+          uint32_t raw[32];
+          tmem_ld32_raw(tl + kRW + c0, raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c8 = 0; c8 < 32; c8 += 8) {
+            const int d0 = c0 + c8;
+            float f[8];
+            if (wrow) {
+#pragma unroll
+              for (int k2 = 0; k2 < 8; ++k2) f[k2] = -__uint_as_float(raw[c8 + k2]);
+            } else {
+              float qv[8];
+              unpack8(*reinterpret_cast<const uint4*>(sKQ + sw128_offset(64 + t, d0, kAtom128)), qv);
+#pragma unroll
+              for (int k2 = 0; k2 < 8; ++k2) f[k2] = et * qv[k2] - __uint_as_float(raw[c8 + k2]);
+            }
+            st_bf16x8(sWQ, sw128_offset(row, d0, kAtom128), f);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars[kWqReady]);
+        mbar_arrive(&bars[kKqFree]);
+      }
+      // the first half of the next chunk's ShortConv anchor, while MMA-c and MMA1 run
+      const bool more = n + 1 < nchunks && !p.writes_off;
+      if (more) {
+        fail = !wwait(&bars[kVFull], (n + 1) & 1, lim, status, s_abort);
+        if (fail) { aborted = true; break; }
+        if (m > 0) anchor(0, NPASS / 2);
+      }
       // ---- E2: Delta~^T -> SB (bf16, TMEM); O^T -> o
-      fail = !bwait(&bars[kAccFull], n & 1, lim, status, s_abort);
-      if (eg_sync_or(fail)) { aborted = true; break; }
+      fail = !wwait(&bars[kAccFull], n & 1, lim, status, s_abort);
+      if (fail) { aborted = true; break; }
       tc_fence_after();
       if (ch == 0) {  // Delta~^T[c, t] = c_t Delta^T[c, t] -> bf16 into SB (A operand of MMA2)
         if (srow) {
@@ -1016,9 +1097,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
             uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int t = 32 * half + 2 * e;
-              pk[e] = pack_bf16x2(gt.c[t] * __uint_as_float(raw[2 * e]), gt.c[t + 1] * __uint_as_float(raw[2 * e + 1]));
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(gt.c + 32 * half + 4 * e4);
+              pk[2 * e4] = pack_bf16x2(c4.x * __uint_as_float(raw[4 * e4]), c4.y * __uint_as_float(raw[4 * e4 + 1]));
+              pk[2 * e4 + 1] = pack_bf16x2(c4.z * __uint_as_float(raw[4 * e4 + 2]), c4.w * __uint_as_float(raw[4 * e4 + 3]));
             }
             tmem_st16_raw(tl + kSB + 16 * half, pk);
           }
@@ -1035,18 +1117,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t raw[32];
           tmem_ld32_raw(tl + kACC + 64 + 32 * half, raw);
           tmem_wait_ld();
+          if (nv == kC) {  // a full chunk: every token valid and inside the tensor
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int t = 32 * half + e;
-            if (t < tmax) op[(size_t)t * H * D] = __float2bfloat16_rn(t < nv ? __uint_as_float(raw[e]) : 0.f);
+            for (int e = 0; e < 32; ++e)
+              op[(size_t)(32 * half + e) * H * D] = __float2bfloat16_rn(__uint_as_float(raw[e]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int t = 32 * half + e;
+              if (t < tmax) op[(size_t)t * H * D] = __float2bfloat16_rn(t < nv ? __uint_as_float(raw[e]) : 0.f);
+            }
           }
         }
       }
+      // the second half of the next chunk's anchor, while MMA2 runs
+      if (more && m > 0) anchor(NPASS / 2, NPASS);
     }
     // ---- the final state, and o past the last chunk
     if (!aborted && nchunks > 0) {
-      const bool okf = bwait(&bars[kRsFull], (nchunks - 1) & 1, lim, status, s_abort);
-      if (!eg_sync_or(!okf)) {
+      const bool okf = wwait(&bars[kRsFull], (nchunks - 1) & 1, lim, status, s_abort);
+      if (okf) {
         tc_fence_after();
         if (srow && S_end) {
 #pragma unroll
