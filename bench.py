@@ -37,6 +37,8 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
     "chunk_scan": "linear_attention_sequence_shortconv_b200/csrc/chunk_scan_kernel.cu",
+    "prism_scan_kernel": "linear_attention_sequence_shortconv_b200/csrc/chunk_scan_kernel.cu",
+    "residual_write_kernel": "linear_attention_sequence_shortconv_b200/csrc/chunk_scan_kernel.cu",
     "recurrent": "linear_attention_sequence_shortconv_b200/csrc/recurrent_kernel.cu",
 }
 
@@ -60,6 +62,22 @@ def algorithmic_work(w, lengths=None):
     flops_th = 10 * C * d + 8 * C * m * d + 6 * d * d + 2 * m * d * d
     return {"tokens": valid_tokens, "token_heads": token_heads,
             "bytes": token_heads * per_th + state, "flops": token_heads * flops_th}
+
+
+def algorithmic_work_split(w, lengths=None):
+    """Bytes each launch of the tensor-core path must move, per token-head (valid
+    tokens): the residual-write launch reads v and gain (I/O dtype) and gamma and
+    alpha (fp32) and writes P~ (bf16, m d_v); the scan reads q, k, v, u (I/O dtype),
+    P~ (bf16) and gamma, beta (fp32), writes o, and reads S0 / writes the final
+    state per sequence-head."""
+    es = 2 if w.dtype == "bf16" else 4
+    m = w.m
+    valid_tokens = int(lengths.sum()) if lengths is not None else w.B * w.T
+    th = valid_tokens * w.H
+    state = w.B * w.H * w.d_v * w.d_k * 4 * (2 if w.with_s0 else 1)
+    prep = th * (es * w.d_v + es * m * w.d_v + 4 * (1 + m) + 2 * m * w.d_v)
+    scan = th * (es * (2 * w.d_k + 2 * w.d_v) + es * m * w.d_k + 2 * m * w.d_v + 8) + state
+    return {"residual_write": prep, "scan": scan}
 
 
 def algorithmic_work_bwd(w, lengths=None):
@@ -391,19 +409,32 @@ def run_ours(args, w):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    # the tensor-core path with residual writes is two launches (more for a cut sequence):
+    # the library records mids[i] between the residual-write launch and the scan
+    use_tc = prism.uses_tensor_cores(w.d_k, w.d_v, w.L, w.W, w.chunk, dtype_code)
+    split = use_tc and w.L > 1
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if split else []
+    for e in mids:
+        e.record(stream)  # creates the event; the call below records it again
     with ClockSampler(local) as clocks:
         for i in range(K):
             flush.zero_()
             starts[i].record(stream)
+            if split:
+                prism.set_split_event(mids[i])
             step()
             ends[i].record(stream)
         torch.cuda.synchronize()
+    prism.set_split_event(None)
     if world > 1:
         dist.barrier()
     if prism.stream_status() != 0:
         raise SystemExit("device status word reports an error in the timed region")
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = max_over_ranks(sum(per_step) / K, dist, dev)
+    if split:
+        prep_ms = max_over_ranks(sum(s.elapsed_time(m) for s, m in zip(starts, mids)) / K, dist, dev)
+        scan_ms = max_over_ranks(sum(m.elapsed_time(e) for m, e in zip(mids, ends)) / K, dist, dev)
     work = algorithmic_work(w, host_inputs["lengths"].numpy() if host_inputs["lengths"] is not None else None)
     value = aggregate_throughput(work["tokens"], world, ms)
 
@@ -448,24 +479,41 @@ def run_ours(args, w):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K2,
                "api": "prism_scan_fwd_host (C ABI, pinned host buffers; two buffer sets on two streams)"}
 
-    # roofline against measured HBM bandwidth.  The duration is the whole step (on the
-    # tensor-core path: the chunk preparation launch and the scan launch), so the
-    # fraction is that of the path, a lower bound for the scan kernel alone.
-    use_tc = prism.uses_tensor_cores(w.d_k, w.d_v, w.L, w.W, w.chunk, dtype_code)
+    # roofline against measured HBM bandwidth.  The dominant kernel is the scan, timed live
+    # by CUDA events on the launching stream (the library records one between its two
+    # launches); "path" is the whole step against the forward's algorithmic bytes
+    # (q, k, v, u, gain, gates read once, o written once), the fraction of the method's
+    # roofline that the step reaches.
     kernel = "chunk_scan" if use_tc else "recurrent"
-    launches_per_step = 1
+    launches_per_step = prism.scan_fwd_launches(w.B, w.T, w.H, w.d_k, w.d_v, w.L, w.W, w.chunk, dtype_code)
     peaks, peak_kind = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    peak_src = f"{peak_kind} (MEASURED_PEAKS hbm_gbs burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s"
+    lens_np = host_inputs["lengths"].numpy() if host_inputs["lengths"] is not None else None
     t_s = ms / 1e3
-    achieved = work["bytes"] / t_s / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(kernel, w.name),
-                "kernel": kernel, "timed": "step = one launch",
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS hbm_gbs burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s",
-                "algorithmic_bytes_per_launch": work["bytes"], "algorithmic_flops_per_launch": work["flops"],
-                "tensor_frac_of_peak": work["flops"] / t_s / 1e12 / peaks["bf16_tflops"],
-                "roofline_time_us": 1e6 * max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
-                                               work["flops"] / (peaks["bf16_tflops"] * 1e12))}
-    roofline["roofline_frac"] = roofline["roofline_time_us"] / (ms * 1e3)
+    path = {"us": ms * 1e3, "algorithmic_bytes": work["bytes"], "achieved_gbs": work["bytes"] / t_s / 1e9,
+            "frac": work["bytes"] / t_s / 1e9 / hbm, "algorithmic_flops": work["flops"],
+            "tensor_frac_of_peak": work["flops"] / t_s / 1e12 / peaks["bf16_tflops"],
+            "roofline_time_us": 1e6 * max(work["bytes"] / (hbm * 1e9), work["flops"] / (peaks["bf16_tflops"] * 1e12))}
+    path["roofline_frac"] = path["roofline_time_us"] / path["us"]
+    if split:
+        sw = algorithmic_work_split(w, lens_np)
+        scan_gbs = sw["scan"] / (scan_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": scan_gbs, "peak": hbm, "unit": "GB/s", "frac": scan_gbs / hbm,
+                    "traffic": recorded_traffic("prism_scan_kernel", w.name), "kernel": "prism_scan_kernel",
+                    "timed": "scan launch(es) of each step, CUDA events on the launching stream",
+                    "kernel_us": scan_ms * 1e3, "algorithmic_bytes_per_launch": sw["scan"], "peak_source": peak_src,
+                    "residual_write": {"kernel": "residual_write_kernel", "us": prep_ms * 1e3,
+                                       "algorithmic_bytes": sw["residual_write"],
+                                       "achieved_gbs": sw["residual_write"] / (prep_ms / 1e3) / 1e9,
+                                       "frac": sw["residual_write"] / (prep_ms / 1e3) / 1e9 / hbm,
+                                       "traffic": recorded_traffic("residual_write_kernel", w.name)},
+                    "path": path}
+    else:
+        roofline = {"bound": "hbm", "achieved": path["achieved_gbs"], "peak": hbm, "unit": "GB/s",
+                    "frac": path["frac"], "traffic": recorded_traffic(kernel, w.name), "kernel": kernel,
+                    "timed": "step = one launch", "kernel_us": ms * 1e3,
+                    "algorithmic_bytes_per_launch": work["bytes"], "peak_source": peak_src, "path": path}
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

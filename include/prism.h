@@ -105,16 +105,18 @@ enum prism_status {
  *
  * chunk: chunk length of the chunkwise-parallel evaluation, a power of two in
  *   [16, 64].  The result does not depend on it beyond rounding.  The bf16
- *   tensor-core path runs chunk == 64 with d_k == d_v in {64, 128} and
- *   L - 1 <= 3; every other supported shape runs the fp32 CUDA-core path, which
- *   evaluates the recurrence token by token.
+ *   tensor-core path runs chunk == 64 with d_k == d_v in {64, 128}; every other
+ *   supported shape runs the fp32 CUDA-core path, which evaluates the recurrence
+ *   token by token.
  * workspace / workspace_bytes: device scratch of at least
  *   prism_scan_fwd_workspace_size(...) bytes (may be NULL when that is 0), 16-byte
  *   aligned, owned by the caller, contents undefined on return.  The tensor-core
- *   path keeps there the inverse T = (I + A)^{-1} of every 64-token chunk as bf16
- *   (B * H * ceil(T / 64) * 8 KB), computed for all chunks at once before the scan;
- *   the token-by-token path needs none.  Too small or NULL: PRISM_ERR_WORKSPACE,
- *   before any launch.
+ *   path writes there, in one launch over all chunks before the scan, the residual
+ *   write vectors alpha_{t,l} r_{t,l} of every token, scaled for the chunk form, as
+ *   bf16 in the layout of gain (B * T * H * (L - 1) * d_v * 2 bytes, rounded up to
+ *   256); a sequence cut into segments (long sequences over few (batch row, head)
+ *   chains) adds three fp32 d_v x d_k states per segment.  The token-by-token path
+ *   needs none.  Too small or NULL: PRISM_ERR_WORKSPACE, before any launch.
  * Errors: PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED, PRISM_ERR_WORKSPACE,
  *   PRISM_ERR_CUDA, as described above.
  */
@@ -209,12 +211,13 @@ int prism_state_affine(const float* S, const float* M, const float* N, float* ou
                        prism_stream_t stream);
 
 /* Size of the device-global scratch behind prism_scan_fwd_static. */
-#define PRISM_STATIC_WORKSPACE_BYTES (32u << 20)
+#define PRISM_STATIC_WORKSPACE_BYTES (192u << 20)
 
 /*
  * prism_scan_fwd_static - prism_scan_fwd_ex without a caller-supplied workspace and
- * without any allocation: the scratch is a file-scope device array of
- * PRISM_STATIC_WORKSPACE_BYTES (32 MiB, 256-byte aligned) inside the library, one per
+ * without any allocation (an entry point of this library; the PRISM write-ups describe
+ * no counterpart): the scratch is a file-scope device array of
+ * PRISM_STATIC_WORKSPACE_BYTES (192 MiB, 256-byte aligned) inside the library, one per
  * device.  The first call on a device looks its address up with cudaGetSymbolAddress
  * (make that first call before any stream capture); later calls reuse it.  The array
  * sits in a module of its own: with lazy module loading (the default of CUDA 12, and
@@ -223,8 +226,9 @@ int prism_state_affine(const float* S, const float* M, const float* N, float* ou
  * library is loaded.  Results are bit-for-bit those of prism_scan_fwd_ex with a
  * workspace.  Sizes whose
  * prism_scan_fwd_workspace_size() exceeds PRISM_STATIC_WORKSPACE_BYTES return
- * PRISM_ERR_WORKSPACE before any launch (the 130M-LM layer, B=16 T=2048 H=6 d=128,
- * needs 24 MiB).  Because the scratch is shared, calls on one device must not overlap
+ * PRISM_ERR_WORKSPACE before any launch (the 130M-LM layer, B=16 T=2048 H=6 d=128
+ * L=4, needs 144 MiB; a 65536-token sequence over 8 heads with L=8 needs more and is
+ * refused).  Because the scratch is shared, calls on one device must not overlap
  * in time: issue them on one stream or order them; calls on one stream may follow each
  * other freely.  Other arguments, conventions and errors as for prism_scan_fwd_ex.
  */
@@ -274,6 +278,12 @@ int prism_prologue_fwd(const void* v, const float* alpha, const void* gain,
  * kernel, 0 if on the CUDA-core token-by-token kernel (sizes as for
  * prism_scan_fwd; unsupported sizes also give 0). */
 int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype);
+
+/* Number of kernel launches one prism_scan_fwd call with these sizes issues on its
+ * stream (0 for invalid sizes).  Tensor-core path: the residual-write launch when
+ * L > 1, then one scan launch, or four (three scans and a fold) when a long sequence
+ * over few (batch row, head) chains is cut into segments.  Token-by-token path: 1. */
+int prism_scan_fwd_launches(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype);
 
 /* prism_prologue_fwd with the residual chain selected by `chain` (see prism_scan_fwd_ex). */
 int prism_prologue_fwd_ex(const void* v, const float* alpha, const void* gain,
@@ -329,6 +339,13 @@ int prism_stream_status(prism_stream_t stream);
  * PRISM_ERR_TIMEOUT instead of waiting, which tests the error path without
  * hanging a GPU.  Host-side setting; applies to launches made after the call. */
 void prism_set_spin_limit(long long limit);
+
+/* Measurement hook: `event` (a cudaEvent_t, or NULL to clear) is recorded on the
+ * stream of the next prism_scan_fwd call that runs the tensor-core path with L > 1,
+ * between its residual-write launch and its scan, and is then forgotten.  Events
+ * recorded by the caller before and after that call then time the two launches
+ * apart.  Process-wide; set it from the thread that makes the call. */
+void prism_set_split_event(void* event);
 
 /* Static description of a status code; never NULL. */
 const char* prism_status_string(int code);

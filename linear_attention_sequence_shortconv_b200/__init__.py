@@ -24,6 +24,8 @@ from ._lib import (  # noqa: F401
     status_string,
     stream_status,
     uses_tensor_cores,
+    scan_fwd_launches,
+    set_split_event,
     version,
     workspace_size,
 )

@@ -43,8 +43,10 @@ EXPORTS = (
     "prism_scan_bwd_workspace_size",
     "prism_state_affine",
     "prism_scan_fwd_uses_tensor_cores",
+    "prism_scan_fwd_launches",
     "prism_stream_status",
     "prism_set_spin_limit",
+    "prism_set_split_event",
     "prism_status_string",
     "prism_version",
 )
@@ -97,10 +99,14 @@ def lib() -> ctypes.CDLL:
     L.prism_state_affine.restype = ci
     L.prism_scan_fwd_uses_tensor_cores.argtypes = [ci] * 6
     L.prism_scan_fwd_uses_tensor_cores.restype = ci
+    L.prism_scan_fwd_launches.argtypes = [ci] * 9
+    L.prism_scan_fwd_launches.restype = ci
     L.prism_stream_status.argtypes = [vp]
     L.prism_stream_status.restype = ci
     L.prism_set_spin_limit.argtypes = [ctypes.c_longlong]
     L.prism_set_spin_limit.restype = None
+    L.prism_set_split_event.argtypes = [vp]
+    L.prism_set_split_event.restype = None
     L.prism_status_string.argtypes = [ci]
     L.prism_status_string.restype = ctypes.c_char_p
     L.prism_version.argtypes = []
@@ -435,6 +441,18 @@ def scan_bwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, dO, L: int, S0=None, 
 def uses_tensor_cores(d_k, d_v, L, W, chunk, dtype_code) -> bool:
     """True if prism_scan_fwd runs these sizes on the tcgen05 chunk kernel."""
     return bool(lib().prism_scan_fwd_uses_tensor_cores(d_k, d_v, L, W, chunk, dtype_code))
+
+
+def scan_fwd_launches(B, T, H, d_k, d_v, L, W, chunk, dtype_code) -> int:
+    """Kernel launches one prism_scan_fwd call with these sizes issues."""
+    return int(lib().prism_scan_fwd_launches(B, T, H, d_k, d_v, L, W, chunk, dtype_code))
+
+
+def set_split_event(event) -> None:
+    """Measurement hook: the next tensor-core forward with L > 1 records ``event`` (a
+    torch.cuda.Event that has been recorded once, so that it exists) between its
+    residual-write launch and its scan.  None clears it."""
+    lib().prism_set_split_event(None if event is None else ctypes.c_void_p(event.cuda_event))
 
 
 def stream_status(stream=None) -> int:

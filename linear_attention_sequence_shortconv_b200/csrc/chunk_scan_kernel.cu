@@ -22,8 +22,11 @@
 //
 // Everything but the last three lines is independent of the state, so the state-dependent
 // chain of a chunk is two MMAs (Q'/W' against S_n, Delta~ against K) and two short
-// tensor-memory epilogues; the rest (the residual chain, the masked Gram products, the
-// inverse, W', Q', U', O_0 and the residual state write) is worked off by other warps.
+// tensor-memory epilogues; the rest (the masked Gram products, the inverse, W', Q', U', O_0
+// and the residual state write) is worked off by other warps.  The residual chain itself
+// (rho, and P~ below) depends on neither the state nor the keys: residual_write_kernel
+// computes it for every chunk of every chain at once, before the scan, and the scan loads
+// P~ by TMA.
 //
 // Tensor-core products (bf16 operands, fp32 accumulators in TMEM, M = 128, one issuing
 // thread each; "x^T" operands come from TMEM or MN-major shared memory):
@@ -36,12 +39,12 @@
 //   c       X0^T x [T;MqkT]^T               -> ACC  ([U'^T | O_0^T])
 //   one     S_n (TMEM) x [-W';Q']^T         -> ACC  ([Delta^T | O^T])
 //   two     Delta~^T (TMEM) x K             -> RS   (S_{n+1})
-// "Fast" chunks (G_63 >= -60) factor the decay as e^{G_t - G_63} c_i: the prologue writes
-// P~ = diag(c) P and U~ = U; other chunks use e^{G_t - G_i} per element, P~ = P and
-// U~ = diag(c) U (scaled in place).
+// "Fast" chunks (G_63 >= -60) factor the decay as e^{G_t - G_63} c_i: the residual-write
+// launch writes P~ = diag(c) P and U~ = U; other chunks use e^{G_t - G_i} per element,
+// P~ = P and U~ = diag(c) U (scaled in place).
 //
-// Warp roles (448 threads): warps 0-7 the epilogue group EG (prologue, Bku/Mqu epilogues,
-// X0, the state epilogues, o), warps 8-11 the key group KG (gate prefix, A and Mqk, the
+// Warp roles (448 threads): warps 0-7 the epilogue group EG (Bku/Mqu epilogues, X0,
+// [-W'; Q'], the state epilogues, o), warps 8-11 the key group KG (gate prefix, A and Mqk, the
 // inverse, Mqk T, K^, W'/Q'; issues its own MMAs), warp 12 the MMA warp (every other MMA),
 // warp 13 the TMA warp.  Hand-overs go through mbarriers; every wait is bounded and gives
 // up once another agent has set the abort flag, so a missed arrival records
@@ -72,6 +75,8 @@ constexpr long long kDrainLimit = 1ll << 18;
 constexpr int kWsLd = 68;  // fp32 row stride of the inverse's scratch (bank padding)
 
 // TMEM columns
+// RU: [K;Q] U_l^T, two slots (directions alternate); RW ([W'; Mqk W']) reuses them once the
+// direction loop is done.
 constexpr uint32_t kRS = 0, kACC = 128, kSB = 256, kRKQ = 320, kRU = 384, kRW = 384;
 
 template <int D>
@@ -88,10 +93,8 @@ struct Lay {
   static constexpr uint32_t WS_BYTES = 64 * kWsLd * 4 + 4096;
   // the inverse's scratch lives in WQ when it fits (WQ is free while the inverse runs)
   static constexpr uint32_t WS = (NA * kAtom128 >= WS_BYTES) ? WQ : WQ + NA * kAtom128;
-  static constexpr uint32_t TAPS = (WS == WQ) ? WQ + NA * kAtom128 : WS + ((WS_BYTES + 1023) / 1024) * 1024;
-  static constexpr uint32_t SMALL = TAPS + D * PRISM_MAX_W * 4;
-  static constexpr uint32_t ALPHA = SMALL + 4096;  // [2][64][PRISM_MAX_L - 1] fp32 step sizes
-  static constexpr uint32_t BYTES = ALPHA + 2 * 64 * (PRISM_MAX_L - 1) * 4;
+  static constexpr uint32_t SMALL = (WS == WQ) ? WQ + NA * kAtom128 : WS + ((WS_BYTES + 1023) / 1024) * 1024;
+  static constexpr uint32_t BYTES = SMALL + 4096;
   static constexpr uint32_t ALLOC = BYTES + 1024;
   static_assert(ALLOC <= 232448, "exceeds the 227 KB opt-in shared memory of sm_100");
 };
@@ -205,16 +208,6 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t base, int kk, uint32_t lbo) 
 }
 
 // ---------------------------------------------------------------- barriers and waits
-__device__ __forceinline__ void eg_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-__device__ __forceinline__ bool eg_sync_or(int v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred q, p;\n\tsetp.ne.s32 q, %1, 0;\n\tbar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(v)
-      : "memory");
-  return r != 0;
-}
 __device__ __forceinline__ void kg_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 __device__ __forceinline__ bool kg_sync_or(int v) {
   uint32_t r;
@@ -363,8 +356,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sZB = sm + Ly::ZB;
   uint8_t* sWQ = sm + Ly::WQ;
   float* sWS = reinterpret_cast<float*>(sm + Ly::WS);
-  float* sTaps = reinterpret_cast<float*>(sm + Ly::TAPS);  // [w][c]
-  float* sAlpha = reinterpret_cast<float*>(sm + Ly::ALPHA);  // [slot][t][l]
   Gates* sGates = reinterpret_cast<Gates*>(sm + Ly::SMALL);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::SMALL + 2 * sizeof(Gates));
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + kNumBars);
@@ -599,12 +590,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ph_kg ^= 1;
       return r;
     };
-    // gate prefix, decay tables and step sizes of chunk n into slot n & 1 (warp 8; the key
+    // gate prefix and decay tables of chunk n into slot n & 1 (warp 8; the key
     // group meets on its barrier afterwards)
     auto gates = [&](int n) {
       if (warp != 8) return;
       Gates& gq = sGates[n & 1];
-      float* al = sAlpha + (n & 1) * 64 * (PRISM_MAX_L - 1);
       const int t0 = tok0 + n * kC;
       const int nv = min(kC, vend - t0);
       float gl[2], bl[2];
@@ -615,18 +605,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t th = ((size_t)b * T + min(t0 + t, T - 1)) * H + h;
         gl[e] = valid ? __ldg(p.gamma + th) : 1.f;
         bl[e] = valid ? __ldg(p.beta + th) : 0.f;
-        for (int l = 0; l < m; ++l) al[t * (PRISM_MAX_L - 1) + l] = valid ? __ldg(p.alpha + th * m + l) : 0.f;
       }
-      const float lg0 = __logf(gl[0]), lg1 = __logf(gl[1]);
-      float x = lg0 + lg1;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += y;
-      }
-      const float G63 = __shfl_sync(0xffffffffu, x, 31);
-      const bool fast = G63 >= -60.f;
-      const float Gv[2] = {x - lg1, x};
+      float Gv[2], G63;
+      chunk_log_decay(gl[0], gl[1], lane, Gv[0], Gv[1], G63);
+      const bool fast = chunk_decay_fast(G63);
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int t = 2 * lane + e;
@@ -682,8 +664,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           float x[32];
           const int tlim = krow ? t : t + 1;  // keep columns i < tlim
-          if (fast) {  // D[t,i] = e^{G_t} e^{-G_i}
+          const int br = q4 & 1;              // this warp's 32-row block against the column half
+          if (fast && br < half) {            // above the diagonal: nothing kept
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = 0.f;
+          } else if (fast) {  // D[t,i] = e^{G_t} e^{-G_i}
             const float rt = bt * et;
+            const int lim_e = br > half ? 32 : tlim - 32 * half;
 #pragma unroll
             for (int e4 = 0; e4 < 32; e4 += 4) {
               const float4 en = *reinterpret_cast<const float4*>(gt.en + 32 * half + e4);
@@ -691,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int k2 = 0; k2 < 4; ++k2) {
                 const int e = e4 + k2;
-                x[e] = (32 * half + e < tlim) ? rt * f[k2] * __uint_as_float(raw[e]) : 0.f;
+                x[e] = e < lim_e ? rt * f[k2] * __uint_as_float(raw[e]) : 0.f;
               }
             }
           } else {  // strongly decaying chunk: e^{G_t - G_i} per element
@@ -802,66 +789,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = 32 * q4 + lane;  // TMEM lane: state row c, or token row
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
     const bool srow = row < D;
-    constexpr int CPT = D / 8;          // prologue threads per token
-    constexpr int TPP = kEG / CPT;      // tokens per prologue pass
-    constexpr int NPASS = kC / TPP;
-    const int pc8 = (tid % CPT) * 8;    // this thread's 8 prologue channels
-    const float* cw_head = p.conv_w + (size_t)h * D * p.W;
-    for (int e = tid; e < D * p.W; e += kEG) sTaps[(e % p.W) * D + e / p.W] = __ldg(cw_head + e);
-    for (int e = D * p.W + tid; e < D * 4; e += kEG) sTaps[e] = 0.f;  // taps W..3 are zero
-    eg_sync();
-    float r[NPASS][8];  // the running residual of the prologue's tokens
-    // r <- r_0 = v - ShortConv anchor of the chunk whose v tile is in VB (its 64 tokens after
-    // 8 rows of history)
-    auto anchor = [&](int ps0, int ps1) {
-#pragma unroll
-      for (int ps = 0; ps < NPASS; ++ps) {
-        if (ps < ps0 || ps >= ps1) continue;
-        const int i = ps * TPP + tid / CPT;
-        const uint8_t* vb = sVB + (pc8 >> 6) * kAtomV;
-        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, v0[8];
-        auto tap = [&](int w, float* vw) {
-          const float4 lo = *reinterpret_cast<const float4*>(sTaps + w * D + pc8);
-          const float4 hi = *reinterpret_cast<const float4*>(sTaps + w * D + pc8 + 4);
-          const float tw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a[e] += tw[e] * vw[e];
-        };
-        if (p.W <= 4) {  // taps W..3 are zero: one unrolled body, every load issued first
-          uint4 raw[4];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) raw[w] = *reinterpret_cast<const uint4*>(vb + sw128_offset(8 + i - w, pc8 & 63, kAtomV));
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            float vw[8];
-            unpack8(raw[w], vw);
-            if (w == 0) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) v0[e] = vw[e];
-            }
-            tap(w, vw);
-          }
-        } else {
-          unpack8(*reinterpret_cast<const uint4*>(vb + sw128_offset(8 + i, pc8 & 63, kAtomV)), v0);
-          tap(0, v0);
-          for (int w = 1; w < p.W; ++w) {
-            float vw[8];
-            unpack8(*reinterpret_cast<const uint4*>(vb + sw128_offset(8 + i - w, pc8 & 63, kAtomV)), vw);
-            tap(w, vw);
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) r[ps][e] = v0[e] - a[e];
-      }
-    };
     bool aborted = false;
     int j = 0;
-    // chunk 0's v tile and anchor (later chunks get theirs while the state MMAs of the
-    // chunk before run)
+    // chunk 0's v tile (later chunks' arrive while the state MMAs of the chunk before run)
     if (nchunks > 0 && !p.writes_off) {
-      const bool okv = wwait(&bars[kVFull], 0, lim, status, s_abort);
-      if (!okv) aborted = true;
-      else if (m > 0) anchor(0, NPASS);
+      if (!wwait(&bars[kVFull], 0, lim, status, s_abort)) aborted = true;
     }
     for (int n = 0; n < nchunks && !aborted; ++n) {
       const int g = n & 1;
@@ -898,11 +830,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
           }
           uint32_t pk[16];
+          const float2 e2 = make_float2(e63, e63);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(__uint_as_float(raw[2 * c]), __uint_as_float(raw[2 * c + 1]));
+          for (int c = 0; c < 16; ++c) {
+            const float2 sv = make_float2(__uint_as_float(raw[2 * c]), __uint_as_float(raw[2 * c + 1]));
+            pk[c] = pack_bf16x2(sv.x, sv.y);
+            const float2 sc = __fmul2_rn(e2, sv);
+            raw[2 * c] = __float_as_uint(sc.x);
+            raw[2 * c + 1] = __float_as_uint(sc.y);
+          }
           tmem_st16_raw(tl + kSB + c0 / 2, pk);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(e63 * __uint_as_float(raw[c]));
           tmem_st32_raw(tl + kRS + c0, raw);
         }
         tmem_wait_st();
@@ -912,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars[kE1Done]);
       const bool fast = gt.fast != 0;
       const int nv = gt.nv;
-      // ---- direction loop: prologue (P~_l) and epilogue ([Bku_l; Mqu_l]) of every direction
+      // ---- direction loop: the epilogue ([Bku_l; Mqu_l]) of every direction
       for (int l = 0; l < m; ++l, ++j) {
         const int s = j & 1;
         uint8_t* sP = sm + Ly::PB + s * NA * kAtom64;
@@ -920,31 +857,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sB = sBQ0 + s * kAtom128;
         fail = !wwait(&bars[kUgFull0 + s], (j >> 1) & 1, lim, status, s_abort);
         if (fail) { aborted = true; break; }
-        // prologue: r_l = chain step of r_{l-1}, P~_l = (c_i or 1) alpha_{i,l} r_l.  Every load
-        // first (the gain rows are then overwritten in place by P~)
-        {
-          uint4 graw[NPASS];
-          float sc[NPASS];
-#pragma unroll
-          for (int ps = 0; ps < NPASS; ++ps) {
-            const int i = ps * TPP + tid / CPT;
-            graw[ps] = *reinterpret_cast<const uint4*>(sP + sw128_offset(i, pc8 & 63, kAtom64) + (pc8 >> 6) * kAtom64);
-            const float al = sAlpha[(g * 64 + i) * (PRISM_MAX_L - 1) + l];  // 0 past the valid tokens
-            sc[ps] = fast ? al * gt.c[i] : al;
-          }
-#pragma unroll
-          for (int ps = 0; ps < NPASS; ++ps) {
-            const int i = ps * TPP + tid / CPT;
-            float gv[8], rho[8];
-            unpack8(graw[ps], gv);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              r[ps][e] = chain_step(r[ps][e], gv[e], CH);
-              rho[e] = sc[ps] * r[ps][e];
-            }
-            st_bf16x8(sP, sw128_offset(i, pc8 & 63, kAtom64) + (pc8 >> 6) * kAtom64, rho);
-          }
-        }
         fail = !wwait(&bars[kRuFull0 + s], (j >> 1) & 1, lim, status, s_abort);
         if (fail) { aborted = true; break; }
         tc_fence_after();
@@ -957,14 +869,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32_raw(tl + kRU + 64 * s + 32 * ch, raw);
           tmem_wait_ld();
           float x[32];
-          if (fast) {
-            const float f = bt * gt.rr[t];
+          // the masks are causal: against this warp's 32-token block of rows, the 32-column
+          // piece [32 ch, 32 ch + 32) is entirely kept, entirely zero or the diagonal block
+          const int br = q4 & 1;
+          if (fast && br != ch) {
+            const float f = br > ch ? bt * gt.rr[t] : 0.f;
+            const float2 f2 = make_float2(f, f);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int i = 32 * ch + e;
-              x[e] = (krow ? i < t : i <= t) ? f * __uint_as_float(raw[e]) : 0.f;
+            for (int e = 0; e < 32; e += 2) {
+              const float2 y = __fmul2_rn(f2, make_float2(__uint_as_float(raw[e]), __uint_as_float(raw[e + 1])));
+              x[e] = y.x;
+              x[e + 1] = y.y;
             }
-          } else {
+          } else if (fast) {
+            const float f = bt * gt.rr[t];
+            const int lim_e = krow ? lane : lane + 1;  // keep columns e < lim_e of the piece
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = e < lim_e ? f * __uint_as_float(raw[e]) : 0.f;
+          } else {  // strongly decaying chunk
             const float Gt = gt.G[t];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -1019,7 +941,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32_raw(tl + kACC + 32 * ch, raw);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] -= __uint_as_float(raw[e]);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 y = __fadd2_rn(make_float2(x[e], x[e + 1]),
+                                        make_float2(-__uint_as_float(raw[e]), -__uint_as_float(raw[e + 1])));
+            x[e] = y.x;
+            x[e + 1] = y.y;
+          }
         }
 #pragma unroll
         for (int c8 = 0; c8 < 32; c8 += 8) st_bf16x8(sBQ0, sw128_offset(row, 32 * ch + c8, kAtom128), x + c8);
@@ -1077,12 +1004,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars[kWqReady]);
         mbar_arrive(&bars[kKqFree]);
       }
-      // the first half of the next chunk's ShortConv anchor, while MMA-c and MMA1 run
-      const bool more = n + 1 < nchunks && !p.writes_off;
-      if (more) {
+      // the next chunk's v tile, loaded while MMA-c and MMA1 run
+      if (n + 1 < nchunks && !p.writes_off) {
         fail = !wwait(&bars[kVFull], (n + 1) & 1, lim, status, s_abort);
         if (fail) { aborted = true; break; }
-        if (m > 0) anchor(0, NPASS / 2);
       }
       // ---- E2: Delta~^T -> SB (bf16, TMEM); O^T -> o
       fail = !wwait(&bars[kAccFull], n & 1, lim, status, s_abort);
@@ -1099,8 +1024,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
               const float4 c4 = *reinterpret_cast<const float4*>(gt.c + 32 * half + 4 * e4);
-              pk[2 * e4] = pack_bf16x2(c4.x * __uint_as_float(raw[4 * e4]), c4.y * __uint_as_float(raw[4 * e4 + 1]));
-              pk[2 * e4 + 1] = pack_bf16x2(c4.z * __uint_as_float(raw[4 * e4 + 2]), c4.w * __uint_as_float(raw[4 * e4 + 3]));
+              const float2 d0 = __fmul2_rn(make_float2(c4.x, c4.y),
+                                           make_float2(__uint_as_float(raw[4 * e4]), __uint_as_float(raw[4 * e4 + 1])));
+              const float2 d1 = __fmul2_rn(make_float2(c4.z, c4.w),
+                                           make_float2(__uint_as_float(raw[4 * e4 + 2]), __uint_as_float(raw[4 * e4 + 3])));
+              pk[2 * e4] = pack_bf16x2(d0.x, d0.y);
+              pk[2 * e4 + 1] = pack_bf16x2(d1.x, d1.y);
             }
             tmem_st16_raw(tl + kSB + 16 * half, pk);
           }
@@ -1121,7 +1050,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e)
               op[(size_t)(32 * half + e) * H * D] = __float2bfloat16_rn(__uint_as_float(raw[e]));
-          } else {
+          } else {  // the last chunk of a sequence
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int t = 32 * half + e;
@@ -1130,8 +1059,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // the second half of the next chunk's anchor, while MMA2 runs
-      if (more && m > 0) anchor(NPASS / 2, NPASS);
     }
     // ---- the final state, and o past the last chunk
     if (!aborted && nchunks > 0) {
@@ -1174,6 +1101,140 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- residual write vectors
+// rho_{t,l} = alpha_{t,l} r_{t,l} of every token, written as P~ (bf16, the layout of gain:
+// [B, T, H, L - 1, D]) for the scan to load by TMA.  r_{t,0} = v_t - ShortConv anchor,
+// r_{t,l} = chain step of r_{t,l-1} with gain g_{t,l}.  In a chunk whose decay is factored
+// (chunk_decay_fast), P~ = e^{G_63 - G_t} rho; else P~ = rho.  Nothing here depends on the
+// state, so every chunk of every chain runs at once, in CTAs of kPrepThreads threads over
+// prep_tokens(D) tokens of one chunk.  A thread owns 8 channels of 4 consecutive tokens: it
+// loads each v row of their ShortConv window once and the gain rows of up to kPrepLevels
+// levels at the same time, so that enough 16-byte loads are in flight to keep HBM busy.
+// Chunks wholly past a row's length are skipped (the scan never reads them); padded tokens
+// of a chunk get zeros.
+constexpr int kPrepThreads = 128;
+constexpr int kPrepTPT = 4;     // consecutive tokens per thread
+constexpr int kPrepLevels = 3;  // residual levels whose gain rows are loaded together
+__host__ __device__ constexpr int prep_tokens(int D) { return kPrepThreads * kPrepTPT / (D / 8); }
+
+__device__ __forceinline__ uint4 ldg16(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+template <int D, int CH, int WM>  // WM >= W: taps held in registers
+__global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
+    residual_write_kernel(const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ gain,
+                          const float* __restrict__ alpha, const float* __restrict__ gamma,
+                          const float* __restrict__ conv_w, const int32_t* __restrict__ lengths,
+                          __nv_bfloat16* __restrict__ ptil, int T, int H, int W, int m, int NC) {
+  constexpr int CPT = D / 8;              // threads per token row
+  constexpr int TPT = kPrepTPT;
+  constexpr int PB = kC / prep_tokens(D);  // CTAs per chunk
+  constexpr int NV = TPT + WM - 1;        // v rows of the threads' ShortConv window
+  constexpr int LB = kPrepLevels;
+  static_assert(PB >= 1 && kC % prep_tokens(D) == 0, "CTA tiling of a chunk");
+  __shared__ float s_c[kC];  // e^{G_63 - G_t} (1 when the chunk's decay is not factored)
+  const int part = blockIdx.x % PB, cidx = blockIdx.x / PB;
+  const int n = cidx % NC, bh = cidx / NC, b = bh / H, h = bh % H;
+  const int len = lengths ? min(max(lengths[b], 0), T) : T;
+  const int t0 = n * kC;
+  if (t0 >= len) return;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int c8 = (tid % CPT) * 8, i0 = part * prep_tokens(D) + (tid / CPT) * TPT;
+  const size_t row0 = ((size_t)b * T + t0 + i0) * H + h;  // (token, head) row of the first token
+  // every load first: the v window, then the gain rows and alphas of the first LB levels
+  uint4 vr[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int t = t0 + i0 - (WM - 1) + j;
+    vr[j] = (t >= 0 && t < T) ? ldg16(v + (((size_t)b * T + t) * H + h) * D + c8) : make_uint4(0, 0, 0, 0);
+  }
+  uint4 gr[LB][TPT];
+  float al[LB][TPT];
+  auto load_levels = [&](int l0) {
+#pragma unroll
+    for (int j = 0; j < LB; ++j)
+#pragma unroll
+      for (int a = 0; a < TPT; ++a) {
+        const bool ok = l0 + j < m && t0 + i0 + a < len;
+        const size_t th = row0 + (size_t)a * H;
+        gr[j][a] = ok ? ldg16(gain + (th * m + l0 + j) * D + c8) : make_uint4(0, 0, 0, 0);
+        al[j][a] = ok ? __ldg(alpha + th * m + l0 + j) : 0.f;
+      }
+  };
+  load_levels(0);
+  if (tid < 32) {
+    const int nv = min(kC, len - t0);
+    float gl[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int t = 2 * lane + e;
+      gl[e] = t < nv ? __ldg(gamma + ((size_t)b * T + t0 + t) * H + h) : 1.f;
+    }
+    float G0, G1, G63;
+    chunk_log_decay(gl[0], gl[1], lane, G0, G1, G63);
+    const bool fast = chunk_decay_fast(G63);
+    s_c[2 * lane] = fast ? __expf(G63 - G0) : 1.f;
+    s_c[2 * lane + 1] = fast ? __expf(G63 - G1) : 1.f;
+  }
+  float r[TPT][8];
+  {
+    float taps[WM][8];
+#pragma unroll
+    for (int w = 0; w < WM; ++w)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) taps[w][e] = w < W ? __ldg(conv_w + ((size_t)h * D + c8 + e) * W + w) : 0.f;
+#pragma unroll
+    for (int a = 0; a < TPT; ++a) {
+      float vt[8];
+      unpack8(vr[a + WM - 1], vt);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r[a][e] = vt[e] - taps[0][e] * vt[e];
+#pragma unroll
+      for (int w = 1; w < WM; ++w) {
+        if (w < W) {
+          float vw[8];
+          unpack8(vr[a + WM - 1 - w], vw);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) r[a][e] -= taps[w][e] * vw[e];
+        }
+      }
+    }
+  }
+  __syncthreads();  // s_c
+  float cs[TPT];
+#pragma unroll
+  for (int a = 0; a < TPT; ++a) cs[a] = s_c[i0 + a];
+  for (int l0 = 0; l0 < m; l0 += LB) {
+    if (l0 > 0) load_levels(l0);
+#pragma unroll
+    for (int j = 0; j < LB; ++j) {
+      if (l0 + j < m) {
+#pragma unroll
+        for (int a = 0; a < TPT; ++a) {
+          const int t = t0 + i0 + a;
+          if (t < T) {
+            float gv[8], rho[8];
+            unpack8(gr[j][a], gv);
+            const float sc = cs[a] * al[j][a];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              r[a][e] = chain_step(r[a][e], gv[e], CH);
+              rho[e] = sc * r[a][e];
+            }
+            uint4 u = make_uint4(0, 0, 0, 0);
+            if (t < len) {
+              u.x = pack_bf16x2(rho[0], rho[1]);
+              u.y = pack_bf16x2(rho[2], rho[3]);
+              u.z = pack_bf16x2(rho[4], rho[5]);
+              u.w = pack_bf16x2(rho[6], rho[7]);
+            }
+            *reinterpret_cast<uint4*>(ptil + ((row0 + (size_t)a * H) * m + l0 + j) * D + c8) = u;
+          }
+        }
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------- segment fold
@@ -1247,6 +1308,12 @@ SegPlan plan_segments(int B, int T, int H) {
   return {(nc + cps - 1) / cps, cps * kC};
 }
 
+// The workspace: P~ (bf16, the shape of gain), 256-byte aligned, then the segments' states.
+size_t ptil_bytes(int B, int T, int H, int D, int L) {
+  const size_t b = (size_t)B * T * H * (L - 1) * D * 2;
+  return (b + 255) & ~size_t(255);
+}
+
 template <int D, int CH>
 cudaError_t set_smem_attr() {
   static std::once_flag attr_once;
@@ -1274,12 +1341,27 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
   if (!encode(&mq, p.q, 4, dims4, str4, box4) || !encode(&mk, p.k, 4, dims4, str4, box4) ||
       !encode(&mv, p.v, 4, dims4, str4, box_v))
     return cudaErrorInvalidValue;
+  __nv_bfloat16* ptil = static_cast<__nv_bfloat16*>(p.workspace);  // P~, the layout of gain
   if (m > 0) {
     const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)m, H, T, B};
     const cuuint64_t str5[4] = {(cuuint64_t)D * 2, (cuuint64_t)m * D * 2, H * m * D * 2, T * H * m * D * 2};
     const cuuint32_t box5[5] = {64, 1, 1, 64, 1};
-    if (!encode(&mu, p.u, 5, dims5, str5, box5) || !encode(&mg, p.gain, 5, dims5, str5, box5))
+    if (!encode(&mu, p.u, 5, dims5, str5, box5) || !encode(&mg, ptil, 5, dims5, str5, box5))
       return cudaErrorInvalidValue;
+    const int NC = (p.T + kC - 1) / kC;
+    const dim3 grid(p.B * p.H * NC * (kC / prep_tokens(D)));
+    const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(p.v);
+    const __nv_bfloat16* gg = static_cast<const __nv_bfloat16*>(p.gain);
+    if (p.W <= 4)
+      residual_write_kernel<D, CH, 4><<<grid, kPrepThreads, 0, stream>>>(vv, gg, p.alpha, p.gamma, p.conv_w,
+                                                                          p.lengths, ptil, p.T, p.H, p.W, m, NC);
+    else
+      residual_write_kernel<D, CH, PRISM_MAX_W><<<grid, kPrepThreads, 0, stream>>>(
+          vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths, ptil, p.T, p.H, p.W, m, NC);
+    if (p.split_event) {
+      const cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(p.split_event), stream);
+      if (e != cudaSuccess) return e;
+    }
   } else {
     mu = mk;
     mg = mk;
@@ -1296,7 +1378,7 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
   }
   // a long sequence over few chains: P segments side by side, three scans and a fold
   const size_t seg_states = (size_t)p.B * p.H * plan.P * D * D;
-  float* wsN = static_cast<float*>(p.workspace);
+  float* wsN = reinterpret_cast<float*>(static_cast<char*>(p.workspace) + ptil_bytes(p.B, p.T, p.H, D, p.L));
   float* wsM = wsN + seg_states;
   float* wsS = wsM + seg_states;
   ScanArgs aN = a;  // each segment from a zero start (the first from S0): N_p
@@ -1330,9 +1412,13 @@ bool chunk_scan_supported(int d_k, int d_v, int L, int W, int chunk, int dtype) 
          L <= PRISM_MAX_L && W >= 1 && W <= PRISM_MAX_W;
 }
 
-size_t chunk_scan_workspace_bytes(int B, int T, int H, int D) {
+size_t chunk_scan_workspace_bytes(int B, int T, int H, int D, int L) {
   const SegPlan plan = plan_segments(B, T, H);
-  return plan.P == 1 ? 0 : 3 * (size_t)B * H * plan.P * D * D * sizeof(float);
+  return ptil_bytes(B, T, H, D, L) + (plan.P == 1 ? 0 : 3 * (size_t)B * H * plan.P * D * D * sizeof(float));
+}
+
+int chunk_scan_launches(int B, int T, int H, int L) {
+  return (L > 1 ? 1 : 0) + (plan_segments(B, T, H).P == 1 ? 1 : 4);
 }
 
 cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream) {

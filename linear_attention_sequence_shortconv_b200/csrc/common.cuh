@@ -36,6 +36,7 @@ struct ScanParams {
                           // slot 0 the initial state, slot n the state after token 64 n - 1,
                           // slot ceil(len / 64) the state after the last valid token
   float* rec_psi;         // v_t - gamma_t S_{t-1} k_t per valid token, [B, T, H, d_v] fp32
+  void* split_event;      // tensor-core path: cudaEvent_t recorded after the residual-write launch (or NULL)
 };
 
 // Tokens per chunk of the chunked backward.
@@ -170,6 +171,27 @@ template <>
 __device__ __forceinline__ void st1<__nv_bfloat16>(__nv_bfloat16* p, float x) {
   *p = __float2bfloat16_rn(x);
 }
+
+// In-chunk cumulative log decay of a 64-token chunk, one warp: lane owns tokens 2 lane and
+// 2 lane + 1 with gates g0, g1 (1 for padded steps); returns G of those tokens and G_63.  The
+// chunk scan and the residual-write launch both call this, so that their per-chunk decisions
+// (such as whether e^{-G} stays finite) agree bit for bit.
+__device__ __forceinline__ void chunk_log_decay(float g0, float g1, int lane, float& G0, float& G1, float& G63) {
+  const float lg0 = __logf(g0), lg1 = __logf(g1);
+  float x = lg0 + lg1;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  G63 = __shfl_sync(0xffffffffu, x, 31);
+  G0 = x - lg1;
+  G1 = x;
+}
+
+// A chunk takes the factored decay e^{G_t - G_i} = e^{G_t} e^{-G_i} (and the residual write
+// vectors scaled by e^{G_63 - G_i}) when its total log decay keeps e^{-G} finite.
+__device__ __forceinline__ bool chunk_decay_fast(float G63) { return G63 >= -60.f; }
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, PRISM_OK, code);

@@ -12,7 +12,8 @@ cudaError_t launch_prologue(const void* v, const float* alpha, const void* gain,
                             int dtype, float* rho, cudaStream_t stream, int chain);
 bool chunk_scan_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
 cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream);
-size_t chunk_scan_workspace_bytes(int B, int T, int H, int D);
+size_t chunk_scan_workspace_bytes(int B, int T, int H, int D, int L);
+int chunk_scan_launches(int B, int T, int H, int L);
 cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, cudaStream_t stream);
 size_t bwd_smem_bytes(int d_k, int d_v, int L);
@@ -36,6 +37,7 @@ int* g_status_ptr[kMaxDevices] = {};
 int g_arch_ok[kMaxDevices] = {};  // 0 unknown, 1 sm_100, -1 other
 constexpr long long kDefaultSpinLimit = 1ll << 18;  // polls; each may suspend up to 20 us
 std::atomic<long long> g_spin_limit{kDefaultSpinLimit};
+std::atomic<void*> g_split_event{nullptr};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool ranges_overlap(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
@@ -108,6 +110,8 @@ const char* prism_status_string(int code) {
   }
 }
 
+void prism_set_split_event(void* event) { g_split_event.store(event); }
+
 void prism_set_spin_limit(long long limit) {
   g_spin_limit.store(limit > 0 ? limit : kDefaultSpinLimit);
 }
@@ -115,10 +119,10 @@ void prism_set_spin_limit(long long limit) {
 size_t prism_scan_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
                                      int dtype) {
   if (check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype) != PRISM_OK) return 0;
-  // the tensor-core scan cuts long sequences over few chains into segments: three fp32
-  // states per segment (its maps from zero and from the identity, and its start state)
+  // the tensor-core scan keeps the residual write vectors (bf16, the shape of gain) and, when
+  // it cuts a long sequence over few chains into segments, three fp32 states per segment
   if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype))
-    return prism::chunk_scan_workspace_bytes(B, T, H, d_k);
+    return prism::chunk_scan_workspace_bytes(B, T, H, d_k, L);
   return 0;
 }
 
@@ -157,9 +161,10 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* 
                       need > 0 ? workspace : nullptr};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t err;
-  if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype))
+  if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype)) {
+    if (L > 1) p.split_event = g_split_event.exchange(nullptr);
     err = prism::launch_chunk_scan(p, s);
-  else
+  } else
     err = prism::launch_recurrent_scan(p, dtype, s);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
@@ -234,6 +239,12 @@ int prism_prologue_fwd_ex(const void* v, const float* alpha, const void* gain, c
   cudaError_t err = prism::launch_prologue(v, alpha, gain, conv_w, lengths, B, T, H, d_v, L, W, dtype,
                                            rho_out, reinterpret_cast<cudaStream_t>(stream), chain);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+int prism_scan_fwd_launches(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype) {
+  if (check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype) != PRISM_OK) return 0;
+  if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype)) return prism::chunk_scan_launches(B, T, H, L);
+  return 1;
 }
 
 int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype) {

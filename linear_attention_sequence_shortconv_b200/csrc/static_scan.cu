@@ -1,4 +1,5 @@
-// prism_scan_fwd_static: the scan for callers that cannot allocate device memory.
+// prism_scan_fwd_static: the scan for callers that cannot allocate device memory.  The
+// PRISM write-ups have no counterpart of this entry point; it is a service of this library.
 //
 // Its scratch is a file-scope device array in this translation unit, which the CUDA
 // runtime registers as a module of its own.  With lazy module loading (the default of

@@ -90,27 +90,53 @@ def _segments(B, T, H):
     return -(-nc // cps)
 
 
+def _ptil(B, T, H, D, L):
+    """Bytes of the residual write vectors the tensor-core scan stages in the workspace:
+    bf16, one d_v row per (token, head, direction), rounded up to 256."""
+    n = B * T * H * (L - 1) * D * 2
+    return -(-n // 256) * 256
+
+
 def test_workspace_size_query(L):
-    # the single-launch scan keeps everything on chip; only a cut sequence needs three fp32
-    # states per segment (its two maps and its start state)
-    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) == 0     # the 130M-LM layer
-    assert prism.workspace_size(128, 1024, 2, 64, 64, 4, 4, 64, 0) == 0     # recsys
+    # the tensor-core scan stages the residual write vectors of every token (bf16, the
+    # layout of gain); a cut sequence adds three fp32 states per segment (its two maps and
+    # its start state)
+    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) == _ptil(16, 2048, 6, 128, 4)  # 130M-LM layer
+    assert _ptil(16, 2048, 6, 128, 4) == 144 << 20
+    assert prism.workspace_size(128, 1024, 2, 64, 64, 4, 4, 64, 0) == _ptil(128, 1024, 2, 64, 4)   # recsys
+    assert prism.workspace_size(16, 2048, 6, 128, 128, 1, 4, 64, 0) == 0   # L = 1: no residual writes
     P = _segments(1, 65536, 8)
     assert P == 18
-    assert prism.workspace_size(1, 65536, 8, 128, 128, 8, 4, 64, 0) == 3 * 8 * P * 128 * 128 * 4
-    assert prism.workspace_size(2, 4096, 1, 64, 64, 2, 4, 64, 0) == 3 * 2 * _segments(2, 4096, 1) * 64 * 64 * 4
+    assert prism.workspace_size(1, 65536, 8, 128, 128, 8, 4, 64, 0) == \
+        _ptil(1, 65536, 8, 128, 8) + 3 * 8 * P * 128 * 128 * 4
+    assert prism.workspace_size(2, 4096, 1, 64, 64, 2, 4, 64, 0) == \
+        _ptil(2, 4096, 1, 64, 2) + 3 * 2 * _segments(2, 4096, 1) * 64 * 64 * 4
+    assert prism.workspace_size(1, 3, 1, 64, 64, 2, 4, 64, 0) == 512   # 384 bytes, rounded up to 256
     assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 1) == 0   # fp32: token-by-token kernel
     assert prism.workspace_size(0, 64, 8, 128, 128, 4, 4, 64, 0) == 0       # invalid sizes
 
 
-def test_workspace_never_exceeds_the_static_scratch(L):
-    # chains x segments never exceeds 148, so no shape needs more than 3 x 148 x 128^2 fp32
+def test_launch_count_query(L):
+    # residual-write launch + one scan; a cut sequence: three scans and a fold instead
+    assert prism.scan_fwd_launches(16, 2048, 6, 128, 128, 4, 4, 64, 0) == 2
+    assert prism.scan_fwd_launches(16, 2048, 6, 128, 128, 1, 4, 64, 0) == 1
+    assert prism.scan_fwd_launches(1, 65536, 8, 128, 128, 8, 4, 64, 0) == 5
+    assert prism.scan_fwd_launches(1, 65536, 8, 128, 128, 1, 4, 64, 0) == 4
+    assert prism.scan_fwd_launches(16, 2048, 6, 128, 128, 4, 4, 64, 1) == 1   # token-by-token
+    assert prism.scan_fwd_launches(16, 2048, 6, 128, 128, 4, 4, 32, 0) == 1
+    assert prism.scan_fwd_launches(0, 2048, 6, 128, 128, 4, 4, 64, 0) == 0
+
+
+def test_segment_states_stay_within_148_chains(L):
+    # chains x segments never exceeds 148, so the segment states never need more than
+    # 3 x 148 x 128^2 fp32 beyond the residual write vectors
     worst = 0
     for B in (1, 2, 3, 5, 8, 37, 74):
         for H in (1, 2, 4, 8):
             for T in (64, 2047, 2048, 65536, 1 << 20):
-                worst = max(worst, prism.workspace_size(B, T, H, 128, 128, 8, 4, 64, 0))
-    assert 0 < worst <= 3 * 148 * 128 * 128 * 4 <= 32 << 20
+                extra = prism.workspace_size(B, T, H, 128, 128, 8, 4, 64, 0) - _ptil(B, T, H, 128, 8)
+                worst = max(worst, extra)
+    assert 0 < worst <= 3 * 148 * 128 * 128 * 4
 
 
 def test_missing_workspace_is_rejected_before_launch(L):
