@@ -115,7 +115,8 @@ enum prism_status {
  *   write vectors alpha_{t,l} r_{t,l} of every token, scaled for the chunk form, as
  *   bf16 in the layout of gain (B * T * H * (L - 1) * d_v * 2 bytes, rounded up to
  *   256); a sequence cut into segments (long sequences over few (batch row, head)
- *   chains) adds three fp32 d_v x d_k states per segment.  The token-by-token path
+ *   chains) adds three fp32 d_v x d_k states per segment, and a scan run in two halves
+ *   (chains that leave SMs idle) adds two fp32 d_v x d_k states per chain.  The token-by-token path
  *   needs none.  Too small or NULL: PRISM_ERR_WORKSPACE, before any launch.
  * Errors: PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED, PRISM_ERR_WORKSPACE,
  *   PRISM_ERR_CUDA, as described above.
@@ -279,10 +280,14 @@ int prism_prologue_fwd(const void* v, const float* alpha, const void* gain,
  * prism_scan_fwd; unsupported sizes also give 0). */
 int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype);
 
-/* Number of kernel launches one prism_scan_fwd call with these sizes issues on its
- * stream (0 for invalid sizes).  Tensor-core path: the residual-write launch when
- * L > 1, then one scan launch, or four (three scans and a fold) when a long sequence
- * over few (batch row, head) chains is cut into segments.  Token-by-token path: 1. */
+/* Number of kernel launches one prism_scan_fwd call with these sizes issues (0 for
+ * invalid sizes).  Tensor-core path: the residual-write launch when L > 1, then one
+ * scan launch, or four (three scans and a fold) when a long sequence over few
+ * (batch row, head) chains is cut into segments; when the chains leave at least 24 of
+ * a B200's SMs idle, L > 1 and the sequence has at least 8 chunks, four: the scan runs
+ * in two halves, and the second half's residual write runs beside the first half's
+ * scan (on two internal streams of the device, forked from and joined back into the
+ * call's stream).  Token-by-token path: 1. */
 int prism_scan_fwd_launches(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype);
 
 /* prism_prologue_fwd with the residual chain selected by `chain` (see prism_scan_fwd_ex). */
@@ -342,9 +347,8 @@ void prism_set_spin_limit(long long limit);
 
 /* Measurement hook: `event` (a cudaEvent_t, or NULL to clear) is recorded on the
  * stream of the next prism_scan_fwd call that runs the tensor-core path with L > 1,
- * between its residual-write launch and its scan, and is then forgotten.  Events
- * recorded by the caller before and after that call then time the two launches
- * apart.  Process-wide; set it from the thread that makes the call. */
+ * after its (first) residual-write launch, and is then forgotten.  Events recorded by
+ * the caller before and after that call then time that launch and the rest apart.  Process-wide; set it from the thread that makes the call. */
 void prism_set_split_event(void* event);
 
 /* Static description of a status code; never NULL. */

@@ -122,6 +122,7 @@ struct ScanArgs {
   int B, T, H, W, m;   // m: residual directions of this launch (0 when writes are off)
   int P, Ts;
   int s_in_identity, write_o, writes_off;
+  int seg_only;        // >= 0: this launch runs only that segment of every chain (one CTA per chain)
   int* status;
   long long spin_limit;
 };
@@ -363,7 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(2 * sizeof(Gates) + 8 * kNumBars + 8 <= 4096, "small region");
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x / p.P, seg = blockIdx.x % p.P, b = bh / p.H, h = bh % p.H;
+  const int bh = p.seg_only >= 0 ? (int)blockIdx.x : (int)blockIdx.x / p.P;
+  const int seg = p.seg_only >= 0 ? p.seg_only : (int)blockIdx.x % p.P, b = bh / p.H, h = bh % p.H;
   const int T = p.T, H = p.H, m = p.m;
   const int len = p.lengths ? min(max(p.lengths[b], 0), T) : T;
   const int tok0 = seg * p.Ts;                         // first token of this CTA's segment
@@ -1113,7 +1115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // loads each v row of their ShortConv window once and the gain rows of up to kPrepLevels
 // levels at the same time, so that enough 16-byte loads are in flight to keep HBM busy.
 // Chunks wholly past a row's length are skipped (the scan never reads them); padded tokens
-// of a chunk get zeros.
+// of a chunk get zeros.  A launch covers chunks [nc0, nc0 + ncn) of every chain.
 constexpr int kPrepThreads = 128;
 constexpr int kPrepTPT = 4;     // consecutive tokens per thread
 constexpr int kPrepLevels = 3;  // residual levels whose gain rows are loaded together
@@ -1126,7 +1128,7 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
     residual_write_kernel(const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ gain,
                           const float* __restrict__ alpha, const float* __restrict__ gamma,
                           const float* __restrict__ conv_w, const int32_t* __restrict__ lengths,
-                          __nv_bfloat16* __restrict__ ptil, int T, int H, int W, int m, int NC) {
+                          __nv_bfloat16* __restrict__ ptil, int T, int H, int W, int m, int nc0, int ncn) {
   constexpr int CPT = D / 8;              // threads per token row
   constexpr int TPT = kPrepTPT;
   constexpr int PB = kC / prep_tokens(D);  // CTAs per chunk
@@ -1135,7 +1137,7 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
   static_assert(PB >= 1 && kC % prep_tokens(D) == 0, "CTA tiling of a chunk");
   __shared__ float s_c[kC];  // e^{G_63 - G_t} (1 when the chunk's decay is not factored)
   const int part = blockIdx.x % PB, cidx = blockIdx.x / PB;
-  const int n = cidx % NC, bh = cidx / NC, b = bh / H, h = bh % H;
+  const int n = nc0 + cidx % ncn, bh = cidx / ncn, b = bh / H, h = bh % H;
   const int len = lengths ? min(max(lengths[b], 0), T) : T;
   const int t0 = n * kC;
   if (t0 >= len) return;
@@ -1308,7 +1310,56 @@ SegPlan plan_segments(int B, int T, int H) {
   return {(nc + cps - 1) / cps, cps * kC};
 }
 
-// The workspace: P~ (bf16, the shape of gain), 256-byte aligned, then the segments' states.
+// Two halves in time.  When the chains of a sequence leave SMs idle during the scan (and
+// the sequence is not cut into segments), the scan runs in two launches: chunks
+// [0, nA), then chunks [nA, NC) from the first launch's end states.  The residual write
+// of the second half runs beside the first scan launch, on the SMs that launch leaves
+// idle, so only the first half's residual write precedes the scan.
+constexpr int kSplitIdleSMs = 24;  // SMs the chains must leave idle
+struct TimeSplit {
+  bool on;
+  int nA;  // chunks of the first half
+};
+TimeSplit time_split(int B, int T, int H, int L) {
+  const int nc = (T + kC - 1) / kC;
+  const bool on = L > 1 && plan_segments(B, T, H).P == 1 && B * H + kSplitIdleSMs <= kPlanSMs && nc >= 8;
+  return {on, (nc + 1) / 2};
+}
+
+// Side streams of a device for the two halves: the first scan launch on a stream of the
+// greatest priority (so that its CTAs take SMs before the second half's residual write),
+// that residual write on a stream of the least priority; fork and join through events on
+// the caller's stream.  Created on first use; a mutex keeps the record / wait sequences of
+// concurrent callers from interleaving.
+struct SideStreams {
+  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaEvent_t forked = nullptr, scan_a = nullptr, res_b = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+std::mutex g_side_mutex;
+SideStreams g_side[kMaxSideDevices];
+
+cudaError_t side_streams(SideStreams** out) {  // with g_side_mutex held
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
+  SideStreams& x = g_side[dev];
+  if (!x.hi) {
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&x.lo, cudaStreamNonBlocking, least)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&x.forked, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&x.scan_a, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&x.res_b, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&x.hi, cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
+  }
+  *out = &x;
+  return cudaSuccess;
+}
+
+// The workspace: P~ (bf16, the shape of gain), 256-byte aligned, then the segments' states
+// or the two halves' hand-over states.
 size_t ptil_bytes(int B, int T, int H, int D, int L) {
   const size_t b = (size_t)B * T * H * (L - 1) * D * 2;
   return (b + 255) & ~size_t(255);
@@ -1342,22 +1393,26 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
       !encode(&mv, p.v, 4, dims4, str4, box_v))
     return cudaErrorInvalidValue;
   __nv_bfloat16* ptil = static_cast<__nv_bfloat16*>(p.workspace);  // P~, the layout of gain
+  const int NC = (p.T + kC - 1) / kC;
+  const TimeSplit split = time_split(p.B, p.T, p.H, p.L);
+  const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(p.v);
+  const __nv_bfloat16* gg = static_cast<const __nv_bfloat16*>(p.gain);
+  auto residual = [&](int nc0, int ncn, cudaStream_t st) {
+    const dim3 grid(p.B * p.H * ncn * (kC / prep_tokens(D)));
+    if (p.W <= 4)
+      residual_write_kernel<D, CH, 4><<<grid, kPrepThreads, 0, st>>>(vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths,
+                                                                      ptil, p.T, p.H, p.W, m, nc0, ncn);
+    else
+      residual_write_kernel<D, CH, PRISM_MAX_W><<<grid, kPrepThreads, 0, st>>>(
+          vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths, ptil, p.T, p.H, p.W, m, nc0, ncn);
+  };
   if (m > 0) {
     const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)m, H, T, B};
     const cuuint64_t str5[4] = {(cuuint64_t)D * 2, (cuuint64_t)m * D * 2, H * m * D * 2, T * H * m * D * 2};
     const cuuint32_t box5[5] = {64, 1, 1, 64, 1};
     if (!encode(&mu, p.u, 5, dims5, str5, box5) || !encode(&mg, ptil, 5, dims5, str5, box5))
       return cudaErrorInvalidValue;
-    const int NC = (p.T + kC - 1) / kC;
-    const dim3 grid(p.B * p.H * NC * (kC / prep_tokens(D)));
-    const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(p.v);
-    const __nv_bfloat16* gg = static_cast<const __nv_bfloat16*>(p.gain);
-    if (p.W <= 4)
-      residual_write_kernel<D, CH, 4><<<grid, kPrepThreads, 0, stream>>>(vv, gg, p.alpha, p.gamma, p.conv_w,
-                                                                          p.lengths, ptil, p.T, p.H, p.W, m, NC);
-    else
-      residual_write_kernel<D, CH, PRISM_MAX_W><<<grid, kPrepThreads, 0, stream>>>(
-          vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths, ptil, p.T, p.H, p.W, m, NC);
+    residual(0, split.on ? split.nA : NC, stream);
     if (p.split_event) {
       const cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(p.split_event), stream);
       if (e != cudaSuccess) return e;
@@ -1370,8 +1425,41 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
   ScanArgs a{static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
              static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha, p.conv_w, p.S0, p.lengths,
              static_cast<__nv_bfloat16*>(p.o), p.S_final, nullptr, nullptr, p.B, p.T, p.H, p.W, m,
-             plan.P, plan.Ts, 0, 1, 0, p.status, p.spin_limit};
+             plan.P, plan.Ts, 0, 1, 0, -1, p.status, p.spin_limit};
   const int grid = p.B * p.H * plan.P;
+  if (split.on) {
+    // the two halves as segments 0 and 1 of a 2-segment plan, one launch each; the first
+    // writes its end states to hand[b, h, 1], where the second reads its start states
+    float* hand = reinterpret_cast<float*>(static_cast<char*>(p.workspace) + ptil_bytes(p.B, p.T, p.H, D, p.L));
+    ScanArgs aA = a;
+    aA.P = 2;
+    aA.Ts = split.nA * kC;
+    aA.seg_only = 0;
+    aA.S_out = hand + (size_t)D * D;
+    ScanArgs aB = aA;
+    aB.seg_only = 1;
+    aB.S_out = nullptr;
+    aB.S_in = hand;
+    {
+      std::lock_guard<std::mutex> lock(g_side_mutex);
+      SideStreams* ss = nullptr;
+      cudaError_t e = side_streams(&ss);
+      if (e == cudaSuccess) e = cudaEventRecord(ss->forked, stream);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->hi, ss->forked, 0);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->lo, ss->forked, 0);
+      if (e != cudaSuccess) return e;
+      prism_scan_kernel<D, CH><<<p.B * p.H, kThreads, Ly::ALLOC, ss->hi>>>(mq, mk, mu, mv, mg, aA);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      residual(split.nA, NC - split.nA, ss->lo);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      if ((e = cudaEventRecord(ss->scan_a, ss->hi)) != cudaSuccess) return e;
+      if ((e = cudaEventRecord(ss->res_b, ss->lo)) != cudaSuccess) return e;
+      if ((e = cudaStreamWaitEvent(stream, ss->scan_a, 0)) != cudaSuccess) return e;
+      if ((e = cudaStreamWaitEvent(stream, ss->res_b, 0)) != cudaSuccess) return e;
+    }
+    prism_scan_kernel<D, CH><<<p.B * p.H, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aB);
+    return cudaGetLastError();
+  }
   if (plan.P == 1) {
     prism_scan_kernel<D, CH><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, a);
     return cudaGetLastError();
@@ -1414,10 +1502,13 @@ bool chunk_scan_supported(int d_k, int d_v, int L, int W, int chunk, int dtype) 
 
 size_t chunk_scan_workspace_bytes(int B, int T, int H, int D, int L) {
   const SegPlan plan = plan_segments(B, T, H);
-  return ptil_bytes(B, T, H, D, L) + (plan.P == 1 ? 0 : 3 * (size_t)B * H * plan.P * D * D * sizeof(float));
+  const size_t states = plan.P > 1 ? 3 * (size_t)B * H * plan.P * D * D
+                                   : (time_split(B, T, H, L).on ? 2 * (size_t)B * H * D * D : 0);
+  return ptil_bytes(B, T, H, D, L) + states * sizeof(float);
 }
 
 int chunk_scan_launches(int B, int T, int H, int L) {
+  if (time_split(B, T, H, L).on) return 4;  // two residual-write launches, two scan launches
   return (L > 1 ? 1 : 0) + (plan_segments(B, T, H).P == 1 ? 1 : 4);
 }
 

@@ -100,11 +100,13 @@ def _ptil(B, T, H, D, L):
 def test_workspace_size_query(L):
     # the tensor-core scan stages the residual write vectors of every token (bf16, the
     # layout of gain); a cut sequence adds three fp32 states per segment (its two maps and
-    # its start state)
-    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) == _ptil(16, 2048, 6, 128, 4)  # 130M-LM layer
+    # its start state); a scan run in two halves adds two fp32 states per chain
+    lm = _ptil(16, 2048, 6, 128, 4) + 2 * 16 * 6 * 128 * 128 * 4
+    assert prism.workspace_size(16, 2048, 6, 128, 128, 4, 4, 64, 0) == lm    # 130M-LM layer: two halves
     assert _ptil(16, 2048, 6, 128, 4) == 144 << 20
-    assert prism.workspace_size(128, 1024, 2, 64, 64, 4, 4, 64, 0) == _ptil(128, 1024, 2, 64, 4)   # recsys
+    assert prism.workspace_size(128, 1024, 2, 64, 64, 4, 4, 64, 0) == _ptil(128, 1024, 2, 64, 4)  # recsys: 256 chains
     assert prism.workspace_size(16, 2048, 6, 128, 128, 1, 4, 64, 0) == 0   # L = 1: no residual writes
+    assert prism.workspace_size(16, 448, 6, 128, 128, 4, 4, 64, 0) == _ptil(16, 448, 6, 128, 4)  # 7 chunks: one launch
     P = _segments(1, 65536, 8)
     assert P == 18
     assert prism.workspace_size(1, 65536, 8, 128, 128, 8, 4, 64, 0) == \
@@ -117,8 +119,11 @@ def test_workspace_size_query(L):
 
 
 def test_launch_count_query(L):
-    # residual-write launch + one scan; a cut sequence: three scans and a fold instead
-    assert prism.scan_fwd_launches(16, 2048, 6, 128, 128, 4, 4, 64, 0) == 2
+    # residual-write launch + one scan; a cut sequence: three scans and a fold instead;
+    # chains that leave SMs idle: two halves (two residual writes, two scans)
+    assert prism.scan_fwd_launches(16, 2048, 6, 128, 128, 4, 4, 64, 0) == 4
+    assert prism.scan_fwd_launches(128, 1024, 2, 64, 64, 4, 4, 64, 0) == 2
+    assert prism.scan_fwd_launches(16, 448, 6, 128, 128, 4, 4, 64, 0) == 2
     assert prism.scan_fwd_launches(16, 2048, 6, 128, 128, 1, 4, 64, 0) == 1
     assert prism.scan_fwd_launches(1, 65536, 8, 128, 128, 8, 4, 64, 0) == 5
     assert prism.scan_fwd_launches(1, 65536, 8, 128, 128, 1, 4, 64, 0) == 4
@@ -128,8 +133,8 @@ def test_launch_count_query(L):
 
 
 def test_segment_states_stay_within_148_chains(L):
-    # chains x segments never exceeds 148, so the segment states never need more than
-    # 3 x 148 x 128^2 fp32 beyond the residual write vectors
+    # chains x segments never exceeds 148, so the segment (or hand-over) states never need
+    # more than 3 x 148 x 128^2 fp32 beyond the residual write vectors
     worst = 0
     for B in (1, 2, 3, 5, 8, 37, 74):
         for H in (1, 2, 4, 8):
