@@ -131,10 +131,18 @@ int prism_scan_fwd(const void* q, const void* k, const void* v,
 
 /*
  * prism_scan_fwd_ex - prism_scan_fwd with the residual chain selected by `chain`
- * (PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU; any other value is PRISM_ERR_INVALID_ARG).
+ * (PRISM_CHAIN_LINEAR or PRISM_CHAIN_GELU; any other value is PRISM_ERR_INVALID_ARG),
+ * and the ShortConv history of the sequences in `conv_state`.
  * For PRISM_CHAIN_GELU the `gain` tensor holds the predictor output p of the exact
  * refinement step r <- r - GELU(p * r) (gist.science PRISM explainer, 2.2), any real value.
- * prism_scan_fwd is prism_scan_fwd_ex with PRISM_CHAIN_LINEAR.
+ * conv_state [B,H,W-1,d_v] dtype (device, 16-byte aligned; NULL: zeros): v_{-W+1}, ...,
+ *   v_{-1}, oldest first, the values of v before token 0 that the ShortConv anchors of
+ *   the first W - 1 tokens read (ICML 2026 PRISM write-up, 消除 Token 间串行: the anchor
+ *   reads the last few tokens).  A sequence scanned in two calls, the second with
+ *   S0 = the first's S_final and conv_state = the first's last W - 1 rows of v, gives
+ *   the result of one call over the whole sequence (the layout of prism_decode_step's
+ *   conv_state).  Ignored when W == 1.
+ * prism_scan_fwd is prism_scan_fwd_ex with PRISM_CHAIN_LINEAR and no history.
  */
 int prism_scan_fwd_ex(const void* q, const void* k, const void* v,
                       const float* gamma, const float* beta,
@@ -142,7 +150,8 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v,
                       const float* conv_w, const float* S0, const int32_t* lengths,
                       int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
                       int dtype, void* o, float* S_final,
-                      void* workspace, size_t workspace_bytes, prism_stream_t stream, int chain);
+                      void* workspace, size_t workspace_bytes, prism_stream_t stream, int chain,
+                      const void* conv_state);
 
 /* Bytes of device workspace prism_scan_fwd needs for these sizes (0 if none).
  * Returns 0 for invalid sizes as well; prism_scan_fwd reports those. */
@@ -238,7 +247,8 @@ int prism_scan_fwd_static(const void* q, const void* k, const void* v,
                           const void* u, const float* alpha, const void* gain,
                           const float* conv_w, const float* S0, const int32_t* lengths,
                           int B, int T, int H, int d_k, int d_v, int L, int W, int chunk,
-                          int dtype, void* o, float* S_final, prism_stream_t stream, int chain);
+                          int dtype, void* o, float* S_final, prism_stream_t stream, int chain,
+                          const void* conv_state);
 
 /*
  * prism_scan_fwd_host - the same operation on HOST buffers: copies every input

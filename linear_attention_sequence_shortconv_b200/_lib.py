@@ -76,14 +76,14 @@ def lib() -> ctypes.CDLL:
     L.prism_scan_fwd.argtypes = [vp, vp, vp, fp, fp, vp, fp, vp, fp, fp, i32p,
                                  ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, fp, vp, cs, vp]
     L.prism_scan_fwd.restype = ci
-    L.prism_scan_fwd_ex.argtypes = L.prism_scan_fwd.argtypes + [ci]
+    L.prism_scan_fwd_ex.argtypes = L.prism_scan_fwd.argtypes + [ci, vp]
     L.prism_scan_fwd_ex.restype = ci
     L.prism_scan_fwd_workspace_size.argtypes = [ci] * 9
     L.prism_scan_fwd_workspace_size.restype = cs
     L.prism_scan_fwd_host.argtypes = ([vp] * 11 + [vp] * 11 + [ci] * 9 + [vp, vp, vp, vp, vp, cs, vp])
     L.prism_scan_fwd_host.restype = ci
     L.prism_scan_fwd_static.argtypes = [vp, vp, vp, fp, fp, vp, fp, vp, fp, fp, i32p,
-                                        ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, fp, vp, ci]
+                                        ci, ci, ci, ci, ci, ci, ci, ci, ci, vp, fp, vp, ci, vp]
     L.prism_scan_fwd_static.restype = ci
     L.prism_prologue_fwd.argtypes = [vp, fp, vp, fp, i32p, ci, ci, ci, ci, ci, ci, ci, fp, vp]
     L.prism_prologue_fwd.restype = ci
@@ -186,7 +186,7 @@ def workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype_code) -> int:
 
 
 def _scan_checks(q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o, S_final, want_state,
-                 stream):
+                 stream, conv_state=None):
     """Argument checks shared by scan_fwd and scan_fwd_static; returns the sizes, the
     device and the (allocated when missing) outputs."""
     dev = _call_device(q, stream)
@@ -210,6 +210,8 @@ def _scan_checks(q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o
         _check(alpha, "alpha", torch.float32, shape=(B, T, H, m), device=dev)
     _check(S0, "S0", torch.float32, required=False, shape=(B, H, d_v, d_k), device=dev)
     _check(lengths, "lengths", torch.int32, required=False, shape=(B,), device=dev)
+    if W > 1:
+        _check(conv_state, "conv_state", dt, required=False, shape=(B, H, W - 1, d_v), device=dev)
     if o is None:
         o = torch.empty((B, T, H, d_v), dtype=dt, device=dev)
     else:
@@ -224,7 +226,7 @@ def _scan_checks(q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o
 
 def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 64,
              S0=None, lengths=None, want_state: bool = True, o=None, S_final=None,
-             workspace=None, stream=None, chain: str = "linear"):
+             workspace=None, stream=None, chain: str = "linear", conv_state=None):
     """PRISM mixer forward on CUDA tensors; returns (o, S_final or None).
 
     ``chain`` picks the residual chain step: "linear" r <- (1 - g) r, or "gelu"
@@ -232,12 +234,14 @@ def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 
 
     Shapes as in include/prism.h: q, k [B,T,H,d_k]; v [B,T,H,d_v]; gamma, beta
     [B,T,H] fp32; u [B,T,H,L-1,d_k]; alpha [B,T,H,L-1] fp32; gain [B,T,H,L-1,d_v];
-    conv_w [H,d_v,W] fp32; S0 [B,H,d_v,d_k] fp32 or None; lengths [B] int32 or None.
+    conv_w [H,d_v,W] fp32; S0 [B,H,d_v,d_k] fp32 or None; lengths [B] int32 or None;
+    conv_state [B,H,W-1,d_v] (the I/O dtype) or None: the values of v before token 0,
+    oldest first, that the first ShortConv anchors read (None: zeros).
     Every tensor must be on one CUDA device; the call runs on that device.
     """
     chain_code = _chain_code(chain)
     (B, T, H, d_k, d_v, W, code), dev, o, S_final = _scan_checks(
-        q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o, S_final, want_state, stream)
+        q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o, S_final, want_state, stream, conv_state)
     with torch.cuda.device(dev):
         ws_bytes = workspace_size(B, T, H, d_k, d_v, L, W, chunk, code)
         if ws_bytes and workspace is None:
@@ -251,7 +255,7 @@ def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 
             B, T, H, d_k, d_v, L, W, chunk, code,
             _ptr(o), _ptr(S_final if want_state else None),
             _ptr(workspace), workspace.numel() if workspace is not None else 0, _stream_handle(stream),
-            chain_code)
+            chain_code, _ptr(conv_state if W > 1 else None))
     if rc != 0:
         raise PrismError(rc, "prism_scan_fwd_ex")
     return o, (S_final if want_state else None)
@@ -259,19 +263,20 @@ def scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 
 
 def scan_fwd_static(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, chunk: int = 64,
                     S0=None, lengths=None, want_state: bool = True, o=None, S_final=None,
-                    stream=None, chain: str = "linear"):
+                    stream=None, chain: str = "linear", conv_state=None):
     """scan_fwd through prism_scan_fwd_static: no workspace argument, and the library
     allocates nothing (its scratch is a device-global array); returns (o, S_final)."""
     chain_code = _chain_code(chain)
     (B, T, H, d_k, d_v, W, code), dev, o, S_final = _scan_checks(
-        q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o, S_final, want_state, stream)
+        q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, o, S_final, want_state, stream, conv_state)
     with torch.cuda.device(dev):
         rc = lib().prism_scan_fwd_static(
             _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(beta),
             _ptr(u if L > 1 else None), _ptr(alpha if L > 1 else None), _ptr(gain if L > 1 else None),
             _ptr(conv_w), _ptr(S0), _ptr(lengths),
             B, T, H, d_k, d_v, L, W, chunk, code,
-            _ptr(o), _ptr(S_final if want_state else None), _stream_handle(stream), chain_code)
+            _ptr(o), _ptr(S_final if want_state else None), _stream_handle(stream), chain_code,
+            _ptr(conv_state if W > 1 else None))
     if rc != 0:
         raise PrismError(rc, "prism_scan_fwd_static")
     return o, (S_final if want_state else None)

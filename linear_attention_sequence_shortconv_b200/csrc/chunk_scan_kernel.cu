@@ -1128,7 +1128,8 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
     residual_write_kernel(const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ gain,
                           const float* __restrict__ alpha, const float* __restrict__ gamma,
                           const float* __restrict__ conv_w, const int32_t* __restrict__ lengths,
-                          __nv_bfloat16* __restrict__ ptil, int T, int H, int W, int m, int nc0, int ncn) {
+                          const __nv_bfloat16* __restrict__ conv_state, __nv_bfloat16* __restrict__ ptil, int T,
+                          int H, int W, int m, int nc0, int ncn) {
   constexpr int CPT = D / 8;              // threads per token row
   constexpr int TPT = kPrepTPT;
   constexpr int PB = kC / prep_tokens(D);  // CTAs per chunk
@@ -1149,7 +1150,12 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int t = t0 + i0 - (WM - 1) + j;
-    vr[j] = (t >= 0 && t < T) ? ldg16(v + (((size_t)b * T + t) * H + h) * D + c8) : make_uint4(0, 0, 0, 0);
+    if (t >= 0)
+      vr[j] = t < T ? ldg16(v + (((size_t)b * T + t) * H + h) * D + c8) : make_uint4(0, 0, 0, 0);
+    else  // before token 0: the sequence's ShortConv history (rows W - 1 + t), else zero
+      vr[j] = (conv_state && t >= 1 - W)
+                  ? ldg16(conv_state + (((size_t)b * H + h) * (W - 1) + (W - 1 + t)) * D + c8)
+                  : make_uint4(0, 0, 0, 0);
   }
   uint4 gr[LB][TPT];
   float al[LB][TPT];
@@ -1397,14 +1403,15 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
   const TimeSplit split = time_split(p.B, p.T, p.H, p.L);
   const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(p.v);
   const __nv_bfloat16* gg = static_cast<const __nv_bfloat16*>(p.gain);
+  const __nv_bfloat16* cs = static_cast<const __nv_bfloat16*>(p.conv_state);
   auto residual = [&](int nc0, int ncn, cudaStream_t st) {
     const dim3 grid(p.B * p.H * ncn * (kC / prep_tokens(D)));
     if (p.W <= 4)
       residual_write_kernel<D, CH, 4><<<grid, kPrepThreads, 0, st>>>(vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths,
-                                                                      ptil, p.T, p.H, p.W, m, nc0, ncn);
+                                                                      cs, ptil, p.T, p.H, p.W, m, nc0, ncn);
     else
       residual_write_kernel<D, CH, PRISM_MAX_W><<<grid, kPrepThreads, 0, st>>>(
-          vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths, ptil, p.T, p.H, p.W, m, nc0, ncn);
+          vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths, cs, ptil, p.T, p.H, p.W, m, nc0, ncn);
   };
   if (m > 0) {
     const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)m, H, T, B};

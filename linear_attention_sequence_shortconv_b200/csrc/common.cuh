@@ -37,6 +37,7 @@ struct ScanParams {
                           // slot ceil(len / 64) the state after the last valid token
   float* rec_psi;         // v_t - gamma_t S_{t-1} k_t per valid token, [B, T, H, d_v] fp32
   void* split_event;      // tensor-core path: cudaEvent_t recorded after the residual-write launch (or NULL)
+  const void* conv_state; // [B, H, W - 1, d_v]: v before token 0, oldest first (NULL: zeros)
 };
 
 // Tokens per chunk of the chunked backward.

@@ -132,21 +132,23 @@ int prism_scan_fwd(const void* q, const void* k, const void* v, const float* gam
                    int L, int W, int chunk, int dtype, void* o, float* S_final, void* workspace,
                    size_t workspace_bytes, prism_stream_t stream) {
   return prism_scan_fwd_ex(q, k, v, gamma, beta, u, alpha, gain, conv_w, S0, lengths, B, T, H, d_k, d_v, L, W,
-                           chunk, dtype, o, S_final, workspace, workspace_bytes, stream, PRISM_CHAIN_LINEAR);
+                           chunk, dtype, o, S_final, workspace, workspace_bytes, stream, PRISM_CHAIN_LINEAR,
+                           nullptr);
 }
 
 int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* gamma, const float* beta,
                       const void* u, const float* alpha, const void* gain, const float* conv_w,
                       const float* S0, const int32_t* lengths, int B, int T, int H, int d_k, int d_v,
                       int L, int W, int chunk, int dtype, void* o, float* S_final, void* workspace,
-                      size_t workspace_bytes, prism_stream_t stream, int chain) {
+                      size_t workspace_bytes, prism_stream_t stream, int chain, const void* conv_state) {
   if (chain != PRISM_CHAIN_LINEAR && chain != PRISM_CHAIN_GELU) return PRISM_ERR_INVALID_ARG;
   int rc = check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype);
   if (rc != PRISM_OK) return rc;
   if (!q || !k || !v || !gamma || !beta || !conv_w || !o) return PRISM_ERR_INVALID_ARG;
   if (L > 1 && (!u || !alpha || !gain)) return PRISM_ERR_INVALID_ARG;
+  if (W == 1) conv_state = nullptr;  // no history to read
   const void* ptrs[] = {q, k, v, gamma, beta, conv_w, o, S0, lengths, S_final, workspace,
-                        L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr};
+                        L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr, conv_state};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return PRISM_ERR_UNSUPPORTED;
   const size_t need = prism_scan_fwd_workspace_size(B, T, H, d_k, d_v, L, W, chunk, dtype);
@@ -159,6 +161,7 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* 
                       L > 1 ? gain : nullptr, conv_w, S0, lengths, o, S_final,
                       B, T, H, d_k, d_v, L, W, chunk, status, g_spin_limit.load(), chain,
                       need > 0 ? workspace : nullptr};
+  p.conv_state = conv_state;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype)) {

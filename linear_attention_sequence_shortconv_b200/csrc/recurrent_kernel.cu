@@ -178,9 +178,11 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   float w[PRISM_MAX_W];
 #pragma unroll
   for (int i = 0; i < PRISM_MAX_W; ++i) w[i] = (i < W) ? p.conv_w[((size_t)h * dv + c) * W + i] : 0.f;
-  float hist[PRISM_MAX_W];  // hist[i] = v_{t-1-i}[c]
+  float hist[PRISM_MAX_W];  // hist[i] = v_{t-1-i}[c]; before token 0 the sequence's history (or zero)
+  const T* cs = static_cast<const T*>(p.conv_state);
 #pragma unroll
-  for (int i = 0; i < PRISM_MAX_W; ++i) hist[i] = 0.f;
+  for (int i = 0; i < PRISM_MAX_W; ++i)
+    hist[i] = (cs && i < W - 1) ? ld1<T>(cs + (((size_t)b * H + h) * (W - 1) + (W - 2 - i)) * dv + c) : 0.f;
 
   float s[EPL];
   const size_t sbase = (((size_t)b * H + h) * dv + c) * dk + 4 * j;

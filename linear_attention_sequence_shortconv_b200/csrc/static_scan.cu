@@ -48,7 +48,7 @@ extern "C" int prism_scan_fwd_static(const void* q, const void* k, const void* v
                                      const float* beta, const void* u, const float* alpha, const void* gain,
                                      const float* conv_w, const float* S0, const int32_t* lengths, int B, int T,
                                      int H, int d_k, int d_v, int L, int W, int chunk, int dtype, void* o,
-                                     float* S_final, prism_stream_t stream, int chain) {
+                                     float* S_final, prism_stream_t stream, int chain, const void* conv_state) {
   if (chain != PRISM_CHAIN_LINEAR && chain != PRISM_CHAIN_GELU) return PRISM_ERR_INVALID_ARG;
   int rc = prism::check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype);
   if (rc != PRISM_OK) return rc;
@@ -63,5 +63,6 @@ extern "C" int prism_scan_fwd_static(const void* q, const void* k, const void* v
     if (rc != PRISM_OK) return rc;
   }
   return prism_scan_fwd_ex(q, k, v, gamma, beta, u, alpha, gain, conv_w, S0, lengths, B, T, H, d_k, d_v, L, W,
-                           chunk, dtype, o, S_final, ws, need > 0 ? kStaticWorkspaceBytes : 0, stream, chain);
+                           chunk, dtype, o, S_final, ws, need > 0 ? kStaticWorkspaceBytes : 0, stream, chain,
+                           conv_state);
 }

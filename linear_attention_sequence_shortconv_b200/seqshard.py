@@ -19,9 +19,8 @@ state from a zero start.  Each rank
      (prism_state_affine): its exact start state;
   4. scans its segment again from that state: its outputs and end state are exact.
 
-The ShortConv history enters a segment as W - 1 inert leading tokens (gamma = 1,
-beta = alpha = 0, q = k = u = gain = 0) that carry the previous segment's last v
-rows: they leave the state untouched and feed the first anchors.
+The ShortConv history enters a segment as the scan's conv_state: the previous
+segment's last W - 1 rows of v, which feed the segment's first anchors.
 
 Every step runs in the library (prism_scan_fwd, prism_state_affine); the two
 exchanges are torch.distributed all-gathers (NCCL over NVLink between GPUs).  The
@@ -56,9 +55,9 @@ class Segment:
 class LibraryOps:
     """The two operations the sharded scan needs, on the library."""
 
-    def scan(self, q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, chain, chunk):
+    def scan(self, q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, chain, chunk, conv_state=None):
         return _lib.scan_fwd(q, k, v, gamma, beta, u, alpha, gain, conv_w, L=L, chunk=chunk, S0=S0,
-                             lengths=lengths, chain=chain)
+                             lengths=lengths, chain=chain, conv_state=conv_state)
 
     def affine(self, S, M, N):
         return _lib.state_affine(S, M, N)
@@ -71,42 +70,30 @@ def halo_rows(v: torch.Tensor, W: int) -> torch.Tensor:
     return v[:, v.shape[1] - (W - 1):].contiguous()
 
 
-def extend(seg: Segment, halo: torch.Tensor) -> Segment:
-    """The segment with the inert history tokens in front (v = halo)."""
-    n = halo.shape[1]
-    if n == 0:
-        return seg
-
-    def lead(x, fill):
-        if x is None:
-            return None
-        pad = torch.full((x.shape[0], n) + tuple(x.shape[2:]), fill, dtype=x.dtype, device=x.device)
-        return torch.cat([pad, x], dim=1).contiguous()
-
-    return Segment(q=lead(seg.q, 0.0), k=lead(seg.k, 0.0), v=torch.cat([halo.to(seg.v.dtype), seg.v], 1).contiguous(),
-                   gamma=lead(seg.gamma, 1.0), beta=lead(seg.beta, 0.0), u=lead(seg.u, 0.0),
-                   alpha=lead(seg.alpha, 0.0), gain=lead(seg.gain, 0.0), start=seg.start - n)
+def conv_history(halo: torch.Tensor) -> torch.Tensor:
+    """Halo rows [B, W-1, H, d_v] as the scan's conv_state [B, H, W-1, d_v]."""
+    return halo.permute(0, 2, 1, 3).contiguous()
 
 
-def local_lengths(lengths: Optional[torch.Tensor], seg: Segment, n_tokens: int, n_halo: int):
-    """Valid tokens of the extended segment per sequence (None: all of them)."""
+def local_lengths(lengths: Optional[torch.Tensor], seg: Segment, n_tokens: int):
+    """Valid tokens of the segment per sequence (None: all of them)."""
     if lengths is None:
         return None
-    lo = seg.start + n_halo  # global index of the first real token
-    return ((lengths.to(torch.int64) - lo).clamp(0, n_tokens) + n_halo).to(torch.int32).contiguous()
+    return (lengths.to(torch.int64) - seg.start).clamp(0, n_tokens).to(torch.int32).contiguous()
 
 
-def segment_map(ext: Segment, conv_w, L: int, lens, chain: str, chunk: int, ops) -> Tuple[torch.Tensor, torch.Tensor]:
-    """(M, N) of an extended segment: S_end = S_start M + N."""
-    _, N = ops.scan(ext.q, ext.k, ext.v, ext.gamma, ext.beta, ext.u, ext.alpha, ext.gain, conv_w, L, None, lens,
-                    chain, chunk)
+def segment_map(seg: Segment, conv_w, L: int, lens, chain: str, chunk: int, ops,
+                conv_state=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(M, N) of a segment: S_end = S_start M + N (conv_state: its ShortConv history)."""
+    _, N = ops.scan(seg.q, seg.k, seg.v, seg.gamma, seg.beta, seg.u, seg.alpha, seg.gain, conv_w, L, None, lens,
+                    chain, chunk, conv_state)
     # the transitions alone: no writes (v = 0, L = 1), start from the identity
-    B, T, H, d_k = ext.k.shape
-    zq = torch.zeros_like(ext.q)
-    zv = torch.zeros((B, T, H, d_k), dtype=ext.v.dtype, device=ext.v.device)
-    zw = torch.zeros((H, d_k, 1), dtype=torch.float32, device=ext.v.device)
-    eye = torch.eye(d_k, dtype=torch.float32, device=ext.v.device).expand(B, H, d_k, d_k).contiguous()
-    _, M = ops.scan(zq, ext.k, zv, ext.gamma, ext.beta, None, None, None, zw, 1, eye, lens, chain, chunk)
+    B, T, H, d_k = seg.k.shape
+    zq = torch.zeros_like(seg.q)
+    zv = torch.zeros((B, T, H, d_k), dtype=seg.v.dtype, device=seg.v.device)
+    zw = torch.zeros((H, d_k, 1), dtype=torch.float32, device=seg.v.device)
+    eye = torch.eye(d_k, dtype=torch.float32, device=seg.v.device).expand(B, H, d_k, d_k).contiguous()
+    _, M = ops.scan(zq, seg.k, zv, seg.gamma, seg.beta, None, None, None, zw, 1, eye, lens, chain, chunk)
     return M, N
 
 
@@ -118,11 +105,10 @@ def start_state(S0, maps: List[Tuple[torch.Tensor, torch.Tensor]], like: torch.T
     return S
 
 
-def scan_segment(ext: Segment, conv_w, L: int, lens, chain: str, chunk: int, S_start, n_halo: int, ops):
+def scan_segment(seg: Segment, conv_w, L: int, lens, chain: str, chunk: int, S_start, ops, conv_state=None):
     """The exact outputs and end state of a segment from its start state."""
-    o, S_end = ops.scan(ext.q, ext.k, ext.v, ext.gamma, ext.beta, ext.u, ext.alpha, ext.gain, conv_w, L,
-                        S_start.contiguous(), lens, chain, chunk)
-    return o[:, n_halo:], S_end
+    return ops.scan(seg.q, seg.k, seg.v, seg.gamma, seg.beta, seg.u, seg.alpha, seg.gain, conv_w, L,
+                    S_start.contiguous(), lens, chain, chunk, conv_state)
 
 
 def scan_fwd_sequence_sharded(seg: Segment, conv_w, L: int, S0=None, lengths=None, chain: str = "linear",
@@ -148,11 +134,10 @@ def scan_fwd_sequence_sharded(seg: Segment, conv_w, L: int, S0=None, lengths=Non
     halos = [torch.empty_like(mine) for _ in range(P)]
     if W > 1:
         dist.all_gather(halos, mine, group=group)
-    halo = halos[rank - 1] if rank > 0 else torch.zeros_like(mine)
-    ext = extend(seg, halo)
-    lens = local_lengths(lengths, ext, n_tokens, W - 1)
+    hist = conv_history(halos[rank - 1]) if rank > 0 and W > 1 else None
+    lens = local_lengths(lengths, seg, n_tokens)
     # 2. this segment's map
-    M, N = segment_map(ext, conv_w, L, lens, chain, chunk, ops)
+    M, N = segment_map(seg, conv_w, L, lens, chain, chunk, ops, hist)
     # 3. every segment's map; fold the earlier ones into this segment's start state
     Ms = [torch.empty_like(M) for _ in range(P)]
     Ns = [torch.empty_like(N) for _ in range(P)]
@@ -160,16 +145,17 @@ def scan_fwd_sequence_sharded(seg: Segment, conv_w, L: int, S0=None, lengths=Non
     dist.all_gather(Ns, N.contiguous(), group=group)
     S_start = start_state(S0, list(zip(Ms[:rank], Ns[:rank])), N, ops)
     # 4. the exact pass
-    return scan_segment(ext, conv_w, L, lens, chain, chunk, S_start, W - 1, ops)
+    return scan_segment(seg, conv_w, L, lens, chain, chunk, S_start, ops, hist)
 
 
 def scan_fwd_segmented(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, P: int, S0=None, lengths=None,
                        chain: str = "linear", chunk: int = 64, ops=None):
     """The whole scan on one device with each sequence cut into P segments that run
     side by side: the segments are stacked along the batch axis (P x B sequences of
-    ceil(T / P) + W - 1 tokens), so each of the three scans has P times the
-    parallelism at 1/P of the length; the maps are folded in P - 1 affine steps.
-    Returns (o [B, T, H, d_v], S_final) as scan_fwd."""
+    ceil(T / P) tokens, each with the previous segment's last W - 1 rows of v as its
+    conv_state), so each of the three scans has P times the parallelism at 1/P of the
+    length; the maps are folded in P - 1 affine steps.  Returns (o [B, T, H, d_v],
+    S_final) as scan_fwd."""
     ops = ops or LibraryOps()
     B, T, H, _ = q.shape
     W = conv_w.shape[-1]
@@ -187,24 +173,25 @@ def scan_fwd_segmented(q, k, v, gamma, beta, u, alpha, gain, conv_w, L: int, P: 
                                           gain=gain).items()}
     if lengths is None:
         lengths = torch.full((B,), T, dtype=torch.int32, device=q.device)
-    exts, lens = [], []
+    segs, lens, hists = [], [], []
     for r in range(P):
         seg = Segment(**{n: None if x is None else x[:, r * Ts:(r + 1) * Ts] for n, x in full.items()},
                       start=r * Ts)
         halo = (full["v"][:, r * Ts - (W - 1):r * Ts] if r > 0 else
                 torch.zeros((B, W - 1) + tuple(v.shape[2:]), dtype=v.dtype, device=v.device))
-        ext = extend(seg, halo)
-        exts.append(ext)
-        lens.append(local_lengths(lengths, ext, Ts, W - 1))
+        segs.append(seg)
+        lens.append(local_lengths(lengths, seg, Ts))
+        hists.append(conv_history(halo))
     # every segment side by side: batch index r * B + b
     cat = lambda xs: None if xs[0] is None else torch.cat(xs, 0).contiguous()
-    stacked = Segment(**{n: cat([getattr(e, n) for e in exts]) for n in full}, start=0)
+    stacked = Segment(**{n: cat([getattr(e, n) for e in segs]) for n in full}, start=0)
     lens_all = torch.cat(lens, 0).contiguous()
-    M, N = segment_map(stacked, conv_w, L, lens_all, chain, chunk, ops)
+    hist = cat(hists) if W > 1 else None
+    M, N = segment_map(stacked, conv_w, L, lens_all, chain, chunk, ops, hist)
     Ms, Ns = M.view(P, B, *M.shape[1:]), N.view(P, B, *N.shape[1:])
     starts = [torch.zeros_like(Ns[0]) if S0 is None else S0]
     for r in range(1, P):
         starts.append(ops.affine(starts[-1].contiguous(), Ms[r - 1].contiguous(), Ns[r - 1].contiguous()))
-    o, S_end = scan_segment(stacked, conv_w, L, lens_all, chain, chunk, torch.cat(starts, 0), W - 1, ops)
+    o, S_end = scan_segment(stacked, conv_w, L, lens_all, chain, chunk, torch.cat(starts, 0), ops, hist)
     o = o.reshape(P, B, Ts, *o.shape[2:]).permute(1, 0, 2, 3, 4).reshape(B, P * Ts, *o.shape[2:])
     return o[:, :T], S_end.view(P, B, *S_end.shape[1:])[P - 1]

@@ -170,10 +170,20 @@ def test_host_entry_invalid_arguments(L):
 def test_unknown_residual_chain_is_rejected(L):
     a = [FAKE] * 9 + [None, None, 2, 8, 2, 64, 64, 4, 4, 64, 0, FAKE, None, None, 0, None]
     for chain in (-1, 2, 7):
-        assert L.prism_scan_fwd_ex(*a, chain) == 1
+        assert L.prism_scan_fwd_ex(*a, chain, None) == 1
         assert L.prism_prologue_fwd_ex(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 64, 4, 4, 0, FAKE, None, chain) == 1
     with pytest.raises(ValueError):
         prism._lib._chain_code("tanh")
+
+
+def test_conv_state_alignment_is_checked_before_launch(L):
+    # B=2 T=8 H=2 d=64 L=4 W=4 bf16, no workspace: a misaligned history is rejected first
+    a = [FAKE] * 9 + [None, None, 2, 8, 2, 64, 64, 4, 4, 64, 0, FAKE, None, None, 0, None, 0]
+    assert L.prism_scan_fwd_ex(*a, FAKE + 4) == 2
+    assert L.prism_scan_fwd_ex(*a, FAKE) == 3          # aligned: then the missing workspace
+    w1 = list(a)
+    w1[17] = 1                                          # W = 1: no history to read, ignored
+    assert L.prism_scan_fwd_ex(*w1, FAKE + 4) == 3
 
 
 def decode_call(lib_, **kw):

@@ -40,13 +40,14 @@ def _sharded_on_gpu(w, bounds, chain="linear"):
             for s, e in zip(bounds[:-1], bounds[1:])]
     ops = seqshard.LibraryOps()
     halos = [seqshard.halo_rows(s.v, W) for s in segs]
-    exts = [seqshard.extend(s, halos[i - 1] if i else torch.zeros_like(halos[0])) for i, s in enumerate(segs)]
-    lens = [seqshard.local_lengths(d["lengths"], e, s.v.shape[1], W - 1) for e, s in zip(exts, segs)]
-    maps = [seqshard.segment_map(e, d["conv_w"], w.L, ln, chain, w.chunk, ops) for e, ln in zip(exts, lens)]
+    hists = [seqshard.conv_history(halos[i - 1]) if i else None for i in range(len(segs))]
+    lens = [seqshard.local_lengths(d["lengths"], s, s.v.shape[1]) for s in segs]
+    maps = [seqshard.segment_map(s, d["conv_w"], w.L, ln, chain, w.chunk, ops, hs)
+            for s, ln, hs in zip(segs, lens, hists)]
     outs, S_end = [], None
-    for r, (e, ln) in enumerate(zip(exts, lens)):
+    for r, (sg, ln, hs) in enumerate(zip(segs, lens, hists)):
         S_start = seqshard.start_state(d["S0"], maps[:r], maps[0][1], ops)
-        o, S_end = seqshard.scan_segment(e, d["conv_w"], w.L, ln, chain, w.chunk, S_start, W - 1, ops)
+        o, S_end = seqshard.scan_segment(sg, d["conv_w"], w.L, ln, chain, w.chunk, S_start, ops, hs)
         outs.append(o)
     torch.cuda.synchronize()
     assert prism.stream_status() == 0

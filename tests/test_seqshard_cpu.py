@@ -25,15 +25,29 @@ def _free_port():
 
 
 class OracleOps:
-    """The library's two operations, restated by the oracle (fp64, CPU)."""
+    """The library's two operations, restated by the oracle (fp64, CPU).  A ShortConv
+    history (conv_state [B, H, W-1, d_v]) is fed to the oracle as W - 1 leading tokens
+    that carry it in v and leave the state alone (gamma = 1; beta = alpha = 0; q, k, u,
+    gain = 0); their outputs are dropped."""
 
-    def scan(self, q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, chain, chunk):
+    def scan(self, q, k, v, gamma, beta, u, alpha, gain, conv_w, L, S0, lengths, chain, chunk, conv_state=None):
         from oracle import prism_seq
 
         n = lambda t: None if t is None else t.double().numpy()
+        h = 0 if conv_state is None else conv_state.shape[2]
+        if h:
+            def lead(x, fill):
+                if x is None:
+                    return None
+                pad = torch.full((x.shape[0], h) + tuple(x.shape[2:]), fill, dtype=x.dtype)
+                return torch.cat([pad, x], 1)
+            q, k, u, gain = lead(q, 0.0), lead(k, 0.0), lead(u, 0.0), lead(gain, 0.0)
+            gamma, beta, alpha = lead(gamma, 1.0), lead(beta, 0.0), lead(alpha, 0.0)
+            v = torch.cat([conv_state.permute(0, 2, 1, 3).to(v.dtype), v], 1)
+            lengths = None if lengths is None else lengths + h
         o, S = prism_seq(n(q), n(k), n(v), n(gamma), n(beta), n(u) if L > 1 else None, n(alpha) if L > 1 else None,
                          n(gain) if L > 1 else None, n(conv_w), S0=n(S0), lengths=n(lengths), chain=chain)
-        return torch.from_numpy(o), torch.from_numpy(S)
+        return torch.from_numpy(o[:, h:]), torch.from_numpy(S)
 
     def affine(self, S, M, N):
         return torch.from_numpy(np.einsum("bhij,bhjk->bhik", S.double().numpy(), M.double().numpy())
@@ -144,13 +158,13 @@ def test_phases_without_collectives():
                                                                       "gain")}, start=s)
             for s, e in zip(bounds[:-1], bounds[1:])]
     halos = [seqshard.halo_rows(s.v, W) for s in segs]
-    exts = [seqshard.extend(s, halos[i - 1] if i else torch.zeros_like(halos[0])) for i, s in enumerate(segs)]
-    lens = [seqshard.local_lengths(None, e, s.v.shape[1], W - 1) for e, s in zip(exts, segs)]
-    maps = [seqshard.segment_map(e, p["conv_w"], L, ln, "linear", 64, ops) for e, ln in zip(exts, lens)]
+    hists = [seqshard.conv_history(halos[i - 1]) if i else None for i in range(len(segs))]
+    lens = [seqshard.local_lengths(None, s, s.v.shape[1]) for s in segs]
+    maps = [seqshard.segment_map(s, p["conv_w"], L, ln, "linear", 64, ops, hs) for s, ln, hs in zip(segs, lens, hists)]
     outs = []
-    for r, (e, ln) in enumerate(zip(exts, lens)):
+    for r, (sg, ln, hs) in enumerate(zip(segs, lens, hists)):
         S_start = seqshard.start_state(p["S0"], maps[:r], maps[0][1], ops)
-        o, S_end = seqshard.scan_segment(e, p["conv_w"], L, ln, "linear", 64, S_start, W - 1, ops)
+        o, S_end = seqshard.scan_segment(sg, p["conv_w"], L, ln, "linear", 64, S_start, ops, hs)
         outs.append(o.numpy())
     n = lambda t: t.numpy()
     o_ref, S_ref = prism_seq(n(p["q"]), n(p["k"]), n(p["v"]), n(p["gamma"]), n(p["beta"]), n(p["u"]), n(p["alpha"]),

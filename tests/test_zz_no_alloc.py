@@ -18,7 +18,7 @@ def _static_call(**kw):
     a.update(kw)
     return prism.lib().prism_scan_fwd_static(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
                                              a["B"], a["T"], a["H"], a["d_k"], a["d_v"], a["L"], a["W"], a["chunk"],
-                                             a["dtype"], FAKE, None, None, a["chain"])
+                                             a["dtype"], FAKE, None, None, a["chain"], None)
 
 
 def test_static_scratch_holds_the_layer_shapes():
