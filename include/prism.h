@@ -296,7 +296,7 @@ int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, 
  * (batch row, head) chains is cut into segments; when the chains leave at least 24 of
  * a B200's SMs idle, L > 1 and the sequence has at least 8 chunks, four: the scan runs
  * in two halves, and the second half's residual write runs beside the first half's
- * scan (on two internal streams of the device, forked from and joined back into the
+ * scan (on an internal stream of the device, forked from and joined back into the
  * call's stream).  Token-by-token path: 1. */
 int prism_scan_fwd_launches(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype);
 

@@ -400,6 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  // this CTA holds its SM: a kernel launched after this one with programmatic dependent
+  // launch (the residual write of a second half) may start once every CTA has got here
+  if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const uint32_t aKQ = smem_u32(sKQ), aKB = smem_u32(sKB), aZB = smem_u32(sZB), aWQ = smem_u32(sWQ);
   const uint32_t aUB0 = smem_u32(sm + Ly::UB), aPB0 = smem_u32(sm + Ly::PB), aBQ0 = smem_u32(sBQ0);
@@ -1332,14 +1335,15 @@ TimeSplit time_split(int B, int T, int H, int L) {
   return {on, (nc + 1) / 2};
 }
 
-// Side streams of a device for the two halves: the first scan launch on a stream of the
-// greatest priority (so that its CTAs take SMs before the second half's residual write),
-// that residual write on a stream of the least priority; fork and join through events on
-// the caller's stream.  Created on first use; a mutex keeps the record / wait sequences of
-// concurrent callers from interleaving.
+// The side stream of a device for the two halves: the first scan launch, then the second
+// half's residual write as a programmatic dependent launch, which starts once every CTA of
+// the scan holds its SM (so it takes only the SMs the scan leaves idle) and does not wait
+// for the scan to finish.  Fork and join through events on the caller's stream; the join
+// event, recorded after both, completes once both have.  Created on first use; a mutex
+// keeps the record / wait sequences of concurrent callers from interleaving.
 struct SideStreams {
-  cudaStream_t hi = nullptr, lo = nullptr;
-  cudaEvent_t forked = nullptr, scan_a = nullptr, res_b = nullptr;
+  cudaStream_t hi = nullptr;
+  cudaEvent_t forked = nullptr, joined = nullptr;
 };
 constexpr int kMaxSideDevices = 64;
 std::mutex g_side_mutex;
@@ -1354,10 +1358,8 @@ cudaError_t side_streams(SideStreams** out) {  // with g_side_mutex held
   if (!x.hi) {
     int least = 0, greatest = 0;
     if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
-    if ((e = cudaStreamCreateWithPriority(&x.lo, cudaStreamNonBlocking, least)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&x.forked, cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&x.scan_a, cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&x.res_b, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&x.joined, cudaEventDisableTiming)) != cudaSuccess) return e;
     if ((e = cudaStreamCreateWithPriority(&x.hi, cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
   }
   *out = &x;
@@ -1404,14 +1406,23 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
   const __nv_bfloat16* vv = static_cast<const __nv_bfloat16*>(p.v);
   const __nv_bfloat16* gg = static_cast<const __nv_bfloat16*>(p.gain);
   const __nv_bfloat16* cs = static_cast<const __nv_bfloat16*>(p.conv_state);
-  auto residual = [&](int nc0, int ncn, cudaStream_t st) {
-    const dim3 grid(p.B * p.H * ncn * (kC / prep_tokens(D)));
+  // the residual write of chunks [nc0, nc0 + ncn); `dependent`: as a programmatic dependent
+  // launch of the kernel before it on the stream
+  auto residual = [&](int nc0, int ncn, cudaStream_t st, bool dependent) -> cudaError_t {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.B * p.H * ncn * (kC / prep_tokens(D)));
+    cfg.blockDim = dim3(kPrepThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
     if (p.W <= 4)
-      residual_write_kernel<D, CH, 4><<<grid, kPrepThreads, 0, st>>>(vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths,
-                                                                      cs, ptil, p.T, p.H, p.W, m, nc0, ncn);
-    else
-      residual_write_kernel<D, CH, PRISM_MAX_W><<<grid, kPrepThreads, 0, st>>>(
-          vv, gg, p.alpha, p.gamma, p.conv_w, p.lengths, cs, ptil, p.T, p.H, p.W, m, nc0, ncn);
+      return cudaLaunchKernelEx(&cfg, residual_write_kernel<D, CH, 4>, vv, gg, p.alpha, p.gamma, p.conv_w,
+                                p.lengths, cs, ptil, p.T, p.H, p.W, m, nc0, ncn);
+    return cudaLaunchKernelEx(&cfg, residual_write_kernel<D, CH, PRISM_MAX_W>, vv, gg, p.alpha, p.gamma, p.conv_w,
+                              p.lengths, cs, ptil, p.T, p.H, p.W, m, nc0, ncn);
   };
   if (m > 0) {
     const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)m, H, T, B};
@@ -1419,7 +1430,8 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
     const cuuint32_t box5[5] = {64, 1, 1, 64, 1};
     if (!encode(&mu, p.u, 5, dims5, str5, box5) || !encode(&mg, ptil, 5, dims5, str5, box5))
       return cudaErrorInvalidValue;
-    residual(0, split.on ? split.nA : NC, stream);
+    const cudaError_t e = residual(0, split.on ? split.nA : NC, stream, false);
+    if (e != cudaSuccess) return e;
     if (p.split_event) {
       const cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(p.split_event), stream);
       if (e != cudaSuccess) return e;
@@ -1453,16 +1465,12 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
       cudaError_t e = side_streams(&ss);
       if (e == cudaSuccess) e = cudaEventRecord(ss->forked, stream);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->hi, ss->forked, 0);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->lo, ss->forked, 0);
       if (e != cudaSuccess) return e;
       prism_scan_kernel<D, CH><<<p.B * p.H, kThreads, Ly::ALLOC, ss->hi>>>(mq, mk, mu, mv, mg, aA);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      residual(split.nA, NC - split.nA, ss->lo);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      if ((e = cudaEventRecord(ss->scan_a, ss->hi)) != cudaSuccess) return e;
-      if ((e = cudaEventRecord(ss->res_b, ss->lo)) != cudaSuccess) return e;
-      if ((e = cudaStreamWaitEvent(stream, ss->scan_a, 0)) != cudaSuccess) return e;
-      if ((e = cudaStreamWaitEvent(stream, ss->res_b, 0)) != cudaSuccess) return e;
+      if ((e = residual(split.nA, NC - split.nA, ss->hi, true)) != cudaSuccess) return e;
+      if ((e = cudaEventRecord(ss->joined, ss->hi)) != cudaSuccess) return e;
+      if ((e = cudaStreamWaitEvent(stream, ss->joined, 0)) != cudaSuccess) return e;
     }
     prism_scan_kernel<D, CH><<<p.B * p.H, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aB);
     return cudaGetLastError();
