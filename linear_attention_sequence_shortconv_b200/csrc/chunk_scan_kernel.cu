@@ -1,7 +1,10 @@
-// Chunkwise-parallel PRISM scan on the 5th-generation tensor cores (tcgen05), one launch.
+// Chunkwise-parallel PRISM scan on the 5th-generation tensor cores (tcgen05): a launch of
+// residual_write_kernel (the residual write vectors of every token), then the scan.
 //
-// One CTA owns one (batch row, head) chain and walks its chunks of C = 64 tokens in
-// order; the fp32 state S (d_v x d_k) stays in tensor memory for the whole sequence.
+// One scan CTA owns one (batch row, head) chain and walks its chunks of C = 64 tokens in
+// order; the fp32 state S (d_v x d_k) stays in tensor memory for the whole sequence (or
+// segment: long sequences over few chains are cut into segments, and a sequence whose
+// chains leave SMs idle runs in two halves; see the host side at the end).
 // Sources: ICML 2026 PRISM write-up (核心迭代形式, 消除 Token 间串行, 消除 Step 间串行,
 // 架构形式) and the PRISM technical summary (2.1, 2.2), which fix the recurrence; the
 // chunk form below is derived from it.
