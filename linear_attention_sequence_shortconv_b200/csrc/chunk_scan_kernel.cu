@@ -76,6 +76,8 @@ constexpr uint32_t kAtom64 = 8192;    // the same with 64 rows
 constexpr uint32_t kAtomV = 9216;     // 72 rows of v: 8 of ShortConv history, then the chunk
 constexpr long long kDrainLimit = 1ll << 18;
 constexpr int kWsLd = 68;  // fp32 row stride of the inverse's scratch (bank padding)
+constexpr int kRankRows = 1024;  // rows the scan ranks by length (longest first) when chains exceed SMs
+constexpr int kPlanSMs = 148;    // SMs of a B200: the segment plan and the chain order assume them
 
 // TMEM columns
 // RU: [K;Q] U_l^T, two slots (directions alternate); RW ([W'; Mqk W']) reuses them once the
@@ -364,10 +366,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::SMALL + 2 * sizeof(Gates));
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  static_assert(2 * sizeof(Gates) + 8 * kNumBars + 8 <= 4096, "small region");
+  static_assert(2 * sizeof(Gates) + 8 * kNumBars + 12 <= 4096, "small region");
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = p.seg_only >= 0 ? (int)blockIdx.x : (int)blockIdx.x / p.P;
+  // The chain of this CTA.  With ragged lengths and one CTA per chain, the CTA of rank r
+  // takes a head of the (r / H)-th longest row (ties: the lower row first): CTAs start in
+  // rank order, so when there are more chains than SMs the long rows start first and the
+  // short ones fill in behind them.
+  int chain = p.seg_only >= 0 ? (int)blockIdx.x : (int)blockIdx.x / p.P;
+  if (p.lengths && (p.P == 1 || p.seg_only >= 0) && p.B <= kRankRows && p.B * p.H > kPlanSMs) {
+    int* s_pick = reinterpret_cast<int*>(s_tmem + 2);
+    const int want = chain / p.H;
+    for (int cand = tid; cand < p.B; cand += kThreads) {
+      const int lc = min(max(p.lengths[cand], 0), p.T);
+      int rank = 0;
+      for (int o = 0; o < p.B; ++o) {
+        const int lo = min(max(p.lengths[o], 0), p.T);
+        rank += (lo > lc || (lo == lc && o < cand)) ? 1 : 0;
+      }
+      if (rank == want) *s_pick = cand;
+    }
+    __syncthreads();
+    chain = *s_pick * p.H + chain % p.H;
+  }
+  const int bh = chain;
   const int seg = p.seg_only >= 0 ? p.seg_only : (int)blockIdx.x % p.P, b = bh / p.H, h = bh % p.H;
   const int T = p.T, H = p.H, m = p.m;
   const int len = p.lengths ? min(max(p.lengths[b], 0), T) : T;
@@ -1309,7 +1331,6 @@ bool encode(CUtensorMap* map, const void* ptr, int rank, const cuuint64_t* dims,
 // device, so that the plan (and with it the rounding of the results and the workspace size)
 // is a function of the sizes alone.  A plan cuts only sequences of at least 32 chunks whose
 // chains fill under half of those SMs, into segments of at least 16 chunks.
-constexpr int kPlanSMs = 148;
 struct SegPlan {
   int P, Ts;
 };

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from linear_attention_sequence_shortconv_b200 import synth
-from oracle import gdn_seq, max_abs_rel_err, residual_chain
+from oracle import gdn_seq, max_abs_rel_err, prism_seq, residual_chain
 from tests.helpers import TOL, gpu_run, oracle_run, rel_err
 
 pytestmark = pytest.mark.gpu
@@ -278,3 +278,19 @@ def test_strongly_decaying_chunks(name, chain):
     o_ref, S_ref = oracle_run(inp, w, chain=chain)
     assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
     assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
+
+
+def test_ragged_rows_exceeding_the_sms():
+    """More chains than SMs with ragged lengths (the scan takes the rows longest first),
+    every chain against the oracle, empty rows included."""
+    w = synth.Workload("ragged160", B=80, T=150, H=2, d_k=64, d_v=64, L=3, chunk=64, lengths_lo=0,
+                       with_s0=True, seed=31)
+    inp = synth.make_inputs(w)
+    inp["lengths"][::7] = 0
+    o, S = gpu_run(inp, w)
+    x = synth.to_float64_numpy(inp)
+    o_ref, S_ref = prism_seq(**x)
+    assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
+    for b, n in enumerate(inp["lengths"].tolist()):
+        assert np.all(o[b, n:] == 0)
