@@ -1151,8 +1151,8 @@ __host__ __device__ constexpr int prep_tokens(int D) { return kPrepThreads * kPr
 
 __device__ __forceinline__ uint4 ldg16(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
-template <int D, int CH, int WM>  // WM >= W: taps held in registers
-__global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
+template <int D, int CH, int WM>  // WM >= W: taps of a head in shared memory
+__global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
     residual_write_kernel(const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ gain,
                           const float* __restrict__ alpha, const float* __restrict__ gamma,
                           const float* __restrict__ conv_w, const int32_t* __restrict__ lengths,
@@ -1165,6 +1165,7 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
   constexpr int LB = kPrepLevels;
   static_assert(PB >= 1 && kC % prep_tokens(D) == 0, "CTA tiling of a chunk");
   __shared__ float s_c[kC];  // e^{G_63 - G_t} (1 when the chunk's decay is not factored)
+  __shared__ __align__(16) float s_taps[WM][D];  // ShortConv taps of the head, tap-major
   const int part = blockIdx.x % PB, cidx = blockIdx.x / PB;
   const int n = nc0 + cidx % ncn, bh = cidx / ncn, b = bh / H, h = bh % H;
   const int len = lengths ? min(max(lengths[b], 0), T) : T;
@@ -1199,6 +1200,10 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
       }
   };
   load_levels(0);
+  for (int e = tid; e < WM * D; e += kPrepThreads) {
+    const int w = e / D, c = e % D;
+    s_taps[w][c] = w < W ? __ldg(conv_w + ((size_t)h * D + c) * W + w) : 0.f;
+  }
   if (tid < 32) {
     const int nv = min(kC, len - t0);
     float gl[2];
@@ -1213,31 +1218,33 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 3 : 2)
     s_c[2 * lane] = fast ? __expf(G63 - G0) : 1.f;
     s_c[2 * lane + 1] = fast ? __expf(G63 - G1) : 1.f;
   }
+  __syncthreads();  // s_taps, s_c
   float r[TPT][8];
   {
-    float taps[WM][8];
-#pragma unroll
-    for (int w = 0; w < WM; ++w)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) taps[w][e] = w < W ? __ldg(conv_w + ((size_t)h * D + c8 + e) * W + w) : 0.f;
+    auto tap8 = [&](int w, float* t8) {
+      const float4 x = *reinterpret_cast<const float4*>(&s_taps[w][c8]);
+      const float4 y = *reinterpret_cast<const float4*>(&s_taps[w][c8 + 4]);
+      t8[0] = x.x; t8[1] = x.y; t8[2] = x.z; t8[3] = x.w; t8[4] = y.x; t8[5] = y.y; t8[6] = y.z; t8[7] = y.w;
+    };
 #pragma unroll
     for (int a = 0; a < TPT; ++a) {
-      float vt[8];
+      float vt[8], tw[8];
       unpack8(vr[a + WM - 1], vt);
+      tap8(0, tw);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) r[a][e] = vt[e] - taps[0][e] * vt[e];
+      for (int e = 0; e < 8; ++e) r[a][e] = vt[e] - tw[e] * vt[e];
 #pragma unroll
       for (int w = 1; w < WM; ++w) {
         if (w < W) {
           float vw[8];
           unpack8(vr[a + WM - 1 - w], vw);
+          tap8(w, tw);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) r[a][e] -= taps[w][e] * vw[e];
+          for (int e = 0; e < 8; ++e) r[a][e] -= tw[e] * vw[e];
         }
       }
     }
   }
-  __syncthreads();  // s_c
   float cs[TPT];
 #pragma unroll
   for (int a = 0; a < TPT; ++a) cs[a] = s_c[i0 + a];
