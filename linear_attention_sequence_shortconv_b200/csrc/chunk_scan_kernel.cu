@@ -376,12 +376,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   int chain = p.seg_only >= 0 ? (int)blockIdx.x : (int)blockIdx.x / p.P;
   if (p.lengths && (p.P == 1 || p.seg_only >= 0) && p.B <= kRankRows && p.B * p.H > kPlanSMs) {
     int* s_pick = reinterpret_cast<int*>(s_tmem + 2);
+    int* s_len = reinterpret_cast<int*>(sBQ0);  // scratch: the [Bku;Mqu] tiles are not in use yet
+    for (int r = tid; r < p.B; r += kThreads) s_len[r] = min(max(p.lengths[r], 0), p.T);
+    __syncthreads();
     const int want = chain / p.H;
     for (int cand = tid; cand < p.B; cand += kThreads) {
-      const int lc = min(max(p.lengths[cand], 0), p.T);
+      const int lc = s_len[cand];
       int rank = 0;
       for (int o = 0; o < p.B; ++o) {
-        const int lo = min(max(p.lengths[o], 0), p.T);
+        const int lo = s_len[o];
         rank += (lo > lc || (lo == lc && o < cand)) ? 1 : 0;
       }
       if (rank == want) *s_pick = cand;

@@ -294,3 +294,21 @@ def test_ragged_rows_exceeding_the_sms():
     assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
     for b, n in enumerate(inp["lengths"].tolist()):
         assert np.all(o[b, n:] == 0)
+
+
+@pytest.mark.parametrize("d,L", [(128, 4), (64, 3)])
+def test_two_halves_with_ragged_rows(d, L):
+    """The scan in two launches (chains that leave SMs idle, 15 chunks), with rows that end
+    inside the first half, inside the second, exactly at the split and an empty row: the
+    hand-over of the end states between the launches, against the oracle."""
+    w = synth.Workload("halves", B=5, T=900, H=2, d_k=d, d_v=d, L=L, chunk=64, with_s0=True, seed=37 + d)
+    import linear_attention_sequence_shortconv_b200 as prism
+    assert prism.scan_fwd_launches(w.B, w.T, w.H, d, d, L, w.W, 64, 0) == 4  # two halves
+    inp = synth.make_inputs(w)
+    inp["lengths"] = torch.tensor([900, 400, 0, 512, 777], dtype=torch.int32)
+    o, S = gpu_run(inp, w)
+    o_ref, S_ref = prism_seq(**synth.to_float64_numpy(inp))
+    assert max_abs_rel_err(o, o_ref) <= TOL["bf16"]
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL["bf16"]
+    for b, n in enumerate(inp["lengths"].tolist()):
+        assert np.all(o[b, n:] == 0)
