@@ -55,6 +55,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <functional>
 #include <mutex>
 
 #include "common.cuh"
@@ -73,7 +74,6 @@ constexpr int kTW = 13;           // TMA warp
 constexpr int kThreads = 448;
 constexpr uint32_t kAtom128 = 16384;  // one 128-row, 128-byte-wide swizzle atom column
 constexpr uint32_t kAtom64 = 8192;    // the same with 64 rows
-constexpr uint32_t kAtomV = 9216;     // 72 rows of v: 8 of ShortConv history, then the chunk
 constexpr long long kDrainLimit = 1ll << 18;
 constexpr int kWsLd = 68;  // fp32 row stride of the inverse's scratch (bank padding)
 constexpr int kRankRows = 1024;  // rows the scan ranks by length (longest first) when chains exceed SMs
@@ -84,16 +84,22 @@ constexpr int kPlanSMs = 148;    // SMs of a B200: the segment plan and the chai
 // direction loop is done.
 constexpr uint32_t kRS = 0, kACC = 128, kSB = 256, kRKQ = 320, kRU = 384, kRW = 384;
 
-template <int D>
+// NU: shared-memory slots for U_l (direction j uses slot j % NU); P~_l always has two.
+// With NU = 3 (many residual directions) the chunk's v tile has no buffer of its own: it
+// is loaded into the [-W'; Q'] buffer once the key group's inverse scratch there is free,
+// and read before [-W'; Q'] is written.
+template <int D, int NU>
 struct Lay {
+  static_assert(NU == 2 || NU == 3, "U slots");
   static constexpr int NA = D / 64;
+  static constexpr bool kVinWQ = NU == 3;
   static constexpr uint32_t KQ = 0;                          // [K;Q] per atom column
   static constexpr uint32_t KB = KQ + NA * kAtom128;         // K for the state update
-  static constexpr uint32_t UB = KB + NA * kAtom64;          // U_l, two slots
-  static constexpr uint32_t PB = UB + 2 * NA * kAtom64;      // gain -> P~_l, two slots
+  static constexpr uint32_t UB = KB + NA * kAtom64;          // U_l, NU slots
+  static constexpr uint32_t PB = UB + NU * NA * kAtom64;     // P~_l, two slots
   static constexpr uint32_t BQ = PB + 2 * NA * kAtom64;      // [Bku_l;Mqu_l], two slots; slot 0 also X0^T
-  static constexpr uint32_t VB = BQ + 2 * kAtom128;          // v, 72 rows
-  static constexpr uint32_t ZB = VB + NA * kAtomV;           // [T; Mqk | MqkT]
+  static constexpr uint32_t VB = BQ + 2 * kAtom128;          // v (64 rows), unless it goes to WQ
+  static constexpr uint32_t ZB = VB + (kVinWQ ? 0 : NA * kAtom64);  // [T; Mqk | MqkT]
   static constexpr uint32_t WQ = ZB + kAtom128;              // [-W'; Q']
   static constexpr uint32_t WS_BYTES = 64 * kWsLd * 4 + 4096;
   // the inverse's scratch lives in WQ when it fits (WQ is free while the inverse runs)
@@ -140,7 +146,8 @@ struct Gates {
 
 // Barriers (one 8-byte word each, in shared memory).
 enum Bar {
-  kKqFull, kKqFree, kKbFull, kVFull, kVFree, kUgFull0, kUgFull1, kSlotFree0, kSlotFree1, kRuFull0, kRuFull1,
+  kKqFull, kKqFree, kKbFull, kVFull, kVFree, kWsFree, kUFull0, kUFull1, kUFull2, kPFull0, kPFull1, kUFree0,
+  kUFree1, kUFree2, kPFree0, kPFree1, kRuFull0, kRuFull1,
   kEpiDone0, kEpiDone1, kE1Done, kKqkFree, kBkupDone, kX0Ready, kZReady, kWqReady, kAccFull, kDlReady, kRsFull,
   kGates0, kGates1, kGFree0, kGFree1, kKgMma, kDrain, kKgDrain, kRwFull, kNumBars
 };
@@ -346,19 +353,20 @@ __device__ __forceinline__ void invert_unit_lower64(float* sA, float* sY, int ti
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int D, int CH>
+template <int D, int NU>
 __global__ void __launch_bounds__(kThreads, 1)
     prism_scan_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_v,
                       const __grid_constant__ CUtensorMap map_g, ScanArgs p) {
-  using Ly = Lay<D>;
+  using Ly = Lay<D, NU>;
   constexpr int NA = Ly::NA;
+  constexpr bool VW = Ly::kVinWQ;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sKQ = sm + Ly::KQ;
   uint8_t* sKB = sm + Ly::KB;
   uint8_t* sBQ0 = sm + Ly::BQ;
-  uint8_t* sVB = sm + Ly::VB;
+  uint8_t* sVB = VW ? sm + Ly::WQ : sm + Ly::VB;  // the chunk's v tile
   uint8_t* sZB = sm + Ly::ZB;
   uint8_t* sWQ = sm + Ly::WQ;
   float* sWS = reinterpret_cast<float*>(sm + Ly::WS);
@@ -437,34 +445,51 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTW) {
     // ================================================================ TMA warp
-    // Lane 0 issues every load in one fixed order that follows their consumption, waiting
-    // (bounded) for each buffer to be released: chunk n's directions from the third on,
-    // then the next chunk's first two directions, its v, [K;Q] and K.  Every wait is on a
-    // release that needs only loads issued before it, so the order cannot deadlock.
+    // Lane 0 issues every load in one fixed order that follows the order in which their
+    // buffers are released, waiting (bounded) for each release.  Per chunk n: P~ of the
+    // directions from the third on (two slots) and U from the (NU + 1)-th on (NU slots);
+    // with v in the [-W'; Q'] buffer, the chunk's v (once the key group's inverse scratch
+    // there is free); then the next chunk's first NU U, first two P~, (v), [K;Q] and K.
+    // Every wait is on a release that needs only loads issued before it, so the order
+    // cannot deadlock.
     if (lane == 0) {
-      int n_kq = 0, n_v = 0, n_kb = 0, j_ug = 0;  // loads issued per stream
+      int n_kq = 0, n_v = 0, n_kb = 0, nu[3] = {0, 0, 0}, np[2] = {0, 0};  // loads issued per stream
       auto prefetch = [&](int n) {  // every tile of chunk n into L2
         const int t0 = tok0 + n * kC;
         for (int a = 0; a < NA; ++a) {
           tma_prefetch_l2_4d(&map_k, 64 * a, h, t0, b);
           tma_prefetch_l2_4d(&map_q, 64 * a, h, t0, b);
-          if (!p.writes_off) tma_prefetch_l2_4d(&map_v, 64 * a, h, t0 - 8, b);
+          if (!p.writes_off) tma_prefetch_l2_4d(&map_v, 64 * a, h, t0, b);
           for (int l = 0; l < m; ++l) {
             tma_prefetch_l2_5d(&map_u, 64 * a, l, h, t0, b);
             tma_prefetch_l2_5d(&map_g, 64 * a, l, h, t0, b);
           }
         }
       };
-      auto ld_ug = [&](int j) -> bool {  // U_l and gain_l of direction j into slot j & 1
-        const int s = j & 1;
-        if (j >= 2 && !bwait(&bars[kSlotFree0 + s], ((j >> 1) - 1) & 1, lim, status, s_abort)) return false;
+      // U_l of direction j into slot j % NU; with NU = 2 P~_l comes with it on the same
+      // barrier (both slots are freed by the same MMAs), else it has its own (ld_p)
+      auto ld_u = [&](int j) -> bool {
+        const int s = j % NU;
+        if (j >= NU && !bwait(&bars[kUFree0 + s], ((j / NU) - 1) & 1, lim, status, s_abort)) return false;
         const int t0 = tok0 + (j / m) * kC, l = j % m;
-        mbar_arrive_expect_tx(&bars[kUgFull0 + s], 2 * NA * kAtom64);
+        mbar_arrive_expect_tx(&bars[kUFull0 + s], (NU == 2 ? 2 : 1) * NA * kAtom64);
         for (int a = 0; a < NA; ++a) {
-          tma_load_5d(sm + Ly::UB + (s * NA + a) * kAtom64, &map_u, &bars[kUgFull0 + s], 64 * a, l, h, t0, b);
-          tma_load_5d(sm + Ly::PB + (s * NA + a) * kAtom64, &map_g, &bars[kUgFull0 + s], 64 * a, l, h, t0, b);
+          tma_load_5d(sm + Ly::UB + (s * NA + a) * kAtom64, &map_u, &bars[kUFull0 + s], 64 * a, l, h, t0, b);
+          if (NU == 2)
+            tma_load_5d(sm + Ly::PB + (s * NA + a) * kAtom64, &map_g, &bars[kUFull0 + s], 64 * a, l, h, t0, b);
         }
-        ++j_ug;
+        ++nu[s];
+        return true;
+      };
+      auto ld_p = [&](int j) -> bool {  // P~_l of direction j into slot j % 2 (NU = 3)
+        if (NU == 2) return true;
+        const int s = j & 1;
+        if (j >= 2 && !bwait(&bars[kPFree0 + s], ((j >> 1) - 1) & 1, lim, status, s_abort)) return false;
+        const int t0 = tok0 + (j / m) * kC, l = j % m;
+        mbar_arrive_expect_tx(&bars[kPFull0 + s], NA * kAtom64);
+        for (int a = 0; a < NA; ++a)
+          tma_load_5d(sm + Ly::PB + (s * NA + a) * kAtom64, &map_g, &bars[kPFull0 + s], 64 * a, l, h, t0, b);
+        ++np[s];
         return true;
       };
       auto ld_kq = [&](int n) -> bool {
@@ -479,12 +504,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++n_kq;
         return true;
       };
+      // v of chunk n: into its own buffer once the epilogue group has read chunk n - 1's,
+      // or (VW) into the [-W'; Q'] buffer once the key group's inverse scratch there is free
       auto ld_v = [&](int n) -> bool {
         if (p.writes_off) return true;
-        if (n >= 1 && !bwait(&bars[kVFree], (n - 1) & 1, lim, status, s_abort)) return false;
-        mbar_arrive_expect_tx(&bars[kVFull], NA * kAtomV);
+        if (VW ? !bwait(&bars[kWsFree], n & 1, lim, status, s_abort)
+               : (n >= 1 && !bwait(&bars[kVFree], (n - 1) & 1, lim, status, s_abort)))
+          return false;
+        mbar_arrive_expect_tx(&bars[kVFull], NA * kAtom64);
         for (int a = 0; a < NA; ++a)
-          tma_load_4d(sVB + a * kAtomV, &map_v, &bars[kVFull], 64 * a, h, tok0 + n * kC - 8, b);
+          tma_load_4d(sVB + a * kAtom64, &map_v, &bars[kVFull], 64 * a, h, tok0 + n * kC, b);
         ++n_v;
         return true;
       };
@@ -506,14 +535,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_prefetch_desc(&map_g);
         }
         if (nchunks > 1) prefetch(1);
-        ok = ld_kq(0) && ld_v(0) && ld_kb(0);
-        for (int l = 0; l < min(m, 2) && ok; ++l) ok = ld_ug(l);
+        ok = ld_kq(0) && (VW || ld_v(0)) && ld_kb(0);
+        for (int l = 0; l < min(m, NU) && ok; ++l) ok = ld_u(l);
+        for (int l = 0; l < min(m, 2) && ok; ++l) ok = ld_p(l);
       }
       for (int n = 0; n < nchunks && ok; ++n) {
-        for (int l = 2; l < m && ok; ++l) ok = ld_ug(n * m + l);
+        for (int l = 2; l < m && ok; ++l) {
+          if (l >= NU) ok = ld_u(n * m + l);
+          ok = ok && ld_p(n * m + l);
+        }
+        if (VW) ok = ok && ld_v(n);
         if (n + 1 < nchunks && ok) {
-          for (int l = 0; l < min(m, 2) && ok; ++l) ok = ld_ug((n + 1) * m + l);
-          ok = ok && ld_v(n + 1) && ld_kq(n + 1) && ld_kb(n + 1);
+          for (int l = 0; l < min(m, NU) && ok; ++l) ok = ld_u((n + 1) * m + l);
+          for (int l = 0; l < min(m, 2) && ok; ++l) ok = ld_p((n + 1) * m + l);
+          ok = ok && (VW || ld_v(n + 1)) && ld_kq(n + 1) && ld_kb(n + 1);
         }
       }
       // drain on an abort: the last phase of every barrier a load was issued on has completed
@@ -521,10 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n_kq > 0) mbar_wait(&bars[kKqFull], (n_kq - 1) & 1, kDrainLimit, status);
         if (n_v > 0) mbar_wait(&bars[kVFull], (n_v - 1) & 1, kDrainLimit, status);
         if (n_kb > 0) mbar_wait(&bars[kKbFull], (n_kb - 1) & 1, kDrainLimit, status);
-        for (int s2 = 0; s2 < 2; ++s2) {
-          const int uses = (j_ug + 1 - s2) / 2;  // loads issued on slot s2
-          if (uses > 0) mbar_wait(&bars[kUgFull0 + s2], (uses - 1) & 1, kDrainLimit, status);
-        }
+#pragma unroll
+        for (int s2 = 0; s2 < 3; ++s2)
+          if (nu[s2] > 0) mbar_wait(&bars[kUFull0 + s2], (nu[s2] - 1) & 1, kDrainLimit, status);
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2)
+          if (np[s2] > 0) mbar_wait(&bars[kPFull0 + s2], (np[s2] - 1) & 1, kDrainLimit, status);
       }
     }
     __syncwarp();
@@ -535,11 +572,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       int j = 0;
       // MMA-b and MMA-e of direction jj (direction l of chunk n)
       auto do_be = [&](int n, int jj, int l) -> bool {
-        const int s = jj & 1;
+        const int s = jj & 1, su = jj % NU;
         if (!bwait(&bars[kEpiDone0 + s], (jj >> 1) & 1, lim, status, s_abort)) return false;
+        if (NU == 3 && !bwait(&bars[kPFull0 + s], (jj >> 1) & 1, lim, status, s_abort)) return false;
         if (l == 0 && !bwait(&bars[kE1Done], n & 1, lim, status, s_abort)) return false;
         tc_fence_after();
-        const uint32_t aP = aPB0 + s * NA * kAtom64, aU = aUB0 + s * NA * kAtom64, aB = aBQ0 + s * kAtom128;
+        const uint32_t aP = aPB0 + s * NA * kAtom64, aU = aUB0 + su * NA * kAtom64, aB = aBQ0 + s * kAtom128;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + kACC, mndesc(aP, kk, kAtom64), kdesc(aB, kk, kAtom128), idesc_bf16(128, 128, 1, 0),
@@ -547,7 +585,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmem + kRS, mndesc(aP, kk, kAtom64), mndesc(aU, kk, kAtom64), idesc_bf16(128, D, 1, 1), 1);
-        mma_commit(&bars[kSlotFree0 + s]);
+        if (NU == 3) mma_commit(&bars[kPFree0 + s]);
+        mma_commit(&bars[kUFree0 + su]);
         if (l == m - 1) mma_commit(&bars[kBkupDone]);
         return true;
       };
@@ -556,11 +595,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // MMA-a of every direction, each followed by MMA-b/e of the direction before it
           ok = bwait(&bars[kKqFull], n & 1, lim, status, s_abort);
           for (int l = 0; l < m && ok; ++l) {
-            const int jj = j + l, s = jj & 1;
-            ok = bwait(&bars[kUgFull0 + s], (jj >> 1) & 1, lim, status, s_abort);
+            const int jj = j + l, s = jj & 1, su = jj % NU;
+            ok = bwait(&bars[kUFull0 + su], (jj / NU) & 1, lim, status, s_abort);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t aU = aUB0 + s * NA * kAtom64;
+            const uint32_t aU = aUB0 + su * NA * kAtom64;
 #pragma unroll
             for (int kk = 0; kk < 4 * NA; ++kk)
               mma_bf16(tmem + kRU + 64 * s, kdesc(aKQ, kk, kAtom128), kdesc(aU, kk, kAtom64),
@@ -745,6 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       kg_sync();
+      if (VW && kt == 0) mbar_arrive(&bars[kWsFree]);  // the inverse's scratch is free: this chunk's v may land
       // ---- Mqk T
       if (kt == 0) {
         tc_fence_after();
@@ -824,8 +864,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool srow = row < D;
     bool aborted = false;
     int j = 0;
-    // chunk 0's v tile (later chunks' arrive while the state MMAs of the chunk before run)
-    if (nchunks > 0 && !p.writes_off) {
+    // chunk 0's v tile (later chunks' arrive while the state MMAs of the chunk before run;
+    // with v in the [-W'; Q'] buffer, each chunk's is waited for in X0)
+    if (!VW && nchunks > 0 && !p.writes_off) {
       if (!wwait(&bars[kVFull], 0, lim, status, s_abort)) aborted = true;
     }
     for (int n = 0; n < nchunks && !aborted; ++n) {
@@ -884,11 +925,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nv = gt.nv;
       // ---- direction loop: the epilogue ([Bku_l; Mqu_l]) of every direction
       for (int l = 0; l < m; ++l, ++j) {
-        const int s = j & 1;
-        uint8_t* sP = sm + Ly::PB + s * NA * kAtom64;
-        uint8_t* sU = sm + Ly::UB + s * NA * kAtom64;
+        const int s = j & 1, su = j % NU;
+        uint8_t* sU = sm + Ly::UB + su * NA * kAtom64;
         uint8_t* sB = sBQ0 + s * kAtom128;
-        fail = !wwait(&bars[kUgFull0 + s], (j >> 1) & 1, lim, status, s_abort);
+        fail = !wwait(&bars[kUFull0 + su], (j / NU) & 1, lim, status, s_abort);
         if (fail) { aborted = true; break; }
         fail = !wwait(&bars[kRuFull0 + s], (j >> 1) & 1, lim, status, s_abort);
         if (fail) { aborted = true; break; }
@@ -951,8 +991,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- X0^T = beta V - (Bku P)^T -> BQ slot 0 (K-major rows c); ACC's Delta half zeroed
       if (!p.writes_off) {
       float x[32];  // beta_t v_t[c], read while the last direction's MMAs finish
+      if (VW) {
+        fail = !wwait(&bars[kVFull], n & 1, lim, status, s_abort);
+        if (fail) { aborted = true; break; }
+      }
       if (srow) {
-        const uint8_t* vcol = sVB + (row >> 6) * kAtomV;
+        const uint8_t* vcol = sVB + (row >> 6) * kAtom64;
 #pragma unroll
         for (int e4 = 0; e4 < 32; e4 += 4) {
           const float4 b4 = *reinterpret_cast<const float4*>(gt.beta + 32 * ch + e4);
@@ -960,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k2 = 0; k2 < 4; ++k2) {
             const int t = 32 * ch + e4 + k2;
-            const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vcol + sw128_offset(8 + t, row & 63, kAtomV)));
+            const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vcol + sw128_offset(t, row & 63, kAtom64)));
             x[e4 + k2] = bb[k2] * vv;
           }
         }
@@ -996,12 +1040,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bars[kX0Ready]);
-        mbar_arrive(&bars[kVFree]);
+        if (!VW) mbar_arrive(&bars[kVFree]);
       }
       }
       // ---- [-W'; Q'] -> WQ (Q' = e Q - Mqk W'): token rows, this warp's half of the columns
       fail = !wwait(&bars[kRwFull], n & 1, lim, status, s_abort);
       if (fail) { aborted = true; break; }
+      // with v in this buffer: every warp of the group has read it (X0Ready completes only
+      // when all eight have arrived; a bounded wait, like every other one)
+      if (VW && !p.writes_off) {
+        fail = !wwait(&bars[kX0Ready], n & 1, lim, status, s_abort);
+        if (fail) { aborted = true; break; }
+      }
       tc_fence_after();
       {
         const bool wrow = row < 64;
@@ -1038,7 +1088,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars[kKqFree]);
       }
       // the next chunk's v tile, loaded while MMA-c and MMA1 run
-      if (n + 1 < nchunks && !p.writes_off) {
+      if (!VW && n + 1 < nchunks && !p.writes_off) {
         fail = !wwait(&bars[kVFull], (n + 1) & 1, lim, status, s_abort);
         if (fail) { aborted = true; break; }
       }
@@ -1407,30 +1457,100 @@ size_t ptil_bytes(int B, int T, int H, int D, int L) {
   return (b + 255) & ~size_t(255);
 }
 
-template <int D, int CH>
+template <int D, int NU>
 cudaError_t set_smem_attr() {
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(prism_scan_kernel<D, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    Lay<D>::ALLOC);
+    attr_err = cudaFuncSetAttribute(prism_scan_kernel<D, NU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Lay<D, NU>::ALLOC);
   });
   return attr_err;
 }
 
+// The scan launches of one call (the residual write vectors are in the workspace): one
+// launch, two halves, or the segments' three launches and fold.  NU: U slots (3 when a
+// chunk has four or more residual directions, so that their loads run ahead).
+template <int D, int NU>
+cudaError_t launch_scans(const ScanParams& p, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
+                         const CUtensorMap& mu, const CUtensorMap& mv, const CUtensorMap& mg, int m,
+                         const TimeSplit& split,
+                         const std::function<cudaError_t(int, int, cudaStream_t, bool)>& residual) {
+  using Ly = Lay<D, NU>;
+  const cudaError_t attr_err = set_smem_attr<D, NU>();
+  if (attr_err != cudaSuccess) return attr_err;
+  const int NC = (p.T + kC - 1) / kC;
+  const SegPlan plan = plan_segments(p.B, p.T, p.H);
+  ScanArgs a{static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
+             static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha, p.conv_w, p.S0, p.lengths,
+             static_cast<__nv_bfloat16*>(p.o), p.S_final, nullptr, nullptr, p.B, p.T, p.H, p.W, m,
+             plan.P, plan.Ts, 0, 1, 0, -1, p.status, p.spin_limit};
+  const int grid = p.B * p.H * plan.P;
+  if (split.on) {
+    // the two halves as segments 0 and 1 of a 2-segment plan, one launch each; the first
+    // writes its end states to hand[b, h, 1], where the second reads its start states
+    float* hand = reinterpret_cast<float*>(static_cast<char*>(p.workspace) + ptil_bytes(p.B, p.T, p.H, D, p.L));
+    ScanArgs aA = a;
+    aA.P = 2;
+    aA.Ts = split.nA * kC;
+    aA.seg_only = 0;
+    aA.S_out = hand + (size_t)D * D;
+    ScanArgs aB = aA;
+    aB.seg_only = 1;
+    aB.S_out = nullptr;
+    aB.S_in = hand;
+    {
+      std::lock_guard<std::mutex> lock(g_side_mutex);
+      SideStreams* ss = nullptr;
+      cudaError_t e = side_streams(&ss);
+      if (e == cudaSuccess) e = cudaEventRecord(ss->forked, stream);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->hi, ss->forked, 0);
+      if (e != cudaSuccess) return e;
+      prism_scan_kernel<D, NU><<<p.B * p.H, kThreads, Ly::ALLOC, ss->hi>>>(mq, mk, mu, mv, mg, aA);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      if ((e = residual(split.nA, NC - split.nA, ss->hi, true)) != cudaSuccess) return e;
+      if ((e = cudaEventRecord(ss->joined, ss->hi)) != cudaSuccess) return e;
+      if ((e = cudaStreamWaitEvent(stream, ss->joined, 0)) != cudaSuccess) return e;
+    }
+    prism_scan_kernel<D, NU><<<p.B * p.H, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aB);
+    return cudaGetLastError();
+  }
+  if (plan.P == 1) {
+    prism_scan_kernel<D, NU><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, a);
+    return cudaGetLastError();
+  }
+  // a long sequence over few chains: P segments side by side, three scans and a fold
+  const size_t seg_states = (size_t)p.B * p.H * plan.P * D * D;
+  float* wsN = reinterpret_cast<float*>(static_cast<char*>(p.workspace) + ptil_bytes(p.B, p.T, p.H, D, p.L));
+  float* wsM = wsN + seg_states;
+  float* wsS = wsM + seg_states;
+  ScanArgs aN = a;  // each segment from a zero start (the first from S0): N_p
+  aN.S_out = wsN;
+  aN.write_o = 0;
+  aN.S_final = nullptr;
+  prism_scan_kernel<D, NU><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aN);
+  ScanArgs aM = aN;  // the transitions alone from the identity: M_p
+  aM.S_out = wsM;
+  aM.s_in_identity = 1;
+  aM.writes_off = 1;
+  aM.m = 0;
+  prism_scan_kernel<D, NU><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aM);
+  segment_fold_kernel<D><<<dim3(D, p.B * p.H), D, 0, stream>>>(wsN, wsM, wsS, plan.P);
+  ScanArgs aF = a;  // every segment again from its exact start state: o and S_final
+  aF.S_in = wsS;
+  prism_scan_kernel<D, NU><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aF);
+  return cudaGetLastError();
+}
+
 template <int D, int CH>
 cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
-  using Ly = Lay<D>;
-  cudaError_t attr_err = set_smem_attr<D, CH>();
-  if (attr_err == cudaSuccess && CH != PRISM_CHAIN_LINEAR) attr_err = set_smem_attr<D, PRISM_CHAIN_LINEAR>();
-  if (attr_err != cudaSuccess) return attr_err;
   const cuuint64_t B = p.B, T = p.T, H = p.H;
   const int m = p.L - 1;
   CUtensorMap mq, mk, mu, mv, mg;
   const cuuint64_t dims4[4] = {(cuuint64_t)D, H, T, B};
   const cuuint64_t str4[3] = {(cuuint64_t)D * 2, H * D * 2, T * H * D * 2};
   const cuuint32_t box4[4] = {64, 1, 64, 1};
-  const cuuint32_t box_v[4] = {64, 1, 72, 1};  // a chunk's v rows and 8 rows of ShortConv history
+  const cuuint32_t box_v[4] = {64, 1, 64, 1};
   if (!encode(&mq, p.q, 4, dims4, str4, box4) || !encode(&mk, p.k, 4, dims4, str4, box4) ||
       !encode(&mv, p.v, 4, dims4, str4, box_v))
     return cudaErrorInvalidValue;
@@ -1474,66 +1594,8 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
     mu = mk;
     mg = mk;
   }
-  const SegPlan plan = plan_segments(p.B, p.T, p.H);
-  ScanArgs a{static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
-             static_cast<const __nv_bfloat16*>(p.v), p.gamma, p.beta, p.alpha, p.conv_w, p.S0, p.lengths,
-             static_cast<__nv_bfloat16*>(p.o), p.S_final, nullptr, nullptr, p.B, p.T, p.H, p.W, m,
-             plan.P, plan.Ts, 0, 1, 0, -1, p.status, p.spin_limit};
-  const int grid = p.B * p.H * plan.P;
-  if (split.on) {
-    // the two halves as segments 0 and 1 of a 2-segment plan, one launch each; the first
-    // writes its end states to hand[b, h, 1], where the second reads its start states
-    float* hand = reinterpret_cast<float*>(static_cast<char*>(p.workspace) + ptil_bytes(p.B, p.T, p.H, D, p.L));
-    ScanArgs aA = a;
-    aA.P = 2;
-    aA.Ts = split.nA * kC;
-    aA.seg_only = 0;
-    aA.S_out = hand + (size_t)D * D;
-    ScanArgs aB = aA;
-    aB.seg_only = 1;
-    aB.S_out = nullptr;
-    aB.S_in = hand;
-    {
-      std::lock_guard<std::mutex> lock(g_side_mutex);
-      SideStreams* ss = nullptr;
-      cudaError_t e = side_streams(&ss);
-      if (e == cudaSuccess) e = cudaEventRecord(ss->forked, stream);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->hi, ss->forked, 0);
-      if (e != cudaSuccess) return e;
-      prism_scan_kernel<D, CH><<<p.B * p.H, kThreads, Ly::ALLOC, ss->hi>>>(mq, mk, mu, mv, mg, aA);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      if ((e = residual(split.nA, NC - split.nA, ss->hi, true)) != cudaSuccess) return e;
-      if ((e = cudaEventRecord(ss->joined, ss->hi)) != cudaSuccess) return e;
-      if ((e = cudaStreamWaitEvent(stream, ss->joined, 0)) != cudaSuccess) return e;
-    }
-    prism_scan_kernel<D, CH><<<p.B * p.H, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aB);
-    return cudaGetLastError();
-  }
-  if (plan.P == 1) {
-    prism_scan_kernel<D, CH><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, a);
-    return cudaGetLastError();
-  }
-  // a long sequence over few chains: P segments side by side, three scans and a fold
-  const size_t seg_states = (size_t)p.B * p.H * plan.P * D * D;
-  float* wsN = reinterpret_cast<float*>(static_cast<char*>(p.workspace) + ptil_bytes(p.B, p.T, p.H, D, p.L));
-  float* wsM = wsN + seg_states;
-  float* wsS = wsM + seg_states;
-  ScanArgs aN = a;  // each segment from a zero start (the first from S0): N_p
-  aN.S_out = wsN;
-  aN.write_o = 0;
-  aN.S_final = nullptr;
-  prism_scan_kernel<D, CH><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aN);
-  ScanArgs aM = aN;  // the transitions alone from the identity: M_p
-  aM.S_out = wsM;
-  aM.s_in_identity = 1;
-  aM.writes_off = 1;
-  aM.m = 0;
-  prism_scan_kernel<D, PRISM_CHAIN_LINEAR><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aM);
-  segment_fold_kernel<D><<<dim3(D, p.B * p.H), D, 0, stream>>>(wsN, wsM, wsS, plan.P);
-  ScanArgs aF = a;  // every segment again from its exact start state: o and S_final
-  aF.S_in = wsS;
-  prism_scan_kernel<D, CH><<<grid, kThreads, Ly::ALLOC, stream>>>(mq, mk, mu, mv, mg, aF);
-  return cudaGetLastError();
+  if (m >= 4) return launch_scans<D, 3>(p, stream, mq, mk, mu, mv, mg, m, split, residual);
+  return launch_scans<D, 2>(p, stream, mq, mk, mu, mv, mg, m, split, residual);
 }
 
 template <int D>
