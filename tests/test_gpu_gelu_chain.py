@@ -23,9 +23,13 @@ CASES = {
     "lm_130m": W["lm_130m"].replace(B=2, T=200, H=3, with_s0=True),
     # tcgen05 chunk kernel at d = 64 with right-padded rows
     "recsys": W["recsys"].replace(B=5, T=260, lengths_lo=30),
-    # token-by-token kernel: fp32 and a long chain (L = 8)
+    # token-by-token kernel: fp32
     "lm_fp32": W["lm_130m"].replace(B=1, T=130, H=2, dtype="fp32"),
+    # tcgen05 chunk kernel with seven residual directions (three U slots)
     "long_ctx": W["long_ctx"].replace(T=150, H=2),
+    # three U slots in the two-halves scan (11 chunks), W = 8, ragged rows
+    "many_dirs_ragged": synth.Workload("mdr", B=4, T=700, H=2, d_k=64, d_v=64, L=6, chunk=64, W=8,
+                                       lengths_lo=100, with_s0=True),
     "d32_L16_W8": synth.Workload("d32", B=2, T=97, H=3, d_k=32, d_v=32, L=16, chunk=32, W=8),
 }
 
