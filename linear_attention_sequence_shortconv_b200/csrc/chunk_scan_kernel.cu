@@ -219,6 +219,14 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk, uint32_t atom_s
 __device__ __forceinline__ uint64_t mndesc(uint32_t base, int kk, uint32_t lbo) {
   return sdesc_sw128(base + (uint32_t)kk * 2048u, lbo, 1024);
 }
+// The same descriptors for K step kk from the step-0 descriptor: only the 14-bit start
+// address field (address / 16, bits 0-13) changes, and every address stays inside shared
+// memory, so the field never carries into the others.  Saves the issuing thread the full
+// descriptor arithmetic per MMA.
+__device__ __forceinline__ uint64_t kdesc_step(uint64_t d0, int kk, uint32_t atom_stride) {
+  return d0 + (((uint32_t)(kk >> 2) * atom_stride + (uint32_t)(kk & 3) * 32u) >> 4);
+}
+__device__ __forceinline__ uint64_t mndesc_step(uint64_t d0, int kk) { return d0 + (uint64_t)kk * 128u; }
 
 // ---------------------------------------------------------------- barriers and waits
 __device__ __forceinline__ void kg_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
@@ -578,13 +586,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (l == 0 && !bwait(&bars[kE1Done], n & 1, lim, status, s_abort)) return false;
         tc_fence_after();
         const uint32_t aP = aPB0 + s * NA * kAtom64, aU = aUB0 + su * NA * kAtom64, aB = aBQ0 + s * kAtom128;
+        const uint64_t dP = mndesc(aP, 0, kAtom64), dB = kdesc(aB, 0, kAtom128), dU = mndesc(aU, 0, kAtom64);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kACC, mndesc(aP, kk, kAtom64), kdesc(aB, kk, kAtom128), idesc_bf16(128, 128, 1, 0),
+          mma_bf16(tmem + kACC, mndesc_step(dP, kk), kdesc_step(dB, kk, kAtom128), idesc_bf16(128, 128, 1, 0),
                    (l > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kRS, mndesc(aP, kk, kAtom64), mndesc(aU, kk, kAtom64), idesc_bf16(128, D, 1, 1), 1);
+          mma_bf16(tmem + kRS, mndesc_step(dP, kk), mndesc_step(dU, kk), idesc_bf16(128, D, 1, 1), 1);
         if (NU == 3) mma_commit(&bars[kPFree0 + s]);
         mma_commit(&bars[kUFree0 + su]);
         if (l == m - 1) mma_commit(&bars[kBkupDone]);
@@ -599,10 +608,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = bwait(&bars[kUFull0 + su], (jj / NU) & 1, lim, status, s_abort);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t aU = aUB0 + su * NA * kAtom64;
+            const uint64_t dKQ = kdesc(aKQ, 0, kAtom128), dU = kdesc(aUB0 + su * NA * kAtom64, 0, kAtom64);
 #pragma unroll
             for (int kk = 0; kk < 4 * NA; ++kk)
-              mma_bf16(tmem + kRU + 64 * s, kdesc(aKQ, kk, kAtom128), kdesc(aU, kk, kAtom64),
+              mma_bf16(tmem + kRU + 64 * s, kdesc_step(dKQ, kk, kAtom128), kdesc_step(dU, kk, kAtom64),
                        idesc_bf16(128, 64, 0, 0), kk > 0);
             mma_commit(&bars[kRuFull0 + s]);
             if (l == m - 1) mma_commit(&bars[kKqkFree]);
@@ -618,19 +627,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = bwait(&bars[kX0Ready], n & 1, lim, status, s_abort) && bwait(&bars[kZReady], n & 1, lim, status, s_abort);
           if (ok) {
             tc_fence_after();
+            const uint64_t dX = kdesc(aBQ0, 0, kAtom128), dZ = kdesc(aZB, 0, kAtom128);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tmem + kACC, kdesc(aBQ0, kk, kAtom128), kdesc(aZB, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
-                       (m > 0 || kk > 0) ? 1u : 0u);
+              mma_bf16(tmem + kACC, kdesc_step(dX, kk, kAtom128), kdesc_step(dZ, kk, kAtom128),
+                       idesc_bf16(128, 128, 0, 0), (m > 0 || kk > 0) ? 1u : 0u);
           }
         }
         // MMA1: S_n x [-W';Q']^T onto ACC
         if (ok) ok = bwait(&bars[kWqReady], n & 1, lim, status, s_abort);
         if (ok) {
           tc_fence_after();
+          const uint64_t dW = kdesc(aWQ, 0, kAtom128);
 #pragma unroll
           for (int kk = 0; kk < 4 * NA; ++kk)
-            mma_ts(tmem + kACC, tmem + kSB + 8 * kk, kdesc(aWQ, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
+            mma_ts(tmem + kACC, tmem + kSB + 8 * kk, kdesc_step(dW, kk, kAtom128), idesc_bf16(128, 128, 0, 0),
                    (!p.writes_off || kk > 0) ? 1u : 0u);
           mma_commit(&bars[kAccFull]);
         }
@@ -638,9 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = bwait(&bars[kDlReady], n & 1, lim, status, s_abort) && bwait(&bars[kKbFull], n & 1, lim, status, s_abort);
         if (ok) {
           tc_fence_after();
+          const uint64_t dK = mndesc(aKB, 0, kAtom64);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + kRS, tmem + kSB + 8 * kk, mndesc(aKB, kk, kAtom64), idesc_bf16(128, D, 0, 1), 1);
+            mma_ts(tmem + kRS, tmem + kSB + 8 * kk, mndesc_step(dK, kk), idesc_bf16(128, D, 0, 1), 1);
           mma_commit(&bars[kRsFull]);
         }
       }
@@ -714,9 +726,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kg_sync_or(fail)) break;
       if (kt == 0) {
         tc_fence_after();
+        const uint64_t dKQ = kdesc(aKQ, 0, kAtom128);
 #pragma unroll
         for (int kk = 0; kk < 4 * NA; ++kk) {
-          const uint64_t a = kdesc(aKQ, kk, kAtom128);
+          const uint64_t a = kdesc_step(dKQ, kk, kAtom128);
           mma_bf16(tmem + kRKQ, a, a, idesc_bf16(128, 64, 0, 0), kk > 0);
         }
         mma_commit(&bars[kKgMma]);
@@ -788,9 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- Mqk T
       if (kt == 0) {
         tc_fence_after();
+        const uint64_t dZk = kdesc(aZB, 0, kAtom128), dZm = mndesc(aZB, 0, kAtom128);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kRKQ, kdesc(aZB, kk, kAtom128), mndesc(aZB, kk, kAtom128), idesc_bf16(128, 64, 0, 1),
+          mma_bf16(tmem + kRKQ, kdesc_step(dZk, kk, kAtom128), mndesc_step(dZm, kk), idesc_bf16(128, 64, 0, 1),
                    kk > 0);
         mma_commit(&bars[kKgMma]);
       }
@@ -834,9 +848,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- [W'; Mqk W'] = [T; MqkT] K^ into RW; the epilogue group turns it into [-W'; Q']
       if (kt == 0) {
         tc_fence_after();
+        const uint64_t dZk = kdesc(aZB, 0, kAtom128), dKm = mndesc(aKQ, 0, kAtom128);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kRW, kdesc(aZB, kk, kAtom128), mndesc(aKQ, kk, kAtom128), idesc_bf16(128, D, 0, 1),
+          mma_bf16(tmem + kRW, kdesc_step(dZk, kk, kAtom128), mndesc_step(dKm, kk), idesc_bf16(128, D, 0, 1),
                    kk > 0);
         mma_commit(&bars[kRwFull]);
       }
