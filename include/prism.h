@@ -105,9 +105,10 @@ enum prism_status {
  *
  * chunk: chunk length of the chunkwise-parallel evaluation, a power of two in
  *   [16, 64].  The result does not depend on it beyond rounding.  The bf16
- *   tensor-core path runs chunk == 64 with d_k == d_v in {64, 128}; every other
- *   supported shape runs the fp32 CUDA-core path, which evaluates the recurrence
- *   token by token.
+ *   tensor-core path runs chunk == 64 with d_k == d_v in {64, 128}.  fp32 with
+ *   d_k == d_v in {16, 32, 64} runs the same chunk decomposition in fp32 FMAs on
+ *   CUDA cores (one launch, chunk length `chunk`).  Every other supported shape runs
+ *   the fp32 CUDA-core path that evaluates the recurrence token by token.
  * workspace / workspace_bytes: device scratch of at least
  *   prism_scan_fwd_workspace_size(...) bytes (may be NULL when that is 0), 16-byte
  *   aligned, owned by the caller, contents undefined on return.  The tensor-core
@@ -116,8 +117,8 @@ enum prism_status {
  *   bf16 in the layout of gain (B * T * H * (L - 1) * d_v * 2 bytes, rounded up to
  *   256); a sequence cut into segments (long sequences over few (batch row, head)
  *   chains) adds three fp32 d_v x d_k states per segment, and a scan run in two halves
- *   (chains that leave SMs idle) adds two fp32 d_v x d_k states per chain.  The token-by-token path
- *   needs none.  Too small or NULL: PRISM_ERR_WORKSPACE, before any launch.
+ *   (chains that leave SMs idle) adds two fp32 d_v x d_k states per chain.  The CUDA-core paths
+ *   need none.  Too small or NULL: PRISM_ERR_WORKSPACE, before any launch.
  * Errors: PRISM_ERR_INVALID_ARG, PRISM_ERR_UNSUPPORTED, PRISM_ERR_WORKSPACE,
  *   PRISM_ERR_CUDA, as described above.
  */
@@ -286,8 +287,8 @@ int prism_prologue_fwd(const void* v, const float* alpha, const void* gain,
                        float* rho_out, prism_stream_t stream);
 
 /* 1 if prism_scan_fwd runs these sizes on the tcgen05 tensor-core chunk
- * kernel, 0 if on the CUDA-core token-by-token kernel (sizes as for
- * prism_scan_fwd; unsupported sizes also give 0). */
+ * kernel, 0 if on a CUDA-core kernel (the fp32 chunk form or token by token;
+ * sizes as for prism_scan_fwd; unsupported sizes also give 0). */
 int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype);
 
 /* Number of kernel launches one prism_scan_fwd call with these sizes issues (0 for

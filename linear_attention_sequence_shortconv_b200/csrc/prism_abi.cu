@@ -14,6 +14,8 @@ bool chunk_scan_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
 cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream);
 size_t chunk_scan_workspace_bytes(int B, int T, int H, int D, int L);
 int chunk_scan_launches(int B, int T, int H, int L);
+bool chunk_fp32_supported(int d_k, int d_v, int chunk, int dtype);
+cudaError_t launch_chunk_fp32(const ScanParams& p, cudaStream_t stream);
 cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t stream);
 cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, cudaStream_t stream);
 size_t bwd_smem_bytes(int d_k, int d_v, int L);
@@ -167,7 +169,9 @@ int prism_scan_fwd_ex(const void* q, const void* k, const void* v, const float* 
   if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype)) {
     if (L > 1) p.split_event = g_split_event.exchange(nullptr);
     err = prism::launch_chunk_scan(p, s);
-  } else
+  } else if (prism::chunk_fp32_supported(d_k, d_v, chunk, dtype))
+    err = prism::launch_chunk_fp32(p, s);
+  else
     err = prism::launch_recurrent_scan(p, dtype, s);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }

@@ -50,9 +50,11 @@ def test_split_bf16_wide_window():
     assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= 2e-2
 
 
-def test_split_fp32_token_path_gelu():
-    """fp32 (the token-by-token kernel), exact GELU chain."""
-    w = synth.Workload("cs_fp32", B=3, T=150, H=2, d_k=64, d_v=64, L=3, chunk=64, W=4, dtype="fp32",
+@pytest.mark.parametrize("d", [64, 128])
+def test_split_fp32_gelu(d):
+    """fp32, exact GELU chain: the fp32 chunk-form kernel (d = 64) and the token-by-token
+    kernel (d = 128)."""
+    w = synth.Workload("cs_fp32", B=3, T=150, H=2, d_k=d, d_v=d, L=3, chunk=64, W=4, dtype="fp32",
                        with_s0=True, seed=53)
     o, S, o_ref, S_ref = _two_calls(w, 61, chain="gelu")
     assert max_abs_rel_err(o, o_ref) <= 1e-4

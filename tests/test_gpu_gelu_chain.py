@@ -23,8 +23,10 @@ CASES = {
     "lm_130m": W["lm_130m"].replace(B=2, T=200, H=3, with_s0=True),
     # tcgen05 chunk kernel at d = 64 with right-padded rows
     "recsys": W["recsys"].replace(B=5, T=260, lengths_lo=30),
-    # token-by-token kernel: fp32
+    # token-by-token kernel: fp32 at d = 128
     "lm_fp32": W["lm_130m"].replace(B=1, T=130, H=2, dtype="fp32"),
+    # fp32 chunk-form kernel: d = 64, several chunks and ragged rows
+    "recsys_fp32": W["recsys"].replace(B=3, T=200, lengths_lo=30, dtype="fp32"),
     # tcgen05 chunk kernel with seven residual directions (three U slots)
     "long_ctx": W["long_ctx"].replace(T=150, H=2),
     # three U slots in the two-halves scan (11 chunks), W = 8, ragged rows
@@ -56,7 +58,7 @@ def test_gelu_chain_parity(name):
             assert np.all(o[b, n:] == 0)
 
 
-@pytest.mark.parametrize("name", ["lm_130m", "lm_fp32"])
+@pytest.mark.parametrize("name", ["lm_130m", "lm_fp32", "recsys_fp32"])
 def test_gelu_chain_parity_wide_predictor(name):
     w = CASES[name]
     inp = _wide_gain(synth.make_inputs(w), w)
