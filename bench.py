@@ -414,6 +414,7 @@ def run_ours(args, w):
     use_tc = prism.uses_tensor_cores(w.d_k, w.d_v, w.L, w.W, w.chunk, dtype_code)
     split = use_tc and w.L > 1
     launches_per_step = prism.scan_fwd_launches(w.B, w.T, w.H, w.d_k, w.d_v, w.L, w.W, w.chunk, dtype_code)
+    first_chunks = prism.scan_fwd_split_chunks(w.B, w.T, w.H, w.d_k, w.d_v, w.L, w.W, w.chunk, dtype_code)
     mids = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if split else []
     for e in mids:
         e.record(stream)  # creates the event; the call below records it again
@@ -498,12 +499,12 @@ def run_ours(args, w):
     path["roofline_frac"] = path["roofline_time_us"] / path["us"]
     if split:
         # with the scan in two halves (four launches) the first residual-write launch covers
-        # the first half's chunks, and the second half's residual write runs beside the
-        # first scan launch: its bytes count in the scan's window
+        # the first launch's chunks (first_chunks of nc), and the second half's residual
+        # write runs beside the first scan launch: its bytes count in the scan's window
         sw = algorithmic_work_split(w, lens_np)
         nc = -(-w.T // w.chunk)
         halves = launches_per_step == 4
-        f_first = ((nc + 1) // 2) / nc if halves else 1.0
+        f_first = first_chunks / nc if halves else 1.0
         rw_first = sw["residual_write"] * f_first
         scan_bytes = sw["scan"] + sw["residual_write"] * (1.0 - f_first)
         scan_gbs = scan_bytes / (scan_ms / 1e3) / 1e9

@@ -298,8 +298,17 @@ int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, 
  * a B200's SMs idle, L > 1 and the sequence has at least 8 chunks, four: the scan runs
  * in two halves, and the second half's residual write runs beside the first half's
  * scan (on an internal stream of the device, forked from and joined back into the
- * call's stream).  Token-by-token path: 1. */
+ * call's stream).  CUDA-core paths: 1. */
 int prism_scan_fwd_launches(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype);
+
+/* Chunks (of 64 tokens) in the first of the two scan launches when prism_scan_fwd runs
+ * these sizes in two halves (see prism_scan_fwd_launches); 0 when it does not, or for
+ * invalid sizes.  The cut is placed so that the second half's residual write, on the SMs
+ * the chains leave idle, ends about when the first scan does: with x = 0.28 chains /
+ * idle SMs, ceil(NC x / (1 + x)) chunks, clamped to [ceil(NC / 4), NC - 1] (11 of 32 for
+ * the 130M-LM layer, B=16 T=2048 H=6).  A measurement aid; results do not depend on it
+ * beyond rounding. */
+int prism_scan_fwd_split_chunks(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype);
 
 /* prism_prologue_fwd with the residual chain selected by `chain` (see prism_scan_fwd_ex). */
 int prism_prologue_fwd_ex(const void* v, const float* alpha, const void* gain,

@@ -25,6 +25,7 @@ from ._lib import (  # noqa: F401
     stream_status,
     uses_tensor_cores,
     scan_fwd_launches,
+    scan_fwd_split_chunks,
     set_split_event,
     version,
     workspace_size,

@@ -44,6 +44,7 @@ EXPORTS = (
     "prism_state_affine",
     "prism_scan_fwd_uses_tensor_cores",
     "prism_scan_fwd_launches",
+    "prism_scan_fwd_split_chunks",
     "prism_stream_status",
     "prism_set_spin_limit",
     "prism_set_split_event",
@@ -101,6 +102,8 @@ def lib() -> ctypes.CDLL:
     L.prism_scan_fwd_uses_tensor_cores.restype = ci
     L.prism_scan_fwd_launches.argtypes = [ci] * 9
     L.prism_scan_fwd_launches.restype = ci
+    L.prism_scan_fwd_split_chunks.argtypes = [ci] * 9
+    L.prism_scan_fwd_split_chunks.restype = ci
     L.prism_stream_status.argtypes = [vp]
     L.prism_stream_status.restype = ci
     L.prism_set_spin_limit.argtypes = [ctypes.c_longlong]
@@ -451,6 +454,11 @@ def uses_tensor_cores(d_k, d_v, L, W, chunk, dtype_code) -> bool:
 def scan_fwd_launches(B, T, H, d_k, d_v, L, W, chunk, dtype_code) -> int:
     """Kernel launches one prism_scan_fwd call with these sizes issues."""
     return int(lib().prism_scan_fwd_launches(B, T, H, d_k, d_v, L, W, chunk, dtype_code))
+
+
+def scan_fwd_split_chunks(B, T, H, d_k, d_v, L, W, chunk, dtype_code) -> int:
+    """Chunks in the first scan launch when the forward runs in two halves, else 0."""
+    return int(lib().prism_scan_fwd_split_chunks(B, T, H, d_k, d_v, L, W, chunk, dtype_code))
 
 
 def set_split_event(event) -> None:

@@ -55,6 +55,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cmath>
 #include <functional>
 #include <mutex>
 
@@ -111,7 +112,8 @@ struct Lay {
 };
 
 // One launch of the scan kernel.  A sequence may be cut into P segments of Ts tokens
-// (Ts a multiple of 64), one CTA each; CTA (b, h, p) scans tokens [p Ts, min((p+1) Ts, len)).
+// (Ts a multiple of 64), one CTA each; CTA (b, h, p) scans tokens [p Ts, min((p+1) Ts, len)),
+// the last segment up to len (the two halves in time have a shorter first segment).
 // Its start state is S0 (p = 0), else the identity (s_in_identity), else S_in[b, h, p],
 // else zero; its end state goes to S_out[b, h, p] when S_out is set, else to S_final from
 // the last segment.  writes_off treats v and the residual writes as zero (the transitions
@@ -413,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int T = p.T, H = p.H, m = p.m;
   const int len = p.lengths ? min(max(p.lengths[b], 0), T) : T;
   const int tok0 = seg * p.Ts;                         // first token of this CTA's segment
-  const int seg_end = min(tok0 + p.Ts, T);             // end of the segment
+  const int seg_end = seg == p.P - 1 ? T : min(tok0 + p.Ts, T);  // end of the segment (the last: T)
   const int vend = min(len, seg_end);                  // end of its valid tokens
   const int nchunks = vend > tok0 ? (vend - tok0 + kC - 1) / kC : 0;
   const long long lim = p.spin_limit;
@@ -1422,8 +1424,14 @@ SegPlan plan_segments(int B, int T, int H) {
 // the sequence is not cut into segments), the scan runs in two launches: chunks
 // [0, nA), then chunks [nA, NC) from the first launch's end states.  The residual write
 // of the second half runs beside the first scan launch, on the SMs that launch leaves
-// idle, so only the first half's residual write precedes the scan.
+// idle, so only the first half's residual write precedes the scan.  The first launch is
+// cut where that write should end about when the first scan does.  On the idle SMs the
+// write of one chunk of every chain takes about x = 0.28 chains / idle SMs chunk times of
+// the scan, so nA = NC x / (1 + x), at least a quarter of the chunks.  The constant is
+// measured on the 130M-LM layer (96 chains): its step time is lowest at nA = 11 of 32
+// chunks (x = 0.52), 2% below nA = 16, and within 1% from 10 to 13.
 constexpr int kSplitIdleSMs = 24;  // SMs the chains must leave idle
+constexpr double kSplitWriteCost = 0.28;
 struct TimeSplit {
   bool on;
   int nA;  // chunks of the first half
@@ -1431,7 +1439,10 @@ struct TimeSplit {
 TimeSplit time_split(int B, int T, int H, int L) {
   const int nc = (T + kC - 1) / kC;
   const bool on = L > 1 && plan_segments(B, T, H).P == 1 && B * H + kSplitIdleSMs <= kPlanSMs && nc >= 8;
-  return {on, (nc + 1) / 2};
+  const int chains = B * H, idle = std::max(kPlanSMs - chains, 1);
+  const double x = kSplitWriteCost * chains / idle;
+  const int nA = (int)std::ceil(nc * x / (1.0 + x));
+  return {on, std::max((nc + 3) / 4, std::min(nc - 1, nA))};
 }
 
 // The side stream of a device for the two halves: the first scan launch, then the second
@@ -1631,6 +1642,11 @@ size_t chunk_scan_workspace_bytes(int B, int T, int H, int D, int L) {
   const size_t states = plan.P > 1 ? 3 * (size_t)B * H * plan.P * D * D
                                    : (time_split(B, T, H, L).on ? 2 * (size_t)B * H * D * D : 0);
   return ptil_bytes(B, T, H, D, L) + states * sizeof(float);
+}
+
+int chunk_scan_split_chunks(int B, int T, int H, int L) {
+  const TimeSplit s = time_split(B, T, H, L);
+  return s.on ? s.nA : 0;
 }
 
 int chunk_scan_launches(int B, int T, int H, int L) {

@@ -14,6 +14,7 @@ bool chunk_scan_supported(int d_k, int d_v, int L, int W, int chunk, int dtype);
 cudaError_t launch_chunk_scan(const ScanParams& p, cudaStream_t stream);
 size_t chunk_scan_workspace_bytes(int B, int T, int H, int D, int L);
 int chunk_scan_launches(int B, int T, int H, int L);
+int chunk_scan_split_chunks(int B, int T, int H, int L);
 bool chunk_fp32_supported(int d_k, int d_v, int chunk, int dtype);
 cudaError_t launch_chunk_fp32(const ScanParams& p, cudaStream_t stream);
 cudaError_t launch_decode_step(const DecodeParams& p, int dtype, cudaStream_t stream);
@@ -252,6 +253,12 @@ int prism_scan_fwd_launches(int B, int T, int H, int d_k, int d_v, int L, int W,
   if (check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype) != PRISM_OK) return 0;
   if (prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype)) return prism::chunk_scan_launches(B, T, H, L);
   return 1;
+}
+
+int prism_scan_fwd_split_chunks(int B, int T, int H, int d_k, int d_v, int L, int W, int chunk, int dtype) {
+  if (check_sizes(B, T, H, d_k, d_v, L, W, chunk, dtype) != PRISM_OK) return 0;
+  if (!prism::chunk_scan_supported(d_k, d_v, L, W, chunk, dtype)) return 0;
+  return prism::chunk_scan_split_chunks(B, T, H, L);
 }
 
 int prism_scan_fwd_uses_tensor_cores(int d_k, int d_v, int L, int W, int chunk, int dtype) {

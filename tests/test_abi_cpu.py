@@ -132,6 +132,29 @@ def test_launch_count_query(L):
     assert prism.scan_fwd_launches(0, 2048, 6, 128, 128, 4, 4, 64, 0) == 0
 
 
+def test_split_point_query():
+    # the first of the two halves ends where the second half's residual write (on the SMs
+    # the chains leave idle) should end about when the first scan does: x = 0.28 chains /
+    # idle SMs, ceil(NC x / (1 + x)) chunks, clamped to [ceil(NC / 4), NC - 1]
+    import math
+
+    def model(B, T, H):
+        nc, chains = -(-T // 64), B * H
+        x = 0.28 * chains / (148 - chains)
+        return max(-(-nc // 4), min(nc - 1, math.ceil(nc * x / (1 + x))))
+
+    assert prism.scan_fwd_split_chunks(16, 2048, 6, 128, 128, 4, 4, 64, 0) == 11 == model(16, 2048, 6)
+    assert prism.scan_fwd_split_chunks(31, 2048, 4, 64, 64, 3, 4, 64, 0) == model(31, 2048, 4) > 16
+    assert prism.scan_fwd_split_chunks(1, 700, 4, 64, 64, 6, 8, 64, 0) == 3  # a quarter of 11 chunks
+    for args in ((128, 1024, 2, 64, 64, 4, 4, 64, 0),      # more chains than idle SMs allow
+                 (16, 448, 6, 128, 128, 4, 4, 64, 0),      # under 8 chunks
+                 (16, 2048, 6, 128, 128, 1, 4, 64, 0),     # L = 1
+                 (1, 65536, 8, 128, 128, 8, 4, 64, 0),     # cut into segments
+                 (16, 2048, 6, 64, 64, 4, 4, 64, 1),       # fp32: a CUDA-core path
+                 (0, 2048, 6, 128, 128, 4, 4, 64, 0)):     # invalid
+        assert prism.scan_fwd_split_chunks(*args) == 0
+
+
 def test_segment_states_stay_within_148_chains(L):
     # chains x segments never exceeds 148, so the segment (or hand-over) states never need
     # more than 3 x 148 x 128^2 fp32 beyond the residual write vectors
