@@ -90,7 +90,9 @@ enum prism_status {
   PRISM_ERR_UNSUPPORTED = 2, /* valid but not implemented: head size, width, alignment, device */
   PRISM_ERR_WORKSPACE = 3,   /* workspace smaller than prism_scan_fwd_workspace_size() */
   PRISM_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
-  PRISM_ERR_TIMEOUT = 5      /* a bounded device-side wait expired (from prism_stream_status) */
+  PRISM_ERR_TIMEOUT = 5,     /* a bounded device-side wait expired (from prism_stream_status) */
+  PRISM_ERR_BOUNDS = 6       /* debug build only: a kernel computed an index outside its buffer
+                                and skipped the access (from prism_stream_status) */
 };
 
 /* Limits of this build (checked; larger values return PRISM_ERR_UNSUPPORTED). */
@@ -355,8 +357,8 @@ int prism_decode_step(const void* q, const void* k, const void* v,
                       void* o, prism_stream_t stream);
 
 /* Synchronises `stream`, then returns and clears the device status word of the
- * current device: PRISM_OK, PRISM_ERR_TIMEOUT, or PRISM_ERR_CUDA if the
- * synchronisation itself failed. */
+ * current device: PRISM_OK, PRISM_ERR_TIMEOUT, PRISM_ERR_BOUNDS (debug build only), or
+ * PRISM_ERR_CUDA if the synchronisation itself failed. */
 int prism_stream_status(prism_stream_t stream);
 
 /* Test hook: the spin limit of the device-side bounded waits (0 restores the
@@ -376,6 +378,20 @@ const char* prism_status_string(int code);
 
 /* (major << 16) | (minor << 8) | patch */
 int prism_version(void);
+
+/* 1 in the debug build of this library (libprism_debug.so, compiled with
+ * PRISM_DEBUG_BOUNDS), 0 in the release build (libprism.so).  Both export the same
+ * functions and compute the same results bit for bit.  In the debug build the kernels
+ * check the global indices they compute against the extents of their buffers (and the
+ * innermost coordinate of every TMA copy against the 16-byte rule); a failed check
+ * records PRISM_ERR_BOUNDS in the device status word and skips the access. */
+int prism_debug_bounds(void);
+
+/* Test hook of the debug build: one launch on `stream` that runs the device-side check
+ * of index i against extent n (no memory is accessed at that index), so that
+ * prism_stream_status then reports PRISM_ERR_BOUNDS exactly when i is outside [0, n).
+ * PRISM_ERR_UNSUPPORTED in the release build; PRISM_ERR_CUDA if the launch fails. */
+int prism_debug_bounds_probe(long long i, long long n, prism_stream_t stream);
 
 #ifdef __cplusplus
 }

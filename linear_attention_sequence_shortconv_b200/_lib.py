@@ -14,7 +14,9 @@ from typing import Optional, Tuple
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libprism.so")
+# PRISM_DEBUG_BOUNDS=1 in the environment loads the debug build (bounds-checked kernels)
+DEBUG_BOUNDS = os.environ.get("PRISM_DEBUG_BOUNDS", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libprism_debug.so" if DEBUG_BOUNDS else "libprism.so")
 
 PRISM_BF16 = 0
 PRISM_FP32 = 1
@@ -27,6 +29,7 @@ STATUS = {
     3: "PRISM_ERR_WORKSPACE",
     4: "PRISM_ERR_CUDA",
     5: "PRISM_ERR_TIMEOUT",
+    6: "PRISM_ERR_BOUNDS",
 }
 
 # Every symbol include/prism.h declares.
@@ -50,6 +53,8 @@ EXPORTS = (
     "prism_set_split_event",
     "prism_status_string",
     "prism_version",
+    "prism_debug_bounds",
+    "prism_debug_bounds_probe",
 )
 
 
@@ -114,6 +119,10 @@ def lib() -> ctypes.CDLL:
     L.prism_status_string.restype = ctypes.c_char_p
     L.prism_version.argtypes = []
     L.prism_version.restype = ci
+    L.prism_debug_bounds.argtypes = []
+    L.prism_debug_bounds.restype = ci
+    L.prism_debug_bounds_probe.argtypes = [ctypes.c_longlong, ctypes.c_longlong, vp]
+    L.prism_debug_bounds_probe.restype = ci
     _lib = L
     return L
 

@@ -1,4 +1,6 @@
-"""Build ``libprism.so`` in-tree with nvcc for sm_100a (no JIT cache)."""
+"""Build ``libprism.so`` and its debug build ``libprism_debug.so`` in-tree with nvcc for
+sm_100a (no JIT cache).  The debug build is compiled with PRISM_DEBUG_BOUNDS: its kernels
+check the global indices they compute and record PRISM_ERR_BOUNDS instead of faulting."""
 from __future__ import annotations
 
 import glob
@@ -11,6 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libprism.so")
+LIB_DEBUG = os.path.join(PKG, "libprism_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -31,25 +34,38 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def needs_rebuild() -> bool:
-    if not os.path.exists(LIB):
+def needs_rebuild(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+def _command(lib: str, debug: bool) -> list[str]:
+    flags = NVCC_FLAGS + (["-DPRISM_DEBUG_BOUNDS"] if debug else [])
+    return [nvcc(), *flags, "-I", INCLUDE, "-I", CSRC, *sources(), "-o", lib + ".tmp"]
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_rebuild():
-        return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *sources(), "-o", LIB + ".tmp"]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
+    """Compile both libraries (side by side) when a source is newer; returns the release
+    library's path."""
+    todo = [(lib, debug) for lib, debug in ((LIB, False), (LIB_DEBUG, True)) if force or needs_rebuild(lib)]
+    procs = []
+    for lib, debug in todo:
+        cmd = _command(lib, debug)
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append((lib, cmd, subprocess.Popen(cmd)))
+    failed = [cmd for _, cmd, proc in procs if proc.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
+    for lib, _, _ in procs:
+        os.replace(lib + ".tmp", lib)
     return LIB
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True)
     print(LIB)
+    print(LIB_DEBUG)

@@ -68,14 +68,21 @@ __global__ void __launch_bounds__(kF32Threads) chunk_fp32_kernel(ScanParams p) {
   const float* conv_state = static_cast<const float*>(p.conv_state);
   float* o = static_cast<float*>(p.o);
   const size_t bh = (size_t)b * H + h;
+  int* status = p.status;
+  // extents of the buffers (the debug build checks every index against them)
+  const long long n_tok = (long long)p.B * T_ * H, n_x = n_tok * D, n_u = n_x * max(m, 1);
 
   // S_0 and the v rows before token 0 (the caller's ShortConv history, or zeros)
   for (int e = tid; e < D * D; e += kF32Threads) {
     const int c = e / D, j = e % D;
-    sS[c * LD + j] = p.S0 ? p.S0[bh * D * D + e] : 0.f;
+    sS[c * LD + j] = p.S0 && in_bounds((long long)(bh * D * D + e), (long long)p.B * H * D * D, status)
+                         ? p.S0[bh * D * D + e]
+                         : 0.f;
   }
   for (int e = tid; e < (W - 1) * D; e += kF32Threads)
-    shist[e] = conv_state ? conv_state[bh * (W - 1) * D + e] : 0.f;
+    shist[e] = conv_state && in_bounds((long long)(bh * (W - 1) * D + e), (long long)p.B * H * (W - 1) * D, status)
+                   ? conv_state[bh * (W - 1) * D + e]
+                   : 0.f;
 
   const int nchunks = (len + C - 1) / C;
   for (int n = 0; n < nchunks; ++n) {
@@ -84,8 +91,8 @@ __global__ void __launch_bounds__(kF32Threads) chunk_fp32_kernel(ScanParams p) {
     // ---- tiles of the chunk (padded tokens: zero vectors, gamma = 1, beta = 0)
     for (int e = tid; e < C * D; e += kF32Threads) {
       const int t = e / D, c = e % D;
-      const bool ok = t < nv;
       const size_t g = (((size_t)b * T_ + t0 + t) * H + h) * D + c;
+      const bool ok = t < nv && in_bounds((long long)g, n_x, status);
       sK[t * LD + c] = ok ? k[g] : 0.f;
       sQ[t * LD + c] = ok ? q[g] : 0.f;
       sV[t * LD + c] = ok ? v[g] : 0.f;
@@ -93,8 +100,8 @@ __global__ void __launch_bounds__(kF32Threads) chunk_fp32_kernel(ScanParams p) {
     }
     for (int e = tid; e < D * D; e += kF32Threads) sSa[(e / D) * LD + e % D] = 0.f;
     if (tid < C) {
-      const bool ok = tid < nv;
       const size_t g = ((size_t)b * T_ + t0 + tid) * H + h;
+      const bool ok = tid < nv && in_bounds((long long)g, n_tok, status);
       slc[tid] = ok ? logf(p.gamma[g]) : 0.f;  // prefix-summed below
       sbet[tid] = ok ? p.beta[g] : 0.f;
     }
@@ -117,7 +124,8 @@ __global__ void __launch_bounds__(kF32Threads) chunk_fp32_kernel(ScanParams p) {
       for (int i = 0; i < W; ++i) {
         const int tau = t - i;
         const float vi = tau >= 0 ? sV[tau * LD + c] : shist[(W - 1 + tau) * D + c];
-        a = fmaf(p.conv_w[((size_t)h * D + c) * W + i], vi, a);
+        const long long wi = ((long long)h * D + c) * W + i;
+        if (in_bounds(wi, (long long)H * D * W, status)) a = fmaf(p.conv_w[wi], vi, a);
       }
       sR[t * LD + c] = t < nv ? sV[t * LD + c] - a : 0.f;
     }
@@ -153,8 +161,8 @@ __global__ void __launch_bounds__(kF32Threads) chunk_fp32_kernel(ScanParams p) {
       __syncthreads();  // T done (l = 0) / the previous direction's products are done
       for (int e = tid; e < C * D; e += kF32Threads) {
         const int t = e / D, c = e % D;
-        const bool ok = t < nv;
         const size_t g = ((((size_t)b * T_ + t0 + t) * H + h) * m + l) * D + c;
+        const bool ok = t < nv && in_bounds((long long)g, n_u, status);
         const float r = ok ? chain_step(sR[t * LD + c], gain[g], p.chain) : 0.f;
         const float al = ok ? p.alpha[(((size_t)b * T_ + t0 + t) * H + h) * m + l] : 0.f;
         sR[t * LD + c] = r;
@@ -248,7 +256,8 @@ __global__ void __launch_bounds__(kF32Threads) chunk_fp32_kernel(ScanParams p) {
       const int t = e / D, c = e % D;
       float a = sO[t * LD + c];
       for (int i = 0; i <= t; ++i) a = fmaf(sM[t * LC + i], sX[i * LD + c], a);
-      if (t < nv) o[(((size_t)b * T_ + t0 + t) * H + h) * D + c] = a;
+      const size_t oi = (((size_t)b * T_ + t0 + t) * H + h) * D + c;
+      if (t < nv && in_bounds((long long)oi, n_x, status)) o[oi] = a;
     }
     // ---- S_{n+1} = b_C S_n + Delta^T diag(b_C / b) K + Sadd
     for (int e = tid; e < D * D; e += kF32Threads) {
@@ -266,10 +275,13 @@ __global__ void __launch_bounds__(kF32Threads) chunk_fp32_kernel(ScanParams p) {
   __syncthreads();
   for (size_t e = tid; e < (size_t)(T_ - len) * D; e += kF32Threads) {
     const int t = len + (int)(e / D), c = (int)(e % D);
-    o[(((size_t)b * T_ + t) * H + h) * D + c] = 0.f;
+    const size_t oi = (((size_t)b * T_ + t) * H + h) * D + c;
+    if (in_bounds((long long)oi, n_x, status)) o[oi] = 0.f;
   }
   if (p.S_final)
-    for (int e = tid; e < D * D; e += kF32Threads) p.S_final[bh * D * D + e] = sS[(e / D) * LD + e % D];
+    for (int e = tid; e < D * D; e += kF32Threads)
+      if (in_bounds((long long)(bh * D * D + e), (long long)p.B * H * D * D, status))
+        p.S_final[bh * D * D + e] = sS[(e / D) * LD + e % D];
 }
 
 template <int D, int C>

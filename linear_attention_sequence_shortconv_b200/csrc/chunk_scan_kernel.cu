@@ -413,7 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = chain;
   const int seg = p.seg_only >= 0 ? p.seg_only : (int)blockIdx.x % p.P, b = bh / p.H, h = bh % p.H;
   const int T = p.T, H = p.H, m = p.m;
-  const int len = p.lengths ? min(max(p.lengths[b], 0), T) : T;
+  // debug build: a chain or segment outside the plan does no work
+  const bool cta_ok = in_bounds(bh, (long long)p.B * H, p.status) && in_bounds(seg, p.P, p.status);
+  const int len = !cta_ok ? 0 : p.lengths ? min(max(p.lengths[b], 0), T) : T;
   const int tok0 = seg * p.Ts;                         // first token of this CTA's segment
   const int seg_end = seg == p.P - 1 ? T : min(tok0 + p.Ts, T);  // end of the segment (the last: T)
   const int vend = min(len, seg_end);                  // end of its valid tokens
@@ -421,11 +423,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long lim = p.spin_limit;
   int* status = p.status;
   const size_t DD = (size_t)D * D;
-  const float* S_start = seg == 0 ? (p.S0 ? p.S0 + (size_t)bh * DD : nullptr)
-                                  : (p.S_in ? p.S_in + ((size_t)bh * p.P + seg) * DD : nullptr);
+  const float* S_start = !cta_ok ? nullptr
+                         : seg == 0 ? (p.S0 ? p.S0 + (size_t)bh * DD : nullptr)
+                                    : (p.S_in ? p.S_in + ((size_t)bh * p.P + seg) * DD : nullptr);
   const bool start_identity = seg > 0 && p.s_in_identity;
-  float* S_end = p.S_out ? p.S_out + ((size_t)bh * p.P + seg) * DD
-                         : (seg == p.P - 1 && p.S_final ? p.S_final + (size_t)bh * DD : nullptr);
+  float* S_end = !cta_ok ? nullptr
+                 : p.S_out ? p.S_out + ((size_t)bh * p.P + seg) * DD
+                           : (seg == p.P - 1 && p.S_final ? p.S_final + (size_t)bh * DD : nullptr);
 
   if (tid == 0) {
     // one arrival each, except the epilogue group's hand-overs: one per warp (8, or the 4
@@ -464,6 +468,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // cannot deadlock.
     if (lane == 0) {
       int n_kq = 0, n_v = 0, n_kb = 0, nu[3] = {0, 0, 0}, np[2] = {0, 0};  // loads issued per stream
+      // debug build: the coordinates of a tile of direction l at token t0 (the innermost,
+      // 64 a, is a multiple of 8 inside [0, D) by construction); on a failure the CTA aborts
+      auto tile_ok = [&](int l, int t0) -> bool {
+        const bool ok = in_bounds(l, max(m, 1), status) && in_bounds(t0, T, status) && in_bounds(h, H, status) &&
+                        in_bounds(b, p.B, status) && tma_x_ok(64 * (NA - 1), 64, D, status);
+        if (!ok) *s_abort = 1;
+        return ok;
+      };
       auto prefetch = [&](int n) {  // every tile of chunk n into L2
         const int t0 = tok0 + n * kC;
         for (int a = 0; a < NA; ++a) {
@@ -482,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j % NU;
         if (j >= NU && !bwait(&bars[kUFree0 + s], ((j / NU) - 1) & 1, lim, status, s_abort)) return false;
         const int t0 = tok0 + (j / m) * kC, l = j % m;
+        if (!tile_ok(l, t0)) return false;
         mbar_arrive_expect_tx(&bars[kUFull0 + s], (NU == 2 ? 2 : 1) * NA * kAtom64);
         for (int a = 0; a < NA; ++a) {
           tma_load_5d(sm + Ly::UB + (s * NA + a) * kAtom64, &map_u, &bars[kUFull0 + s], 64 * a, l, h, t0, b);
@@ -496,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j & 1;
         if (j >= 2 && !bwait(&bars[kPFree0 + s], ((j >> 1) - 1) & 1, lim, status, s_abort)) return false;
         const int t0 = tok0 + (j / m) * kC, l = j % m;
+        if (!tile_ok(l, t0)) return false;
         mbar_arrive_expect_tx(&bars[kPFull0 + s], NA * kAtom64);
         for (int a = 0; a < NA; ++a)
           tma_load_5d(sm + Ly::PB + (s * NA + a) * kAtom64, &map_g, &bars[kPFull0 + s], 64 * a, l, h, t0, b);
@@ -505,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto ld_kq = [&](int n) -> bool {
         if (n >= 1 && !bwait(&bars[kKqFree], (n - 1) & 1, lim, status, s_abort)) return false;
         const int t0 = tok0 + n * kC;
+        if (!tile_ok(0, t0)) return false;
         mbar_arrive_expect_tx(&bars[kKqFull], 2 * NA * kAtom64);
         for (int a = 0; a < NA; ++a) {
           tma_load_4d(sKQ + a * kAtom128, &map_k, &bars[kKqFull], 64 * a, h, t0, b);
@@ -521,6 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (VW ? !bwait(&bars[kWsFree], n & 1, lim, status, s_abort)
                : (n >= 1 && !bwait(&bars[kVFree], (n - 1) & 1, lim, status, s_abort)))
           return false;
+        if (!tile_ok(0, tok0 + n * kC)) return false;
         mbar_arrive_expect_tx(&bars[kVFull], NA * kAtom64);
         for (int a = 0; a < NA; ++a)
           tma_load_4d(sVB + a * kAtom64, &map_v, &bars[kVFull], 64 * a, h, tok0 + n * kC, b);
@@ -529,6 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto ld_kb = [&](int n) -> bool {
         if (n >= 1 && !bwait(&bars[kRsFull], (n - 1) & 1, lim, status, s_abort)) return false;
+        if (!tile_ok(0, tok0 + n * kC)) return false;
         mbar_arrive_expect_tx(&bars[kKbFull], NA * kAtom64);
         for (int a = 0; a < NA; ++a)
           tma_load_4d(sKB + a * kAtom64, &map_k, &bars[kKbFull], 64 * a, h, tok0 + n * kC, b);
@@ -689,8 +706,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = 2 * lane + e;
         const bool valid = t < nv;
         const size_t th = ((size_t)b * T + min(t0 + t, T - 1)) * H + h;
-        gl[e] = valid ? __ldg(p.gamma + th) : 1.f;
-        bl[e] = valid ? __ldg(p.beta + th) : 0.f;
+        const bool ld = valid && in_bounds((long long)th, (long long)p.B * T * H, status);
+        gl[e] = ld ? __ldg(p.gamma + th) : 1.f;
+        bl[e] = ld ? __ldg(p.beta + th) : 0.f;
       }
       float Gv[2], G63;
       chunk_log_decay(gl[0], gl[1], lane, Gv[0], Gv[1], G63);
@@ -1141,12 +1159,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (srow && p.write_o) {  // o[t0 + t, c] = O^T[c, t]; zero past the sequence's length
         __nv_bfloat16* op = p.o + (((size_t)b * T + t0) * H + h) * D + row;
         const int tmax = min(kC, seg_end - t0);
+        // debug build: the first and the last token row this thread writes (the rows between
+        // lie between them)
+        const long long o0 = (((long long)b * T + t0) * H + h) * D + row, on = (long long)p.B * T * H * D;
+        const bool o_ok = in_bounds(o0, on, status) && in_bounds(o0 + (long long)(tmax - 1) * H * D, on, status);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t raw[32];
           tmem_ld32_raw(tl + kACC + 64 + 32 * half, raw);
           tmem_wait_ld();
-          if (nv == kC) {  // a full chunk: every token valid and inside the tensor
+          if (!o_ok) {
+          } else if (nv == kC) {  // a full chunk: every token valid and inside the tensor
 #pragma unroll
             for (int e = 0; e < 32; ++e)
               op[(size_t)(32 * half + e) * H * D] = __float2bfloat16_rn(__uint_as_float(raw[e]));
@@ -1188,12 +1211,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = tid; e < D * D; e += kEG)
           S_end[e] = start_identity ? (e / D == e % D ? 1.f : 0.f) : (S_start ? S_start[e] : 0.f);
       }
-      if (p.write_o) {  // o = 0 for the segment's tokens past its last chunk
+      if (p.write_o && cta_ok) {  // o = 0 for the segment's tokens past its last chunk
         const int tz = tok0 + nchunks * kC;
         const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
         for (size_t e = tid; e < (size_t)max(seg_end - tz, 0) * D; e += kEG) {
           const int t = tz + (int)(e / D), c = (int)(e % D);
-          p.o[(((size_t)b * T + t) * H + h) * D + c] = zero;
+          const size_t oi = (((size_t)b * T + t) * H + h) * D + c;
+          if (in_bounds((long long)oi, (long long)p.B * T * H * D, status)) p.o[oi] = zero;
         }
       }
     }
@@ -1226,8 +1250,8 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
     residual_write_kernel(const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ gain,
                           const float* __restrict__ alpha, const float* __restrict__ gamma,
                           const float* __restrict__ conv_w, const int32_t* __restrict__ lengths,
-                          const __nv_bfloat16* __restrict__ conv_state, __nv_bfloat16* __restrict__ ptil, int T,
-                          int H, int W, int m, int nc0, int ncn) {
+                          const __nv_bfloat16* __restrict__ conv_state, __nv_bfloat16* __restrict__ ptil, int B,
+                          int T, int H, int W, int m, int nc0, int ncn, int* status) {
   constexpr int CPT = D / 8;              // threads per token row
   constexpr int TPT = kPrepTPT;
   constexpr int PB = kC / prep_tokens(D);  // CTAs per chunk
@@ -1238,6 +1262,7 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
   __shared__ __align__(16) float s_taps[WM][D];  // ShortConv taps of the head, tap-major
   const int part = blockIdx.x % PB, cidx = blockIdx.x / PB;
   const int n = nc0 + cidx % ncn, bh = cidx / ncn, b = bh / H, h = bh % H;
+  if (!in_bounds(bh, (long long)B * H, status)) return;  // debug build: a chain outside the batch
   const int len = lengths ? min(max(lengths[b], 0), T) : T;
   const int t0 = n * kC;
   if (t0 >= len) return;
@@ -1249,11 +1274,14 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int t = t0 + i0 - (WM - 1) + j;
+    const size_t vi = (((size_t)b * T + t) * H + h) * D + c8;
+    const size_t ci = (((size_t)b * H + h) * (W - 1) + (W - 1 + t)) * D + c8;
     if (t >= 0)
-      vr[j] = t < T ? ldg16(v + (((size_t)b * T + t) * H + h) * D + c8) : make_uint4(0, 0, 0, 0);
+      vr[j] = t < T && in_bounds((long long)vi + 7, (long long)B * T * H * D, status) ? ldg16(v + vi)
+                                                                                       : make_uint4(0, 0, 0, 0);
     else  // before token 0: the sequence's ShortConv history (rows W - 1 + t), else zero
-      vr[j] = (conv_state && t >= 1 - W)
-                  ? ldg16(conv_state + (((size_t)b * H + h) * (W - 1) + (W - 1 + t)) * D + c8)
+      vr[j] = (conv_state && t >= 1 - W && in_bounds((long long)ci + 7, (long long)B * H * (W - 1) * D, status))
+                  ? ldg16(conv_state + ci)
                   : make_uint4(0, 0, 0, 0);
   }
   uint4 gr[LB][TPT];
@@ -1263,8 +1291,9 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
     for (int j = 0; j < LB; ++j)
 #pragma unroll
       for (int a = 0; a < TPT; ++a) {
-        const bool ok = l0 + j < m && t0 + i0 + a < len;
         const size_t th = row0 + (size_t)a * H;
+        const bool ok = l0 + j < m && t0 + i0 + a < len &&
+                        in_bounds((long long)((th * m + l0 + j) * D + c8) + 7, (long long)B * T * H * m * D, status);
         gr[j][a] = ok ? ldg16(gain + (th * m + l0 + j) * D + c8) : make_uint4(0, 0, 0, 0);
         al[j][a] = ok ? __ldg(alpha + th * m + l0 + j) : 0.f;
       }
@@ -1272,7 +1301,9 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
   load_levels(0);
   for (int e = tid; e < WM * D; e += kPrepThreads) {
     const int w = e / D, c = e % D;
-    s_taps[w][c] = w < W ? __ldg(conv_w + ((size_t)h * D + c) * W + w) : 0.f;
+    s_taps[w][c] = w < W && in_bounds(((long long)h * D + c) * W + w, (long long)H * D * W, status)
+                       ? __ldg(conv_w + ((size_t)h * D + c) * W + w)
+                       : 0.f;
   }
   if (tid < 32) {
     const int nv = min(kC, len - t0);
@@ -1280,7 +1311,8 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int t = 2 * lane + e;
-      gl[e] = t < nv ? __ldg(gamma + ((size_t)b * T + t0 + t) * H + h) : 1.f;
+      const size_t gi = ((size_t)b * T + t0 + t) * H + h;
+      gl[e] = t < nv && in_bounds((long long)gi, (long long)B * T * H, status) ? __ldg(gamma + gi) : 1.f;
     }
     float G0, G1, G63;
     chunk_log_decay(gl[0], gl[1], lane, G0, G1, G63);
@@ -1342,7 +1374,9 @@ __global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
               u.z = pack_bf16x2(rho[4], rho[5]);
               u.w = pack_bf16x2(rho[6], rho[7]);
             }
-            *reinterpret_cast<uint4*>(ptil + ((row0 + (size_t)a * H) * m + l0 + j) * D + c8) = u;
+            const size_t pi = ((row0 + (size_t)a * H) * m + l0 + j) * D + c8;
+            if (in_bounds((long long)pi + 7, (long long)B * T * H * m * D, status))
+              *reinterpret_cast<uint4*>(ptil + pi) = u;
           }
         }
       }
@@ -1600,9 +1634,9 @@ cudaError_t launch_dc(const ScanParams& p, cudaStream_t stream) {
     cfg.numAttrs = dependent ? 1 : 0;
     if (p.W <= 4)
       return cudaLaunchKernelEx(&cfg, residual_write_kernel<D, CH, 4>, vv, gg, p.alpha, p.gamma, p.conv_w,
-                                p.lengths, cs, ptil, p.T, p.H, p.W, m, nc0, ncn);
+                                p.lengths, cs, ptil, p.B, p.T, p.H, p.W, m, nc0, ncn, p.status);
     return cudaLaunchKernelEx(&cfg, residual_write_kernel<D, CH, PRISM_MAX_W>, vv, gg, p.alpha, p.gamma, p.conv_w,
-                              p.lengths, cs, ptil, p.T, p.H, p.W, m, nc0, ncn);
+                              p.lengths, cs, ptil, p.B, p.T, p.H, p.W, m, nc0, ncn, p.status);
   };
   if (m > 0) {
     const cuuint64_t dims5[5] = {(cuuint64_t)D, (cuuint64_t)m, H, T, B};

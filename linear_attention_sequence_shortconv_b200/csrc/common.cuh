@@ -198,4 +198,33 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, PRISM_OK, code);
 }
 
+// The debug build (compiled with PRISM_DEBUG_BOUNDS, libprism_debug.so) checks the global
+// indices the kernels compute against the extents of their buffers, and the innermost
+// coordinate of every TMA copy against the 16-byte rule.  A failed check records
+// PRISM_ERR_BOUNDS in the status word and the access is skipped, so a bad index shows up
+// in prism_stream_status instead of as a fault.  The release build compiles every check to
+// `true`.
+#ifdef PRISM_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+
+// 0 <= i < n (always true in the release build)
+__device__ __forceinline__ bool in_bounds(long long i, long long n, int* status) {
+  if (!kDebugBounds) return true;
+  if (i >= 0 && i < n) return true;
+  record_status(status, PRISM_ERR_BOUNDS);
+  return false;
+}
+
+// a TMA box of bf16 elements starting at innermost coordinate x inside [0, extent): x a
+// multiple of 8 (16 bytes) and x + box <= extent (always true in the release build)
+__device__ __forceinline__ bool tma_x_ok(int x, int box, int extent, int* status) {
+  if (!kDebugBounds) return true;
+  if (x >= 0 && (x & 7) == 0 && x + box <= extent) return true;
+  record_status(status, PRISM_ERR_BOUNDS);
+  return false;
+}
+
 }  // namespace prism

@@ -93,9 +93,23 @@ namespace {
 using prism::check_sizes;
 using prism::device_setup;
 
+// one thread: the device-side index check on (i, n), nothing accessed
+__global__ void bounds_probe_kernel(long long i, long long n, int* status) { prism::in_bounds(i, n, status); }
+
 }  // namespace
 
 extern "C" {
+
+int prism_debug_bounds(void) { return prism::kDebugBounds ? 1 : 0; }
+
+int prism_debug_bounds_probe(long long i, long long n, prism_stream_t stream) {
+  if (!prism::kDebugBounds) return PRISM_ERR_UNSUPPORTED;
+  int* status = nullptr;
+  const int rc = device_setup(&status);
+  if (rc != PRISM_OK) return rc;
+  bounds_probe_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(i, n, status);
+  return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
 
 int prism_version(void) {
   return (PRISM_VERSION_MAJOR << 16) | (PRISM_VERSION_MINOR << 8) | PRISM_VERSION_PATCH;
@@ -109,6 +123,7 @@ const char* prism_status_string(int code) {
     case PRISM_ERR_WORKSPACE: return "PRISM_ERR_WORKSPACE: workspace smaller than prism_scan_fwd_workspace_size()";
     case PRISM_ERR_CUDA: return "PRISM_ERR_CUDA: a CUDA runtime call or kernel launch failed";
     case PRISM_ERR_TIMEOUT: return "PRISM_ERR_TIMEOUT: a bounded device-side wait expired";
+    case PRISM_ERR_BOUNDS: return "PRISM_ERR_BOUNDS: a kernel computed an index outside its buffer (debug build)";
     default: return "PRISM: unknown status code";
   }
 }

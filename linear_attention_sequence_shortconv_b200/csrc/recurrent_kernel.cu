@@ -109,7 +109,10 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   const int T_ = p.T, H = p.H, dk = p.d_k, dv = p.d_v, m = p.L - 1, W = p.W;
   const bool row_ok = row < dv;
   const int c = row_ok ? row : dv - 1;  // idle rows shadow the last real row (no stores)
-  const int len = p.lengths ? min(max(p.lengths[b], 0), T_) : T_;
+  // debug build: a block outside the batch or the heads reads and writes nothing
+  const bool blk_ok = in_bounds(b, p.B, p.status) && in_bounds(h, H, p.status);
+  const int len = !blk_ok ? 0 : p.lengths ? min(max(p.lengths[b], 0), T_) : T_;
+  const long long n_o = (long long)p.B * T_ * H * dv;
   const TileLayout L(TT, dk, m, RPB, (int)sizeof(T));
   const int nrows = min(RPB, dv - row0);  // rows of this block that exist
 
@@ -124,6 +127,8 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   auto load_tile = [&](int ti, int buf) {
     uint8_t* base = smem + buf * L.bytes;
     const int t0 = ti * TT, nt = min(TT, len - t0);
+    // debug build: the tile's last (token, head) row lies inside the tensors
+    if (nt > 0 && !in_bounds(((long long)b * T_ + t0 + nt - 1) * H + h, (long long)p.B * T_ * H, p.status)) return;
     const int vec = 16 / (int)sizeof(T);  // elements per 16-byte chunk
     const int kchunks = dk / vec;
     // k, q: [nt][dk]
@@ -182,14 +187,14 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
   const T* cs = static_cast<const T*>(p.conv_state);
 #pragma unroll
   for (int i = 0; i < PRISM_MAX_W; ++i)
-    hist[i] = (cs && i < W - 1) ? ld1<T>(cs + (((size_t)b * H + h) * (W - 1) + (W - 2 - i)) * dv + c) : 0.f;
+    hist[i] = (cs && blk_ok && i < W - 1) ? ld1<T>(cs + (((size_t)b * H + h) * (W - 1) + (W - 2 - i)) * dv + c) : 0.f;
 
   float s[EPL];
   const size_t sbase = (((size_t)b * H + h) * dv + c) * dk + 4 * j;
 #pragma unroll
   for (int e = 0; e < EPL; e += 4) {
-    const float4 f =
-        p.S0 ? __ldg(reinterpret_cast<const float4*>(p.S0 + sbase + e * LPR)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 f = p.S0 && blk_ok ? __ldg(reinterpret_cast<const float4*>(p.S0 + sbase + e * LPR))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
     s[e] = f.x; s[e + 1] = f.y; s[e + 2] = f.z; s[e + 3] = f.w;
   }
 
@@ -290,15 +295,19 @@ __global__ void __launch_bounds__(kBlock) recurrent_scan_kernel(ScanParams p, in
           oq += s[e] * f.x + s[e + 1] * f.y + s[e + 2] * f.z + s[e + 3] * f.w;
         }
         oq = row_sum<LPR>(oq);
-        if (row_ok && j == 0) st1<T>(o + (((size_t)b * T_ + t0 + i) * H + h) * dv + c, oq);
+        const size_t oi = (((size_t)b * T_ + t0 + i) * H + h) * dv + c;
+        if (row_ok && j == 0 && in_bounds((long long)oi, n_o, p.status)) st1<T>(o + oi, oq);
       }
     }
     __syncthreads();  // the buffer is refilled next iteration
   }
   cp_async_wait_0();
-  if (o && row_ok && j == 0)
-    for (int t = len; t < T_; ++t) st1<T>(o + (((size_t)b * T_ + t) * H + h) * dv + c, 0.f);
-  if (row_ok && p.S_final) {
+  if (o && row_ok && j == 0 && blk_ok)
+    for (int t = len; t < T_; ++t) {
+      const size_t oi = (((size_t)b * T_ + t) * H + h) * dv + c;
+      if (in_bounds((long long)oi, n_o, p.status)) st1<T>(o + oi, 0.f);
+    }
+  if (row_ok && p.S_final && blk_ok) {
 #pragma unroll
     for (int e = 0; e < EPL; e += 4)
       *reinterpret_cast<float4*>(p.S_final + sbase + e * LPR) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);

@@ -41,9 +41,22 @@ def test_version_matches_header(L):
 
 
 def test_status_strings(L):
-    for code in range(6):
+    for code in range(7):
         assert prism.status_string(code).startswith("PRISM")
+    assert "BOUNDS" in prism.status_string(6)
     assert "unknown" in prism.status_string(99)
+
+
+def test_debug_build_exports_the_same_symbols(L):
+    # the bounds-checked debug build is a second library with the same ABI; it reports itself
+    # through prism_debug_bounds (the release build: 0, and its probe hook is unsupported)
+    D = ctypes.CDLL(prism_build.LIB_DEBUG)
+    for name in declared_functions():
+        assert hasattr(D, name), name
+    D.prism_debug_bounds.restype = ctypes.c_int
+    assert D.prism_debug_bounds() == 1
+    assert L.prism_debug_bounds() == 0
+    assert L.prism_debug_bounds_probe(5, 4, None) == 2  # PRISM_ERR_UNSUPPORTED, no CUDA call
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails before any CUDA call
