@@ -58,6 +58,7 @@ struct DecodeParams {
   float* S;
   void* o;
   int B, H, d_k, d_v, L, W, chain;
+  int* status;  // device status word (the debug build's bounds checks record there)
 };
 
 // Pointers and sizes of one prism_scan_bwd call (device pointers).

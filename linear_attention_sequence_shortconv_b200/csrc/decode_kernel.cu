@@ -28,6 +28,9 @@ __global__ void __launch_bounds__(kLanes * 128) decode_step_kernel(DecodeParams 
   extern __shared__ float sh[];  // k [d_k], q [d_k], u [m][d_k] as fp32
   const int bh = blockIdx.x, h = bh % p.H;
   const int dk = p.d_k, dv = p.d_v, m = p.L - 1;
+  // debug build: a block or a state row outside the batch reads and writes no global memory
+  // (no early return: every thread still meets the barrier below)
+  const bool bh_ok = in_bounds(bh, (long long)p.B * p.H, p.status);
   float* sk = sh;
   float* sq = sh + dk;
   float* su = sh + 2 * dk;
@@ -35,28 +38,30 @@ __global__ void __launch_bounds__(kLanes * 128) decode_step_kernel(DecodeParams 
   const T* qin = static_cast<const T*>(p.q) + (size_t)bh * dk;
   const T* uin = static_cast<const T*>(p.u) + (size_t)bh * m * dk;
   for (int j = threadIdx.x; j < dk; j += blockDim.x) {
-    sk[j] = ld1<T>(kin + j);
-    sq[j] = ld1<T>(qin + j);
+    sk[j] = bh_ok ? ld1<T>(kin + j) : 0.f;
+    sq[j] = bh_ok ? ld1<T>(qin + j) : 0.f;
   }
-  for (int j = threadIdx.x; j < m * dk; j += blockDim.x) su[j] = ld1<T>(uin + j);
+  for (int j = threadIdx.x; j < m * dk; j += blockDim.x) su[j] = bh_ok ? ld1<T>(uin + j) : 0.f;
 
   const int c = threadIdx.x / kLanes, lane = threadIdx.x % kLanes;
+  const bool ok = bh_ok && in_bounds(c, dv, p.status);
   const int groups = dk / (4 * kLanes);
   float* Srow = p.S + ((size_t)bh * dv + c) * dk;
   float4 s[kMaxGroups];
 #pragma unroll
   for (int i = 0; i < kMaxGroups; ++i)
-    if (i < groups) s[i] = *reinterpret_cast<const float4*>(Srow + 16 * i + 4 * lane);
-  const float gam = __ldg(p.gamma + bh), bet = __ldg(p.beta + bh);
-  const float vc = ld1<T>(static_cast<const T*>(p.v) + (size_t)bh * dv + c);
+    if (i < groups) s[i] = ok ? *reinterpret_cast<const float4*>(Srow + 16 * i + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float gam = ok ? __ldg(p.gamma + bh) : 1.f, bet = ok ? __ldg(p.beta + bh) : 0.f;
+  const float vc = ok ? ld1<T>(static_cast<const T*>(p.v) + (size_t)bh * dv + c) : 0.f;
   // ShortConv anchor from the carried history (oldest first)
   const float* w = p.conv_w + ((size_t)h * dv + c) * p.W;
   T* hist = static_cast<T*>(p.conv_state) + (size_t)bh * (p.W - 1) * dv + c;
   float hv[PRISM_MAX_W];
-  float a = __ldg(w) * vc;
+  float a = ok ? __ldg(w) * vc : 0.f;
 #pragma unroll
   for (int i = 1; i < PRISM_MAX_W; ++i) {
-    if (i < p.W) {
+    hv[i] = 0.f;
+    if (ok && i < p.W) {
       hv[i] = ld_plain(hist + (size_t)(p.W - 1 - i) * dv);  // v_{t-i}
       a += __ldg(w + i) * hv[i];
     }
@@ -87,7 +92,7 @@ __global__ void __launch_bounds__(kLanes * 128) decode_step_kernel(DecodeParams 
     }
   }
   // residual chain and its rank-m write
-  if (m > 0) {
+  if (m > 0 && ok) {
     const T* g = static_cast<const T*>(p.gain) + (size_t)bh * m * dv + c;
     const float* al = p.alpha + (size_t)bh * m;
     float r = vc - a;
@@ -114,12 +119,12 @@ __global__ void __launch_bounds__(kLanes * 128) decode_step_kernel(DecodeParams 
     if (i < groups) {
       const float4 qq = *reinterpret_cast<const float4*>(sq + 16 * i + 4 * lane);
       oc += s[i].x * qq.x + s[i].y * qq.y + s[i].z * qq.z + s[i].w * qq.w;
-      *reinterpret_cast<float4*>(Srow + 16 * i + 4 * lane) = s[i];
+      if (ok) *reinterpret_cast<float4*>(Srow + 16 * i + 4 * lane) = s[i];
     }
   }
   oc += __shfl_xor_sync(0xffffffffu, oc, 1);
   oc += __shfl_xor_sync(0xffffffffu, oc, 2);
-  if (lane == 0) {
+  if (lane == 0 && ok) {
     st1<T>(static_cast<T*>(p.o) + (size_t)bh * dv + c, oc);
     // history <- (v_{t-W+2}, ..., v_t), oldest first: slot W-2-i takes v_{t-i}; this thread
     // read channel c's old history above, so the shift reuses those values

@@ -328,7 +328,7 @@ int prism_decode_step(const void* q, const void* k, const void* v, const float* 
   rc = device_setup(&status);
   if (rc != PRISM_OK) return rc;
   prism::DecodeParams p{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr,
-                        conv_w, W > 1 ? conv_state : nullptr, S, o, B, H, d_k, d_v, L, W, chain};
+                        conv_w, W > 1 ? conv_state : nullptr, S, o, B, H, d_k, d_v, L, W, chain, status};
   cudaError_t err = prism::launch_decode_step(p, dtype, reinterpret_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }

@@ -2,8 +2,9 @@
 the global indices they compute against their buffers' extents and record
 PRISM_ERR_BOUNDS instead of faulting.  On valid inputs it must report nothing and give the
 release build's results bit for bit, on every forward path: the tensor-core scan (plain,
-in two halves, cut into segments, ragged rows), the fp32 chunk form and the token-by-token
-kernel.  Its probe hook shows that a failed device-side check reaches prism_stream_status.
+in two halves, cut into segments, ragged rows), the fp32 chunk form, the token-by-token
+kernel, and the decode step.  Its probe hook shows that a failed device-side check
+reaches prism_stream_status.
 
 The debug library is loaded in a child process (PRISM_DEBUG_BOUNDS=1 selects it), which
 writes its outputs to a file that this process compares with the release library's.
@@ -54,6 +55,20 @@ def _run_all():
             out[f"{name}_{chain}_o"] = o.float().cpu().numpy()
             out[f"{name}_{chain}_S"] = S.cpu().numpy()
             out[f"{name}_{chain}_status"] = np.array(status)
+    # decode: a few tokens of two cases, the state and the ShortConv history carried in place
+    for name in ("tc_d128", "fp32_chunk"):
+        w = CASES[name]
+        d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in synth.make_inputs(w).items()}
+        S = torch.zeros((w.B, w.H, w.d_v, w.d_k), dtype=torch.float32, device="cuda")
+        hist = torch.zeros((w.B, w.H, w.W - 1, w.d_v), dtype=d["v"].dtype, device="cuda")
+        for t in range(3):
+            tok = {n: d[n][:, t].contiguous() for n in ("q", "k", "v", "gamma", "beta", "u", "alpha", "gain")}
+            o = prism.decode_step(tok["q"], tok["k"], tok["v"], tok["gamma"], tok["beta"], tok["u"], tok["alpha"],
+                                  tok["gain"], d["conv_w"], hist, S, L=w.L)
+            out[f"decode_{name}_{t}_o"] = o.float().cpu().numpy()
+        out[f"decode_{name}_status"] = np.array(prism.stream_status())
+        out[f"decode_{name}_S"] = S.cpu().numpy()
+        out[f"decode_{name}_hist"] = hist.float().cpu().numpy()
     return out
 
 
