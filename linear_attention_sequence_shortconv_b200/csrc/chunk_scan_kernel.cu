@@ -1233,20 +1233,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 // r_{t,l} = chain step of r_{t,l-1} with gain g_{t,l}.  In a chunk whose decay is factored
 // (chunk_decay_fast), P~ = e^{G_63 - G_t} rho; else P~ = rho.  Nothing here depends on the
 // state, so every chunk of every chain runs at once, in CTAs of kPrepThreads threads over
-// prep_tokens(D) tokens of one chunk.  A thread owns 8 channels of 4 consecutive tokens: it
+// prep_tokens(D) tokens of one chunk.  A thread owns 8 channels of 2 consecutive tokens: it
 // loads each v row of their ShortConv window once and the gain rows of up to kPrepLevels
 // levels at the same time, so that enough 16-byte loads are in flight to keep HBM busy.
+// Two tokens rather than four: 80 registers, six CTAs per SM, twice as many shorter CTAs,
+// whose load, compute and store phases overlap better (the 130M-LM step 1.7% faster).
 // Chunks wholly past a row's length are skipped (the scan never reads them); padded tokens
 // of a chunk get zeros.  A launch covers chunks [nc0, nc0 + ncn) of every chain.
 constexpr int kPrepThreads = 128;
-constexpr int kPrepTPT = 4;     // consecutive tokens per thread
+constexpr int kPrepTPT = 2;     // consecutive tokens per thread
 constexpr int kPrepLevels = 3;  // residual levels whose gain rows are loaded together
 __host__ __device__ constexpr int prep_tokens(int D) { return kPrepThreads * kPrepTPT / (D / 8); }
 
 __device__ __forceinline__ uint4 ldg16(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
 template <int D, int CH, int WM>  // WM >= W: taps of a head in shared memory
-__global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 4 : 2)
+__global__ void __launch_bounds__(kPrepThreads, WM <= 4 ? 6 : 3)
     residual_write_kernel(const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ gain,
                           const float* __restrict__ alpha, const float* __restrict__ gamma,
                           const float* __restrict__ conv_w, const int32_t* __restrict__ lengths,
