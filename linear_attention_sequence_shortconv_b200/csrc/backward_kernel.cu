@@ -72,6 +72,8 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(BwdParams p) {
   const int rb = blockIdx.x, nrb = gridDim.x;
   const int c_raw = rb * RB + tid / LPR, j = tid % LPR;
   const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
+  // debug build: a block outside the batch touches no memory (block-uniform)
+  if (!in_bounds(bh, (long long)p.B * p.H, p.status)) return;
   const int T_ = p.T, H = p.H, dk = p.d_k, dv = p.d_v, m = p.L - 1, W = p.W;
   const int NV = (2 + m) * dk + (2 + m);
   const int len = p.lengths ? min(max(p.lengths[b], 0), T_) : T_;

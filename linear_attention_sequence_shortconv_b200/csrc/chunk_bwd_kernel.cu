@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(kAdjBlock) adjoint_scan_kernel(ChunkBwdParams 
   const int row0 = blockIdx.x * RPB;
   const int row = row0 + lrow;
   const int h = blockIdx.y, b = blockIdx.z;
+  // debug build: a block outside the batch or the heads touches no memory (block-uniform)
+  if (!in_bounds(b, p.B, p.status) || !in_bounds(h, p.H, p.status)) return;
   const int T_ = p.T, H = p.H, dk = p.d, dv = p.d, m = p.L - 1;
   const bool row_ok = row < dv;
   const int c = row_ok ? row : dv - 1;
@@ -407,6 +409,10 @@ __global__ void __launch_bounds__(kGradThreads) chunk_grad_kernel(ChunkBwdParams
   float* sred = sm + Ly::RED;
 
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // debug build: a block outside the batch, the heads or the chunks touches no memory
+  if (!in_bounds(b, p.B, p.status) || !in_bounds(h, p.H, p.status) ||
+      !in_bounds(n, (p.T + kBwdChunk - 1) / kBwdChunk, p.status))
+    return;
   const int T_ = p.T, H = p.H, W = p.W;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15, warp = tid >> 5, lane = tid & 31;
   const int len = p.lengths ? min(max(p.lengths[b], 0), T_) : T_;

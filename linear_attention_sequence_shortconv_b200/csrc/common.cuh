@@ -90,6 +90,7 @@ struct BwdParams {
   float* dconv_w;     // [H, d_v, W]
   float* dS0;
   int B, T, H, d_k, d_v, L, W, chain;
+  int* status;        // device status word (the debug build's bounds checks record there)
 };
 
 // Pointers and sizes of the chunked backward (d_k = d_v = d; device pointers).
@@ -125,6 +126,7 @@ struct ChunkBwdParams {
   float* dconv_w;
   float* dS0;
   int B, T, H, d, L, W, chain;
+  int* status;          // device status word (the debug build's bounds checks record there)
 };
 
 // One step of the residual chain.  Exact form (gist.science PRISM explainer, 2.2

@@ -416,7 +416,7 @@ int prism_scan_bwd(const void* q, const void* k, const void* v, const float* gam
                              reinterpret_cast<float*>(wsb + ws.gu), reinterpret_cast<float*>(wsb + ws.hs),
                              reinterpret_cast<float*>(wsb + ws.part), dq, dk, dv, dgamma, dbeta,
                              L > 1 ? du : nullptr, L > 1 ? dalpha : nullptr, L > 1 ? dgain : nullptr, dconv_w, dS0,
-                             B, T, H, d_k, L, W, chain};
+                             B, T, H, d_k, L, W, chain, status};
     err = prism::launch_chunk_bwd(cp, dtype, s);
     return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
   }
@@ -436,7 +436,7 @@ int prism_scan_bwd(const void* q, const void* k, const void* v, const float* gam
   prism::BwdParams bp{q, k, v, gamma, beta, L > 1 ? u : nullptr, L > 1 ? alpha : nullptr, L > 1 ? gain : nullptr,
                       conv_w, S0, lengths, dO, dS_final, states, dq, dk, dv, dgamma, dbeta,
                       L > 1 ? du : nullptr, L > 1 ? dalpha : nullptr, L > 1 ? dgain : nullptr, dconv_part, part,
-                      dconv_w, dS0, B, T, H, d_k, d_v, L, W, chain};
+                      dconv_w, dS0, B, T, H, d_k, d_v, L, W, chain, status};
   err = prism::launch_scan_bwd(bp, dtype, s);
   return err == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }

@@ -3,7 +3,7 @@ the global indices they compute against their buffers' extents and record
 PRISM_ERR_BOUNDS instead of faulting.  On valid inputs it must report nothing and give the
 release build's results bit for bit, on every forward path: the tensor-core scan (plain,
 in two halves, cut into segments, ragged rows), the fp32 chunk form, the token-by-token
-kernel, and the decode step.  Its probe hook shows that a failed device-side check
+kernel, the decode step, and both backward paths.  Its probe hook shows that a failed device-side check
 reaches prism_stream_status.
 
 The debug library is loaded in a child process (PRISM_DEBUG_BOUNDS=1 selects it), which
@@ -69,6 +69,19 @@ def _run_all():
         out[f"decode_{name}_status"] = np.array(prism.stream_status())
         out[f"decode_{name}_S"] = S.cpu().numpy()
         out[f"decode_{name}_hist"] = hist.float().cpu().numpy()
+    # backward: the chunked path (d = 64, ragged rows) and the token-by-token one (fp32, d = 32)
+    for name, w in (("bwd_chunked", synth.Workload("h", B=2, T=150, H=2, d_k=64, d_v=64, L=3, chunk=64,
+                                                   lengths_lo=70, with_s0=True, seed=88)),
+                    ("bwd_token", synth.Workload("i", B=1, T=60, H=2, d_k=32, d_v=32, L=3, chunk=32, dtype="fp32",
+                                                 with_s0=True, seed=89))):
+        inp = synth.make_inputs(w)
+        d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+        dO = torch.randn((w.B, w.T, w.H, w.d_v), generator=torch.Generator().manual_seed(7)).to(inp["v"].dtype)
+        g = prism.scan_bwd(d["q"], d["k"], d["v"], d["gamma"], d["beta"], d["u"], d["alpha"], d["gain"],
+                           d["conv_w"], dO.cuda(), L=w.L, S0=d["S0"], lengths=d["lengths"])
+        out[f"{name}_status"] = np.array(prism.stream_status())
+        for n, t in g.items():
+            out[f"{name}_{n}"] = t.cpu().numpy()
     return out
 
 
