@@ -107,3 +107,16 @@ def test_fp32_chunk_conv_state_split():
     o_ref, S_ref = prism_seq(**x, chain="gelu")
     assert max_abs_rel_err(o, o_ref) <= TOL
     assert max_abs_rel_err(S2.cpu().numpy(), S_ref, slice_axes=(0, 1)) <= TOL
+
+
+@pytest.mark.parametrize("T,chunk", [(1, 16), (15, 16), (16, 16), (17, 16), (33, 16), (1, 64), (63, 64), (65, 64)])
+def test_fp32_chunk_boundary_lengths(T, chunk):
+    """Sequences of one token, one short of a chunk, exactly one chunk, one past it, and two
+    chunks plus one, with an initial state and the ShortConv window reaching before token 0."""
+    w = synth.Workload("j", B=2, T=T, H=2, d_k=16, d_v=16, L=3, chunk=chunk, W=4, dtype="fp32", with_s0=True,
+                       seed=90 + T)
+    inp = synth.make_inputs(w)
+    o, S = gpu_run(inp, w)
+    o_ref, S_ref = oracle_run(inp, w)
+    assert max_abs_rel_err(o, o_ref) <= TOL
+    assert max_abs_rel_err(S, S_ref, slice_axes=(0, 1)) <= TOL
