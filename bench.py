@@ -514,7 +514,8 @@ def run_ours(args, w):
                               "beside the first), CUDA events on the call's stream" if halves else
                               "scan launch(es) of each step, CUDA events on the launching stream"),
                     "kernel_us": scan_ms * 1e3, "algorithmic_bytes_per_launch": scan_bytes, "peak_source": peak_src,
-                    "residual_write": {"kernel": "residual_write_kernel" + (" (first half)" if halves else ""),
+                    "residual_write": {"kernel": "residual_write_kernel" + (
+                                           f" (chunks 0-{first_chunks - 1}, first launch)" if halves else ""),
                                        "us": prep_ms * 1e3, "algorithmic_bytes": rw_first,
                                        "achieved_gbs": rw_first / (prep_ms / 1e3) / 1e9,
                                        "frac": rw_first / (prep_ms / 1e3) / 1e9 / hbm,
